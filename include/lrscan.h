@@ -1,0 +1,183 @@
+/*
+ * lrscan.h -- C ABI of the B200 (sm_100a) fused linear-recurrence scan library.
+ *
+ * The operation.  A linear recurrence h_t = a_t (.) h_{t-1} + b_t with readout y_t = f(h_t),
+ * run over the whole sequence in one pass on the GPU instead of one dispatch per step, with a
+ * backward pass that stores only the states at segment boundaries and recomputes the rest
+ * ("mlx-recurrence", Apple Developer Forums thread 840535: opening paragraphs, and the list of
+ * kernels under "Current kernels").  The associative operator (a2,b2) o (a1,b1) =
+ * (a2 a1, a2 b1 + b2) that lets the sequence be split into chunks is the one stated in the
+ * K-Search / mlx-mamba blog post (techtrendfeed repost, paragraph after Table 1).  The
+ * time-varying selective scan with ZOH or bilinear discretisation follows "lrnnx: A library for
+ * Linear RNNs" (ai.info summary, Key Contributions 2 and 3).
+ *
+ * Kinds (per-kind definitions, t = 0..L-1, h_{-1} = 0):
+ *   LR_RGLRU   h_t = a_t h_{t-1} + b_t, y_t = h_t.                                  state [B, D]
+ *   LR_ROTLRU  pair k = channels (2k, 2k+1) = (re, im); lambda_t = mag_k g_t[k] e^{i theta_k};
+ *              h_t = lambda_t h_{t-1} + b_t (complex), y_t = h_t.                   state [B, D]
+ *   LR_S6      per (d, n): abar, beta = disc(dt_t[d], A[d,n]);
+ *              h_t[d,n] = abar h_{t-1}[d,n] + beta B_t[n] x_t[d];
+ *              y_t[d] = (sum_n C_t[n] h_t[d,n] + D_d x_t[d]) * silu(z_t[d]).     state [B, D, N]
+ *   LR_SSD     per head h, group g = h / (H / G): abar_t, beta_t = disc(dt_t[h], A_h);
+ *              h_t[p,n] = abar_t h_{t-1}[p,n] + beta_t x_t[p] B_t[g,n];
+ *              y_t[p] = sum_n C_t[g,n] h_t[p,n] + D_h x_t[p]  (times silu(z_t[p]) if z).
+ *                                                                                state [B, H, P, N]
+ *   LR_GLA     S_t = g_t S_{t-1} + k_t v_t^T (K x V), o_t = S_t^T q_t.          state [B, H, K, V]
+ *   disc ZOH:      abar = exp(dt A), beta = (exp(dt A) - 1) / A.
+ *   disc BILINEAR: abar = (1 + dt A/2) / (1 - dt A/2), beta = dt / (1 - dt A/2).
+ *
+ * Layouts.  Row-major, last index contiguous, token-major:
+ *   rglru   a, b, y, dy, da, db            [B, L, D]              io dtype
+ *   rotlru  b, y, dy, db                   [B, L, D] (re, im interleaved)   io dtype
+ *           g, dg                          [B, L, D/2]            io dtype
+ *           mag, theta, dmag, dtheta       [D/2]                  f32
+ *   s6      x, delta, z, y, dy, dx, ddelta, dz   [B, L, D]        io dtype
+ *           A, dA [D, N] f32;  Bm, Cm [B, L, N] io;  dBm, dCm [B, L, N] f32;  Dskip, dDskip [D] f32
+ *   ssd     x, z, y, dy, dx, dz [B, L, H, P] io;  delta, ddelta [B, L, H] io;
+ *           A, dA, Dskip, dDskip [H] f32;  Bm, Cm [B, L, G, N] io;  dBm, dCm [B, L, G, N] f32
+ *   gla     q, k, dq, dk [B, L, H, K] io;  v, o, dy, dv [B, L, H, V] io;  g, dg [B, L, H] io
+ *   (for GLA the descriptor's N field carries K and P carries V).
+ *
+ * Ownership.  The caller allocates and frees every buffer: inputs, outputs, gradients, the
+ * checkpoint buffer (lr_ckpt_bytes) and the workspace (lr_workspace_bytes).  The library
+ * allocates nothing and frees nothing, and keeps no pointer after a call returns.  All pointers
+ * passed to lr_scan_fwd / lr_scan_bwd are device pointers.
+ *
+ * Asynchrony and errors.  lr_scan_fwd / lr_scan_bwd validate on the host and enqueue work on the
+ * given CUDA stream (a cudaStream_t passed as void*; NULL = legacy default stream); the returned
+ * status covers validation and launch errors only.  Faults the kernels detect themselves (a
+ * bounded wait that gave up, a failed bounds check in a checking build) are recorded in the
+ * workspace and reported by lr_get_error.  Kernels never trap, assert or spin without a bound.
+ *
+ * Alignment.  Every pointer must be 16-byte aligned and the innermost dimension of every
+ * per-token tensor must span a multiple of 16 bytes (LR_ERR_ALIGNMENT otherwise).
+ *
+ * Gradients are written, not accumulated.
+ */
+#ifndef LRSCAN_H
+#define LRSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LRSCAN_VERSION 1
+
+typedef enum {
+    LR_OK = 0,
+    LR_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, non-positive or inconsistent shape   */
+    LR_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (see lr_validate) */
+    LR_ERR_ALIGNMENT = 3,     /* pointer or innermost extent not 16-byte aligned                */
+    LR_ERR_WORKSPACE = 4,     /* workspace smaller than lr_workspace_bytes                      */
+    LR_ERR_CUDA = 5,          /* a CUDA runtime call failed (launch, memset, copy)              */
+    LR_ERR_TIMEOUT = 6,       /* device: a bounded wait gave up (reported by lr_get_error)      */
+    LR_ERR_DEVICE_CHECK = 7   /* device: a bounds/consistency check failed (lr_get_error)       */
+} lr_status;
+
+typedef enum { LR_RGLRU = 0, LR_ROTLRU = 1, LR_S6 = 2, LR_SSD = 3, LR_GLA = 4 } lr_kind;
+typedef enum { LR_DISC_NONE = 0, LR_DISC_ZOH = 1, LR_DISC_BILINEAR = 2 } lr_disc;
+typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
+
+/* flags */
+#define LR_HAS_Z 1u       /* S6 / SSD: multiply the readout by silu(z)   */
+#define LR_HAS_DSKIP 2u   /* S6 / SSD: add the D-skip term D * x         */
+/* Test hook for the failure path: the tiles of the first segment never publish their carry, so
+ * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
+ * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
+#define LR_TEST_WITHHOLD_CARRY 0x80000000u
+
+/* Problem descriptor.  Unused dimensions are 0.  S6: D, N.  SSD: H, P, N, G, chunk.
+ * GLA: H, P (= V), N (= K), chunk.  rglru / rotlru: D.  segment = checkpoint segment length S
+ * (the backward pass stores the state every S steps and recomputes inside a segment). */
+typedef struct {
+    int32_t kind;      /* lr_kind  */
+    int32_t disc;      /* lr_disc  (S6 / SSD: ZOH or BILINEAR; others: NONE) */
+    int32_t io;        /* lr_dtype of per-token tensors                         */
+    uint32_t flags;    /* LR_HAS_Z | LR_HAS_DSKIP                               */
+    int64_t B, L, D, H, P, N, G;
+    int32_t chunk;     /* SSD / GLA chunk length Q (0 = default 64)             */
+    int32_t segment;   /* checkpoint segment length S                           */
+} lr_desc;
+
+/* Inputs, per kind (unused members NULL).  Device pointers. */
+typedef struct {
+    const void *a, *b;            /* rglru a, b; rotlru b                    */
+    const void *g;                /* rotlru magnitude gate; gla forget gate  */
+    const float *mag, *theta;     /* rotlru                                  */
+    const void *x, *delta;        /* s6 / ssd                                */
+    const float *A;               /* s6 [D,N] / ssd [H]                      */
+    const void *Bm, *Cm;          /* s6 / ssd                                */
+    const float *Dskip;           /* s6 [D] / ssd [H] (LR_HAS_DSKIP)         */
+    const void *z;                /* s6 / ssd (LR_HAS_Z)                     */
+    const void *q, *k, *v;        /* gla                                     */
+} lr_inputs;
+
+/* Gradients, per kind (unused members NULL).  Device pointers. */
+typedef struct {
+    void *da, *db, *dg;           /* rglru da, db; rotlru db, dg; gla dg     */
+    float *dmag, *dtheta;         /* rotlru                                  */
+    void *dx, *ddelta;            /* s6 / ssd                                */
+    float *dA, *dBm, *dCm, *dDskip;
+    void *dz;
+    void *dq, *dk, *dv;           /* gla                                     */
+} lr_grads;
+
+/* Host-side check of a descriptor: LR_OK, or the status lr_scan_fwd would return for it
+ * (INVALID_ARG for inconsistent shapes, UNSUPPORTED for a valid request outside this build's
+ * limits, ALIGNMENT for innermost extents that are not multiples of 16 bytes). */
+lr_status lr_validate(const lr_desc *desc);
+
+/* Bytes of the checkpoint buffer: ceil(L/S) states, f32 (slot k = state after k*S steps).
+ * The forward pass writes it and the backward pass reads it.  0 on an invalid descriptor. */
+size_t lr_ckpt_bytes(const lr_desc *desc);
+
+/* Bytes of scratch the forward (backward = 0) or backward (backward = 1) pass needs: per-tile
+ * carry records and flags, parameter-gradient partial sums and the error word.  The content need
+ * not be initialised; each call resets what it uses.  0 on an invalid descriptor. */
+size_t lr_workspace_bytes(const lr_desc *desc, int backward);
+
+/* Forward pass over the whole sequence: writes y and the segment checkpoints.
+ *   desc, in   problem and input pointers (see the layout table above)
+ *   y          output, same layout and dtype as the kind's per-token output
+ *   ckpt       checkpoint buffer of lr_ckpt_bytes(desc) bytes (written)
+ *   ws         workspace of ws_bytes >= lr_workspace_bytes(desc, 0) bytes
+ *   stream     cudaStream_t as void*
+ * Returns LR_OK once the work is enqueued. */
+lr_status lr_scan_fwd(const lr_desc *desc, const lr_inputs *in, void *y, void *ckpt, void *ws,
+                      size_t ws_bytes, void *stream);
+
+/* Backward pass: recomputes the states inside each segment from ckpt and runs the adjoint
+ * recurrence in reverse; writes every non-NULL gradient required by the kind
+ * (rglru: da, db; rotlru: db, dg, dmag, dtheta; s6: dx, ddelta, dA, dBm, dCm, dDskip if
+ * LR_HAS_DSKIP, dz if LR_HAS_Z; ssd: the same with per-head dA, dDskip; gla: dq, dk, dv, dg).
+ *   dy         upstream gradient of y (io dtype, y's layout)
+ *   ckpt       the buffer the matching lr_scan_fwd call wrote
+ *   ws         workspace of ws_bytes >= lr_workspace_bytes(desc, 1) bytes */
+lr_status lr_scan_bwd(const lr_desc *desc, const lr_inputs *in, const void *dy, const void *ckpt,
+                      lr_grads *grads, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads and clears the device-side error record in `ws`.  Every
+ * lr_scan_fwd / lr_scan_bwd call resets that record when it starts, so this reports the most
+ * recent call that used `ws`.  LR_OK, LR_ERR_TIMEOUT or LR_ERR_DEVICE_CHECK; LR_ERR_CUDA
+ * if the synchronisation itself failed.  `info`, if non-NULL, receives a kernel-specific code. */
+lr_status lr_get_error(void *ws, void *stream, int32_t *info);
+
+/* Static, human-readable name of a status. */
+const char *lr_status_string(lr_status s);
+
+/* Names of the kernels the last lr_scan_fwd / lr_scan_bwd call on this host thread launched,
+ * separated by '+' (a fingerprint that lets tests check which code path ran). */
+const char *lr_last_dispatch(void);
+
+/* Number of kernel launches the last lr_scan_fwd / lr_scan_bwd call on this thread enqueued. */
+int lr_last_launch_count(void);
+
+int lr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LRSCAN_H */

@@ -1,0 +1,182 @@
+// common.cuh -- device-side building blocks shared by the scan kernels (sm_100a).
+//
+//  * TMA tile copies (cp.async.bulk.tensor, no multicast) completing on an mbarrier, and TMA
+//    tile stores through bulk groups;
+//  * mbarrier waits with an iteration bound: a wait that gives up records LR_ERR_TIMEOUT in the
+//    workspace error record and returns false instead of spinning forever;
+//  * acquire / release flag accesses for the single-pass chained scan across tiles;
+//  * the workspace header (error record and tile tickets).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lrscan.h"
+
+namespace lrs {
+
+// ----------------------------------------------------------------------------- workspace header
+// First 256 bytes of every workspace.  Zeroed by the host (cudaMemsetAsync) before each call.
+struct WsHeader {
+    unsigned int err;       // first device-side error status (0 = none)
+    int info;               // kernel-specific detail of that error
+    unsigned int ticket[6]; // dynamic tile tickets, one per kernel of a call
+    unsigned int pad[56];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+// Bounded waits give up after this long (ns of %globaltimer) and record LR_ERR_TIMEOUT.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void record_error(WsHeader* hdr, unsigned int code, int info) {
+    if (atomicCAS(&hdr->err, 0u, code) == 0u) atomicExch(&hdr->info, info);
+}
+
+// ------------------------------------------------------------------------------ numeric I/O
+template <typename T> struct IO;
+template <> struct IO<float> {
+    static __device__ __forceinline__ float ld(const float* p) { return *p; }
+    static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
+};
+template <> struct IO<__nv_bfloat16> {
+    static __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+// ------------------------------------------------------------------------------ smem addresses
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`.  Returns false (and records LR_ERR_TIMEOUT) if the
+// phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WsHeader* hdr, int info) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_error(hdr, LR_ERR_TIMEOUT, info);
+    return false;
+}
+
+// ------------------------------------------------------------------------------------- TMA
+// 3-D tiled load global -> shared, completion counted on `bar` (bytes).  No multicast.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 3-D tiled store shared -> global (out-of-range rows/columns of the box are clipped).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------- cross-CTA flag protocol
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned int* p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Status of a tile's carry record in the chained scan.
+enum : unsigned int { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2 };
+
+// Poll `flag` until it is non-zero, for at most kWaitLimitNs.  Returns the flag, or kFlagNone
+// after giving up (an error is then recorded).
+__device__ __forceinline__ unsigned int wait_flag(const unsigned int* flag, WsHeader* hdr, int info) {
+    unsigned int f = ld_acquire(flag);
+    if (f != kFlagNone) return f;
+    const unsigned long long t0 = global_ns();
+    for (int i = 0;; ++i) {
+        f = ld_acquire(flag);
+        if (f != kFlagNone) return f;
+        if (i > 16) __nanosleep(128);
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_error(hdr, LR_ERR_TIMEOUT, info);
+    return kFlagNone;
+}
+
+// Dynamic tile ticket: tiles are numbered in the order CTAs start, so that every tile a CTA may
+// wait on belongs to a CTA that has already started.
+__device__ __forceinline__ unsigned int take_ticket(WsHeader* hdr, int which) {
+    return atomicAdd(&hdr->ticket[which], 1u);
+}
+
+// ------------------------------------------------------------------------- complex helpers
+struct cpx {
+    float r, i;
+};
+__device__ __forceinline__ cpx cmul(cpx a, cpx b) {
+    return {fmaf(a.r, b.r, -a.i * b.i), fmaf(a.r, b.i, a.i * b.r)};
+}
+__device__ __forceinline__ cpx cfma(cpx a, cpx b, cpx c) {  // a*b + c
+    return {fmaf(a.r, b.r, fmaf(-a.i, b.i, c.r)), fmaf(a.r, b.i, fmaf(a.i, b.r, c.i))};
+}
+__device__ __forceinline__ cpx conjc(cpx a) { return {a.r, -a.i}; }
+
+}  // namespace lrs

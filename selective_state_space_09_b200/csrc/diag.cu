@@ -1,0 +1,668 @@
+// diag.cu -- diagonal chassis: rglru_scan and rotlru_scan, forward and backward (sm_100a).
+//
+// Recurrence h_t = c_t h_{t-1} + b_t with a real (rglru) or complex (rotlru) diagonal
+// coefficient c_t, read out as y_t = h_t ("mlx-recurrence", Apple Developer Forums thread
+// 840535, "Current kernels": rglru_scan, rotlru_scan).  The sequence is cut into checkpoint
+// segments of S steps; chunks compose with the associative operator
+// (c2, b2) o (c1, b1) = (c2 c1, c2 b1 + b2) of the K-Search / mlx-mamba post (techtrendfeed
+// repost, paragraph after Table 1).
+//
+// Tiling.  One CTA owns one tile = (batch row b, channel block, segment): S steps x CB units
+// (rglru: 32 real channels; rotlru: 16 complex pairs = 32 floats).  The CTA loads the whole tile
+// into shared memory with TMA (one box per tensor, ragged tails zero-filled by the TMA unit),
+// splits it into NG time groups of S/NG steps (one thread per unit per group), scans each group
+// sequentially in fp32, combines the groups in shared memory and chains the tiles of a row
+// through a single-pass look-back over per-tile carry records (aggregate first, inclusive
+// prefix once known; bounded waits).  Results are written back into the tile's shared-memory
+// slots and stored with TMA.
+//
+// Forward: carries flow to later segments; the carry entering each segment is the segment
+// checkpoint (written to ckpt).  Backward ("segment checkpointing with recomputation during the
+// backward pass", same post): each tile starts from its checkpoint, recomputes its states into
+// registers, runs the adjoint recurrence G_t = dy_t + conj(c_{t+1}) G_{t+1} with carries flowing
+// to earlier segments, and writes the input gradients; rotlru's parameter gradients are summed
+// per tile into partials that a second kernel reduces in a fixed order.
+#include <stdio.h>
+
+#include "common.cuh"
+#include "host_common.h"
+
+namespace lrs {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxSeg = 256;  // TMA box rows; S <= 256 keeps the tile in one box per tensor
+
+__device__ __forceinline__ float one_of(float) { return 1.0f; }
+__device__ __forceinline__ cpx one_of(cpx) { return {1.0f, 0.0f}; }
+__device__ __forceinline__ float zero_of(float) { return 0.0f; }
+__device__ __forceinline__ cpx zero_of(cpx) { return {0.0f, 0.0f}; }
+__device__ __forceinline__ float mulx(float a, float b) { return a * b; }
+__device__ __forceinline__ cpx mulx(cpx a, cpx b) { return cmul(a, b); }
+__device__ __forceinline__ float fmax_(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ cpx fmax_(cpx a, cpx b, cpx c) { return cfma(a, b, c); }
+__device__ __forceinline__ float conjx(float a) { return a; }
+__device__ __forceinline__ cpx conjx(cpx a) { return conjc(a); }
+__device__ __forceinline__ float addx(float a, float b) { return a + b; }
+__device__ __forceinline__ cpx addx(cpx a, cpx b) { return {a.r + b.r, a.i + b.i}; }
+
+template <typename V> struct Agg {
+    V m;  // product of coefficients over the span
+    V v;  // local result with zero carry-in
+};
+
+struct DiagArgs {
+    int B, L, D, S, nseg, ncb;  // D = real channels of b / y
+    unsigned int dflags;        // lr_desc flags (LR_TEST_WITHHOLD_CARRY)
+    const float* mag;           // rotlru
+    const float* theta;         // rotlru
+    float* ckpt;                // [nseg, B, D] f32
+    WsHeader* hdr;
+    unsigned int* flags;        // [B * ncb * nseg]
+    void* agg;                  // Agg<V>[tiles][CB]
+    void* pre;                  // V[tiles][CB]
+    float2* partial;            // rotlru bwd: [B * nseg][D/2] (dmag, dtheta)
+};
+
+// Per-kind description.  Unit = the element one thread carries through time.
+template <int KIND, typename T> struct Kind;
+
+template <typename T> struct Kind<LR_RGLRU, T> {
+    using V = float;
+    static constexpr int CB = 32;        // units (channels) per tile
+    static constexpr int NG = 8;         // time groups
+    static constexpr int CW = CB;        // coefficient-tensor columns per tile
+    static constexpr int BW = CB;        // b / y columns per tile
+    struct Unit {
+        __device__ Unit(const DiagArgs&, int) {}
+        __device__ __forceinline__ V coef(const T* C, int t, int u) const {
+            return IO<T>::ld(C + t * CW + u);
+        }
+    };
+    static __device__ __forceinline__ V ldb(const T* Bs, int t, int u) { return IO<T>::ld(Bs + t * BW + u); }
+    static __device__ __forceinline__ void stb(T* Bs, int t, int u, V v) { IO<T>::st(Bs + t * BW + u, v); }
+    static __device__ __forceinline__ void st_ckpt(float* p, int chan0, V v) { p[chan0] = v; }
+    static __device__ __forceinline__ V ld_ckpt(const float* p, int chan0) { return p[chan0]; }
+    static constexpr int chans_per_unit = 1;
+};
+
+template <typename T> struct Kind<LR_ROTLRU, T> {
+    using V = cpx;
+    static constexpr int CB = 16;        // complex pairs per tile
+    static constexpr int NG = 16;
+    static constexpr int CW = CB;        // g columns (one per pair)
+    static constexpr int BW = 2 * CB;    // b / y columns (re, im interleaved)
+    struct Unit {
+        float mag, cs, sn;
+        __device__ Unit(const DiagArgs& a, int pair) {
+            bool ok = pair < a.D / 2;
+            mag = ok ? a.mag[pair] : 0.0f;
+            float th = ok ? a.theta[pair] : 0.0f;
+            sincosf(th, &sn, &cs);
+        }
+        __device__ __forceinline__ V coef(const T* C, int t, int u) const {
+            float m = mag * IO<T>::ld(C + t * CW + u);
+            return {m * cs, m * sn};
+        }
+    };
+    static __device__ __forceinline__ V ldb(const T* Bs, int t, int u) {
+        return {IO<T>::ld(Bs + t * BW + 2 * u), IO<T>::ld(Bs + t * BW + 2 * u + 1)};
+    }
+    static __device__ __forceinline__ void stb(T* Bs, int t, int u, V v) {
+        IO<T>::st(Bs + t * BW + 2 * u, v.r);
+        IO<T>::st(Bs + t * BW + 2 * u + 1, v.i);
+    }
+    static __device__ __forceinline__ void st_ckpt(float* p, int chan0, V v) {
+        p[chan0] = v.r;
+        p[chan0 + 1] = v.i;
+    }
+    static __device__ __forceinline__ V ld_ckpt(const float* p, int chan0) { return {p[chan0], p[chan0 + 1]}; }
+    static constexpr int chans_per_unit = 2;
+};
+
+// Shared-memory plan of one tile.
+template <int KIND, typename T, bool BWD> struct Smem {
+    using K = Kind<KIND, T>;
+    using V = typename K::V;
+    static __host__ __device__ constexpr size_t coef_bytes() { return size_t(kMaxSeg) * K::CW * sizeof(T); }
+    static __host__ __device__ constexpr size_t b_bytes() { return size_t(kMaxSeg) * K::BW * sizeof(T); }
+    static __host__ __device__ constexpr size_t off_coef() { return 128; }
+    static __host__ __device__ constexpr size_t off_b() { return off_coef() + coef_bytes(); }
+    static __host__ __device__ constexpr size_t off_dy() { return off_b() + b_bytes(); }
+    static __host__ __device__ constexpr size_t off_aggf() { return off_dy() + (BWD ? b_bytes() : 0); }
+    static __host__ __device__ constexpr size_t off_aggr() { return off_aggf() + sizeof(Agg<V>) * K::NG * K::CB; }
+    static __host__ __device__ constexpr size_t off_carry() {
+        return off_aggr() + (BWD ? sizeof(Agg<V>) * K::NG * K::CB : 0);
+    }
+    static __host__ __device__ constexpr size_t off_red() { return off_carry() + 2 * sizeof(V) * K::CB; }
+    static __host__ __device__ constexpr size_t off_misc() {
+        return off_red() + (BWD ? sizeof(float2) * K::NG * K::CB : 0);
+    }
+    static __host__ __device__ constexpr size_t total() { return off_misc() + 64 + 128; }
+};
+
+template <typename V>
+__device__ __forceinline__ void st_cg(V* p, V v) {
+    if constexpr (sizeof(V) == 4) {
+        __stcg(reinterpret_cast<float*>(p), *reinterpret_cast<float*>(&v));
+    } else {
+        __stcg(reinterpret_cast<float2*>(p), *reinterpret_cast<float2*>(&v));
+    }
+}
+template <typename V>
+__device__ __forceinline__ V ld_cg(const V* p) {
+    V v;
+    if constexpr (sizeof(V) == 4) {
+        *reinterpret_cast<float*>(&v) = __ldcg(reinterpret_cast<const float*>(p));
+    } else {
+        *reinterpret_cast<float2*>(&v) = __ldcg(reinterpret_cast<const float2*>(p));
+    }
+    return v;
+}
+template <typename V>
+__device__ __forceinline__ void st_cg_agg(Agg<V>* p, Agg<V> a) {
+    st_cg(&p->m, a.m);
+    st_cg(&p->v, a.v);
+}
+template <typename V>
+__device__ __forceinline__ Agg<V> ld_cg_agg(const Agg<V>* p) {
+    return {ld_cg(&p->m), ld_cg(&p->v)};
+}
+
+// Dynamic shared memory, re-aligned to 128 bytes.
+__device__ __forceinline__ char* smem_base() {
+    extern __shared__ char dyn_smem[];
+    uintptr_t p = reinterpret_cast<uintptr_t>(dyn_smem);
+    return reinterpret_cast<char*>((p + 127) & ~uintptr_t(127)) ;
+}
+
+// --------------------------------------------------------------------------------- forward
+template <int KIND, typename T>
+__global__ void __launch_bounds__(kThreads)
+diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
+                const __grid_constant__ CUtensorMap mapY, DiagArgs a) {
+    using K = Kind<KIND, T>;
+    using V = typename K::V;
+    using SM = Smem<KIND, T, false>;
+    constexpr int CB = K::CB, NG = K::NG;
+    char* sm = smem_base();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+    T* Cs = reinterpret_cast<T*>(sm + SM::off_coef());
+    T* Bs = reinterpret_cast<T*>(sm + SM::off_b());
+    Agg<V>* aggF = reinterpret_cast<Agg<V>*>(sm + SM::off_aggf());
+    V* carryS = reinterpret_cast<V*>(sm + SM::off_carry());
+    int* misc = reinterpret_cast<int*>(sm + SM::off_misc());
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = tid / CB, u = tid % CB;
+
+    if (tid == 0) {
+        unsigned int tk = take_ticket(a.hdr, 0);
+        int per_seg = a.B * a.ncb;
+        int seg = tk / per_seg, rem = tk % per_seg;
+        misc[0] = seg;
+        misc[1] = rem / a.ncb;
+        misc[2] = rem % a.ncb;
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+    const int seg = misc[0], b = misc[1], cb = misc[2];
+    const int t0g = seg * a.S;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + K::BW) * sizeof(T)));
+        tma_load_3d(Cs, &mapC, bar, cb * K::CW, t0g, b);
+        tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
+    }
+    const int unit = cb * CB + u;  // global unit index (channel or pair)
+    typename K::Unit U(a, unit);
+    const int nt = min(a.S, a.L - t0g);
+    const int spg = (a.S + NG - 1) / NG;
+    const int j0 = grp * spg, j1 = min(j0 + spg, nt);
+    bool ok = mbar_wait(bar, 0, a.hdr, 100);
+
+    // group aggregate with zero carry-in
+    V P = one_of(V{}), h = zero_of(V{});
+    if (ok) {
+        for (int j = j0; j < j1; ++j) {
+            V c = U.coef(Cs, j, u);
+            P = mulx(c, P);
+            h = fmax_(c, h, K::ldb(Bs, j, u));
+        }
+    }
+    aggF[grp * CB + u] = {P, h};
+    __syncthreads();
+
+    // tile carry through the chained look-back (warp 0, one lane per unit)
+    const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
+    if (warp == 0) {
+        const bool act = lane < CB && unit < units;
+        const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
+        Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
+        V* preRec = reinterpret_cast<V*>(a.pre);
+        Agg<V> tile{one_of(V{}), zero_of(V{})};
+        if (lane < CB) {
+            for (int g = 0; g < NG; ++g) {
+                Agg<V> ag = aggF[g * CB + lane];
+                tile.v = fmax_(ag.m, tile.v, ag.v);
+                tile.m = mulx(ag.m, tile.m);
+            }
+        }
+        const bool has_succ = seg + 1 < a.nseg;
+        if (seg > 0 && has_succ) {
+            if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+        }
+        V carry = zero_of(V{});
+        if (seg > 0) {
+            V Pc = one_of(V{}), hc = zero_of(V{});
+            int j = seg - 1;
+            while (true) {
+                unsigned int f = wait_flag(&a.flags[row + j], a.hdr, 101);
+                if (f == kFlagPrefix) {
+                    V st = act ? ld_cg(&preRec[(row + j) * CB + lane]) : zero_of(V{});
+                    carry = fmax_(Pc, st, hc);
+                    break;
+                }
+                if (f == kFlagAgg) {
+                    Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + j) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
+                    hc = fmax_(Pc, ag.v, hc);
+                    Pc = mulx(Pc, ag.m);
+                    if (--j < 0) { carry = hc; break; }
+                    continue;
+                }
+                carry = hc;  // gave up (error recorded): continue with what is known
+                break;
+            }
+        }
+        const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == 0;
+        if (has_succ && !withhold) {
+            if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
+        }
+        if (act) K::st_ckpt(a.ckpt + ((size_t)seg * a.B + b) * a.D, unit * K::chans_per_unit, carry);
+        if (lane < CB) carryS[lane] = carry;
+    }
+    __syncthreads();
+
+    // apply: recompute the group with its true carry-in, write y into the b slot
+    V hh = carryS[u];
+    for (int g = 0; g < grp; ++g) {
+        Agg<V> ag = aggF[g * CB + u];
+        hh = fmax_(ag.m, hh, ag.v);
+    }
+    if (ok) {
+        for (int j = j0; j < j1; ++j) {
+            V c = U.coef(Cs, j, u);
+            hh = fmax_(c, hh, K::ldb(Bs, j, u));
+            K::stb(Bs, j, u, hh);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        tma_store_3d(&mapY, Bs, cb * K::BW, t0g, b);
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+}
+
+// -------------------------------------------------------------------------------- backward
+template <int KIND, typename T>
+__global__ void __launch_bounds__(kThreads)
+diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
+                const __grid_constant__ CUtensorMap mapDY, const __grid_constant__ CUtensorMap mapDC,
+                const __grid_constant__ CUtensorMap mapDB, DiagArgs a) {
+    using K = Kind<KIND, T>;
+    using V = typename K::V;
+    using SM = Smem<KIND, T, true>;
+    constexpr int CB = K::CB, NG = K::NG;
+    constexpr int SPG = kMaxSeg / NG;
+    char* sm = smem_base();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+    T* Cs = reinterpret_cast<T*>(sm + SM::off_coef());
+    T* Bs = reinterpret_cast<T*>(sm + SM::off_b());
+    T* Ds = reinterpret_cast<T*>(sm + SM::off_dy());
+    Agg<V>* aggF = reinterpret_cast<Agg<V>*>(sm + SM::off_aggf());
+    Agg<V>* aggR = reinterpret_cast<Agg<V>*>(sm + SM::off_aggr());
+    V* carryS = reinterpret_cast<V*>(sm + SM::off_carry());
+    float2* red = reinterpret_cast<float2*>(sm + SM::off_red());
+    int* misc = reinterpret_cast<int*>(sm + SM::off_misc());
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = tid / CB, u = tid % CB;
+
+    if (tid == 0) {
+        unsigned int tk = take_ticket(a.hdr, 1);
+        int per_seg = a.B * a.ncb;
+        int seg = a.nseg - 1 - (int)(tk / per_seg), rem = tk % per_seg;
+        misc[0] = seg;
+        misc[1] = rem / a.ncb;
+        misc[2] = rem % a.ncb;
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+    const int seg = misc[0], b = misc[1], cb = misc[2];
+    const int t0g = seg * a.S;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + 2 * K::BW) * sizeof(T)));
+        tma_load_3d(Cs, &mapC, bar, cb * K::CW, t0g, b);
+        tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
+        tma_load_3d(Ds, &mapDY, bar, cb * K::BW, t0g, b);
+    }
+    const int unit = cb * CB + u;
+    const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
+    typename K::Unit U(a, unit);
+    if (tid < CB) {
+        V c0 = zero_of(V{});
+        if (unit < units)
+            c0 = K::ld_ckpt(a.ckpt + ((size_t)seg * a.B + b) * a.D, unit * K::chans_per_unit);
+        carryS[tid] = c0;
+    }
+    const int nt = min(a.S, a.L - t0g);
+    const int spg = (a.S + NG - 1) / NG;
+    const int j0 = grp * spg, j1 = min(j0 + spg, nt);
+    const int n = max(j1 - j0, 0);
+    bool ok = mbar_wait(bar, 0, a.hdr, 200);
+
+    // forward aggregate of the group
+    {
+        V P = one_of(V{}), h = zero_of(V{});
+        if (ok)
+            for (int j = j0; j < j1; ++j) {
+                V c = U.coef(Cs, j, u);
+                P = mulx(c, P);
+                h = fmax_(c, h, K::ldb(Bs, j, u));
+            }
+        aggF[grp * CB + u] = {P, h};
+    }
+    __syncthreads();
+    // states of the group, from the segment checkpoint, kept in registers
+    V hin = carryS[u];
+    for (int g = 0; g < grp; ++g) {
+        Agg<V> ag = aggF[g * CB + u];
+        hin = fmax_(ag.m, hin, ag.v);
+    }
+    V hreg[SPG];
+    {
+        V h = hin;
+#pragma unroll
+        for (int j = 0; j < SPG; ++j) {
+            if (j < n) {
+                V c = U.coef(Cs, j0 + j, u);
+                h = fmax_(c, h, K::ldb(Bs, j0 + j, u));
+            }
+            hreg[j] = h;
+        }
+    }
+    // reverse aggregate of the group: outgoing carry = v + m * incoming
+    {
+        V M = one_of(V{}), r = zero_of(V{});
+        if (ok)
+            for (int j = j1 - 1; j >= j0; --j) {
+                V cc = conjx(U.coef(Cs, j, u));
+                V G = addx(K::ldb(Ds, j, u), r);
+                r = mulx(cc, G);
+                M = mulx(cc, M);
+            }
+        aggR[grp * CB + u] = {M, r};
+    }
+    __syncthreads();
+
+    // tile carry from later segments (warp 0)
+    if (warp == 0) {
+        const bool act = lane < CB && unit < units;
+        const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
+        Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
+        V* preRec = reinterpret_cast<V*>(a.pre);
+        Agg<V> tile{one_of(V{}), zero_of(V{})};
+        if (lane < CB)
+            for (int g = NG - 1; g >= 0; --g) {
+                Agg<V> ag = aggR[g * CB + lane];
+                tile.v = fmax_(ag.m, tile.v, ag.v);
+                tile.m = mulx(ag.m, tile.m);
+            }
+        const bool has_pred = seg > 0;  // earlier segment waits on this one
+        if (has_pred && seg + 1 < a.nseg) {
+            if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+        }
+        V carry = zero_of(V{});
+        if (seg + 1 < a.nseg) {
+            V Mc = one_of(V{}), vc = zero_of(V{});
+            int j = seg + 1;
+            while (true) {
+                unsigned int f = wait_flag(&a.flags[row + j], a.hdr, 201);
+                if (f == kFlagPrefix) {
+                    V st = act ? ld_cg(&preRec[(row + j) * CB + lane]) : zero_of(V{});
+                    carry = fmax_(Mc, st, vc);
+                    break;
+                }
+                if (f == kFlagAgg) {
+                    Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + j) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
+                    vc = fmax_(Mc, ag.v, vc);
+                    Mc = mulx(Mc, ag.m);
+                    if (++j >= a.nseg) { carry = vc; break; }
+                    continue;
+                }
+                carry = vc;
+                break;
+            }
+        }
+        const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == a.nseg - 1;
+        if (has_pred && !withhold) {
+            if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
+        }
+        if (lane < CB) carryS[CB + lane] = carry;
+    }
+    __syncthreads();
+
+    // adjoint sweep of the group with its true carry; gradients into the shared slots
+    V r = carryS[CB + u];
+    for (int g = NG - 1; g > grp; --g) {
+        Agg<V> ag = aggR[g * CB + u];
+        r = fmax_(ag.m, r, ag.v);
+    }
+    float acc_mag = 0.0f, acc_th = 0.0f;
+#pragma unroll
+    for (int jj = SPG - 1; jj >= 0; --jj) {
+        if (jj < n && ok) {
+            const int j = j0 + jj;
+            V G = addx(K::ldb(Ds, j, u), r);
+            V hp = jj > 0 ? hreg[jj > 0 ? jj - 1 : 0] : hin;
+            if constexpr (KIND == LR_RGLRU) {
+                float c = IO<T>::ld(Cs + j * K::CW + u);
+                IO<T>::st(Ds + j * K::BW + u, G);       // db
+                IO<T>::st(Cs + j * K::CW + u, G * hp);  // da
+                r = c * G;
+            } else {
+                float gt = IO<T>::ld(Cs + j * K::CW + u);
+                float m = U.mag * gt;
+                cpx lam{m * U.cs, m * U.sn};
+                K::stb(Ds, j, u, G);                               // db
+                cpx dl = cmul(G, conjc(hp));                        // dlambda = G conj(h_{t-1})
+                float dm = fmaf(dl.r, U.cs, dl.i * U.sn);           // Re(dlambda e^{-i theta})
+                IO<T>::st(Cs + j * K::CW + u, U.mag * dm);          // dg
+                acc_mag = fmaf(gt, dm, acc_mag);
+                acc_th = fmaf(m, fmaf(dl.i, U.cs, -dl.r * U.sn), acc_th);
+                r = cmul(conjc(lam), G);
+            }
+        }
+    }
+    if constexpr (KIND == LR_ROTLRU) {
+        red[grp * CB + u] = make_float2(acc_mag, acc_th);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if constexpr (KIND == LR_ROTLRU) {
+        if (tid < CB && unit < units) {
+            float sm_ = 0.0f, st_ = 0.0f;
+            for (int g = 0; g < NG; ++g) {
+                float2 v = red[g * CB + tid];
+                sm_ += v.x;
+                st_ += v.y;
+            }
+            a.partial[((size_t)b * a.nseg + seg) * (a.D / 2) + unit] = make_float2(sm_, st_);
+        }
+    }
+    if (tid == 0 && ok) {
+        tma_store_3d(&mapDC, Cs, cb * K::CW, t0g, b);
+        tma_store_3d(&mapDB, Ds, cb * K::BW, t0g, b);
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+}
+
+// Fixed-order reduction of rotlru's per-tile parameter partials over (batch row, segment).
+__global__ void rotlru_param_reduce(const float2* __restrict__ partial, int rows, int K,
+                                    float* __restrict__ dmag, float* __restrict__ dtheta) {
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= K) return;
+    float s0 = 0.0f, s1 = 0.0f;
+    for (int r = 0; r < rows; ++r) {
+        float2 v = __ldg(&partial[(size_t)r * K + k]);
+        s0 += v.x;
+        s1 += v.y;
+    }
+    dmag[k] = s0;
+    dtheta[k] = s1;
+}
+
+// ------------------------------------------------------------------------------ host side
+struct Geo {
+    int nseg, ncb, tiles, cb;
+};
+
+Geo geo(const lr_desc& d) {
+    Geo g;
+    g.nseg = (int)((d.L + d.segment - 1) / d.segment);
+    int units = d.kind == LR_RGLRU ? (int)d.D : (int)(d.D / 2);
+    g.cb = d.kind == LR_RGLRU ? 32 : 16;
+    g.ncb = (units + g.cb - 1) / g.cb;
+    g.tiles = (int)d.B * g.ncb * g.nseg;
+    return g;
+}
+
+struct DiagWs {
+    size_t flags, agg, pre, partial, end;
+};
+
+DiagWs ws_plan(const lr_desc& d, bool bwd) {
+    Geo g = geo(d);
+    size_t vs = d.kind == LR_RGLRU ? 4 : 8;
+    WsCursor c;
+    DiagWs w;
+    w.flags = c.take(sizeof(unsigned int) * g.tiles);
+    w.agg = c.take(2 * vs * g.cb * (size_t)g.tiles);
+    w.pre = c.take(vs * g.cb * (size_t)g.tiles);
+    w.partial = (bwd && d.kind == LR_ROTLRU) ? c.take(sizeof(float2) * d.B * g.nseg * (d.D / 2)) : 0;
+    w.end = c.off;
+    return w;
+}
+
+template <int KIND, typename T, bool BWD>
+void set_smem_attr(const void* fn) {
+    static bool done = false;  // per instantiation
+    if (!done) {
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Smem<KIND, T, BWD>::total());
+        done = true;
+    }
+}
+
+template <int KIND, typename T>
+lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                     cudaStream_t st) {
+    using K = Kind<KIND, T>;
+    Geo g = geo(d);
+    DiagWs w = ws_plan(d, false);
+    const int es = sizeof(T);
+    CUtensorMap mC, mB, mY;
+    const void* coef = KIND == LR_RGLRU ? in.a : in.g;
+    uint64_t coefC = KIND == LR_RGLRU ? d.D : d.D / 2;
+    bool ok = make_tmap_3d(&mC, coef, es, coefC, d.L, d.B, K::CW, d.segment) &&
+              make_tmap_3d(&mB, in.b, es, d.D, d.L, d.B, K::BW, d.segment) &&
+              make_tmap_3d(&mY, y, es, d.D, d.L, d.B, K::BW, d.segment);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
+               (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
+               nullptr};
+    auto fn = diag_fwd_kernel<KIND, T>;
+    set_smem_attr<KIND, T, false>((const void*)fn);
+    note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : "rotlru_fwd_tile");
+    fn<<<g.tiles, kThreads, Smem<KIND, T, false>::total(), st>>>(mC, mB, mY, a);
+    return check_launch();
+}
+
+template <int KIND, typename T>
+lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                     const lr_grads& gr, char* ws, cudaStream_t st) {
+    using K = Kind<KIND, T>;
+    Geo g = geo(d);
+    DiagWs w = ws_plan(d, true);
+    const int es = sizeof(T);
+    CUtensorMap mC, mB, mDY, mDC, mDB;
+    const void* coef = KIND == LR_RGLRU ? in.a : in.g;
+    void* dcoef = KIND == LR_RGLRU ? gr.da : gr.dg;
+    uint64_t coefC = KIND == LR_RGLRU ? d.D : d.D / 2;
+    bool ok = make_tmap_3d(&mC, coef, es, coefC, d.L, d.B, K::CW, d.segment) &&
+              make_tmap_3d(&mB, in.b, es, d.D, d.L, d.B, K::BW, d.segment) &&
+              make_tmap_3d(&mDY, dy, es, d.D, d.L, d.B, K::BW, d.segment) &&
+              make_tmap_3d(&mDC, dcoef, es, coefC, d.L, d.B, K::CW, d.segment) &&
+              make_tmap_3d(&mDB, gr.db, es, d.D, d.L, d.B, K::BW, d.segment);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
+               (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
+               w.partial ? (float2*)(ws + w.partial) : nullptr};
+    auto fn = diag_bwd_kernel<KIND, T>;
+    set_smem_attr<KIND, T, true>((const void*)fn);
+    note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : "rotlru_bwd_tile");
+    fn<<<g.tiles, kThreads, Smem<KIND, T, true>::total(), st>>>(mC, mB, mDY, mDC, mDB, a);
+    lr_status s = check_launch();
+    if (s != LR_OK) return s;
+    if (KIND == LR_ROTLRU) {
+        int K2 = (int)(d.D / 2);
+        note_launch("rotlru_param_reduce");
+        rotlru_param_reduce<<<(K2 + 127) / 128, 128, 0, st>>>(a.partial, (int)d.B * g.nseg, K2,
+                                                             gr.dmag, gr.dtheta);
+        s = check_launch();
+    }
+    return s;
+}
+
+}  // namespace
+
+size_t diag_ws_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).end; }
+size_t diag_flag_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).agg; }
+
+lr_status diag_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                   cudaStream_t st) {
+    if (d.kind == LR_RGLRU)
+        return d.io == LR_F32 ? launch_fwd<LR_RGLRU, float>(d, in, y, ckpt, ws, st)
+                              : launch_fwd<LR_RGLRU, __nv_bfloat16>(d, in, y, ckpt, ws, st);
+    return d.io == LR_F32 ? launch_fwd<LR_ROTLRU, float>(d, in, y, ckpt, ws, st)
+                          : launch_fwd<LR_ROTLRU, __nv_bfloat16>(d, in, y, ckpt, ws, st);
+}
+
+lr_status diag_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                   const lr_grads& gr, char* ws, cudaStream_t st) {
+    if (d.kind == LR_RGLRU)
+        return d.io == LR_F32 ? launch_bwd<LR_RGLRU, float>(d, in, dy, ckpt, gr, ws, st)
+                              : launch_bwd<LR_RGLRU, __nv_bfloat16>(d, in, dy, ckpt, gr, ws, st);
+    return d.io == LR_F32 ? launch_bwd<LR_ROTLRU, float>(d, in, dy, ckpt, gr, ws, st)
+                          : launch_bwd<LR_ROTLRU, __nv_bfloat16>(d, in, dy, ckpt, gr, ws, st);
+}
+
+}  // namespace lrs

@@ -1,0 +1,64 @@
+// host_common.h -- host-side helpers shared by the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lrscan.h"
+
+namespace lrs {
+
+// Round up to a multiple of `a`.
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Records the name of a kernel about to be launched on this host thread (fingerprint for
+// lr_last_dispatch / lr_last_launch_count).
+void note_launch(const char* name);
+
+// Converts the last CUDA error into a status.
+lr_status check_launch();
+
+// Builds a tiled TMA descriptor of a rank-3 row-major tensor [d2][d1][d0] (d0 contiguous) of
+// element size `esize` (4 = f32, 2 = bf16) with box [1][box1][box0].  Returns false if the
+// driver rejects the description.
+bool make_tmap_3d(CUtensorMap* map, const void* base, int esize, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint32_t box0, uint32_t box1);
+
+// Byte offset bookkeeping for a workspace: a 256-byte header followed by regions.
+struct WsCursor {
+    size_t off = 256;
+    size_t take(size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    }
+};
+
+// Per-kind entry points (defined in the kernel files).  *_supported: whether this build has
+// kernels for the (already validated) descriptor.
+bool s6_supported(const lr_desc& d);
+bool chunk_supported(const lr_desc& d);
+size_t diag_ws_bytes(const lr_desc& d, bool bwd);
+size_t diag_flag_bytes(const lr_desc& d, bool bwd);
+lr_status diag_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                   cudaStream_t st);
+lr_status diag_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                   const lr_grads& gr, char* ws, cudaStream_t st);
+
+size_t s6_ws_bytes(const lr_desc& d, bool bwd);
+size_t s6_flag_bytes(const lr_desc& d, bool bwd);
+lr_status s6_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                 cudaStream_t st);
+lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                 const lr_grads& gr, char* ws, cudaStream_t st);
+
+size_t chunk_ws_bytes(const lr_desc& d, bool bwd);
+size_t chunk_flag_bytes(const lr_desc& d, bool bwd);
+lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                    cudaStream_t st);
+lr_status chunk_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                    const lr_grads& gr, char* ws, cudaStream_t st);
+
+}  // namespace lrs

@@ -6,7 +6,8 @@ so that both sides see bit-identical inputs.
 
 Draw order is fixed (the order of the ``_draw`` calls below) and every tensor is drawn in fp32 on
 the generator's device and then rounded to the I/O dtype (round-to-nearest-even for bf16).
-Parameters (``A``, ``D``, ``mag``, ``theta``) stay fp32.
+Parameters (``A``, ``Dskip``, ``mag``, ``theta``) stay fp32.  Key names follow the C ABI's
+``lr_inputs`` members (``Bm``, ``Cm``, ``Dskip`` for the selective scans' B, C and D).
 
 Workloads (token-major layouts, last index contiguous):
 
@@ -92,8 +93,8 @@ def s6(B, L, D, N, seed=0, io="bf16", device="cpu", with_z=True, with_D=True):
     z = r.randn(B, L, D)
     dy = r.randn(B, L, D)
     t = _DT[io]
-    return {"x": x.to(t), "delta": delta.to(t), "A": A.contiguous(), "B": Bm.to(t),
-            "C": Cm.to(t), "D": Dskip if with_D else None, "z": z.to(t) if with_z else None,
+    return {"x": x.to(t), "delta": delta.to(t), "A": A.contiguous(), "Bm": Bm.to(t),
+            "Cm": Cm.to(t), "Dskip": Dskip if with_D else None, "z": z.to(t) if with_z else None,
             "dy": dy.to(t)}
 
 
@@ -110,8 +111,8 @@ def ssd(B, L, H, P, N, G=1, seed=0, io="bf16", device="cpu", with_z=False, with_
     dy = r.randn(B, L, H, P)
     z = r.randn(B, L, H, P) if with_z else None
     t = _DT[io]
-    return {"x": x.to(t), "delta": delta.to(t), "A": A, "B": Bm.to(t), "C": Cm.to(t),
-            "D": Dskip if with_D else None, "z": z.to(t) if z is not None else None,
+    return {"x": x.to(t), "delta": delta.to(t), "A": A, "Bm": Bm.to(t), "Cm": Cm.to(t),
+            "Dskip": Dskip if with_D else None, "z": z.to(t) if z is not None else None,
             "dy": dy.to(t)}
 
 

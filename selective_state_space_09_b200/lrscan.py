@@ -1,0 +1,274 @@
+"""Thin Python binding of the C ABI in ``include/lrscan.h`` (argument marshalling only).
+
+Every step of the scan runs in the CUDA library ``_lrscan.so``; this module only builds the
+descriptor and pointer structs from torch tensors and passes torch's current CUDA stream.  torch
+supplies device memory and streams, nothing else.  Importing it without the built library raises
+``ImportError``: there is no CPU fallback.
+
+Layouts and dtypes are those of the header (token-major, row-major).  ``Plan`` holds the
+checkpoint buffer and workspace of one problem so that repeated calls allocate nothing.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lrscan.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError("CUDA scan library %s is not built (run selective_state_space_09_b200/build.py "
+                      "or __graft_entry__.build())" % LIB_PATH)
+
+KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
+DISC = {"none": 0, "zoh": 1, "bilinear": 2}
+IO = {torch.float32: 0, torch.bfloat16: 1}
+HAS_Z, HAS_DSKIP = 1, 2
+STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
+          "workspace too small", "CUDA runtime error", "device wait timed out",
+          "device consistency check failed"]
+
+
+class LrScanError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = int(status)
+        msg = lib.lr_status_string(self.status).decode()
+        super().__init__("%s: %s (status %d)" % (where, msg, self.status))
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("disc", ctypes.c_int32), ("io", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("B", ctypes.c_int64), ("L", ctypes.c_int64),
+                ("D", ctypes.c_int64), ("H", ctypes.c_int64), ("P", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("G", ctypes.c_int64), ("chunk", ctypes.c_int32),
+                ("segment", ctypes.c_int32)]
+
+
+_IN = ["a", "b", "g", "mag", "theta", "x", "delta", "A", "Bm", "Cm", "Dskip", "z", "q", "k", "v"]
+_GR = ["da", "db", "dg", "dmag", "dtheta", "dx", "ddelta", "dA", "dBm", "dCm", "dDskip", "dz",
+       "dq", "dk", "dv"]
+
+
+class Inputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _IN]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _GR]
+
+
+def _load():
+    L = ctypes.CDLL(LIB_PATH)
+    vp, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    pd = ctypes.POINTER(Desc)
+    L.lr_validate.argtypes = [pd]
+    L.lr_validate.restype = st
+    L.lr_ckpt_bytes.argtypes = [pd]
+    L.lr_ckpt_bytes.restype = sz
+    L.lr_workspace_bytes.argtypes = [pd, ctypes.c_int]
+    L.lr_workspace_bytes.restype = sz
+    L.lr_scan_fwd.argtypes = [pd, ctypes.POINTER(Inputs), vp, vp, vp, sz, vp]
+    L.lr_scan_fwd.restype = st
+    L.lr_scan_bwd.argtypes = [pd, ctypes.POINTER(Inputs), vp, vp, ctypes.POINTER(Grads), vp, sz, vp]
+    L.lr_scan_bwd.restype = st
+    L.lr_get_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    L.lr_get_error.restype = st
+    L.lr_status_string.argtypes = [st]
+    L.lr_status_string.restype = ctypes.c_char_p
+    L.lr_last_dispatch.restype = ctypes.c_char_p
+    L.lr_last_launch_count.restype = ctypes.c_int
+    L.lr_version.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def make_desc(kind, io=torch.float32, B=1, L=1, D=0, H=0, P=0, N=0, G=0, segment=1, chunk=0,
+              disc="none", has_z=False, has_d=False):
+    return Desc(KIND[kind], DISC[disc], IO[io], (HAS_Z if has_z else 0) | (HAS_DSKIP if has_d else 0),
+                B, L, D, H, P, N, G, chunk, segment)
+
+
+def validate(desc):
+    return int(lib.lr_validate(ctypes.byref(desc)))
+
+
+def ckpt_bytes(desc):
+    return int(lib.lr_ckpt_bytes(ctypes.byref(desc)))
+
+
+def workspace_bytes(desc, backward):
+    return int(lib.lr_workspace_bytes(ctypes.byref(desc), 1 if backward else 0))
+
+
+def last_dispatch():
+    return lib.lr_last_dispatch().decode()
+
+
+def last_launch_count():
+    return int(lib.lr_last_launch_count())
+
+
+def _check(status, where):
+    if status != 0:
+        raise LrScanError(status, where)
+
+
+class Plan:
+    """Checkpoint buffer and workspace of one problem, allocated once on ``device``."""
+
+    def __init__(self, desc, device="cuda"):
+        s = validate(desc)
+        if s != 0:
+            raise LrScanError(s, "lr_validate")
+        self.desc = desc
+        self.device = torch.device(device)
+        nck = ckpt_bytes(desc)
+        nws = max(workspace_bytes(desc, False), workspace_bytes(desc, True))
+        self.ckpt = torch.empty(max(nck // 4, 4), dtype=torch.float32, device=self.device)
+        self.ws = torch.empty(max((nws + 15) // 16, 16), dtype=torch.float32, device=self.device).view(torch.uint8)
+        self.ws_bytes = self.ws.numel()
+
+    def fwd(self, inp, y):
+        """inp: dict of tensors named as in ``Inputs`` (a, b, g, mag, theta, x, delta, A, Bm,
+        Cm, Dskip, z, q, k, v); y: output tensor (written)."""
+        ii = Inputs(*[_ptr(inp.get(n)) for n in _IN])
+        _check(lib.lr_scan_fwd(ctypes.byref(self.desc), ctypes.byref(ii), _ptr(y), _ptr(self.ckpt),
+                               _ptr(self.ws), self.ws_bytes, _stream()), "lr_scan_fwd")
+        return y
+
+    def bwd(self, inp, dy, grads):
+        """grads: dict of output tensors named as in ``Grads`` (written)."""
+        ii = Inputs(*[_ptr(inp.get(n)) for n in _IN])
+        gg = Grads(*[_ptr(grads.get(n)) for n in _GR])
+        _check(lib.lr_scan_bwd(ctypes.byref(self.desc), ctypes.byref(ii), _ptr(dy), _ptr(self.ckpt),
+                               ctypes.byref(gg), _ptr(self.ws), self.ws_bytes, _stream()), "lr_scan_bwd")
+        return grads
+
+    def device_error(self):
+        """Synchronises and returns (status, info) of the device-side error record."""
+        info = ctypes.c_int32(0)
+        s = lib.lr_get_error(_ptr(self.ws), _stream(), ctypes.byref(info))
+        return int(s), int(info.value)
+
+    def ckpt_view(self):
+        """The checkpoint buffer as an f32 tensor of ceil(L/S) states."""
+        d = self.desc
+        nseg = (d.L + d.segment - 1) // d.segment
+        shapes = {0: (nseg, d.B, d.D), 1: (nseg, d.B, d.D), 2: (nseg, d.B, d.D, d.N),
+                  3: (nseg, d.B, d.H, d.P, d.N), 4: (nseg, d.B, d.H, d.N, d.P)}
+        shp = shapes[d.kind]
+        n = 1
+        for s in shp:
+            n *= s
+        return self.ckpt[:n].view(*shp)
+
+
+# ------------------------------------------------------------------ per-kind convenience plans
+def plan_for(kind, inp, segment, disc="none", chunk=0):
+    """Build the Plan of a kind from its input tensors (shapes read from the tensors)."""
+    if kind == "rglru":
+        B, L, D = inp["a"].shape
+        d = make_desc("rglru", inp["a"].dtype, B, L, D=D, segment=segment)
+    elif kind == "rotlru":
+        B, L, D = inp["b"].shape
+        d = make_desc("rotlru", inp["b"].dtype, B, L, D=D, segment=segment)
+    elif kind == "s6":
+        B, L, D = inp["x"].shape
+        N = inp["A"].shape[1]
+        d = make_desc("s6", inp["x"].dtype, B, L, D=D, N=N, segment=segment, disc=disc,
+                      has_z=inp.get("z") is not None, has_d=inp.get("Dskip") is not None)
+    elif kind == "ssd":
+        B, L, H, P = inp["x"].shape
+        G, N = inp["Bm"].shape[2], inp["Bm"].shape[3]
+        d = make_desc("ssd", inp["x"].dtype, B, L, H=H, P=P, N=N, G=G, segment=segment,
+                      chunk=chunk, disc=disc, has_z=inp.get("z") is not None,
+                      has_d=inp.get("Dskip") is not None)
+    elif kind == "gla":
+        B, L, H, K = inp["q"].shape
+        V = inp["v"].shape[3]
+        d = make_desc("gla", inp["q"].dtype, B, L, H=H, P=V, N=K, segment=segment, chunk=chunk)
+    else:
+        raise KeyError(kind)
+    return Plan(d, inp[next(k for k in inp if inp[k] is not None)].device)
+
+
+def alloc_outputs(kind, inp):
+    """Output tensor and empty gradient tensors for a kind (shapes/dtypes of the header)."""
+    e = torch.empty_like
+    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
+    if kind == "rglru":
+        return e(inp["b"]), {"da": e(inp["a"]), "db": e(inp["b"])}
+    if kind == "rotlru":
+        return e(inp["b"]), {"db": e(inp["b"]), "dg": e(inp["g"]), "dmag": e(inp["mag"]),
+                             "dtheta": e(inp["theta"])}
+    if kind in ("s6", "ssd"):
+        g = {"dx": e(inp["x"]), "ddelta": e(inp["delta"]), "dA": e(inp["A"]), "dBm": f32(inp["Bm"]),
+             "dCm": f32(inp["Cm"])}
+        if inp.get("Dskip") is not None:
+            g["dDskip"] = e(inp["Dskip"])
+        if inp.get("z") is not None:
+            g["dz"] = e(inp["z"])
+        return e(inp["x"]), g
+    if kind == "gla":
+        return e(inp["v"]), {"dq": e(inp["q"]), "dk": e(inp["k"]), "dv": e(inp["v"]), "dg": e(inp["g"])}
+    raise KeyError(kind)
+
+
+# ---------------------------------------------------------------------- autograd wrappers
+class _ScanFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, kind, names, segment, disc, chunk, *tensors):
+        inp = {n: t.contiguous() if t is not None else None for n, t in zip(names, tensors)}
+        plan = plan_for(kind, inp, segment, disc, chunk)
+        y, _ = alloc_outputs(kind, inp)
+        plan.fwd(inp, y)
+        ctx.kind, ctx.names, ctx.plan = kind, names, plan
+        ctx.save_for_backward(*[inp[n] for n in names])
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        inp = dict(zip(ctx.names, ctx.saved_tensors))
+        _, grads = alloc_outputs(ctx.kind, inp)
+        ctx.plan.bwd(inp, dy.contiguous(), grads)
+        out = []
+        for n in ctx.names:
+            t = inp[n]
+            out.append(grads.get("d" + n) if t is not None else None)
+        return (None, None, None, None, None) + tuple(out)
+
+
+def rglru(a, b, segment=128):
+    """y = rglru_scan(a, b): h_t = a_t h_{t-1} + b_t, y_t = h_t.  a, b: [B, L, D]."""
+    return _ScanFn.apply("rglru", ("a", "b"), segment, "none", 0, a, b)
+
+
+def rotlru(b, g, mag, theta, segment=256):
+    """y = rotlru_scan: lambda_t = mag g_t e^{i theta}, h_t = lambda_t h_{t-1} + b_t (pairs)."""
+    return _ScanFn.apply("rotlru", ("b", "g", "mag", "theta"), segment, "none", 0, b, g, mag, theta)
+
+
+def s6(x, delta, A, B, C, D=None, z=None, disc="zoh", segment=256):
+    """Selective scan S6 with fused D skip and silu(z) gate.  x, delta, z: [B, L, D]."""
+    return _ScanFn.apply("s6", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z"), segment, disc, 0,
+                         x, delta, A, B, C, D, z)
+
+
+def ssd(x, delta, A, B, C, D=None, z=None, disc="zoh", chunk=64, segment=256):
+    """Head-wise SSD scan.  x, z: [B, L, H, P]; delta: [B, L, H]; B, C: [B, L, G, N]."""
+    return _ScanFn.apply("ssd", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z"), segment, disc, chunk,
+                         x, delta, A, B, C, D, z)
+
+
+def gla(q, k, v, g, chunk=64, segment=256):
+    """GLA scan: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t."""
+    return _ScanFn.apply("gla", ("q", "k", "v", "g"), segment, "none", chunk, q, k, v, g)

@@ -1,0 +1,108 @@
+"""Host-side tests of the C-ABI library (no GPU needed): it loads, exports every function the
+header declares, and its validation / size queries follow the documented rules.  No call here
+reaches a CUDA runtime function."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lrscan.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from selective_state_space_09_b200 import build
+    build.build()
+    from selective_state_space_09_b200 import lrscan
+    return lrscan
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(lr_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["lr_scan_fwd", "lr_scan_bwd", "lr_ckpt_bytes", "lr_workspace_bytes",
+              "lr_get_error", "lr_status_string", "lr_last_dispatch", "lr_validate"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    so = ctypes.CDLL(L.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(so, n), n
+
+
+def test_status_strings(L):
+    for s, want in enumerate(L.STATUS):
+        assert L.lib.lr_status_string(s).decode() == want
+    assert L.lib.lr_version() == 1
+
+
+def _ok(lrs, **kw):
+    return lrs.validate(lrs.make_desc(**kw))
+
+
+def test_validation_rules(L):
+    import torch
+    f32, bf = torch.float32, torch.bfloat16
+    assert _ok(L, kind="rglru", io=f32, B=1, L=1024, D=256, segment=128) == 0
+    assert _ok(L, kind="rglru", io=f32, B=1, L=1, D=4, segment=1) == 0
+    assert _ok(L, kind="rglru", io=f32, B=1, L=10, D=3, segment=4) == 3        # 12 B rows
+    assert _ok(L, kind="rglru", io=f32, B=0, L=10, D=4, segment=4) == 1
+    assert _ok(L, kind="rglru", io=f32, B=1, L=10, D=4, segment=0) == 1
+    assert _ok(L, kind="rglru", io=f32, B=1, L=1000, D=4, segment=512) == 2    # S > 256
+    assert _ok(L, kind="rglru", io=f32, B=1, L=10, D=4, segment=4, disc="zoh") == 1
+    assert _ok(L, kind="rotlru", io=f32, B=16, L=16384, D=4096, segment=256) == 0
+    assert _ok(L, kind="rotlru", io=f32, B=1, L=8, D=5, segment=4) == 1        # odd D
+    assert _ok(L, kind="rotlru", io=f32, B=1, L=8, D=4, segment=4) == 3        # g rows 8 B
+    # kinds whose kernels a build lacks report UNSUPPORTED (2) for otherwise valid requests
+    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256, disc="zoh") in (0, 2)
+    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256) == 1  # no disc
+    assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=256,
+               chunk=64, disc="zoh") in (0, 2)
+    assert _ok(L, kind="ssd", io=bf, B=2, L=64, H=32, P=64, N=128, G=3, segment=64,
+               disc="zoh") == 1                                                  # H % G
+    assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=256, chunk=64) in (0, 2)
+    assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=256,
+               disc="zoh") == 1
+
+
+def test_size_queries(L):
+    import torch
+    d = L.make_desc("rotlru", torch.float32, B=16, L=16384, D=4096, segment=256)
+    assert L.ckpt_bytes(d) == 64 * 16 * 4096 * 4                    # 16 MiB of checkpoints
+    assert L.workspace_bytes(d, False) > 256 and L.workspace_bytes(d, True) > 256
+    d = L.make_desc("rglru", torch.float32, B=1, L=1000, D=256, segment=128)
+    assert L.ckpt_bytes(d) == 8 * 1 * 256 * 4                       # ceil(1000/128) = 8
+    bad = L.make_desc("rglru", torch.float32, B=1, L=1000, D=3, segment=128)
+    assert L.ckpt_bytes(bad) == 0 and L.workspace_bytes(bad, True) == 0
+
+
+def test_calls_rejected_before_any_launch(L):
+    """Invalid requests return their status from host-side validation (no CUDA call made)."""
+    import torch
+    d = L.make_desc("rglru", torch.float32, B=1, L=16, D=32, segment=8)
+    ii = L.Inputs()  # all NULL
+    s = L.lib.lr_scan_fwd(ctypes.byref(d), ctypes.byref(ii), None, None, None, 0, None)
+    assert s == 1
+    bad = L.make_desc("rglru", torch.float32, B=1, L=16, D=6, segment=8)
+    s = L.lib.lr_scan_fwd(ctypes.byref(bad), ctypes.byref(ii), None, None, None, 0, None)
+    assert s == 3
+    # misaligned pointer
+    ii = L.Inputs(a=ctypes.c_void_p(0x1004), b=ctypes.c_void_p(0x2000))
+    s = L.lib.lr_scan_fwd(ctypes.byref(d), ctypes.byref(ii), ctypes.c_void_p(0x3000),
+                          ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), 1 << 20, None)
+    assert s == 3
+    # workspace too small
+    ii = L.Inputs(a=ctypes.c_void_p(0x1000), b=ctypes.c_void_p(0x2000))
+    s = L.lib.lr_scan_fwd(ctypes.byref(d), ctypes.byref(ii), ctypes.c_void_p(0x3000),
+                          ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), 16, None)
+    assert s == 4
+    assert L.last_launch_count() == 0

@@ -1,0 +1,122 @@
+"""GPU parity of the diagonal kinds (rglru_scan, rotlru_scan) against the fp64 oracle.
+
+Cases span several tiles and ragged tails in time (L not a multiple of the segment) and in
+channels (D not a multiple of the 32-channel tile), the degenerate L = 1 / S = 1 / L < S cases,
+bf16 I/O, the rglru workload at full size and the long-sequence rotlru workload at full size on
+sampled units.  Tolerance: max|err| <= 1e-5 max|ref| for fp32 I/O, 2e-2 for bf16, per tensor
+(y, checkpoints and every gradient).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import TOL, assert_close, run_gpu, to64
+from selective_state_space_09_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+RGLRU_CASES = [
+    # B, L, D, S, io
+    (1, 1024, 256, 128, "f32"),     # the rglru workload itself
+    (2, 1000, 96, 64, "f32"),       # ragged L, 3 channel blocks
+    (3, 37, 40, 8, "f32"),          # ragged channels (40 = 32 + 8)
+    (1, 1, 32, 1, "f32"),           # single step
+    (2, 5, 64, 16, "f32"),          # L < S
+    (1, 700, 64, 256, "f32"),       # maximum segment
+    (2, 300, 128, 100, "bf16"),
+    (1, 129, 8, 1, "f32"),          # S = 1: a checkpoint every step
+]
+
+
+@pytest.mark.parametrize("B,L,D,S,io", RGLRU_CASES)
+def test_rglru_parity(B, L, D, S, io):
+    inp = inputs.rglru(B, L, D, seed=B * 1000 + L, io=io)
+    y, ck, gr, plan, disp = run_gpu("rglru", inp, S)
+    tol = TOL[inp["a"].dtype]
+    ry, rck = oracle.rglru_fwd(inp["a"], inp["b"], S=S)
+    rg = oracle.rglru_bwd(inp["a"], inp["b"], inp["dy"])
+    assert_close("y", y, ry, tol)
+    assert_close("ckpt", ck, rck, max(tol, 1e-5))
+    assert_close("da", gr["da"], rg["a"], tol)
+    assert_close("db", gr["db"], rg["b"], tol)
+    assert disp == ("rglru_fwd_tile", "rglru_bwd_tile")
+    assert plan.device_error() == (0, 0)
+
+
+ROTLRU_CASES = [
+    (2, 1000, 64, 64, "f32"),
+    (1, 333, 40, 256, "f32"),       # 20 pairs: ragged pair block
+    (3, 17, 8, 4, "f32"),
+    (2, 600, 64, 128, "bf16"),
+    (1, 1, 32, 1, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,L,D,S,io", ROTLRU_CASES)
+def test_rotlru_parity(B, L, D, S, io):
+    inp = inputs.rotlru(B, L, D, seed=B * 1000 + L, io=io)
+    y, ck, gr, plan, disp = run_gpu("rotlru", inp, S)
+    tol = TOL[inp["b"].dtype]
+    ry, rck = oracle.rotlru_fwd(inp["b"], inp["g"], inp["mag"], inp["theta"], S=S)
+    rg = oracle.rotlru_bwd(inp["b"], inp["g"], inp["mag"], inp["theta"], inp["dy"])
+    assert_close("y", y, ry, tol)
+    assert_close("ckpt", ck, rck, max(tol, 1e-5))
+    assert_close("db", gr["db"], rg["b"], tol)
+    assert_close("dg", gr["dg"], rg["g"], tol)
+    assert_close("dmag", gr["dmag"], rg["mag"], max(tol, 1e-5))
+    assert_close("dtheta", gr["dtheta"], rg["theta"], max(tol, 1e-5))
+    assert disp == ("rotlru_fwd_tile", "rotlru_bwd_tile+rotlru_param_reduce")
+    assert plan.device_error() == (0, 0)
+
+
+def test_diag_deterministic():
+    """Two runs give bitwise-identical outputs (no order-dependent reductions, no races)."""
+    inp = inputs.rotlru(2, 777, 96, seed=5)
+    a = run_gpu("rotlru", inp, 64)
+    b = run_gpu("rotlru", inp, 64)
+    for k in ("db", "dg", "dmag", "dtheta"):
+        assert torch.equal(a[2][k], b[2][k]), k
+    assert torch.equal(a[0], b[0])
+
+
+def test_withheld_carry_times_out_and_context_survives():
+    """Failure path: tiles of the first segment withhold their carry; later tiles wait out
+    their bound, record LR_ERR_TIMEOUT (status 6) and finish.  A normal call afterwards on the
+    same context is correct."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.rglru(1, 256, 32, seed=3)
+    y, ck, gr, plan, _ = run_gpu("rglru", inp, 64, flags=0x80000000)
+    status, info = plan.device_error()
+    assert status == 6 and info in (101, 201)
+    y, ck, gr, plan, _ = run_gpu("rglru", inp, 64)
+    assert plan.device_error() == (0, 0)
+    assert_close("y", y, oracle.rglru_fwd(inp["a"], inp["b"]), 1e-5)
+
+
+@pytest.mark.slow
+def test_rotlru_full_size_sampled():
+    """The long-sequence rotlru workload (B=16, D=4096, L=16384, S=256) on the GPU; the oracle
+    recomputes sampled pairs (all batch rows of a pair, so the parameter gradients, which sum
+    over batch and time, are checked too)."""
+    w = inputs.WORKLOADS["rotlru"]
+    inp = inputs.rotlru(w["B"], w["L"], w["D"], seed=0, device="cuda")
+    y, ck, gr, plan, _ = run_gpu("rotlru", inp, w["segment"])
+    assert plan.device_error() == (0, 0)
+    rng = np.random.default_rng(0)
+    pairs = sorted(set([0, w["D"] // 2 - 1] + list(rng.integers(0, w["D"] // 2, size=4))))
+    oracle.set_threads(8)
+    for k in pairs:
+        sl = slice(2 * k, 2 * k + 2)
+        b = to64(inp["b"][:, :, sl])
+        g = to64(inp["g"][:, :, k:k + 1])
+        mag, th = to64(inp["mag"][k:k + 1]), to64(inp["theta"][k:k + 1])
+        dy = to64(inp["dy"][:, :, sl])
+        ry, rck = oracle.rotlru_fwd(b, g, mag, th, S=w["segment"])
+        rg = oracle.rotlru_bwd(b, g, mag, th, dy)
+        assert_close("y[%d]" % k, y[:, :, sl], ry, 1e-5)
+        assert_close("ckpt[%d]" % k, ck[:, :, sl], rck, 1e-5)
+        assert_close("db[%d]" % k, gr["db"][:, :, sl], rg["b"], 1e-5)
+        assert_close("dg[%d]" % k, gr["dg"][:, :, k:k + 1], rg["g"], 1e-5)
+        assert_close("dmag[%d]" % k, gr["dmag"][k:k + 1], rg["mag"], 1e-5)
+        assert_close("dtheta[%d]" % k, gr["dtheta"][k:k + 1], rg["theta"], 1e-5)

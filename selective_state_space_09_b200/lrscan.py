@@ -134,7 +134,7 @@ class Plan:
         nck = ckpt_bytes(desc)
         nws = max(workspace_bytes(desc, False), workspace_bytes(desc, True))
         self.ckpt = torch.empty(max(nck // 4, 4), dtype=torch.float32, device=self.device)
-        self.ws = torch.empty(max((nws + 15) // 16, 16), dtype=torch.float32, device=self.device).view(torch.uint8)
+        self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=self.device)
         self.ws_bytes = self.ws.numel()
 
     def fwd(self, inp, y):

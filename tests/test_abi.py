@@ -106,3 +106,13 @@ def test_calls_rejected_before_any_launch(L):
                           ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), 16, None)
     assert s == 4
     assert L.last_launch_count() == 0
+
+
+def test_plan_buffers_cover_the_queried_sizes(L):
+    import torch
+    for d in (L.make_desc("rotlru", torch.float32, B=2, L=1000, D=64, segment=64),
+              L.make_desc("rglru", torch.bfloat16, B=3, L=77, D=96, segment=16)):
+        p = L.Plan(d, "cpu")
+        assert p.ws_bytes >= max(L.workspace_bytes(d, False), L.workspace_bytes(d, True))
+        assert p.ckpt.numel() * 4 >= L.ckpt_bytes(d)
+        assert p.ckpt_view().shape[0] == (d.L + d.segment - 1) // d.segment

@@ -169,6 +169,35 @@ __device__ __forceinline__ Agg<V> ld_cg_agg(const Agg<V>* p) {
     return {ld_cg(&p->m), ld_cg(&p->v)};
 }
 
+// Carry entering tile k of a row, deterministic whatever the timing: walk towards the start
+// of the chain (dir = -1: earlier segments, forward pass; dir = +1: later segments, backward
+// pass) until a tile that has published its inclusive prefix (or the end of the row), then fold
+// the aggregates of the tiles in between in chain order, x <- m x + v.  That is the same
+// sequence of operations as a purely chained scan, so the result does not depend on which
+// records happened to be ready.  Waits are bounded; a wait that gives up counts as a zero
+// prefix (the error is recorded).
+template <typename V>
+__device__ V lookback_carry(const unsigned int* flags, const Agg<V>* aggRec, const V* preRec,
+                            size_t row, int k, int dir, int nseg, int CB, int lane, bool act,
+                            WsHeader* hdr, int info) {
+    int j = k + dir;
+    V x = zero_of(V{});
+    while (j >= 0 && j < nseg) {
+        unsigned int f = wait_flag(&flags[row + j], hdr, info);
+        if (f == kFlagPrefix) {
+            if (act) x = ld_cg(&preRec[(row + j) * CB + lane]);
+            break;
+        }
+        if (f != kFlagAgg) break;  // gave up: zero prefix
+        j += dir;
+    }
+    for (int i = j - dir; i != k; i -= dir) {
+        Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + i) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
+        x = fmax_(ag.m, x, ag.v);
+    }
+    return x;
+}
+
 // Dynamic shared memory, re-aligned to 128 bytes.
 __device__ __forceinline__ char* smem_base() {
     extern __shared__ char dyn_smem[];
@@ -256,28 +285,8 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             __syncwarp();
             if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
         }
-        V carry = zero_of(V{});
-        if (seg > 0) {
-            V Pc = one_of(V{}), hc = zero_of(V{});
-            int j = seg - 1;
-            while (true) {
-                unsigned int f = wait_flag(&a.flags[row + j], a.hdr, 101);
-                if (f == kFlagPrefix) {
-                    V st = act ? ld_cg(&preRec[(row + j) * CB + lane]) : zero_of(V{});
-                    carry = fmax_(Pc, st, hc);
-                    break;
-                }
-                if (f == kFlagAgg) {
-                    Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + j) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
-                    hc = fmax_(Pc, ag.v, hc);
-                    Pc = mulx(Pc, ag.m);
-                    if (--j < 0) { carry = hc; break; }
-                    continue;
-                }
-                carry = hc;  // gave up (error recorded): continue with what is known
-                break;
-            }
-        }
+        const V carry = lookback_carry(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane, act,
+                                       a.hdr, 101);
         const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == 0;
         if (has_succ && !withhold) {
             if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));
@@ -436,28 +445,8 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             __syncwarp();
             if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
         }
-        V carry = zero_of(V{});
-        if (seg + 1 < a.nseg) {
-            V Mc = one_of(V{}), vc = zero_of(V{});
-            int j = seg + 1;
-            while (true) {
-                unsigned int f = wait_flag(&a.flags[row + j], a.hdr, 201);
-                if (f == kFlagPrefix) {
-                    V st = act ? ld_cg(&preRec[(row + j) * CB + lane]) : zero_of(V{});
-                    carry = fmax_(Mc, st, vc);
-                    break;
-                }
-                if (f == kFlagAgg) {
-                    Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + j) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
-                    vc = fmax_(Mc, ag.v, vc);
-                    Mc = mulx(Mc, ag.m);
-                    if (++j >= a.nseg) { carry = vc; break; }
-                    continue;
-                }
-                carry = vc;
-                break;
-            }
-        }
+        const V carry = lookback_carry(a.flags, aggRec, preRec, row, seg, +1, a.nseg, CB, lane, act,
+                                       a.hdr, 201);
         const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == a.nseg - 1;
         if (has_pred && !withhold) {
             if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));

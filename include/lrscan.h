@@ -177,6 +177,31 @@ int lr_last_launch_count(void);
 
 int lr_version(void);
 
+/* lr_rglru_fwd_noalloc -- the rglru forward pass for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists for deployment, not for the method.
+ *
+ * Who needs it: code that runs inside a framework owning every device byte through its own pool
+ * (and offering no scratch buffer to plug-ins), hosts that only let a plug-in run a fixed
+ * callback on the tensors they hand over, and latency-critical loops where cudaMalloc / cudaFree
+ * would synchronise the device.  Such callers cannot provide the workspace lr_scan_fwd needs.
+ *
+ * It computes exactly what lr_scan_fwd computes for LR_RGLRU (same kernel): y [B, L, D] and the
+ * segment checkpoints `ckpt` (lr_ckpt_bytes(desc) bytes), from device inputs a, b.  Its scratch
+ * is a 1 MiB array inside the library (held by every GPU that loads the library until the
+ * process exits); the call allocates nothing.  Limit: problems whose forward workspace
+ * (lr_workspace_bytes(desc, 0), about 390 bytes per tile of 32 channels x S steps per batch row)
+ * exceeds 1 MiB are rejected with LR_ERR_WORKSPACE.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All calls on a device
+ * share the array and each call clears the part that must start at zero, so calls that overlap
+ * on the GPU (unordered streams) race and must be avoided.  With `check` non-zero the call
+ * synchronises `stream` and returns the kernel's device-side status (LR_ERR_TIMEOUT if a bounded
+ * wait gave up); otherwise it returns once the work is enqueued.  Other statuses as
+ * lr_scan_fwd (LR_ERR_INVALID_ARG also for a kind other than LR_RGLRU). */
+lr_status lr_rglru_fwd_noalloc(const lr_desc *desc, const void *a, const void *b, void *y,
+                               void *ckpt, void *stream, int check);
+
 #ifdef __cplusplus
 }
 #endif

@@ -97,6 +97,8 @@ void begin_call() {
 
 }  // namespace
 
+void reset_dispatch() { begin_call(); }
+
 void note_launch(const char* name) {
     if (!t_dispatch.empty()) t_dispatch += "+";
     t_dispatch += name;

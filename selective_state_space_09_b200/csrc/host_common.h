@@ -17,6 +17,9 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // lr_last_dispatch / lr_last_launch_count).
 void note_launch(const char* name);
 
+// Clears this host thread's launch fingerprint (start of an entry-point call).
+void reset_dispatch();
+
 // Converts the last CUDA error into a status.
 lr_status check_launch();
 

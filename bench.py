@@ -38,8 +38,8 @@ NAMES = {
     "ssd": "Mamba-2 SSD scan (mamba-370m-like), bf16, B=2 H=32 P=64 N=128 L=4096, chunk 64, S=256, ZOH",
     "rglru": "rglru_scan, f32, B=1 D=256 L=1024, S=128",
     "gla": "GLA scan, bf16, B=4 H=16 K=V=128 L=2048, chunk 64, S=256",
-    "s6_zoh": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=256, ZOH, D skip + silu(z)",
-    "s6_bilinear": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=256, bilinear, D skip + silu(z)",
+    "s6_zoh": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, ZOH, D skip + silu(z)",
+    "s6_bilinear": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, bilinear, D skip + silu(z)",
     "rotlru": "rotlru_scan, f32, B=16 D=4096 L=16384, S=256",
 }
 INPUT_NAMES = {
@@ -152,10 +152,17 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ workloads
+BATCH_OVERRIDE = None  # --batch: a smaller batch of the same workload (profiling captures)
+
+
 def workload_inputs(name, device, seed):
     from selective_state_space_09_b200 import inputs
     w = dict(inputs.WORKLOADS[name])
-    inp = inputs.workload(name, seed=seed, device=device)
+    if BATCH_OVERRIDE:
+        w["B"] = BATCH_OVERRIDE
+        inp = inputs.workload(name, seed=seed, device=device, B=BATCH_OVERRIDE)
+    else:
+        inp = inputs.workload(name, seed=seed, device=device)
     return w, inp
 
 
@@ -428,7 +435,11 @@ def main():
     ap.add_argument("--workload", default=None, help="headline workload (default: ssd if built)")
     ap.add_argument("--only-headline", action="store_true", help="skip the per-kind lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (small profiling cases only)")
     args = ap.parse_args()
+    global BATCH_OVERRIDE
+    BATCH_OVERRIDE = args.batch
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

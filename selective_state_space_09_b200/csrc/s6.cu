@@ -1,0 +1,589 @@
+// s6.cu -- selective scan S6 (time-varying diagonal A with per-step dt, B, C), forward and
+// backward, fused D skip and silu(z) gate, ZOH or bilinear discretisation (sm_100a).
+//
+// Definition ("lrnnx: A library for Linear RNNs", ai.info summary, Key Contributions 2-3: time-
+// varying layers with ZOH / bilinear discretisation inside a fused scan and output projection):
+//   per (b, d, n):  abar, beta = disc(dt_t[d], A[d,n])
+//     ZOH:       abar = exp(dt A),              beta = (exp(dt A) - 1) / A
+//     bilinear:  abar = (1 + dt A/2)/(1 - dt A/2), beta = dt / (1 - dt A/2)
+//   h_t[n] = abar h_{t-1}[n] + beta B_t[n] x_t,   y_t = (sum_n C_t[n] h_t[n] + D x_t) silu(z_t).
+// Segment checkpoints and recompute follow the mlx-recurrence post (Apple Developer Forums
+// thread 840535, segment checkpointing with recomputation during the backward pass).
+//
+// Work split.  The scan is bound by the per-(t, d, n) arithmetic (one exp or reciprocal and a
+// handful of FMAs per state per step), not by HBM, so the layout keeps states in registers and
+// avoids cross-thread traffic on the recurrence: a CTA owns one batch row and 64 channels for the
+// whole sequence; two threads per channel (lanes l and l^16 of a warp) hold 8 of its 16 states
+// each, so the readout sum over n is one shuffle.  Segments of S <= 64 steps are staged in shared
+// memory by TMA (x, dt, z, dy as [S][64] bf16 tiles, B, C as [S][16]); outputs are written back
+// into the consumed tile slots and stored with TMA.  The forward pass double-buffers segments and
+// writes the state entering each segment to the checkpoint buffer.
+//
+// Backward, per segment in reverse order (the adjoint carry G stays in registers across
+// segments): (A) from the checkpoint, run the segment forward and keep the state at every 8-step
+// sub-block boundary in shared memory; (C) for each sub-block in reverse, recompute its 8 steps
+// keeping h_t and abar_t in registers, then run the adjoint recurrence
+// G_t[n] = ds_t C_t[n] + abar_{t+1} G_{t+1}[n] (ds = dy silu(z)) backwards through them and form
+// every gradient.  dB_t[n] and dC_t[n] (sums over channels) are reduced over the 16 channels of a
+// half-warp with a butterfly, then over the CTA's four warps in a fixed order, giving one partial
+// per 64-channel block; dA and dD partials are per batch row.  A small kernel sums the partials in
+// a fixed order (deterministic results).
+#include "common.cuh"
+#include "host_common.h"
+
+namespace lrs {
+namespace {
+
+constexpr int kDB = 64;       // channels per CTA
+constexpr int kNH = 8;        // states per thread (N = 16)
+constexpr int kN = 2 * kNH;
+constexpr int kThreads = 128; // 64 channels x 2 halves
+constexpr int kMaxS = 64;     // segment rows per TMA box
+constexpr int kSub = 8;       // backward sub-block length
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sigm(float z) { return rcp(1.0f + ex2(-z * kLog2e)); }
+__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// 8 consecutive bf16 -> float
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* out) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        out[2 * i] = f.x;
+        out[2 * i + 1] = f.y;
+    }
+}
+
+struct S6Args {
+    int B, L, D, S, nseg, ncb;
+    int disc;            // LR_DISC_ZOH / LR_DISC_BILINEAR
+    int has_z, has_d;
+    const float* A;      // [D, N]
+    const float* Dskip;  // [D]
+    float* ckpt;         // [nseg, B, D, N]
+    WsHeader* hdr;
+    float* pdB;          // [ncb, B, L, N]
+    float* pdC;          // [ncb, B, L, N]
+    float* pdA;          // [B, D, N]
+    float* pdD;          // [B, D]
+};
+
+// Per-thread constants of the discretisation for its 8 states.
+struct Disc {
+    float a2[kNH];  // ZOH: A log2(e); bilinear: A / 2
+    float ia[kNH];  // ZOH: 1 / A
+    float A[kNH];
+};
+
+template <int DISC>
+__device__ __forceinline__ void coef(const Disc& c, int j, float dt, float& ab, float& be) {
+    if (DISC == LR_DISC_ZOH) {
+        ab = ex2(dt * c.a2[j]);
+        be = (ab - 1.0f) * c.ia[j];
+    } else {
+        float r = rcp(fmaf(-dt, c.a2[j], 1.0f));
+        ab = fmaf(dt * c.a2[j], r, r);  // (1 + dt A/2) r
+        be = dt * r;
+    }
+}
+
+// beta from abar (cheaper than a second transcendental in the backward sweep)
+template <int DISC>
+__device__ __forceinline__ float beta_of(const Disc& c, int j, float dt, float ab) {
+    if (DISC == LR_DISC_ZOH) return (ab - 1.0f) * c.ia[j];
+    return dt * 0.5f * (ab + 1.0f);  // dt / (1 - dt A/2) = dt (abar + 1) / 2
+}
+
+__device__ __forceinline__ char* smem_base() {
+    extern __shared__ char dyn_smem[];
+    uintptr_t p = reinterpret_cast<uintptr_t>(dyn_smem);
+    return reinterpret_cast<char*>((p + 127) & ~uintptr_t(127));
+}
+
+constexpr size_t kTileDT = size_t(kMaxS) * kDB * 2;  // [S][64] bf16
+constexpr size_t kTileBC = size_t(kMaxS) * kN * 2;   // [S][16] bf16
+
+// ----------------------------------------------------------------------------------- forward
+// Shared memory per stage: X, DT, Z tiles and B, C tiles.
+constexpr size_t kFwdStage = 3 * kTileDT + 2 * kTileBC;
+constexpr size_t kFwdSmem = 128 + 2 * kFwdStage + 128;
+
+template <int DISC>
+__global__ void __launch_bounds__(kThreads)
+s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
+              const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mB,
+              const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mY, S6Args a) {
+    char* sm = smem_base();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);  // bar[0], bar[1]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = lane >> 4, dl = warp * 16 + (lane & 15);
+    const int b = blockIdx.x / a.ncb, cb = blockIdx.x % a.ncb;
+    const int d = cb * kDB + dl;
+    const bool dok = d < a.D;
+    auto stage = [&](int s, int which) -> char* { return sm + 128 + s * kFwdStage + which * kTileDT; };
+    auto stageBC = [&](int s, int which) -> __nv_bfloat16* {
+        return reinterpret_cast<__nv_bfloat16*>(sm + 128 + s * kFwdStage + 3 * kTileDT + which * kTileBC);
+    };
+    const uint32_t bytes = (uint32_t)(a.S * kDB * 2 * (a.has_z ? 3 : 2) + 2 * a.S * kN * 2);
+    auto issue = [&](int k, int s) {
+        mbar_arrive_expect_tx(&bar[s], bytes);
+        const int t0 = k * a.S;
+        tma_load_3d(stage(s, 0), &mX, &bar[s], cb * kDB, t0, b);
+        tma_load_3d(stage(s, 1), &mDT, &bar[s], cb * kDB, t0, b);
+        if (a.has_z) tma_load_3d(stage(s, 2), &mZ, &bar[s], cb * kDB, t0, b);
+        tma_load_3d(stageBC(s, 0), &mB, &bar[s], 0, t0, b);
+        tma_load_3d(stageBC(s, 1), &mC, &bar[s], 0, t0, b);
+    };
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        issue(0, 0);
+    }
+    Disc c;
+#pragma unroll
+    for (int j = 0; j < kNH; ++j) {
+        float A = dok ? a.A[(size_t)d * kN + half * kNH + j] : -1.0f;
+        c.A[j] = A;
+        c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
+        c.ia[j] = 1.0f / A;
+    }
+    const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
+    float h[kNH];
+#pragma unroll
+    for (int j = 0; j < kNH; ++j) h[j] = 0.0f;
+    __syncthreads();
+
+    bool ok = true;
+    for (int k = 0; k < a.nseg; ++k) {
+        const int s = k & 1;
+        if (tid == 0 && k + 1 < a.nseg) {
+            if (k >= 1) bulk_wait_read_all();  // store of segment k-1 has read stage s^1
+            issue(k + 1, s ^ 1);
+        }
+        ok = ok && mbar_wait(&bar[s], (k >> 1) & 1, a.hdr, 300);
+        if (dok) {
+            float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + half * kNH;
+#pragma unroll
+            for (int j = 0; j < kNH; ++j) ck[j] = h[j];
+        }
+        const int nt = min(a.S, a.L - k * a.S);
+        __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(stage(s, 0));
+        const __nv_bfloat16* DT = reinterpret_cast<const __nv_bfloat16*>(stage(s, 1));
+        const __nv_bfloat16* Z = reinterpret_cast<const __nv_bfloat16*>(stage(s, 2));
+        const __nv_bfloat16* Bs = stageBC(s, 0);
+        const __nv_bfloat16* Cs = stageBC(s, 1);
+        if (ok) {
+            for (int t = 0; t < nt; ++t) {
+                const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                float Bv[kNH], Cv[kNH];
+                ld8(Bs + t * kN + half * kNH, Bv);
+                ld8(Cs + t * kN + half * kNH, Cv);
+                float sacc = 0.0f;
+#pragma unroll
+                for (int j = 0; j < kNH; ++j) {
+                    float ab, be;
+                    coef<DISC>(c, j, dt, ab, be);
+                    h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
+                    sacc = fmaf(Cv[j], h[j], sacc);
+                }
+                sacc += __shfl_xor_sync(0xffffffffu, sacc, 16);
+                if (half == 0) {
+                    float yv = fmaf(Dd, xv, sacc);
+                    if (a.has_z) {
+                        const float zv = bf(Z + t * kDB + dl);
+                        yv *= zv * sigm(zv);
+                    }
+                    X[t * kDB + dl] = __float2bfloat16_rn(yv);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tma_store_3d(&mY, X, cb * kDB, k * a.S, b);
+            bulk_commit();
+        }
+    }
+    if (tid == 0) bulk_wait_read_all();
+}
+
+// ---------------------------------------------------------------------------------- backward
+// Shared memory: X, DT, Z, DY tiles, B, C tiles, sub-block boundary states, per-warp dB/dC.
+constexpr size_t kOffX = 128;
+constexpr size_t kOffB = kOffX + 4 * kTileDT;
+constexpr size_t kOffBnd = kOffB + 2 * kTileBC;
+constexpr size_t kBndBytes = size_t(kMaxS / kSub) * kThreads * kNH * 4;
+constexpr size_t kOffRed = kOffBnd + kBndBytes;
+constexpr size_t kRedBytes = size_t(4) * kMaxS * 2 * kN * 4;
+constexpr size_t kBwdSmem = kOffRed + kRedBytes + 128;
+
+template <int DISC>
+__global__ void __launch_bounds__(kThreads)
+s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
+              const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mDY,
+              const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
+              const __grid_constant__ CUtensorMap mdX, const __grid_constant__ CUtensorMap mdDT,
+              const __grid_constant__ CUtensorMap mdZ, S6Args a) {
+    char* sm = smem_base();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+    __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(sm + kOffX);
+    __nv_bfloat16* DT = reinterpret_cast<__nv_bfloat16*>(sm + kOffX + kTileDT);
+    __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(sm + kOffX + 2 * kTileDT);
+    __nv_bfloat16* DY = reinterpret_cast<__nv_bfloat16*>(sm + kOffX + 3 * kTileDT);
+    const __nv_bfloat16* Bs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB);
+    const __nv_bfloat16* Cs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB + kTileBC);
+    float* bnd = reinterpret_cast<float*>(sm + kOffBnd);  // [sub-block][thread][kNH]
+    float* red = reinterpret_cast<float*>(sm + kOffRed);  // [warp][t][2][kN]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = lane >> 4, q = lane & 15, dl = warp * 16 + q;
+    const int b = blockIdx.x / a.ncb, cb = blockIdx.x % a.ncb;
+    const int d = cb * kDB + dl;
+    const bool dok = d < a.D;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    Disc c;
+#pragma unroll
+    for (int j = 0; j < kNH; ++j) {
+        float A = dok ? a.A[(size_t)d * kN + half * kNH + j] : -1.0f;
+        c.A[j] = A;
+        c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
+        c.ia[j] = 1.0f / A;
+    }
+    const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
+    float G[kNH], anext[kNH], dA[kNH];
+#pragma unroll
+    for (int j = 0; j < kNH; ++j) G[j] = anext[j] = dA[j] = 0.0f;
+    float dD = 0.0f;
+    const uint32_t bytes = (uint32_t)(a.S * kDB * 2 * (a.has_z ? 4 : 3) + 2 * a.S * kN * 2);
+    __syncthreads();
+
+    bool ok = true;
+    int phase = 0;
+    for (int k = a.nseg - 1; k >= 0; --k, phase ^= 1) {
+        const int t0 = k * a.S;
+        const int nt = min(a.S, a.L - t0);
+        if (tid == 0) {
+            bulk_wait_read_all();  // previous segment's gradient tiles have left shared memory
+            mbar_arrive_expect_tx(&bar[0], bytes);
+            tma_load_3d(X, &mX, &bar[0], cb * kDB, t0, b);
+            tma_load_3d(DT, &mDT, &bar[0], cb * kDB, t0, b);
+            if (a.has_z) tma_load_3d(Z, &mZ, &bar[0], cb * kDB, t0, b);
+            tma_load_3d(DY, &mDY, &bar[0], cb * kDB, t0, b);
+            tma_load_3d(const_cast<__nv_bfloat16*>(Bs), &mB, &bar[0], 0, t0, b);
+            tma_load_3d(const_cast<__nv_bfloat16*>(Cs), &mC, &bar[0], 0, t0, b);
+        }
+        float h[kNH];
+        {
+            const float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + (dok ? d : 0)) * kN + half * kNH;
+#pragma unroll
+            for (int j = 0; j < kNH; ++j) h[j] = dok ? ck[j] : 0.0f;
+        }
+        ok = ok && mbar_wait(&bar[0], phase, a.hdr, 400);
+        const int nsb = (nt + kSub - 1) / kSub;
+        // (A) segment forward, keeping sub-block boundary states
+        for (int sb = 0; sb < nsb; ++sb) {
+            float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
+#pragma unroll
+            for (int j = 0; j < kNH; ++j) bp[j] = h[j];
+            const int te = min(nt, (sb + 1) * kSub);
+            for (int t = sb * kSub; t < te; ++t) {
+                const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                float Bv[kNH];
+                ld8(Bs + t * kN + half * kNH, Bv);
+#pragma unroll
+                for (int j = 0; j < kNH; ++j) {
+                    float ab, be;
+                    coef<DISC>(c, j, dt, ab, be);
+                    h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
+                }
+            }
+        }
+        // (C) sub-blocks in reverse: recompute into registers, then the adjoint sweep
+        for (int sb = nsb - 1; sb >= 0; --sb) {
+            const int tb = sb * kSub;
+            const int n = min(kSub, nt - tb);
+            float h0[kNH], hr[kSub][kNH], ar[kSub][kNH];
+            {
+                const float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
+#pragma unroll
+                for (int j = 0; j < kNH; ++j) h0[j] = h[j] = bp[j];
+            }
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) {
+                if (i < n) {
+                    const int t = tb + i;
+                    const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                    float Bv[kNH];
+                    ld8(Bs + t * kN + half * kNH, Bv);
+#pragma unroll
+                    for (int j = 0; j < kNH; ++j) {
+                        float ab, be;
+                        coef<DISC>(c, j, dt, ab, be);
+                        h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
+                        hr[i][j] = h[j];
+                        ar[i][j] = ab;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = kSub - 1; i >= 0; --i) {
+                if (i < n) {
+                    const int t = tb + i;
+                    const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                    const float dyv = bf(DY + t * kDB + dl);
+                    float Bv[kNH], Cv[kNH];
+                    ld8(Bs + t * kN + half * kNH, Bv);
+                    ld8(Cs + t * kN + half * kNH, Cv);
+                    // readout and gate
+                    float sacc = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < kNH; ++j) sacc = fmaf(Cv[j], hr[i][j], sacc);
+                    sacc += __shfl_xor_sync(0xffffffffu, sacc, 16);
+                    const float s = fmaf(Dd, xv, sacc);
+                    float ds = dyv, dz = 0.0f;
+                    if (a.has_z) {
+                        const float zv = bf(Z + t * kDB + dl);
+                        const float sg = sigm(zv);
+                        ds = dyv * zv * sg;
+                        dz = dyv * s * sg * fmaf(zv, 1.0f - sg, 1.0f);
+                    }
+                    float v[2 * kNH];  // dB (x n), dC (x n) contributions of this channel
+                    float dxa = 0.0f, dta = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < kNH; ++j) {
+                        const float ab = ar[i][j];
+                        const float be = beta_of<DISC>(c, j, dt, ab);
+                        const float hp = i > 0 ? hr[i > 0 ? i - 1 : 0][j] : h0[j];
+                        G[j] = fmaf(anext[j], G[j], ds * Cv[j]);
+                        v[kNH + j] = ds * hr[i][j];
+                        const float u = G[j] * be;
+                        v[j] = u * xv;
+                        dxa = fmaf(u, Bv[j], dxa);
+                        const float dab = G[j] * hp;
+                        const float w = G[j] * (Bv[j] * xv);  // d loss / d beta
+                        if (DISC == LR_DISC_ZOH) {
+                            dta = fmaf(dab, c.A[j] * ab, fmaf(w, ab, dta));
+                            dA[j] = fmaf(dab, dt * ab, fmaf(w, (dt * ab - be) * c.ia[j], dA[j]));
+                        } else {
+                            const float r = 0.5f * (ab + 1.0f);  // 1 / (1 - dt A / 2)
+                            const float r2 = r * r;
+                            dta = fmaf(dab, c.A[j] * r2, fmaf(w, fmaf(0.5f * dt * c.A[j], r2, r), dta));
+                            dA[j] = fmaf(dab, dt * r2, fmaf(w, 0.5f * dt * dt * r2, dA[j]));
+                        }
+                        anext[j] = ab;
+                    }
+                    dxa += __shfl_xor_sync(0xffffffffu, dxa, 16);
+                    dta += __shfl_xor_sync(0xffffffffu, dta, 16);
+                    // dB / dC: sum over the 16 channels of this half-warp (butterfly; lane q
+                    // ends with the sum of value q)
+#pragma unroll
+                    for (int m = 8; m >= 1; m >>= 1) {
+#pragma unroll
+                        for (int i2 = 0; i2 < m; ++i2) {
+                            const bool up = (q & m) != 0;
+                            const float send = up ? v[i2] : v[i2 + m];
+                            const float keep = up ? v[i2 + m] : v[i2];
+                            v[i2] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                        }
+                    }
+                    red[((size_t)(warp * kMaxS + t) * 2 + (q >> 3)) * kN + half * kNH + (q & 7)] = v[0];
+                    if (half == 0) {
+                        X[t * kDB + dl] = __float2bfloat16_rn(fmaf(ds, Dd, dxa));
+                        DT[t * kDB + dl] = __float2bfloat16_rn(dta);
+                        if (a.has_z) Z[t * kDB + dl] = __float2bfloat16_rn(dz);
+                        dD = fmaf(ds, xv, dD);
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tma_store_3d(&mdX, X, cb * kDB, t0, b);
+            tma_store_3d(&mdDT, DT, cb * kDB, t0, b);
+            if (a.has_z) tma_store_3d(&mdZ, Z, cb * kDB, t0, b);
+            bulk_commit();
+        }
+        // per-CTA partial dB / dC of this segment: fixed-order sum over the four warps
+        for (int e = tid; e < nt * 2 * kN; e += kThreads) {
+            const int t = e / (2 * kN), r = e % (2 * kN);
+            float sum = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sum += red[((size_t)(w * kMaxS + t) * 2) * kN + r];
+            float* dst = (r < kN ? a.pdB : a.pdC) + (((size_t)cb * a.B + b) * a.L + t0 + t) * kN + (r % kN);
+            *dst = sum;
+        }
+        __syncthreads();
+    }
+    if (dok) {
+        float* pa = a.pdA + ((size_t)b * a.D + d) * kN + half * kNH;
+#pragma unroll
+        for (int j = 0; j < kNH; ++j) pa[j] = dA[j];
+        if (half == 0) a.pdD[(size_t)b * a.D + d] = dD;
+    }
+    if (tid == 0) bulk_wait_read_all();
+}
+
+// Fixed-order sums of the partials: dB, dC over channel blocks; dA, dD over batch rows.
+__global__ void s6_reduce_kernel(S6Args a, float* __restrict__ dBm, float* __restrict__ dCm,
+                                 float* __restrict__ dAo, float* __restrict__ dDo) {
+    const size_t nBC = (size_t)a.B * a.L * kN;
+    const size_t nA = (size_t)a.D * kN;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nBC + nA + a.D;
+         i += (size_t)gridDim.x * blockDim.x) {
+        if (i < nBC) {
+            float sb = 0.0f, sc = 0.0f;
+            for (int cb = 0; cb < a.ncb; ++cb) {
+                sb += a.pdB[(size_t)cb * nBC + i];
+                sc += a.pdC[(size_t)cb * nBC + i];
+            }
+            dBm[i] = sb;
+            dCm[i] = sc;
+        } else if (i < nBC + nA) {
+            const size_t j = i - nBC;
+            float s = 0.0f;
+            for (int bb = 0; bb < a.B; ++bb) s += a.pdA[(size_t)bb * nA + j];
+            dAo[j] = s;
+        } else if (dDo) {
+            const size_t j = i - nBC - nA;
+            float s = 0.0f;
+            for (int bb = 0; bb < a.B; ++bb) s += a.pdD[(size_t)bb * a.D + j];
+            dDo[j] = s;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------ host side
+struct S6Ws {
+    size_t pdB, pdC, pdA, pdD, end;
+};
+
+S6Ws ws_plan(const lr_desc& d) {
+    const size_t ncb = (d.D + kDB - 1) / kDB;
+    WsCursor c;
+    S6Ws w;
+    w.pdB = c.take(sizeof(float) * ncb * d.B * d.L * kN);
+    w.pdC = c.take(sizeof(float) * ncb * d.B * d.L * kN);
+    w.pdA = c.take(sizeof(float) * d.B * d.D * kN);
+    w.pdD = c.take(sizeof(float) * d.B * d.D);
+    w.end = c.off;
+    return w;
+}
+
+S6Args make_args(const lr_desc& d, const lr_inputs& in, void* ckpt, char* ws, bool bwd) {
+    S6Args a{};
+    a.B = (int)d.B;
+    a.L = (int)d.L;
+    a.D = (int)d.D;
+    a.S = d.segment;
+    a.nseg = (int)((d.L + d.segment - 1) / d.segment);
+    a.ncb = (int)((d.D + kDB - 1) / kDB);
+    a.disc = d.disc;
+    a.has_z = (d.flags & LR_HAS_Z) ? 1 : 0;
+    a.has_d = (d.flags & LR_HAS_DSKIP) ? 1 : 0;
+    a.A = in.A;
+    a.Dskip = in.Dskip;
+    a.ckpt = (float*)ckpt;
+    a.hdr = (WsHeader*)ws;
+    if (bwd) {
+        S6Ws w = ws_plan(d);
+        a.pdB = (float*)(ws + w.pdB);
+        a.pdC = (float*)(ws + w.pdC);
+        a.pdA = (float*)(ws + w.pdA);
+        a.pdD = (float*)(ws + w.pdD);
+    }
+    return a;
+}
+
+template <typename F>
+void set_smem(F fn, size_t bytes) {
+    cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+bool s6_supported(const lr_desc& d) {
+    return d.io == LR_BF16 && d.N == kN && d.segment <= kMaxS && d.segment % kSub == 0 &&
+           d.D <= (1 << 24) && d.L <= (1 << 30);
+}
+
+size_t s6_ws_bytes(const lr_desc& d, bool bwd) { return bwd ? ws_plan(d).end : 256; }
+size_t s6_flag_bytes(const lr_desc&, bool) { return 256; }
+
+lr_status s6_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                 cudaStream_t st) {
+    S6Args a = make_args(d, in, ckpt, ws, false);
+    CUtensorMap mX, mDT, mZ, mB, mC, mY;
+    const uint32_t S = (uint32_t)d.segment;
+    bool ok = make_tmap_3d(&mX, in.x, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mDT, in.delta, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mZ, a.has_z ? in.z : in.x, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mB, in.Bm, 2, kN, d.L, d.B, kN, S) &&
+              make_tmap_3d(&mC, in.Cm, 2, kN, d.L, d.B, kN, S) &&
+              make_tmap_3d(&mY, y, 2, d.D, d.L, d.B, kDB, S);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    const int grid = a.B * a.ncb;
+    if (d.disc == LR_DISC_ZOH) {
+        set_smem(s6_fwd_kernel<LR_DISC_ZOH>, kFwdSmem);
+        note_launch("s6_fwd_zoh");
+        s6_fwd_kernel<LR_DISC_ZOH><<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
+    } else {
+        set_smem(s6_fwd_kernel<LR_DISC_BILINEAR>, kFwdSmem);
+        note_launch("s6_fwd_bilinear");
+        s6_fwd_kernel<LR_DISC_BILINEAR><<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
+    }
+    return check_launch();
+}
+
+lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                 const lr_grads& gr, char* ws, cudaStream_t st) {
+    S6Args a = make_args(d, in, const_cast<void*>(ckpt), ws, true);
+    CUtensorMap mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ;
+    const uint32_t S = (uint32_t)d.segment;
+    bool ok = make_tmap_3d(&mX, in.x, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mDT, in.delta, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mZ, a.has_z ? in.z : in.x, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mDY, dy, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mB, in.Bm, 2, kN, d.L, d.B, kN, S) &&
+              make_tmap_3d(&mC, in.Cm, 2, kN, d.L, d.B, kN, S) &&
+              make_tmap_3d(&mdX, gr.dx, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mdDT, gr.ddelta, 2, d.D, d.L, d.B, kDB, S) &&
+              make_tmap_3d(&mdZ, a.has_z ? gr.dz : gr.dx, 2, d.D, d.L, d.B, kDB, S);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    const int grid = a.B * a.ncb;
+    if (d.disc == LR_DISC_ZOH) {
+        set_smem(s6_bwd_kernel<LR_DISC_ZOH>, kBwdSmem);
+        note_launch("s6_bwd_zoh");
+        s6_bwd_kernel<LR_DISC_ZOH><<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
+    } else {
+        set_smem(s6_bwd_kernel<LR_DISC_BILINEAR>, kBwdSmem);
+        note_launch("s6_bwd_bilinear");
+        s6_bwd_kernel<LR_DISC_BILINEAR><<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
+    }
+    lr_status s = check_launch();
+    if (s != LR_OK) return s;
+    note_launch("s6_param_reduce");
+    s6_reduce_kernel<<<4 * 148, 256, 0, st>>>(a, gr.dBm, gr.dCm, gr.dA, a.has_d ? gr.dDskip : nullptr);
+    return check_launch();
+}
+
+}  // namespace lrs

@@ -4,12 +4,7 @@
 #include "host_common.h"
 
 namespace lrs {
-bool s6_supported(const lr_desc&) { return false; }
 bool chunk_supported(const lr_desc&) { return false; }
-size_t s6_ws_bytes(const lr_desc&, bool) { return 256; }
-size_t s6_flag_bytes(const lr_desc&, bool) { return 256; }
-lr_status s6_fwd(const lr_desc&, const lr_inputs&, void*, void*, char*, cudaStream_t) { return LR_ERR_UNSUPPORTED; }
-lr_status s6_bwd(const lr_desc&, const lr_inputs&, const void*, const void*, const lr_grads&, char*, cudaStream_t) { return LR_ERR_UNSUPPORTED; }
 size_t chunk_ws_bytes(const lr_desc&, bool) { return 256; }
 size_t chunk_flag_bytes(const lr_desc&, bool) { return 256; }
 lr_status chunk_fwd(const lr_desc&, const lr_inputs&, void*, void*, char*, cudaStream_t) { return LR_ERR_UNSUPPORTED; }

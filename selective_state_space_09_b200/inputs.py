@@ -19,7 +19,7 @@ Workloads (token-major layouts, last index contiguous):
   ``x, B, C ~ N(0,1)/sqrt(N)``; ``D_h ~ N(0,1)``.
 * ``gla``    bf16, B=4, H=16, K=V=128, L=2048, chunk 64, segment 256.
   ``g = sigmoid(N(3,1))`` per (b,t,h); ``q, k ~ N(0,1)`` L2-normalised per (b,t,h); ``v ~ N(0,1)``.
-* ``s6``     bf16 I/O, B=8, D=2048, N=16, L=2048, segment 256, ZOH or bilinear.
+* ``s6``     bf16 I/O, B=8, D=2048, N=16, L=2048, segment 64, ZOH or bilinear.
   ``dt = softplus(N(-3,1))``; ``A[d,n] = -(n+1)``; ``B, C ~ N(0,1)`` per (b,t,n); ``x, z, D ~ N(0,1)``.
 * ``rotlru`` fp32, B=16, D=4096 (2048 interleaved pairs), L=16384, segment 256.
   ``mag ~ U(0.95, 0.9999)`` and ``theta ~ U(0, pi/8)`` per pair; ``g = sigmoid(N(2,1))`` per
@@ -36,8 +36,8 @@ WORKLOADS = {
     "ssd": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=64,
                 segment=256, disc="zoh"),
     "gla": dict(kind="gla", io="bf16", B=4, H=16, K=128, V=128, L=2048, chunk=64, segment=256),
-    "s6_zoh": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=256, disc="zoh"),
-    "s6_bilinear": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=256,
+    "s6_zoh": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64, disc="zoh"),
+    "s6_bilinear": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64,
                         disc="bilinear"),
     "rotlru": dict(kind="rotlru", io="f32", B=16, D=4096, L=16384, segment=256),
 }

@@ -63,7 +63,10 @@ def test_validation_rules(L):
     assert _ok(L, kind="rotlru", io=f32, B=1, L=8, D=5, segment=4) == 1        # odd D
     assert _ok(L, kind="rotlru", io=f32, B=1, L=8, D=4, segment=4) == 3        # g rows 8 B
     # kinds whose kernels a build lacks report UNSUPPORTED (2) for otherwise valid requests
-    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256, disc="zoh") in (0, 2)
+    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=64, disc="zoh") == 0
+    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256, disc="zoh") == 2
+    assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=8, segment=64, disc="zoh") == 2
+    assert _ok(L, kind="s6", io=f32, B=8, L=2048, D=2048, N=16, segment=64, disc="zoh") == 2
     assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256) == 1  # no disc
     assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=256,
                chunk=64, disc="zoh") in (0, 2)

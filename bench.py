@@ -507,6 +507,7 @@ def main():
             "bwd_frac_hbm": round(r["bwd_gbs"] / pk["hbm_gbs"], 4),
             "step_frac_hbm": round(r["step_gbs"] / pk["hbm_gbs"], 4),
             "kernels": r["fwd_kernels"] + " | " + r["bwd_kernels"],
+            "traffic_bwd": ncu_traffic(r["bwd_kernels"].split("+")[0]),
             "peak_mem_gib": round(r["peak_mem_bytes"] / 2 ** 30, 3), "l2": r["l2"],
         }
     line = {

@@ -35,9 +35,9 @@ sys.path.insert(0, ROOT)
 METRIC = "fwd+bwd scan tokens/s & achieved HBM GB/s (% of B200 peak) per scan kind"
 BENCH_ORDER = ["ssd", "rglru", "gla", "s6_zoh", "s6_bilinear", "rotlru"]
 NAMES = {
-    "ssd": "Mamba-2 SSD scan (mamba-370m-like), bf16, B=2 H=32 P=64 N=128 L=4096, chunk 64, S=256, ZOH",
+    "ssd": "Mamba-2 SSD scan (mamba-370m-like), bf16, B=2 H=32 P=64 N=128 L=4096, chunk 128, S=128, ZOH",
     "rglru": "rglru_scan, f32, B=1 D=256 L=1024, S=128",
-    "gla": "GLA scan, bf16, B=4 H=16 K=V=128 L=2048, chunk 64, S=256",
+    "gla": "GLA scan, bf16, B=4 H=16 K=V=128 L=2048, chunk 128, S=128",
     "s6_zoh": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, ZOH, D skip + silu(z)",
     "s6_bilinear": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, bilinear, D skip + silu(z)",
     "rotlru": "rotlru_scan, f32, B=16 D=4096 L=16384, S=256",

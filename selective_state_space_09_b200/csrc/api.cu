@@ -110,8 +110,8 @@ lr_status check_launch() {
     return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 
-bool make_tmap_3d(CUtensorMap* map, const void* base, int esize_, uint64_t d0, uint64_t d1,
-                  uint64_t d2, uint32_t box0, uint32_t box1) {
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -122,6 +122,32 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int esize_, uint64_t d0, u
             q == cudaDriverEntryPointSuccess)
             encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     });
+    return encode;
+}
+}  // namespace
+
+bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const uint64_t* dims,
+               const uint64_t* strides, const uint32_t* box, bool swizzle128) {
+    auto encode = tmap_encoder();
+    if (!encode || rank < 2 || rank > 5) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], e[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        e[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
+    CUresult r = encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, int esize_, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint32_t box0, uint32_t box1) {
+    auto encode = tmap_encoder();
     if (!encode) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {d0 * esize_, d0 * d1 * esize_};

@@ -1,0 +1,458 @@
+// chunk.cu -- chunked-matmul chassis: ssd_scan and gla_scan on tcgen05 tensor cores (sm_100a).
+//
+// Both kinds are the recurrence S_t = e^{lam_t} S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t with a
+// scalar decay per step and head ("mlx-recurrence", Apple Developer Forums thread 840535,
+// "Current kernels": ssd_scan state [B, H, Dh, N], gla_scan state [B, H, Dh, Dh]):
+//   gla:  q, k, v per head, lam = log g, beta = 1;
+//   ssd:  q = C_t, k = B_t (shared by the heads of a group), v = x_t, lam = dt A_h,
+//         beta = (e^{dt A_h} - 1) / A_h (ZOH), y = o + D_h x.
+// The chunked form evaluates a chunk of Q = 128 steps with dense products (chunk-local cumulative
+// log decay l_t):
+//   o_t = sum_{s<=t} e^{l_t - l_s} beta_s (q_t . k_s) v_s  +  e^{l_t} q_t S_in
+//   S_out = e^{l_Q} S_in + sum_s e^{l_Q - l_s} beta_s k_s v_s^T
+// and chunks compose with the associative operator of the K-Search / mlx-mamba post (techtrendfeed
+// repost, paragraph after Table 1) -- here with a scalar coefficient e^{l_Q} and a matrix state.
+//
+// Forward tile = (batch row, head, chunk).  TMA brings q, k (128 x 128) and v (128 x V) into
+// 128-byte-swizzled shared-memory tiles; tcgen05 computes, with fp32 accumulators in TMEM,
+//   G1: Sqk = Q K^T                 (128 x 128 x K)
+//   G2: Y   = P V                   (P = masked, decayed, beta-scaled Sqk, written as bf16)
+//   G4: Sl  = K^T (w . V)           (w_s = e^{l_Q - l_s} beta_s; the chunk's own state increment)
+//   G3: Y2  = Q S_in                (S_in as bf16)
+// and y = Y + e^{l_t} Y2 (+ D x).  The state entering each chunk comes from a single-pass
+// decoupled look-back: a tile publishes its aggregate (e^{l_Q}, Sl) as soon as G4 is done, walks
+// back to the nearest chunk that has published its inclusive state, and folds the aggregates in
+// chain order (deterministic).  The inclusive states are the checkpoints: the checkpoint segment
+// equals the chunk (128 steps), slot c = state entering chunk c.
+#include "common.cuh"
+#include "host_common.h"
+#include "tc.cuh"
+
+namespace lrs {
+namespace {
+
+constexpr int kQ = 128;        // chunk length (rows of every tile, M of every MMA)
+constexpr int kKD = 128;       // key / state-row dimension (N of SSD, K of GLA)
+constexpr int kThreads = 128;  // 4 warps: thread i <-> row / TMEM lane i
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+struct ChunkArgs {
+    int kind;                 // LR_SSD / LR_GLA
+    int B, L, H, G, nchunk;   // G = groups (SSD), H heads
+    int VD;                   // value dim (SSD P, GLA V)
+    const __nv_bfloat16* lam; // SSD: dt [B, L, H]; GLA: g [B, L, H]
+    const float* A;           // SSD [H]
+    const float* Dskip;       // SSD [H] or null
+    float* ckpt;              // [nchunk, B, H, KD, VD] f32
+    WsHeader* hdr;
+    unsigned int* flags;      // [B*H*nchunk]
+    float* agg;               // [B*H*nchunk][KD][VD]
+    float* aggA;              // [B*H*nchunk] chunk decay e^{l_Q}
+    unsigned int dflags;
+};
+
+__device__ __forceinline__ char* smem_base1024() {
+    extern __shared__ char dyn_smem[];
+    uintptr_t p = reinterpret_cast<uintptr_t>(dyn_smem);
+    return reinterpret_cast<char*>((p + 1023) & ~uintptr_t(1023));
+}
+
+// Per-step log decay and beta of row t (t >= L gives no decay, no input).
+__device__ __forceinline__ void step_coef(const ChunkArgs& a, int b, int h, int t, float& lam, float& beta) {
+    lam = 0.0f;
+    beta = 0.0f;
+    if (t >= a.L) return;
+    const float v = __bfloat162float(a.lam[((size_t)b * a.L + t) * a.H + h]);
+    if (a.kind == LR_SSD) {
+        const float Ah = a.A[h];
+        lam = v * Ah;
+        beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+    } else {
+        lam = __logf(v);
+        beta = 1.0f;
+    }
+}
+
+// Inclusive prefix sum over the 128 threads of the CTA (tmp: 4 floats of shared memory).
+__device__ __forceinline__ float cta_inclusive_sum(float x, float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    float add = 0.0f;
+    for (int w = 0; w < warp; ++w) add += tmp[w];
+    __syncthreads();
+    return x + add;
+}
+
+// Shared-memory plan of the forward tile (offsets from a 1024-aligned base).
+template <int VD>
+struct FwdSmem {
+    static constexpr size_t kQt = 0;                                  // 128 x 128 bf16
+    static constexpr size_t kKt = kQt + kQ * kKD * 2;                 // 128 x 128
+    static constexpr size_t kVt = kKt + kQ * kKD * 2;                 // 128 x VD
+    static constexpr size_t kVs = kVt + kQ * VD * 2;                  // scaled copy of V
+    static constexpr size_t kPt = kVs + kQ * VD * 2;                  // 128 x 128 (P), then y
+    static constexpr size_t kSt = kPt + kQ * kQ * 2;                  // KD x VD (S_in bf16)
+    static constexpr size_t kL2 = kSt + kKD * VD * 2;                 // l * log2e [128]
+    static constexpr size_t kBeta = kL2 + kQ * 4;                     // beta [128]
+    static constexpr size_t kTmp = kBeta + kQ * 4;                    // scan scratch, misc
+    static constexpr size_t kBar = kTmp + 64;                         // 6 mbarriers
+    static constexpr size_t kTmem = kBar + 64;                        // TMEM base address
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;                     // + alignment slack
+};
+
+// TMEM columns of the forward tile
+constexpr uint32_t kColS1 = 0;    // 128: Q K^T, then Y2
+constexpr uint32_t kColY = 128;   // VD
+constexpr uint32_t kColSl = 256;  // VD
+
+template <int VD>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mY,
+                 ChunkArgs a) {
+    using SM = FwdSmem<VD>;
+    char* sm = smem_base1024();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);  // 0 load, 1 G1, 2 G2, 3 G4, 4 G3
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* l2 = reinterpret_cast<float*>(sm + SM::kL2);
+    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    int* misc = reinterpret_cast<int*>(sm + SM::kTmp + 32);
+    const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sV = smem_u32(sm + SM::kVt),
+                   sVs = smem_u32(sm + SM::kVs), sP = smem_u32(sm + SM::kPt), sS = smem_u32(sm + SM::kSt);
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    if (tid == 0) {
+        const unsigned int tk = take_ticket(a.hdr, 0);
+        const int per = a.B * a.H;
+        misc[0] = tk / per;           // chunk
+        misc[1] = (tk % per) / a.H;   // batch row
+        misc[2] = tk % a.H;           // head
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int c = misc[0], b = misc[1], h = misc[2];
+    const int t0 = c * kQ;
+    const int qk_head = a.kind == LR_SSD ? h / (a.H / a.G) : h;
+    const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;  // record index of this tile
+
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2 + kQ * VD * 2));
+        for (int j = 0; j < kKD / 64; ++j) {
+            tma_load_4d(sm + SM::kQt + j * kQ * 128, &mQ, &bar[0], 64 * j, qk_head, t0, b);
+            tma_load_4d(sm + SM::kKt + j * kQ * 128, &mK, &bar[0], 64 * j, qk_head, t0, b);
+        }
+        for (int j = 0; j < VD / 64; ++j) tma_load_4d(sm + SM::kVt + j * kQ * 128, &mV, &bar[0], 64 * j, h, t0, b);
+    }
+    // decays of this chunk: l_t inclusive cumulative log decay, beta_t
+    float lam, beta;
+    step_coef(a, b, h, t0 + tid, lam, beta);
+    const float lt = cta_inclusive_sum(lam, tmp);
+    l2[tid] = lt * kLog2e;
+    betas[tid] = beta;
+    __syncthreads();
+    const float lQ2 = l2[kQ - 1];  // l_Q log2e
+
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 500);
+    if (tid == 0 && ok) {  // G1: Q K^T
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kColS1, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);
+        tc::commit(&bar[1]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 501);
+    tc::fence_after_sync();
+    // P[t, s] = Sqk[t, s] e^{l_t - l_s} beta_s for s <= t, as a K-major bf16 tile
+    {
+        const int t = tid;
+        const float lt2 = l2[t];
+        char* P = sm + SM::kPt;
+        for (int s0 = 0; s0 < kQ; s0 += 16) {
+            float v[16];
+            tc::ld16(tmem + kColS1 + ((uint32_t)(warp * 32) << 16) + s0, v);
+            tc::wait_ld();
+            __align__(16) __nv_bfloat16 pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int s = s0 + i;
+                const float p = (s <= t) ? v[i] * ex2(lt2 - l2[s]) * betas[s] : 0.0f;
+                pk[i] = __float2bfloat16_rn(p);
+            }
+            *reinterpret_cast<uint4*>(P + tc::sw128_off(t, s0, kQ)) = *reinterpret_cast<uint4*>(&pk[0]);
+            *reinterpret_cast<uint4*>(P + tc::sw128_off(t, s0 + 8, kQ)) = *reinterpret_cast<uint4*>(&pk[8]);
+        }
+        // scaled copy of V: row s times w_s = e^{l_Q - l_s} beta_s
+        const float w = ex2(lQ2 - l2[t]) * betas[t];
+        const char* V = sm + SM::kVt;
+        char* Vs = sm + SM::kVs;
+        for (int v0 = 0; v0 < VD; v0 += 8) {
+            uint4 raw = *reinterpret_cast<const uint4*>(V + tc::sw128_off(t, v0, kQ));
+            __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float2 f = __bfloat1622float2(hv[i]);
+                hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
+            }
+            *reinterpret_cast<uint4*>(Vs + tc::sw128_off(t, v0, kQ)) = raw;
+        }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kColY, sP, 0, kQ, sV, 1, kQ, kQ, VD, kQ, 0);      // G2: Y = P V
+        tc::commit(&bar[2]);
+        tc::mma_tiles(tmem + kColSl, sK, 1, kQ, sVs, 1, kQ, kKD, VD, kQ, 0);  // G4: Sl = K^T (w V)
+        tc::commit(&bar[3]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[3], 0, a.hdr, 502);
+    tc::fence_after_sync();
+
+    // publish the aggregate (e^{l_Q}, Sl) of this chunk
+    const int kd = tid;  // state row / TMEM lane
+    const bool has_succ = c + 1 < a.nchunk;
+    float* myagg = a.agg + tile * kKD * VD + (size_t)kd * VD;
+    if (c > 0 && has_succ) {
+        for (int v0 = 0; v0 < VD; v0 += 16) {
+            float v[16];
+            tc::ld16(tmem + kColSl + ((uint32_t)(warp * 32) << 16) + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                __stcg(reinterpret_cast<float4*>(myagg + v0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+        if (tid == 0) __stcg(&a.aggA[tile], ex2(lQ2));
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) st_release(&a.flags[tile], kFlagAgg);
+    }
+
+    // look-back: state entering this chunk (row kd), deterministic fold in chain order
+    const size_t row0 = ((size_t)b * a.H + h) * a.nchunk;
+    int j = c - 1;
+    while (j >= 0) {
+        unsigned int f = wait_flag(&a.flags[row0 + j], a.hdr, 503);
+        if (f == kFlagPrefix || f == kFlagNone) break;
+        --j;
+    }
+    // j: nearest chunk with a published inclusive state (its state is ckpt slot j + 1), or -1
+    float* ck_in = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + kd) * VD;
+    char* St = sm + SM::kSt;
+    for (int v0 = 0; v0 < VD; v0 += 16) {
+        float x[16];
+        if (j >= 0) {
+            const float* src = a.ckpt + ((((size_t)(j + 1) * a.B + b) * a.H + h) * kKD + kd) * VD + v0;
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
+                x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+        }
+        for (int i = j + 1; i < c; ++i) {
+            const float ai = __ldcg(&a.aggA[row0 + i]);
+            const float* src = a.agg + (row0 + i) * kKD * VD + (size_t)kd * VD + v0;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+                float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
+                x[e] = fmaf(ai, x[e], f.x); x[e + 1] = fmaf(ai, x[e + 1], f.y);
+                x[e + 2] = fmaf(ai, x[e + 2], f.z); x[e + 3] = fmaf(ai, x[e + 3], f.w);
+            }
+        }
+        // checkpoint slot c = state entering this chunk (the predecessor writes the same bits as its
+        // inclusive state); bf16 copy as the MN-major B operand of G3
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(ck_in + v0 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        __align__(16) __nv_bfloat16 pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = __float2bfloat16_rn(x[i]);
+        *reinterpret_cast<uint4*>(St + tc::sw128_off(kd, v0, kKD)) = *reinterpret_cast<uint4*>(&pk[0]);
+        *reinterpret_cast<uint4*>(St + tc::sw128_off(kd, v0 + 8, kKD)) = *reinterpret_cast<uint4*>(&pk[8]);
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok && c > 0) {  // G3: Y2 = Q S_in (reuses the Sqk columns)
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kColS1, sQ, 0, kQ, sS, 1, kKD, kQ, VD, kKD, 0);
+        tc::commit(&bar[4]);
+    }
+    // inclusive state of this chunk: S_out = e^{l_Q} S_in + Sl  ->  checkpoint slot c + 1
+    const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && c == 0;
+    if (has_succ) {
+        const float aq = ex2(lQ2);
+        float* ck_out = a.ckpt + ((((size_t)(c + 1) * a.B + b) * a.H + h) * kKD + kd) * VD;
+        for (int v0 = 0; v0 < VD; v0 += 16) {
+            float v[16];
+            tc::ld16(tmem + kColSl + ((uint32_t)(warp * 32) << 16) + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 sin = *reinterpret_cast<const float4*>(ck_in + v0 + i);
+                __stcg(reinterpret_cast<float4*>(ck_out + v0 + i),
+                       make_float4(fmaf(aq, sin.x, v[i]), fmaf(aq, sin.y, v[i + 1]), fmaf(aq, sin.z, v[i + 2]),
+                                   fmaf(aq, sin.w, v[i + 3])));
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !withhold) st_release(&a.flags[tile], kFlagPrefix);
+    }
+
+    // output rows: y_t = Y_t + e^{l_t} Y2_t (+ D x_t)
+    ok = ok && mbar_wait(&bar[2], 0, a.hdr, 504);
+    if (c > 0) ok = ok && mbar_wait(&bar[4], 0, a.hdr, 505);
+    tc::fence_after_sync();
+    {
+        const int t = tid;
+        const float Et = ex2(l2[t]);
+        const float Dh = (a.kind == LR_SSD && a.Dskip) ? a.Dskip[h] : 0.0f;
+        char* Yo = sm + SM::kPt;  // P is no longer needed (G2 complete)
+        const char* V = sm + SM::kVt;
+        for (int v0 = 0; v0 < VD; v0 += 16) {
+            float y1[16], y2[16];
+            tc::ld16(tmem + kColY + ((uint32_t)(warp * 32) << 16) + v0, y1);
+            if (c > 0) tc::ld16(tmem + kColS1 + ((uint32_t)(warp * 32) << 16) + v0, y2);
+            tc::wait_ld();
+            __align__(16) __nv_bfloat16 pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 8) {
+                uint4 raw = *reinterpret_cast<const uint4*>(V + tc::sw128_off(t, v0 + i, kQ));
+                const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float yv = y1[i + e] + (c > 0 ? Et * y2[i + e] : 0.0f);
+                    yv = fmaf(Dh, __bfloat162float(xv[e]), yv);
+                    pk[i + e] = __float2bfloat16_rn(yv);
+                }
+            }
+            *reinterpret_cast<uint4*>(Yo + tc::sw128_off(t, v0, kQ)) = *reinterpret_cast<uint4*>(&pk[0]);
+            *reinterpret_cast<uint4*>(Yo + tc::sw128_off(t, v0 + 8, kQ)) = *reinterpret_cast<uint4*>(&pk[8]);
+        }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        for (int jj = 0; jj < VD / 64; ++jj) tma_store_4d(&mY, sm + SM::kPt + jj * kQ * 128, 64 * jj, h, t0, b);
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------ host side
+struct ChunkWs {
+    size_t flags, agg, aggA, end;
+};
+
+ChunkWs ws_plan(const lr_desc& d) {
+    const size_t tiles = (size_t)d.B * d.H * ((d.L + kQ - 1) / kQ);
+    const size_t VD = (size_t)d.P;
+    WsCursor c;
+    ChunkWs w;
+    w.flags = c.take(sizeof(unsigned int) * tiles);
+    w.aggA = c.take(sizeof(float) * tiles);
+    w.agg = c.take(sizeof(float) * tiles * kKD * VD);
+    w.end = c.off;
+    return w;
+}
+
+// rank-4 map of a [B, L, X, W] bf16 tensor (W contiguous) with box [1, 128 rows, 1, 64 cols]
+bool map4(CUtensorMap* m, const void* p, uint64_t W, uint64_t X, uint64_t L, uint64_t B, bool swz) {
+    uint64_t dims[4] = {W, X, L, B};
+    uint64_t str[3] = {W * 2, X * W * 2, L * X * W * 2};
+    uint32_t box[4] = {64, 1, (uint32_t)kQ, 1};
+    return make_tmap(m, p, 2, 4, dims, str, box, swz);
+}
+
+}  // namespace
+
+bool chunk_supported(const lr_desc& d) {
+    if (d.io != LR_BF16) return false;
+    if (d.N != kKD || (d.P != 64 && d.P != 128)) return false;
+    if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
+    if (d.kind == LR_SSD && (d.disc != LR_DISC_ZOH || (d.flags & LR_HAS_Z))) return false;
+    return d.L <= (1 << 28) && d.H <= 4096;
+}
+
+size_t chunk_ws_bytes(const lr_desc& d, bool) { return ws_plan(d).end; }
+size_t chunk_flag_bytes(const lr_desc& d, bool) { return ws_plan(d).aggA; }
+
+lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
+                    cudaStream_t st) {
+    ChunkWs w = ws_plan(d);
+    ChunkArgs a{};
+    a.kind = d.kind;
+    a.B = (int)d.B;
+    a.L = (int)d.L;
+    a.H = (int)d.H;
+    a.G = d.kind == LR_SSD ? (int)d.G : (int)d.H;
+    a.nchunk = (int)((d.L + kQ - 1) / kQ);
+    a.VD = (int)d.P;
+    a.lam = (const __nv_bfloat16*)(d.kind == LR_SSD ? in.delta : in.g);
+    a.A = in.A;
+    a.Dskip = (d.kind == LR_SSD && (d.flags & LR_HAS_DSKIP)) ? in.Dskip : nullptr;
+    a.ckpt = (float*)ckpt;
+    a.hdr = (WsHeader*)ws;
+    a.flags = (unsigned int*)(ws + w.flags);
+    a.agg = (float*)(ws + w.agg);
+    a.aggA = (float*)(ws + w.aggA);
+    a.dflags = d.flags;
+    CUtensorMap mQ, mK, mV, mY;
+    const void* q = d.kind == LR_SSD ? in.Cm : in.q;
+    const void* k = d.kind == LR_SSD ? in.Bm : in.k;
+    const void* v = d.kind == LR_SSD ? in.x : in.v;
+    const uint64_t QX = d.kind == LR_SSD ? (uint64_t)d.G : (uint64_t)d.H;
+    bool ok = map4(&mQ, q, kKD, QX, d.L, d.B, true) && map4(&mK, k, kKD, QX, d.L, d.B, true) &&
+              map4(&mV, v, d.P, d.H, d.L, d.B, true) && map4(&mY, y, d.P, d.H, d.L, d.B, true);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    const int grid = a.B * a.H * a.nchunk;
+    if (d.P == 64) {
+        using SM = FwdSmem<64>;
+        cudaFuncSetAttribute(chunk_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        note_launch(d.kind == LR_SSD ? "ssd_fwd_chunk" : "gla_fwd_chunk");
+        chunk_fwd_kernel<64><<<grid, kThreads, SM::kAlloc, st>>>(mQ, mK, mV, mY, a);
+    } else {
+        using SM = FwdSmem<128>;
+        cudaFuncSetAttribute(chunk_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        note_launch(d.kind == LR_SSD ? "ssd_fwd_chunk" : "gla_fwd_chunk");
+        chunk_fwd_kernel<128><<<grid, kThreads, SM::kAlloc, st>>>(mQ, mK, mV, mY, a);
+    }
+    return check_launch();
+}
+
+lr_status chunk_bwd(const lr_desc&, const lr_inputs&, const void*, const void*, const lr_grads&, char*,
+                    cudaStream_t) {
+    return LR_ERR_UNSUPPORTED;
+}
+
+}  // namespace lrs

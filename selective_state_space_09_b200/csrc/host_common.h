@@ -29,6 +29,12 @@ lr_status check_launch();
 bool make_tmap_3d(CUtensorMap* map, const void* base, int esize, uint64_t d0, uint64_t d1,
                   uint64_t d2, uint32_t box0, uint32_t box1);
 
+// Builds a tiled TMA descriptor of a row-major tensor of rank 2..5 (dims[0] contiguous;
+// strides[i] = byte stride of dimension i+1).  swizzle128 selects the 128-byte swizzle (box[0] *
+// esize must then be 128).  Returns false if the driver rejects the description.
+bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const uint64_t* dims,
+               const uint64_t* strides, const uint32_t* box, bool swizzle128);
+
 // Byte offset bookkeeping for a workspace: a 256-byte header followed by regions.
 struct WsCursor {
     size_t off = 256;

@@ -14,10 +14,11 @@ Workloads (token-major layouts, last index contiguous):
 * ``rglru``  fp32, B=1, D=256, L=1024, segment 128.
   ``a = sigmoid(Lam)^(8 r)``, ``Lam ~ U(2, 6)`` per channel, ``r = sigmoid(N(0,1))`` per step and
   channel; ``b = sqrt(1 - a^2) N(0,1)``.
-* ``ssd``    bf16 I/O, B=2, H=32, P=64, N=128, L=4096, G=1, chunk 64, segment 256, ZOH.
+* ``ssd``    bf16 I/O, B=2, H=32, P=64, N=128, L=4096, G=1, ZOH; evaluated in chunks of 128 steps,
+  which are also the checkpoint segments.
   ``dt = softplus(N(-2,1))`` per (b,t,h); ``A_h = -exp(U(log 1, log 16))``;
   ``x, B, C ~ N(0,1)/sqrt(N)``; ``D_h ~ N(0,1)``.
-* ``gla``    bf16, B=4, H=16, K=V=128, L=2048, chunk 64, segment 256.
+* ``gla``    bf16, B=4, H=16, K=V=128, L=2048; chunks (and checkpoint segments) of 128 steps.
   ``g = sigmoid(N(3,1))`` per (b,t,h); ``q, k ~ N(0,1)`` L2-normalised per (b,t,h); ``v ~ N(0,1)``.
 * ``s6``     bf16 I/O, B=8, D=2048, N=16, L=2048, segment 64, ZOH or bilinear.
   ``dt = softplus(N(-3,1))``; ``A[d,n] = -(n+1)``; ``B, C ~ N(0,1)`` per (b,t,n); ``x, z, D ~ N(0,1)``.
@@ -33,9 +34,9 @@ import torch
 
 WORKLOADS = {
     "rglru": dict(kind="rglru", io="f32", B=1, D=256, L=1024, segment=128),
-    "ssd": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=64,
-                segment=256, disc="zoh"),
-    "gla": dict(kind="gla", io="bf16", B=4, H=16, K=128, V=128, L=2048, chunk=64, segment=256),
+    "ssd": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=128,
+                segment=128, disc="zoh"),
+    "gla": dict(kind="gla", io="bf16", B=4, H=16, K=128, V=128, L=2048, chunk=128, segment=128),
     "s6_zoh": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64, disc="zoh"),
     "s6_bilinear": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64,
                         disc="bilinear"),

@@ -68,11 +68,16 @@ def test_validation_rules(L):
     assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=8, segment=64, disc="zoh") == 2
     assert _ok(L, kind="s6", io=f32, B=8, L=2048, D=2048, N=16, segment=64, disc="zoh") == 2
     assert _ok(L, kind="s6", io=bf, B=8, L=2048, D=2048, N=16, segment=256) == 1  # no disc
+    assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=128,
+               chunk=128, disc="zoh") == 0
     assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=256,
-               chunk=64, disc="zoh") in (0, 2)
+               chunk=64, disc="zoh") == 2                                        # chunk != 128
+    assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=128,
+               disc="bilinear") == 2
     assert _ok(L, kind="ssd", io=bf, B=2, L=64, H=32, P=64, N=128, G=3, segment=64,
                disc="zoh") == 1                                                  # H % G
-    assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=256, chunk=64) in (0, 2)
+    assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=128, chunk=128) == 0
+    assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=96, N=128, segment=128) == 2
     assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=256,
                disc="zoh") == 1
 

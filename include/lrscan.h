@@ -50,7 +50,8 @@
  * workspace and reported by lr_get_error.  Kernels never trap, assert or spin without a bound.
  *
  * Alignment.  Every pointer must be 16-byte aligned and the innermost dimension of every
- * per-token tensor must span a multiple of 16 bytes (LR_ERR_ALIGNMENT otherwise).
+ * per-token tensor must span a multiple of 16 bytes (LR_ERR_ALIGNMENT otherwise) -- except the
+ * per-head dt of SSD and g of GLA ([B, L, H]), which may have any H.
  *
  * Gradients are written, not accumulated.
  */

@@ -48,13 +48,13 @@ lr_status validate(const lr_desc* d) {
         case LR_SSD: {
             if (d->disc != LR_DISC_ZOH && d->disc != LR_DISC_BILINEAR) return LR_ERR_INVALID_ARG;
             if (d->H < 1 || d->P < 1 || d->N < 1 || d->G < 1 || d->H % d->G) return LR_ERR_INVALID_ARG;
-            if ((d->P * es) % 16 || (d->N * es) % 16 || (d->H * es) % 16) return LR_ERR_ALIGNMENT;
+            if ((d->P * es) % 16 || (d->N * es) % 16) return LR_ERR_ALIGNMENT;
             return chunk_supported(*d) ? LR_OK : LR_ERR_UNSUPPORTED;
         }
         case LR_GLA: {
             if (d->disc != LR_DISC_NONE) return LR_ERR_INVALID_ARG;
             if (d->H < 1 || d->P < 1 || d->N < 1) return LR_ERR_INVALID_ARG;
-            if ((d->P * es) % 16 || (d->N * es) % 16 || (d->H * es) % 16) return LR_ERR_ALIGNMENT;
+            if ((d->P * es) % 16 || (d->N * es) % 16) return LR_ERR_ALIGNMENT;
             return chunk_supported(*d) ? LR_OK : LR_ERR_UNSUPPORTED;
         }
     }

@@ -124,3 +124,24 @@ def test_plan_buffers_cover_the_queried_sizes(L):
         assert p.ws_bytes >= max(L.workspace_bytes(d, False), L.workspace_bytes(d, True))
         assert p.ckpt.numel() * 4 >= L.ckpt_bytes(d)
         assert p.ckpt_view().shape[0] == (d.L + d.segment - 1) // d.segment
+
+
+def test_every_gpu_test_case_passes_host_validation(L):
+    """The descriptors of the GPU parity cases are valid for this build (checked on the CPU, so a
+    shape-rule mistake does not cost a GPU run)."""
+    import torch
+    import test_gpu_diag as gd
+    import test_gpu_s6 as gs
+    import test_gpu_chunk as gc
+    f32, bf = torch.float32, torch.bfloat16
+    for B, Lq, D, S, io in gd.RGLRU_CASES:
+        assert _ok(L, kind="rglru", io=f32 if io == "f32" else bf, B=B, L=Lq, D=D, segment=S) == 0
+    for B, Lq, D, S, io in gd.ROTLRU_CASES:
+        assert _ok(L, kind="rotlru", io=f32 if io == "f32" else bf, B=B, L=Lq, D=D, segment=S) == 0
+    for B, Lq, D, S, disc, wz, wd in gs.CASES:
+        assert _ok(L, kind="s6", io=bf, B=B, L=Lq, D=D, N=16, segment=S, disc=disc, has_z=wz, has_d=wd) == 0
+    for B, Lq, H, P, G in gc.SSD_CASES:
+        assert _ok(L, kind="ssd", io=bf, B=B, L=Lq, H=H, P=P, N=128, G=G, segment=128, chunk=128,
+                   disc="zoh", has_d=True) == 0
+    for B, Lq, H, V in gc.GLA_CASES:
+        assert _ok(L, kind="gla", io=bf, B=B, L=Lq, H=H, P=V, N=128, segment=128, chunk=128) == 0

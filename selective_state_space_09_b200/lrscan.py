@@ -164,7 +164,7 @@ class Plan:
         d = self.desc
         nseg = (d.L + d.segment - 1) // d.segment
         shapes = {0: (nseg, d.B, d.D), 1: (nseg, d.B, d.D), 2: (nseg, d.B, d.D, d.N),
-                  3: (nseg, d.B, d.H, d.P, d.N), 4: (nseg, d.B, d.H, d.N, d.P)}
+                  3: (nseg, d.B, d.H, d.N, d.P), 4: (nseg, d.B, d.H, d.N, d.P)}
         shp = shapes[d.kind]
         n = 1
         for s in shp:

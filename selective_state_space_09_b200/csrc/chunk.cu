@@ -404,8 +404,9 @@ bool chunk_supported(const lr_desc& d) {
     return d.L <= (1 << 28) && d.H <= 4096;
 }
 
-size_t chunk_ws_bytes(const lr_desc& d, bool) { return ws_plan(d).end; }
-size_t chunk_flag_bytes(const lr_desc& d, bool) { return ws_plan(d).aggA; }
+size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only);
+size_t chunk_ws_bytes(const lr_desc& d, bool bwd) { return bwd ? chunk_bwd_ws_end(d, false) : ws_plan(d).end; }
+size_t chunk_flag_bytes(const lr_desc& d, bool bwd) { return bwd ? chunk_bwd_ws_end(d, true) : ws_plan(d).aggA; }
 
 lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
                     cudaStream_t st) {
@@ -450,9 +451,559 @@ lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, 
     return check_launch();
 }
 
-lr_status chunk_bwd(const lr_desc&, const lr_inputs&, const void*, const void*, const lr_grads&, char*,
-                    cudaStream_t) {
-    return LR_ERR_UNSUPPORTED;
+// =========================================================================================
+// Backward.  Tile = (batch row, head, chunk), chunks taken in reverse order.  With the chunk's
+// entering state S_in (checkpoint slot c), its inclusive state S_out (slot c + 1), the upstream
+// gradient dO and the adjoint dS_out of S_out, the chunk's gradients are (l: chunk-local
+// cumulative log decay, E_t = e^{l_t}, W_s = e^{l_Q - l_s}, a = e^{l_Q}):
+//   dq  = Pd K + diag(E) dO S_in^T            Pd[t,s] = (dO V^T)[t,s] e^{l_t - l_s} beta_s, s <= t
+//   dk  = Pd^T Q + diag(W beta) V dS_out^T
+//   dv  = P^T dO + diag(W beta) K dS_out       P[t,s]  = (Q K^T)[t,s] e^{l_t - l_s} beta_s, s <= t
+//   dS_in = a dS_out + Q^T diag(E) dO         (the adjoint handed to the previous chunk)
+//   dl_t  = q_t . dq_t - k_t . dk_t  (+ <dS_out, S_out> at the chunk's last step)
+//   d lam_r = sum_{t >= r} dl_t ;   d beta_s = k_s . dk_s / beta_s
+// (gla: dg = d lam / g; ssd: d dt = d lam A + d beta abar, dA = sum(d lam dt + d beta
+// (dt abar - beta) / A), dx = dv + D dy, dB / dC = sums of dk / dq over the heads of a group.)
+// The adjoint carry dS_out comes from a reverse decoupled look-back over per-chunk records
+// (aggregate (a, Q^T diag(E) dO), inclusive dS_in), folded in chain order.
+// =========================================================================================
+namespace {
+
+template <int VD>
+struct BwdSmem {
+    static constexpr size_t kQt = 0;                      // Q (never scaled); dq staging at the end
+    static constexpr size_t kKt = kQt + kQ * kKD * 2;     // K, then diag(W beta) K; dk staging
+    static constexpr size_t kVt = kKt + kQ * kKD * 2;     // V, then diag(W beta) V; dv / dx staging
+    static constexpr size_t kOt = kVt + kQ * VD * 2;      // dO, then diag(E) dO
+    static constexpr size_t kPt = kOt + kQ * VD * 2;      // P, then dS_out (bf16, KD x VD)
+    static constexpr size_t kPdt = kPt + kQ * kQ * 2;     // Pd, then S_in (bf16, KD x VD)
+    static constexpr size_t kL2 = kPdt + kQ * kQ * 2;     // l log2e [128]
+    static constexpr size_t kBeta = kL2 + kQ * 4;         // beta [128]
+    static constexpr size_t kLam = kBeta + kQ * 4;        // raw per-step input (dt or g) [128]
+    static constexpr size_t kRed = kLam + kQ * 4;         // reduction scratch [128]
+    static constexpr size_t kTmp = kRed + kQ * 4;         // scan scratch, misc
+    static constexpr size_t kBar = kTmp + 64;
+    static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;
+};
+
+constexpr uint32_t kR0 = 0, kR1 = 128, kR2 = 256, kR3 = 384;
+
+struct ChunkBwdArgs {
+    ChunkArgs f;              // shapes, decays, checkpoints (read), header
+    const __nv_bfloat16* kg;  // k (GLA) / B (SSD) in global memory, for the k . dk row dots
+    const __nv_bfloat16* dy;  // upstream gradient [B, L, H, VD]
+    __nv_bfloat16* dlam;      // GLA dg / SSD ddt [B, L, H]
+    float* dBm;               // SSD [B, L, G, N] (accumulated over heads)
+    float* dCm;
+    unsigned int* flags;      // reverse-chain records
+    float* agg;
+    float* aggA;
+    float* pre;
+    float* pdA;               // SSD per-tile partials
+    float* pdD;
+};
+
+__device__ __forceinline__ void fold16(float* x, float a, const float* src) {
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
+        x[e] = fmaf(a, x[e], f.x);
+        x[e + 1] = fmaf(a, x[e + 1], f.y);
+        x[e + 2] = fmaf(a, x[e + 2], f.z);
+        x[e + 3] = fmaf(a, x[e + 3], f.w);
+    }
+}
+
+// Scale row r (cols [0, cols)) of an SW128 tile with `rows` rows by w, in place.
+__device__ __forceinline__ void scale_row(char* tile, int r, int cols, int rows, float w) {
+    for (int c0 = 0; c0 < cols; c0 += 8) {
+        uint4 raw = *reinterpret_cast<const uint4*>(tile + tc::sw128_off(r, c0, rows));
+        __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(hv[i]);
+            hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
+        }
+        *reinterpret_cast<uint4*>(tile + tc::sw128_off(r, c0, rows)) = raw;
+    }
+}
+
+template <int VD>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mO,
+                 const __grid_constant__ CUtensorMap mdQ, const __grid_constant__ CUtensorMap mdK,
+                 const __grid_constant__ CUtensorMap mdV, ChunkBwdArgs bw) {
+    using SM = BwdSmem<VD>;
+    const ChunkArgs& a = bw.f;
+    char* sm = smem_base1024();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* l2 = reinterpret_cast<float*>(sm + SM::kL2);
+    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
+    float* red = reinterpret_cast<float*>(sm + SM::kRed);
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    int* misc = reinterpret_cast<int*>(sm + SM::kTmp + 32);
+    const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sV = smem_u32(sm + SM::kVt),
+                   sO = smem_u32(sm + SM::kOt), sP = smem_u32(sm + SM::kPt), sPd = smem_u32(sm + SM::kPdt);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const bool ssd = a.kind == LR_SSD;
+    const uint32_t colDv = kR1, colDSl = ssd ? kR1 + 64 : kR0;
+
+    if (tid == 0) {
+        const unsigned int tk = take_ticket(a.hdr, 1);
+        const int per = a.B * a.H;
+        misc[0] = a.nchunk - 1 - (int)(tk / per);
+        misc[1] = (tk % per) / a.H;
+        misc[2] = tk % a.H;
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int c = misc[0], b = misc[1], h = misc[2];
+    const int t0 = c * kQ;
+    const int gq = ssd ? h / (a.H / a.G) : h;
+    const size_t row0 = ((size_t)b * a.H + h) * a.nchunk;
+    const size_t tile = row0 + c;
+    const bool last = c + 1 >= a.nchunk;
+
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2 + 2 * kQ * VD * 2));
+        for (int j = 0; j < kKD / 64; ++j) {
+            tma_load_4d(sm + SM::kQt + j * kQ * 128, &mQ, &bar[0], 64 * j, gq, t0, b);
+            tma_load_4d(sm + SM::kKt + j * kQ * 128, &mK, &bar[0], 64 * j, gq, t0, b);
+        }
+        for (int j = 0; j < VD / 64; ++j) {
+            tma_load_4d(sm + SM::kVt + j * kQ * 128, &mV, &bar[0], 64 * j, h, t0, b);
+            tma_load_4d(sm + SM::kOt + j * kQ * 128, &mO, &bar[0], 64 * j, h, t0, b);
+        }
+    }
+    const int r = tid;  // this thread's row (time step in the chunk, or state row kd)
+    const int tr = t0 + r;
+    float lam, beta;
+    step_coef(a, b, h, tr, lam, beta);
+    const float lt = cta_inclusive_sum(lam, tmp);
+    l2[r] = lt * kLog2e;
+    betas[r] = beta;
+    __syncthreads();
+    const float lQ2 = l2[kQ - 1];
+
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 600);
+    if (tid == 0 && ok) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kR0, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);  // Q K^T
+        tc::mma_tiles(tmem + kR1, sO, 0, kQ, sV, 0, kQ, kQ, kQ, VD, 0);   // dO V^T
+        tc::commit(&bar[1]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 601);
+    tc::fence_after_sync();
+    {  // P and Pd (bf16), row r
+        const float lr2 = l2[r];
+        char* P = sm + SM::kPt;
+        char* Pd = sm + SM::kPdt;
+        for (int s0 = 0; s0 < kQ; s0 += 16) {
+            float qk[16], dv[16];
+            tc::ld16(tmem + kR0 + lane_off + s0, qk);
+            tc::ld16(tmem + kR1 + lane_off + s0, dv);
+            tc::wait_ld();
+            __align__(16) __nv_bfloat16 pk[16], pd[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int s = s0 + i;
+                const float f = (s <= r) ? ex2(lr2 - l2[s]) * betas[s] : 0.0f;
+                pk[i] = __float2bfloat16_rn(qk[i] * f);
+                pd[i] = __float2bfloat16_rn(dv[i] * f);
+            }
+            *reinterpret_cast<uint4*>(P + tc::sw128_off(r, s0, kQ)) = *reinterpret_cast<uint4*>(&pk[0]);
+            *reinterpret_cast<uint4*>(P + tc::sw128_off(r, s0 + 8, kQ)) = *reinterpret_cast<uint4*>(&pk[8]);
+            *reinterpret_cast<uint4*>(Pd + tc::sw128_off(r, s0, kQ)) = *reinterpret_cast<uint4*>(&pd[0]);
+            *reinterpret_cast<uint4*>(Pd + tc::sw128_off(r, s0 + 8, kQ)) = *reinterpret_cast<uint4*>(&pd[8]);
+        }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kR2, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, 0);  // dq  = Pd K
+        tc::mma_tiles(tmem + kR3, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, 0);  // dk  = Pd^T Q
+        tc::mma_tiles(tmem + colDv, sP, 1, kQ, sO, 1, kQ, kQ, VD, kQ, 0);  // dv  = P^T dO
+        tc::commit(&bar[2]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[2], 0, a.hdr, 602);
+    float dD_part = 0.0f;
+    {
+        // D-skip gradient part (ssd): sum_v dy x of row r, before V is rescaled
+        char* V = sm + SM::kVt;
+        char* O = sm + SM::kOt;
+        if (ssd) {
+            for (int v0 = 0; v0 < VD; v0 += 8) {
+                uint4 xr = *reinterpret_cast<const uint4*>(V + tc::sw128_off(r, v0, kQ));
+                uint4 orw = *reinterpret_cast<const uint4*>(O + tc::sw128_off(r, v0, kQ));
+                const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&xr);
+                const __nv_bfloat16* ov = reinterpret_cast<const __nv_bfloat16*>(&orw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dD_part = fmaf(__bfloat162float(xv[e]), __bfloat162float(ov[e]), dD_part);
+            }
+        }
+        const float E = ex2(l2[r]);
+        const float wb = ex2(lQ2 - l2[r]) * betas[r];
+        scale_row(O, r, VD, kQ, E);                   // diag(E) dO
+        scale_row(V, r, VD, kQ, wb);                  // diag(W beta) V
+        scale_row(sm + SM::kKt, r, kKD, kQ, wb);      // diag(W beta) K
+        // S_in (checkpoint slot c) as bf16, rows kd x cols v, in the Pd region
+        const float* sin = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + r) * VD;
+        char* St = sm + SM::kPdt;
+        for (int v0 = 0; v0 < VD; v0 += 8) {
+            const float4 f0 = __ldcg(reinterpret_cast<const float4*>(sin + v0));
+            const float4 f1 = __ldcg(reinterpret_cast<const float4*>(sin + v0 + 4));
+            __align__(16) __nv_bfloat162 pk[4] = {__floats2bfloat162_rn(f0.x, f0.y), __floats2bfloat162_rn(f0.z, f0.w),
+                                                  __floats2bfloat162_rn(f1.x, f1.y), __floats2bfloat162_rn(f1.z, f1.w)};
+            *reinterpret_cast<uint4*>(St + tc::sw128_off(r, v0, kKD)) = *reinterpret_cast<uint4*>(pk);
+        }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kR2, sO, 0, kQ, sPd, 0, kKD, kQ, kKD, VD, 1);   // dq += diag(E) dO S_in^T
+        tc::mma_tiles(tmem + colDSl, sQ, 1, kQ, sO, 1, kQ, kKD, VD, kQ, 0);  // dSl = Q^T diag(E) dO
+        tc::commit(&bar[3]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[3], 0, a.hdr, 603);
+    tc::fence_after_sync();
+
+    // reverse chain: aggregate (a, dSl) of this chunk
+    const float aq = ex2(lQ2);
+    float* myagg = bw.agg + tile * kKD * VD + (size_t)r * VD;
+    if (c > 0 && !last) {
+        for (int v0 = 0; v0 < VD; v0 += 16) {
+            float v[16];
+            tc::ld16(tmem + colDSl + lane_off + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                __stcg(reinterpret_cast<float4*>(myagg + v0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+        if (tid == 0) __stcg(&bw.aggA[tile], aq);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) st_release(&bw.flags[tile], kFlagAgg);
+    }
+    // dS_out: walk to the nearest later chunk with an inclusive adjoint, fold in chain order
+    int j = c + 1;
+    while (j < a.nchunk) {
+        const unsigned int f = wait_flag(&bw.flags[row0 + j], a.hdr, 604);
+        if (f == kFlagPrefix || f == kFlagNone) break;
+        ++j;
+    }
+    float xdot = 0.0f;  // <dS_out, S_out> restricted to row r
+    float* mypre = bw.pre + tile * kKD * VD + (size_t)r * VD;
+    char* dSt = sm + SM::kPt;
+    const float* sout = a.ckpt + ((((size_t)(c + 1) * a.B + b) * a.H + h) * kKD + r) * VD;
+    for (int v0 = 0; v0 < VD; v0 += 16) {
+        float x[16];
+        if (j < a.nchunk) {
+            const float* src = bw.pre + (row0 + j) * kKD * VD + (size_t)r * VD + v0;
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
+                x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+        }
+        for (int i = j - 1; i > c; --i)
+            fold16(x, __ldcg(&bw.aggA[row0 + i]), bw.agg + (row0 + i) * kKD * VD + (size_t)r * VD + v0);
+        if (!last) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 so = __ldcg(reinterpret_cast<const float4*>(sout + v0 + i));
+                xdot = fmaf(x[i], so.x, fmaf(x[i + 1], so.y, fmaf(x[i + 2], so.z, fmaf(x[i + 3], so.w, xdot))));
+            }
+        }
+        __align__(16) __nv_bfloat16 pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = __float2bfloat16_rn(x[i]);
+        *reinterpret_cast<uint4*>(dSt + tc::sw128_off(r, v0, kKD)) = *reinterpret_cast<uint4*>(&pk[0]);
+        *reinterpret_cast<uint4*>(dSt + tc::sw128_off(r, v0 + 8, kKD)) = *reinterpret_cast<uint4*>(&pk[8]);
+        if (c > 0) {  // inclusive adjoint handed to chunk c - 1: a dS_out + dSl
+            float v[16];
+            tc::ld16(tmem + colDSl + lane_off + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                __stcg(reinterpret_cast<float4*>(mypre + v0 + i),
+                       make_float4(fmaf(aq, x[i], v[i]), fmaf(aq, x[i + 1], v[i + 1]), fmaf(aq, x[i + 2], v[i + 2]),
+                                   fmaf(aq, x[i + 3], v[i + 3])));
+        }
+    }
+    const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && last;
+    if (c > 0) {
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !withhold) st_release(&bw.flags[tile], kFlagPrefix);
+    }
+    red[r] = xdot;
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok && !last) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem + kR3, sV, 0, kQ, sP, 0, kKD, kQ, kKD, VD, 1);    // dk += diag(W b) V dS_out^T
+        tc::mma_tiles(tmem + colDv, sK, 0, kQ, sP, 1, kKD, kQ, VD, kKD, 1);  // dv += diag(W b) K dS_out
+        tc::commit(&bar[4]);
+    }
+    __syncwarp();
+    if (!last) ok = ok && mbar_wait(&bar[4], 0, a.hdr, 605);
+    tc::fence_after_sync();
+    float X = 0.0f;  // <dS_out, S_out>
+    for (int i = 0; i < kQ; ++i) X += red[i];
+
+    // final epilogue, row r: dq, dk, dv (dx), dl
+    const bool valid = tr < a.L;
+    float qdq = 0.0f, kdk = 0.0f;
+    {
+        char* Q = sm + SM::kQt;
+        char* K = sm + SM::kKt;
+        const __nv_bfloat16* kglob = bw.kg + (((size_t)b * a.L + min(tr, a.L - 1)) * (ssd ? a.G : a.H) + gq) * kKD;
+        for (int k0 = 0; k0 < kKD; k0 += 16) {
+            float dq[16], dk[16];
+            tc::ld16(tmem + kR2 + lane_off + k0, dq);
+            tc::ld16(tmem + kR3 + lane_off + k0, dk);
+            tc::wait_ld();
+            __align__(16) __nv_bfloat16 oq[16], ok2[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 8) {
+                uint4 qr = *reinterpret_cast<const uint4*>(Q + tc::sw128_off(r, k0 + i, kQ));
+                uint4 kr = valid ? *reinterpret_cast<const uint4*>(kglob + k0 + i) : make_uint4(0, 0, 0, 0);
+                const __nv_bfloat16* qv = reinterpret_cast<const __nv_bfloat16*>(&qr);
+                const __nv_bfloat16* kv = reinterpret_cast<const __nv_bfloat16*>(&kr);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    qdq = fmaf(__bfloat162float(qv[e]), dq[i + e], qdq);
+                    kdk = fmaf(__bfloat162float(kv[e]), dk[i + e], kdk);
+                    oq[i + e] = __float2bfloat16_rn(dq[i + e]);
+                    ok2[i + e] = __float2bfloat16_rn(dk[i + e]);
+                }
+            }
+            if (ssd) {
+                if (valid) {
+                    float* dC = bw.dCm + (((size_t)b * a.L + tr) * a.G + gq) * kKD + k0;
+                    float* dB = bw.dBm + (((size_t)b * a.L + tr) * a.G + gq) * kKD + k0;
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        atomicAdd(reinterpret_cast<float4*>(dC + i), make_float4(dq[i], dq[i + 1], dq[i + 2], dq[i + 3]));
+                        atomicAdd(reinterpret_cast<float4*>(dB + i), make_float4(dk[i], dk[i + 1], dk[i + 2], dk[i + 3]));
+                    }
+                }
+            } else {
+                *reinterpret_cast<uint4*>(Q + tc::sw128_off(r, k0, kQ)) = *reinterpret_cast<uint4*>(&oq[0]);
+                *reinterpret_cast<uint4*>(Q + tc::sw128_off(r, k0 + 8, kQ)) = *reinterpret_cast<uint4*>(&oq[8]);
+                *reinterpret_cast<uint4*>(K + tc::sw128_off(r, k0, kQ)) = *reinterpret_cast<uint4*>(&ok2[0]);
+                *reinterpret_cast<uint4*>(K + tc::sw128_off(r, k0 + 8, kQ)) = *reinterpret_cast<uint4*>(&ok2[8]);
+            }
+        }
+        // dv (gla) / dx = dv + D dy (ssd) into the V region
+        char* V = sm + SM::kVt;
+        const float Dh = (ssd && a.Dskip) ? a.Dskip[h] : 0.0f;
+        const __nv_bfloat16* dyr = bw.dy + (((size_t)b * a.L + min(tr, a.L - 1)) * a.H + h) * VD;
+        for (int v0 = 0; v0 < VD; v0 += 16) {
+            float dv[16];
+            tc::ld16(tmem + colDv + lane_off + v0, dv);
+            tc::wait_ld();
+            __align__(16) __nv_bfloat16 o[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 8) {
+                uint4 yr = (valid && ssd) ? *reinterpret_cast<const uint4*>(dyr + v0 + i) : make_uint4(0, 0, 0, 0);
+                const __nv_bfloat16* yv = reinterpret_cast<const __nv_bfloat16*>(&yr);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[i + e] = __float2bfloat16_rn(fmaf(Dh, __bfloat162float(yv[e]), dv[i + e]));
+            }
+            *reinterpret_cast<uint4*>(V + tc::sw128_off(r, v0, kQ)) = *reinterpret_cast<uint4*>(&o[0]);
+            *reinterpret_cast<uint4*>(V + tc::sw128_off(r, v0 + 8, kQ)) = *reinterpret_cast<uint4*>(&o[8]);
+        }
+    }
+    // decay and beta gradients
+    float dl = qdq - kdk + (r == kQ - 1 ? X : 0.0f);
+    if (!valid) dl = 0.0f;
+    const float incl = cta_inclusive_sum(dl, tmp);
+    if (tid == kQ - 1) red[0] = incl;  // total
+    __syncthreads();
+    const float dlam = red[0] - incl + dl;  // sum over t >= r
+    float dA_part = 0.0f;
+    if (valid) {
+        const float raw = __bfloat162float(a.lam[((size_t)b * a.L + tr) * a.H + h]);
+        float out;
+        if (ssd) {
+            const float Ah = a.A[h];
+            const float ab = ex2(raw * Ah * kLog2e);
+            const float dbeta = beta != 0.0f ? kdk / beta : 0.0f;
+            out = dlam * Ah + dbeta * ab;
+            dA_part = dlam * raw + dbeta * (raw * ab - beta) / Ah;
+        } else {
+            out = dlam / raw;
+        }
+        bw.dlam[((size_t)b * a.L + tr) * a.H + h] = __float2bfloat16_rn(out);
+    }
+    if (ssd) {  // per-tile partials of dA_h and dD_h (fixed-order sums)
+        __syncthreads();
+        red[r] = dA_part;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.0f;
+            for (int i = 0; i < kQ; ++i) s += red[i];
+            bw.pdA[tile] = s;
+        }
+        __syncthreads();
+        red[r] = dD_part;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.0f;
+            for (int i = 0; i < kQ; ++i) s += red[i];
+            bw.pdD[tile] = s;
+        }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        if (!ssd) {
+            for (int jj = 0; jj < kKD / 64; ++jj) {
+                tma_store_4d(&mdQ, sm + SM::kQt + jj * kQ * 128, 64 * jj, h, t0, b);
+                tma_store_4d(&mdK, sm + SM::kKt + jj * kQ * 128, 64 * jj, h, t0, b);
+            }
+        }
+        for (int jj = 0; jj < VD / 64; ++jj) tma_store_4d(&mdV, sm + SM::kVt + jj * kQ * 128, 64 * jj, h, t0, b);
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// Fixed-order sums of the per-tile SSD parameter partials over batch rows and chunks.
+__global__ void ssd_param_reduce(const float* __restrict__ pdA, const float* __restrict__ pdD, int B, int H,
+                                 int nchunk, float* __restrict__ dA, float* __restrict__ dD) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    float sa = 0.0f, sd = 0.0f;
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < nchunk; ++c) {
+            const size_t t = ((size_t)b * H + h) * nchunk + c;
+            sa += pdA[t];
+            sd += pdD[t];
+        }
+    dA[h] = sa;
+    if (dD) dD[h] = sd;
+}
+
+struct ChunkBwdWs {
+    size_t flags, aggA, pdA, pdD, agg, pre, end;
+};
+
+ChunkBwdWs bwd_plan(const lr_desc& d) {
+    const size_t tiles = (size_t)d.B * d.H * ((d.L + kQ - 1) / kQ);
+    const size_t VD = (size_t)d.P;
+    WsCursor c;
+    ChunkBwdWs w;
+    w.flags = c.take(sizeof(unsigned int) * tiles);
+    w.aggA = c.take(sizeof(float) * tiles);
+    w.pdA = c.take(sizeof(float) * tiles);
+    w.pdD = c.take(sizeof(float) * tiles);
+    w.agg = c.take(sizeof(float) * tiles * kKD * VD);
+    w.pre = c.take(sizeof(float) * tiles * kKD * VD);
+    w.end = c.off;
+    return w;
+}
+
+}  // namespace
+
+size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only) {
+    ChunkBwdWs w = bwd_plan(d);
+    return flags_only ? w.aggA : w.end;
+}
+
+lr_status chunk_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
+                    const lr_grads& gr, char* ws, cudaStream_t st) {
+    ChunkBwdWs w = bwd_plan(d);
+    ChunkBwdArgs bw{};
+    ChunkArgs& a = bw.f;
+    a.kind = d.kind;
+    a.B = (int)d.B;
+    a.L = (int)d.L;
+    a.H = (int)d.H;
+    a.G = d.kind == LR_SSD ? (int)d.G : (int)d.H;
+    a.nchunk = (int)((d.L + kQ - 1) / kQ);
+    a.VD = (int)d.P;
+    a.lam = (const __nv_bfloat16*)(d.kind == LR_SSD ? in.delta : in.g);
+    a.A = in.A;
+    a.Dskip = (d.kind == LR_SSD && (d.flags & LR_HAS_DSKIP)) ? in.Dskip : nullptr;
+    a.ckpt = (float*)const_cast<void*>(ckpt);
+    a.hdr = (WsHeader*)ws;
+    a.dflags = d.flags;
+    bw.kg = (const __nv_bfloat16*)(d.kind == LR_SSD ? in.Bm : in.k);
+    bw.dy = (const __nv_bfloat16*)dy;
+    bw.dlam = (__nv_bfloat16*)(d.kind == LR_SSD ? gr.ddelta : gr.dg);
+    bw.dBm = gr.dBm;
+    bw.dCm = gr.dCm;
+    bw.flags = (unsigned int*)(ws + w.flags);
+    bw.agg = (float*)(ws + w.agg);
+    bw.aggA = (float*)(ws + w.aggA);
+    bw.pre = (float*)(ws + w.pre);
+    bw.pdA = (float*)(ws + w.pdA);
+    bw.pdD = (float*)(ws + w.pdD);
+    const bool ssd = d.kind == LR_SSD;
+    if (ssd) {
+        const size_t n = (size_t)d.B * d.L * d.G * kKD * sizeof(float);
+        if (cudaMemsetAsync(gr.dBm, 0, n, st) != cudaSuccess || cudaMemsetAsync(gr.dCm, 0, n, st) != cudaSuccess)
+            return LR_ERR_CUDA;
+    }
+    CUtensorMap mQ, mK, mV, mO, mdQ, mdK, mdV;
+    const void* q = ssd ? in.Cm : in.q;
+    const void* k = ssd ? in.Bm : in.k;
+    const void* v = ssd ? in.x : in.v;
+    const uint64_t QX = ssd ? (uint64_t)d.G : (uint64_t)d.H;
+    bool okm = map4(&mQ, q, kKD, QX, d.L, d.B, true) && map4(&mK, k, kKD, QX, d.L, d.B, true) &&
+               map4(&mV, v, d.P, d.H, d.L, d.B, true) && map4(&mO, dy, d.P, d.H, d.L, d.B, true) &&
+               map4(&mdV, ssd ? gr.dx : gr.dv, d.P, d.H, d.L, d.B, true) &&
+               map4(&mdQ, ssd ? gr.dx : gr.dq, ssd ? d.P : kKD, d.H, d.L, d.B, true) &&
+               map4(&mdK, ssd ? gr.dx : gr.dk, ssd ? d.P : kKD, d.H, d.L, d.B, true);
+    if (!okm) return LR_ERR_INVALID_ARG;
+    const int grid = a.B * a.H * a.nchunk;
+    if (d.P == 64) {
+        using SM = BwdSmem<64>;
+        cudaFuncSetAttribute(chunk_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        note_launch(ssd ? "ssd_bwd_chunk" : "gla_bwd_chunk");
+        chunk_bwd_kernel<64><<<grid, kThreads, SM::kAlloc, st>>>(mQ, mK, mV, mO, mdQ, mdK, mdV, bw);
+    } else {
+        using SM = BwdSmem<128>;
+        cudaFuncSetAttribute(chunk_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        note_launch(ssd ? "ssd_bwd_chunk" : "gla_bwd_chunk");
+        chunk_bwd_kernel<128><<<grid, kThreads, SM::kAlloc, st>>>(mQ, mK, mV, mO, mdQ, mdK, mdV, bw);
+    }
+    lr_status s = check_launch();
+    if (s != LR_OK || !ssd) return s;
+    note_launch("ssd_param_reduce");
+    ssd_param_reduce<<<(a.H + 127) / 128, 128, 0, st>>>(bw.pdA, bw.pdD, a.B, a.H, a.nchunk, gr.dA,
+                                                         (d.flags & LR_HAS_DSKIP) ? gr.dDskip : nullptr);
+    return check_launch();
 }
 
 }  // namespace lrs

@@ -1,43 +1,43 @@
 """GPU parity of the chunked-matmul kinds (SSD, GLA; tcgen05 tensor cores) against the fp64
-oracle.  bf16 I/O, tolerance max|err| <= 2e-2 max|ref| per tensor.  Cases cover several chunks
-chained through the look-back, a ragged last chunk (L not a multiple of 128), a single chunk,
-several heads per group (SSD), and the workloads at full size on sampled heads."""
+oracle.  bf16 I/O, tolerance max|err| <= 2e-2 max|ref| per tensor (y, checkpoints, every
+gradient).  Cases cover several chunks chained through the forward and reverse look-backs, a
+ragged last chunk (L not a multiple of 128), a single chunk, several heads per group (SSD), both
+value widths (64, 128), and the workloads at full size on sampled heads."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from helpers import assert_close, gpu_inputs, to64
-from selective_state_space_09_b200 import inputs, lrscan
+from helpers import assert_close, run_gpu, to64
+from selective_state_space_09_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
 
-
-def fwd_only(kind, inp, disc="none"):
-    g = gpu_inputs(inp)
-    g.pop("dy")
-    g = {k: v for k, v in g.items() if v is not None}
-    plan = lrscan.plan_for(kind, g, 128, disc, 128)
-    y, _ = lrscan.alloc_outputs(kind, g)
-    plan.fwd(g, y)
-    disp = lrscan.last_dispatch()
-    torch.cuda.synchronize()
-    return y, plan.ckpt_view().clone(), plan, disp
-
-
 SSD_CASES = [(1, 512, 4, 64, 1), (2, 300, 8, 64, 2), (1, 128, 2, 64, 1), (1, 77, 8, 64, 1)]
 
 
+def _ssd_ref(inp):
+    a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], None)
+    ry, rck = oracle.ssd_fwd(*a, disc="zoh", S=128)
+    rg = oracle.ssd_bwd(*a, inp["dy"], disc="zoh")
+    return ry, rck, rg
+
+
 @pytest.mark.parametrize("B,L,H,P,G", SSD_CASES)
-def test_ssd_forward(B, L, H, P, G):
+def test_ssd_parity(B, L, H, P, G):
     inp = inputs.ssd(B, L, H, P, 128, G=G, seed=B * 31 + L)
-    y, ck, plan, disp = fwd_only("ssd", inp, "zoh")
-    ry, rck = oracle.ssd_fwd(inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"],
-                             None, disc="zoh", S=128)
+    y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc="zoh", chunk=128)
+    ry, rck, rg = _ssd_ref(inp)
     assert_close("y", y, ry, TOL)
     assert_close("ckpt", ck.transpose(-1, -2), rck, TOL)   # kernel state [N, P], oracle [P, N]
-    assert disp == "ssd_fwd_chunk"
+    assert_close("dx", gr["dx"], rg["x"], TOL)
+    assert_close("ddelta", gr["ddelta"], rg["delta"], TOL)
+    assert_close("dA", gr["dA"], rg["A"], TOL)
+    assert_close("dB", gr["dBm"], rg["B"], TOL)
+    assert_close("dC", gr["dCm"], rg["C"], TOL)
+    assert_close("dD", gr["dDskip"], rg["D"], TOL)
+    assert disp == ("ssd_fwd_chunk", "ssd_bwd_chunk+ssd_param_reduce")
     assert plan.device_error() == (0, 0)
 
 
@@ -45,11 +45,70 @@ GLA_CASES = [(1, 512, 2, 128), (2, 300, 3, 128), (1, 128, 1, 128), (2, 200, 2, 6
 
 
 @pytest.mark.parametrize("B,L,H,V", GLA_CASES)
-def test_gla_forward(B, L, H, V):
+def test_gla_parity(B, L, H, V):
     inp = inputs.gla(B, L, H, 128, V, seed=B * 17 + L)
-    y, ck, plan, disp = fwd_only("gla", inp)
+    y, ck, gr, plan, disp = run_gpu("gla", inp, 128, chunk=128)
     ry, rck = oracle.gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], S=128)
+    rg = oracle.gla_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["dy"])
     assert_close("o", y, ry, TOL)
     assert_close("ckpt", ck, rck, TOL)
-    assert disp == "gla_fwd_chunk"
+    for gk, rk in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g")):
+        assert_close(gk, gr[gk], rg[rk], TOL)
+    assert disp == ("gla_fwd_chunk", "gla_bwd_chunk")
     assert plan.device_error() == (0, 0)
+
+
+def test_gla_deterministic():
+    inp = inputs.gla(2, 384, 2, 128, 128, seed=3)
+    a = run_gpu("gla", inp, 128, chunk=128)
+    b = run_gpu("gla", inp, 128, chunk=128)
+    assert torch.equal(a[0], b[0])
+    for k in a[2]:
+        assert torch.equal(a[2][k], b[2][k]), k
+
+
+@pytest.mark.slow
+def test_ssd_full_size_sampled():
+    """The SSD workload (B=2, H=32, P=64, N=128, L=4096).  The oracle recomputes sampled heads over
+    both batch rows (dA, dD exact per head); dB and dC (sums over the 32 heads of batch row 0) are
+    checked against the oracle on the whole of batch row 0."""
+    w = inputs.WORKLOADS["ssd"]
+    inp = inputs.ssd(w["B"], w["L"], w["H"], w["P"], w["N"], seed=0, device="cuda")
+    y, ck, gr, plan, _ = run_gpu("ssd", inp, w["segment"], disc="zoh", chunk=w["chunk"])
+    assert plan.device_error() == (0, 0)
+    oracle.set_threads(8)
+    for h in (0, 13, 31):
+        sl = slice(h, h + 1)
+        sub = {"x": inp["x"][:, :, sl], "delta": inp["delta"][:, :, sl], "A": inp["A"][sl],
+               "Bm": inp["Bm"], "Cm": inp["Cm"], "Dskip": inp["Dskip"][sl], "dy": inp["dy"][:, :, sl]}
+        sub = {k: to64(v) for k, v in sub.items()}
+        ry, rck, rg = _ssd_ref(sub)
+        assert_close("y[h=%d]" % h, y[:, :, sl], ry, TOL)
+        assert_close("ckpt[h=%d]" % h, ck[:, :, sl].transpose(-1, -2), rck, TOL)
+        assert_close("dx[h=%d]" % h, gr["dx"][:, :, sl], rg["x"], TOL)
+        assert_close("ddelta[h=%d]" % h, gr["ddelta"][:, :, sl], rg["delta"], TOL)
+        assert_close("dA[h=%d]" % h, gr["dA"][sl], rg["A"], TOL)
+        assert_close("dD[h=%d]" % h, gr["dDskip"][sl], rg["D"], TOL)
+    sub = {k: (to64(v[0:1]) if k not in ("A", "Dskip") else to64(v)) for k, v in inp.items() if v is not None}
+    sub["z"] = None
+    _, _, rg = _ssd_ref(sub)
+    assert_close("dB[b=0]", gr["dBm"][0:1], rg["B"], TOL)
+    assert_close("dC[b=0]", gr["dCm"][0:1], rg["C"], TOL)
+
+
+@pytest.mark.slow
+def test_gla_full_size_sampled():
+    """The GLA workload (B=4, H=16, K=V=128, L=2048) on sampled (batch row, head) units."""
+    w = inputs.WORKLOADS["gla"]
+    inp = inputs.gla(w["B"], w["L"], w["H"], w["K"], w["V"], seed=0, device="cuda")
+    y, ck, gr, plan, _ = run_gpu("gla", inp, w["segment"], chunk=w["chunk"])
+    assert plan.device_error() == (0, 0)
+    oracle.set_threads(4)
+    for b, h in ((0, 0), (3, 15), (1, 7)):
+        sub = {k: to64(v[b:b + 1, :, h:h + 1]) for k, v in inp.items()}
+        ry, rck = oracle.gla_fwd(sub["q"], sub["k"], sub["v"], sub["g"], S=128)
+        rg = oracle.gla_bwd(sub["q"], sub["k"], sub["v"], sub["g"], sub["dy"])
+        assert_close("o[%d,%d]" % (b, h), y[b:b + 1, :, h:h + 1], ry, TOL)
+        assert_close("ckpt[%d,%d]" % (b, h), ck[:, b:b + 1, h:h + 1], rck, TOL)
+        for gk, rk in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g")):
+            assert_close("%s[%d,%d]" % (gk, b, h), gr[gk][b:b + 1, :, h:h + 1], rg[rk], TOL)

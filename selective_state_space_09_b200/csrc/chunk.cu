@@ -95,35 +95,139 @@ __device__ __forceinline__ float cta_inclusive_sum(float x, float* tmp) {
     return x + add;
 }
 
-// Shared-memory plan of the forward tile (offsets from a 1024-aligned base).
+// Nearest chunk, walking from `c` in direction `dir`, whose inclusive record is published
+// (flags read four at a time; an unpublished flag is waited for, with a bound).  Returns `stop`
+// (-1 or nchunk) if the walk leaves the row.  A wait that gives up counts as published (the
+// error is recorded and the caller proceeds with whatever the record holds).
+__device__ __forceinline__ int find_prefix(const unsigned int* flags, int c, int dir, int nchunk,
+                                           WsHeader* hdr, int info) {
+    int j = c + dir;
+    const int stop = dir < 0 ? -1 : nchunk;
+    while (j != stop) {
+        unsigned int f[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int jj = j + k * dir;
+            f[k] = (jj >= 0 && jj < nchunk) ? ld_acquire(&flags[jj]) : kFlagPrefix;
+        }
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+            const int jj = j + k * dir;
+            if (jj < 0 || jj >= nchunk) return stop;
+            unsigned int fk = f[k];
+            if (fk == kFlagNone) fk = wait_flag(&flags[jj], hdr, info);
+            if (fk != kFlagAgg) return jj;  // prefix (or a wait that gave up)
+        }
+        j += 4 * dir;
+    }
+    return stop;
+}
+
+// x[0..16) = fold in chain order of the aggregates first .. last (x <- a_i x + agg_i) starting
+// from the 16 values at `pre` (or zero).  agg_row0 points at the caller's row inside record 0;
+// records are `rec_stride` floats apart and indexed row0 + i.  dir = +1 folds i = first .. last-1
+// upwards, dir = -1 folds i = first .. last+1 downwards.  Loads of up to three records are issued
+// together.
+__device__ __forceinline__ void fold_chain(float* x, const float* pre, const float* agg_row0, size_t rec_stride,
+                                           const float* aggA, size_t row0, int first, int last, int dir) {
+    float4 p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = pre ? __ldcg(reinterpret_cast<const float4*>(pre) + e) : make_float4(0, 0, 0, 0);
+    int i = first;
+    while (i != last) {
+        float4 r[3][4];
+        float ar[3];
+        int n = 0;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int ii = i + k * dir;
+            const bool live = dir > 0 ? ii < last : ii > last;
+            if (live) {
+                const float* src = agg_row0 + (row0 + ii) * rec_stride;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) r[k][e] = __ldcg(reinterpret_cast<const float4*>(src) + e);
+                ar[k] = __ldcg(&aggA[row0 + ii]);
+                n = k + 1;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            if (k < n) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    p[e].x = fmaf(ar[k], p[e].x, r[k][e].x);
+                    p[e].y = fmaf(ar[k], p[e].y, r[k][e].y);
+                    p[e].z = fmaf(ar[k], p[e].z, r[k][e].z);
+                    p[e].w = fmaf(ar[k], p[e].w, r[k][e].w);
+                }
+            }
+        }
+        i += n * dir;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        x[4 * e] = p[e].x;
+        x[4 * e + 1] = p[e].y;
+        x[4 * e + 2] = p[e].z;
+        x[4 * e + 3] = p[e].w;
+    }
+}
+
+// Fire-and-forget vector add of four floats to global memory (relaxed, gpu scope).
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
+// Scale row r (cols [0, cols)) of an SW128 tile with `rows` rows by w, in place.
+__device__ __forceinline__ void scale_row(char* tile, int r, int cols, int rows, float w) {
+    for (int c0 = 0; c0 < cols; c0 += 8) {
+        uint4 raw = *reinterpret_cast<const uint4*>(tile + tc::sw128_off(r, c0, rows));
+        __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(hv[i]);
+            hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
+        }
+        *reinterpret_cast<uint4*>(tile + tc::sw128_off(r, c0, rows)) = raw;
+    }
+}
+
+// Shared-memory plan of the forward tile (offsets from a 1024-aligned base).  P lives in tensor
+// memory, K is rescaled in place once Q K^T is done, and the output is staged in the Q tile after
+// the last product that reads Q, so the SSD tile (V = 64) needs under 100 KB: two CTAs per SM.
 template <int VD>
 struct FwdSmem {
-    static constexpr size_t kQt = 0;                                  // 128 x 128 bf16
-    static constexpr size_t kKt = kQt + kQ * kKD * 2;                 // 128 x 128
-    static constexpr size_t kVt = kKt + kQ * kKD * 2;                 // 128 x VD
-    static constexpr size_t kVs = kVt + kQ * VD * 2;                  // scaled copy of V
-    static constexpr size_t kPt = kVs + kQ * VD * 2;                  // 128 x 128 (P), then y
-    static constexpr size_t kSt = kPt + kQ * kQ * 2;                  // KD x VD (S_in bf16)
-    static constexpr size_t kL2 = kSt + kKD * VD * 2;                 // l * log2e [128]
-    static constexpr size_t kBeta = kL2 + kQ * 4;                     // beta [128]
-    static constexpr size_t kTmp = kBeta + kQ * 4;                    // scan scratch, misc
-    static constexpr size_t kBar = kTmp + 64;                         // 6 mbarriers
-    static constexpr size_t kTmem = kBar + 64;                        // TMEM base address
+    static constexpr size_t kQt = 0;                       // 128 x 128 bf16 (q / C), then y staging
+    static constexpr size_t kKt = kQt + kQ * kKD * 2;      // 128 x 128 (k / B), then diag(w) K
+    static constexpr size_t kVt = kKt + kQ * kKD * 2;      // 128 x VD (v / x)
+    static constexpr size_t kSt = kVt + kQ * VD * 2;       // KD x VD (S_in bf16)
+    static constexpr size_t kL2 = kSt + kKD * VD * 2;      // l * log2e [128]
+    static constexpr size_t kBeta = kL2 + kQ * 4;          // beta [128]
+    static constexpr size_t kTmp = kBeta + kQ * 4;         // scan scratch, misc
+    static constexpr size_t kBar = kTmp + 64;              // mbarriers
+    static constexpr size_t kTmem = kBar + 64;             // TMEM base address
     static constexpr size_t kEnd = kTmem + 64;
-    static constexpr size_t kAlloc = kEnd + 1024;                     // + alignment slack
+    static constexpr size_t kAlloc = kEnd + 1024;          // + alignment slack
+    static constexpr uint32_t kTmemCols = VD <= 64 ? 256 : 512;
+    static constexpr int kMinBlocks = VD <= 64 ? 2 : 1;
+    static_assert(kAlloc <= 232448, "forward tile exceeds the shared memory of one CTA");
 };
 
-// TMEM columns of the forward tile
-constexpr uint32_t kColS1 = 0;    // 128: Q K^T, then Y2
-constexpr uint32_t kColY = 128;   // VD
-constexpr uint32_t kColSl = 256;  // VD
+// TMEM columns of the forward tile: Q K^T (f32, 128 columns), overwritten in place by P (bf16
+// pairs, 64 columns) and later by Y2; Y; Sl.
+constexpr uint32_t kColS1 = 0;
+constexpr uint32_t kColY = 128;
+template <int VD> constexpr uint32_t col_sl() { return 128 + VD; }
 
 template <int VD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, FwdSmem<VD>::kMinBlocks)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                  const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mY,
                  ChunkArgs a) {
     using SM = FwdSmem<VD>;
+    constexpr uint32_t kColSl = col_sl<VD>();
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);  // 0 load, 1 G1, 2 G2, 3 G4, 4 G3
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
@@ -132,8 +236,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
     int* misc = reinterpret_cast<int*>(sm + SM::kTmp + 32);
     const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sV = smem_u32(sm + SM::kVt),
-                   sVs = smem_u32(sm + SM::kVs), sP = smem_u32(sm + SM::kPt), sS = smem_u32(sm + SM::kSt);
+                   sS = smem_u32(sm + SM::kSt);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
     if (tid == 0) {
         const unsigned int tk = take_ticket(a.hdr, 0);
@@ -145,7 +250,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    if (warp == 0) tc::tmem_alloc(tmem_slot, SM::kTmemCols);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -181,48 +286,46 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     __syncwarp();
     ok = ok && mbar_wait(&bar[1], 0, a.hdr, 501);
     tc::fence_after_sync();
-    // P[t, s] = Sqk[t, s] e^{l_t - l_s} beta_s for s <= t, as a K-major bf16 tile
     {
+        // P[t, s] = Sqk[t, s] e^{l_t - l_s} beta_s (s <= t) as bf16 pairs, written over the Sqk
+        // columns it has already read (32 f32 columns in, 16 packed columns out, lower addresses)
         const int t = tid;
         const float lt2 = l2[t];
-        char* P = sm + SM::kPt;
-        for (int s0 = 0; s0 < kQ; s0 += 16) {
-            float v[16];
-            tc::ld16(tmem + kColS1 + ((uint32_t)(warp * 32) << 16) + s0, v);
+#pragma unroll 1
+        for (int s0 = 0; s0 < kQ; s0 += 32) {
+            uint32_t pk[16];
+            if (s0 > warp * 32 + 31) {  // every row of this warp is above the diagonal block
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                tc::st16(tmem + kColS1 + lane_off + (s0 >> 1), pk);
+                continue;
+            }
+            float v[32];
+            tc::ld16(tmem + kColS1 + lane_off + s0, v);
+            tc::ld16(tmem + kColS1 + lane_off + s0 + 16, v + 16);
             tc::wait_ld();
-            __align__(16) __nv_bfloat16 pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int s = s0 + i;
-                const float p = (s <= t) ? v[i] * ex2(lt2 - l2[s]) * betas[s] : 0.0f;
-                pk[i] = __float2bfloat16_rn(p);
+                const int s = s0 + 2 * i;
+                const float p0 = (s <= t) ? v[2 * i] * ex2(lt2 - l2[s]) * betas[s] : 0.0f;
+                const float p1 = (s + 1 <= t) ? v[2 * i + 1] * ex2(lt2 - l2[s + 1]) * betas[s + 1] : 0.0f;
+                __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+                pk[i] = *reinterpret_cast<uint32_t*>(&pr);
             }
-            *reinterpret_cast<uint4*>(P + tc::sw128_off(t, s0, kQ)) = *reinterpret_cast<uint4*>(&pk[0]);
-            *reinterpret_cast<uint4*>(P + tc::sw128_off(t, s0 + 8, kQ)) = *reinterpret_cast<uint4*>(&pk[8]);
+            tc::st16(tmem + kColS1 + lane_off + (s0 >> 1), pk);
         }
-        // scaled copy of V: row s times w_s = e^{l_Q - l_s} beta_s
-        const float w = ex2(lQ2 - l2[t]) * betas[t];
-        const char* V = sm + SM::kVt;
-        char* Vs = sm + SM::kVs;
-        for (int v0 = 0; v0 < VD; v0 += 8) {
-            uint4 raw = *reinterpret_cast<const uint4*>(V + tc::sw128_off(t, v0, kQ));
-            __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float2 f = __bfloat1622float2(hv[i]);
-                hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
-            }
-            *reinterpret_cast<uint4*>(Vs + tc::sw128_off(t, v0, kQ)) = raw;
-        }
+        tc::wait_st();
+        // K rows scaled by w_s = e^{l_Q - l_s} beta_s (the A operand of G4); G1 is complete
+        scale_row(sm + SM::kKt, t, kKD, kQ, ex2(lQ2 - l2[t]) * betas[t]);
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     if (tid == 0 && ok) {
         tc::fence_after_sync();
-        tc::mma_tiles(tmem + kColY, sP, 0, kQ, sV, 1, kQ, kQ, VD, kQ, 0);      // G2: Y = P V
+        tc::mma_ts_tiles(tmem + kColY, tmem + kColS1, sV, 1, kQ, VD, kQ, 0);  // G2: Y = P V
         tc::commit(&bar[2]);
-        tc::mma_tiles(tmem + kColSl, sK, 1, kQ, sVs, 1, kQ, kKD, VD, kQ, 0);  // G4: Sl = K^T (w V)
+        tc::mma_tiles(tmem + kColSl, sK, 1, kQ, sV, 1, kQ, kKD, VD, kQ, 0);   // G4: Sl = (w K)^T V
         tc::commit(&bar[3]);
     }
     __syncwarp();
@@ -236,7 +339,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     if (c > 0 && has_succ) {
         for (int v0 = 0; v0 < VD; v0 += 16) {
             float v[16];
-            tc::ld16(tmem + kColSl + ((uint32_t)(warp * 32) << 16) + v0, v);
+            tc::ld16(tmem + kColSl + lane_off + v0, v);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
@@ -250,93 +353,70 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
 
     // look-back: state entering this chunk (row kd), deterministic fold in chain order
     const size_t row0 = ((size_t)b * a.H + h) * a.nchunk;
-    int j = c - 1;
-    while (j >= 0) {
-        unsigned int f = wait_flag(&a.flags[row0 + j], a.hdr, 503);
-        if (f == kFlagPrefix || f == kFlagNone) break;
-        --j;
-    }
-    // j: nearest chunk with a published inclusive state (its state is ckpt slot j + 1), or -1
+    const int j = find_prefix(a.flags + row0, c, -1, a.nchunk, a.hdr, 503);
+    // j: nearest earlier chunk with a published inclusive state (checkpoint slot j + 1), or -1.
+    // For every 16 columns: fold (prefix, aggregates j+1 .. c-1) into the entering state S_in
+    // (checkpoint slot c, written by the predecessor as its inclusive state; chunk 0 writes the
+    // zero slot), its bf16 copy (MN-major B of G3), and the inclusive state
+    // S_out = e^{l_Q} S_in + Sl into slot c + 1.
     float* ck_in = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + kd) * VD;
+    float* ck_out = a.ckpt + ((((size_t)(c + 1) * a.B + b) * a.H + h) * kKD + kd) * VD;
+    const float* pre_row = j >= 0 ? a.ckpt + ((((size_t)(j + 1) * a.B + b) * a.H + h) * kKD + kd) * VD : nullptr;
+    const float aq = ex2(lQ2);
     char* St = sm + SM::kSt;
+#pragma unroll 1
     for (int v0 = 0; v0 < VD; v0 += 16) {
         float x[16];
-        if (j >= 0) {
-            const float* src = a.ckpt + ((((size_t)(j + 1) * a.B + b) * a.H + h) * kKD + kd) * VD + v0;
+        fold_chain(x, pre_row ? pre_row + v0 : nullptr, a.agg + (size_t)kd * VD + v0, (size_t)kKD * VD,
+                   a.aggA, row0, j + 1, c, +1);
+        if (c == 0) {  // slot 0 (zero state); later slots are written by the predecessor
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
-                x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(ck_in + v0 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
         }
-        for (int i = j + 1; i < c; ++i) {
-            const float ai = __ldcg(&a.aggA[row0 + i]);
-            const float* src = a.agg + (row0 + i) * kKD * VD + (size_t)kd * VD + v0;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-                float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
-                x[e] = fmaf(ai, x[e], f.x); x[e + 1] = fmaf(ai, x[e + 1], f.y);
-                x[e + 2] = fmaf(ai, x[e + 2], f.z); x[e + 3] = fmaf(ai, x[e + 3], f.w);
-            }
-        }
-        // checkpoint slot c = state entering this chunk (the predecessor writes the same bits as its
-        // inclusive state); bf16 copy as the MN-major B operand of G3
-#pragma unroll
-        for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(ck_in + v0 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
         __align__(16) __nv_bfloat16 pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = __float2bfloat16_rn(x[i]);
         *reinterpret_cast<uint4*>(St + tc::sw128_off(kd, v0, kKD)) = *reinterpret_cast<uint4*>(&pk[0]);
         *reinterpret_cast<uint4*>(St + tc::sw128_off(kd, v0 + 8, kKD)) = *reinterpret_cast<uint4*>(&pk[8]);
+        if (has_succ) {
+            float v[16];
+            tc::ld16(tmem + kColSl + lane_off + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                __stcg(reinterpret_cast<float4*>(ck_out + v0 + i),
+                       make_float4(fmaf(aq, x[i], v[i]), fmaf(aq, x[i + 1], v[i + 1]), fmaf(aq, x[i + 2], v[i + 2]),
+                                   fmaf(aq, x[i + 3], v[i + 3])));
+        }
     }
+    const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && c == 0;
+    if (has_succ) __threadfence();
+    ok = ok && mbar_wait(&bar[2], 0, a.hdr, 504);  // G2 done: P's columns can take Y2
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    if (tid == 0 && ok && c > 0) {  // G3: Y2 = Q S_in (reuses the Sqk columns)
+    if (tid == 0 && has_succ && !withhold) st_release(&a.flags[tile], kFlagPrefix);
+    if (tid == 0 && ok && c > 0) {  // G3: Y2 = Q S_in (in the Sqk / P columns)
         tc::fence_after_sync();
         tc::mma_tiles(tmem + kColS1, sQ, 0, kQ, sS, 1, kKD, kQ, VD, kKD, 0);
         tc::commit(&bar[4]);
     }
-    // inclusive state of this chunk: S_out = e^{l_Q} S_in + Sl  ->  checkpoint slot c + 1
-    const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && c == 0;
-    if (has_succ) {
-        const float aq = ex2(lQ2);
-        float* ck_out = a.ckpt + ((((size_t)(c + 1) * a.B + b) * a.H + h) * kKD + kd) * VD;
-        for (int v0 = 0; v0 < VD; v0 += 16) {
-            float v[16];
-            tc::ld16(tmem + kColSl + ((uint32_t)(warp * 32) << 16) + v0, v);
-            tc::wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                const float4 sin = *reinterpret_cast<const float4*>(ck_in + v0 + i);
-                __stcg(reinterpret_cast<float4*>(ck_out + v0 + i),
-                       make_float4(fmaf(aq, sin.x, v[i]), fmaf(aq, sin.y, v[i + 1]), fmaf(aq, sin.z, v[i + 2]),
-                                   fmaf(aq, sin.w, v[i + 3])));
-            }
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && !withhold) st_release(&a.flags[tile], kFlagPrefix);
-    }
-
-    // output rows: y_t = Y_t + e^{l_t} Y2_t (+ D x_t)
-    ok = ok && mbar_wait(&bar[2], 0, a.hdr, 504);
+    __syncwarp();
     if (c > 0) ok = ok && mbar_wait(&bar[4], 0, a.hdr, 505);
     tc::fence_after_sync();
+
+    // output rows: y_t = Y_t + e^{l_t} Y2_t (+ D x_t), staged in the Q tile (G3 is complete)
     {
         const int t = tid;
         const float Et = ex2(l2[t]);
         const float Dh = (a.kind == LR_SSD && a.Dskip) ? a.Dskip[h] : 0.0f;
-        char* Yo = sm + SM::kPt;  // P is no longer needed (G2 complete)
+        char* Yo = sm + SM::kQt;
         const char* V = sm + SM::kVt;
         for (int v0 = 0; v0 < VD; v0 += 16) {
             float y1[16], y2[16];
-            tc::ld16(tmem + kColY + ((uint32_t)(warp * 32) << 16) + v0, y1);
-            if (c > 0) tc::ld16(tmem + kColS1 + ((uint32_t)(warp * 32) << 16) + v0, y2);
+            tc::ld16(tmem + kColY + lane_off + v0, y1);
+            if (c > 0) tc::ld16(tmem + kColS1 + lane_off + v0, y2);
             tc::wait_ld();
             __align__(16) __nv_bfloat16 pk[16];
 #pragma unroll
@@ -358,14 +438,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     tc::fence_before_sync();
     __syncthreads();
     if (tid == 0 && ok) {
-        for (int jj = 0; jj < VD / 64; ++jj) tma_store_4d(&mY, sm + SM::kPt + jj * kQ * 128, 64 * jj, h, t0, b);
+        for (int jj = 0; jj < VD / 64; ++jj) tma_store_4d(&mY, sm + SM::kQt + jj * kQ * 128, 64 * jj, h, t0, b);
         bulk_commit();
         bulk_wait_read_all();
     }
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 512);
+        tc::tmem_dealloc(tmem, SM::kTmemCols);
     }
 }
 
@@ -400,7 +480,7 @@ bool chunk_supported(const lr_desc& d) {
     if (d.io != LR_BF16) return false;
     if (d.N != kKD || (d.P != 64 && d.P != 128)) return false;
     if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
-    if (d.kind == LR_SSD && (d.disc != LR_DISC_ZOH || (d.flags & LR_HAS_Z))) return false;
+    if (d.kind == LR_SSD && (d.disc != LR_DISC_ZOH || (d.flags & LR_HAS_Z) || d.P != 64)) return false;
     return d.L <= (1 << 28) && d.H <= 4096;
 }
 
@@ -477,7 +557,8 @@ struct BwdSmem {
     static constexpr size_t kOt = kVt + kQ * VD * 2;      // dO, then diag(E) dO
     static constexpr size_t kPt = kOt + kQ * VD * 2;      // P, then dS_out (bf16, KD x VD)
     static constexpr size_t kPdt = kPt + kQ * kQ * 2;     // Pd, then S_in (bf16, KD x VD)
-    static constexpr size_t kL2 = kPdt + kQ * kQ * 2;     // l log2e [128]
+    static constexpr size_t kYt = kPdt + kQ * kQ * 2;     // dy, unscaled (ssd, V = 64: dx = dv + D dy)
+    static constexpr size_t kL2 = kYt + (VD <= 64 ? kQ * VD * 2 : 0);  // l log2e [128]
     static constexpr size_t kBeta = kL2 + kQ * 4;         // beta [128]
     static constexpr size_t kLam = kBeta + kQ * 4;        // raw per-step input (dt or g) [128]
     static constexpr size_t kRed = kLam + kQ * 4;         // reduction scratch [128]
@@ -486,6 +567,7 @@ struct BwdSmem {
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
+    static_assert(kAlloc <= 232448, "backward tile exceeds the shared memory of one CTA");
 };
 
 constexpr uint32_t kR0 = 0, kR1 = 128, kR2 = 256, kR3 = 384;
@@ -504,31 +586,6 @@ struct ChunkBwdArgs {
     float* pdA;               // SSD per-tile partials
     float* pdD;
 };
-
-__device__ __forceinline__ void fold16(float* x, float a, const float* src) {
-#pragma unroll
-    for (int e = 0; e < 16; e += 4) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
-        x[e] = fmaf(a, x[e], f.x);
-        x[e + 1] = fmaf(a, x[e + 1], f.y);
-        x[e + 2] = fmaf(a, x[e + 2], f.z);
-        x[e + 3] = fmaf(a, x[e + 3], f.w);
-    }
-}
-
-// Scale row r (cols [0, cols)) of an SW128 tile with `rows` rows by w, in place.
-__device__ __forceinline__ void scale_row(char* tile, int r, int cols, int rows, float w) {
-    for (int c0 = 0; c0 < cols; c0 += 8) {
-        uint4 raw = *reinterpret_cast<const uint4*>(tile + tc::sw128_off(r, c0, rows));
-        __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 f = __bfloat1622float2(hv[i]);
-            hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
-        }
-        *reinterpret_cast<uint4*>(tile + tc::sw128_off(r, c0, rows)) = raw;
-    }
-}
 
 template <int VD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -554,11 +611,23 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     const uint32_t colDv = kR1, colDSl = ssd ? kR1 + 64 : kR0;
 
     if (tid == 0) {
-        const unsigned int tk = take_ticket(a.hdr, 1);
-        const int per = a.B * a.H;
-        misc[0] = a.nchunk - 1 - (int)(tk / per);
-        misc[1] = (tk % per) / a.H;
-        misc[2] = tk % a.H;
+        // Tiles are numbered along diagonals key = (nchunk - 1 - c) + h, so that tiles running at
+        // the same time sit at different chunks of different heads (SSD's dB / dC sums over heads
+        // then do not collide), while every tile's reverse-chain dependency (c + 1, key - 1) has
+        // a smaller number.
+        unsigned int tk = take_ticket(a.hdr, 1);
+        int key = 0, lo = 0, n = 0;
+        for (;; ++key) {
+            lo = max(0, key - (a.nchunk - 1));
+            const int hi = min(a.H - 1, key);
+            n = hi - lo + 1;
+            if (tk < (unsigned int)(a.B * n)) break;
+            tk -= a.B * n;
+        }
+        const int hh = lo + (int)(tk % n);
+        misc[0] = a.nchunk - 1 - (key - hh);
+        misc[1] = (int)(tk / n);
+        misc[2] = hh;
         for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -576,7 +645,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     const bool last = c + 1 >= a.nchunk;
 
     if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2 + 2 * kQ * VD * 2));
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2 + (ssd ? 3 : 2) * kQ * VD * 2));
         for (int j = 0; j < kKD / 64; ++j) {
             tma_load_4d(sm + SM::kQt + j * kQ * 128, &mQ, &bar[0], 64 * j, gq, t0, b);
             tma_load_4d(sm + SM::kKt + j * kQ * 128, &mK, &bar[0], 64 * j, gq, t0, b);
@@ -584,6 +653,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
         for (int j = 0; j < VD / 64; ++j) {
             tma_load_4d(sm + SM::kVt + j * kQ * 128, &mV, &bar[0], 64 * j, h, t0, b);
             tma_load_4d(sm + SM::kOt + j * kQ * 128, &mO, &bar[0], 64 * j, h, t0, b);
+            if (ssd) tma_load_4d(sm + SM::kYt + j * kQ * 128, &mO, &bar[0], 64 * j, h, t0, b);
         }
     }
     const int r = tid;  // this thread's row (time step in the chunk, or state row kd)
@@ -660,7 +730,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
         const float wb = ex2(lQ2 - l2[r]) * betas[r];
         scale_row(O, r, VD, kQ, E);                   // diag(E) dO
         scale_row(V, r, VD, kQ, wb);                  // diag(W beta) V
-        scale_row(sm + SM::kKt, r, kKD, kQ, wb);      // diag(W beta) K
         // S_in (checkpoint slot c) as bf16, rows kd x cols v, in the Pd region
         const float* sin = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + r) * VD;
         char* St = sm + SM::kPdt;
@@ -702,38 +771,27 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
         __syncthreads();
         if (tid == 0) st_release(&bw.flags[tile], kFlagAgg);
     }
-    // dS_out: walk to the nearest later chunk with an inclusive adjoint, fold in chain order
-    int j = c + 1;
-    while (j < a.nchunk) {
-        const unsigned int f = wait_flag(&bw.flags[row0 + j], a.hdr, 604);
-        if (f == kFlagPrefix || f == kFlagNone) break;
-        ++j;
-    }
+    // dS_out: nearest later chunk with an inclusive adjoint, then the fold in chain order
+    const int j = find_prefix(bw.flags + row0, c, +1, a.nchunk, a.hdr, 604);
     float xdot = 0.0f;  // <dS_out, S_out> restricted to row r
     float* mypre = bw.pre + tile * kKD * VD + (size_t)r * VD;
     char* dSt = sm + SM::kPt;
     const float* sout = a.ckpt + ((((size_t)(c + 1) * a.B + b) * a.H + h) * kKD + r) * VD;
+    const float* pre_row = j < a.nchunk ? bw.pre + (row0 + j) * kKD * VD + (size_t)r * VD : nullptr;
+#pragma unroll 1
     for (int v0 = 0; v0 < VD; v0 += 16) {
-        float x[16];
-        if (j < a.nchunk) {
-            const float* src = bw.pre + (row0 + j) * kKD * VD + (size_t)r * VD + v0;
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
-                x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = 0.0f;
-        }
-        for (int i = j - 1; i > c; --i)
-            fold16(x, __ldcg(&bw.aggA[row0 + i]), bw.agg + (row0 + i) * kKD * VD + (size_t)r * VD + v0);
+        float4 so[4];
         if (!last) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                const float4 so = __ldcg(reinterpret_cast<const float4*>(sout + v0 + i));
-                xdot = fmaf(x[i], so.x, fmaf(x[i + 1], so.y, fmaf(x[i + 2], so.z, fmaf(x[i + 3], so.w, xdot))));
-            }
+            for (int e = 0; e < 4; ++e) so[e] = __ldcg(reinterpret_cast<const float4*>(sout + v0) + e);
+        }
+        float x[16];
+        fold_chain(x, pre_row ? pre_row + v0 : nullptr, bw.agg + (size_t)r * VD + v0, (size_t)kKD * VD, bw.aggA,
+                   row0, j - 1, c, -1);
+        if (!last) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                xdot = fmaf(x[4 * e], so[e].x, fmaf(x[4 * e + 1], so[e].y, fmaf(x[4 * e + 2], so[e].z, fmaf(x[4 * e + 3], so[e].w, xdot))));
         }
         __align__(16) __nv_bfloat16 pk[16];
 #pragma unroll
@@ -763,8 +821,8 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     __syncthreads();
     if (tid == 0 && ok && !last) {
         tc::fence_after_sync();
-        tc::mma_tiles(tmem + kR3, sV, 0, kQ, sP, 0, kKD, kQ, kKD, VD, 1);    // dk += diag(W b) V dS_out^T
-        tc::mma_tiles(tmem + colDv, sK, 0, kQ, sP, 1, kKD, kQ, VD, kKD, 1);  // dv += diag(W b) K dS_out
+        tc::mma_tiles(tmem + kR3, sV, 0, kQ, sP, 0, kKD, kQ, kKD, VD, 1);     // dk += diag(W b) V dS_out^T
+        tc::mma_tiles(tmem + colDSl, sK, 0, kQ, sP, 1, kKD, kQ, VD, kKD, 0);  // K dS_out (dSl is consumed)
         tc::commit(&bar[4]);
     }
     __syncwarp();
@@ -779,7 +837,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
     {
         char* Q = sm + SM::kQt;
         char* K = sm + SM::kKt;
-        const __nv_bfloat16* kglob = bw.kg + (((size_t)b * a.L + min(tr, a.L - 1)) * (ssd ? a.G : a.H) + gq) * kKD;
         for (int k0 = 0; k0 < kKD; k0 += 16) {
             float dq[16], dk[16];
             tc::ld16(tmem + kR2 + lane_off + k0, dq);
@@ -789,7 +846,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 16; i += 8) {
                 uint4 qr = *reinterpret_cast<const uint4*>(Q + tc::sw128_off(r, k0 + i, kQ));
-                uint4 kr = valid ? *reinterpret_cast<const uint4*>(kglob + k0 + i) : make_uint4(0, 0, 0, 0);
+                uint4 kr = *reinterpret_cast<const uint4*>(K + tc::sw128_off(r, k0 + i, kQ));
                 const __nv_bfloat16* qv = reinterpret_cast<const __nv_bfloat16*>(&qr);
                 const __nv_bfloat16* kv = reinterpret_cast<const __nv_bfloat16*>(&kr);
 #pragma unroll
@@ -806,8 +863,8 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
                     float* dB = bw.dBm + (((size_t)b * a.L + tr) * a.G + gq) * kKD + k0;
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
-                        atomicAdd(reinterpret_cast<float4*>(dC + i), make_float4(dq[i], dq[i + 1], dq[i + 2], dq[i + 3]));
-                        atomicAdd(reinterpret_cast<float4*>(dB + i), make_float4(dk[i], dk[i + 1], dk[i + 2], dk[i + 3]));
+                        red_add4(dC + i, dq[i], dq[i + 1], dq[i + 2], dq[i + 3]);
+                        red_add4(dB + i, dk[i], dk[i + 1], dk[i + 2], dk[i + 3]);
                     }
                 }
             } else {
@@ -820,15 +877,21 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__
         // dv (gla) / dx = dv + D dy (ssd) into the V region
         char* V = sm + SM::kVt;
         const float Dh = (ssd && a.Dskip) ? a.Dskip[h] : 0.0f;
-        const __nv_bfloat16* dyr = bw.dy + (((size_t)b * a.L + min(tr, a.L - 1)) * a.H + h) * VD;
+        const char* Yt = sm + SM::kYt;
+        const float wbr = ex2(lQ2 - l2[r]) * betas[r];
         for (int v0 = 0; v0 < VD; v0 += 16) {
-            float dv[16];
+            float dv[16], dvi[16];
             tc::ld16(tmem + colDv + lane_off + v0, dv);
+            if (!last) tc::ld16(tmem + colDSl + lane_off + v0, dvi);
             tc::wait_ld();
+            if (!last) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dv[i] = fmaf(wbr, dvi[i], dv[i]);
+            }
             __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
             for (int i = 0; i < 16; i += 8) {
-                uint4 yr = (valid && ssd) ? *reinterpret_cast<const uint4*>(dyr + v0 + i) : make_uint4(0, 0, 0, 0);
+                uint4 yr = ssd ? *reinterpret_cast<const uint4*>(Yt + tc::sw128_off(r, v0 + i, kQ)) : make_uint4(0, 0, 0, 0);
                 const __nv_bfloat16* yv = reinterpret_cast<const __nv_bfloat16*>(&yr);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[i + e] = __float2bfloat16_rn(fmaf(Dh, __bfloat162float(yv[e]), dv[i + e]));

@@ -71,6 +71,18 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b
         : "memory");
 }
 
+// D[tmem] = A[tmem] * B (+ D if accumulate): A (M = 128 rows = lanes, bf16 pairs packed in 32-bit
+// columns, K/2 columns) read from tensor memory.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -91,6 +103,34 @@ __device__ __forceinline__ void ld16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Store 16 32-bit columns of this thread's lane.
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// M = 128 x N x K product with A in tensor memory (a_tmem: K/2 columns) and B an SW128 tile.
+__device__ __forceinline__ void mma_ts_tiles(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int b_mn, int b_rows,
+                                             int N, int K, uint32_t accumulate_first) {
+    const uint32_t idesc = idesc_bf16(128, N, 0, b_mn);
+    for (int k = 0; k < K; k += 16) {
+        uint32_t b_addr, b_lbo;
+        if (b_mn) {
+            b_addr = b_base + (uint32_t)k * 128u;
+            b_lbo = (uint32_t)b_rows * 128u;
+        } else {
+            b_addr = b_base + (uint32_t)(k >> 6) * b_rows * 128u + (uint32_t)(k & 63) * 2u;
+            b_lbo = 16;
+        }
+        mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), desc_sw128(b_addr, b_lbo, 1024), idesc,
+               (k > 0 || accumulate_first) ? 1u : 0u);
+    }
+}
 
 // Issue an M x N x K product as K/16 MMAs over SW128 tiles.
 //   a: K-major (a_mn = 0: rows = M, 64-wide blocks along K of `a_rows` rows) or MN-major

@@ -47,8 +47,6 @@ INPUT_NAMES = {
     "s6": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z"], "ssd": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z"],
     "gla": ["q", "k", "v", "g"],
 }
-PARAM_GRADS = {"rglru": [], "rotlru": ["dmag", "dtheta"], "s6": ["dA", "dDskip"], "ssd": ["dA", "dDskip"],
-               "gla": []}
 FALLBACK_HBM = 6650.0
 
 
@@ -190,7 +188,7 @@ def tokens_of(w):
 def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu_sample=False):
     import torch
     import torch.distributed as dist
-    from selective_state_space_09_b200 import lrscan
+    from selective_state_space_09_b200 import dp, lrscan
 
     w, inp = workload_inputs(name, device, seed=1000 + rank)
     kind = w["kind"]
@@ -198,14 +196,12 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
     plan = lrscan.plan_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0))
     y, grads = lrscan.alloc_outputs(kind, ai)
     dy = inp["dy"]
-    pgrads = [grads[k] for k in PARAM_GRADS[kind] if k in grads]
 
     def step():
         plan.fwd(ai, y)
         plan.bwd(ai, dy, grads)
         if world > 1:
-            for t in pgrads:
-                dist.all_reduce(t)
+            dp.reduce_param_grads(kind, grads)
 
     for _ in range(warmup):
         step()
@@ -235,8 +231,7 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         e1.record()
         plan.bwd(ai, dy, grads)
         if world > 1:
-            for t in pgrads:
-                dist.all_reduce(t)
+            dp.reduce_param_grads(kind, grads)
         e2.record()
     torch.cuda.synchronize()
     if world > 1:
@@ -267,16 +262,17 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         "l2": "flushed between steps" if flush else "inputs larger than L2",
     }
     if e2e:
-        res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, pgrads, w)
+        res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
     del fl
     return res
 
 
-def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, pgrads, w):
+def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
     """Same step through the public API from pinned host buffers: every step copies its inputs
     host->device, runs forward and backward, and copies y and all gradients back."""
     import torch
     import torch.distributed as dist
+    from selective_state_space_09_b200 import dp
     h_in = {k: v.to("cpu").pin_memory() for k, v in ai.items()}
     h_dy = dy.to("cpu").pin_memory()
     h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -291,8 +287,7 @@ def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, pgrads, w):
         plan.fwd(d_in, y)
         plan.bwd(d_in, d_dy, grads)
         if world > 1:
-            for t in pgrads:
-                dist.all_reduce(t)
+            dp.reduce_param_grads(kind, grads)
         h_y.copy_(y, non_blocking=True)
         for k in grads:
             h_g[k].copy_(grads[k], non_blocking=True)

@@ -89,6 +89,11 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
  * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
 #define LR_TEST_WITHHOLD_CARRY 0x80000000u
+/* Test hook for the work distribution: SSD kernels that loop over the heads of a group inside one
+ * CTA take the largest head blocks they support (16 heads) instead of sizing the blocks to fill
+ * the GPU.  Results are bitwise identical with and without it; small test problems use it to
+ * cover the multi-head pipelines. */
+#define LR_TEST_MAX_HEAD_BLOCK 0x40000000u
 
 /* Problem descriptor.  Unused dimensions are 0.  S6: D, N.  SSD: H, P, N, G, chunk.
  * GLA: H, P (= V), N (= K), chunk.  rglru / rotlru: D.  segment = checkpoint segment length S

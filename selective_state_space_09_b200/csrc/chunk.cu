@@ -24,23 +24,11 @@
 // back to the nearest chunk that has published its inclusive state, and folds the aggregates in
 // chain order (deterministic).  The inclusive states are the checkpoints: the checkpoint segment
 // equals the chunk (128 steps), slot c = state entering chunk c.
-#include "common.cuh"
-#include "host_common.h"
-#include "tc.cuh"
+#include "chunk_common.cuh"
 
 namespace lrs {
+using namespace chunkc;
 namespace {
-
-constexpr int kQ = 128;        // chunk length (rows of every tile, M of every MMA)
-constexpr int kKD = 128;       // key / state-row dimension (N of SSD, K of GLA)
-constexpr int kThreads = 128;  // 4 warps: thread i <-> row / TMEM lane i
-constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 struct ChunkArgs {
     int kind;                 // LR_SSD / LR_GLA
@@ -57,12 +45,6 @@ struct ChunkArgs {
     unsigned int dflags;
 };
 
-__device__ __forceinline__ char* smem_base1024() {
-    extern __shared__ char dyn_smem[];
-    uintptr_t p = reinterpret_cast<uintptr_t>(dyn_smem);
-    return reinterpret_cast<char*>((p + 1023) & ~uintptr_t(1023));
-}
-
 // Per-step log decay and beta of row t (t >= L gives no decay, no input).
 __device__ __forceinline__ void step_coef(const ChunkArgs& a, int b, int h, int t, float& lam, float& beta) {
     lam = 0.0f;
@@ -77,22 +59,6 @@ __device__ __forceinline__ void step_coef(const ChunkArgs& a, int b, int h, int 
         lam = __logf(v);
         beta = 1.0f;
     }
-}
-
-// Inclusive prefix sum over the 128 threads of the CTA (tmp: 4 floats of shared memory).
-__device__ __forceinline__ float cta_inclusive_sum(float x, float* tmp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) tmp[warp] = x;
-    __syncthreads();
-    float add = 0.0f;
-    for (int w = 0; w < warp; ++w) add += tmp[w];
-    __syncthreads();
-    return x + add;
 }
 
 // Nearest chunk, walking from `c` in direction `dir`, whose inclusive record is published
@@ -170,27 +136,6 @@ __device__ __forceinline__ void fold_chain(float* x, const float* pre, const flo
         x[4 * e + 1] = p[e].y;
         x[4 * e + 2] = p[e].z;
         x[4 * e + 3] = p[e].w;
-    }
-}
-
-// Fire-and-forget vector add of four floats to global memory (relaxed, gpu scope).
-__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
-    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
-
-// Scale row r (cols [0, cols)) of an SW128 tile with `rows` rows by w, in place.
-__device__ __forceinline__ void scale_row(char* tile, int r, int cols, int rows, float w) {
-    for (int c0 = 0; c0 < cols; c0 += 8) {
-        uint4 raw = *reinterpret_cast<const uint4*>(tile + tc::sw128_off(r, c0, rows));
-        __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 f = __bfloat1622float2(hv[i]);
-            hv[i] = __floats2bfloat162_rn(f.x * w, f.y * w);
-        }
-        *reinterpret_cast<uint4*>(tile + tc::sw128_off(r, c0, rows)) = raw;
     }
 }
 
@@ -466,14 +411,6 @@ ChunkWs ws_plan(const lr_desc& d) {
     return w;
 }
 
-// rank-4 map of a [B, L, X, W] bf16 tensor (W contiguous) with box [1, 128 rows, 1, 64 cols]
-bool map4(CUtensorMap* m, const void* p, uint64_t W, uint64_t X, uint64_t L, uint64_t B, bool swz) {
-    uint64_t dims[4] = {W, X, L, B};
-    uint64_t str[3] = {W * 2, X * W * 2, L * X * W * 2};
-    uint32_t box[4] = {64, 1, (uint32_t)kQ, 1};
-    return make_tmap(m, p, 2, 4, dims, str, box, swz);
-}
-
 }  // namespace
 
 bool chunk_supported(const lr_desc& d) {
@@ -485,11 +422,18 @@ bool chunk_supported(const lr_desc& d) {
 }
 
 size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only);
-size_t chunk_ws_bytes(const lr_desc& d, bool bwd) { return bwd ? chunk_bwd_ws_end(d, false) : ws_plan(d).end; }
-size_t chunk_flag_bytes(const lr_desc& d, bool bwd) { return bwd ? chunk_bwd_ws_end(d, true) : ws_plan(d).aggA; }
+size_t chunk_ws_bytes(const lr_desc& d, bool bwd) {
+    if (d.kind == LR_SSD) return bwd ? ssd_bwd_ws_bytes(d) : ssd_fwd_ws_bytes(d);
+    return bwd ? chunk_bwd_ws_end(d, false) : ws_plan(d).end;
+}
+size_t chunk_flag_bytes(const lr_desc& d, bool bwd) {
+    if (d.kind == LR_SSD) return bwd ? ssd_bwd_flag_bytes(d) : ssd_fwd_flag_bytes(d);
+    return bwd ? chunk_bwd_ws_end(d, true) : ws_plan(d).aggA;
+}
 
 lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
                     cudaStream_t st) {
+    if (d.kind == LR_SSD) return ssd_fwd(d, in, y, ckpt, ws, st);
     ChunkWs w = ws_plan(d);
     ChunkArgs a{};
     a.kind = d.kind;
@@ -1005,6 +949,7 @@ size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only) {
 
 lr_status chunk_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
                     const lr_grads& gr, char* ws, cudaStream_t st) {
+    if (d.kind == LR_SSD) return ssd_bwd(d, in, dy, ckpt, gr, ws, st);
     ChunkBwdWs w = bwd_plan(d);
     ChunkBwdArgs bw{};
     ChunkArgs& a = bw.f;

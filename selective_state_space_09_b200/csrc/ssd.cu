@@ -1,0 +1,1088 @@
+// ssd.cu -- the SSD scan (state-space duality form of Mamba-2) on tcgen05, organised around the
+// heads of a group sharing B_t and C_t.
+//
+// Recurrence per head h ("mlx-recurrence", Apple Developer Forums thread 840535, "Current
+// kernels": ssd_scan, state [B, H, Dh, N]; the chunked evaluation of the K-Search / mlx-mamba
+// post, paragraph after Table 1):
+//   S_t = e^{dt_t A_h} S_{t-1} + beta_t B_t x_t^T,  beta_t = (e^{dt_t A_h} - 1) / A_h  (ZOH)
+//   y_t = S_t^T C_t + D_h x_t
+// With 128-step chunks, l_t the chunk-local inclusive cumulative log decay, w_t = e^{l_Q - l_t}
+// beta_t and E_t = e^{l_t}:
+//   S_out = e^{l_Q} S_in + Sl,               Sl = B^T diag(w) X
+//   Y     = (M o Lmask) X + diag(E) C S_in,  M = C B^T,  Lmask[t, s] = e^{l_t - l_s} beta_s (s <= t)
+// M is the same for every head of a group: the output kernel computes it once per (batch row,
+// chunk) and runs the group's heads through it.
+//
+// Forward = three launches, none of which waits on another CTA:
+//   ssd_state_kernel  (batch row, chunk, block of 4 heads): Sl of every chunk but the last,
+//                     written into checkpoint slot c + 1; e^{l_Q} per chunk;
+//   ssd_pass_kernel   elementwise over (batch row, head, state element): slot c <- e^{l_Q, c-1}
+//                     slot c-1 + Sl_{c-1}, in place, so slot c ends as the state entering chunk c;
+//   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x.
+#include "chunk_common.cuh"
+
+namespace lrs {
+using namespace chunkc;
+namespace {
+
+constexpr int kP = 64;    // head dimension (value columns)
+constexpr int kHS = 4;    // heads per CTA of the state kernel
+
+struct SsdArgs {
+    int B, L, H, G, HpG, nchunk;  // HpG: heads per group
+    const __nv_bfloat16* dt;      // [B, L, H]
+    const float* A;               // [H]
+    const float* Dskip;           // [H] or null
+    const float* ckpt;            // [nchunk][B][H][N][P] f32 (state entering each chunk)
+    float* decay;                 // [B][H][nchunk] e^{l_Q}
+    WsHeader* hdr;
+};
+
+// Per-step log decay and beta of head h at step t (t >= L: no decay, no input).
+__device__ __forceinline__ void ssd_coef(const SsdArgs& a, int b, int h, int t, float& lam, float& beta) {
+    lam = 0.0f;
+    beta = 0.0f;
+    if (t >= a.L) return;
+    const float v = __bfloat162float(a.dt[((size_t)b * a.L + t) * a.H + h]);
+    const float Ah = a.A[h];
+    lam = v * Ah;
+    beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+}
+
+// ------------------------------------------------------------------------- state increments
+struct StateSmem {
+    static constexpr size_t kR = 0;                                  // 128 x 128 bf16 (B or C)
+    static constexpr size_t kZ = kR + kQ * kKD * 2;                  // kHS tiles 128 x 64 (x or dy)
+    static constexpr size_t kTmp = kZ + (size_t)kHS * kQ * kP * 2;   // scan scratch, l_Q per head
+    static constexpr size_t kBar = kTmp + 128;
+    static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;
+    static_assert(2 * kAlloc <= 232448, "two state CTAs per SM");
+};
+
+// One CTA per (chunk, batch row, group, block of kHS heads):
+//   dir > 0: Sl_c = B^T diag(w) x_h for chunk c = 0 .. nchunk-2, into slot c + 1 of `out`;
+//   dir < 0: U_c = C^T diag(E) dy_h for chunk c = 1 .. nchunk-1, into slot c - 1 of `out`
+//            (the adjoint handed from chunk c to the state leaving chunk c - 1).
+// `decay[(b H + h) nchunk + c]` receives e^{l_Q} of the chunk.
+__global__ void __launch_bounds__(kThreads, 2)
+ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ, SsdArgs a,
+                 float* out, int nblk, int dir) {
+    using SM = StateSmem;
+    char* sm = smem_base1024();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+    int idx = blockIdx.x;
+    const int blk = idx % nblk;
+    idx /= nblk;
+    const int g = idx % a.G;
+    idx /= a.G;
+    const int b = idx % a.B;
+    const int c = idx / a.B + (dir > 0 ? 0 : 1);
+    const int slot = dir > 0 ? c + 1 : c - 1;
+    const int t0 = c * kQ;
+    const int hfirst = g * a.HpG + blk * kHS;
+    const int nh = min(kHS, a.HpG - blk * kHS);
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 256);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(kQ * kKD * 2 + nh * kQ * kP * 2));
+        for (int j = 0; j < kKD / 64; ++j) tma_load_4d(sm + SM::kR + j * kQ * 128, &mR, &bar[0], 64 * j, g, t0, b);
+        for (int j = 0; j < nh; ++j) tma_load_4d(sm + SM::kZ + j * kQ * 128, &mZ, &bar[0], 0, hfirst + j, t0, b);
+    }
+    float l[kHS], beta[kHS];
+#pragma unroll
+    for (int j = 0; j < kHS; ++j) {
+        l[j] = beta[j] = 0.0f;
+        if (j < nh) ssd_coef(a, b, hfirst + j, t0 + tid, l[j], beta[j]);
+    }
+    cta_inclusive_sum_n<kHS>(l, tmp);
+    if (tid == kQ - 1) {
+#pragma unroll
+        for (int j = 0; j < kHS; ++j) tmp[16 + j] = l[j];
+    }
+    __syncthreads();
+    float f[kHS];
+#pragma unroll
+    for (int j = 0; j < kHS; ++j) {
+        const float lQ2 = tmp[16 + j] * kLog2e, lt2 = l[j] * kLog2e;
+        f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] : ex2(lt2);
+        if (tid == j && j < nh) a.decay[((size_t)b * a.H + hfirst + j) * a.nchunk + c] = ex2(lQ2);
+    }
+
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 700);
+#pragma unroll
+    for (int j = 0; j < kHS; ++j)
+        if (j < nh) scale_row(sm + SM::kZ + j * kQ * 128, tid, kP, kQ, f[j]);
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {  // per head: R^T (f o Z), M = state rows (128), N = 64, K = 128 steps
+        tc::fence_after_sync();
+        for (int j = 0; j < nh; ++j)
+            tc::mma_tiles(tmem + kP * j, smem_u32(sm + SM::kR), 1, kQ, smem_u32(sm + SM::kZ + j * kQ * 128), 1, kQ,
+                          kKD, kP, kQ, 0);
+        tc::commit(&bar[1]);
+    }
+    __syncwarp();
+    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 701);
+    tc::fence_after_sync();
+    for (int j = 0; j < nh; ++j) {
+        float* dst = out + ((((size_t)slot * a.B + b) * a.H + hfirst + j) * kKD + tid) * kP;
+#pragma unroll
+        for (int v0 = 0; v0 < kP; v0 += 16) {
+            float v[16];
+            tc::ld16(tmem + kP * j + lane_off + v0, v);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                __stcg(reinterpret_cast<float4*>(dst + v0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------------------- state passing
+// In place over the slots of `buf` ([nchunk][B*H][n4] float4), one thread per (b h, float4):
+//   dir > 0: slot 0 = 0; slot c = decay_{c-1} slot_{c-1} + slot_c, c = 1 .. nchunk-1
+//   dir < 0: slot nchunk-1 = 0; slot c = decay_{c+1} slot_{c+1} + slot_c, c = nchunk-2 .. 0
+// Loads of eight slots are issued ahead of their dependent updates.
+__global__ void __launch_bounds__(256)
+ssd_pass_kernel(float4* buf, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir) {
+    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (size_t)BH * n4) return;
+    const size_t stride = (size_t)BH * n4;
+    const float* dec = decay + (e / n4) * nchunk;
+    float4* p = buf + e;
+    float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const int first = dir > 0 ? 0 : nchunk - 1;
+    p[(size_t)first * stride] = s;
+    for (int k0 = 1; k0 < nchunk; k0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
+            if (k0 + k < nchunk) v[k] = __ldcg(p + (size_t)c * stride);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k0 + k < nchunk) {
+                const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
+                const float d = dec[c - dir];
+                s = make_float4(fmaf(d, s.x, v[k].x), fmaf(d, s.y, v[k].y), fmaf(d, s.z, v[k].z), fmaf(d, s.w, v[k].w));
+                p[(size_t)c * stride] = s;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------- outputs
+// Shared memory of the output CTA: C and B of the chunk, a ring of three x tiles (each becomes
+// the y staging tile of its head), two bf16 S_in tiles, the current head's decays.
+struct OutSmem {
+    static constexpr size_t kC = 0;                          // 128 x 128 bf16
+    static constexpr size_t kB = kC + kQ * kKD * 2;          // 128 x 128 bf16
+    static constexpr size_t kX = kB + kQ * kKD * 2;          // 3 x (128 x 64) bf16
+    static constexpr size_t kSt = kX + 3 * kQ * kP * 2;      // 2 x (128 x 64) bf16, [n][p]
+    static constexpr size_t kL2 = kSt + 2 * kKD * kP * 2;    // l log2e [128]
+    static constexpr size_t kBeta = kL2 + kQ * 4;            // beta [128]
+    static constexpr size_t kCf = kBeta + kQ * 4;            // column factors [4 warps][128]
+    static constexpr size_t kTmp = kCf + 4 * kQ * 4;         // scan scratch
+    static constexpr size_t kBar = kTmp + 64;                // 0 C/B, 1 M, 2..4 x ring, 5..6 MMA
+    static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;
+    static_assert(kAlloc <= 232448, "output CTA exceeds the shared memory of one CTA");
+};
+// TMEM columns: M = C B^T (f32, 128), then two head buffers of P (bf16 pairs, 64), Y (64), Y2 (64).
+__device__ __forceinline__ uint32_t col_p(int j) { return 128u + 192u * j; }
+__device__ __forceinline__ uint32_t col_y(int j) { return 192u + 192u * j; }
+__device__ __forceinline__ uint32_t col_y2(int j) { return 256u + 192u * j; }
+
+// One CTA per (chunk, batch row, group, block of hb heads), heads software-pipelined:
+//   prep(i): decays of head i, S_in -> bf16 tile, P = M o Lmask -> TMEM (bf16 pairs);
+//   issue(i): Y = P X (A from TMEM), Y2 = C S_in;
+//   finish(i - 1): y = Y + E Y2 + D x -> the x tile -> TMA store; the freed x slot loads head i + 2.
+__global__ void __launch_bounds__(kThreads, 1)
+ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
+               const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a, int hb,
+               int nblk) {
+    using SM = OutSmem;
+    char* sm = smem_base1024();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
+    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
+    float* cf = reinterpret_cast<float*>(sm + SM::kCf);
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    const uint32_t sC = smem_u32(sm + SM::kC), sB = smem_u32(sm + SM::kB);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+    int idx = blockIdx.x;
+    const int blk = idx % nblk;
+    idx /= nblk;
+    const int g = idx % a.G;
+    idx /= a.G;
+    const int b = idx % a.B;
+    const int c = idx / a.B;
+    const int t0 = c * kQ;
+    const int hfirst = g * a.HpG + blk * hb;
+    const int nh = min(hb, a.HpG - blk * hb);
+    const bool has_in = c > 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < 7; ++i) mbar_init(&bar[i], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2));
+        for (int j = 0; j < kKD / 64; ++j) {
+            tma_load_4d(sm + SM::kC + j * kQ * 128, &mC, &bar[0], 64 * j, g, t0, b);
+            tma_load_4d(sm + SM::kB + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
+        }
+        for (int i = 0; i < min(3, nh); ++i) {
+            mbar_arrive_expect_tx(&bar[2 + i], (uint32_t)(kQ * kP * 2));
+            tma_load_4d(sm + SM::kX + i * kQ * 128, &mX, &bar[2 + i], 0, hfirst + i, t0, b);
+        }
+    }
+    // S_in rows (row n = tid) of the next head, prefetched into registers
+    float4 sreg[16];
+    auto load_s = [&](int h) {
+        const float* src = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + tid) * kP;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sreg[e] = __ldcg(reinterpret_cast<const float4*>(src) + e);
+    };
+    if (has_in) load_s(hfirst);
+
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 710);
+    if (tid == 0 && ok) {
+        tc::fence_after_sync();
+        tc::mma_tiles(tmem, sC, 0, kQ, sB, 0, kQ, kQ, kQ, kKD, 0);  // M = C B^T
+        tc::commit(&bar[1]);
+    }
+    __syncwarp();
+
+    float Eprev = 0.0f, Dprev = 0.0f;
+    auto finish = [&](int i, float E, float Dh) {
+        const int j = i & 1, xb = i % 3;
+        ok = ok && mbar_wait(&bar[5 + j], (uint32_t)((i >> 1) & 1), a.hdr, 713);
+        ok = ok && mbar_wait(&bar[2 + xb], (uint32_t)((i / 3) & 1), a.hdr, 714);  // x rows read below
+        tc::fence_after_sync();
+        char* X = sm + SM::kX + xb * kQ * 128;
+#pragma unroll
+        for (int v0 = 0; v0 < kP; v0 += 16) {
+            float y1[16], y2[16];
+            tc::ld16(tmem + col_y(j) + lane_off + v0, y1);
+            if (has_in) tc::ld16(tmem + col_y2(j) + lane_off + v0, y2);
+            tc::wait_ld();
+#pragma unroll
+            for (int hh = 0; hh < 16; hh += 8) {
+                uint4* px = reinterpret_cast<uint4*>(X + tc::sw128_off(tid, v0 + hh, kQ));
+                uint4 raw = *px;
+                __nv_bfloat162* xv = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 xf = __bfloat1622float2(xv[e]);
+                    float o0 = y1[hh + 2 * e], o1 = y1[hh + 2 * e + 1];
+                    if (has_in) {
+                        o0 = fmaf(E, y2[hh + 2 * e], o0);
+                        o1 = fmaf(E, y2[hh + 2 * e + 1], o1);
+                    }
+                    xv[e] = __floats2bfloat162_rn(fmaf(Dh, xf.x, o0), fmaf(Dh, xf.y, o1));
+                }
+                *px = raw;
+            }
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&mY, X, 0, hfirst + i, t0, b);
+            bulk_commit();
+            bulk_wait_read_all();
+            if (i + 3 < nh) {
+                mbar_arrive_expect_tx(&bar[2 + xb], (uint32_t)(kQ * kP * 2));
+                tma_load_4d(X, &mX, &bar[2 + xb], 0, hfirst + i + 3, t0, b);
+            }
+        }
+    };
+
+    for (int i = 0; i < nh; ++i) {
+        const int h = hfirst + i, j = i & 1;
+        // ---- prep(i): decays, S_in tile, P
+        float lam, beta;
+        ssd_coef(a, b, h, t0 + tid, lam, beta);
+        const float lt = cta_inclusive_sum(lam, tmp);
+        const float lt2 = lt * kLog2e;
+        l2s[tid] = lt2;
+        betas[tid] = beta;
+        __syncthreads();
+        const float Ecur = ex2(lt2);
+        const float Dcur = a.Dskip ? a.Dskip[h] : 0.0f;
+        float* cfw = cf + warp * kQ;
+        const float l0 = l2s[32 * warp];
+        for (int s = lane; s < 32 * warp; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
+        __syncwarp();
+        if (has_in) {
+            char* St = sm + SM::kSt + j * kKD * kP * 2;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+                __align__(16) __nv_bfloat162 pk[4] = {
+                    __floats2bfloat162_rn(sreg[e].x, sreg[e].y), __floats2bfloat162_rn(sreg[e].z, sreg[e].w),
+                    __floats2bfloat162_rn(sreg[e + 1].x, sreg[e + 1].y),
+                    __floats2bfloat162_rn(sreg[e + 1].z, sreg[e + 1].w)};
+                *reinterpret_cast<uint4*>(St + tc::sw128_off(tid, 4 * e, kKD)) = *reinterpret_cast<uint4*>(pk);
+            }
+        }
+        if (i == 0) ok = ok && mbar_wait(&bar[1], 0, a.hdr, 711);
+        tc::fence_after_sync();
+        {
+            const float rf = ex2(lt2 - l0);
+            const uint32_t pcol = tmem + col_p(j) + lane_off;
+#pragma unroll 1
+            for (int sb = 0; sb < 4; ++sb) {
+                uint32_t pk[16];
+                if (sb > warp) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                    tc::st16(pcol + 16 * sb, pk);
+                    continue;
+                }
+                float v[32];
+                tc::ld16(tmem + lane_off + 32 * sb, v);
+                tc::ld16(tmem + lane_off + 32 * sb + 16, v + 16);
+                tc::wait_ld();
+                if (sb < warp) {
+                    const float* cfb = cfw + 32 * sb;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * q] * (rf * cfb[2 * q]),
+                                                                  v[2 * q + 1] * (rf * cfb[2 * q + 1]));
+                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int s = 32 * sb + 2 * q;
+                        const float p0 = s <= tid ? v[2 * q] * (ex2(lt2 - l2s[s]) * betas[s]) : 0.0f;
+                        const float p1 = s + 1 <= tid ? v[2 * q + 1] * (ex2(lt2 - l2s[s + 1]) * betas[s + 1]) : 0.0f;
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                }
+                tc::st16(pcol + 16 * sb, pk);
+            }
+            tc::wait_st();
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- issue(i)
+        if (tid == 0 && ok) {
+            ok = mbar_wait(&bar[2 + i % 3], (uint32_t)((i / 3) & 1), a.hdr, 712);
+            tc::fence_after_sync();
+            tc::mma_ts_tiles(tmem + col_y(j), tmem + col_p(j), smem_u32(sm + SM::kX + (i % 3) * kQ * 128), 1, kQ, kP,
+                             kQ, 0);
+            if (has_in)
+                tc::mma_tiles(tmem + col_y2(j), sC, 0, kQ, smem_u32(sm + SM::kSt + j * kKD * kP * 2), 1, kKD, kQ, kP,
+                              kKD, 0);
+            tc::commit(&bar[5 + j]);
+        }
+        __syncwarp();
+        if (has_in && i + 1 < nh) load_s(h + 1);
+        if (i > 0) finish(i - 1, Eprev, Dprev);
+        Eprev = Ecur;
+        Dprev = Dcur;
+    }
+    if (nh > 0) finish(nh - 1, Eprev, Dprev);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+struct SsdFwdWs {
+    size_t decay, end;
+};
+SsdFwdWs fwd_plan(const lr_desc& d) {
+    const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
+    WsCursor cur;
+    SsdFwdWs w;
+    w.decay = cur.take(sizeof(float) * d.B * d.H * nchunk);
+    w.end = cur.off;
+    return w;
+}
+
+SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char* ws, float* decay) {
+    SsdArgs a{};
+    a.B = (int)d.B;
+    a.L = (int)d.L;
+    a.H = (int)d.H;
+    a.G = (int)d.G;
+    a.HpG = (int)(d.H / d.G);
+    a.nchunk = (int)((d.L + kQ - 1) / kQ);
+    a.dt = (const __nv_bfloat16*)in.delta;
+    a.A = in.A;
+    a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
+    a.ckpt = (const float*)ckpt;
+    a.decay = decay;
+    a.hdr = (WsHeader*)ws;
+    return a;
+}
+
+// Heads per output CTA: the group's heads split into the fewest blocks that give at least one
+// CTA per SM, blocks of at most 16 heads (always 16 under LR_TEST_MAX_HEAD_BLOCK).
+int out_heads_per_cta(const lr_desc& d, int nchunk) {
+    const int HpG = (int)(d.H / d.G);
+    const long units = (long)nchunk * d.B * d.G;
+    int hb = HpG < 16 ? HpG : 16;
+    if (d.flags & LR_TEST_MAX_HEAD_BLOCK) return hb;
+    while (hb > 1 && units * ((HpG + hb - 1) / hb) < 148) hb = (hb + 1) / 2;
+    return hb;
+}
+
+// =========================================================================================
+// Backward.  With G_c the adjoint of the state leaving chunk c (G_{last} = 0):
+//   U_c = C^T diag(E) dy_h                   (ssd_state_kernel, dir < 0)
+//   G_{c-1} = e^{l_Q, c} G_c + U_c            (ssd_pass_kernel, dir < 0)
+// and per (chunk, head), with S2 = dy x^T, Pd = S2 o Lmask, P = M o Lmask, R = Pd o M:
+//   dC += Pd B + diag(E) dy S_in^T            dB += Pd^T C + diag(w) x G^T   (summed over heads)
+//   dx  = P^T dy + diag(w) B G + D dy
+//   dl_t = rowsum_t(R) + E_t dy_t . (C S_in)_t - colsum_t(R) - w_t x_t . (B G)_t  (+ X at t = Q-1)
+//   X = <G, S_out> = e^{l_Q} <G, S_in> + sum_s w_s x_s . (B G)_s
+//   d lam_r = sum_{t >= r} dl_t;  d beta_s = (colsum_s(R) + w_s x_s . (B G)_s) / beta_s
+//   d dt = d lam A + d beta e^{dt A};  dA_h += d lam dt + d beta (dt e^{dt A} - beta) / A;  dD_h += dy . x
+// (rowsum_t(R) = C_t . dC_t and colsum_s(R) = B_s . dB_s restricted to the chunk's own terms;
+// here they come straight from the fp32 accumulators of M and S2.)
+// =========================================================================================
+struct SsdGradArgs {
+    SsdArgs a;
+    const float* G;        // [nchunk][B][H][N][P] adjoint of each chunk's outgoing state
+    __nv_bfloat16* ddt;    // [B, L, H]
+    float* dB;             // [B, L, G, N]
+    float* dC;
+    float* pdA;            // [B][H][nchunk] per-chunk partials of dA_h, dD_h
+    float* pdD;
+    int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
+};
+
+struct GradSmem {
+    static constexpr size_t kQt = 0;                       // C tile 128 x 128 bf16
+    static constexpr size_t kKt = kQt + kQ * kKD * 2;      // B tile
+    static constexpr size_t kReg = kKt + kQ * kKD * 2;     // two 32 KB regions: {x, dy} of a head or Pd
+    static constexpr size_t kPt = kReg + 2 * kQ * kQ * 2;  // P, then the dx staging tile
+    static constexpr size_t kSt = kPt + kQ * kQ * 2;       // S_in bf16 [n][p]
+    static constexpr size_t kGt = kSt + kKD * kP * 2;      // G bf16 [n][p]
+    static constexpr size_t kL2 = kGt + kKD * kP * 2;      // l log2e [128]
+    static constexpr size_t kBeta = kL2 + kQ * 4;          // beta [128]
+    static constexpr size_t kCf = kBeta + kQ * 4;          // column factors [4][128]
+    static constexpr size_t kRowp = kCf + 4 * kQ * 4;      // row sums of R [2][128]
+    static constexpr size_t kColp = kRowp + 2 * kQ * 4;    // column sums of R [4][128]
+    static constexpr size_t kQdq = kColp + 4 * kQ * 4;     // E dy . Y2 [2][128]
+    static constexpr size_t kKdk = kQdq + 2 * kQ * 4;      // w x . BG [2][128]
+    static constexpr size_t kDd = kKdk + 2 * kQ * 4;       // dy . x [2][128]
+    static constexpr size_t kGs = kDd + 2 * kQ * 4;        // <G, S_in> partials [256]
+    static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
+    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A, 4 batch 1, 5 batch 2
+    static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;
+    static_assert(kAlloc <= 232448, "gradient CTA exceeds the shared memory of one CTA");
+};
+// TMEM columns: dC (0), dB (128); phase A: M (256), S2 (384); phase B: dV1 (256), BG (320), Y2 (384).
+constexpr uint32_t kGdC = 0, kGdB = 128, kGM = 256, kGS2 = 384, kGdV = 256, kGBG = 320, kGY2 = 384;
+
+__device__ __forceinline__ void wg0_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum).
+__device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    wg0_bar();
+    float add = 0.0f;
+    for (int w = 0; w < warp; ++w) add += tmp[w];
+    wg0_bar();
+    return x + add;
+}
+// Sum over the 128 threads of warpgroup 0, fixed order, result in every thread.
+__device__ __forceinline__ float wg0_sum(float x, float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) tmp[8 + warp] = x;
+    wg0_bar();
+    const float s = (tmp[8] + tmp[9]) + (tmp[10] + tmp[11]);
+    wg0_bar();
+    return s;
+}
+
+// Pack 8 floats into 8 bf16 (one 16-byte chunk).
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    uint4 r;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+    return r;
+}
+
+// One CTA per (chunk, batch row, group, block of hb heads), 256 threads: warpgroup wg handles
+// columns [64 wg, 64 wg + 64) (or [32 wg, ...) of 64-wide tensors) of TMEM lane / row 32 wq + lane.
+// Per head: phase A (M = C B^T, S2 = dy x^T) -> E1 (P, Pd, row / column sums of R) -> batch 1
+// (Pd B, Pd^T C into dC, dB; P^T dy, B G, C S_in) -> E2 (dx, inter-chunk row dots, scaling of dy
+// by E and x by w) -> batch 2 (diag(E) dy S_in^T, diag(w) x G^T into dC, dB) while warpgroup 0
+// turns the row terms into d dt.  The {x, dy} region of head i + 1 is loaded into the region that
+// held Pd of head i, so loads overlap the tail of each head.
+__global__ void __launch_bounds__(256, 1)
+ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
+                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
+                const __grid_constant__ CUtensorMap mdX, SsdGradArgs ga, int hb, int nblk) {
+    using SM = GradSmem;
+    const SsdArgs& a = ga.a;
+    char* sm = smem_base1024();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
+    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
+    float* cf = reinterpret_cast<float*>(sm + SM::kCf);
+    float* rowp = reinterpret_cast<float*>(sm + SM::kRowp);
+    float* colp = reinterpret_cast<float*>(sm + SM::kColp);
+    float* qdqp = reinterpret_cast<float*>(sm + SM::kQdq);
+    float* kdkp = reinterpret_cast<float*>(sm + SM::kKdk);
+    float* ddp = reinterpret_cast<float*>(sm + SM::kDd);
+    float* gsp = reinterpret_cast<float*>(sm + SM::kGs);
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sP = smem_u32(sm + SM::kPt),
+                   sS = smem_u32(sm + SM::kSt), sG = smem_u32(sm + SM::kGt);
+    const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
+    const int row = tid & 127;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+
+    int idx = blockIdx.x;
+    const int blk = idx % nblk;
+    idx /= nblk;
+    const int g = idx % a.G;
+    idx /= a.G;
+    const int b = idx % a.B;
+    const int c = idx / a.B;
+    const int t0 = c * kQ;
+    const int hfirst = g * a.HpG + blk * hb;
+    const int nh = min(hb, a.HpG - blk * hb);
+    const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
+
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (tid < 32) tc::tmem_alloc(tmem_slot, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto region = [&](int r) { return sm + SM::kReg + (size_t)r * kQ * kQ * 2; };
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2));
+        for (int j = 0; j < kKD / 64; ++j) {
+            tma_load_4d(sm + SM::kQt + j * kQ * 128, &mC, &bar[0], 64 * j, g, t0, b);
+            tma_load_4d(sm + SM::kKt + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
+        }
+        mbar_arrive_expect_tx(&bar[1], (uint32_t)(2 * kQ * kP * 2));
+        tma_load_4d(region(0), &mX, &bar[1], 0, hfirst, t0, b);
+        tma_load_4d(region(0) + kQ * kP * 2, &mdY, &bar[1], 0, hfirst, t0, b);
+    }
+    // S_in and G rows (row n = row, columns [32 wg, 32 wg + 32)) of the next head, in registers
+    float4 sin_r[8], g_r[8];
+    auto load_sg = [&](int h) {
+        const size_t off = ((((size_t)c * a.B + b) * a.H + h) * kKD + row) * kP + 32 * wg;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sin_r[e] = has_in ? __ldcg(reinterpret_cast<const float4*>(a.ckpt + off) + e) : make_float4(0, 0, 0, 0);
+            g_r[e] = has_out ? __ldcg(reinterpret_cast<const float4*>(ga.G + off) + e) : make_float4(0, 0, 0, 0);
+        }
+    };
+    load_sg(hfirst);
+    auto load_dt = [&](int h) {
+        return (wg == 0 && t0 + row < a.L) ? a.dt[((size_t)b * a.L + t0 + row) * a.H + h] : __float2bfloat16_rn(0.0f);
+    };
+    __nv_bfloat16 dt_next = load_dt(hfirst);
+    bool ok = true;
+
+    for (int i = 0; i < nh; ++i) {
+        const int h = hfirst + i, r = i & 1, pr = r ^ 1;
+        char* Xt = region(r);
+        char* Ot = region(r) + kQ * kP * 2;
+        char* Pdt = region(pr);
+        const uint32_t sX = smem_u32(Xt), sO = smem_u32(Ot), sPd = smem_u32(Pdt);
+        // ------------------------------------------------------------ prep(i)
+        if (i > 0) {
+            ok = ok && mbar_wait(&bar[5], (uint32_t)((i - 1) & 1), a.hdr, 720);
+            tc::fence_after_sync();
+        }
+        const float dt_raw = __bfloat162float(dt_next);
+        float lam = 0.0f, beta = 0.0f;
+        if (wg == 0 && t0 + row < a.L) {
+            const float Ah = a.A[h];
+            lam = dt_raw * Ah;
+            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+        }
+        if (wg == 0) {
+            const float lt = wg0_inclusive_sum(lam, tmp);
+            l2s[row] = lt * kLog2e;
+            betas[row] = beta;
+        }
+        if (i + 1 < nh) dt_next = load_dt(h + 1);
+        // S_in / G rows -> bf16 tiles, <G, S_in> partial
+        {
+            float gs = 0.0f;
+            char* St = sm + SM::kSt;
+            char* Gt = sm + SM::kGt;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float fs[8] = {sin_r[e].x, sin_r[e].y, sin_r[e].z, sin_r[e].w,
+                                     sin_r[e + 1].x, sin_r[e + 1].y, sin_r[e + 1].z, sin_r[e + 1].w};
+                const float fg[8] = {g_r[e].x, g_r[e].y, g_r[e].z, g_r[e].w, g_r[e + 1].x, g_r[e + 1].y, g_r[e + 1].z,
+                                     g_r[e + 1].w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) gs = fmaf(fs[q], fg[q], gs);
+                const int col = 32 * wg + 4 * e;
+                if (has_in) *reinterpret_cast<uint4*>(St + tc::sw128_off(row, col, kKD)) = pack8(fs);
+                if (has_out) *reinterpret_cast<uint4*>(Gt + tc::sw128_off(row, col, kKD)) = pack8(fg);
+            }
+            gsp[tid] = gs;
+        }
+        if (i + 1 < nh) load_sg(h + 1);
+        if (tid == 0) {
+            if (i == 0) ok = ok && mbar_wait(&bar[0], 0, a.hdr, 721);
+            bulk_wait_read_all();  // the previous head's dx store has left the P tile
+        }
+        ok = ok && mbar_wait(&bar[1 + r], (uint32_t)((i >> 1) & 1), a.hdr, 722);  // x, dy (read by E2 too)
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0 && ok) {  // phase A
+            tc::fence_after_sync();
+            tc::mma_tiles(tmem + kGM, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);   // M  = C B^T
+            tc::mma_tiles(tmem + kGS2, sO, 0, kQ, sX, 0, kQ, kQ, kQ, kP, 0);   // S2 = dy x^T
+            tc::commit(&bar[3]);
+        }
+        // column factors cf[w][s] = e^{l_{32 w} - l_s} beta_s (s < 32 w), two per thread
+#pragma unroll
+        for (int k = tid; k < 4 * kQ; k += 256) {
+            const int w = k >> 7, s = k & 127;
+            if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]) * betas[s];
+        }
+        // warpgroup 0 keeps its row's <G, S_in> partials: warpgroup 1 rewrites them for the next
+        // head while warpgroup 0 is still turning this head's row terms into d dt
+        const float gs_row = wg == 0 ? gsp[row] + gsp[row + kQ] : 0.0f;
+        __syncthreads();
+        // ------------------------------------------------------------ E1(i)
+        ok = ok && mbar_wait(&bar[3], (uint32_t)(i & 1), a.hdr, 723);
+        tc::fence_after_sync();
+        {
+            const float l2r = l2s[row];
+            const float rf = ex2(l2r - l2s[32 * wq]);
+            float rsum = 0.0f;
+#pragma unroll 1
+            for (int sb = wg; sb < 4; sb += 2) {
+                const int s0 = 32 * sb;
+                if (sb > wq) {  // above the diagonal: zero rows of P and Pd
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < 32; k += 8) {
+                        *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, s0 + k, kQ)) = z;
+                        *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = z;
+                    }
+                    colp[wq * kQ + s0 + lane] = 0.0f;
+                    continue;
+                }
+                float m[32], s2[32];
+                tc::ld16(tmem + kGM + lane_off + s0, m);
+                tc::ld16(tmem + kGM + lane_off + s0 + 16, m + 16);
+                tc::ld16(tmem + kGS2 + lane_off + s0, s2);
+                tc::ld16(tmem + kGS2 + lane_off + s0 + 16, s2 + 16);
+                tc::wait_ld();
+                float rr[32];
+                if (sb < wq) {
+                    const float* cfb = cf + wq * kQ + s0;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const float f = rf * cfb[k];
+                        const float mk = m[k];
+                        m[k] = mk * f;            // P
+                        s2[k] *= f;               // Pd
+                        rr[k] = s2[k] * mk;       // R = Pd o M
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int s = s0 + k;
+                        const float f = s <= row ? ex2(l2r - l2s[s]) * betas[s] : 0.0f;
+                        const float mk = m[k];
+                        m[k] = mk * f;
+                        s2[k] *= f;
+                        rr[k] = s2[k] * mk;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 32; k += 8) {
+                    *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, s0 + k, kQ)) = pack8(m + k);
+                    *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = pack8(s2 + k);
+                }
+#pragma unroll
+                for (int k = 0; k < 32; ++k) rsum += rr[k];
+                // column sums over this warp's 32 rows: lane l ends with column s0 + l
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const bool up = (lane & off) != 0;
+#pragma unroll
+                    for (int k = 0; k < off; ++k) {
+                        const float send = up ? rr[k] : rr[k + off];
+                        const float keep = up ? rr[k + off] : rr[k];
+                        rr[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    }
+                }
+                colp[wq * kQ + s0 + lane] = rr[0];
+            }
+            rowp[wg * kQ + row] = rsum;
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0 && ok) {  // batch 1
+            tc::fence_after_sync();
+            const uint32_t acc = i > 0 ? 1u : 0u;
+            tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
+            tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
+            tc::mma_tiles(tmem + kGdV, sP, 1, kQ, sO, 1, kQ, kQ, kP, kQ, 0);      // dV1 = P^T dy
+            if (has_out) tc::mma_tiles(tmem + kGBG, sK, 0, kQ, sG, 1, kKD, kQ, kP, kKD, 0);  // B G
+            if (has_in) tc::mma_tiles(tmem + kGY2, sQ, 0, kQ, sS, 1, kKD, kQ, kP, kKD, 0);   // C S_in
+            tc::commit(&bar[4]);
+        }
+        ok = ok && mbar_wait(&bar[4], (uint32_t)(i & 1), a.hdr, 724);
+        tc::fence_after_sync();
+        if (tid == 0 && ok && i + 1 < nh) {  // Pd is consumed: its region takes {x, dy} of head i + 1
+            mbar_arrive_expect_tx(&bar[1 + pr], (uint32_t)(2 * kQ * kP * 2));
+            tma_load_4d(region(pr), &mX, &bar[1 + pr], 0, h + 1, t0, b);
+            tma_load_4d(region(pr) + kQ * kP * 2, &mdY, &bar[1 + pr], 0, h + 1, t0, b);
+        }
+        // ------------------------------------------------------------ E2(i)
+        {
+            const float l2r = l2s[row];
+            const float E = ex2(l2r);
+            const float w = ex2(l2s[kQ - 1] - l2r) * betas[row];
+            const float Dh = a.Dskip ? a.Dskip[h] : 0.0f;
+            float qdq = 0.0f, kdk = 0.0f, dd = 0.0f;
+#pragma unroll
+            for (int v0 = 0; v0 < 32; v0 += 16) {
+                const int col = 32 * wg + v0;
+                float dv[16], bg[16], y2[16];
+                tc::ld16(tmem + kGdV + lane_off + col, dv);
+                if (has_out) tc::ld16(tmem + kGBG + lane_off + col, bg);
+                if (has_in) tc::ld16(tmem + kGY2 + lane_off + col, y2);
+                tc::wait_ld();
+#pragma unroll
+                for (int hh = 0; hh < 16; hh += 8) {
+                    uint4* px = reinterpret_cast<uint4*>(Xt + tc::sw128_off(row, col + hh, kQ));
+                    uint4* po = reinterpret_cast<uint4*>(Ot + tc::sw128_off(row, col + hh, kQ));
+                    uint4 xr = *px, orr = *po;
+                    const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&xr);
+                    const __nv_bfloat162* ov = reinterpret_cast<const __nv_bfloat162*>(&orr);
+                    float xs[8], os[8], dx[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 xf = __bfloat1622float2(xv[e]), of = __bfloat1622float2(ov[e]);
+                        xs[2 * e] = xf.x;
+                        xs[2 * e + 1] = xf.y;
+                        os[2 * e] = of.x;
+                        os[2 * e + 1] = of.y;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int k = hh + e;
+                        float dvk = dv[k];
+                        if (has_out) {
+                            dvk = fmaf(w, bg[k], dvk);
+                            kdk = fmaf(xs[e], bg[k], kdk);
+                        }
+                        if (has_in) qdq = fmaf(os[e], y2[k], qdq);
+                        dd = fmaf(os[e], xs[e], dd);
+                        dx[e] = fmaf(Dh, os[e], dvk);
+                        xs[e] *= w;
+                        os[e] *= E;
+                    }
+                    *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, col + hh, kQ)) = pack8(dx);
+                    *px = pack8(xs);
+                    *po = pack8(os);
+                }
+            }
+            qdqp[wg * kQ + row] = E * qdq;
+            kdkp[wg * kQ + row] = w * kdk;
+            ddp[wg * kQ + row] = dd;
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0 && ok) {  // batch 2, then the dx store
+            tc::fence_after_sync();
+            if (has_in) tc::mma_tiles(tmem + kGdC, sO, 0, kQ, sS, 0, kKD, kQ, kKD, kP, 1);   // dC += (E dy) S_in^T
+            if (has_out) tc::mma_tiles(tmem + kGdB, sX, 0, kQ, sG, 0, kKD, kQ, kKD, kP, 1);  // dB += (w x) G^T
+            tc::commit(&bar[5]);
+            tma_store_4d(&mdX, sm + SM::kPt, 0, h, t0, b);
+            bulk_commit();
+        }
+        // ------------------------------------------------------------ d dt, dA, dD (warpgroup 0)
+        if (wg == 0) {
+            const int t = row;
+            const bool valid = t0 + t < a.L;
+            const float cs = (colp[t] + colp[kQ + t]) + (colp[2 * kQ + t] + colp[3 * kQ + t]);
+            const float rs = rowp[t] + rowp[kQ + t];
+            const float qi = qdqp[t] + qdqp[kQ + t];
+            const float ki = kdkp[t] + kdkp[kQ + t];
+            const float ddv = ddp[t] + ddp[kQ + t];
+            const float kisum = wg0_sum(ki, tmp);
+            const float gs = wg0_sum(gs_row, tmp);
+            const float X = ex2(l2s[kQ - 1]) * gs + kisum;
+            float dl = rs + qi - cs - ki + (t == kQ - 1 ? X : 0.0f);
+            if (!valid) dl = 0.0f;
+            const float incl = wg0_inclusive_sum(dl, tmp);
+            if (t == kQ - 1) tmp[16] = incl;
+            wg0_bar();
+            const float dlam = tmp[16] - incl + dl;
+            float dA_part = 0.0f;
+            if (valid) {
+                const float Ah = a.A[h];
+                const float bt = betas[t];
+                const float ab = ex2(dt_raw * Ah * kLog2e);
+                const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
+                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(dlam * Ah + dbeta * ab);
+                dA_part = dlam * dt_raw + dbeta * (dt_raw * ab - bt) / Ah;
+            }
+            const float sA = wg0_sum(dA_part, tmp);
+            const float sD = wg0_sum(valid ? ddv : 0.0f, tmp);
+            if (t == 0) {
+                const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
+                ga.pdA[tile] = sA;
+                ga.pdD[tile] = sD;
+            }
+        }
+    }
+    // dC, dB of this (batch row, chunk, group): rows t, columns [64 wg, 64 wg + 64).  Every lane
+    // takes part in the (warp-collective) TMEM loads; rows past L are not stored.
+    ok = ok && mbar_wait(&bar[5], (uint32_t)((nh - 1) & 1), a.hdr, 725);
+    tc::fence_after_sync();
+    {
+        const bool vrow = t0 + row < a.L;
+        const size_t base = (((size_t)b * a.L + (vrow ? t0 + row : 0)) * a.G + g) * kKD + 64 * wg;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            float* dst = (which == 0 ? ga.dC : ga.dB) + base;
+            const uint32_t col = (which == 0 ? kGdC : kGdB) + 64 * wg;
+#pragma unroll
+            for (int v0 = 0; v0 < 64; v0 += 16) {
+                float v[16];
+                tc::ld16(tmem + col + lane_off + v0, v);
+                tc::wait_ld();
+                if (vrow) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4) {
+                        if (ga.accumulate)
+                            red_add4(dst + v0 + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+                        else
+                            *reinterpret_cast<float4*>(dst + v0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    }
+                }
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid < 32) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// dA_h, dD_h: fixed-order sums of the per-chunk partials over batch rows and chunks (one warp per
+// head; lane-strided partial sums, then a fixed butterfly).
+__global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __restrict__ pdD, int B, int H, int nchunk,
+                              float* __restrict__ dA, float* __restrict__ dD) {
+    const int h = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= H) return;
+    float sa = 0.0f, sd = 0.0f;
+    for (int bb = 0; bb < B; ++bb)
+        for (int c = lane; c < nchunk; c += 32) {
+            const size_t t = ((size_t)bb * H + h) * nchunk + c;
+            sa += pdA[t];
+            sd += pdD[t];
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, o);
+        sd += __shfl_xor_sync(0xffffffffu, sd, o);
+    }
+    if (lane == 0) {
+        dA[h] = sa;
+        if (dD) dD[h] = sd;
+    }
+}
+
+struct SsdBwdWs {
+    size_t decay, pdA, pdD, G, end;
+};
+SsdBwdWs bwd_plan(const lr_desc& d) {
+    const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
+    const size_t tiles = (size_t)d.B * d.H * nchunk;
+    WsCursor cur;
+    SsdBwdWs w;
+    w.decay = cur.take(sizeof(float) * tiles);
+    w.pdA = cur.take(sizeof(float) * tiles);
+    w.pdD = cur.take(sizeof(float) * tiles);
+    w.G = cur.take(sizeof(float) * tiles * kKD * kP);
+    w.end = cur.off;
+    return w;
+}
+
+// Heads per gradient CTA: the group's heads split into the fewest blocks (at most 16 heads each)
+// that occupy about three quarters of the SMs or more (always 16 under LR_TEST_MAX_HEAD_BLOCK).
+int grad_heads_per_cta(const lr_desc& d, int nchunk) {
+    const int HpG = (int)(d.H / d.G);
+    const long units = (long)nchunk * d.B * d.G;
+    int hb = HpG < 16 ? HpG : 16;
+    if (d.flags & LR_TEST_MAX_HEAD_BLOCK) return hb;
+    while (hb > 1 && units * ((HpG + hb - 1) / hb) < 110) hb = (hb + 1) / 2;
+    return hb;
+}
+
+}  // namespace
+
+size_t ssd_fwd_ws_bytes(const lr_desc& d) { return fwd_plan(d).end; }
+size_t ssd_fwd_flag_bytes(const lr_desc&) { return 256; }
+
+lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
+    const SsdFwdWs w = fwd_plan(d);
+    SsdArgs a = make_args(d, in, ckpt, ws, (float*)(ws + w.decay));
+    CUtensorMap mC, mB, mX, mY;
+    bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
+              map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    const int nblk_s = (a.HpG + kHS - 1) / kHS;
+    if (a.nchunk > 1) {
+        cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
+        note_launch("ssd_chunk_state");
+        const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
+        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mB, mX, a, (float*)ckpt, nblk_s, +1);
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
+    {
+        const int n4 = kKD * kP / 4;
+        const size_t total = (size_t)a.B * a.H * n4;
+        note_launch("ssd_state_pass");
+        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)ckpt, a.decay, a.B * a.H, n4,
+                                                                         a.nchunk, +1);
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
+    const int hb = out_heads_per_cta(d, a.nchunk);
+    const int nblk_o = (a.HpG + hb - 1) / hb;
+    cudaFuncSetAttribute(ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
+    note_launch("ssd_chunk_out");
+    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, kThreads, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, hb, nblk_o);
+    return check_launch();
+}
+
+size_t ssd_bwd_ws_bytes(const lr_desc& d) { return bwd_plan(d).end; }
+size_t ssd_bwd_flag_bytes(const lr_desc&) { return 256; }
+
+lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt, const lr_grads& gr,
+                  char* ws, cudaStream_t st) {
+    const SsdBwdWs w = bwd_plan(d);
+    SsdGradArgs ga{};
+    ga.a = make_args(d, in, ckpt, ws, (float*)(ws + w.decay));
+    const SsdArgs& a = ga.a;
+    ga.G = (const float*)(ws + w.G);
+    ga.ddt = (__nv_bfloat16*)gr.ddelta;
+    ga.dB = gr.dBm;
+    ga.dC = gr.dCm;
+    ga.pdA = (float*)(ws + w.pdA);
+    ga.pdD = (float*)(ws + w.pdD);
+    CUtensorMap mC, mB, mX, mdY, mdX;
+    bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
+              map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true) &&
+              map4(&mdX, gr.dx, kP, d.H, d.L, d.B, true);
+    if (!ok) return LR_ERR_INVALID_ARG;
+    float* Gbuf = (float*)(ws + w.G);
+    const int nblk_s = (a.HpG + kHS - 1) / kHS;
+    if (a.nchunk > 1) {
+        cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
+        note_launch("ssd_chunk_state");
+        const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
+        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, a, Gbuf, nblk_s, -1);
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
+    {
+        const int n4 = kKD * kP / 4;
+        const size_t total = (size_t)a.B * a.H * n4;
+        note_launch("ssd_state_pass");
+        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)Gbuf, a.decay, a.B * a.H, n4,
+                                                                         a.nchunk, -1);
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
+    const int hb = grad_heads_per_cta(d, a.nchunk);
+    const int nblk = (a.HpG + hb - 1) / hb;
+    ga.accumulate = nblk > 1 ? 1 : 0;
+    if (ga.accumulate) {
+        const size_t n = (size_t)d.B * d.L * d.G * kKD * sizeof(float);
+        if (cudaMemsetAsync(gr.dBm, 0, n, st) != cudaSuccess || cudaMemsetAsync(gr.dCm, 0, n, st) != cudaSuccess)
+            return LR_ERR_CUDA;
+    }
+    cudaFuncSetAttribute(ssd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
+    note_launch("ssd_chunk_grad");
+    ssd_grad_kernel<<<a.nchunk * a.B * a.G * nblk, 256, GradSmem::kAlloc, st>>>(mC, mB, mX, mdY, mdX, ga, hb, nblk);
+    lr_status s = check_launch();
+    if (s != LR_OK) return s;
+    note_launch("ssd_param_reduce");
+    ssd_param_sum<<<(a.H + 7) / 8, 256, 0, st>>>(ga.pdA, ga.pdD, a.B, a.H, a.nchunk, gr.dA,
+                                                 (d.flags & LR_HAS_DSKIP) ? gr.dDskip : nullptr);
+    return check_launch();
+}
+
+}  // namespace lrs

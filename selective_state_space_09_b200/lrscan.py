@@ -23,6 +23,8 @@ KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
 DISC = {"none": 0, "zoh": 1, "bilinear": 2}
 IO = {torch.float32: 0, torch.bfloat16: 1}
 HAS_Z, HAS_DSKIP = 1, 2
+# test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
+TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
 STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
           "workspace too small", "CUDA runtime error", "device wait timed out",
           "device consistency check failed"]

@@ -245,7 +245,7 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         t = torch.tensor([step_ms, fwd_mean, bwd_mean], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         step_ms, fwd_mean, bwd_mean = (float(v) for v in t.tolist())
-    fwd_b, bwd_b = algorithmic_bytes(kind, inp, y, grads, lrscan.ckpt_bytes(plan.desc))
+    fwd_b, bwd_b = algorithmic_bytes(kind, inp, y, grads, plan.ckpt_view().numel() * 4)  # f32 states
     res = {
         "workload": name, "kind": kind, "desc": NAMES[name],
         "tokens_per_step": tokens_of(w) * world,

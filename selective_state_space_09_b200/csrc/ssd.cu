@@ -163,20 +163,34 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------- state passing
-// In place over the slots of `buf` ([nchunk][B*H][n4] float4), one thread per (b h, float4):
-//   dir > 0: slot 0 = 0; slot c = decay_{c-1} slot_{c-1} + slot_c, c = 1 .. nchunk-1
-//   dir < 0: slot nchunk-1 = 0; slot c = decay_{c+1} slot_{c+1} + slot_c, c = nchunk-2 .. 0
+constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf16 SW128 tile
+
+// One thread per (b h, four consecutive state elements (n, p .. p+3)) of the f32 slots of `buf`
+// ([nchunk][B*H][N*P/4] float4), walking the chunks in order:
+//   dir > 0: slot 0 = 0; slot c = decay_{c-1} slot_{c-1} + slot_c (c = 1 .. nchunk-1), in place;
+//            every slot is also written as bf16 into `tiles` ([nchunk][B*H] tiles, tensor-core
+//            order), the B operand of C S_in in the output and gradient kernels;
+//   dir < 0: G_{nchunk-1} = 0; G_c = decay_{c+1} G_{c+1} + slot_c (slot c holds U_{c+1}), written
+//            only as bf16 tiles.
 // Loads of eight slots are issued ahead of their dependent updates.
 __global__ void __launch_bounds__(256)
-ssd_pass_kernel(float4* buf, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir) {
+ssd_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir) {
     const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= (size_t)BH * n4) return;
     const size_t stride = (size_t)BH * n4;
-    const float* dec = decay + (e / n4) * nchunk;
+    const int bh = (int)(e / n4), q = (int)(e % n4);
+    const float* dec = decay + (size_t)bh * nchunk;
+    const uint32_t toff = tc::sw128_off(q / (kP / 4), (q % (kP / 4)) * 4, kKD);
+    auto put = [&](int c, float4 v) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        *reinterpret_cast<uint2*>(tiles + ((size_t)c * BH + bh) * kTileBytes + toff) = u;
+    };
     float4* p = buf + e;
     float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     const int first = dir > 0 ? 0 : nchunk - 1;
-    p[(size_t)first * stride] = s;
+    if (dir > 0) p[(size_t)first * stride] = s;
+    put(first, s);
     for (int k0 = 1; k0 < nchunk; k0 += 8) {
         float4 v[8];
 #pragma unroll
@@ -190,26 +204,30 @@ ssd_pass_kernel(float4* buf, const float* __restrict__ decay, int BH, int n4, in
                 const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
                 const float d = dec[c - dir];
                 s = make_float4(fmaf(d, s.x, v[k].x), fmaf(d, s.y, v[k].y), fmaf(d, s.z, v[k].z), fmaf(d, s.w, v[k].w));
-                p[(size_t)c * stride] = s;
+                if (dir > 0) p[(size_t)c * stride] = s;
+                put(c, s);
             }
         }
     }
 }
 
 // ---------------------------------------------------------------------------------- outputs
+constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernels)
+
 // Shared memory of the output CTA: C and B of the chunk, a ring of three x tiles (each becomes
-// the y staging tile of its head), two bf16 S_in tiles, the current head's decays.
+// the y staging tile of its head), two bf16 S_in tiles, per-head dt, the current head's decays.
 struct OutSmem {
     static constexpr size_t kC = 0;                          // 128 x 128 bf16
     static constexpr size_t kB = kC + kQ * kKD * 2;          // 128 x 128 bf16
     static constexpr size_t kX = kB + kQ * kKD * 2;          // 3 x (128 x 64) bf16
     static constexpr size_t kSt = kX + 3 * kQ * kP * 2;      // 2 x (128 x 64) bf16, [n][p]
-    static constexpr size_t kL2 = kSt + 2 * kKD * kP * 2;    // l log2e [128]
+    static constexpr size_t kDt = kSt + 2 * kTileBytes;      // dt of every head [kMaxHB][128] f32
+    static constexpr size_t kL2 = kDt + kMaxHB * kQ * 4;     // l log2e [128]
     static constexpr size_t kBeta = kL2 + kQ * 4;            // beta [128]
     static constexpr size_t kCf = kBeta + kQ * 4;            // column factors [4 warps][128]
     static constexpr size_t kTmp = kCf + 4 * kQ * 4;         // scan scratch
-    static constexpr size_t kBar = kTmp + 64;                // 0 C/B, 1 M, 2..4 x ring, 5..6 MMA
-    static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kBar = kTmp + 64;                // 0 C/B, 1 M, 2..4 x ring, 5..6 MMA, 7..8 S_in
+    static constexpr size_t kTmem = kBar + 128;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kAlloc <= 232448, "output CTA exceeds the shared memory of one CTA");
@@ -219,18 +237,31 @@ __device__ __forceinline__ uint32_t col_p(int j) { return 128u + 192u * j; }
 __device__ __forceinline__ uint32_t col_y(int j) { return 192u + 192u * j; }
 __device__ __forceinline__ uint32_t col_y2(int j) { return 256u + 192u * j; }
 
+// dt of the CTA's heads at the chunk's steps into shared memory ([head][step], 0 past L).
+__device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, int b, int t0, int hfirst, int nh, int row) {
+    const bool valid = t0 + row < a.L;
+    const __nv_bfloat16* src = a.dt + ((size_t)b * a.L + (valid ? t0 + row : 0)) * a.H + hfirst;
+    float v[kMaxHB];
+#pragma unroll
+    for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? __bfloat162float(src[i]) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxHB; ++i) dts[i * kQ + row] = v[i];
+}
+
 // One CTA per (chunk, batch row, group, block of hb heads), heads software-pipelined:
-//   prep(i): decays of head i, S_in -> bf16 tile, P = M o Lmask -> TMEM (bf16 pairs);
-//   issue(i): Y = P X (A from TMEM), Y2 = C S_in;
-//   finish(i - 1): y = Y + E Y2 + D x -> the x tile -> TMA store; the freed x slot loads head i + 2.
+//   prep(i): decays of head i, P = M o Lmask -> TMEM (bf16 pairs);
+//   issue(i): Y = P X (A from TMEM), Y2 = C S_in (S_in tile bulk-copied two heads ahead);
+//   finish(i - 1): y = Y + E Y2 + D x -> the x tile -> TMA store; the freed x slot loads head
+//   i + 2 and the freed S_in slot head i + 1.
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
-               const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a, int hb,
-               int nblk) {
+               const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
+               const char* stiles, int hb, int nblk) {
     using SM = OutSmem;
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    float* dts = reinterpret_cast<float*>(sm + SM::kDt);
     float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
     float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
     float* cf = reinterpret_cast<float*>(sm + SM::kCf);
@@ -250,9 +281,10 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     const int hfirst = g * a.HpG + blk * hb;
     const int nh = min(hb, a.HpG - blk * hb);
     const bool has_in = c > 0;
+    auto stile = [&](int h) { return stiles + (((size_t)c * a.B + b) * a.H + h) * kTileBytes; };
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 9; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -271,15 +303,14 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             mbar_arrive_expect_tx(&bar[2 + i], (uint32_t)(kQ * kP * 2));
             tma_load_4d(sm + SM::kX + i * kQ * 128, &mX, &bar[2 + i], 0, hfirst + i, t0, b);
         }
+        if (has_in) {
+            for (int i = 0; i < min(2, nh); ++i) {
+                mbar_arrive_expect_tx(&bar[7 + i], kTileBytes);
+                bulk_load(sm + SM::kSt + i * kTileBytes, stile(hfirst + i), kTileBytes, &bar[7 + i]);
+            }
+        }
     }
-    // S_in rows (row n = tid) of the next head, prefetched into registers
-    float4 sreg[16];
-    auto load_s = [&](int h) {
-        const float* src = a.ckpt + ((((size_t)c * a.B + b) * a.H + h) * kKD + tid) * kP;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sreg[e] = __ldcg(reinterpret_cast<const float4*>(src) + e);
-    };
-    if (has_in) load_s(hfirst);
+    load_dts(a, dts, b, t0, hfirst, nh, tid);
 
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 710);
     if (tid == 0 && ok) {
@@ -326,6 +357,10 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         if (tid == 0) {
             tma_store_4d(&mY, X, 0, hfirst + i, t0, b);
             bulk_commit();
+            if (has_in && i + 2 < nh) {  // S_in slot j is free (the MMAs of head i are complete)
+                mbar_arrive_expect_tx(&bar[7 + j], kTileBytes);
+                bulk_load(sm + SM::kSt + j * kTileBytes, stile(hfirst + i + 2), kTileBytes, &bar[7 + j]);
+            }
             bulk_wait_read_all();
             if (i + 3 < nh) {
                 mbar_arrive_expect_tx(&bar[2 + xb], (uint32_t)(kQ * kP * 2));
@@ -336,9 +371,13 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
 
     for (int i = 0; i < nh; ++i) {
         const int h = hfirst + i, j = i & 1;
-        // ---- prep(i): decays, S_in tile, P
-        float lam, beta;
-        ssd_coef(a, b, h, t0 + tid, lam, beta);
+        // ---- prep(i): decays, P
+        float lam = 0.0f, beta = 0.0f;
+        if (t0 + tid < a.L) {
+            const float Ah = a.A[h];
+            lam = dts[i * kQ + tid] * Ah;
+            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+        }
         const float lt = cta_inclusive_sum(lam, tmp);
         const float lt2 = lt * kLog2e;
         l2s[tid] = lt2;
@@ -350,17 +389,6 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         const float l0 = l2s[32 * warp];
         for (int s = lane; s < 32 * warp; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
         __syncwarp();
-        if (has_in) {
-            char* St = sm + SM::kSt + j * kKD * kP * 2;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-                __align__(16) __nv_bfloat162 pk[4] = {
-                    __floats2bfloat162_rn(sreg[e].x, sreg[e].y), __floats2bfloat162_rn(sreg[e].z, sreg[e].w),
-                    __floats2bfloat162_rn(sreg[e + 1].x, sreg[e + 1].y),
-                    __floats2bfloat162_rn(sreg[e + 1].z, sreg[e + 1].w)};
-                *reinterpret_cast<uint4*>(St + tc::sw128_off(tid, 4 * e, kKD)) = *reinterpret_cast<uint4*>(pk);
-            }
-        }
         if (i == 0) ok = ok && mbar_wait(&bar[1], 0, a.hdr, 711);
         tc::fence_after_sync();
         {
@@ -401,27 +429,27 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             }
             tc::wait_st();
         }
-        fence_proxy_async_smem();
         tc::fence_before_sync();
         __syncthreads();
         // ---- issue(i)
         if (tid == 0 && ok) {
             ok = mbar_wait(&bar[2 + i % 3], (uint32_t)((i / 3) & 1), a.hdr, 712);
+            if (has_in) ok = ok && mbar_wait(&bar[7 + j], (uint32_t)((i >> 1) & 1), a.hdr, 715);
             tc::fence_after_sync();
             tc::mma_ts_tiles(tmem + col_y(j), tmem + col_p(j), smem_u32(sm + SM::kX + (i % 3) * kQ * 128), 1, kQ, kP,
                              kQ, 0);
             if (has_in)
-                tc::mma_tiles(tmem + col_y2(j), sC, 0, kQ, smem_u32(sm + SM::kSt + j * kKD * kP * 2), 1, kKD, kQ, kP,
+                tc::mma_tiles(tmem + col_y2(j), sC, 0, kQ, smem_u32(sm + SM::kSt + j * kTileBytes), 1, kKD, kQ, kP,
                               kKD, 0);
             tc::commit(&bar[5 + j]);
         }
         __syncwarp();
-        if (has_in && i + 1 < nh) load_s(h + 1);
         if (i > 0) finish(i - 1, Eprev, Dprev);
         Eprev = Ecur;
         Dprev = Dcur;
     }
     if (nh > 0) finish(nh - 1, Eprev, Dprev);
+    if (tid == 0) bulk_wait_all();
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -486,7 +514,8 @@ int out_heads_per_cta(const lr_desc& d, int nchunk) {
 // =========================================================================================
 struct SsdGradArgs {
     SsdArgs a;
-    const float* G;        // [nchunk][B][H][N][P] adjoint of each chunk's outgoing state
+    const char* gtiles;    // [nchunk][B][H] bf16 tiles: adjoint of each chunk's outgoing state
+    const char* stiles;    // [nchunk][B][H] bf16 tiles: state entering each chunk
     __nv_bfloat16* ddt;    // [B, L, H]
     float* dB;             // [B, L, G, N]
     float* dC;
@@ -502,7 +531,8 @@ struct GradSmem {
     static constexpr size_t kPt = kReg + 2 * kQ * kQ * 2;  // P, then the dx staging tile
     static constexpr size_t kSt = kPt + kQ * kQ * 2;       // S_in bf16 [n][p]
     static constexpr size_t kGt = kSt + kKD * kP * 2;      // G bf16 [n][p]
-    static constexpr size_t kL2 = kGt + kKD * kP * 2;      // l log2e [128]
+    static constexpr size_t kDt = kGt + kKD * kP * 2;      // dt of every head [kMaxHB][128] f32
+    static constexpr size_t kL2 = kDt + kMaxHB * kQ * 4;   // l log2e [128]
     static constexpr size_t kBeta = kL2 + kQ * 4;          // beta [128]
     static constexpr size_t kCf = kBeta + kQ * 4;          // column factors [4][128]
     static constexpr size_t kRowp = kCf + 4 * kQ * 4;      // row sums of R [2][128]
@@ -512,7 +542,7 @@ struct GradSmem {
     static constexpr size_t kDd = kKdk + 2 * kQ * 4;       // dy . x [2][128]
     static constexpr size_t kGs = kDd + 2 * kQ * 4;        // <G, S_in> partials [256]
     static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
-    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A, 4 batch 1, 5 batch 2
+    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A, 4 batch 1, 5 batch 2, 6 S_in/G
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
@@ -585,6 +615,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     float* ddp = reinterpret_cast<float*>(sm + SM::kDd);
     float* gsp = reinterpret_cast<float*>(sm + SM::kGs);
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    float* dts = reinterpret_cast<float*>(sm + SM::kDt);
     const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sP = smem_u32(sm + SM::kPt),
                    sS = smem_u32(sm + SM::kSt), sG = smem_u32(sm + SM::kGt);
     const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
@@ -604,7 +635,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
 
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 7; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -624,21 +655,20 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         tma_load_4d(region(0), &mX, &bar[1], 0, hfirst, t0, b);
         tma_load_4d(region(0) + kQ * kP * 2, &mdY, &bar[1], 0, hfirst, t0, b);
     }
-    // S_in and G rows (row n = row, columns [32 wg, 32 wg + 32)) of the next head, in registers
-    float4 sin_r[8], g_r[8];
+    // S_in and G tiles of head h (bulk copies; phase completes also when neither exists)
     auto load_sg = [&](int h) {
-        const size_t off = ((((size_t)c * a.B + b) * a.H + h) * kKD + row) * kP + 32 * wg;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            sin_r[e] = has_in ? __ldcg(reinterpret_cast<const float4*>(a.ckpt + off) + e) : make_float4(0, 0, 0, 0);
-            g_r[e] = has_out ? __ldcg(reinterpret_cast<const float4*>(ga.G + off) + e) : make_float4(0, 0, 0, 0);
+        const size_t tile = (((size_t)c * a.B + b) * a.H + h) * kTileBytes;
+        const uint32_t bytes = (has_in ? kTileBytes : 0u) + (has_out ? kTileBytes : 0u);
+        if (bytes == 0) {
+            mbar_arrive(&bar[6]);
+            return;
         }
+        mbar_arrive_expect_tx(&bar[6], bytes);
+        if (has_in) bulk_load(sm + SM::kSt, ga.stiles + tile, kTileBytes, &bar[6]);
+        if (has_out) bulk_load(sm + SM::kGt, ga.gtiles + tile, kTileBytes, &bar[6]);
     };
-    load_sg(hfirst);
-    auto load_dt = [&](int h) {
-        return (wg == 0 && t0 + row < a.L) ? a.dt[((size_t)b * a.L + t0 + row) * a.H + h] : __float2bfloat16_rn(0.0f);
-    };
-    __nv_bfloat16 dt_next = load_dt(hfirst);
+    if (tid == 0) load_sg(hfirst);
+    if (wg == 0) load_dts(a, dts, b, t0, hfirst, nh, row);
     bool ok = true;
 
     for (int i = 0; i < nh; ++i) {
@@ -651,8 +681,9 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (i > 0) {
             ok = ok && mbar_wait(&bar[5], (uint32_t)((i - 1) & 1), a.hdr, 720);
             tc::fence_after_sync();
+            if (tid == 0) load_sg(h);  // the S_in / G tiles are free again
         }
-        const float dt_raw = __bfloat162float(dt_next);
+        const float dt_raw = wg == 0 ? dts[i * kQ + row] : 0.0f;
         float lam = 0.0f, beta = 0.0f;
         if (wg == 0 && t0 + row < a.L) {
             const float Ah = a.A[h];
@@ -664,27 +695,6 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             l2s[row] = lt * kLog2e;
             betas[row] = beta;
         }
-        if (i + 1 < nh) dt_next = load_dt(h + 1);
-        // S_in / G rows -> bf16 tiles, <G, S_in> partial
-        {
-            float gs = 0.0f;
-            char* St = sm + SM::kSt;
-            char* Gt = sm + SM::kGt;
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const float fs[8] = {sin_r[e].x, sin_r[e].y, sin_r[e].z, sin_r[e].w,
-                                     sin_r[e + 1].x, sin_r[e + 1].y, sin_r[e + 1].z, sin_r[e + 1].w};
-                const float fg[8] = {g_r[e].x, g_r[e].y, g_r[e].z, g_r[e].w, g_r[e + 1].x, g_r[e + 1].y, g_r[e + 1].z,
-                                     g_r[e + 1].w};
-#pragma unroll
-                for (int q = 0; q < 8; ++q) gs = fmaf(fs[q], fg[q], gs);
-                const int col = 32 * wg + 4 * e;
-                if (has_in) *reinterpret_cast<uint4*>(St + tc::sw128_off(row, col, kKD)) = pack8(fs);
-                if (has_out) *reinterpret_cast<uint4*>(Gt + tc::sw128_off(row, col, kKD)) = pack8(fg);
-            }
-            gsp[tid] = gs;
-        }
-        if (i + 1 < nh) load_sg(h + 1);
         if (tid == 0) {
             if (i == 0) ok = ok && mbar_wait(&bar[0], 0, a.hdr, 721);
             bulk_wait_read_all();  // the previous head's dx store has left the P tile
@@ -705,9 +715,6 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             const int w = k >> 7, s = k & 127;
             if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]) * betas[s];
         }
-        // warpgroup 0 keeps its row's <G, S_in> partials: warpgroup 1 rewrites them for the next
-        // head while warpgroup 0 is still turning this head's row terms into d dt
-        const float gs_row = wg == 0 ? gsp[row] + gsp[row + kQ] : 0.0f;
         __syncthreads();
         // ------------------------------------------------------------ E1(i)
         ok = ok && mbar_wait(&bar[3], (uint32_t)(i & 1), a.hdr, 723);
@@ -778,6 +785,27 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 colp[wq * kQ + s0 + lane] = rr[0];
             }
             rowp[wg * kQ + row] = rsum;
+        }
+        // S_in and G tiles of this head: <G, S_in> partial over this thread's row / columns
+        ok = ok && mbar_wait(&bar[6], (uint32_t)(i & 1), a.hdr, 726);
+        {
+            float gs = 0.0f;
+            if (has_in && has_out) {
+#pragma unroll
+                for (int k = 0; k < 32; k += 8) {
+                    const uint32_t off = tc::sw128_off(row, 32 * wg + k, kKD);
+                    uint4 sr = *reinterpret_cast<const uint4*>(sm + SM::kSt + off);
+                    uint4 gr = *reinterpret_cast<const uint4*>(sm + SM::kGt + off);
+                    const __nv_bfloat162* sv = reinterpret_cast<const __nv_bfloat162*>(&sr);
+                    const __nv_bfloat162* gv = reinterpret_cast<const __nv_bfloat162*>(&gr);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 sf = __bfloat1622float2(sv[e]), gf = __bfloat1622float2(gv[e]);
+                        gs = fmaf(sf.x, gf.x, fmaf(sf.y, gf.y, gs));
+                    }
+                }
+            }
+            gsp[tid] = gs;
         }
         fence_proxy_async_smem();
         tc::fence_before_sync();
@@ -874,7 +902,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             const float ki = kdkp[t] + kdkp[kQ + t];
             const float ddv = ddp[t] + ddp[kQ + t];
             const float kisum = wg0_sum(ki, tmp);
-            const float gs = wg0_sum(gs_row, tmp);
+            const float gs = wg0_sum(gsp[t] + gsp[kQ + t], tmp);
             const float X = ex2(l2s[kQ - 1]) * gs + kisum;
             float dl = rs + qi - cs - ki + (t == kQ - 1 ? X : 0.0f);
             if (!valid) dl = 0.0f;
@@ -963,7 +991,7 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
 }
 
 struct SsdBwdWs {
-    size_t decay, pdA, pdD, G, end;
+    size_t decay, pdA, pdD, U, gtiles, end;
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
@@ -973,7 +1001,8 @@ SsdBwdWs bwd_plan(const lr_desc& d) {
     w.decay = cur.take(sizeof(float) * tiles);
     w.pdA = cur.take(sizeof(float) * tiles);
     w.pdD = cur.take(sizeof(float) * tiles);
-    w.G = cur.take(sizeof(float) * tiles * kKD * kP);
+    w.U = cur.take(sizeof(float) * tiles * kKD * kP);
+    w.gtiles = cur.take((size_t)kTileBytes * tiles);
     w.end = cur.off;
     return w;
 }
@@ -1000,6 +1029,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     CUtensorMap mC, mB, mX, mY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
+    char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     if (!ok) return LR_ERR_INVALID_ARG;
     const int nblk_s = (a.HpG + kHS - 1) / kHS;
     if (a.nchunk > 1) {
@@ -1014,8 +1044,8 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
         const int n4 = kKD * kP / 4;
         const size_t total = (size_t)a.B * a.H * n4;
         note_launch("ssd_state_pass");
-        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)ckpt, a.decay, a.B * a.H, n4,
-                                                                         a.nchunk, +1);
+        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)ckpt, stiles, a.decay, a.B * a.H,
+                                                                         n4, a.nchunk, +1);
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1023,7 +1053,8 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     const int nblk_o = (a.HpG + hb - 1) / hb;
     cudaFuncSetAttribute(ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
-    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, kThreads, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, hb, nblk_o);
+    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, kThreads, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, stiles, hb,
+                                                                                      nblk_o);
     return check_launch();
 }
 
@@ -1036,7 +1067,8 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     SsdGradArgs ga{};
     ga.a = make_args(d, in, ckpt, ws, (float*)(ws + w.decay));
     const SsdArgs& a = ga.a;
-    ga.G = (const float*)(ws + w.G);
+    ga.gtiles = ws + w.gtiles;
+    ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     ga.ddt = (__nv_bfloat16*)gr.ddelta;
     ga.dB = gr.dBm;
     ga.dC = gr.dCm;
@@ -1047,13 +1079,13 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true) &&
               map4(&mdX, gr.dx, kP, d.H, d.L, d.B, true);
     if (!ok) return LR_ERR_INVALID_ARG;
-    float* Gbuf = (float*)(ws + w.G);
+    float* Ubuf = (float*)(ws + w.U);
     const int nblk_s = (a.HpG + kHS - 1) / kHS;
     if (a.nchunk > 1) {
         cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
         note_launch("ssd_chunk_state");
         const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, a, Gbuf, nblk_s, -1);
+        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, a, Ubuf, nblk_s, -1);
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1061,8 +1093,8 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         const int n4 = kKD * kP / 4;
         const size_t total = (size_t)a.B * a.H * n4;
         note_launch("ssd_state_pass");
-        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)Gbuf, a.decay, a.B * a.H, n4,
-                                                                         a.nchunk, -1);
+        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)Ubuf, ws + w.gtiles, a.decay,
+                                                                         a.B * a.H, n4, a.nchunk, -1);
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }

@@ -26,7 +26,7 @@ using namespace chunkc;
 namespace {
 
 constexpr int kP = 64;    // head dimension (value columns)
-constexpr int kHS = 4;    // heads per CTA of the state kernel
+constexpr int kHS = 2;    // heads per CTA of the state kernel
 
 struct SsdArgs {
     int B, L, H, G, HpG, nchunk;  // HpG: heads per group
@@ -58,7 +58,8 @@ struct StateSmem {
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
-    static_assert(2 * kAlloc <= 232448, "two state CTAs per SM");
+    static_assert(3 * (kAlloc + 1024) <= 233472, "three state CTAs per SM");
+    static_assert(kHS == 2, "the f32 staging uses the R tile and the two Z tiles");
 };
 
 // One CTA per (chunk, batch row, group, block of kHS heads):
@@ -66,9 +67,9 @@ struct StateSmem {
 //   dir < 0: U_c = C^T diag(E) dy_h for chunk c = 1 .. nchunk-1, into slot c - 1 of `out`
 //            (the adjoint handed from chunk c to the state leaving chunk c - 1).
 // `decay[(b H + h) nchunk + c]` receives e^{l_Q} of the chunk.
-__global__ void __launch_bounds__(kThreads, 2)
-ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ, SsdArgs a,
-                 float* out, int nblk, int dir) {
+__global__ void __launch_bounds__(kThreads, 3)
+ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
+                 const __grid_constant__ CUtensorMap mOut, SsdArgs a, int nblk, int dir) {
     using SM = StateSmem;
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
@@ -95,7 +96,7 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 256);
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 128);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -142,23 +143,41 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
     __syncwarp();
     ok = ok && mbar_wait(&bar[1], 0, a.hdr, 701);
     tc::fence_after_sync();
+    // f32 results through shared memory (head j: the R tile for j = 0, the two Z tiles for j = 1;
+    // all MMAs are complete) in the 128-byte-swizzled layout of two 32-column TMA boxes
     for (int j = 0; j < nh; ++j) {
-        float* dst = out + ((((size_t)slot * a.B + b) * a.H + hfirst + j) * kKD + tid) * kP;
+        char* stage = sm + (j == 0 ? SM::kR : SM::kZ);
 #pragma unroll
         for (int v0 = 0; v0 < kP; v0 += 16) {
             float v[16];
             tc::ld16(tmem + kP * j + lane_off + v0, v);
             tc::wait_ld();
+            char* box = stage + (v0 >> 5) * (kKD * 128);
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-                __stcg(reinterpret_cast<float4*>(dst + v0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+            for (int k = 0; k < 4; ++k) {
+                const int chunk = ((v0 & 31) >> 2) + k;
+                *reinterpret_cast<float4*>(box + tid * 128 + ((chunk ^ (tid & 7)) << 4)) =
+                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
         }
     }
+    fence_proxy_async_smem();
     tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && ok) {
+        for (int j = 0; j < nh; ++j) {
+            const char* stage = sm + (j == 0 ? SM::kR : SM::kZ);
+            const int bh = b * a.H + hfirst + j;
+            tma_store_4d(&mOut, stage, 0, 0, bh, slot);
+            tma_store_4d(&mOut, stage + kKD * 128, 32, 0, bh, slot);
+        }
+        bulk_commit();
+        bulk_wait_read_all();
+    }
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 256);
+        tc::tmem_dealloc(tmem, 128);
     }
 }
 
@@ -222,7 +241,8 @@ struct OutSmem {
     static constexpr size_t kX = kB + kQ * kKD * 2;          // 3 x (128 x 64) bf16
     static constexpr size_t kSt = kX + 3 * kQ * kP * 2;      // 2 x (128 x 64) bf16, [n][p]
     static constexpr size_t kDt = kSt + 2 * kTileBytes;      // dt of every head [kMaxHB][128] f32
-    static constexpr size_t kL2 = kDt + kMaxHB * kQ * 4;     // l log2e [128]
+    static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;     // A, D of every head [2][kMaxHB]
+    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;      // l log2e [128]
     static constexpr size_t kBeta = kL2 + kQ * 4;            // beta [128]
     static constexpr size_t kCf = kBeta + kQ * 4;            // column factors [4 warps][128]
     static constexpr size_t kTmp = kCf + 4 * kQ * 4;         // scan scratch
@@ -237,8 +257,14 @@ __device__ __forceinline__ uint32_t col_p(int j) { return 128u + 192u * j; }
 __device__ __forceinline__ uint32_t col_y(int j) { return 192u + 192u * j; }
 __device__ __forceinline__ uint32_t col_y2(int j) { return 256u + 192u * j; }
 
-// dt of the CTA's heads at the chunk's steps into shared memory ([head][step], 0 past L).
-__device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, int b, int t0, int hfirst, int nh, int row) {
+// dt of the CTA's heads at the chunk's steps into shared memory ([head][step], 0 past L), and
+// A_h, D_h of the heads (ad[0 .. kMaxHB), ad[kMaxHB ..)).
+__device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad, int b, int t0, int hfirst, int nh,
+                                         int row) {
+    if (row < nh) {
+        ad[row] = a.A[hfirst + row];
+        ad[kMaxHB + row] = a.Dskip ? a.Dskip[hfirst + row] : 0.0f;
+    }
     const bool valid = t0 + row < a.L;
     const __nv_bfloat16* src = a.dt + ((size_t)b * a.L + (valid ? t0 + row : 0)) * a.H + hfirst;
     float v[kMaxHB];
@@ -262,6 +288,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
     float* dts = reinterpret_cast<float*>(sm + SM::kDt);
+    float* ad = reinterpret_cast<float*>(sm + SM::kAD);
     float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
     float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
     float* cf = reinterpret_cast<float*>(sm + SM::kCf);
@@ -310,7 +337,8 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             }
         }
     }
-    load_dts(a, dts, b, t0, hfirst, nh, tid);
+    load_dts(a, dts, ad, b, t0, hfirst, nh, tid);
+    __syncthreads();
 
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 710);
     if (tid == 0 && ok) {
@@ -361,20 +389,21 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
                 mbar_arrive_expect_tx(&bar[7 + j], kTileBytes);
                 bulk_load(sm + SM::kSt + j * kTileBytes, stile(hfirst + i + 2), kTileBytes, &bar[7 + j]);
             }
-            bulk_wait_read_all();
-            if (i + 3 < nh) {
-                mbar_arrive_expect_tx(&bar[2 + xb], (uint32_t)(kQ * kP * 2));
-                tma_load_4d(X, &mX, &bar[2 + xb], 0, hfirst + i + 3, t0, b);
+            if (i >= 1 && i + 2 < nh) {  // head i - 1's y has left its slot: it takes x of head i + 2
+                const int xo = (i + 2) % 3;
+                bulk_wait_read_1();
+                mbar_arrive_expect_tx(&bar[2 + xo], (uint32_t)(kQ * kP * 2));
+                tma_load_4d(sm + SM::kX + xo * kQ * 128, &mX, &bar[2 + xo], 0, hfirst + i + 2, t0, b);
             }
         }
     };
 
     for (int i = 0; i < nh; ++i) {
-        const int h = hfirst + i, j = i & 1;
+        const int j = i & 1;
         // ---- prep(i): decays, P
         float lam = 0.0f, beta = 0.0f;
         if (t0 + tid < a.L) {
-            const float Ah = a.A[h];
+            const float Ah = ad[i];
             lam = dts[i * kQ + tid] * Ah;
             beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
         }
@@ -384,7 +413,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         betas[tid] = beta;
         __syncthreads();
         const float Ecur = ex2(lt2);
-        const float Dcur = a.Dskip ? a.Dskip[h] : 0.0f;
+        const float Dcur = ad[kMaxHB + i];
         float* cfw = cf + warp * kQ;
         const float l0 = l2s[32 * warp];
         for (int s = lane; s < 32 * warp; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
@@ -456,6 +485,15 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
+}
+
+// TMA map of the f32 state slots [nslot][B*H][N][P], boxes of 32 columns x 128 rows (128-byte
+// swizzle), written by the state kernel.
+bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
+    uint64_t dims[4] = {(uint64_t)kP, (uint64_t)kKD, (uint64_t)BH, (uint64_t)nslot};
+    uint64_t str[3] = {kP * 4, (uint64_t)kKD * kP * 4, (uint64_t)BH * kKD * kP * 4};
+    uint32_t box[4] = {32, (uint32_t)kKD, 1, 1};
+    return make_tmap(m, base, 4, 4, dims, str, box, true);
 }
 
 struct SsdFwdWs {
@@ -532,7 +570,8 @@ struct GradSmem {
     static constexpr size_t kSt = kPt + kQ * kQ * 2;       // S_in bf16 [n][p]
     static constexpr size_t kGt = kSt + kKD * kP * 2;      // G bf16 [n][p]
     static constexpr size_t kDt = kGt + kKD * kP * 2;      // dt of every head [kMaxHB][128] f32
-    static constexpr size_t kL2 = kDt + kMaxHB * kQ * 4;   // l log2e [128]
+    static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;   // A, D of every head [2][kMaxHB]
+    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;    // l log2e [128]
     static constexpr size_t kBeta = kL2 + kQ * 4;          // beta [128]
     static constexpr size_t kCf = kBeta + kQ * 4;          // column factors [4][128]
     static constexpr size_t kRowp = kCf + 4 * kQ * 4;      // row sums of R [2][128]
@@ -616,6 +655,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     float* gsp = reinterpret_cast<float*>(sm + SM::kGs);
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
     float* dts = reinterpret_cast<float*>(sm + SM::kDt);
+    float* ad = reinterpret_cast<float*>(sm + SM::kAD);
     const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sP = smem_u32(sm + SM::kPt),
                    sS = smem_u32(sm + SM::kSt), sG = smem_u32(sm + SM::kGt);
     const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
@@ -668,7 +708,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (has_out) bulk_load(sm + SM::kGt, ga.gtiles + tile, kTileBytes, &bar[6]);
     };
     if (tid == 0) load_sg(hfirst);
-    if (wg == 0) load_dts(a, dts, b, t0, hfirst, nh, row);
+    if (wg == 0) load_dts(a, dts, ad, b, t0, hfirst, nh, row);
+    __syncthreads();
     bool ok = true;
 
     for (int i = 0; i < nh; ++i) {
@@ -686,7 +727,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         const float dt_raw = wg == 0 ? dts[i * kQ + row] : 0.0f;
         float lam = 0.0f, beta = 0.0f;
         if (wg == 0 && t0 + row < a.L) {
-            const float Ah = a.A[h];
+            const float Ah = ad[i];
             lam = dt_raw * Ah;
             beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
         }
@@ -832,7 +873,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             const float l2r = l2s[row];
             const float E = ex2(l2r);
             const float w = ex2(l2s[kQ - 1] - l2r) * betas[row];
-            const float Dh = a.Dskip ? a.Dskip[h] : 0.0f;
+            const float Dh = ad[kMaxHB + i];
             float qdq = 0.0f, kdk = 0.0f, dd = 0.0f;
 #pragma unroll
             for (int v0 = 0; v0 < 32; v0 += 16) {
@@ -912,7 +953,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             const float dlam = tmp[16] - incl + dl;
             float dA_part = 0.0f;
             if (valid) {
-                const float Ah = a.A[h];
+                const float Ah = ad[i];
                 const float bt = betas[t];
                 const float ab = ex2(dt_raw * Ah * kLog2e);
                 const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
@@ -1033,10 +1074,12 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     if (!ok) return LR_ERR_INVALID_ARG;
     const int nblk_s = (a.HpG + kHS - 1) / kHS;
     if (a.nchunk > 1) {
+        CUtensorMap mS;
+        if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
         cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
         note_launch("ssd_chunk_state");
         const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mB, mX, a, (float*)ckpt, nblk_s, +1);
+        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mB, mX, mS, a, nblk_s, +1);
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1082,10 +1125,12 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     float* Ubuf = (float*)(ws + w.U);
     const int nblk_s = (a.HpG + kHS - 1) / kHS;
     if (a.nchunk > 1) {
+        CUtensorMap mU;
+        if (!map_states(&mU, Ubuf, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
         cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
         note_launch("ssd_chunk_state");
         const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, a, Ubuf, nblk_s, -1);
+        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, mU, a, nblk_s, -1);
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }

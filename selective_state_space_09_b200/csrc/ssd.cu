@@ -233,30 +233,6 @@ ssd_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int B
 // ---------------------------------------------------------------------------------- outputs
 constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernels)
 
-// Shared memory of the output CTA: C and B of the chunk, a ring of three x tiles (each becomes
-// the y staging tile of its head), two bf16 S_in tiles, per-head dt, the current head's decays.
-struct OutSmem {
-    static constexpr size_t kC = 0;                          // 128 x 128 bf16
-    static constexpr size_t kB = kC + kQ * kKD * 2;          // 128 x 128 bf16
-    static constexpr size_t kX = kB + kQ * kKD * 2;          // 3 x (128 x 64) bf16
-    static constexpr size_t kSt = kX + 3 * kQ * kP * 2;      // 2 x (128 x 64) bf16, [n][p]
-    static constexpr size_t kDt = kSt + 2 * kTileBytes;      // dt of every head [kMaxHB][128] f32
-    static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;     // A, D of every head [2][kMaxHB]
-    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;      // l log2e [128]
-    static constexpr size_t kBeta = kL2 + kQ * 4;            // beta [128]
-    static constexpr size_t kCf = kBeta + kQ * 4;            // column factors [4 warps][128]
-    static constexpr size_t kTmp = kCf + 4 * kQ * 4;         // scan scratch
-    static constexpr size_t kBar = kTmp + 64;                // 0 C/B, 1 M, 2..4 x ring, 5..6 MMA, 7..8 S_in
-    static constexpr size_t kTmem = kBar + 128;
-    static constexpr size_t kEnd = kTmem + 64;
-    static constexpr size_t kAlloc = kEnd + 1024;
-    static_assert(kAlloc <= 232448, "output CTA exceeds the shared memory of one CTA");
-};
-// TMEM columns: M = C B^T (f32, 128), then two head buffers of P (bf16 pairs, 64), Y (64), Y2 (64).
-__device__ __forceinline__ uint32_t col_p(int j) { return 128u + 192u * j; }
-__device__ __forceinline__ uint32_t col_y(int j) { return 192u + 192u * j; }
-__device__ __forceinline__ uint32_t col_y2(int j) { return 256u + 192u * j; }
-
 // dt of the CTA's heads at the chunk's steps into shared memory ([head][step], 0 past L), and
 // A_h, D_h of the heads (ad[0 .. kMaxHB), ad[kMaxHB ..)).
 __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad, int b, int t0, int hfirst, int nh,
@@ -274,12 +250,58 @@ __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad
     for (int i = 0; i < kMaxHB; ++i) dts[i * kQ + row] = v[i];
 }
 
-// One CTA per (chunk, batch row, group, block of hb heads), heads software-pipelined:
-//   prep(i): decays of head i, P = M o Lmask -> TMEM (bf16 pairs);
-//   issue(i): Y = P X (A from TMEM), Y2 = C S_in (S_in tile bulk-copied two heads ahead);
-//   finish(i - 1): y = Y + E Y2 + D x -> the x tile -> TMA store; the freed x slot loads head
-//   i + 2 and the freed S_in slot head i + 1.
-__global__ void __launch_bounds__(kThreads, 1)
+// Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
+__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
+
+// Inclusive prefix sum over the 128 threads of warpgroup wg (same order as cta_inclusive_sum).
+__device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
+    const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 3;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[w] = x;
+    wg_sync(wg);
+    float add = 0.0f;
+    for (int k = 0; k < w; ++k) add += tmp[k];
+    wg_sync(wg);
+    return x + add;
+}
+
+// Shared memory of the output CTA: C and B of the chunk; per warpgroup a ring of three x tiles
+// (each becomes the y staging tile of its head) and one bf16 S_in tile; dt, A, D of every head;
+// per warpgroup the current head's decays and column factors.
+struct OutSmem {
+    static constexpr size_t kC = 0;                          // 128 x 128 bf16
+    static constexpr size_t kB = kC + kQ * kKD * 2;          // 128 x 128 bf16
+    static constexpr size_t kX = kB + kQ * kKD * 2;          // [2 warpgroups][3] x (128 x 64) bf16
+    static constexpr size_t kSt = kX + 6 * kQ * kP * 2;      // [2] x (128 x 64) bf16, [n][p]
+    static constexpr size_t kDt = kSt + 2 * kTileBytes;      // dt of every head [kMaxHB][128] f32
+    static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;     // A, D of every head [2][kMaxHB]
+    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;      // l log2e [2][128]
+    static constexpr size_t kBeta = kL2 + 2 * kQ * 4;        // beta [2][128]
+    static constexpr size_t kCf = kBeta + 2 * kQ * 4;        // column factors [2][4 warps][128]
+    static constexpr size_t kTmp = kCf + 2 * 4 * kQ * 4;     // scan scratch [2][16]
+    static constexpr size_t kBar = kTmp + 128;               // 0 C/B, 1 M; 2 + 5 wg: x ring (3), S_in, MMA
+    static constexpr size_t kTmem = kBar + 128;
+    static constexpr size_t kEnd = kTmem + 64;
+    static constexpr size_t kAlloc = kEnd + 1024;
+    static_assert(kAlloc <= 232448, "output CTA exceeds the shared memory of one CTA");
+};
+// TMEM columns: M = C B^T (f32, 128), then per warpgroup P (bf16 pairs, 64), Y (64), Y2 (64).
+__device__ __forceinline__ uint32_t col_p(int w) { return 128u + 192u * w; }
+__device__ __forceinline__ uint32_t col_y(int w) { return 192u + 192u * w; }
+__device__ __forceinline__ uint32_t col_y2(int w) { return 256u + 192u * w; }
+
+// One CTA per (chunk, batch row, group, block of hb heads), 256 threads.  M = C B^T is computed
+// once; warpgroup w takes heads w, w + 2, ... through its own TMEM buffer, so one warpgroup's
+// epilogues overlap the other's products.  Per head (thread = row t of the chunk):
+//   prep: decays of the head, P = M o Lmask -> TMEM (bf16 pairs);
+//   issue (one thread): Y = P X (A from TMEM), Y2 = C S_in;
+//   finish: y = Y + E Y2 + D x -> the x tile -> TMA store; the freed S_in slot loads the
+//   warpgroup's next head and the x slot freed one head earlier the head after next.
+__global__ void __launch_bounds__(256, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
                const char* stiles, int hb, int nblk) {
@@ -287,15 +309,18 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    const int tid = threadIdx.x, wg = tid >> 7, wt = tid & 127, wq = (tid >> 5) & 3, lane = tid & 31;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     float* dts = reinterpret_cast<float*>(sm + SM::kDt);
     float* ad = reinterpret_cast<float*>(sm + SM::kAD);
-    float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
-    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
-    float* cf = reinterpret_cast<float*>(sm + SM::kCf);
-    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
+    float* l2s = reinterpret_cast<float*>(sm + SM::kL2) + wg * kQ;
+    float* betas = reinterpret_cast<float*>(sm + SM::kBeta) + wg * kQ;
+    float* cfw = reinterpret_cast<float*>(sm + SM::kCf) + (wg * 4 + wq) * kQ;
+    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp) + wg * 16;
+    uint64_t* wbar = bar + 2 + 5 * wg;  // x ring 0..2, S_in 3, MMA 4
+    char* Xs = sm + SM::kX + (size_t)wg * 3 * kQ * kP * 2;
+    char* St = sm + SM::kSt + (size_t)wg * kTileBytes;
     const uint32_t sC = smem_u32(sm + SM::kC), sB = smem_u32(sm + SM::kB);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
     int idx = blockIdx.x;
     const int blk = idx % nblk;
@@ -307,15 +332,16 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     const int t0 = c * kQ;
     const int hfirst = g * a.HpG + blk * hb;
     const int nh = min(hb, a.HpG - blk * hb);
+    const int nmine = (nh - wg + 1) / 2;  // heads wg, wg + 2, ...
     const bool has_in = c > 0;
     auto stile = [&](int h) { return stiles + (((size_t)c * a.B + b) * a.H + h) * kTileBytes; };
 
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 12; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    if (tid < 32) tc::tmem_alloc(tmem_slot, 512);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -326,44 +352,112 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             tma_load_4d(sm + SM::kC + j * kQ * 128, &mC, &bar[0], 64 * j, g, t0, b);
             tma_load_4d(sm + SM::kB + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
         }
-        for (int i = 0; i < min(3, nh); ++i) {
-            mbar_arrive_expect_tx(&bar[2 + i], (uint32_t)(kQ * kP * 2));
-            tma_load_4d(sm + SM::kX + i * kQ * 128, &mX, &bar[2 + i], 0, hfirst + i, t0, b);
+    }
+    if (wt == 0) {
+        for (int u = 0; u < min(3, nmine); ++u) {
+            mbar_arrive_expect_tx(&wbar[u], (uint32_t)(kQ * kP * 2));
+            tma_load_4d(Xs + u * kQ * 128, &mX, &wbar[u], 0, hfirst + wg + 2 * u, t0, b);
         }
-        if (has_in) {
-            for (int i = 0; i < min(2, nh); ++i) {
-                mbar_arrive_expect_tx(&bar[7 + i], kTileBytes);
-                bulk_load(sm + SM::kSt + i * kTileBytes, stile(hfirst + i), kTileBytes, &bar[7 + i]);
-            }
+        if (has_in && nmine > 0) {
+            mbar_arrive_expect_tx(&wbar[3], kTileBytes);
+            bulk_load(St, stile(hfirst + wg), kTileBytes, &wbar[3]);
         }
     }
-    load_dts(a, dts, ad, b, t0, hfirst, nh, tid);
+    if (wg == 0) load_dts(a, dts, ad, b, t0, hfirst, nh, wt);
     __syncthreads();
-
-    bool ok = mbar_wait(&bar[0], 0, a.hdr, 710);
-    if (tid == 0 && ok) {
-        tc::fence_after_sync();
-        tc::mma_tiles(tmem, sC, 0, kQ, sB, 0, kQ, kQ, kQ, kKD, 0);  // M = C B^T
+    bool ok = true;
+    if (tid == 0) {
+        ok = mbar_wait(&bar[0], 0, a.hdr, 710);
+        if (ok) {
+            tc::fence_after_sync();
+            tc::mma_tiles(tmem, sC, 0, kQ, sB, 0, kQ, kQ, kQ, kKD, 0);  // M = C B^T
+        }
         tc::commit(&bar[1]);
     }
-    __syncwarp();
+    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 711);
+    tc::fence_after_sync();
 
-    float Eprev = 0.0f, Dprev = 0.0f;
-    auto finish = [&](int i, float E, float Dh) {
-        const int j = i & 1, xb = i % 3;
-        ok = ok && mbar_wait(&bar[5 + j], (uint32_t)((i >> 1) & 1), a.hdr, 713);
-        ok = ok && mbar_wait(&bar[2 + xb], (uint32_t)((i / 3) & 1), a.hdr, 714);  // x rows read below
+    for (int u = 0; u < nmine; ++u) {
+        const int i = wg + 2 * u, xs = u % 3;
+        // ---- prep: decays, column factors, P
+        float lam = 0.0f, beta = 0.0f;
+        if (t0 + wt < a.L) {
+            const float Ah = ad[i];
+            lam = dts[i * kQ + wt] * Ah;
+            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+        }
+        const float lt2 = wg_inclusive_sum(lam, tmp, wg) * kLog2e;
+        l2s[wt] = lt2;
+        betas[wt] = beta;
+        wg_sync(wg);
+        const float E = ex2(lt2);
+        const float Dh = ad[kMaxHB + i];
+        const float l0 = l2s[32 * wq];
+        for (int s = lane; s < 32 * wq; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
+        __syncwarp();
+        {
+            const float rf = ex2(lt2 - l0);
+            const uint32_t pcol = tmem + col_p(wg) + lane_off;
+#pragma unroll 1
+            for (int sb = 0; sb < 4; ++sb) {
+                uint32_t pk[16];
+                if (sb > wq) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                    tc::st16(pcol + 16 * sb, pk);
+                    continue;
+                }
+                float v[32];
+                tc::ld16(tmem + lane_off + 32 * sb, v);
+                tc::ld16(tmem + lane_off + 32 * sb + 16, v + 16);
+                tc::wait_ld();
+                if (sb < wq) {
+                    const float* cfb = cfw + 32 * sb;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * q] * (rf * cfb[2 * q]),
+                                                                  v[2 * q + 1] * (rf * cfb[2 * q + 1]));
+                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int s = 32 * sb + 2 * q;
+                        const float p0 = s <= wt ? v[2 * q] * (ex2(lt2 - l2s[s]) * betas[s]) : 0.0f;
+                        const float p1 = s + 1 <= wt ? v[2 * q + 1] * (ex2(lt2 - l2s[s + 1]) * betas[s + 1]) : 0.0f;
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                }
+                tc::st16(pcol + 16 * sb, pk);
+            }
+            tc::wait_st();
+        }
+        tc::fence_before_sync();
+        wg_sync(wg);
+        // ---- issue
+        if (wt == 0 && ok) {
+            ok = mbar_wait(&wbar[xs], (uint32_t)((u / 3) & 1), a.hdr, 712);
+            if (has_in) ok = ok && mbar_wait(&wbar[3], (uint32_t)(u & 1), a.hdr, 715);
+            tc::fence_after_sync();
+            tc::mma_ts_tiles(tmem + col_y(wg), tmem + col_p(wg), smem_u32(Xs + xs * kQ * 128), 1, kQ, kP, kQ, 0);
+            if (has_in) tc::mma_tiles(tmem + col_y2(wg), sC, 0, kQ, smem_u32(St), 1, kKD, kQ, kP, kKD, 0);
+            tc::commit(&wbar[4]);
+        }
+        // ---- finish
+        ok = ok && mbar_wait(&wbar[4], (uint32_t)(u & 1), a.hdr, 713);
+        ok = ok && mbar_wait(&wbar[xs], (uint32_t)((u / 3) & 1), a.hdr, 714);  // x rows read below
         tc::fence_after_sync();
-        char* X = sm + SM::kX + xb * kQ * 128;
+        char* X = Xs + xs * kQ * 128;
 #pragma unroll
         for (int v0 = 0; v0 < kP; v0 += 16) {
             float y1[16], y2[16];
-            tc::ld16(tmem + col_y(j) + lane_off + v0, y1);
-            if (has_in) tc::ld16(tmem + col_y2(j) + lane_off + v0, y2);
+            tc::ld16(tmem + col_y(wg) + lane_off + v0, y1);
+            if (has_in) tc::ld16(tmem + col_y2(wg) + lane_off + v0, y2);
             tc::wait_ld();
 #pragma unroll
             for (int hh = 0; hh < 16; hh += 8) {
-                uint4* px = reinterpret_cast<uint4*>(X + tc::sw128_off(tid, v0 + hh, kQ));
+                uint4* px = reinterpret_cast<uint4*>(X + tc::sw128_off(wt, v0 + hh, kQ));
                 uint4 raw = *px;
                 __nv_bfloat162* xv = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
@@ -381,107 +475,26 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         }
         fence_proxy_async_smem();
         tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
+        wg_sync(wg);
+        if (wt == 0) {
             tma_store_4d(&mY, X, 0, hfirst + i, t0, b);
             bulk_commit();
-            if (has_in && i + 2 < nh) {  // S_in slot j is free (the MMAs of head i are complete)
-                mbar_arrive_expect_tx(&bar[7 + j], kTileBytes);
-                bulk_load(sm + SM::kSt + j * kTileBytes, stile(hfirst + i + 2), kTileBytes, &bar[7 + j]);
+            if (has_in && u + 1 < nmine) {  // the S_in slot is free: the products of this head are done
+                mbar_arrive_expect_tx(&wbar[3], kTileBytes);
+                bulk_load(St, stile(hfirst + i + 2), kTileBytes, &wbar[3]);
             }
-            if (i >= 1 && i + 2 < nh) {  // head i - 1's y has left its slot: it takes x of head i + 2
-                const int xo = (i + 2) % 3;
+            if (u >= 1 && u + 2 < nmine) {  // the previous head's y has left its slot
+                const int xo = (u + 2) % 3;
                 bulk_wait_read_1();
-                mbar_arrive_expect_tx(&bar[2 + xo], (uint32_t)(kQ * kP * 2));
-                tma_load_4d(sm + SM::kX + xo * kQ * 128, &mX, &bar[2 + xo], 0, hfirst + i + 2, t0, b);
+                mbar_arrive_expect_tx(&wbar[xo], (uint32_t)(kQ * kP * 2));
+                tma_load_4d(Xs + xo * kQ * 128, &mX, &wbar[xo], 0, hfirst + i + 4, t0, b);
             }
         }
-    };
-
-    for (int i = 0; i < nh; ++i) {
-        const int j = i & 1;
-        // ---- prep(i): decays, P
-        float lam = 0.0f, beta = 0.0f;
-        if (t0 + tid < a.L) {
-            const float Ah = ad[i];
-            lam = dts[i * kQ + tid] * Ah;
-            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
-        }
-        const float lt = cta_inclusive_sum(lam, tmp);
-        const float lt2 = lt * kLog2e;
-        l2s[tid] = lt2;
-        betas[tid] = beta;
-        __syncthreads();
-        const float Ecur = ex2(lt2);
-        const float Dcur = ad[kMaxHB + i];
-        float* cfw = cf + warp * kQ;
-        const float l0 = l2s[32 * warp];
-        for (int s = lane; s < 32 * warp; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
-        __syncwarp();
-        if (i == 0) ok = ok && mbar_wait(&bar[1], 0, a.hdr, 711);
-        tc::fence_after_sync();
-        {
-            const float rf = ex2(lt2 - l0);
-            const uint32_t pcol = tmem + col_p(j) + lane_off;
-#pragma unroll 1
-            for (int sb = 0; sb < 4; ++sb) {
-                uint32_t pk[16];
-                if (sb > warp) {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) pk[q] = 0u;
-                    tc::st16(pcol + 16 * sb, pk);
-                    continue;
-                }
-                float v[32];
-                tc::ld16(tmem + lane_off + 32 * sb, v);
-                tc::ld16(tmem + lane_off + 32 * sb + 16, v + 16);
-                tc::wait_ld();
-                if (sb < warp) {
-                    const float* cfb = cfw + 32 * sb;
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * q] * (rf * cfb[2 * q]),
-                                                                  v[2 * q + 1] * (rf * cfb[2 * q + 1]));
-                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int s = 32 * sb + 2 * q;
-                        const float p0 = s <= tid ? v[2 * q] * (ex2(lt2 - l2s[s]) * betas[s]) : 0.0f;
-                        const float p1 = s + 1 <= tid ? v[2 * q + 1] * (ex2(lt2 - l2s[s + 1]) * betas[s + 1]) : 0.0f;
-                        __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-                        pk[q] = *reinterpret_cast<uint32_t*>(&pr);
-                    }
-                }
-                tc::st16(pcol + 16 * sb, pk);
-            }
-            tc::wait_st();
-        }
-        tc::fence_before_sync();
-        __syncthreads();
-        // ---- issue(i)
-        if (tid == 0 && ok) {
-            ok = mbar_wait(&bar[2 + i % 3], (uint32_t)((i / 3) & 1), a.hdr, 712);
-            if (has_in) ok = ok && mbar_wait(&bar[7 + j], (uint32_t)((i >> 1) & 1), a.hdr, 715);
-            tc::fence_after_sync();
-            tc::mma_ts_tiles(tmem + col_y(j), tmem + col_p(j), smem_u32(sm + SM::kX + (i % 3) * kQ * 128), 1, kQ, kP,
-                             kQ, 0);
-            if (has_in)
-                tc::mma_tiles(tmem + col_y2(j), sC, 0, kQ, smem_u32(sm + SM::kSt + j * kTileBytes), 1, kKD, kQ, kP,
-                              kKD, 0);
-            tc::commit(&bar[5 + j]);
-        }
-        __syncwarp();
-        if (i > 0) finish(i - 1, Eprev, Dprev);
-        Eprev = Ecur;
-        Dprev = Dcur;
     }
-    if (nh > 0) finish(nh - 1, Eprev, Dprev);
-    if (tid == 0) bulk_wait_all();
+    if (wt == 0) bulk_wait_all();
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (tid < 32) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
@@ -571,17 +584,17 @@ struct GradSmem {
     static constexpr size_t kGt = kSt + kKD * kP * 2;      // G bf16 [n][p]
     static constexpr size_t kDt = kGt + kKD * kP * 2;      // dt of every head [kMaxHB][128] f32
     static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;   // A, D of every head [2][kMaxHB]
-    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;    // l log2e [128]
-    static constexpr size_t kBeta = kL2 + kQ * 4;          // beta [128]
-    static constexpr size_t kCf = kBeta + kQ * 4;          // column factors [4][128]
-    static constexpr size_t kRowp = kCf + 4 * kQ * 4;      // row sums of R [2][128]
+    static constexpr size_t kL2 = kAD + 2 * kMaxHB * 4;    // l log2e [2 heads in flight][128]
+    static constexpr size_t kBeta = kL2 + 2 * kQ * 4;      // beta [2][128]
+    static constexpr size_t kCf = kBeta + 2 * kQ * 4;      // column factors [2][4][128]
+    static constexpr size_t kRowp = kCf + 2 * 4 * kQ * 4;  // row sums of R [2][128]
     static constexpr size_t kColp = kRowp + 2 * kQ * 4;    // column sums of R [4][128]
     static constexpr size_t kQdq = kColp + 4 * kQ * 4;     // E dy . Y2 [2][128]
     static constexpr size_t kKdk = kQdq + 2 * kQ * 4;      // w x . BG [2][128]
     static constexpr size_t kDd = kKdk + 2 * kQ * 4;       // dy . x [2][128]
     static constexpr size_t kGs = kDd + 2 * kQ * 4;        // <G, S_in> partials [256]
     static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
-    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A, 4 batch 1, 5 batch 2, 6 S_in/G
+    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A (+ batch 2), 4 batch 1 (dV1, BG, Y2), 5 batch 1 (dC, dB), 6 S_in/G
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
@@ -592,8 +605,14 @@ constexpr uint32_t kGdC = 0, kGdB = 128, kGM = 256, kGS2 = 384, kGdV = 256, kGBG
 
 __device__ __forceinline__ void wg0_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum).
-__device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp) {
+// Thread that issues the gradient kernel's products after the prologue: warpgroup 1 idles while
+// they run, and an issuing thread blocks while the tensor pipe is full, so warpgroup 0 stays free
+// to prepare the next head's decays and to reduce the current head's row terms.
+constexpr int kIssuer = 128;
+
+// Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum);
+// *total receives the sum of all 128 values.
+__device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp, float* total = nullptr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -604,17 +623,24 @@ __device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp) {
     wg0_bar();
     float add = 0.0f;
     for (int w = 0; w < warp; ++w) add += tmp[w];
+    if (total) *total = ((tmp[0] + tmp[1]) + tmp[2]) + tmp[3];
     wg0_bar();
     return x + add;
 }
-// Sum over the 128 threads of warpgroup 0, fixed order, result in every thread.
-__device__ __forceinline__ float wg0_sum(float x, float* tmp) {
+// Sums of two values over the 128 threads of warpgroup 0, fixed order, results in every thread.
+__device__ __forceinline__ float2 wg0_sum2(float x, float y, float* tmp) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) tmp[8 + warp] = x;
+    for (int o = 16; o > 0; o >>= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+        y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (lane == 0) {
+        tmp[8 + warp] = x;
+        tmp[12 + warp] = y;
+    }
     wg0_bar();
-    const float s = (tmp[8] + tmp[9]) + (tmp[10] + tmp[11]);
+    const float2 s = make_float2((tmp[8] + tmp[9]) + (tmp[10] + tmp[11]), (tmp[12] + tmp[13]) + (tmp[14] + tmp[15]));
     wg0_bar();
     return s;
 }
@@ -630,11 +656,13 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 
 // One CTA per (chunk, batch row, group, block of hb heads), 256 threads: warpgroup wg handles
 // columns [64 wg, 64 wg + 64) (or [32 wg, ...) of 64-wide tensors) of TMEM lane / row 32 wq + lane.
-// Per head: phase A (M = C B^T, S2 = dy x^T) -> E1 (P, Pd, row / column sums of R) -> batch 1
-// (Pd B, Pd^T C into dC, dB; P^T dy, B G, C S_in) -> E2 (dx, inter-chunk row dots, scaling of dy
-// by E and x by w) -> batch 2 (diag(E) dy S_in^T, diag(w) x G^T into dC, dB) while warpgroup 0
-// turns the row terms into d dt.  The {x, dy} region of head i + 1 is loaded into the region that
-// held Pd of head i, so loads overlap the tail of each head.
+// Per head i:
+//   E1: P, Pd (bf16 tiles) and the row / column sums of R from M and S2 of head i;
+//   batch 1: Pd B, Pd^T C into dC, dB (committed first: Pd's region then takes {x, dy} of head
+//     i + 1), then P^T dy, B G, C S_in; warpgroup 0 meanwhile prepares the decays of head i + 1;
+//   E2: dx, the inter-chunk row dots, dy scaled by E and x by w in place;
+//   batch 2: diag(E) dy S_in^T, diag(w) x G^T into dC, dB, issued with phase A of head i + 1
+//     (M = C B^T, S2 = dy x^T) while warpgroup 0 turns head i's row terms into d dt.
 __global__ void __launch_bounds__(256, 1)
 ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                 const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
@@ -644,9 +672,9 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
-    float* l2s = reinterpret_cast<float*>(sm + SM::kL2);
-    float* betas = reinterpret_cast<float*>(sm + SM::kBeta);
-    float* cf = reinterpret_cast<float*>(sm + SM::kCf);
+    float* l2all = reinterpret_cast<float*>(sm + SM::kL2);
+    float* betall = reinterpret_cast<float*>(sm + SM::kBeta);
+    float* cfall = reinterpret_cast<float*>(sm + SM::kCf);
     float* rowp = reinterpret_cast<float*>(sm + SM::kRowp);
     float* colp = reinterpret_cast<float*>(sm + SM::kColp);
     float* qdqp = reinterpret_cast<float*>(sm + SM::kQdq);
@@ -685,17 +713,12 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     auto region = [&](int r) { return sm + SM::kReg + (size_t)r * kQ * kQ * 2; };
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2));
-        for (int j = 0; j < kKD / 64; ++j) {
-            tma_load_4d(sm + SM::kQt + j * kQ * 128, &mC, &bar[0], 64 * j, g, t0, b);
-            tma_load_4d(sm + SM::kKt + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
-        }
-        mbar_arrive_expect_tx(&bar[1], (uint32_t)(2 * kQ * kP * 2));
-        tma_load_4d(region(0), &mX, &bar[1], 0, hfirst, t0, b);
-        tma_load_4d(region(0) + kQ * kP * 2, &mdY, &bar[1], 0, hfirst, t0, b);
-    }
-    // S_in and G tiles of head h (bulk copies; phase completes also when neither exists)
+    auto load_xdy = [&](int r, int h) {  // {x, dy} of head h into region r
+        mbar_arrive_expect_tx(&bar[1 + r], (uint32_t)(2 * kQ * kP * 2));
+        tma_load_4d(region(r), &mX, &bar[1 + r], 0, h, t0, b);
+        tma_load_4d(region(r) + kQ * kP * 2, &mdY, &bar[1 + r], 0, h, t0, b);
+    };
+    // S_in and G tiles of head h (bulk copies; the phase completes also when neither exists)
     auto load_sg = [&](int h) {
         const size_t tile = (((size_t)c * a.B + b) * a.H + h) * kTileBytes;
         const uint32_t bytes = (has_in ? kTileBytes : 0u) + (has_out ? kTileBytes : 0u);
@@ -707,10 +730,58 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (has_in) bulk_load(sm + SM::kSt, ga.stiles + tile, kTileBytes, &bar[6]);
         if (has_out) bulk_load(sm + SM::kGt, ga.gtiles + tile, kTileBytes, &bar[6]);
     };
-    if (tid == 0) load_sg(hfirst);
-    if (wg == 0) load_dts(a, dts, ad, b, t0, hfirst, nh, row);
-    __syncthreads();
+    // phase A of head i ({x, dy} in region i & 1): M = C B^T, S2 = dy x^T
+    auto phase_a = [&](int i) {
+        const uint32_t sXi = smem_u32(region(i & 1)), sOi = sXi + kQ * kP * 2;
+        tc::mma_tiles(tmem + kGM, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);
+        tc::mma_tiles(tmem + kGS2, sOi, 0, kQ, sXi, 0, kQ, kQ, kQ, kP, 0);
+    };
+    // decays of head i into buffer i & 1 (warpgroup 0): l log2e, beta, column factors
+    // cf[w][s] = e^{l_{32 w} - l_s} beta_s (s < 32 w)
+    auto decays = [&](int i) {
+        float* l2s = l2all + (i & 1) * kQ;
+        float* betas = betall + (i & 1) * kQ;
+        float* cf = cfall + (i & 1) * 4 * kQ;
+        float lam = 0.0f, beta = 0.0f;
+        if (t0 + row < a.L) {
+            const float Ah = ad[i];
+            lam = dts[i * kQ + row] * Ah;
+            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+        }
+        const float lt = wg0_inclusive_sum(lam, tmp);
+        l2s[row] = lt * kLog2e;
+        betas[row] = beta;
+        wg0_bar();
+#pragma unroll
+        for (int k = row; k < 4 * kQ; k += kQ) {
+            const int w = k >> 7, s = k & 127;
+            if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]) * betas[s];
+        }
+    };
+
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2));
+        for (int j = 0; j < kKD / 64; ++j) {
+            tma_load_4d(sm + SM::kQt + j * kQ * 128, &mC, &bar[0], 64 * j, g, t0, b);
+            tma_load_4d(sm + SM::kKt + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
+        }
+        load_xdy(0, hfirst);
+        load_sg(hfirst);
+    }
+    if (wg == 0) {
+        load_dts(a, dts, ad, b, t0, hfirst, nh, row);
+        wg0_bar();
+        decays(0);
+    }
     bool ok = true;
+    if (tid == 0) {
+        ok = mbar_wait(&bar[0], 0, a.hdr, 721) && mbar_wait(&bar[1], 0, a.hdr, 722);
+        if (ok) {
+            tc::fence_after_sync();
+            phase_a(0);
+        }
+        tc::commit(&bar[3]);
+    }
 
     for (int i = 0; i < nh; ++i) {
         const int h = hfirst + i, r = i & 1, pr = r ^ 1;
@@ -718,48 +789,17 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         char* Ot = region(r) + kQ * kP * 2;
         char* Pdt = region(pr);
         const uint32_t sX = smem_u32(Xt), sO = smem_u32(Ot), sPd = smem_u32(Pdt);
-        // ------------------------------------------------------------ prep(i)
-        if (i > 0) {
-            ok = ok && mbar_wait(&bar[5], (uint32_t)((i - 1) & 1), a.hdr, 720);
-            tc::fence_after_sync();
-            if (tid == 0) load_sg(h);  // the S_in / G tiles are free again
-        }
-        const float dt_raw = wg == 0 ? dts[i * kQ + row] : 0.0f;
-        float lam = 0.0f, beta = 0.0f;
-        if (wg == 0 && t0 + row < a.L) {
-            const float Ah = ad[i];
-            lam = dt_raw * Ah;
-            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
-        }
-        if (wg == 0) {
-            const float lt = wg0_inclusive_sum(lam, tmp);
-            l2s[row] = lt * kLog2e;
-            betas[row] = beta;
-        }
-        if (tid == 0) {
-            if (i == 0) ok = ok && mbar_wait(&bar[0], 0, a.hdr, 721);
-            bulk_wait_read_all();  // the previous head's dx store has left the P tile
-        }
-        ok = ok && mbar_wait(&bar[1 + r], (uint32_t)((i >> 1) & 1), a.hdr, 722);  // x, dy (read by E2 too)
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0 && ok) {  // phase A
-            tc::fence_after_sync();
-            tc::mma_tiles(tmem + kGM, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);   // M  = C B^T
-            tc::mma_tiles(tmem + kGS2, sO, 0, kQ, sX, 0, kQ, kQ, kQ, kP, 0);   // S2 = dy x^T
-            tc::commit(&bar[3]);
-        }
-        // column factors cf[w][s] = e^{l_{32 w} - l_s} beta_s (s < 32 w), two per thread
-#pragma unroll
-        for (int k = tid; k < 4 * kQ; k += 256) {
-            const int w = k >> 7, s = k & 127;
-            if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]) * betas[s];
-        }
-        __syncthreads();
-        // ------------------------------------------------------------ E1(i)
-        ok = ok && mbar_wait(&bar[3], (uint32_t)(i & 1), a.hdr, 723);
+        const float* l2s = l2all + r * kQ;
+        const float* betas = betall + r * kQ;
+        const float* cf = cfall + r * 4 * kQ;
+        // ---- phase A of head i and batch 2 of head i - 1 complete: S_in, G and Pd's region are free
+        ok = ok && mbar_wait(&bar[3], (uint32_t)(i & 1), a.hdr, 720);
+        ok = ok && mbar_wait(&bar[1 + r], (uint32_t)((i >> 1) & 1), a.hdr, 727);  // x, dy (read by E2)
         tc::fence_after_sync();
+        if (tid == 0 && i > 0) load_sg(h);
+        if (tid == kIssuer) bulk_wait_read_all();  // the previous head's dx store has left the P tile
+        __syncthreads();
+        // ---- E1
         {
             const float l2r = l2s[row];
             const float rf = ex2(l2r - l2s[32 * wq]);
@@ -851,24 +891,26 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         fence_proxy_async_smem();
         tc::fence_before_sync();
         __syncthreads();
-        if (tid == 0 && ok) {  // batch 1
+        // ---- batch 1: the dC / dB terms first (they free Pd's region), then dV1, B G, C S_in
+        if (tid == kIssuer && ok) {
             tc::fence_after_sync();
             const uint32_t acc = i > 0 ? 1u : 0u;
             tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
             tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
+            tc::commit(&bar[5]);
             tc::mma_tiles(tmem + kGdV, sP, 1, kQ, sO, 1, kQ, kQ, kP, kQ, 0);      // dV1 = P^T dy
             if (has_out) tc::mma_tiles(tmem + kGBG, sK, 0, kQ, sG, 1, kKD, kQ, kP, kKD, 0);  // B G
             if (has_in) tc::mma_tiles(tmem + kGY2, sQ, 0, kQ, sS, 1, kKD, kQ, kP, kKD, 0);   // C S_in
             tc::commit(&bar[4]);
         }
+        if (wg == 0 && i + 1 < nh) decays(i + 1);
+        if (tid == kIssuer && ok && i + 1 < nh) {  // Pd consumed: its region takes {x, dy} of head i + 1
+            ok = mbar_wait(&bar[5], (uint32_t)(i & 1), a.hdr, 728);
+            load_xdy(pr, h + 1);
+        }
         ok = ok && mbar_wait(&bar[4], (uint32_t)(i & 1), a.hdr, 724);
         tc::fence_after_sync();
-        if (tid == 0 && ok && i + 1 < nh) {  // Pd is consumed: its region takes {x, dy} of head i + 1
-            mbar_arrive_expect_tx(&bar[1 + pr], (uint32_t)(2 * kQ * kP * 2));
-            tma_load_4d(region(pr), &mX, &bar[1 + pr], 0, h + 1, t0, b);
-            tma_load_4d(region(pr) + kQ * kP * 2, &mdY, &bar[1 + pr], 0, h + 1, t0, b);
-        }
-        // ------------------------------------------------------------ E2(i)
+        // ---- E2
         {
             const float l2r = l2s[row];
             const float E = ex2(l2r);
@@ -925,15 +967,22 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         fence_proxy_async_smem();
         tc::fence_before_sync();
         __syncthreads();
-        if (tid == 0 && ok) {  // batch 2, then the dx store
-            tc::fence_after_sync();
-            if (has_in) tc::mma_tiles(tmem + kGdC, sO, 0, kQ, sS, 0, kKD, kQ, kKD, kP, 1);   // dC += (E dy) S_in^T
-            if (has_out) tc::mma_tiles(tmem + kGdB, sX, 0, kQ, sG, 0, kKD, kQ, kKD, kP, 1);  // dB += (w x) G^T
-            tc::commit(&bar[5]);
-            tma_store_4d(&mdX, sm + SM::kPt, 0, h, t0, b);
-            bulk_commit();
+        // ---- batch 2, the dx store, phase A of head i + 1 (one commit for all products)
+        if (tid == kIssuer) {
+            if (ok) {
+                tc::fence_after_sync();
+                if (has_in) tc::mma_tiles(tmem + kGdC, sO, 0, kQ, sS, 0, kKD, kQ, kKD, kP, 1);   // dC += (E dy) S_in^T
+                if (has_out) tc::mma_tiles(tmem + kGdB, sX, 0, kQ, sG, 0, kKD, kQ, kKD, kP, 1);  // dB += (w x) G^T
+                tma_store_4d(&mdX, sm + SM::kPt, 0, h, t0, b);
+                bulk_commit();
+                if (i + 1 < nh) {
+                    ok = mbar_wait(&bar[1 + pr], (uint32_t)(((i + 1) >> 1) & 1), a.hdr, 729);
+                    if (ok) phase_a(i + 1);
+                }
+            }
+            tc::commit(&bar[3]);
         }
-        // ------------------------------------------------------------ d dt, dA, dD (warpgroup 0)
+        // ---- d dt, dA, dD of head i (warpgroup 0)
         if (wg == 0) {
             const int t = row;
             const bool valid = t0 + t < a.L;
@@ -942,36 +991,34 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             const float qi = qdqp[t] + qdqp[kQ + t];
             const float ki = kdkp[t] + kdkp[kQ + t];
             const float ddv = ddp[t] + ddp[kQ + t];
-            const float kisum = wg0_sum(ki, tmp);
-            const float gs = wg0_sum(gsp[t] + gsp[kQ + t], tmp);
-            const float X = ex2(l2s[kQ - 1]) * gs + kisum;
+            const float2 kg = wg0_sum2(ki, gsp[t] + gsp[kQ + t], tmp);  // sum_s w x . BG, <G, S_in>
+            const float X = ex2(l2s[kQ - 1]) * kg.y + kg.x;
             float dl = rs + qi - cs - ki + (t == kQ - 1 ? X : 0.0f);
             if (!valid) dl = 0.0f;
-            const float incl = wg0_inclusive_sum(dl, tmp);
-            if (t == kQ - 1) tmp[16] = incl;
-            wg0_bar();
-            const float dlam = tmp[16] - incl + dl;
+            float total;
+            const float incl = wg0_inclusive_sum(dl, tmp, &total);
+            const float dlam = total - incl + dl;
             float dA_part = 0.0f;
             if (valid) {
                 const float Ah = ad[i];
                 const float bt = betas[t];
+                const float dt_raw = dts[i * kQ + t];
                 const float ab = ex2(dt_raw * Ah * kLog2e);
                 const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
                 ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(dlam * Ah + dbeta * ab);
                 dA_part = dlam * dt_raw + dbeta * (dt_raw * ab - bt) / Ah;
             }
-            const float sA = wg0_sum(dA_part, tmp);
-            const float sD = wg0_sum(valid ? ddv : 0.0f, tmp);
+            const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
             if (t == 0) {
                 const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
-                ga.pdA[tile] = sA;
-                ga.pdD[tile] = sD;
+                ga.pdA[tile] = sAD.x;
+                ga.pdD[tile] = sAD.y;
             }
         }
     }
     // dC, dB of this (batch row, chunk, group): rows t, columns [64 wg, 64 wg + 64).  Every lane
     // takes part in the (warp-collective) TMEM loads; rows past L are not stored.
-    ok = ok && mbar_wait(&bar[5], (uint32_t)((nh - 1) & 1), a.hdr, 725);
+    ok = ok && mbar_wait(&bar[3], (uint32_t)(nh & 1), a.hdr, 725);
     tc::fence_after_sync();
     {
         const bool vrow = t0 + row < a.L;
@@ -997,7 +1044,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             }
         }
     }
-    if (tid == 0) bulk_wait_all();
+    if (tid == kIssuer) bulk_wait_all();
     tc::fence_before_sync();
     __syncthreads();
     if (tid < 32) {
@@ -1096,8 +1143,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     const int nblk_o = (a.HpG + hb - 1) / hb;
     cudaFuncSetAttribute(ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
-    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, kThreads, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, stiles, hb,
-                                                                                      nblk_o);
+    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, 256, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, stiles, hb, nblk_o);
     return check_launch();
 }
 

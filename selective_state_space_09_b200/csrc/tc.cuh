@@ -114,22 +114,28 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Descriptor of an SW128 tile at the start of a product: the start address advances by a
+// compile-time number of 16-byte units per K = 16 step, so the per-step descriptor is the base
+// descriptor plus a small constant (the address field is the low 14 bits and never carries:
+// shared memory ends below 256 KB).
+//   K-major (mn = 0): +32 bytes per step inside a 64-wide block, +rows * 128 bytes per block;
+//   MN-major (mn = 1): +16 rows = 2048 bytes per step.
+__device__ __forceinline__ uint64_t tile_desc(uint32_t base, int mn, int rows) {
+    return desc_sw128(base, mn ? (uint32_t)rows * 128u : 16u, 1024);
+}
+__device__ __forceinline__ uint32_t tile_step(int k, int mn, int rows) {
+    return mn ? (uint32_t)k * 8u : (uint32_t)(k >> 6) * (uint32_t)rows * 8u + (uint32_t)((k & 63) >> 3);
+}
+
 // M = 128 x N x K product with A in tensor memory (a_tmem: K/2 columns) and B an SW128 tile.
 __device__ __forceinline__ void mma_ts_tiles(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int b_mn, int b_rows,
                                              int N, int K, uint32_t accumulate_first) {
     const uint32_t idesc = idesc_bf16(128, N, 0, b_mn);
-    for (int k = 0; k < K; k += 16) {
-        uint32_t b_addr, b_lbo;
-        if (b_mn) {
-            b_addr = b_base + (uint32_t)k * 128u;
-            b_lbo = (uint32_t)b_rows * 128u;
-        } else {
-            b_addr = b_base + (uint32_t)(k >> 6) * b_rows * 128u + (uint32_t)(k & 63) * 2u;
-            b_lbo = 16;
-        }
-        mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), desc_sw128(b_addr, b_lbo, 1024), idesc,
+    const uint64_t b0 = tile_desc(b_base, b_mn, b_rows);
+#pragma unroll
+    for (int k = 0; k < K; k += 16)
+        mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), b0 + tile_step(k, b_mn, b_rows), idesc,
                (k > 0 || accumulate_first) ? 1u : 0u);
-    }
 }
 
 // Issue an M x N x K product as K/16 MMAs over SW128 tiles.
@@ -140,25 +146,11 @@ __device__ __forceinline__ void mma_tiles(uint32_t d_tmem, uint32_t a_base, int 
                                           uint32_t b_base, int b_mn, int b_rows, int M, int N, int K,
                                           uint32_t accumulate_first) {
     const uint32_t idesc = idesc_bf16(M, N, a_mn, b_mn);
-    for (int k = 0; k < K; k += 16) {
-        uint32_t a_addr, b_addr, a_lbo, b_lbo;
-        if (a_mn) {  // K runs along rows: 16 rows = 2048 bytes
-            a_addr = a_base + (uint32_t)k * 128u;
-            a_lbo = (uint32_t)a_rows * 128u;
-        } else {     // K runs along columns: block k/64, 32 bytes per 16 inside the row
-            a_addr = a_base + (uint32_t)(k >> 6) * a_rows * 128u + (uint32_t)(k & 63) * 2u;
-            a_lbo = 16;
-        }
-        if (b_mn) {
-            b_addr = b_base + (uint32_t)k * 128u;
-            b_lbo = (uint32_t)b_rows * 128u;
-        } else {
-            b_addr = b_base + (uint32_t)(k >> 6) * b_rows * 128u + (uint32_t)(k & 63) * 2u;
-            b_lbo = 16;
-        }
-        mma(d_tmem, desc_sw128(a_addr, a_lbo, 1024), desc_sw128(b_addr, b_lbo, 1024), idesc,
+    const uint64_t a0 = tile_desc(a_base, a_mn, a_rows), b0 = tile_desc(b_base, b_mn, b_rows);
+#pragma unroll
+    for (int k = 0; k < K; k += 16)
+        mma(d_tmem, a0 + tile_step(k, a_mn, a_rows), b0 + tile_step(k, b_mn, b_rows), idesc,
             (k > 0 || accumulate_first) ? 1u : 0u);
-    }
 }
 
 }  // namespace tc

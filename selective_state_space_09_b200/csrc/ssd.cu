@@ -568,6 +568,7 @@ struct SsdGradArgs {
     const char* gtiles;    // [nchunk][B][H] bf16 tiles: adjoint of each chunk's outgoing state
     const char* stiles;    // [nchunk][B][H] bf16 tiles: state entering each chunk
     __nv_bfloat16* ddt;    // [B, L, H]
+    __nv_bfloat16* dx;     // [B, L, H, P]
     float* dB;             // [B, L, G, N]
     float* dC;
     float* pdA;            // [B][H][nchunk] per-chunk partials of dA_h, dD_h
@@ -578,9 +579,8 @@ struct SsdGradArgs {
 struct GradSmem {
     static constexpr size_t kQt = 0;                       // C tile 128 x 128 bf16
     static constexpr size_t kKt = kQt + kQ * kKD * 2;      // B tile
-    static constexpr size_t kReg = kKt + kQ * kKD * 2;     // two 32 KB regions: {x, dy} of a head or Pd
-    static constexpr size_t kPt = kReg + 2 * kQ * kQ * 2;  // P, then the dx staging tile
-    static constexpr size_t kSt = kPt + kQ * kQ * 2;       // S_in bf16 [n][p]
+    static constexpr size_t kReg = kKt + kQ * kKD * 2;     // three 32 KB slots: {x, dy}, P, Pd (rotating)
+    static constexpr size_t kSt = kReg + 3 * kQ * kQ * 2;  // S_in bf16 [n][p]
     static constexpr size_t kGt = kSt + kKD * kP * 2;      // G bf16 [n][p]
     static constexpr size_t kDt = kGt + kKD * kP * 2;      // dt of every head [kMaxHB][128] f32
     static constexpr size_t kAD = kDt + kMaxHB * kQ * 4;   // A, D of every head [2][kMaxHB]
@@ -594,7 +594,7 @@ struct GradSmem {
     static constexpr size_t kDd = kKdk + 2 * kQ * 4;       // dy . x [2][128]
     static constexpr size_t kGs = kDd + 2 * kQ * 4;        // <G, S_in> partials [256]
     static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
-    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 regions, 3 phase A (+ batch 2), 4 batch 1 (dV1, BG, Y2), 5 batch 1 (dC, dB), 6 S_in/G
+    static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 + 7 slots, 3 phase A (+ batch 2), 4 batch 1 (dV1, BG, Y2), 5 batch 1 (dC, dB), 6 S_in/G
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
@@ -609,6 +609,9 @@ __device__ __forceinline__ void wg0_bar() { asm volatile("bar.sync 1, 128;" ::: 
 // they run, and an issuing thread blocks while the tensor pipe is full, so warpgroup 0 stays free
 // to prepare the next head's decays and to reduce the current head's row terms.
 constexpr int kIssuer = 128;
+// Thread (another warp of warpgroup 1) that loads {x, dy} of the next head as soon as batch 1a has
+// consumed P, while the issuing thread may still be blocked issuing batch 1b.
+constexpr int kLoader = 160;
 
 // Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum);
 // *total receives the sum of all 128 values.
@@ -665,8 +668,8 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 //     (M = C B^T, S2 = dy x^T) while warpgroup 0 turns head i's row terms into d dt.
 __global__ void __launch_bounds__(256, 1)
 ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
-                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
-                const __grid_constant__ CUtensorMap mdX, SsdGradArgs ga, int hb, int nblk) {
+                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY, SsdGradArgs ga,
+                int hb, int nblk) {
     using SM = GradSmem;
     const SsdArgs& a = ga.a;
     char* sm = smem_base1024();
@@ -684,8 +687,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
     float* dts = reinterpret_cast<float*>(sm + SM::kDt);
     float* ad = reinterpret_cast<float*>(sm + SM::kAD);
-    const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sP = smem_u32(sm + SM::kPt),
-                   sS = smem_u32(sm + SM::kSt), sG = smem_u32(sm + SM::kGt);
+    const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sS = smem_u32(sm + SM::kSt),
+                   sG = smem_u32(sm + SM::kGt);
     const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
     const int row = tid & 127;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -703,7 +706,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -712,11 +715,15 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Three 32 KB slots rotate per head i: {x, dy} in slot i % 3, P in (i + 1) % 3, Pd in (i + 2) % 3.
+    // P is consumed first (batch 1a), so its slot takes {x, dy} of head i + 1; Pd's slot takes P of
+    // head i + 1 and the {x, dy} slot (free after batch 2) Pd of head i + 1.
     auto region = [&](int r) { return sm + SM::kReg + (size_t)r * kQ * kQ * 2; };
-    auto load_xdy = [&](int r, int h) {  // {x, dy} of head h into region r
-        mbar_arrive_expect_tx(&bar[1 + r], (uint32_t)(2 * kQ * kP * 2));
-        tma_load_4d(region(r), &mX, &bar[1 + r], 0, h, t0, b);
-        tma_load_4d(region(r) + kQ * kP * 2, &mdY, &bar[1 + r], 0, h, t0, b);
+    auto slot_bar = [&](int r) { return r < 2 ? &bar[1 + r] : &bar[7]; };
+    auto load_xdy = [&](int r, int h) {  // {x, dy} of head h into slot r
+        mbar_arrive_expect_tx(slot_bar(r), (uint32_t)(2 * kQ * kP * 2));
+        tma_load_4d(region(r), &mX, slot_bar(r), 0, h, t0, b);
+        tma_load_4d(region(r) + kQ * kP * 2, &mdY, slot_bar(r), 0, h, t0, b);
     };
     // S_in and G tiles of head h (bulk copies; the phase completes also when neither exists)
     auto load_sg = [&](int h) {
@@ -732,7 +739,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     };
     // phase A of head i ({x, dy} in region i & 1): M = C B^T, S2 = dy x^T
     auto phase_a = [&](int i) {
-        const uint32_t sXi = smem_u32(region(i & 1)), sOi = sXi + kQ * kP * 2;
+        const uint32_t sXi = smem_u32(region(i % 3)), sOi = sXi + kQ * kP * 2;
         tc::mma_tiles(tmem + kGM, sQ, 0, kQ, sK, 0, kQ, kQ, kQ, kKD, 0);
         tc::mma_tiles(tmem + kGS2, sOi, 0, kQ, sXi, 0, kQ, kQ, kQ, kP, 0);
     };
@@ -784,20 +791,20 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     }
 
     for (int i = 0; i < nh; ++i) {
-        const int h = hfirst + i, r = i & 1, pr = r ^ 1;
-        char* Xt = region(r);
-        char* Ot = region(r) + kQ * kP * 2;
-        char* Pdt = region(pr);
-        const uint32_t sX = smem_u32(Xt), sO = smem_u32(Ot), sPd = smem_u32(Pdt);
+        const int h = hfirst + i, r = i & 1, xs = i % 3, ps = (i + 1) % 3, ds = (i + 2) % 3;
+        char* Xt = region(xs);
+        char* Ot = region(xs) + kQ * kP * 2;
+        char* Pt = region(ps);
+        char* Pdt = region(ds);
+        const uint32_t sX = smem_u32(Xt), sO = smem_u32(Ot), sP = smem_u32(Pt), sPd = smem_u32(Pdt);
         const float* l2s = l2all + r * kQ;
         const float* betas = betall + r * kQ;
         const float* cf = cfall + r * 4 * kQ;
         // ---- phase A of head i and batch 2 of head i - 1 complete: S_in, G and Pd's region are free
         ok = ok && mbar_wait(&bar[3], (uint32_t)(i & 1), a.hdr, 720);
-        ok = ok && mbar_wait(&bar[1 + r], (uint32_t)((i >> 1) & 1), a.hdr, 727);  // x, dy (read by E2)
+        ok = ok && mbar_wait(slot_bar(xs), (uint32_t)((i / 3) & 1), a.hdr, 727);  // x, dy (read by E2)
         tc::fence_after_sync();
         if (tid == 0 && i > 0) load_sg(h);
-        if (tid == kIssuer) bulk_wait_read_all();  // the previous head's dx store has left the P tile
         __syncthreads();
         // ---- E1
         {
@@ -811,7 +818,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int k = 0; k < 32; k += 8) {
-                        *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, s0 + k, kQ)) = z;
+                        *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = z;
                         *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = z;
                     }
                     colp[wq * kQ + s0 + lane] = 0.0f;
@@ -847,7 +854,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 }
 #pragma unroll
                 for (int k = 0; k < 32; k += 8) {
-                    *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, s0 + k, kQ)) = pack8(m + k);
+                    *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = pack8(m + k);
                     *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = pack8(s2 + k);
                 }
 #pragma unroll
@@ -891,31 +898,30 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         fence_proxy_async_smem();
         tc::fence_before_sync();
         __syncthreads();
-        // ---- batch 1: the dC / dB terms first (they free Pd's region), then dV1, B G, C S_in
+        // ---- batch 1: dV1, B G, C S_in first (E2 needs them; P's slot then takes {x, dy} of head
+        // i + 1), then the dC / dB terms, which run while E2 works
         if (tid == kIssuer && ok) {
             tc::fence_after_sync();
             const uint32_t acc = i > 0 ? 1u : 0u;
-            tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
-            tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
-            tc::commit(&bar[5]);
             tc::mma_tiles(tmem + kGdV, sP, 1, kQ, sO, 1, kQ, kQ, kP, kQ, 0);      // dV1 = P^T dy
             if (has_out) tc::mma_tiles(tmem + kGBG, sK, 0, kQ, sG, 1, kKD, kQ, kP, kKD, 0);  // B G
             if (has_in) tc::mma_tiles(tmem + kGY2, sQ, 0, kQ, sS, 1, kKD, kQ, kP, kKD, 0);   // C S_in
             tc::commit(&bar[4]);
+            tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
+            tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
+            tc::commit(&bar[5]);
         }
         if (wg == 0 && i + 1 < nh) decays(i + 1);
-        if (tid == kIssuer && ok && i + 1 < nh) {  // Pd consumed: its region takes {x, dy} of head i + 1
-            ok = mbar_wait(&bar[5], (uint32_t)(i & 1), a.hdr, 728);
-            load_xdy(pr, h + 1);
-        }
         ok = ok && mbar_wait(&bar[4], (uint32_t)(i & 1), a.hdr, 724);
         tc::fence_after_sync();
+        if (tid == kLoader && ok && i + 1 < nh) load_xdy(ps, h + 1);  // P consumed
         // ---- E2
         {
             const float l2r = l2s[row];
             const float E = ex2(l2r);
             const float w = ex2(l2s[kQ - 1] - l2r) * betas[row];
             const float Dh = ad[kMaxHB + i];
+            __nv_bfloat16* dxrow = ga.dx + (((size_t)b * a.L + min(t0 + row, a.L - 1)) * a.H + h) * kP;
             float qdq = 0.0f, kdk = 0.0f, dd = 0.0f;
 #pragma unroll
             for (int v0 = 0; v0 < 32; v0 += 16) {
@@ -955,7 +961,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                         xs[e] *= w;
                         os[e] *= E;
                     }
-                    *reinterpret_cast<uint4*>(sm + SM::kPt + tc::sw128_off(row, col + hh, kQ)) = pack8(dx);
+                    if (t0 + row < a.L) *reinterpret_cast<uint4*>(dxrow + col + hh) = pack8(dx);
                     *px = pack8(xs);
                     *po = pack8(os);
                 }
@@ -973,10 +979,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 tc::fence_after_sync();
                 if (has_in) tc::mma_tiles(tmem + kGdC, sO, 0, kQ, sS, 0, kKD, kQ, kKD, kP, 1);   // dC += (E dy) S_in^T
                 if (has_out) tc::mma_tiles(tmem + kGdB, sX, 0, kQ, sG, 0, kKD, kQ, kKD, kP, 1);  // dB += (w x) G^T
-                tma_store_4d(&mdX, sm + SM::kPt, 0, h, t0, b);
-                bulk_commit();
                 if (i + 1 < nh) {
-                    ok = mbar_wait(&bar[1 + pr], (uint32_t)(((i + 1) >> 1) & 1), a.hdr, 729);
+                    ok = mbar_wait(slot_bar(ps), (uint32_t)(((i + 1) / 3) & 1), a.hdr, 729);
                     if (ok) phase_a(i + 1);
                 }
             }
@@ -1044,7 +1048,6 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             }
         }
     }
-    if (tid == kIssuer) bulk_wait_all();
     tc::fence_before_sync();
     __syncthreads();
     if (tid < 32) {
@@ -1159,14 +1162,14 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.gtiles = ws + w.gtiles;
     ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     ga.ddt = (__nv_bfloat16*)gr.ddelta;
+    ga.dx = (__nv_bfloat16*)gr.dx;
     ga.dB = gr.dBm;
     ga.dC = gr.dCm;
     ga.pdA = (float*)(ws + w.pdA);
     ga.pdD = (float*)(ws + w.pdD);
-    CUtensorMap mC, mB, mX, mdY, mdX;
+    CUtensorMap mC, mB, mX, mdY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
-              map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true) &&
-              map4(&mdX, gr.dx, kP, d.H, d.L, d.B, true);
+              map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true);
     if (!ok) return LR_ERR_INVALID_ARG;
     float* Ubuf = (float*)(ws + w.U);
     const int nblk_s = (a.HpG + kHS - 1) / kHS;
@@ -1199,7 +1202,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     }
     cudaFuncSetAttribute(ssd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
     note_launch("ssd_chunk_grad");
-    ssd_grad_kernel<<<a.nchunk * a.B * a.G * nblk, 256, GradSmem::kAlloc, st>>>(mC, mB, mX, mdY, mdX, ga, hb, nblk);
+    ssd_grad_kernel<<<a.nchunk * a.B * a.G * nblk, 256, GradSmem::kAlloc, st>>>(mC, mB, mX, mdY, ga, hb, nblk);
     lr_status s = check_launch();
     if (s != LR_OK) return s;
     note_launch("ssd_param_reduce");

@@ -177,6 +177,14 @@ lr_status lr_get_error(void *ws, void *stream, int32_t *info);
 /* Static, human-readable name of a status. */
 const char *lr_status_string(lr_status s);
 
+/* Timing hook (benchmarks).  While set, on this host thread, every kernel launch of an
+ * lr_scan_fwd / lr_scan_bwd call first records events[k] on the call's stream, k = 0, 1, ...
+ * counting the launches of that call (launches past n record nothing).  Kernel k then runs between
+ * events[k] and events[k + 1] (the last one until whatever the caller records after the call).
+ * events: n cudaEvent_t handles passed as void*, owned by the caller; NULL or n = 0 turns the
+ * hook off.  Records only; never synchronises. */
+void lr_set_launch_events(void *const *events, int n);
+
 /* Names of the kernels the last lr_scan_fwd / lr_scan_bwd call on this host thread launched,
  * separated by '+' (a fingerprint that lets tests check which code path ran). */
 const char *lr_last_dispatch(void);

@@ -15,6 +15,9 @@ namespace lrs {
 namespace {
 thread_local std::string t_dispatch;
 thread_local int t_launches = 0;
+thread_local void* const* t_events = nullptr;  // lr_set_launch_events
+thread_local int t_nevents = 0;
+thread_local cudaStream_t t_stream = nullptr;  // stream of the current entry-point call
 
 int esize(int io) { return io == LR_BF16 ? 2 : 4; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -102,8 +105,12 @@ void reset_dispatch() { begin_call(); }
 void note_launch(const char* name) {
     if (!t_dispatch.empty()) t_dispatch += "+";
     t_dispatch += name;
+    if (t_events && t_launches < t_nevents && t_events[t_launches])
+        cudaEventRecord(static_cast<cudaEvent_t>(t_events[t_launches]), t_stream);
     ++t_launches;
 }
+
+void set_launch_stream(cudaStream_t st) { t_stream = st; }
 
 lr_status check_launch() {
     cudaError_t e = cudaGetLastError();
@@ -210,6 +217,7 @@ lr_status lr_scan_fwd(const lr_desc* desc, const lr_inputs* in, void* y, void* c
     if (!aligned16(y) || !aligned16(ckpt) || !aligned16(ws)) return LR_ERR_ALIGNMENT;
     if (ws_size < ws_bytes(d, false)) return LR_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    set_launch_stream(st);
     if (cudaMemsetAsync(ws, 0, flag_bytes(d, false), st) != cudaSuccess) return LR_ERR_CUDA;
     switch (d.kind) {
         case LR_RGLRU:
@@ -252,6 +260,7 @@ lr_status lr_scan_bwd(const lr_desc* desc, const lr_inputs* in, const void* dy, 
     if (!aligned16(dy) || !aligned16(ckpt) || !aligned16(ws)) return LR_ERR_ALIGNMENT;
     if (ws_size < ws_bytes(d, true)) return LR_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    set_launch_stream(st);
     if (cudaMemsetAsync(ws, 0, flag_bytes(d, true), st) != cudaSuccess) return LR_ERR_CUDA;
     switch (d.kind) {
         case LR_RGLRU:
@@ -289,5 +298,10 @@ const char* lr_status_string(lr_status s) {
 const char* lr_last_dispatch(void) { return t_dispatch.c_str(); }
 
 int lr_last_launch_count(void) { return t_launches; }
+
+void lr_set_launch_events(void* const* events, int n) {
+    t_events = (events && n > 0) ? events : nullptr;
+    t_nevents = t_events ? n : 0;
+}
 
 }  // extern "C"

@@ -167,6 +167,16 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the previous kernel of
+// the stream is still running.  pdl_launch_dependents lets the next kernel start its independent
+// prologue; pdl_wait blocks the calling thread until the previous kernel has completed and its
+// writes are visible (it returns at once when there is no such kernel).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------- cross-CTA flag protocol
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
     unsigned int v;

@@ -20,6 +20,9 @@ void note_launch(const char* name);
 // Clears this host thread's launch fingerprint (start of an entry-point call).
 void reset_dispatch();
 
+// Stream of the current entry-point call (where the timing hook records its events).
+void set_launch_stream(cudaStream_t st);
+
 // Converts the last CUDA error into a status.
 lr_status check_launch();
 
@@ -34,6 +37,25 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int esize, uint64_t d0, ui
 // esize must then be 128).  Returns false if the driver rejects the description.
 bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const uint64_t* dims,
                const uint64_t* strides, const uint32_t* box, bool swizzle128);
+
+// Launches `kernel` on `st` with programmatic stream serialization: it may start while the
+// previous kernel of the stream runs and must call pdl_wait before touching that kernel's outputs
+// (or anything it reads).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Byte offset bookkeeping for a workspace: a 256-byte header followed by regions.
 struct WsCursor {

@@ -66,6 +66,7 @@ extern "C" lr_status lr_rglru_fwd_noalloc(const lr_desc* desc, const void* a, co
     s = scratch_address(&ws);
     if (s != LR_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    set_launch_stream(st);
     if (cudaMemsetAsync(ws, 0, diag_flag_bytes(*desc, false), st) != cudaSuccess) return LR_ERR_CUDA;
     lr_inputs in{};
     in.a = a;

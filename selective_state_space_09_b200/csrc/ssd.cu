@@ -89,6 +89,7 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
     const int t0 = c * kQ;
     const int hfirst = g * a.HpG + blk * kHS;
     const int nh = min(kHS, a.HpG - blk * kHS);
+    pdl_launch_dependents();
 
     if (tid == 0) {
         mbar_init(&bar[0], 1);
@@ -113,6 +114,7 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
         if (j < nh) ssd_coef(a, b, hfirst + j, t0 + tid, l[j], beta[j]);
     }
     cta_inclusive_sum_n<kHS>(l, tmp);
+    pdl_wait();  // the previous kernel of the stream may still read what this one writes
     if (tid == kQ - 1) {
 #pragma unroll
         for (int j = 0; j < kHS; ++j) tmp[16 + j] = l[j];
@@ -193,8 +195,16 @@ constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf1
 //            only as bf16 tiles.
 // Loads of eight slots are issued ahead of their dependent updates.
 __global__ void __launch_bounds__(256)
-ssd_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir) {
+ssd_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir,
+                float4* zero0, float4* zero1, size_t nzero4) {
+    pdl_launch_dependents();
+    pdl_wait();
     const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // zero0 / zero1 (the backward's dB, dC when several CTAs add into them): nzero4 float4 each
+    for (size_t z = e; z < nzero4; z += (size_t)gridDim.x * blockDim.x) {
+        zero0[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        zero1[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
     if (e >= (size_t)BH * n4) return;
     const size_t stride = (size_t)BH * n4;
     const int bh = (int)(e / n4), q = (int)(e % n4);
@@ -335,6 +345,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     const int nmine = (nh - wg + 1) / 2;  // heads wg, wg + 2, ...
     const bool has_in = c > 0;
     auto stile = [&](int h) { return stiles + (((size_t)c * a.B + b) * a.H + h) * kTileBytes; };
+    pdl_launch_dependents();
 
     if (tid == 0) {
         for (int i = 0; i < 12; ++i) mbar_init(&bar[i], 1);
@@ -358,6 +369,9 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             mbar_arrive_expect_tx(&wbar[u], (uint32_t)(kQ * kP * 2));
             tma_load_4d(Xs + u * kQ * 128, &mX, &wbar[u], 0, hfirst + wg + 2 * u, t0, b);
         }
+    }
+    pdl_wait();  // the S_in tiles come from the previous kernel
+    if (wt == 0) {
         if (has_in && nmine > 0) {
             mbar_arrive_expect_tx(&wbar[3], kTileBytes);
             bulk_load(St, stile(hfirst + wg), kTileBytes, &wbar[3]);
@@ -538,15 +552,41 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     return a;
 }
 
-// Heads per output CTA: the group's heads split into the fewest blocks that give at least one
-// CTA per SM, blocks of at most 16 heads (always 16 under LR_TEST_MAX_HEAD_BLOCK).
+// Number of SMs of the current device (queried once).
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+                                                          cudaSuccess && v > 0)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
+
+// Heads per output CTA (at most 16; 16 under LR_TEST_MAX_HEAD_BLOCK): the block size that
+// minimises waves x per-CTA time, a CTA taking about 2 units per head of each warpgroup (two
+// warpgroups alternate heads) plus 1 unit of prologue (C, B loads and C B^T).
 int out_heads_per_cta(const lr_desc& d, int nchunk) {
     const int HpG = (int)(d.H / d.G);
     const long units = (long)nchunk * d.B * d.G;
-    int hb = HpG < 16 ? HpG : 16;
-    if (d.flags & LR_TEST_MAX_HEAD_BLOCK) return hb;
-    while (hb > 1 && units * ((HpG + hb - 1) / hb) < 148) hb = (hb + 1) / 2;
-    return hb;
+    const int top = HpG < 16 ? HpG : 16;
+    if (d.flags & LR_TEST_MAX_HEAD_BLOCK) return top;
+    int best = top;
+    long best_cost = -1;
+    for (int hb = top; hb >= 1; hb = hb > 1 ? (hb + 1) / 2 : 0) {
+        const long ctas = units * ((HpG + hb - 1) / hb);
+        const long waves = (ctas + sm_count() - 1) / sm_count();
+        const long cost = waves * (2 * ((hb + 1) / 2) + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = hb;
+        }
+        if (hb == 1) break;
+    }
+    return best;
 }
 
 // =========================================================================================
@@ -704,6 +744,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     const int hfirst = g * a.HpG + blk * hb;
     const int nh = min(hb, a.HpG - blk * hb);
     const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
+    pdl_launch_dependents();
 
     if (tid == 0) {
         for (int i = 0; i < 8; ++i) mbar_init(&bar[i], 1);
@@ -773,8 +814,9 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             tma_load_4d(sm + SM::kKt + j * kQ * 128, &mB, &bar[0], 64 * j, g, t0, b);
         }
         load_xdy(0, hfirst);
-        load_sg(hfirst);
     }
+    pdl_wait();  // the G tiles (and the zeroed dB, dC) come from the previous kernel
+    if (tid == 0) load_sg(hfirst);
     if (wg == 0) {
         load_dts(a, dts, ad, b, t0, hfirst, nh, row);
         wg0_bar();
@@ -1060,6 +1102,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
 // head; lane-strided partial sums, then a fixed butterfly).
 __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __restrict__ pdD, int B, int H, int nchunk,
                               float* __restrict__ dA, float* __restrict__ dD) {
+    pdl_wait();
     const int h = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (h >= H) return;
@@ -1129,7 +1172,9 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
         cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
         note_launch("ssd_chunk_state");
         const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mB, mX, mS, a, nblk_s, +1);
+        cudaError_t e = launch_pdl(ssd_state_kernel, dim3(grid), dim3(kThreads), StateSmem::kAlloc, st, mB, mX, mS, a,
+                                   nblk_s, +1);
+        if (e != cudaSuccess) return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1137,8 +1182,10 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
         const int n4 = kKD * kP / 4;
         const size_t total = (size_t)a.B * a.H * n4;
         note_launch("ssd_state_pass");
-        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)ckpt, stiles, a.decay, a.B * a.H,
-                                                                         n4, a.nchunk, +1);
+        cudaError_t e = launch_pdl(ssd_pass_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
+                                   (float4*)ckpt, stiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, +1,
+                                   (float4*)nullptr, (float4*)nullptr, (size_t)0);
+        if (e != cudaSuccess) return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1146,7 +1193,9 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     const int nblk_o = (a.HpG + hb - 1) / hb;
     cudaFuncSetAttribute(ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
-    ssd_out_kernel<<<a.nchunk * a.B * a.G * nblk_o, 256, OutSmem::kAlloc, st>>>(mC, mB, mX, mY, a, stiles, hb, nblk_o);
+    if (launch_pdl(ssd_out_kernel, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
+                   a, (const char*)stiles, hb, nblk_o) != cudaSuccess)
+        return LR_ERR_CUDA;
     return check_launch();
 }
 
@@ -1179,35 +1228,38 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
         note_launch("ssd_chunk_state");
         const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        ssd_state_kernel<<<grid, kThreads, StateSmem::kAlloc, st>>>(mC, mdY, mU, a, nblk_s, -1);
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
-    {
-        const int n4 = kKD * kP / 4;
-        const size_t total = (size_t)a.B * a.H * n4;
-        note_launch("ssd_state_pass");
-        ssd_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((float4*)Ubuf, ws + w.gtiles, a.decay,
-                                                                         a.B * a.H, n4, a.nchunk, -1);
+        cudaError_t e = launch_pdl(ssd_state_kernel, dim3(grid), dim3(kThreads), StateSmem::kAlloc, st, mC, mdY, mU,
+                                   a, nblk_s, -1);
+        if (e != cudaSuccess) return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
     const int hb = grad_heads_per_cta(d, a.nchunk);
     const int nblk = (a.HpG + hb - 1) / hb;
-    ga.accumulate = nblk > 1 ? 1 : 0;
-    if (ga.accumulate) {
-        const size_t n = (size_t)d.B * d.L * d.G * kKD * sizeof(float);
-        if (cudaMemsetAsync(gr.dBm, 0, n, st) != cudaSuccess || cudaMemsetAsync(gr.dCm, 0, n, st) != cudaSuccess)
-            return LR_ERR_CUDA;
+    ga.accumulate = nblk > 1 ? 1 : 0;  // several head blocks add into dB, dC: the pass kernel zeroes them
+    {
+        const int n4 = kKD * kP / 4;
+        const size_t total = (size_t)a.B * a.H * n4;
+        const size_t nzero4 = ga.accumulate ? (size_t)d.B * d.L * d.G * kKD / 4 : 0;
+        note_launch("ssd_state_pass");
+        cudaError_t e = launch_pdl(ssd_pass_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
+                                   (float4*)Ubuf, ws + w.gtiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, -1,
+                                   (float4*)gr.dBm, (float4*)gr.dCm, nzero4);
+        if (e != cudaSuccess) return LR_ERR_CUDA;
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
     }
     cudaFuncSetAttribute(ssd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
     note_launch("ssd_chunk_grad");
-    ssd_grad_kernel<<<a.nchunk * a.B * a.G * nblk, 256, GradSmem::kAlloc, st>>>(mC, mB, mX, mdY, ga, hb, nblk);
+    if (launch_pdl(ssd_grad_kernel, dim3(a.nchunk * a.B * a.G * nblk), dim3(256), GradSmem::kAlloc, st, mC, mB, mX, mdY,
+                   ga, hb, nblk) != cudaSuccess)
+        return LR_ERR_CUDA;
     lr_status s = check_launch();
     if (s != LR_OK) return s;
     note_launch("ssd_param_reduce");
-    ssd_param_sum<<<(a.H + 7) / 8, 256, 0, st>>>(ga.pdA, ga.pdD, a.B, a.H, a.nchunk, gr.dA,
-                                                 (d.flags & LR_HAS_DSKIP) ? gr.dDskip : nullptr);
+    if (launch_pdl(ssd_param_sum, dim3((a.H + 7) / 8), dim3(256), 0, st, (const float*)ga.pdA, (const float*)ga.pdD,
+                   a.B, a.H, a.nchunk, gr.dA, (d.flags & LR_HAS_DSKIP) ? gr.dDskip : (float*)nullptr) != cudaSuccess)
+        return LR_ERR_CUDA;
     return check_launch();
 }
 

@@ -78,6 +78,8 @@ def _load():
     L.lr_status_string.restype = ctypes.c_char_p
     L.lr_last_dispatch.restype = ctypes.c_char_p
     L.lr_last_launch_count.restype = ctypes.c_int
+    L.lr_set_launch_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+    L.lr_set_launch_events.restype = None
     L.lr_version.restype = ctypes.c_int
     return L
 
@@ -117,6 +119,18 @@ def last_dispatch():
 
 def last_launch_count():
     return int(lib.lr_last_launch_count())
+
+
+def set_launch_events(events):
+    """Timing hook: each kernel launch of the following calls on this thread first records
+    events[k] (torch.cuda.Event, already created) on the call's stream; None turns it off."""
+    if not events:
+        lib.lr_set_launch_events(None, 0)
+        set_launch_events._keep = None
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    set_launch_events._keep = arr  # the library keeps the pointer until the hook is reset
+    lib.lr_set_launch_events(arr, len(events))
 
 
 def _check(status, where):

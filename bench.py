@@ -72,16 +72,16 @@ def src_sha():
     return h.hexdigest()[:12]
 
 
-def ncu_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+def ncu_traffic(kernel, pas=None):
+    """DRAM bytes per launch of `kernel` (of pass `pas` when the name occurs in both passes) from
+    the committed ncu summary, if it was taken on the current kernel sources (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
     except Exception:
         return None
-    e = d.get(kernel)
+    e = d.get("%s@%s" % (kernel, pas)) or d.get(kernel)
     if not e or e.get("src_sha") != src_sha():
         return None
     return e.get("bytes_per_launch")
@@ -580,7 +580,7 @@ def main():
     dom_row = max(h["kernels_timed"], key=lambda r: r["ms"])
     roofline = kernel_roofline(dom_row, pk)
     roofline.update({
-        "traffic": ncu_traffic(dom_row["kernel"]), "kernel": dom_row["kernel"], "pass": dom_row["pass"],
+        "traffic": ncu_traffic(dom_row["kernel"], dom_row["pass"]), "kernel": dom_row["kernel"], "pass": dom_row["pass"],
         "algorithmic_bytes_per_launch": dom_row["bytes"], "algorithmic_flops_per_launch": dom_row["flops"],
         "ms_per_launch": round(dom_row["ms"], 5),
         "note": "of %s peak (burst GEMM / copy); kernel time from CUDA events the library records "

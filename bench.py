@@ -212,11 +212,27 @@ def kernel_cost(w, name, pas, pass_bytes):
             per = 2 * Q * (Q * P + 2 * Q * N + Q * P + 2 * P * N + 2 * N * P)
             fl = head_chunks * per + nc * B * G * 2 * Q * Q * N
             return 3 * tok + 2 * bc + 2 * dt + 2 * nc * tile + 2 * B * L * G * N * 4, fl
-    if kind == "gla" and name.startswith("gla_"):
+    if kind == "gla":
         B, L, H, K, V = w["B"], w["L"], w["H"], w["K"], w["V"]
-        hc = -(-L // 128) * B * H
-        nprod = 4 if pas == "fwd" else 9
-        return pass_bytes, hc * nprod * 2 * 128 * 128 * max(K, V)
+        Q = 128
+        nc = -(-L // Q)
+        tk = B * L * H * K * 2             # q, k, dq, dk (bf16)
+        tv = B * L * H * V * 2             # v, o, dO, dv
+        g = B * L * H * 2
+        slot = B * H * K * V * 4
+        tile = B * H * K * V * 2
+        hc = nc * B * H
+        prod = 2 * Q * Q * max(K, V)       # one 128 x 128 x 128 product
+        if name == "gla_chunk_state":
+            return tk + tv + g + (nc - 1) * slot, (nc - 1) * B * H * 2 * K * V * Q
+        if name == "gla_state_pass":
+            if pas == "fwd":
+                return (nc - 1) * slot + nc * slot + nc * tile, 0
+            return (nc - 1) * slot + nc * tile, 0
+        if name == "gla_chunk_out":
+            return 2 * tk + 2 * tv + g + nc * tile, hc * 3 * prod
+        if name == "gla_chunk_grad":
+            return 4 * tk + 3 * tv + 2 * g + 2 * nc * tile, hc * 9 * prod
     return pass_bytes, 0
 
 

@@ -180,8 +180,8 @@ lr_status lr_validate(const lr_desc* desc) { return validate(desc); }
 size_t lr_ckpt_bytes(const lr_desc* desc) {
     if (validate(desc) != LR_OK) return 0;
     size_t nseg = (size_t)((desc->L + desc->segment - 1) / desc->segment);
-    // SSD: the f32 states are followed by a bf16 copy of each in tensor-core tile order
-    const size_t per = desc->kind == LR_SSD ? sizeof(float) + 2 : sizeof(float);
+    // SSD, GLA: the f32 states are followed by a bf16 copy of each in tensor-core tile order
+    const size_t per = (desc->kind == LR_SSD || desc->kind == LR_GLA) ? sizeof(float) + 2 : sizeof(float);
     return nseg * state_elems(*desc) * per;
 }
 

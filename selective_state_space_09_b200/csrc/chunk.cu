@@ -424,16 +424,19 @@ bool chunk_supported(const lr_desc& d) {
 size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only);
 size_t chunk_ws_bytes(const lr_desc& d, bool bwd) {
     if (d.kind == LR_SSD) return bwd ? ssd_bwd_ws_bytes(d) : ssd_fwd_ws_bytes(d);
+    if (d.kind == LR_GLA) return gla_ws_bytes(d, bwd);
     return bwd ? chunk_bwd_ws_end(d, false) : ws_plan(d).end;
 }
 size_t chunk_flag_bytes(const lr_desc& d, bool bwd) {
     if (d.kind == LR_SSD) return bwd ? ssd_bwd_flag_bytes(d) : ssd_fwd_flag_bytes(d);
+    if (d.kind == LR_GLA) return gla_flag_bytes(d, bwd);
     return bwd ? chunk_bwd_ws_end(d, true) : ws_plan(d).aggA;
 }
 
 lr_status chunk_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
                     cudaStream_t st) {
     if (d.kind == LR_SSD) return ssd_fwd(d, in, y, ckpt, ws, st);
+    if (d.kind == LR_GLA) return gla_fwd(d, in, y, ckpt, ws, st);
     ChunkWs w = ws_plan(d);
     ChunkArgs a{};
     a.kind = d.kind;
@@ -950,6 +953,7 @@ size_t chunk_bwd_ws_end(const lr_desc& d, bool flags_only) {
 lr_status chunk_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
                     const lr_grads& gr, char* ws, cudaStream_t st) {
     if (d.kind == LR_SSD) return ssd_bwd(d, in, dy, ckpt, gr, ws, st);
+    if (d.kind == LR_GLA) return gla_bwd(d, in, dy, ckpt, gr, ws, st);
     ChunkBwdWs w = bwd_plan(d);
     ChunkBwdArgs bw{};
     ChunkArgs& a = bw.f;

@@ -95,6 +95,11 @@ lr_status chunk_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const
 size_t ssd_fwd_ws_bytes(const lr_desc& d);
 size_t ssd_fwd_flag_bytes(const lr_desc& d);
 lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st);
+size_t gla_ws_bytes(const lr_desc& d, bool bwd);
+size_t gla_flag_bytes(const lr_desc& d, bool bwd);
+lr_status gla_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st);
+lr_status gla_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt, const lr_grads& gr,
+                  char* ws, cudaStream_t st);
 size_t ssd_bwd_ws_bytes(const lr_desc& d);
 size_t ssd_bwd_flag_bytes(const lr_desc& d);
 lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt, const lr_grads& gr,

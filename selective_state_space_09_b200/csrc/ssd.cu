@@ -16,7 +16,7 @@
 // Forward = three launches, none of which waits on another CTA:
 //   ssd_state_kernel  (batch row, chunk, block of 4 heads): Sl of every chunk but the last,
 //                     written into checkpoint slot c + 1; e^{l_Q} per chunk;
-//   ssd_pass_kernel   elementwise over (batch row, head, state element): slot c <- e^{l_Q, c-1}
+//   state_pass_kernel  elementwise over (batch row, head, state element): slot c <- e^{l_Q, c-1}
 //                     slot c-1 + Sl_{c-1}, in place, so slot c ends as the state entering chunk c;
 //   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x.
 #include "chunk_common.cuh"
@@ -26,6 +26,7 @@ using namespace chunkc;
 namespace {
 
 constexpr int kP = 64;    // head dimension (value columns)
+constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf16 SW128 tile
 constexpr int kHS = 2;    // heads per CTA of the state kernel
 
 struct SsdArgs {
@@ -180,63 +181,6 @@ ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__
     if (warp == 0) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 128);
-    }
-}
-
-// ---------------------------------------------------------------------------- state passing
-constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf16 SW128 tile
-
-// One thread per (b h, four consecutive state elements (n, p .. p+3)) of the f32 slots of `buf`
-// ([nchunk][B*H][N*P/4] float4), walking the chunks in order:
-//   dir > 0: slot 0 = 0; slot c = decay_{c-1} slot_{c-1} + slot_c (c = 1 .. nchunk-1), in place;
-//            every slot is also written as bf16 into `tiles` ([nchunk][B*H] tiles, tensor-core
-//            order), the B operand of C S_in in the output and gradient kernels;
-//   dir < 0: G_{nchunk-1} = 0; G_c = decay_{c+1} G_{c+1} + slot_c (slot c holds U_{c+1}), written
-//            only as bf16 tiles.
-// Loads of eight slots are issued ahead of their dependent updates.
-__global__ void __launch_bounds__(256)
-ssd_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir,
-                float4* zero0, float4* zero1, size_t nzero4) {
-    pdl_launch_dependents();
-    pdl_wait();
-    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    // zero0 / zero1 (the backward's dB, dC when several CTAs add into them): nzero4 float4 each
-    for (size_t z = e; z < nzero4; z += (size_t)gridDim.x * blockDim.x) {
-        zero0[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        zero1[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
-    if (e >= (size_t)BH * n4) return;
-    const size_t stride = (size_t)BH * n4;
-    const int bh = (int)(e / n4), q = (int)(e % n4);
-    const float* dec = decay + (size_t)bh * nchunk;
-    const uint32_t toff = tc::sw128_off(q / (kP / 4), (q % (kP / 4)) * 4, kKD);
-    auto put = [&](int c, float4 v) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-        uint2 u = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-        *reinterpret_cast<uint2*>(tiles + ((size_t)c * BH + bh) * kTileBytes + toff) = u;
-    };
-    float4* p = buf + e;
-    float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const int first = dir > 0 ? 0 : nchunk - 1;
-    if (dir > 0) p[(size_t)first * stride] = s;
-    put(first, s);
-    for (int k0 = 1; k0 < nchunk; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
-            if (k0 + k < nchunk) v[k] = __ldcg(p + (size_t)c * stride);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            if (k0 + k < nchunk) {
-                const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
-                const float d = dec[c - dir];
-                s = make_float4(fmaf(d, s.x, v[k].x), fmaf(d, s.y, v[k].y), fmaf(d, s.z, v[k].z), fmaf(d, s.w, v[k].w));
-                if (dir > 0) p[(size_t)c * stride] = s;
-                put(c, s);
-            }
-        }
     }
 }
 
@@ -592,7 +536,7 @@ int out_heads_per_cta(const lr_desc& d, int nchunk) {
 // =========================================================================================
 // Backward.  With G_c the adjoint of the state leaving chunk c (G_{last} = 0):
 //   U_c = C^T diag(E) dy_h                   (ssd_state_kernel, dir < 0)
-//   G_{c-1} = e^{l_Q, c} G_c + U_c            (ssd_pass_kernel, dir < 0)
+//   G_{c-1} = e^{l_Q, c} G_c + U_c            (state_pass_kernel, dir < 0)
 // and per (chunk, head), with S2 = dy x^T, Pd = S2 o Lmask, P = M o Lmask, R = Pd o M:
 //   dC += Pd B + diag(E) dy S_in^T            dB += Pd^T C + diag(w) x G^T   (summed over heads)
 //   dx  = P^T dy + diag(w) B G + D dy
@@ -643,8 +587,6 @@ struct GradSmem {
 // TMEM columns: dC (0), dB (128); phase A: M (256), S2 (384); phase B: dV1 (256), BG (320), Y2 (384).
 constexpr uint32_t kGdC = 0, kGdB = 128, kGM = 256, kGS2 = 384, kGdV = 256, kGBG = 320, kGY2 = 384;
 
-__device__ __forceinline__ void wg0_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
 // Thread that issues the gradient kernel's products after the prologue: warpgroup 1 idles while
 // they run, and an issuing thread blocks while the tensor pipe is full, so warpgroup 0 stays free
 // to prepare the next head's decays and to reduce the current head's row terms.
@@ -652,50 +594,6 @@ constexpr int kIssuer = 128;
 // Thread (another warp of warpgroup 1) that loads {x, dy} of the next head as soon as batch 1a has
 // consumed P, while the issuing thread may still be blocked issuing batch 1b.
 constexpr int kLoader = 160;
-
-// Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum);
-// *total receives the sum of all 128 values.
-__device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp, float* total = nullptr) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) tmp[warp] = x;
-    wg0_bar();
-    float add = 0.0f;
-    for (int w = 0; w < warp; ++w) add += tmp[w];
-    if (total) *total = ((tmp[0] + tmp[1]) + tmp[2]) + tmp[3];
-    wg0_bar();
-    return x + add;
-}
-// Sums of two values over the 128 threads of warpgroup 0, fixed order, results in every thread.
-__device__ __forceinline__ float2 wg0_sum2(float x, float y, float* tmp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        x += __shfl_xor_sync(0xffffffffu, x, o);
-        y += __shfl_xor_sync(0xffffffffu, y, o);
-    }
-    if (lane == 0) {
-        tmp[8 + warp] = x;
-        tmp[12 + warp] = y;
-    }
-    wg0_bar();
-    const float2 s = make_float2((tmp[8] + tmp[9]) + (tmp[10] + tmp[11]), (tmp[12] + tmp[13]) + (tmp[14] + tmp[15]));
-    wg0_bar();
-    return s;
-}
-
-// Pack 8 floats into 8 bf16 (one 16-byte chunk).
-__device__ __forceinline__ uint4 pack8(const float* f) {
-    uint4 r;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-    return r;
-}
 
 // One CTA per (chunk, batch row, group, block of hb heads), 256 threads: warpgroup wg handles
 // columns [64 wg, 64 wg + 64) (or [32 wg, ...) of 64-wide tensors) of TMEM lane / row 32 wq + lane.
@@ -896,8 +794,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 }
 #pragma unroll
                 for (int k = 0; k < 32; k += 8) {
-                    *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = pack8(m + k);
-                    *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = pack8(s2 + k);
+                    *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = pack_bf16x8(m + k);
+                    *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = pack_bf16x8(s2 + k);
                 }
 #pragma unroll
                 for (int k = 0; k < 32; ++k) rsum += rr[k];
@@ -1003,9 +901,9 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                         xs[e] *= w;
                         os[e] *= E;
                     }
-                    if (t0 + row < a.L) *reinterpret_cast<uint4*>(dxrow + col + hh) = pack8(dx);
-                    *px = pack8(xs);
-                    *po = pack8(os);
+                    if (t0 + row < a.L) *reinterpret_cast<uint4*>(dxrow + col + hh) = pack_bf16x8(dx);
+                    *px = pack_bf16x8(xs);
+                    *po = pack_bf16x8(os);
                 }
             }
             qdqp[wg * kQ + row] = E * qdq;
@@ -1182,7 +1080,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
         const int n4 = kKD * kP / 4;
         const size_t total = (size_t)a.B * a.H * n4;
         note_launch("ssd_state_pass");
-        cudaError_t e = launch_pdl(ssd_pass_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
+        cudaError_t e = launch_pdl(state_pass_kernel<kP>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
                                    (float4*)ckpt, stiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, +1,
                                    (float4*)nullptr, (float4*)nullptr, (size_t)0);
         if (e != cudaSuccess) return LR_ERR_CUDA;
@@ -1242,7 +1140,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         const size_t total = (size_t)a.B * a.H * n4;
         const size_t nzero4 = ga.accumulate ? (size_t)d.B * d.L * d.G * kKD / 4 : 0;
         note_launch("ssd_state_pass");
-        cudaError_t e = launch_pdl(ssd_pass_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
+        cudaError_t e = launch_pdl(state_pass_kernel<kP>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
                                    (float4*)Ubuf, ws + w.gtiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, -1,
                                    (float4*)gr.dBm, (float4*)gr.dCm, nzero4);
         if (e != cudaSuccess) return LR_ERR_CUDA;

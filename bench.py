@@ -236,11 +236,28 @@ def kernel_cost(w, name, pas, pass_bytes):
     return pass_bytes, 0
 
 
+# S6 is bound by plain ALU work: per (t, d, n) element, FMA-pipe ops and MUFU (ex2 / rcp) results
+# (forward 7 + 1, backward 25 + 2).  Peak element rate = 148 SMs x min(128 FMA lanes / ops,
+# 16 MUFU lanes / results) x the maximum SM clock (1,965 MHz).
+S6_ALU = {"fwd": (7, 1), "bwd": (25, 2)}
+SM_COUNT, SM_MAX_HZ = 148, 1.965e9
+
+
+def kernel_alu(w, name, pas):
+    if w["kind"] != "s6" or name.endswith("param_reduce"):
+        return None
+    fma, mufu = S6_ALU[pas]
+    elems = w["B"] * w["L"] * w["D"] * w["N"]
+    peak = SM_COUNT * SM_MAX_HZ * min(128.0 / fma, 16.0 / mufu)
+    return {"elements": elems, "peak_elems_per_s": peak}
+
+
 def kernel_table(w, names, ms, pas, pass_bytes):
     rows = []
     for k, (n, t) in enumerate(zip(names, ms)):
         b, f = kernel_cost(w, n, pas, pass_bytes)
-        rows.append({"pass": pas, "index": k, "kernel": n, "ms": t, "bytes": b, "flops": f})
+        rows.append({"pass": pas, "index": k, "kernel": n, "ms": t, "bytes": b, "flops": f,
+                     "alu": kernel_alu(w, n, pas)})
     return rows
 
 
@@ -250,6 +267,12 @@ def kernel_roofline(row, pk):
     t_hbm = row["bytes"] / (pk["hbm_gbs"] * 1e9)
     t_tc = row["flops"] / (pk["bf16_tflops"] * 1e12)
     sec = row["ms"] * 1e-3
+    alu = row.get("alu")
+    if alu and alu["elements"] / alu["peak_elems_per_s"] > max(t_hbm, t_tc):
+        ach = alu["elements"] / sec / 1e9
+        pk_g = alu["peak_elems_per_s"] / 1e9
+        return {"bound": "alu", "achieved": round(ach, 1), "peak": round(pk_g, 1), "unit": "Gelem/s",
+                "frac": round(ach / pk_g, 4)}
     if t_tc > t_hbm:
         ach = row["flops"] / sec / 1e12
         return {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",

@@ -13,11 +13,14 @@
 // Work split.  The scan is bound by the per-(t, d, n) arithmetic (one exp or reciprocal and a
 // handful of FMAs per state per step), not by HBM, so the layout keeps states in registers and
 // avoids cross-thread traffic on the recurrence: a CTA owns one batch row and 64 channels for the
-// whole sequence; two threads per channel (lanes l and l^16 of a warp) hold 8 of its 16 states
-// each, so the readout sum over n is one shuffle.  Segments of S <= 64 steps are staged in shared
-// memory by TMA (x, dt, z, dy as [S][64] bf16 tiles, B, C as [S][16]); outputs are written back
-// into the consumed tile slots and stored with TMA.  The forward pass double-buffers segments and
-// writes the state entering each segment to the checkpoint buffer.
+// whole sequence; kTPC = 2 threads per channel (lanes q and q + 16 of a warp) hold 8 of its 16
+// states each, so the readout sum over n is one shuffle.  (4 or 8 threads per channel give more
+// warps but repeat the per-(step, channel) work -- loads, gate, reductions, outputs -- on every
+// thread; both measured slower on the S6 workload.)
+// Segments of S <= 64 steps are staged in shared memory by TMA (x, dt, z, dy as [S][64] bf16
+// tiles, B, C as [S][16]); outputs are written back into the consumed tile slots and stored with
+// TMA.  The forward pass double-buffers segments and writes the state entering each segment to the
+// checkpoint buffer.
 //
 // Backward, per segment in reverse order (the adjoint carry G stays in registers across
 // segments): (A) from the checkpoint, run the segment forward and keep the state at every 8-step
@@ -25,21 +28,25 @@
 // keeping h_t and abar_t in registers, then run the adjoint recurrence
 // G_t[n] = ds_t C_t[n] + abar_{t+1} G_{t+1}[n] (ds = dy silu(z)) backwards through them and form
 // every gradient.  dB_t[n] and dC_t[n] (sums over channels) are reduced over the 16 channels of a
-// half-warp with a butterfly, then over the CTA's four warps in a fixed order, giving one partial
-// per 64-channel block; dA and dD partials are per batch row.  A small kernel sums the partials in
-// a fixed order (deterministic results).
+// warp with a butterfly, then over the CTA's warps in a fixed order once per sub-block, giving
+// one partial per 64-channel block; dA and dD partials are per batch row.  A small kernel sums the
+// partials in a fixed order (deterministic results).
 #include "common.cuh"
 #include "host_common.h"
 
 namespace lrs {
 namespace {
 
-constexpr int kDB = 64;       // channels per CTA
-constexpr int kNH = 8;        // states per thread (N = 16)
-constexpr int kN = 2 * kNH;
-constexpr int kThreads = 128; // 64 channels x 2 halves
-constexpr int kMaxS = 64;     // segment rows per TMA box
-constexpr int kSub = 8;       // backward sub-block length
+constexpr int kDB = 64;                // channels per CTA
+constexpr int kN = 16;                 // states per channel
+constexpr int kTPC = 2;                // threads per channel
+constexpr int kNH = kN / kTPC;         // states per thread
+constexpr int kCPW = 32 / kTPC;        // channels per warp
+constexpr int kThreads = kDB * kTPC;   // 512
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxS = 64;              // segment rows per TMA box
+constexpr int kSub = 8;                // backward sub-block length
+static_assert(2 * kNH == kCPW, "the dB / dC reduce-scatter over a warp's channels leaves one value per lane");
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float ex2(float x) {
@@ -55,16 +62,20 @@ __device__ __forceinline__ float rcp(float x) {
 __device__ __forceinline__ float sigm(float z) { return rcp(1.0f + ex2(-z * kLog2e)); }
 __device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// 8 consecutive bf16 -> float
-__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* out) {
-    uint4 v = *reinterpret_cast<const uint4*>(p);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+// kNH consecutive bf16 -> float (this thread's states of a B or C row)
+__device__ __forceinline__ void ldn(const __nv_bfloat16* p, float* out) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 f = __bfloat1622float2(h[i]);
-        out[2 * i] = f.x;
-        out[2 * i + 1] = f.y;
+    for (int i = 0; i < kNH; i += 2) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p + i));
+        out[i] = f.x;
+        out[i + 1] = f.y;
     }
+}
+// sum over the kTPC threads of a channel (lanes l, l + kCPW, l + 2 kCPW, ...)
+__device__ __forceinline__ float chan_sum(float x) {
+#pragma unroll
+    for (int o = kCPW; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
 }
 
 struct S6Args {
@@ -129,7 +140,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     char* sm = smem_base();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm);  // bar[0], bar[1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, dl = warp * 16 + (lane & 15);
+    const int part = lane / kCPW, dl = warp * kCPW + (lane % kCPW);
     const int b = blockIdx.x / a.ncb, cb = blockIdx.x % a.ncb;
     const int d = cb * kDB + dl;
     const bool dok = d < a.D;
@@ -157,7 +168,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     Disc c;
 #pragma unroll
     for (int j = 0; j < kNH; ++j) {
-        float A = dok ? a.A[(size_t)d * kN + half * kNH + j] : -1.0f;
+        float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
         c.A[j] = A;
         c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
         c.ia[j] = 1.0f / A;
@@ -177,7 +188,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         }
         ok = ok && mbar_wait(&bar[s], (k >> 1) & 1, a.hdr, 300);
         if (dok) {
-            float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + half * kNH;
+            float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + part * kNH;
 #pragma unroll
             for (int j = 0; j < kNH; ++j) ck[j] = h[j];
         }
@@ -191,8 +202,8 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int t = 0; t < nt; ++t) {
                 const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
                 float Bv[kNH], Cv[kNH];
-                ld8(Bs + t * kN + half * kNH, Bv);
-                ld8(Cs + t * kN + half * kNH, Cv);
+                ldn(Bs + t * kN + part * kNH, Bv);
+                ldn(Cs + t * kN + part * kNH, Cv);
                 float sacc = 0.0f;
 #pragma unroll
                 for (int j = 0; j < kNH; ++j) {
@@ -201,8 +212,8 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
                     sacc = fmaf(Cv[j], h[j], sacc);
                 }
-                sacc += __shfl_xor_sync(0xffffffffu, sacc, 16);
-                if (half == 0) {
+                sacc = chan_sum(sacc);
+                if (part == 0) {
                     float yv = fmaf(Dd, xv, sacc);
                     if (a.has_z) {
                         const float zv = bf(Z + t * kDB + dl);
@@ -229,7 +240,7 @@ constexpr size_t kOffB = kOffX + 4 * kTileDT;
 constexpr size_t kOffBnd = kOffB + 2 * kTileBC;
 constexpr size_t kBndBytes = size_t(kMaxS / kSub) * kThreads * kNH * 4;
 constexpr size_t kOffRed = kOffBnd + kBndBytes;
-constexpr size_t kRedBytes = size_t(4) * kMaxS * 2 * kN * 4;
+constexpr size_t kRedBytes = size_t(kWarps) * kSub * 2 * kN * 4;  // per-warp dB / dC of one sub-block
 constexpr size_t kBwdSmem = kOffRed + kRedBytes + 128;
 
 template <int DISC>
@@ -248,10 +259,10 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     const __nv_bfloat16* Bs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB);
     const __nv_bfloat16* Cs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB + kTileBC);
     float* bnd = reinterpret_cast<float*>(sm + kOffBnd);  // [sub-block][thread][kNH]
-    float* red = reinterpret_cast<float*>(sm + kOffRed);  // [warp][t][2][kN]
+    float* red = reinterpret_cast<float*>(sm + kOffRed);  // [warp][step of the sub-block][2][kN]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, q = lane & 15, dl = warp * 16 + q;
+    const int part = lane / kCPW, q = lane % kCPW, dl = warp * kCPW + q;
     const int b = blockIdx.x / a.ncb, cb = blockIdx.x % a.ncb;
     const int d = cb * kDB + dl;
     const bool dok = d < a.D;
@@ -263,7 +274,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     Disc c;
 #pragma unroll
     for (int j = 0; j < kNH; ++j) {
-        float A = dok ? a.A[(size_t)d * kN + half * kNH + j] : -1.0f;
+        float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
         c.A[j] = A;
         c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
         c.ia[j] = 1.0f / A;
@@ -293,7 +304,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         }
         float h[kNH];
         {
-            const float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + (dok ? d : 0)) * kN + half * kNH;
+            const float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + (dok ? d : 0)) * kN + part * kNH;
 #pragma unroll
             for (int j = 0; j < kNH; ++j) h[j] = dok ? ck[j] : 0.0f;
         }
@@ -308,7 +319,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int t = sb * kSub; t < te; ++t) {
                 const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
                 float Bv[kNH];
-                ld8(Bs + t * kN + half * kNH, Bv);
+                ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
                 for (int j = 0; j < kNH; ++j) {
                     float ab, be;
@@ -333,7 +344,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     const int t = tb + i;
                     const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
                     float Bv[kNH];
-                    ld8(Bs + t * kN + half * kNH, Bv);
+                    ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
                     for (int j = 0; j < kNH; ++j) {
                         float ab, be;
@@ -351,13 +362,13 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
                     const float dyv = bf(DY + t * kDB + dl);
                     float Bv[kNH], Cv[kNH];
-                    ld8(Bs + t * kN + half * kNH, Bv);
-                    ld8(Cs + t * kN + half * kNH, Cv);
+                    ldn(Bs + t * kN + part * kNH, Bv);
+                    ldn(Cs + t * kN + part * kNH, Cv);
                     // readout and gate
                     float sacc = 0.0f;
 #pragma unroll
                     for (int j = 0; j < kNH; ++j) sacc = fmaf(Cv[j], hr[i][j], sacc);
-                    sacc += __shfl_xor_sync(0xffffffffu, sacc, 16);
+                    sacc = chan_sum(sacc);
                     const float s = fmaf(Dd, xv, sacc);
                     float ds = dyv, dz = 0.0f;
                     if (a.has_z) {
@@ -391,12 +402,13 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                         }
                         anext[j] = ab;
                     }
-                    dxa += __shfl_xor_sync(0xffffffffu, dxa, 16);
-                    dta += __shfl_xor_sync(0xffffffffu, dta, 16);
-                    // dB / dC: sum over the 16 channels of this half-warp (butterfly; lane q
-                    // ends with the sum of value q)
+                    dxa = chan_sum(dxa);
+                    dta = chan_sum(dta);
+                    // dB / dC: sum over the kCPW channels of the warp that hold the same states
+                    // (butterfly over lanes differing in the channel bits; lane q ends with the
+                    // sum of value q)
 #pragma unroll
-                    for (int m = 8; m >= 1; m >>= 1) {
+                    for (int m = kCPW / 2; m >= 1; m >>= 1) {
 #pragma unroll
                         for (int i2 = 0; i2 < m; ++i2) {
                             const bool up = (q & m) != 0;
@@ -405,8 +417,8 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                             v[i2] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                         }
                     }
-                    red[((size_t)(warp * kMaxS + t) * 2 + (q >> 3)) * kN + half * kNH + (q & 7)] = v[0];
-                    if (half == 0) {
+                    red[((size_t)(warp * kSub + i) * 2 + q / kNH) * kN + part * kNH + (q % kNH)] = v[0];
+                    if (part == 0) {
                         X[t * kDB + dl] = __float2bfloat16_rn(fmaf(ds, Dd, dxa));
                         DT[t * kDB + dl] = __float2bfloat16_rn(dta);
                         if (a.has_z) Z[t * kDB + dl] = __float2bfloat16_rn(dz);
@@ -414,6 +426,17 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     }
                 }
             }
+            // this sub-block's dB / dC partial of the CTA: fixed-order sum over the warps
+            __syncthreads();
+            for (int e = tid; e < n * 2 * kN; e += kThreads) {
+                const int i = e / (2 * kN), r = e % (2 * kN);
+                float sum = 0.0f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) sum += red[((size_t)(w * kSub + i) * 2) * kN + r];
+                float* dst = (r < kN ? a.pdB : a.pdC) + (((size_t)cb * a.B + b) * a.L + t0 + tb + i) * kN + (r % kN);
+                *dst = sum;
+            }
+            __syncthreads();
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -423,22 +446,13 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             if (a.has_z) tma_store_3d(&mdZ, Z, cb * kDB, t0, b);
             bulk_commit();
         }
-        // per-CTA partial dB / dC of this segment: fixed-order sum over the four warps
-        for (int e = tid; e < nt * 2 * kN; e += kThreads) {
-            const int t = e / (2 * kN), r = e % (2 * kN);
-            float sum = 0.0f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) sum += red[((size_t)(w * kMaxS + t) * 2) * kN + r];
-            float* dst = (r < kN ? a.pdB : a.pdC) + (((size_t)cb * a.B + b) * a.L + t0 + t) * kN + (r % kN);
-            *dst = sum;
-        }
         __syncthreads();
     }
     if (dok) {
-        float* pa = a.pdA + ((size_t)b * a.D + d) * kN + half * kNH;
+        float* pa = a.pdA + ((size_t)b * a.D + d) * kN + part * kNH;
 #pragma unroll
         for (int j = 0; j < kNH; ++j) pa[j] = dA[j];
-        if (half == 0) a.pdD[(size_t)b * a.D + d] = dD;
+        if (part == 0) a.pdD[(size_t)b * a.D + d] = dD;
     }
     if (tid == 0) bulk_wait_read_all();
 }

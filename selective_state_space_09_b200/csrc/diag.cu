@@ -105,12 +105,12 @@ template <typename T> struct Kind<LR_ROTLRU, T> {
             return {m * cs, m * sn};
         }
     };
-    static __device__ __forceinline__ V ldb(const T* Bs, int t, int u) {
-        return {IO<T>::ld(Bs + t * BW + 2 * u), IO<T>::ld(Bs + t * BW + 2 * u + 1)};
+    static __device__ __forceinline__ V ldb(const T* Bs, int t, int u) {  // (re, im) in one access
+        const float2 v = IO<T>::ld2(Bs + t * BW + 2 * u);
+        return {v.x, v.y};
     }
     static __device__ __forceinline__ void stb(T* Bs, int t, int u, V v) {
-        IO<T>::st(Bs + t * BW + 2 * u, v.r);
-        IO<T>::st(Bs + t * BW + 2 * u + 1, v.i);
+        IO<T>::st2(Bs + t * BW + 2 * u, make_float2(v.r, v.i));
     }
     static __device__ __forceinline__ void st_ckpt(float* p, int chan0, V v) {
         p[chan0] = v.r;
@@ -198,6 +198,21 @@ __device__ V lookback_carry(const unsigned int* flags, const Agg<V>* aggRec, con
     return x;
 }
 
+// The carry entering tile k when its neighbour k + dir has already published its inclusive prefix
+// (or does not exist): read while the tile's own loads are in flight.  Returns whether every lane
+// found it (otherwise the caller takes the look-back above, which yields the same value once the
+// neighbour's prefix is out).
+template <typename V>
+__device__ __forceinline__ bool early_carry(const unsigned int* flags, const V* preRec, size_t row, int k, int dir,
+                                            int nseg, int CB, int lane, bool act, V& x) {
+    x = zero_of(V{});
+    const int j = k + dir;
+    if (j < 0 || j >= nseg) return true;
+    const bool ready = ld_acquire(&flags[row + j]) == kFlagPrefix;
+    if (ready && act) x = ld_cg(&preRec[(row + j) * CB + lane]);
+    return __all_sync(0xffffffffu, ready);
+}
+
 // Dynamic shared memory, re-aligned to 128 bytes.
 __device__ __forceinline__ char* smem_base() {
     extern __shared__ char dyn_smem[];
@@ -245,6 +260,14 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
     }
     const int unit = cb * CB + u;  // global unit index (channel or pair)
+    const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
+    const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
+    Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
+    V* preRec = reinterpret_cast<V*>(a.pre);
+    const bool act = warp == 0 && lane < CB && unit < units;
+    V carry = zero_of(V{});
+    bool have = false;
+    if (warp == 0) have = early_carry(a.flags, preRec, row, seg, -1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     const int nt = min(a.S, a.L - t0g);
     const int spg = (a.S + NG - 1) / NG;
@@ -263,13 +286,12 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     aggF[grp * CB + u] = {P, h};
     __syncthreads();
 
-    // tile carry through the chained look-back (warp 0, one lane per unit)
-    const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
+    // tile carry through the chained look-back (warp 0, one lane per unit); the carry is usually
+    // known already (early_carry), and this tile's own prefix is published after the other warps
+    // have been released
+    const bool has_succ = seg + 1 < a.nseg;
+    V pub = zero_of(V{});
     if (warp == 0) {
-        const bool act = lane < CB && unit < units;
-        const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
-        Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
-        V* preRec = reinterpret_cast<V*>(a.pre);
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB) {
             for (int g = 0; g < NG; ++g) {
@@ -278,26 +300,29 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
                 tile.m = mulx(ag.m, tile.m);
             }
         }
-        const bool has_succ = seg + 1 < a.nseg;
-        if (seg > 0 && has_succ) {
-            if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+        if (!have) {
+            if (seg > 0 && has_succ) {
+                if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+            }
+            carry = lookback_carry(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane, act, a.hdr, 101);
         }
-        const V carry = lookback_carry(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane, act,
-                                       a.hdr, 101);
-        const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == 0;
-        if (has_succ && !withhold) {
-            if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
-        }
+        pub = fmax_(tile.m, carry, tile.v);
         if (act) K::st_ckpt(a.ckpt + ((size_t)seg * a.B + b) * a.D, unit * K::chans_per_unit, carry);
         if (lane < CB) carryS[lane] = carry;
     }
     __syncthreads();
+    if (warp == 0) {
+        const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == 0;
+        if (has_succ && !withhold) {
+            if (act) st_cg(&preRec[(row + seg) * CB + lane], pub);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
+        }
+    }
 
     // apply: recompute the group with its true carry-in, write y into the b slot
     V hh = carryS[u];
@@ -323,7 +348,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 
 // -------------------------------------------------------------------------------- backward
 template <int KIND, typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)  // two tiles per SM (shared memory)
 diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapDY, const __grid_constant__ CUtensorMap mapDC,
                 const __grid_constant__ CUtensorMap mapDB, DiagArgs a) {
@@ -353,21 +378,31 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         misc[0] = seg;
         misc[1] = rem / a.ncb;
         misc[2] = rem % a.ncb;
-        mbar_init(bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
+    // coefficients and b (the forward recompute) on bar[0], dy (the adjoint) on bar[1]
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + 2 * K::BW) * sizeof(T)));
-        tma_load_3d(Cs, &mapC, bar, cb * K::CW, t0g, b);
-        tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
-        tma_load_3d(Ds, &mapDY, bar, cb * K::BW, t0g, b);
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(a.S * (K::CW + K::BW) * sizeof(T)));
+        tma_load_3d(Cs, &mapC, &bar[0], cb * K::CW, t0g, b);
+        tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
+        mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
+        tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
     }
     const int unit = cb * CB + u;
     const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
+    const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
+    Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
+    V* preRec = reinterpret_cast<V*>(a.pre);
+    const bool act = warp == 0 && lane < CB && unit < units;
+    V carry = zero_of(V{});
+    bool have = false;
+    if (warp == 0) have = early_carry(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     if (tid < CB) {
         V c0 = zero_of(V{});
@@ -379,7 +414,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int spg = (a.S + NG - 1) / NG;
     const int j0 = grp * spg, j1 = min(j0 + spg, nt);
     const int n = max(j1 - j0, 0);
-    bool ok = mbar_wait(bar, 0, a.hdr, 200);
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 200);
 
     // forward aggregate of the group
     {
@@ -412,6 +447,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         }
     }
     // reverse aggregate of the group: outgoing carry = v + m * incoming
+    ok = mbar_wait(&bar[1], 0, a.hdr, 202) && ok;
     {
         V M = one_of(V{}), r = zero_of(V{});
         if (ok)
@@ -425,12 +461,10 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     }
     __syncthreads();
 
-    // tile carry from later segments (warp 0)
+    // tile carry from later segments (warp 0; usually known already, see the forward kernel)
+    const bool has_pred = seg > 0;  // earlier segment waits on this one
+    V pub = zero_of(V{});
     if (warp == 0) {
-        const bool act = lane < CB && unit < units;
-        const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
-        Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
-        V* preRec = reinterpret_cast<V*>(a.pre);
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB)
             for (int g = NG - 1; g >= 0; --g) {
@@ -438,25 +472,28 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
                 tile.v = fmax_(ag.m, tile.v, ag.v);
                 tile.m = mulx(ag.m, tile.m);
             }
-        const bool has_pred = seg > 0;  // earlier segment waits on this one
-        if (has_pred && seg + 1 < a.nseg) {
-            if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+        if (!have) {
+            if (has_pred && seg + 1 < a.nseg) {
+                if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+            }
+            carry = lookback_carry(a.flags, aggRec, preRec, row, seg, +1, a.nseg, CB, lane, act, a.hdr, 201);
         }
-        const V carry = lookback_carry(a.flags, aggRec, preRec, row, seg, +1, a.nseg, CB, lane, act,
-                                       a.hdr, 201);
+        pub = fmax_(tile.m, carry, tile.v);
+        if (lane < CB) carryS[CB + lane] = carry;
+    }
+    __syncthreads();
+    if (warp == 0) {
         const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == a.nseg - 1;
         if (has_pred && !withhold) {
-            if (act) st_cg(&preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v));
+            if (act) st_cg(&preRec[(row + seg) * CB + lane], pub);
             __threadfence();
             __syncwarp();
             if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
         }
-        if (lane < CB) carryS[CB + lane] = carry;
     }
-    __syncthreads();
 
     // adjoint sweep of the group with its true carry; gradients into the shared slots
     V r = carryS[CB + u];
@@ -514,19 +551,40 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     }
 }
 
-// Fixed-order reduction of rotlru's per-tile parameter partials over (batch row, segment).
-__global__ void rotlru_param_reduce(const float2* __restrict__ partial, int rows, int K,
-                                    float* __restrict__ dmag, float* __restrict__ dtheta) {
-    int k = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= K) return;
-    float s0 = 0.0f, s1 = 0.0f;
-    for (int r = 0; r < rows; ++r) {
-        float2 v = __ldg(&partial[(size_t)r * K + k]);
-        s0 += v.x;
-        s1 += v.y;
+// Fixed-order reduction of rotlru's per-tile parameter partials over (batch row, segment).  A
+// block owns kRedPairs pairs; its kRedSlices slices each sum every kRedSlices-th row (rows in
+// increasing order), and the slices are then folded by a fixed pairwise tree, so the result does
+// not depend on timing.
+constexpr int kRedPairs = 16, kRedSlices = 64;
+__global__ void __launch_bounds__(kRedPairs * kRedSlices)
+rotlru_param_reduce(const float2* __restrict__ partial, int rows, int K, float* __restrict__ dmag,
+                    float* __restrict__ dtheta) {
+    __shared__ float2 red[kRedSlices][kRedPairs];
+    const int x = threadIdx.x % kRedPairs, y = threadIdx.x / kRedPairs;
+    const int k = blockIdx.x * kRedPairs + x;
+    float2 acc = make_float2(0.0f, 0.0f);
+    if (k < K) {
+#pragma unroll 8
+        for (int r = y; r < rows; r += kRedSlices) {
+            const float2 v = __ldg(&partial[(size_t)r * K + k]);
+            acc.x += v.x;
+            acc.y += v.y;
+        }
     }
-    dmag[k] = s0;
-    dtheta[k] = s1;
+    red[y][x] = acc;
+    __syncthreads();
+#pragma unroll
+    for (int off = kRedSlices / 2; off > 0; off >>= 1) {
+        if (y < off) {
+            red[y][x].x += red[y + off][x].x;
+            red[y][x].y += red[y + off][x].y;
+        }
+        __syncthreads();
+    }
+    if (y == 0 && k < K) {
+        dmag[k] = red[0][x].x;
+        dtheta[k] = red[0][x].y;
+    }
 }
 
 // ------------------------------------------------------------------------------ host side
@@ -628,8 +686,8 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
     if (KIND == LR_ROTLRU) {
         int K2 = (int)(d.D / 2);
         note_launch("rotlru_param_reduce");
-        rotlru_param_reduce<<<(K2 + 127) / 128, 128, 0, st>>>(a.partial, (int)d.B * g.nseg, K2,
-                                                             gr.dmag, gr.dtheta);
+        rotlru_param_reduce<<<(K2 + kRedPairs - 1) / kRedPairs, kRedPairs * kRedSlices, 0, st>>>(
+            a.partial, (int)d.B * g.nseg, K2, gr.dmag, gr.dtheta);
         s = check_launch();
     }
     return s;

@@ -199,12 +199,9 @@ def kernel_cost(w, name, pas, pass_bytes):
         slot = B * H * N * P * 4           # one f32 state slot
         tile = B * H * N * P * 2           # one bf16 state slot
         head_chunks = nc * B * H
-        if name == "ssd_chunk_state":
-            return tok + bc + dt + (nc - 1) * slot, (nc - 1) * B * H * 2 * N * P * Q
-        if name == "ssd_state_pass":
-            if pas == "fwd":
-                return (nc - 1) * slot + nc * slot + nc * tile, 0
-            return (nc - 1) * slot + nc * tile, 0
+        if name == "ssd_state_scan":       # x (dy), B (C), dt in; every slot out (f32 + tile; tile)
+            out = nc * (slot + tile) if pas == "fwd" else nc * tile
+            return tok + bc + dt + out, (nc - 1) * B * H * 2 * N * P * Q
         if name == "ssd_chunk_out":
             fl = head_chunks * (2 * Q * P * Q + 2 * Q * P * N) + nc * B * G * 2 * Q * Q * N
             return 2 * tok + 2 * bc + dt + nc * tile, fl

@@ -72,6 +72,32 @@ __device__ __forceinline__ void cta_inclusive_sum_n(float (&x)[NV], float* tmp) 
 
 __device__ __forceinline__ void wg0_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// cta_inclusive_sum_n over the 128 threads of warpgroup 0 (named barrier 1; tmp: 4 * NV floats).
+template <int NV>
+__device__ __forceinline__ void wg0_inclusive_sum_n(float (&x)[NV], float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const float y = __shfl_up_sync(0xffffffffu, x[j], o);
+            if (lane >= o) x[j] += y;
+        }
+    }
+    if (lane == 31) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) tmp[warp * NV + j] = x[j];
+    }
+    wg0_bar();
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        float add = 0.0f;
+        for (int w = 0; w < warp; ++w) add += tmp[w * NV + j];
+        x[j] += add;
+    }
+    wg0_bar();
+}
+
 // Inclusive prefix sum over the 128 threads of warpgroup 0 (same order as cta_inclusive_sum);
 // *total receives the sum of all 128 values.
 __device__ __forceinline__ float wg0_inclusive_sum(float x, float* tmp, float* total = nullptr) {

@@ -13,11 +13,10 @@
 // M is the same for every head of a group: the output kernel computes it once per (batch row,
 // chunk) and runs the group's heads through it.
 //
-// Forward = three launches, none of which waits on another CTA:
-//   ssd_state_kernel  (batch row, chunk, block of 4 heads): Sl of every chunk but the last,
-//                     written into checkpoint slot c + 1; e^{l_Q} per chunk;
-//   state_pass_kernel  elementwise over (batch row, head, state element): slot c <- e^{l_Q, c-1}
-//                     slot c-1 + Sl_{c-1}, in place, so slot c ends as the state entering chunk c;
+// Forward = two launches, none of which waits on another CTA:
+//   ssd_scan_kernel   (batch row, head): runs through the chunks, S_{c+1} = e^{l_Q,c} S_c + Sl_c
+//                     with Sl_c on tcgen05 and S in registers; slot c of the checkpoint <- S_c
+//                     (f32, and a bf16 tile copy for the tensor cores);
 //   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x.
 #include "chunk_common.cuh"
 
@@ -27,7 +26,6 @@ namespace {
 
 constexpr int kP = 64;    // head dimension (value columns)
 constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf16 SW128 tile
-constexpr int kHS = 2;    // heads per CTA of the state kernel
 
 struct SsdArgs {
     int B, L, H, G, HpG, nchunk;  // HpG: heads per group
@@ -35,152 +33,302 @@ struct SsdArgs {
     const float* A;               // [H]
     const float* Dskip;           // [H] or null
     const float* ckpt;            // [nchunk][B][H][N][P] f32 (state entering each chunk)
-    float* decay;                 // [B][H][nchunk] e^{l_Q}
     WsHeader* hdr;
 };
 
-// Per-step log decay and beta of head h at step t (t >= L: no decay, no input).
-__device__ __forceinline__ void ssd_coef(const SsdArgs& a, int b, int h, int t, float& lam, float& beta) {
-    lam = 0.0f;
-    beta = 0.0f;
-    if (t >= a.L) return;
-    const float v = __bfloat162float(a.dt[((size_t)b * a.L + t) * a.H + h]);
-    const float Ah = a.A[h];
-    lam = v * Ah;
-    beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+// Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
+__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
+
+// Inclusive prefix sum over the 128 threads of warpgroup wg (same order as cta_inclusive_sum).
+__device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
+    const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 3;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[w] = x;
+    wg_sync(wg);
+    float add = 0.0f;
+    for (int k = 0; k < w; ++k) add += tmp[k];
+    wg_sync(wg);
+    return x + add;
 }
 
-// ------------------------------------------------------------------------- state increments
-struct StateSmem {
-    static constexpr size_t kR = 0;                                  // 128 x 128 bf16 (B or C)
-    static constexpr size_t kZ = kR + kQ * kKD * 2;                  // kHS tiles 128 x 64 (x or dy)
-    static constexpr size_t kTmp = kZ + (size_t)kHS * kQ * kP * 2;   // scan scratch, l_Q per head
-    static constexpr size_t kBar = kTmp + 128;
-    static constexpr size_t kTmem = kBar + 64;
-    static constexpr size_t kEnd = kTmem + 64;
+// -------------------------------------------------------------------- chunk states, scanned
+// One CTA per (batch row, head) walks the chunks in order (dir > 0) or in reverse (dir < 0):
+//   dir > 0: S_0 = 0,      S_{c+1} = e^{l_Q,c} S_c + B_c^T diag(w) x_c    slot c <- S_c
+//            (the f32 checkpoint and its bf16 tile copy);
+//   dir < 0: G_{last} = 0, G_{c-1} = e^{l_Q,c} G_c + C_c^T diag(E) dy_c   slot c <- G_c (bf16 tile).
+// Only the fold is sequential; the chunk products are independent, so the CTA runs as a pipeline of
+// roles joined by mbarriers:
+//   warps 0-3 (prep, thread = step t): decays of kScanPrepGroup chunks at a time (inclusive sums of
+//     dt A), then per chunk, once its tiles are in, row t of x (dy) scaled by w_t (E_t) in place;
+//   warp 8 lane 0 (issue): the tcgen05 product of each prepared chunk into one of kScanBufs TMEM
+//     buffers;
+//   warp 10 lane 0 (load): the TMA loads of the chunk tiles into a ring of NS stages, each stage
+//     refilled as soon as the product that reads it has completed;
+//   warps 4-7 (fold, thread = state row n, all 64 columns in registers): S <- e^{l_Q} S + product,
+//     then S leaves through shared memory (f32: TMA store of two 32-column boxes; bf16 tile: one
+//     bulk copy, the tile already in its global format);
+//   warp 9: zeroes the dB, dC accumulators of the gradient kernel when asked to (backward);
+//   warp 11 (dt): dt of every chunk into a ring in shared memory, kDtRing chunks ahead (kept out of
+//     the prep warps: their barriers and arrivals would wait for loads in flight).
+// No CTA waits on another.
+// NS stages: 3 when the f32 states are staged too (forward), 4 otherwise.
+constexpr int kScanBufs = 4, kDecRing = 16, kScanPrepGroup = 4, kDtRing = 8;
+constexpr int kScanThreads = 384;
+template <int NS, bool F32> struct ScanSmem {
+    static constexpr size_t kRt = (size_t)kQ * kKD * 2;            // R tile (B or C), 128 x 128 bf16
+    static constexpr size_t kStage = kRt + (size_t)kQ * kP * 2;      // then the Z tile (x or dy)
+    static constexpr size_t kF32 = (size_t)NS * kStage;             // f32 state staging, 2 boxes
+    static constexpr size_t kBf = kF32 + (F32 ? (size_t)kKD * kP * 4 : 0);  // bf16 tile staging
+    static constexpr size_t kTmp = kBf + kTileBytes;                 // prep scan scratch [4][4], l_Q [4]
+    static constexpr size_t kDecP = kTmp + 128;                      // e^{l_Q}: prep -> issue [kDecRing]
+    static constexpr size_t kDecF = kDecP + 4 * kDecRing;            // e^{l_Q}: issue -> fold [kDecRing]
+    static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128] f32
+    static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 4;   // full, scaled, prod, bfree, dt full / empty
+    static constexpr size_t kTmem = kBar + 8 * (NS + 3 * kScanBufs + 2 * kDtRing);
+    static constexpr size_t kEnd = kTmem + 16;
     static constexpr size_t kAlloc = kEnd + 1024;
-    static_assert(3 * (kAlloc + 1024) <= 233472, "three state CTAs per SM");
-    static_assert(kHS == 2, "the f32 staging uses the R tile and the two Z tiles");
+    static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of SW128 tiles");
+    static_assert(kAlloc <= 232448, "scan CTA exceeds the shared memory of one CTA");
+    // the prep role writes e^{l_Q} at most NS + kScanPrepGroup chunks ahead of the issuing thread;
+    // kScanBufs >= NS keeps every mbarrier at most one phase ahead of its waiters
+    static_assert(kScanBufs >= NS && NS + kScanPrepGroup < kDecRing, "ring sizes");
+    static_assert(kDtRing % kScanPrepGroup == 0 && kDtRing >= 2 * kScanPrepGroup, "dt ring holds two prep groups");
 };
 
-// One CTA per (chunk, batch row, group, block of kHS heads):
-//   dir > 0: Sl_c = B^T diag(w) x_h for chunk c = 0 .. nchunk-2, into slot c + 1 of `out`;
-//   dir < 0: U_c = C^T diag(E) dy_h for chunk c = 1 .. nchunk-1, into slot c - 1 of `out`
-//            (the adjoint handed from chunk c to the state leaving chunk c - 1).
-// `decay[(b H + h) nchunk + c]` receives e^{l_Q} of the chunk.
-__global__ void __launch_bounds__(kThreads, 3)
-ssd_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
-                 const __grid_constant__ CUtensorMap mOut, SsdArgs a, int nblk, int dir) {
-    using SM = StateSmem;
+template <int NS, bool F32>
+__global__ void __launch_bounds__(kScanThreads, 1)
+ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
+                const __grid_constant__ CUtensorMap mS, SsdArgs a, char* __restrict__ tiles, int dir,
+                float4* zero0, float4* zero1, size_t nzero4) {
+    using SM = ScanSmem<NS, F32>;
     char* sm = smem_base1024();
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+    uint64_t* scaled = full + NS;
+    uint64_t* prod = scaled + kScanBufs;
+    uint64_t* bfree = prod + kScanBufs;
+    uint64_t* dtfull = bfree + kScanBufs;
+    uint64_t* dtempty = dtfull + kDtRing;
+    float* dtr = reinterpret_cast<float*>(sm + SM::kDt);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-
-    int idx = blockIdx.x;
-    const int blk = idx % nblk;
-    idx /= nblk;
-    const int g = idx % a.G;
-    idx /= a.G;
-    const int b = idx % a.B;
-    const int c = idx / a.B + (dir > 0 ? 0 : 1);
-    const int slot = dir > 0 ? c + 1 : c - 1;
-    const int t0 = c * kQ;
-    const int hfirst = g * a.HpG + blk * kHS;
-    const int nh = min(kHS, a.HpG - blk * kHS);
+    float* decp = reinterpret_cast<float*>(sm + SM::kDecP);
+    float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, g = h / a.HpG;
+    const int BH = a.B * a.H;
+    const int nk = a.nchunk - 1;  // chunks with a product
+    auto chunk_of = [&](int k) { return dir > 0 ? k : a.nchunk - 1 - k; };
+    auto stage = [&](int k) { return sm + (size_t)(k % NS) * SM::kStage; };
+    auto load = [&](int k) {
+        char* st = stage(k);
+        uint64_t* bar = &full[k % NS];
+        const int t0 = chunk_of(k) * kQ;
+        mbar_arrive_expect_tx(bar, (uint32_t)SM::kStage);
+        for (int j = 0; j < kKD / 64; ++j) tma_load_4d(st + j * kQ * 128, &mR, bar, 64 * j, g, t0, b);
+        tma_load_4d(st + SM::kRt, &mZ, bar, 0, h, t0, b);
+    };
     pdl_launch_dependents();
-
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+    if (tid == 256) {
+        for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < kScanBufs; ++i) {
+            mbar_init(&scaled[i], 128);
+            mbar_init(&prod[i], 2);  // the product's commit and the issuing thread (e^{l_Q} handed on)
+            mbar_init(&bfree[i], 128);
+        }
+        for (int i = 0; i < kDtRing; ++i) {
+            mbar_init(&dtfull[i], 32);
+            mbar_init(&dtempty[i], 1);
+        }
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 128);
+    if (warp == 8) tc::tmem_alloc(tmem_slot, 64 * kScanBufs);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(kQ * kKD * 2 + nh * kQ * kP * 2));
-        for (int j = 0; j < kKD / 64; ++j) tma_load_4d(sm + SM::kR + j * kQ * 128, &mR, &bar[0], 64 * j, g, t0, b);
-        for (int j = 0; j < nh; ++j) tma_load_4d(sm + SM::kZ + j * kQ * 128, &mZ, &bar[0], 0, hfirst + j, t0, b);
-    }
-    float l[kHS], beta[kHS];
-#pragma unroll
-    for (int j = 0; j < kHS; ++j) {
-        l[j] = beta[j] = 0.0f;
-        if (j < nh) ssd_coef(a, b, hfirst + j, t0 + tid, l[j], beta[j]);
-    }
-    cta_inclusive_sum_n<kHS>(l, tmp);
-    pdl_wait();  // the previous kernel of the stream may still read what this one writes
-    if (tid == kQ - 1) {
-#pragma unroll
-        for (int j = 0; j < kHS; ++j) tmp[16 + j] = l[j];
-    }
-    __syncthreads();
-    float f[kHS];
-#pragma unroll
-    for (int j = 0; j < kHS; ++j) {
-        const float lQ2 = tmp[16 + j] * kLog2e, lt2 = l[j] * kLog2e;
-        f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] : ex2(lt2);
-        if (tid == j && j < nh) a.decay[((size_t)b * a.H + hfirst + j) * a.nchunk + c] = ex2(lQ2);
-    }
+    bool ok = true;
 
-    bool ok = mbar_wait(&bar[0], 0, a.hdr, 700);
+    if (warp < 4) {
+        // ------------------------------------------------------------------------- prep
+        constexpr int NG = kScanPrepGroup;
+        const int t = tid;
+        const float Ah = a.A[h];
+        for (int k0 = 0; k0 < nk; k0 += NG) {
+            float l[NG], beta[NG], f[NG];
 #pragma unroll
-    for (int j = 0; j < kHS; ++j)
-        if (j < nh) scale_row(sm + SM::kZ + j * kQ * 128, tid, kP, kQ, f[j]);
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && ok) {  // per head: R^T (f o Z), M = state rows (128), N = 64, K = 128 steps
-        tc::fence_after_sync();
-        for (int j = 0; j < nh; ++j)
-            tc::mma_tiles(tmem + kP * j, smem_u32(sm + SM::kR), 1, kQ, smem_u32(sm + SM::kZ + j * kQ * 128), 1, kQ,
-                          kKD, kP, kQ, 0);
-        tc::commit(&bar[1]);
-    }
-    __syncwarp();
-    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 701);
-    tc::fence_after_sync();
-    // f32 results through shared memory (head j: the R tile for j = 0, the two Z tiles for j = 1;
-    // all MMAs are complete) in the 128-byte-swizzled layout of two 32-column TMA boxes
-    for (int j = 0; j < nh; ++j) {
-        char* stage = sm + (j == 0 ? SM::kR : SM::kZ);
+            for (int j = 0; j < NG; ++j) {
+                const int k = k0 + j;
+                ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
+                l[j] = dtr[(k % kDtRing) * kQ + t] * Ah;  // a step past L has dt = 0: no decay, no input
+                beta[j] = (ex2(l[j] * kLog2e) - 1.0f) / Ah;
+            }
+            wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
+            if (t == 0) {
 #pragma unroll
-        for (int v0 = 0; v0 < kP; v0 += 16) {
-            float v[16];
-            tc::ld16(tmem + kP * j + lane_off + v0, v);
-            tc::wait_ld();
-            char* box = stage + (v0 >> 5) * (kKD * 128);
+                for (int j = 0; j < NG; ++j) mbar_arrive(&dtempty[(k0 + j) % kDtRing]);
+            }
+            if (t == kQ - 1) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int chunk = ((v0 & 31) >> 2) + k;
-                *reinterpret_cast<float4*>(box + tid * 128 + ((chunk ^ (tid & 7)) << 4)) =
-                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                for (int j = 0; j < NG; ++j) tmp[4 * NG + j] = l[j];
+            }
+            wg_sync(0);
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+                const float lQ2 = tmp[4 * NG + j] * kLog2e, lt2 = l[j] * kLog2e;
+                f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] : ex2(lt2);
+                if (t == 0) decp[(k0 + j) % kDecRing] = ex2(lQ2);
+            }
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+                const int k = k0 + j;
+                if (k >= nk) break;
+                ok = ok && mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1), a.hdr, 740);
+                char* z = stage(k) + SM::kRt;
+                uint4 raw[kP / 8];  // the whole row first: its loads overlap
+#pragma unroll
+                for (int c = 0; c < kP / 8; ++c) raw[c] = *reinterpret_cast<const uint4*>(z + tc::sw128_off(t, 8 * c, kQ));
+#pragma unroll
+                for (int c = 0; c < kP / 8; ++c) {
+                    __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw[c]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 v = __bfloat1622float2(hv[i]);
+                        hv[i] = __floats2bfloat162_rn(v.x * f[j], v.y * f[j]);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < kP / 8; ++c) *reinterpret_cast<uint4*>(z + tc::sw128_off(t, 8 * c, kQ)) = raw[c];
+                fence_proxy_async_smem();
+                mbar_arrive(&scaled[k % kScanBufs]);
             }
         }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------------------ issue
+        if (lane == 0) {
+            for (int k = 0; k < nk; ++k) {
+                const int buf = k % kScanBufs, use = k / kScanBufs;
+                ok = ok && mbar_wait(&scaled[buf], (uint32_t)(use & 1), a.hdr, 741);
+                if (k >= kScanBufs) ok = ok && mbar_wait(&bfree[buf], (uint32_t)((use - 1) & 1), a.hdr, 742);
+                tc::fence_after_sync();
+                decf[k % kDecRing] = decp[k % kDecRing];
+                if (ok)
+                    tc::mma_tiles(tmem + 64 * buf, smem_u32(stage(k)), 1, kQ, smem_u32(stage(k) + SM::kRt), 1, kQ,
+                                  kKD, kP, kQ, 0);
+                tc::commit(&prod[buf]);
+                mbar_arrive(&prod[buf]);
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------------------- load
+        if (lane == 0) {
+            for (int k = 0; k < nk && k < NS; ++k) load(k);
+            for (int k = 0; k + NS < nk; ++k) {  // the product of chunk k has read its stage
+                ok = ok && mbar_wait(&prod[k % kScanBufs], (uint32_t)((k / kScanBufs) & 1), a.hdr, 743);
+                if (ok) load(k + NS);
+            }
+        }
+    } else if (warp == 11) {
+        // --------------------------------------------------------------------------- dt
+        // one prep group (kScanPrepGroup chunks) per batch of loads: an arrival waits for every load
+        // of the thread in flight, so the loads of a group are all issued before the first one
+        constexpr int NG = kScanPrepGroup;
+        for (int k0 = 0; k0 < nk; k0 += NG) {
+            if (k0 >= kDtRing) {
+#pragma unroll
+                for (int j = 0; j < NG; ++j) {
+                    const int k = k0 + j;
+                    ok = ok && mbar_wait(&dtempty[k % kDtRing], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
+                }
+            }
+            float v[NG][kQ / 32];
+#pragma unroll
+            for (int j = 0; j < NG; ++j)
+#pragma unroll
+                for (int i = 0; i < kQ / 32; ++i) {
+                    const int k = k0 + j, tt = chunk_of(k) * kQ + lane + 32 * i;
+                    v[j][i] = k < nk && tt < a.L ? __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]) : 0.0f;
+                }
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+                const int slot = (k0 + j) % kDtRing;
+#pragma unroll
+                for (int i = 0; i < kQ / 32; ++i) dtr[slot * kQ + lane + 32 * i] = v[j][i];
+                mbar_arrive(&dtfull[slot]);
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------------------- zero
+        pdl_wait();  // the previous kernel of the stream may still read dB, dC
+        for (size_t z = (size_t)blockIdx.x * 32 + lane; z < nzero4; z += (size_t)gridDim.x * 32) {
+            zero0[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            zero1[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+    } else {
+        // ------------------------------------------------------------------------- fold
+        const int n = tid - 128, fl = n == 0;  // fl: the thread that issues the copies
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        float S[kP];
+#pragma unroll
+        for (int i = 0; i < kP; ++i) S[i] = 0.0f;
+        pdl_wait();  // the previous kernel of the stream may still read the slots
+        // S into slot c through the staging buffers (free: the copies of the previous slot have
+        // read them before the first barrier)
+        auto put = [&](int c) {
+            if (fl) bulk_wait_read_all();
+            wg_sync(1);
+            if constexpr (F32) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    char* box = sm + SM::kF32 + j * (kKD * 128);  // columns 32 j .. 32 j + 31
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<float4*>(box + n * 128 + ((i ^ (n & 7)) << 4)) =
+                            make_float4(S[32 * j + 4 * i], S[32 * j + 4 * i + 1], S[32 * j + 4 * i + 2],
+                                        S[32 * j + 4 * i + 3]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<uint4*>(sm + SM::kBf + tc::sw128_off(n, 8 * i, kKD)) = pack_bf16x8(S + 8 * i);
+            fence_proxy_async_smem();
+            wg_sync(1);
+            if (fl) {
+                if constexpr (F32) {
+                    tma_store_4d(&mS, sm + SM::kF32, 0, 0, bh, c);
+                    tma_store_4d(&mS, sm + SM::kF32 + kKD * 128, 32, 0, bh, c);
+                }
+                bulk_store(tiles + ((size_t)c * BH + bh) * kTileBytes, sm + SM::kBf, kTileBytes);
+                bulk_commit();
+            }
+        };
+        put(dir > 0 ? 0 : a.nchunk - 1);
+        for (int k = 0; k < nk; ++k) {
+            const int buf = k % kScanBufs;
+            ok = ok && mbar_wait(&prod[buf], (uint32_t)((k / kScanBufs) & 1), a.hdr, 744);
+            tc::fence_after_sync();
+            float v[kP];
+#pragma unroll
+            for (int j = 0; j < kP; j += 16) tc::ld16(tmem + 64 * buf + j + lane_off, v + j);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            mbar_arrive(&bfree[buf]);
+            const float d = decf[k % kDecRing];
+#pragma unroll
+            for (int i = 0; i < kP; ++i) S[i] = fmaf(d, S[i], v[i]);
+            put(chunk_of(k) + dir);
+        }
+        if (fl) bulk_wait_all();
     }
-    fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    if (tid == 0 && ok) {
-        for (int j = 0; j < nh; ++j) {
-            const char* stage = sm + (j == 0 ? SM::kR : SM::kZ);
-            const int bh = b * a.H + hfirst + j;
-            tma_store_4d(&mOut, stage, 0, 0, bh, slot);
-            tma_store_4d(&mOut, stage + kKD * 128, 32, 0, bh, slot);
-        }
-        bulk_commit();
-        bulk_wait_read_all();
-    }
-    __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 128);
+        tc::tmem_dealloc(tmem, 64 * kScanBufs);
     }
 }
 
@@ -202,25 +350,6 @@ __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad
     for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? __bfloat162float(src[i]) : 0.0f;
 #pragma unroll
     for (int i = 0; i < kMaxHB; ++i) dts[i * kQ + row] = v[i];
-}
-
-// Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
-__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
-
-// Inclusive prefix sum over the 128 threads of warpgroup wg (same order as cta_inclusive_sum).
-__device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
-    const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 3;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) tmp[w] = x;
-    wg_sync(wg);
-    float add = 0.0f;
-    for (int k = 0; k < w; ++k) add += tmp[k];
-    wg_sync(wg);
-    return x + add;
 }
 
 // Shared memory of the output CTA: C and B of the chunk; per warpgroup a ring of three x tiles
@@ -459,7 +588,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
 }
 
 // TMA map of the f32 state slots [nslot][B*H][N][P], boxes of 32 columns x 128 rows (128-byte
-// swizzle), written by the state kernel.
+// swizzle), written by the scan kernel.
 bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
     uint64_t dims[4] = {(uint64_t)kP, (uint64_t)kKD, (uint64_t)BH, (uint64_t)nslot};
     uint64_t str[3] = {kP * 4, (uint64_t)kKD * kP * 4, (uint64_t)BH * kKD * kP * 4};
@@ -468,18 +597,16 @@ bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
 }
 
 struct SsdFwdWs {
-    size_t decay, end;
+    size_t end;  // the workspace holds only the header
 };
-SsdFwdWs fwd_plan(const lr_desc& d) {
-    const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
+SsdFwdWs fwd_plan(const lr_desc&) {
     WsCursor cur;
     SsdFwdWs w;
-    w.decay = cur.take(sizeof(float) * d.B * d.H * nchunk);
     w.end = cur.off;
     return w;
 }
 
-SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char* ws, float* decay) {
+SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char* ws) {
     SsdArgs a{};
     a.B = (int)d.B;
     a.L = (int)d.L;
@@ -491,7 +618,6 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     a.A = in.A;
     a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
     a.ckpt = (const float*)ckpt;
-    a.decay = decay;
     a.hdr = (WsHeader*)ws;
     return a;
 }
@@ -535,8 +661,7 @@ int out_heads_per_cta(const lr_desc& d, int nchunk) {
 
 // =========================================================================================
 // Backward.  With G_c the adjoint of the state leaving chunk c (G_{last} = 0):
-//   U_c = C^T diag(E) dy_h                   (ssd_state_kernel, dir < 0)
-//   G_{c-1} = e^{l_Q, c} G_c + U_c            (state_pass_kernel, dir < 0)
+//   G_{c-1} = e^{l_Q, c} G_c + U_c,  U_c = C^T diag(E) dy_h      (ssd_scan_kernel, dir < 0)
 // and per (chunk, head), with S2 = dy x^T, Pd = S2 o Lmask, P = M o Lmask, R = Pd o M:
 //   dC += Pd B + diag(E) dy S_in^T            dB += Pd^T C + diag(w) x G^T   (summed over heads)
 //   dx  = P^T dy + diag(w) B G + D dy
@@ -1023,17 +1148,15 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
 }
 
 struct SsdBwdWs {
-    size_t decay, pdA, pdD, U, gtiles, end;
+    size_t pdA, pdD, gtiles, end;
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     const size_t tiles = (size_t)d.B * d.H * nchunk;
     WsCursor cur;
     SsdBwdWs w;
-    w.decay = cur.take(sizeof(float) * tiles);
     w.pdA = cur.take(sizeof(float) * tiles);
     w.pdD = cur.take(sizeof(float) * tiles);
-    w.U = cur.take(sizeof(float) * tiles * kKD * kP);
     w.gtiles = cur.take((size_t)kTileBytes * tiles);
     w.end = cur.off;
     return w;
@@ -1056,34 +1179,22 @@ size_t ssd_fwd_ws_bytes(const lr_desc& d) { return fwd_plan(d).end; }
 size_t ssd_fwd_flag_bytes(const lr_desc&) { return 256; }
 
 lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
-    const SsdFwdWs w = fwd_plan(d);
-    SsdArgs a = make_args(d, in, ckpt, ws, (float*)(ws + w.decay));
+    SsdArgs a = make_args(d, in, ckpt, ws);
     CUtensorMap mC, mB, mX, mY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
     char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     if (!ok) return LR_ERR_INVALID_ARG;
-    const int nblk_s = (a.HpG + kHS - 1) / kHS;
-    if (a.nchunk > 1) {
-        CUtensorMap mS;
-        if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
-        cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
-        note_launch("ssd_chunk_state");
-        const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        cudaError_t e = launch_pdl(ssd_state_kernel, dim3(grid), dim3(kThreads), StateSmem::kAlloc, st, mB, mX, mS, a,
-                                   nblk_s, +1);
-        if (e != cudaSuccess) return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
+    using ScanF = ScanSmem<3, true>;
+    cudaFuncSetAttribute(ssd_scan_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
+    note_launch("ssd_state_scan");
+    CUtensorMap mS;
+    if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
+    if (launch_pdl(ssd_scan_kernel<3, true>, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, a,
+                   stiles, +1,
+                   (float4*)nullptr, (float4*)nullptr, (size_t)0) != cudaSuccess)
+        return LR_ERR_CUDA;
     {
-        const int n4 = kKD * kP / 4;
-        const size_t total = (size_t)a.B * a.H * n4;
-        note_launch("ssd_state_pass");
-        cudaError_t e = launch_pdl(state_pass_kernel<kP>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
-                                   (float4*)ckpt, stiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, +1,
-                                   (float4*)nullptr, (float4*)nullptr, (size_t)0);
-        if (e != cudaSuccess) return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
@@ -1104,7 +1215,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
                   char* ws, cudaStream_t st) {
     const SsdBwdWs w = bwd_plan(d);
     SsdGradArgs ga{};
-    ga.a = make_args(d, in, ckpt, ws, (float*)(ws + w.decay));
+    ga.a = make_args(d, in, ckpt, ws);
     const SsdArgs& a = ga.a;
     ga.gtiles = ws + w.gtiles;
     ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
@@ -1118,32 +1229,19 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true);
     if (!ok) return LR_ERR_INVALID_ARG;
-    float* Ubuf = (float*)(ws + w.U);
-    const int nblk_s = (a.HpG + kHS - 1) / kHS;
-    if (a.nchunk > 1) {
-        CUtensorMap mU;
-        if (!map_states(&mU, Ubuf, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
-        cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem::kAlloc);
-        note_launch("ssd_chunk_state");
-        const int grid = (a.nchunk - 1) * a.B * a.G * nblk_s;
-        cudaError_t e = launch_pdl(ssd_state_kernel, dim3(grid), dim3(kThreads), StateSmem::kAlloc, st, mC, mdY, mU,
-                                   a, nblk_s, -1);
-        if (e != cudaSuccess) return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
     const int hb = grad_heads_per_cta(d, a.nchunk);
     const int nblk = (a.HpG + hb - 1) / hb;
-    ga.accumulate = nblk > 1 ? 1 : 0;  // several head blocks add into dB, dC: the pass kernel zeroes them
+    ga.accumulate = nblk > 1 ? 1 : 0;  // several head blocks add into dB, dC: the scan kernel zeroes them
     {
-        const int n4 = kKD * kP / 4;
-        const size_t total = (size_t)a.B * a.H * n4;
         const size_t nzero4 = ga.accumulate ? (size_t)d.B * d.L * d.G * kKD / 4 : 0;
-        note_launch("ssd_state_pass");
-        cudaError_t e = launch_pdl(state_pass_kernel<kP>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st,
-                                   (float4*)Ubuf, ws + w.gtiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, -1,
-                                   (float4*)gr.dBm, (float4*)gr.dCm, nzero4);
-        if (e != cudaSuccess) return LR_ERR_CUDA;
+        using ScanB = ScanSmem<4, false>;
+        cudaFuncSetAttribute(ssd_scan_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
+        note_launch("ssd_state_scan");
+        // no f32 states in this direction (the map argument is unused)
+        if (launch_pdl(ssd_scan_kernel<4, false>, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC,
+                       a,
+                       ws + w.gtiles, -1, (float4*)gr.dBm, (float4*)gr.dCm, nzero4) != cudaSuccess)
+            return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }

@@ -16,9 +16,8 @@ TOL = 2e-2
 
 SSD_CASES = [(1, 512, 4, 64, 1), (2, 300, 8, 64, 2), (1, 128, 2, 64, 1), (1, 77, 8, 64, 1),
              (1, 384, 12, 64, 1), (2, 260, 10, 64, 2), (1, 520, 40, 64, 2)]
-SSD_FWD = ("ssd_chunk_state+ssd_state_pass+ssd_chunk_out", "ssd_state_pass+ssd_chunk_out")
-SSD_BWD = ("ssd_chunk_state+ssd_state_pass+ssd_chunk_grad+ssd_param_reduce",
-           "ssd_state_pass+ssd_chunk_grad+ssd_param_reduce")
+SSD_FWD = ("ssd_state_scan+ssd_chunk_out",)
+SSD_BWD = ("ssd_state_scan+ssd_chunk_grad+ssd_param_reduce",)
 
 
 def _ssd_ref(inp):

@@ -63,10 +63,24 @@ def peaks():
                 "source": "fallback"}
 
 
-def src_sha():
+# Sources each kernel family is built from (its own file and the headers it includes): a committed
+# ncu figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "ssd": ("ssd.cu", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
+    "gla": ("gla.cu", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
+    "s6": ("s6.cu", "common.cuh", "host_common.h"),
+    "rglru": ("diag.cu", "common.cuh", "host_common.h"),
+    "rotlru": ("diag.cu", "common.cuh", "host_common.h"),
+}
+
+
+def src_sha(kernel=None):
+    """Hash of the kernel family's sources (of every source when `kernel` is None)."""
     h = hashlib.sha1()
     cdir = os.path.join(ROOT, "selective_state_space_09_b200", "csrc")
-    for n in sorted(os.listdir(cdir)):
+    fam = kernel.split("_")[0] if kernel else None
+    names = KERNEL_SOURCES.get(fam) or sorted(os.listdir(cdir))
+    for n in names:
         with open(os.path.join(cdir, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:12]
@@ -82,7 +96,7 @@ def ncu_traffic(kernel, pas=None):
     except Exception:
         return None
     e = d.get("%s@%s" % (kernel, pas)) or d.get(kernel)
-    if not e or e.get("src_sha") != src_sha():
+    if not e or e.get("src_sha") != src_sha(kernel):
         return None
     return e.get("bytes_per_launch")
 

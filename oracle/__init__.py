@@ -8,7 +8,10 @@ precision); this module only marshals numpy arrays to it.
 Every function takes numpy arrays (any float dtype; bf16 inputs must already be widened exactly,
 e.g. ``tensor.double().numpy()``) in the token-major layouts documented in ``lr_oracle.c`` and
 returns float64 arrays.  ``S`` (segment length) > 0 additionally returns the checkpointed states
-after k*S steps, k = 0..ceil(L/S)-1.
+after k*S steps, k = 0..ceil(L/S)-1.  Every forward takes an optional initial state ``h0`` (zero
+when omitted) and, with ``final=True``, also returns the state after the last step, both in the
+kind's state layout: rglru / rotlru [B, D], S6 [B, D, N], SSD [B, H, P, N], GLA [B, H, K, V].
+Results are returned as ``y``, ``(y, ck)``, ``(y, hL)`` or ``(y, ck, hL)``.
 
 Sources: the mlx-recurrence post (Apple Developer Forums thread 840535, "Current kernels" and the
 segment-checkpointing paragraph), "lrnnx: A library for Linear RNNs" (ai.info summary, Key
@@ -33,15 +36,15 @@ def load(path):
     i64, dp, ci = ctypes.c_int64, ctypes.POINTER(ctypes.c_double), ctypes.c_int
     L.orc_set_threads.argtypes = [ci]
     L.orc_get_threads.restype = ci
-    L.orc_rglru_fwd.argtypes = [i64, i64, i64, dp, dp, dp, i64, dp]
+    L.orc_rglru_fwd.argtypes = [i64, i64, i64, dp, dp, dp, i64, dp, dp, dp]
     L.orc_rglru_bwd.argtypes = [i64, i64, i64, dp, dp, dp, dp, dp]
-    L.orc_rotlru_fwd.argtypes = [i64, i64, i64, dp, dp, dp, dp, dp, i64, dp]
+    L.orc_rotlru_fwd.argtypes = [i64, i64, i64, dp, dp, dp, dp, dp, i64, dp, dp, dp]
     L.orc_rotlru_bwd.argtypes = [i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp]
-    L.orc_s6_fwd.argtypes = [i64, i64, i64, i64, ci] + [dp] * 8 + [i64, dp]
+    L.orc_s6_fwd.argtypes = [i64, i64, i64, i64, ci] + [dp] * 8 + [i64, dp, dp, dp]
     L.orc_s6_bwd.argtypes = [i64, i64, i64, i64, ci] + [dp] * 15
-    L.orc_ssd_fwd.argtypes = [i64, i64, i64, i64, i64, i64, ci] + [dp] * 8 + [i64, dp]
+    L.orc_ssd_fwd.argtypes = [i64, i64, i64, i64, i64, i64, ci] + [dp] * 8 + [i64, dp, dp, dp]
     L.orc_ssd_bwd.argtypes = [i64, i64, i64, i64, i64, i64, ci] + [dp] * 15
-    L.orc_gla_fwd.argtypes = [i64, i64, i64, i64, i64] + [dp] * 5 + [i64, dp]
+    L.orc_gla_fwd.argtypes = [i64, i64, i64, i64, i64] + [dp] * 5 + [i64, dp, dp, dp]
     L.orc_gla_bwd.argtypes = [i64, i64, i64, i64, i64] + [dp] * 9
     return L
 
@@ -79,14 +82,31 @@ def _nseg(L, S):
     return (L + S - 1) // S if S and S > 0 else 0
 
 
+def _state(h0, shape):
+    """Initial state as a contiguous float64 array of `shape` (None stays None)."""
+    if h0 is None:
+        return None
+    h0 = _f64(h0)
+    if h0.shape != tuple(shape):
+        raise ValueError("initial state has shape %s, expected %s" % (h0.shape, tuple(shape)))
+    return h0
+
+
+def _ret(y, ck, hL, S, final):
+    out = (y,) + ((ck,) if S else ()) + ((hL,) if final else ())
+    return out[0] if len(out) == 1 else out
+
+
 # ---------------------------------------------------------------------------------------- rglru
-def rglru_fwd(a, b, S=0):
+def rglru_fwd(a, b, S=0, h0=None, final=False):
     a, b = _f64(a), _f64(b)
     B, L, D = a.shape
     y = np.empty_like(a)
     ck = np.empty((_nseg(L, S), B, D)) if S else None
-    lib().orc_rglru_fwd(B, L, D, _p(a), _p(b), _p(y), int(S or 0), _p(ck))
-    return (y, ck) if S else y
+    h0 = _state(h0, (B, D))
+    hL = np.empty((B, D)) if final else None
+    lib().orc_rglru_fwd(B, L, D, _p(a), _p(b), _p(y), int(S or 0), _p(ck), _p(h0), _p(hL))
+    return _ret(y, ck, hL, S, final)
 
 
 def rglru_bwd(a, b, dy):
@@ -98,13 +118,16 @@ def rglru_bwd(a, b, dy):
 
 
 # --------------------------------------------------------------------------------------- rotlru
-def rotlru_fwd(b, g, mag, theta, S=0):
+def rotlru_fwd(b, g, mag, theta, S=0, h0=None, final=False):
     b, g, mag, theta = _f64(b), _f64(g), _f64(mag), _f64(theta)
     B, L, D = b.shape
     y = np.empty_like(b)
     ck = np.empty((_nseg(L, S), B, D)) if S else None
-    lib().orc_rotlru_fwd(B, L, D, _p(b), _p(g), _p(mag), _p(theta), _p(y), int(S or 0), _p(ck))
-    return (y, ck) if S else y
+    h0 = _state(h0, (B, D))
+    hL = np.empty((B, D)) if final else None
+    lib().orc_rotlru_fwd(B, L, D, _p(b), _p(g), _p(mag), _p(theta), _p(y), int(S or 0), _p(ck),
+                         _p(h0), _p(hL))
+    return _ret(y, ck, hL, S, final)
 
 
 def rotlru_bwd(b, g, mag, theta, dy):
@@ -118,16 +141,18 @@ def rotlru_bwd(b, g, mag, theta, dy):
 
 
 # ------------------------------------------------------------------------------------------- S6
-def s6_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0):
+def s6_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False):
     x, delta, A, Bm, Cm = map(_f64, (x, delta, A, Bm, Cm))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, D = x.shape
     N = A.shape[1]
     y = np.empty_like(x)
     ck = np.empty((_nseg(L, S), B, D, N)) if S else None
+    h0 = _state(h0, (B, D, N))
+    hL = np.empty((B, D, N)) if final else None
     lib().orc_s6_fwd(B, L, D, N, DISC[disc], _p(x), _p(delta), _p(A), _p(Bm), _p(Cm),
-                     _p(Dskip), _p(z), _p(y), int(S or 0), _p(ck))
-    return (y, ck) if S else y
+                     _p(Dskip), _p(z), _p(y), int(S or 0), _p(ck), _p(h0), _p(hL))
+    return _ret(y, ck, hL, S, final)
 
 
 def s6_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
@@ -146,16 +171,18 @@ def s6_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
 
 
 # ------------------------------------------------------------------------------------------ SSD
-def ssd_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0):
+def ssd_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False):
     x, delta, A, Bm, Cm = map(_f64, (x, delta, A, Bm, Cm))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
     y = np.empty_like(x)
     ck = np.empty((_nseg(L, S), B, H, P, N)) if S else None
+    h0 = _state(h0, (B, H, P, N))
+    hL = np.empty((B, H, P, N)) if final else None
     lib().orc_ssd_fwd(B, L, H, P, N, G, DISC[disc], _p(x), _p(delta), _p(A), _p(Bm), _p(Cm),
-                      _p(Dskip), _p(z), _p(y), int(S or 0), _p(ck))
-    return (y, ck) if S else y
+                      _p(Dskip), _p(z), _p(y), int(S or 0), _p(ck), _p(h0), _p(hL))
+    return _ret(y, ck, hL, S, final)
 
 
 def ssd_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
@@ -174,14 +201,17 @@ def ssd_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
 
 
 # ------------------------------------------------------------------------------------------ GLA
-def gla_fwd(q, k, v, g, S=0):
+def gla_fwd(q, k, v, g, S=0, h0=None, final=False):
     q, k, v, g = map(_f64, (q, k, v, g))
     B, L, H, K = q.shape
     V = v.shape[3]
     o = np.empty_like(v)
     ck = np.empty((_nseg(L, S), B, H, K, V)) if S else None
-    lib().orc_gla_fwd(B, L, H, K, V, _p(q), _p(k), _p(v), _p(g), _p(o), int(S or 0), _p(ck))
-    return (o, ck) if S else o
+    h0 = _state(h0, (B, H, K, V))
+    hL = np.empty((B, H, K, V)) if final else None
+    lib().orc_gla_fwd(B, L, H, K, V, _p(q), _p(k), _p(v), _p(g), _p(o), int(S or 0), _p(ck),
+                      _p(h0), _p(hL))
+    return _ret(o, ck, hL, S, final)
 
 
 def gla_bwd(q, k, v, g, do):

@@ -33,8 +33,13 @@
  *     B, C shared by the heads of a group and an optional z gate; GLA: o_t = S_t^T q_t.
  *
  * Checkpoints: every *_fwd may also return the state after k*S steps for k = 0..ceil(L/S)-1
- * (slot 0 is the zero initial state) -- the segment checkpoints of the mlx-recurrence post's
+ * (slot 0 is the initial state) -- the segment checkpoints of the mlx-recurrence post's
  * "segment checkpointing with recomputation during the backward pass".
+ *
+ * Initial and final state (decode and continuation): every *_fwd takes an optional initial state
+ * h0 (NULL = zero) and optionally returns the state after the last step in hL, both in the kind's
+ * state layout (rglru, rotlru [B, D]; S6 [B, D, N]; SSD [B, H, P, N]; GLA [B, H, K, V]).  Running
+ * L1 steps and then L2 steps from the returned state is the same recurrence as L1 + L2 steps.
  *
  * Layouts are row-major, last index contiguous, token-major:
  *   per-token tensors [B, L, ...]; parameters as documented per function.
@@ -121,18 +126,19 @@ static void discretise_grad(int disc, double dt, double A, double *da_ddt, doubl
 /* ------------------------------------------------------------------------------------------ */
 
 void orc_rglru_fwd(int64_t B, int64_t L, int64_t D, const double *a, const double *b, double *y,
-                   int64_t S, double *ck)
+                   int64_t S, double *ck, const double *h0, double *hL)
 {
 #pragma omp parallel for collapse(2) schedule(static) num_threads(ORC_NT)
     for (int64_t bi = 0; bi < B; ++bi)
         for (int64_t d = 0; d < D; ++d) {
-            double h = 0.0;
+            double h = h0 ? h0[bi * D + d] : 0.0;
             for (int64_t t = 0; t < L; ++t) {
                 if (ck && S > 0 && t % S == 0) ck[((t / S) * B + bi) * D + d] = h;
                 int64_t i = (bi * L + t) * D + d;
                 h = a[i] * h + b[i];
                 y[i] = h;
             }
+            if (hL) hL[bi * D + d] = h;
         }
 }
 
@@ -176,14 +182,15 @@ void orc_rglru_bwd(int64_t B, int64_t L, int64_t D, const double *a, const doubl
 /* ------------------------------------------------------------------------------------------ */
 
 void orc_rotlru_fwd(int64_t B, int64_t L, int64_t D, const double *b, const double *g,
-                    const double *mag, const double *theta, double *y, int64_t S, double *ck)
+                    const double *mag, const double *theta, double *y, int64_t S, double *ck,
+                    const double *h0, double *hL)
 {
     int64_t K = D / 2;
 #pragma omp parallel for collapse(2) schedule(static) num_threads(ORC_NT)
     for (int64_t bi = 0; bi < B; ++bi)
         for (int64_t k = 0; k < K; ++k) {
             double c = cos(theta[k]), s = sin(theta[k]);
-            double hr = 0.0, hi = 0.0;
+            double hr = h0 ? h0[bi * D + 2 * k] : 0.0, hi = h0 ? h0[bi * D + 2 * k + 1] : 0.0;
             for (int64_t t = 0; t < L; ++t) {
                 if (ck && S > 0 && t % S == 0) {
                     ck[((t / S) * B + bi) * D + 2 * k] = hr;
@@ -198,6 +205,10 @@ void orc_rotlru_fwd(int64_t B, int64_t L, int64_t D, const double *b, const doub
                 hi = ni;
                 y[i] = hr;
                 y[i + 1] = hi;
+            }
+            if (hL) {
+                hL[bi * D + 2 * k] = hr;
+                hL[bi * D + 2 * k + 1] = hi;
             }
         }
 }
@@ -273,7 +284,8 @@ void orc_rotlru_bwd(int64_t B, int64_t L, int64_t D, const double *b, const doub
 
 void orc_s6_fwd(int64_t B, int64_t L, int64_t D, int64_t N, int disc, const double *x,
                 const double *dt, const double *A, const double *Bm, const double *Cm,
-                const double *Dskip, const double *z, double *y, int64_t S, double *ck)
+                const double *Dskip, const double *z, double *y, int64_t S, double *ck,
+                const double *h0, double *hL)
 {
 #pragma omp parallel num_threads(ORC_NT)
     {
@@ -281,7 +293,7 @@ void orc_s6_fwd(int64_t B, int64_t L, int64_t D, int64_t N, int disc, const doub
 #pragma omp for collapse(2) schedule(static)
         for (int64_t bi = 0; bi < B; ++bi)
             for (int64_t d = 0; d < D; ++d) {
-                for (int64_t n = 0; n < N; ++n) h[n] = 0.0;
+                for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[(bi * D + d) * N + n] : 0.0;
                 for (int64_t t = 0; t < L; ++t) {
                     if (ck && S > 0 && t % S == 0)
                         for (int64_t n = 0; n < N; ++n)
@@ -297,6 +309,8 @@ void orc_s6_fwd(int64_t B, int64_t L, int64_t D, int64_t N, int disc, const doub
                     if (Dskip) s += Dskip[d] * xv;
                     y[i] = z ? s * z[i] * sigm(z[i]) : s;
                 }
+                if (hL)
+                    for (int64_t n = 0; n < N; ++n) hL[(bi * D + d) * N + n] = h[n];
             }
         free(h);
     }
@@ -408,7 +422,7 @@ void orc_s6_bwd(int64_t B, int64_t L, int64_t D, int64_t N, int disc, const doub
 void orc_ssd_fwd(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t Gn, int disc,
                  const double *x, const double *dt, const double *A, const double *Bm,
                  const double *Cm, const double *Dskip, const double *z, double *y, int64_t S,
-                 double *ck)
+                 double *ck, const double *h0, double *hL)
 {
     int64_t hpg = H / Gn;
 #pragma omp parallel num_threads(ORC_NT)
@@ -418,7 +432,10 @@ void orc_ssd_fwd(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t 
         for (int64_t bi = 0; bi < B; ++bi)
             for (int64_t hh = 0; hh < H; ++hh) {
                 int64_t gi = hh / hpg;
-                memset(h, 0, sizeof(double) * (size_t)(P * N));
+                if (h0)
+                    memcpy(h, h0 + (bi * H + hh) * P * N, sizeof(double) * (size_t)(P * N));
+                else
+                    memset(h, 0, sizeof(double) * (size_t)(P * N));
                 for (int64_t t = 0; t < L; ++t) {
                     if (ck && S > 0 && t % S == 0)
                         memcpy(ck + (((t / S) * B + bi) * H + hh) * P * N, h,
@@ -439,6 +456,7 @@ void orc_ssd_fwd(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t 
                         y[i] = z ? s * z[i] * sigm(z[i]) : s;
                     }
                 }
+                if (hL) memcpy(hL + (bi * H + hh) * P * N, h, sizeof(double) * (size_t)(P * N));
             }
         free(h);
     }
@@ -565,7 +583,7 @@ void orc_ssd_bwd(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t 
 
 void orc_gla_fwd(int64_t B, int64_t L, int64_t H, int64_t K, int64_t V, const double *q,
                  const double *k, const double *v, const double *g, double *o, int64_t S,
-                 double *ck)
+                 double *ck, const double *h0, double *hL)
 {
 #pragma omp parallel num_threads(ORC_NT)
     {
@@ -573,7 +591,10 @@ void orc_gla_fwd(int64_t B, int64_t L, int64_t H, int64_t K, int64_t V, const do
 #pragma omp for collapse(2) schedule(static)
         for (int64_t bi = 0; bi < B; ++bi)
             for (int64_t hh = 0; hh < H; ++hh) {
-                memset(St, 0, sizeof(double) * (size_t)(K * V));
+                if (h0)
+                    memcpy(St, h0 + (bi * H + hh) * K * V, sizeof(double) * (size_t)(K * V));
+                else
+                    memset(St, 0, sizeof(double) * (size_t)(K * V));
                 for (int64_t t = 0; t < L; ++t) {
                     if (ck && S > 0 && t % S == 0)
                         memcpy(ck + (((t / S) * B + bi) * H + hh) * K * V, St,
@@ -592,6 +613,7 @@ void orc_gla_fwd(int64_t B, int64_t L, int64_t H, int64_t K, int64_t V, const do
                         ot[j] = s;
                     }
                 }
+                if (hL) memcpy(hL + (bi * H + hh) * K * V, St, sizeof(double) * (size_t)(K * V));
             }
         free(St);
     }

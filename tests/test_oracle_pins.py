@@ -455,6 +455,112 @@ def test_prefix_and_stepwise_equivalence(orc):
         assert rel_err((h * Cm[:, t, None, :]).sum(-1), y[:, t]) < 1e-11
 
 
+# ----------------------------------------- initial / final state (decode and continuation)
+def _split_runs(orc):
+    """(name, full-run callable, state shape) for every kind on small random inputs; the callable
+    takes (slice of steps, h0) and returns (y, h_final)."""
+    rng = np.random.default_rng(41)
+    B, L = 2, 11
+    cases = []
+    a = rng.uniform(-1.1, 1.1, (B, L, 3))
+    b = rng.normal(size=(B, L, 3))
+    cases.append(("rglru", L, lambda sl, h0: orc.rglru_fwd(a[:, sl], b[:, sl], h0=h0, final=True), (B, 3)))
+    br = rng.normal(size=(B, L, 4))
+    g = rng.uniform(0.5, 1.0, (B, L, 2))
+    mag, th = rng.uniform(0.8, 1.0, 2), rng.uniform(0, 1, 2)
+    cases.append(("rotlru", L, lambda sl, h0: orc.rotlru_fwd(br[:, sl], g[:, sl], mag, th, h0=h0, final=True),
+                  (B, 4)))
+    D, N = 3, 2
+    x, z = rng.normal(size=(B, L, D)), rng.normal(size=(B, L, D))
+    dt = rng.uniform(0.05, 0.5, (B, L, D))
+    A6 = -rng.uniform(0.3, 3, (D, N))
+    B6, C6, D6 = rng.normal(size=(B, L, N)), rng.normal(size=(B, L, N)), rng.normal(size=D)
+    cases.append(("s6", L, lambda sl, h0: orc.s6_fwd(x[:, sl], dt[:, sl], A6, B6[:, sl], C6[:, sl], D6, z[:, sl],
+                                                     disc="bilinear", h0=h0, final=True), (B, D, N)))
+    H, P, Ns, G = 4, 3, 5, 2
+    xs = rng.normal(size=(B, L, H, P))
+    dts = rng.uniform(0.05, 0.5, (B, L, H))
+    As = -rng.uniform(0.3, 3, H)
+    Bs, Cs = rng.normal(size=(B, L, G, Ns)), rng.normal(size=(B, L, G, Ns))
+    Ds = rng.normal(size=H)
+    cases.append(("ssd", L, lambda sl, h0: orc.ssd_fwd(xs[:, sl], dts[:, sl], As, Bs[:, sl], Cs[:, sl], Ds, None,
+                                                      disc="zoh", h0=h0, final=True), (B, H, P, Ns)))
+    K, V = 3, 5
+    q, k = rng.normal(size=(B, L, 2, K)), rng.normal(size=(B, L, 2, K))
+    v, gg = rng.normal(size=(B, L, 2, V)), rng.uniform(0.5, 1.0, (B, L, 2))
+    cases.append(("gla", L, lambda sl, h0: orc.gla_fwd(q[:, sl], k[:, sl], v[:, sl], gg[:, sl], h0=h0, final=True),
+                  (B, 2, K, V)))
+    return cases
+
+
+def test_split_runs_compose(orc):
+    """P7 for the state interface: L1 steps, then L - L1 steps from the returned state, equals the
+    whole run (outputs and final state), for every split point and for one step at a time."""
+    for name, L, run, shape in _split_runs(orc):
+        y, hL = run(slice(0, L), None)
+        y0, hz = run(slice(0, L), np.zeros(shape))
+        assert rel_err(y0, y) == 0.0 and rel_err(hz, hL) == 0.0, name
+        for L1 in (1, 4, L - 1):
+            y1, h1 = run(slice(0, L1), None)
+            y2, h2 = run(slice(L1, L), h1)
+            assert rel_err(np.concatenate([y1, y2], axis=1), y) < REL, (name, L1)
+            assert rel_err(h2, hL) < REL, (name, L1)
+        h, ys = None, []
+        for t in range(L):
+            yt, h = run(slice(t, t + 1), h)
+            ys.append(yt)
+        assert rel_err(np.concatenate(ys, axis=1), y) < REL and rel_err(h, hL) < REL, name
+
+
+def test_initial_state_closed_forms(orc):
+    """With zero inputs the state only decays from h0: brute-force products of the per-step
+    coefficients applied to h0, read out per kind.  Non-square P x N and K x V make a transposed
+    state layout fail."""
+    rng = np.random.default_rng(43)
+    B, L = 2, 7
+    # rglru: y_t = (prod_{r<=t} a_r) h0
+    a = rng.uniform(-1.1, 1.1, (B, L, 3))
+    h0 = rng.normal(size=(B, 3))
+    y = orc.rglru_fwd(a, np.zeros((B, L, 3)), h0=h0)
+    assert rel_err(y, np.cumprod(a, axis=1) * h0[:, None]) < REL
+    # rotlru: h_t = (prod m_r) e^{i (t+1) theta} h0
+    g = rng.uniform(0.5, 1.0, (B, L, 2))
+    mag, th = rng.uniform(0.8, 1.0, 2), rng.uniform(0, 1, 2)
+    h0 = rng.normal(size=(B, 4))
+    y = orc.rotlru_fwd(np.zeros((B, L, 4)), g, mag, th, h0=h0)
+    hc = h0[:, 0::2] + 1j * h0[:, 1::2]
+    ref = np.cumprod(mag * g, axis=1) * np.exp(1j * th * np.arange(1, L + 1)[:, None]) * hc[:, None]
+    assert rel_err(y[..., 0::2], ref.real) < REL and rel_err(y[..., 1::2], ref.imag) < REL
+    # SSD: y_t[p] = sum_n C_t[n] (prod_{r<=t} e^{dt_r A}) h0[p, n]
+    H, P, N = 2, 3, 5
+    dt = rng.uniform(0.05, 0.5, (B, L, H))
+    A = -rng.uniform(0.3, 3, H)
+    Cm = rng.normal(size=(B, L, 1, N))
+    h0 = rng.normal(size=(B, H, P, N))
+    y = orc.ssd_fwd(np.zeros((B, L, H, P)), dt, A, rng.normal(size=(B, L, 1, N)), Cm, None, None, h0=h0)
+    dec = np.exp(np.cumsum(dt * A, axis=1))                       # [B, L, H]
+    ref = np.einsum("bln,bhpn,blh->blhp", Cm[:, :, 0], h0, dec)
+    assert rel_err(y, ref) < REL
+    # S6: y_t = (sum_n C_t[n] prod_r abar_r[n] h0[n]) silu(z_t)
+    D6, N6 = 2, 3
+    dt6 = rng.uniform(0.05, 0.5, (B, L, D6))
+    A6 = -rng.uniform(0.3, 3, (D6, N6))
+    C6, z6 = rng.normal(size=(B, L, N6)), rng.normal(size=(B, L, D6))
+    h0 = rng.normal(size=(B, D6, N6))
+    y = orc.s6_fwd(np.zeros((B, L, D6)), dt6, A6, rng.normal(size=(B, L, N6)), C6, None, z6, disc="zoh", h0=h0)
+    dec6 = np.exp(np.cumsum(dt6[..., None] * A6[None, None], axis=1))   # [B, L, D, N]
+    ref = np.einsum("bln,bldn,bdn->bld", C6, dec6, h0) * silu(z6)
+    assert rel_err(y, ref) < REL
+    # GLA: o_t = (prod_{r<=t} g_r) S0^T q_t
+    K, V = 3, 5
+    gg = rng.uniform(0.5, 1.0, (B, L, 2))
+    q = rng.normal(size=(B, L, 2, K))
+    S0 = rng.normal(size=(B, 2, K, V))
+    o = orc.gla_fwd(q, np.zeros((B, L, 2, K)), np.zeros((B, L, 2, V)), gg, h0=S0)
+    ref = np.einsum("blh,bhkv,blhk->blhv", np.cumprod(gg, axis=1), S0, q)
+    assert rel_err(o, ref) < REL
+
+
 # ------------------------------------------------------------------- golden fixtures
 def _golden(name):
     with open(os.path.join(GOLDEN, name)) as f:
@@ -500,6 +606,11 @@ def test_planted_mistakes_are_caught(tmp_path):
                               "St[i * V + j] = St[i * V + j] + kt[i] * vt[j];"),
         # ZOH beta = dt instead of expm1(u)/A
         "euler_beta": ("*beta = (A != 0.0) ? expm1(u) / A : dt;", "*beta = dt;"),
+        # SSD ignores its initial state
+        "ssd_h0_ignored": ("                if (h0)\n                    memcpy(h, h0 + (bi * H + hh) * P * N",
+                           "                if (0)\n                    memcpy(h, h0 + (bi * H + hh) * P * N"),
+        # rglru returns the first step's state as the final one
+        "rglru_stale_final": ("if (hL) hL[bi * D + d] = h;", "if (hL) hL[bi * D + d] = y[(bi * L) * D + d];"),
     }
     import oracle as real
     for name, (old, new) in mutants.items():
@@ -515,7 +626,8 @@ def test_planted_mistakes_are_caught(tmp_path):
             failed = 0
             for test, args in ((test_rglru_closed_form, ()), (test_rotlru_closed_form, ()),
                                (test_gla_closed_form, ()),
-                               (test_s6_closed_form_with_scipy_discretisation, ("zoh",))):
+                               (test_s6_closed_form_with_scipy_discretisation, ("zoh",)),
+                               (test_split_runs_compose, ()), (test_initial_state_closed_forms, ())):
                 try:
                     test(real, *args)
                 except AssertionError:

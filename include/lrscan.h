@@ -168,6 +168,29 @@ lr_status lr_scan_fwd(const lr_desc *desc, const lr_inputs *in, void *y, void *c
 lr_status lr_scan_bwd(const lr_desc *desc, const lr_inputs *in, const void *dy, const void *ckpt,
                       lr_grads *grads, void *ws, size_t ws_bytes, void *stream);
 
+/* Decode and continuation (forward only): advances the recurrence by desc->L steps from the
+ * state `state_in` and writes the outputs of those steps and the state after the last one.  One
+ * token per call (L = 1) is the decode step; a longer call continues a sequence.  Running L1
+ * steps and then L2 steps from the returned state is the same recurrence as L1 + L2 steps (the
+ * recurrence h_t = a_t h_{t-1} + b_t of the mlx-recurrence post, Apple Developer Forums thread
+ * 840535, "Current kernels"; one-token decode as in the mlx-mamba post, techtrendfeed repost,
+ * paragraph after Table 1).
+ *   desc        as for lr_scan_fwd; `segment` and `chunk` are ignored.  Limits of this path:
+ *               S6 N <= 32; SSD N <= 128; GLA K (desc->N) <= 128 (LR_ERR_UNSUPPORTED beyond).
+ *               SSD takes ZOH or BILINEAR and may have a z gate here.
+ *   in          per-token inputs of the L steps, [B, L, ...] as for lr_scan_fwd (contiguous)
+ *   state_in    f32 state entering the call, NULL for the zero state; layouts:
+ *                 rglru, rotlru [B, D] (rotlru re, im interleaved per pair);  S6 [B, D, N];
+ *                 SSD [B, H, N, P] (row n, column p: the layout of the checkpoint slots);
+ *                 GLA [B, H, K, V]
+ *   state_out   f32 state after the last step (written); may be the same buffer as state_in
+ *   y           outputs of the L steps (io dtype, the kind's output layout)
+ * Pointers need the alignment of their element type only (rotlru b, y: two elements).  No
+ * workspace, no checkpoint; nothing is allocated and nothing synchronises, so the call can be
+ * captured in a CUDA graph.  Returns LR_OK once the work is enqueued. */
+lr_status lr_step(const lr_desc *desc, const lr_inputs *in, const void *state_in, void *state_out,
+                  void *y, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device-side error record in `ws`.  Every
  * lr_scan_fwd / lr_scan_bwd call resets that record when it starts, so this reports the most
  * recent call that used `ws`.  LR_OK, LR_ERR_TIMEOUT or LR_ERR_DEVICE_CHECK; LR_ERR_CUDA
@@ -185,11 +208,11 @@ const char *lr_status_string(lr_status s);
  * hook off.  Records only; never synchronises. */
 void lr_set_launch_events(void *const *events, int n);
 
-/* Names of the kernels the last lr_scan_fwd / lr_scan_bwd call on this host thread launched,
+/* Names of the kernels the last lr_scan_fwd / lr_scan_bwd / lr_step call on this host thread launched,
  * separated by '+' (a fingerprint that lets tests check which code path ran). */
 const char *lr_last_dispatch(void);
 
-/* Number of kernel launches the last lr_scan_fwd / lr_scan_bwd call on this thread enqueued. */
+/* Number of kernel launches the last lr_scan_fwd / lr_scan_bwd / lr_step call on this thread enqueued. */
 int lr_last_launch_count(void);
 
 int lr_version(void);

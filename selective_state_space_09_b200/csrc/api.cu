@@ -270,6 +270,71 @@ lr_status lr_scan_bwd(const lr_desc* desc, const lr_inputs* in, const void* dy, 
     }
 }
 
+lr_status lr_step(const lr_desc* desc, const lr_inputs* in, const void* state_in, void* state_out, void* y,
+                  void* stream) {
+    begin_call();
+    if (!desc || !in || !state_out || !y) return LR_ERR_INVALID_ARG;
+    const lr_desc& d = *desc;
+    if (d.kind < LR_RGLRU || d.kind > LR_GLA) return LR_ERR_INVALID_ARG;
+    if (d.io != LR_F32 && d.io != LR_BF16) return LR_ERR_INVALID_ARG;
+    if (d.B < 1 || d.L < 1) return LR_ERR_INVALID_ARG;
+    if (d.B > (1 << 20) || d.L > (1ll << 30)) return LR_ERR_UNSUPPORTED;
+    const size_t es = (size_t)esize(d.io);
+    struct Need {
+        const void* p;
+        size_t align;
+    } need[10];
+    int nn = 0;
+    switch (d.kind) {
+        case LR_RGLRU:
+            if (d.disc != LR_DISC_NONE || d.D < 1) return LR_ERR_INVALID_ARG;
+            need[nn++] = {in->a, es};
+            need[nn++] = {in->b, es};
+            need[nn++] = {y, es};
+            break;
+        case LR_ROTLRU:
+            if (d.disc != LR_DISC_NONE || d.D < 2 || d.D % 2) return LR_ERR_INVALID_ARG;
+            need[nn++] = {in->b, 2 * es};
+            need[nn++] = {in->g, es};
+            need[nn++] = {in->mag, 4};
+            need[nn++] = {in->theta, 4};
+            need[nn++] = {y, 2 * es};
+            break;
+        case LR_S6:
+        case LR_SSD:
+            if (d.disc != LR_DISC_ZOH && d.disc != LR_DISC_BILINEAR) return LR_ERR_INVALID_ARG;
+            if (d.kind == LR_S6 && (d.D < 1 || d.N < 1)) return LR_ERR_INVALID_ARG;
+            if (d.kind == LR_SSD && (d.H < 1 || d.P < 1 || d.N < 1 || d.G < 1 || d.H % d.G))
+                return LR_ERR_INVALID_ARG;
+            need[nn++] = {in->x, es};
+            need[nn++] = {in->delta, es};
+            need[nn++] = {in->A, 4};
+            need[nn++] = {in->Bm, es};
+            need[nn++] = {in->Cm, es};
+            need[nn++] = {y, es};
+            if (d.flags & LR_HAS_DSKIP) need[nn++] = {in->Dskip, 4};
+            if (d.flags & LR_HAS_Z) need[nn++] = {in->z, es};
+            break;
+        case LR_GLA:
+            if (d.disc != LR_DISC_NONE || d.H < 1 || d.P < 1 || d.N < 1) return LR_ERR_INVALID_ARG;
+            need[nn++] = {in->q, es};
+            need[nn++] = {in->k, es};
+            need[nn++] = {in->v, es};
+            need[nn++] = {in->g, es};
+            need[nn++] = {y, es};
+            break;
+    }
+    for (int i = 0; i < nn; ++i) {
+        if (!need[i].p) return LR_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(need[i].p) % need[i].align) return LR_ERR_ALIGNMENT;
+    }
+    if ((reinterpret_cast<uintptr_t>(state_in) | reinterpret_cast<uintptr_t>(state_out)) % 4) return LR_ERR_ALIGNMENT;
+    if (!step_supported(d)) return LR_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    set_launch_stream(st);
+    return step_run(d, *in, static_cast<const float*>(state_in), static_cast<float*>(state_out), y, st);
+}
+
 lr_status lr_get_error(void* ws, void* stream, int32_t* info) {
     if (!ws) return LR_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -105,4 +105,9 @@ size_t ssd_bwd_flag_bytes(const lr_desc& d);
 lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt, const lr_grads& gr,
                   char* ws, cudaStream_t st);
 
+// decode / continuation (step.cu)
+bool step_supported(const lr_desc& d);
+lr_status step_run(const lr_desc& d, const lr_inputs& in, const float* s_in, float* s_out, void* y,
+                   cudaStream_t st);
+
 }  // namespace lrs

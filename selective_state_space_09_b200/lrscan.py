@@ -81,6 +81,8 @@ def _load():
     L.lr_set_launch_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
     L.lr_set_launch_events.restype = None
     L.lr_version.restype = ctypes.c_int
+    L.lr_step.argtypes = [pd, ctypes.POINTER(Inputs), vp, vp, vp, vp]
+    L.lr_step.restype = st
     return L
 
 
@@ -189,8 +191,8 @@ class Plan:
 
 
 # ------------------------------------------------------------------ per-kind convenience plans
-def plan_for(kind, inp, segment, disc="none", chunk=0):
-    """Build the Plan of a kind from its input tensors (shapes read from the tensors)."""
+def desc_for(kind, inp, segment=1, disc="none", chunk=0):
+    """Descriptor of a kind from its input tensors (shapes read from the tensors)."""
     if kind == "rglru":
         B, L, D = inp["a"].shape
         d = make_desc("rglru", inp["a"].dtype, B, L, D=D, segment=segment)
@@ -214,7 +216,64 @@ def plan_for(kind, inp, segment, disc="none", chunk=0):
         d = make_desc("gla", inp["q"].dtype, B, L, H=H, P=V, N=K, segment=segment, chunk=chunk)
     else:
         raise KeyError(kind)
+    return d
+
+
+def plan_for(kind, inp, segment, disc="none", chunk=0):
+    """Build the Plan of a kind from its input tensors (shapes read from the tensors)."""
+    d = desc_for(kind, inp, segment, disc, chunk)
     return Plan(d, inp[next(k for k in inp if inp[k] is not None)].device)
+
+
+# ------------------------------------------------------------------------ decode / continuation
+# per-token inputs of each kind (the rest are parameters)
+TOKEN_INPUTS = {"rglru": ("a", "b"), "rotlru": ("b", "g"), "s6": ("x", "delta", "Bm", "Cm", "z"),
+                "ssd": ("x", "delta", "Bm", "Cm", "z"), "gla": ("q", "k", "v", "g")}
+
+
+def state_shape(desc):
+    """Shape of the f32 state lr_step reads and writes (see lrscan.h)."""
+    d = desc
+    return {0: (d.B, d.D), 1: (d.B, d.D), 2: (d.B, d.D, d.N), 3: (d.B, d.H, d.N, d.P),
+            4: (d.B, d.H, d.N, d.P)}[d.kind]
+
+
+def step(desc, inp, y, state_out, state_in=None):
+    """lr_step: advance by desc.L steps from state_in (None: zero state) into state_out (may be
+    state_in), writing the steps' outputs into y."""
+    ii = Inputs(*[_ptr(inp.get(n)) for n in _IN])
+    _check(lib.lr_step(ctypes.byref(desc), ctypes.byref(ii), _ptr(state_in), _ptr(state_out), _ptr(y),
+                       _stream()), "lr_step")
+    return y
+
+
+class DecodeGraph:
+    """T one-token steps captured once in a CUDA graph; ``replay()`` runs them all.
+
+    ``seq``: the kind's inputs, token tensors time-major and contiguous, [T, B, 1, ...] (token t's
+    inputs are ``seq[name][t]``), parameters as usual; ``state``: the f32 state, advanced in place;
+    ``y``: [T, B, 1, ...] outputs.  Every replay continues from whatever ``state`` holds."""
+
+    def __init__(self, kind, seq, state, y, disc="none"):
+        toks = TOKEN_INPUTS[kind]
+        T = y.shape[0]
+        self.kind, self.T, self.state, self.y = kind, T, state, y
+        first = {n: (seq[n][0] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}
+        self.desc = desc_for(kind, first, 1, disc)
+        self.calls = [({n: (seq[n][t] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}, y[t])
+                      for t in range(T)]
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # one eager step (on scratch buffers) settles lazy initialisation
+            step(self.desc, self.calls[0][0], torch.empty_like(y[0]), state.clone(), state)
+        torch.cuda.current_stream().wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            for inp, yt in self.calls:
+                step(self.desc, inp, yt, state, state)
+
+    def replay(self):
+        self.graph.replay()
 
 
 def alloc_outputs(kind, inp):

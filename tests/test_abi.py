@@ -116,6 +116,35 @@ def test_calls_rejected_before_any_launch(L):
     assert L.last_launch_count() == 0
 
 
+def test_step_calls_rejected_before_any_launch(L):
+    """lr_step's host-side checks: missing pointers, misalignment, the limits of the step path."""
+    import torch
+    V = ctypes.c_void_p
+    d = L.make_desc("rglru", torch.float32, B=2, L=1, D=32)
+    ok = L.Inputs(a=V(0x1000), b=V(0x2000))
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(ok), None, None, V(0x3000), None) == 1  # no state_out
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(L.Inputs()), None, V(0x4000), V(0x3000), None) == 1
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(ok), V(0x1002), V(0x4000), V(0x3000), None) == 3
+    bad = L.Inputs(a=V(0x1001), b=V(0x2000))
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(bad), None, V(0x4000), V(0x3000), None) == 3
+    # rotlru b and y are read as (re, im) pairs: two elements of alignment
+    d = L.make_desc("rotlru", torch.float32, B=1, L=1, D=8)
+    ii = L.Inputs(b=V(0x1004), g=V(0x2000), mag=V(0x3000), theta=V(0x3100))
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(ii), None, V(0x4000), V(0x5000), None) == 3
+    # limits of the step path: S6 N <= 32, SSD / GLA N <= 128; SSD heads divisible by groups
+    s6in = L.Inputs(x=V(0x1000), delta=V(0x2000), A=V(0x3000), Bm=V(0x4000), Cm=V(0x5000))
+    d = L.make_desc("s6", torch.bfloat16, B=1, L=1, D=8, N=64, disc="zoh")
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(s6in), None, V(0x6000), V(0x7000), None) == 2
+    d = L.make_desc("ssd", torch.bfloat16, B=1, L=1, H=4, P=8, N=256, G=1, disc="zoh")
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(s6in), None, V(0x6000), V(0x7000), None) == 2
+    d = L.make_desc("ssd", torch.bfloat16, B=1, L=1, H=4, P=8, N=16, G=3, disc="zoh")
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(s6in), None, V(0x6000), V(0x7000), None) == 1
+    d = L.make_desc("gla", torch.bfloat16, B=1, L=1, H=2, P=8, N=16, disc="zoh")
+    gin = L.Inputs(q=V(0x1000), k=V(0x2000), v=V(0x3000), g=V(0x4000))
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(gin), None, V(0x6000), V(0x7000), None) == 1
+    assert L.last_launch_count() == 0
+
+
 def test_plan_buffers_cover_the_queried_sizes(L):
     import torch
     for d in (L.make_desc("rotlru", torch.float32, B=2, L=1000, D=64, segment=64),

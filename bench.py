@@ -412,8 +412,42 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
     }
     if e2e:
         res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
+    if world == 1:
+        res["decode"] = run_decode(kind, ai, w)
     del fl
     return res
+
+
+def run_decode(kind, ai, w, T=256, reps=20):
+    """Decode: one token per batch row per step through lr_step, T steps captured in a CUDA graph
+    (the first T tokens of the workload, state carried in place), timed over `reps` replays with
+    CUDA events.  Outside the fwd+bwd timed region; the state stays in L2, so this measures the
+    per-token latency of the step path, not HBM bandwidth."""
+    import torch
+    from selective_state_space_09_b200 import lrscan
+    toks = lrscan.TOKEN_INPUTS[kind]
+    seq = {n: (v[:, :T].transpose(0, 1).unsqueeze(2).contiguous() if n in toks and v is not None else v)
+           for n, v in ai.items()}
+    first = {n: (v[0] if n in toks and v is not None else v) for n, v in seq.items()}
+    desc = lrscan.desc_for(kind, first, 1, w.get("disc", "none"))
+    state = torch.zeros(lrscan.state_shape(desc), dtype=torch.float32, device=ai[toks[0]].device)
+    out = ai["v"] if kind == "gla" else (ai["b"] if kind in ("rglru", "rotlru") else ai["x"])
+    y = torch.empty((T, out.shape[0], 1) + tuple(out.shape[2:]), dtype=out.dtype, device=out.device)
+    graph = lrscan.DecodeGraph(kind, seq, state, y, w.get("disc", "none"))
+    for _ in range(3):
+        graph.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    us = ms * 1e3 / (T * reps)
+    B = out.shape[0]
+    return {"tokens_per_s": B / (us * 1e-6), "us_per_step": round(us, 3), "batch": B, "steps_per_graph": T,
+            "state_bytes": state.numel() * 4, "kernel": lrscan.last_dispatch() or kind + "_step"}
 
 
 def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
@@ -657,6 +691,10 @@ def main():
                                     kernel=max(r["kernels_timed"], key=lambda q: q["ms"])["kernel"]),
             "peak_mem_gib": round(r["peak_mem_bytes"] / 2 ** 30, 3), "l2": r["l2"],
         }
+        if "decode" in r:
+            d = dict(r["decode"])
+            d["tokens_per_s"] = round(d["tokens_per_s"], 1)
+            per_kind[name]["decode"] = d
     line = {
         "metric": METRIC, "value": round(h["tokens_per_s"], 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

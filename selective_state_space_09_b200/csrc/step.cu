@@ -7,7 +7,7 @@
 // The state is f32 in the kind's state layout and stays in registers across the call's steps:
 //   rglru   [B, D]        one thread per channel
 //   rotlru  [B, D]        one thread per complex pair (re, im interleaved)
-//   S6      [B, D, N]     one thread per (b, d), N <= 32 states
+//   S6      [B, D, N]     one thread per (b, d, n), N <= 32, the readout reduced by shuffles
 //   SSD     [B, H, N, P]  matrix state S[n][p] (the layout of the checkpoint slots), and
 //   GLA     [B, H, K, V]  S[k][v]: one kernel for both, since an SSD step is a GLA step with
 //                         q = C_t, k = beta_t B_t, v = x_t and forget gate abar_t; one CTA per
@@ -87,41 +87,42 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + ex2(-z * k
 
 constexpr int kS6MaxN = 32;
 
+// One thread per (b, d, n): NL lanes (a power of two >= N, at most 32) per channel, the readout
+// sum over n by butterfly shuffles within those lanes (lanes n >= N hold zero).
 template <typename T>
 __global__ void __launch_bounds__(256)
 s6_step_kernel(const T* __restrict__ x, const T* __restrict__ delta, const float* __restrict__ A,
                const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ Dskip,
                const T* __restrict__ z, T* __restrict__ y, const float* s_in, float* s_out, int B, int L, int D,
-               int N, int disc) {
-    const size_t u = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (u >= (size_t)B * D) return;
-    const int bi = (int)(u / D), d = (int)(u % D);
-    float h[kS6MaxN];
-#pragma unroll
-    for (int n = 0; n < kS6MaxN; ++n) h[n] = (n < N && s_in) ? s_in[u * N + n] : 0.0f;
-    const float Dd = Dskip ? Dskip[d] : 0.0f;
+               int N, int NL, int disc) {
+    const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t u = gtid / NL;  // channel (b, d)
+    const int n = (int)(gtid % NL);
+    const bool live = u < (size_t)B * D;  // whole groups of NL lanes share this
+    const bool act = live && n < N;
+    const int bi = live ? (int)(u / D) : 0, d = live ? (int)(u % D) : 0;
+    float h = (act && s_in) ? s_in[u * N + n] : 0.0f;
+    const float An = act ? A[(size_t)d * N + n] : 0.0f;
+    const float Dd = (live && Dskip) ? Dskip[d] : 0.0f;
     for (int t = 0; t < L; ++t) {
         const size_t i = ((size_t)bi * L + t) * D + d;
-        const float xv = IO<T>::ld(x + i), dt = IO<T>::ld(delta + i);
-        const T* Bt = Bm + ((size_t)bi * L + t) * N;
-        const T* Ct = Cm + ((size_t)bi * L + t) * N;
-        float s = 0.0f;
-#pragma unroll
-        for (int n = 0; n < kS6MaxN; ++n) {
-            if (n < N) {
-                float ab, be;
-                disc_coef(disc, dt, A[(size_t)d * N + n], ab, be);
-                h[n] = fmaf(ab, h[n], be * IO<T>::ld(Bt + n) * xv);
-                s = fmaf(IO<T>::ld(Ct + n), h[n], s);
-            }
+        float xv = 0.0f, s = 0.0f;
+        if (act) {
+            const size_t bt = ((size_t)bi * L + t) * N + n;
+            xv = IO<T>::ld(x + i);
+            float ab, be;
+            disc_coef(disc, IO<T>::ld(delta + i), An, ab, be);
+            h = fmaf(ab, h, be * IO<T>::ld(Bm + bt) * xv);
+            s = IO<T>::ld(Cm + bt) * h;
         }
-        s = fmaf(Dd, xv, s);
-        if (z) s *= silu_f(IO<T>::ld(z + i));
-        IO<T>::st(y + i, s);
+        for (int o = NL / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, NL);
+        if (live && n == 0) {
+            s = fmaf(Dd, xv, s);
+            if (z) s *= silu_f(IO<T>::ld(z + i));
+            IO<T>::st(y + i, s);
+        }
     }
-#pragma unroll
-    for (int n = 0; n < kS6MaxN; ++n)
-        if (n < N) s_out[u * N + n] = h[n];
+    if (act) s_out[u * N + n] = h;
 }
 
 // ------------------------------------------------------------------- SSD / GLA matrix state
@@ -236,12 +237,14 @@ lr_status step_impl(const lr_desc& d, const lr_inputs& in, const float* s_in, fl
             return check_launch();
         }
         case LR_S6: {
-            const size_t n = (size_t)d.B * d.D;
+            int NL = 1;
+            while (NL < d.N) NL *= 2;
+            const size_t n = (size_t)d.B * d.D * NL;
             note_launch("s6_step");
             s6_step_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
                 (const T*)in.x, (const T*)in.delta, in.A, (const T*)in.Bm, (const T*)in.Cm,
                 (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr, (d.flags & LR_HAS_Z) ? (const T*)in.z : nullptr,
-                (T*)y, s_in, s_out, B, L, (int)d.D, (int)d.N, (int)d.disc);
+                (T*)y, s_in, s_out, B, L, (int)d.D, (int)d.N, NL, (int)d.disc);
             return check_launch();
         }
         default: {

@@ -25,7 +25,7 @@ import numpy as np
 
 from . import build as _build
 
-DISC = {"none": 0, "zoh": 1, "bilinear": 2}
+DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 
 _lib = None
 

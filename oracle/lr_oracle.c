@@ -52,7 +52,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_DISC_NONE = 0, ORC_DISC_ZOH = 1, ORC_DISC_BILINEAR = 2 };
+enum { ORC_DISC_NONE = 0, ORC_DISC_ZOH = 1, ORC_DISC_BILINEAR = 2, ORC_DISC_DIRAC = 3, ORC_DISC_ZOH_EULER = 4 };
 
 static int g_threads = 0;
 
@@ -82,7 +82,14 @@ static void *xcalloc(size_t n, size_t sz)
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Discretisation (lrnnx summary, Key Contributions 2-3: ZOH and bilinear).                    */
+/* Discretisation (lrnnx summary, Key Contributions 2-3, which name ZOH, bilinear, dirac and    */
+/* asynchronous discretisation without defining them):                                         */
+/*   ZOH        abar = e^{dt A}, beta = (e^{dt A} - 1) / A   (exact zero-order hold)           */
+/*   bilinear   abar = (1 + dt A/2) / (1 - dt A/2), beta = dt / (1 - dt A/2)   (Tustin)         */
+/*   dirac      abar = e^{dt A}, beta = 1   (the input an impulse at the sample: it enters the  */
+/*              state undamped)                                                                */
+/*   ZOH-Euler  abar = e^{dt A}, beta = dt  (zero-order hold for A, Euler for B: the form the   */
+/*              selective-scan kernels the lrnnx kernels derive from use)                       */
 /* ------------------------------------------------------------------------------------------ */
 
 /* abar and beta for one (dt, A) pair.  beta multiplies B*x in the state update. */
@@ -92,6 +99,12 @@ static void discretise(int disc, double dt, double A, double *abar, double *beta
         double u = dt * A;
         *abar = exp(u);
         *beta = (A != 0.0) ? expm1(u) / A : dt;        /* limit A -> 0: beta -> dt */
+    } else if (disc == ORC_DISC_DIRAC) {
+        *abar = exp(dt * A);
+        *beta = 1.0;
+    } else if (disc == ORC_DISC_ZOH_EULER) {
+        *abar = exp(dt * A);
+        *beta = dt;
     } else {                                             /* bilinear (Tustin)        */
         double v = 1.0 - 0.5 * dt * A;
         *abar = (1.0 + 0.5 * dt * A) / v;
@@ -110,6 +123,12 @@ static void discretise_grad(int disc, double dt, double A, double *da_ddt, doubl
         *da_dA = dt * ab;
         *db_ddt = ab;
         *db_dA = (A != 0.0) ? (dt * ab - be) / A : 0.5 * dt * dt;
+    } else if (disc == ORC_DISC_DIRAC || disc == ORC_DISC_ZOH_EULER) {
+        double ab = exp(dt * A);
+        *da_ddt = A * ab;
+        *da_dA = dt * ab;
+        *db_ddt = disc == ORC_DISC_ZOH_EULER ? 1.0 : 0.0;
+        *db_dA = 0.0;
     } else {
         double v = 1.0 - 0.5 * dt * A;
         double v2 = v * v;

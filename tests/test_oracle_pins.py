@@ -34,10 +34,18 @@ def rel_err(x, ref):
 # ------------------------------------------------------------------------ independent helpers
 def scipy_disc(dt, A, method):
     """(abar, beta) of dh/dt = A h + u sampled at step dt, from scipy (matrix exponential for
-    ZOH, generalised bilinear transform with alpha = 1/2 for Tustin)."""
-    Ad, Bd, _, _, _ = cont2discrete((np.array([[A]]), np.array([[1.0]]), np.array([[1.0]]),
-                                     np.array([[0.0]])), float(dt), method=method)
-    return Ad[0, 0], Bd[0, 0]
+    ZOH, generalised bilinear transform with alpha = 1/2 for Tustin).  The two mixed schemes take
+    abar from scipy's ZOH and beta from their definition: dirac (an impulse input enters the state
+    undamped, beta = 1) and ZOH-Euler (beta from scipy's forward Euler, dt)."""
+    def c2d(m):
+        Ad, Bd, _, _, _ = cont2discrete((np.array([[A]]), np.array([[1.0]]), np.array([[1.0]]),
+                                         np.array([[0.0]])), float(dt), method=m)
+        return Ad[0, 0], Bd[0, 0]
+    if method == "dirac":
+        return c2d("zoh")[0], 1.0
+    if method == "zoh_euler":
+        return c2d("zoh")[0], c2d("euler")[1]
+    return c2d(method)
 
 
 def closed_form(a, b):
@@ -118,7 +126,7 @@ def test_rotlru_closed_form(orc):
                 assert abs(got - ref[kk * 3 - 1]) < REL * max(1.0, abs(ref).max())
 
 
-@pytest.mark.parametrize("disc", ["zoh", "bilinear"])
+@pytest.mark.parametrize("disc", ["zoh", "bilinear", "dirac", "zoh_euler"])
 def test_s6_closed_form_with_scipy_discretisation(orc, disc):
     """S6 output as the quadratic form y_t = (sum_{s<=t} sum_n C_t[n] (prod abar) beta_s B_s[n]
     x_s + D x_t) silu(z_t), with abar and beta from scipy's discretisation."""
@@ -275,7 +283,7 @@ def test_rotlru_zero_angle_is_rglru(orc):
     assert rel_err(gr["g"], mag * (r_re["a"] + r_im["a"])) < 1e-11
 
 
-@pytest.mark.parametrize("disc", ["zoh", "bilinear"])
+@pytest.mark.parametrize("disc", ["zoh", "bilinear", "dirac", "zoh_euler"])
 def test_s6_with_headwise_parameters_is_ssd(orc, disc):
     rng = np.random.default_rng(8)
     B, L, H, P, N = 2, 10, 3, 2, 4
@@ -390,7 +398,7 @@ def test_fd_rotlru(orc):
               inp, ["b", "g", "mag", "theta"], dy)
 
 
-@pytest.mark.parametrize("disc", ["zoh", "bilinear"])
+@pytest.mark.parametrize("disc", ["zoh", "bilinear", "dirac", "zoh_euler"])
 def test_fd_s6(orc, disc):
     rng = np.random.default_rng(12)
     B, L, D, N = 2, 5, 3, 2
@@ -405,7 +413,7 @@ def test_fd_s6(orc, disc):
     _fd_check(f, b, inp, ["x", "delta", "A", "B", "C", "D", "z"], dy)
 
 
-@pytest.mark.parametrize("disc", ["zoh", "bilinear"])
+@pytest.mark.parametrize("disc", ["zoh", "bilinear", "dirac", "zoh_euler"])
 def test_fd_ssd(orc, disc):
     rng = np.random.default_rng(13)
     B, L, H, P, N, G = 1, 5, 4, 2, 3, 2
@@ -611,6 +619,10 @@ def test_planted_mistakes_are_caught(tmp_path):
                            "                if (0)\n                    memcpy(h, h0 + (bi * H + hh) * P * N"),
         # rglru returns the first step's state as the final one
         "rglru_stale_final": ("if (hL) hL[bi * D + d] = h;", "if (hL) hL[bi * D + d] = y[(bi * L) * D + d];"),
+        # ZOH-Euler: the dt-dependence of beta dropped from the gradient
+        "euler_dbeta_dropped": ("*db_ddt = disc == ORC_DISC_ZOH_EULER ? 1.0 : 0.0;", "*db_ddt = 0.0;"),
+        # dirac read as an Euler input (beta = dt)
+        "dirac_as_euler": ("        *beta = 1.0;", "        *beta = dt;"),
     }
     import oracle as real
     for name, (old, new) in mutants.items():
@@ -627,7 +639,9 @@ def test_planted_mistakes_are_caught(tmp_path):
             for test, args in ((test_rglru_closed_form, ()), (test_rotlru_closed_form, ()),
                                (test_gla_closed_form, ()),
                                (test_s6_closed_form_with_scipy_discretisation, ("zoh",)),
-                               (test_split_runs_compose, ()), (test_initial_state_closed_forms, ())):
+                               (test_split_runs_compose, ()), (test_initial_state_closed_forms, ()),
+                               (test_s6_closed_form_with_scipy_discretisation, ("dirac",)),
+                               (test_fd_s6, ("zoh_euler",))):
                 try:
                     test(real, *args)
                 except AssertionError:

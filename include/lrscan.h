@@ -23,8 +23,12 @@
  *              y_t[p] = sum_n C_t[g,n] h_t[p,n] + D_h x_t[p]  (times silu(z_t[p]) if z).
  *                                                                                state [B, H, P, N]
  *   LR_GLA     S_t = g_t S_{t-1} + k_t v_t^T (K x V), o_t = S_t^T q_t.          state [B, H, K, V]
- *   disc ZOH:      abar = exp(dt A), beta = (exp(dt A) - 1) / A.
- *   disc BILINEAR: abar = (1 + dt A/2) / (1 - dt A/2), beta = dt / (1 - dt A/2).
+ *   disc ZOH:       abar = exp(dt A), beta = (exp(dt A) - 1) / A.
+ *   disc BILINEAR:  abar = (1 + dt A/2) / (1 - dt A/2), beta = dt / (1 - dt A/2).
+ *   disc DIRAC:     abar = exp(dt A), beta = 1 (the input an impulse at the sample time).
+ *   disc ZOH_EULER: abar = exp(dt A), beta = dt (zero-order hold for A, Euler for B).
+ *   (The lrnnx summary names ZOH, bilinear and dirac discretisation without defining them; the
+ *   readings above are this library's.)
  *
  * Layouts.  Row-major, last index contiguous, token-major:
  *   rglru   a, b, y, dy, da, db            [B, L, D]              io dtype
@@ -79,7 +83,13 @@ typedef enum {
 } lr_status;
 
 typedef enum { LR_RGLRU = 0, LR_ROTLRU = 1, LR_S6 = 2, LR_SSD = 3, LR_GLA = 4 } lr_kind;
-typedef enum { LR_DISC_NONE = 0, LR_DISC_ZOH = 1, LR_DISC_BILINEAR = 2 } lr_disc;
+typedef enum {
+    LR_DISC_NONE = 0,
+    LR_DISC_ZOH = 1,
+    LR_DISC_BILINEAR = 2,
+    LR_DISC_DIRAC = 3,
+    LR_DISC_ZOH_EULER = 4
+} lr_disc;
 typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
 
 /* flags */
@@ -100,7 +110,7 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * (the backward pass stores the state every S steps and recomputes inside a segment). */
 typedef struct {
     int32_t kind;      /* lr_kind  */
-    int32_t disc;      /* lr_disc  (S6 / SSD: ZOH or BILINEAR; others: NONE) */
+    int32_t disc;      /* lr_disc  (S6 / SSD: ZOH, BILINEAR, DIRAC or ZOH_EULER; others: NONE) */
     int32_t io;        /* lr_dtype of per-token tensors                         */
     uint32_t flags;    /* LR_HAS_Z | LR_HAS_DSKIP                               */
     int64_t B, L, D, H, P, N, G;

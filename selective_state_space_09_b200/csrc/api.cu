@@ -43,13 +43,13 @@ lr_status validate(const lr_desc* d) {
             return LR_OK;
         }
         case LR_S6: {
-            if (d->disc != LR_DISC_ZOH && d->disc != LR_DISC_BILINEAR) return LR_ERR_INVALID_ARG;
+            if (d->disc < LR_DISC_ZOH || d->disc > LR_DISC_ZOH_EULER) return LR_ERR_INVALID_ARG;
             if (d->D < 1 || d->N < 1) return LR_ERR_INVALID_ARG;
             if ((d->D * es) % 16 || (d->N * es) % 16) return LR_ERR_ALIGNMENT;
             return s6_supported(*d) ? LR_OK : LR_ERR_UNSUPPORTED;
         }
         case LR_SSD: {
-            if (d->disc != LR_DISC_ZOH && d->disc != LR_DISC_BILINEAR) return LR_ERR_INVALID_ARG;
+            if (d->disc < LR_DISC_ZOH || d->disc > LR_DISC_ZOH_EULER) return LR_ERR_INVALID_ARG;
             if (d->H < 1 || d->P < 1 || d->N < 1 || d->G < 1 || d->H % d->G) return LR_ERR_INVALID_ARG;
             if ((d->P * es) % 16 || (d->N * es) % 16) return LR_ERR_ALIGNMENT;
             return chunk_supported(*d) ? LR_OK : LR_ERR_UNSUPPORTED;
@@ -302,7 +302,7 @@ lr_status lr_step(const lr_desc* desc, const lr_inputs* in, const void* state_in
             break;
         case LR_S6:
         case LR_SSD:
-            if (d.disc != LR_DISC_ZOH && d.disc != LR_DISC_BILINEAR) return LR_ERR_INVALID_ARG;
+            if (d.disc < LR_DISC_ZOH || d.disc > LR_DISC_ZOH_EULER) return LR_ERR_INVALID_ARG;
             if (d.kind == LR_S6 && (d.D < 1 || d.N < 1)) return LR_ERR_INVALID_ARG;
             if (d.kind == LR_SSD && (d.H < 1 || d.P < 1 || d.N < 1 || d.G < 1 || d.H % d.G))
                 return LR_ERR_INVALID_ARG;

@@ -3,7 +3,8 @@
 // Both kinds are the recurrence S_t = e^{lam_t} S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t with a
 // scalar decay per step and head ("mlx-recurrence", Apple Developer Forums thread 840535,
 // "Current kernels": ssd_scan, gla_scan), evaluated in 128-step chunks on tcgen05 tensor cores:
-// per pass, a chunk-state kernel, an elementwise state-passing kernel and a chunk kernel.
+// per pass, the chunk states (SSD: one scan kernel; GLA: a chunk-state kernel and an elementwise
+// state-passing kernel) and a chunk kernel.
 #include "chunk_common.cuh"
 
 namespace lrs {
@@ -13,7 +14,9 @@ bool chunk_supported(const lr_desc& d) {
     if (d.io != LR_BF16) return false;
     if (d.N != kKD || (d.P != 64 && d.P != 128)) return false;
     if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
-    if (d.kind == LR_SSD && (d.disc != LR_DISC_ZOH || (d.flags & LR_HAS_Z) || d.P != 64)) return false;
+    // SSD: the decays are kept as chunk-local log sums, so abar = e^{dt A} > 0 is required (ZOH,
+    // dirac, ZOH-Euler; bilinear abar can be negative)
+    if (d.kind == LR_SSD && (d.disc == LR_DISC_BILINEAR || (d.flags & LR_HAS_Z) || d.P != 64)) return false;
     return d.L <= (1 << 28) && d.H <= 4096;
 }
 

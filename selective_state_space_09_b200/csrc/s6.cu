@@ -1,11 +1,15 @@
 // s6.cu -- selective scan S6 (time-varying diagonal A with per-step dt, B, C), forward and
-// backward, fused D skip and silu(z) gate, ZOH or bilinear discretisation (sm_100a).
+// backward, fused D skip and silu(z) gate, ZOH, bilinear, dirac or ZOH-Euler discretisation
+// (sm_100a).
 //
 // Definition ("lrnnx: A library for Linear RNNs", ai.info summary, Key Contributions 2-3: time-
-// varying layers with ZOH / bilinear discretisation inside a fused scan and output projection):
+// varying layers with ZOH / bilinear / dirac discretisation inside a fused scan and output
+// projection; the schemes are named there, the formulas below are this library's readings):
 //   per (b, d, n):  abar, beta = disc(dt_t[d], A[d,n])
 //     ZOH:       abar = exp(dt A),              beta = (exp(dt A) - 1) / A
 //     bilinear:  abar = (1 + dt A/2)/(1 - dt A/2), beta = dt / (1 - dt A/2)
+//     dirac:     abar = exp(dt A),              beta = 1
+//     ZOH-Euler: abar = exp(dt A),              beta = dt
 //   h_t[n] = abar h_{t-1}[n] + beta B_t[n] x_t,   y_t = (sum_n C_t[n] h_t[n] + D x_t) silu(z_t).
 // Segment checkpoints and recompute follow the mlx-recurrence post (Apple Developer Forums
 // thread 840535, segment checkpointing with recomputation during the backward pass).
@@ -80,7 +84,7 @@ __device__ __forceinline__ float chan_sum(float x) {
 
 struct S6Args {
     int B, L, D, S, nseg, ncb;
-    int disc;            // LR_DISC_ZOH / LR_DISC_BILINEAR
+    int disc;            // LR_DISC_ZOH / _BILINEAR / _DIRAC / _ZOH_EULER
     int has_z, has_d;
     const float* A;      // [D, N]
     const float* Dskip;  // [D]
@@ -94,20 +98,20 @@ struct S6Args {
 
 // Per-thread constants of the discretisation for its 8 states.
 struct Disc {
-    float a2[kNH];  // ZOH: A log2(e); bilinear: A / 2
+    float a2[kNH];  // bilinear: A / 2; the others (abar = e^{dt A}): A log2(e)
     float ia[kNH];  // ZOH: 1 / A
     float A[kNH];
 };
 
 template <int DISC>
 __device__ __forceinline__ void coef(const Disc& c, int j, float dt, float& ab, float& be) {
-    if (DISC == LR_DISC_ZOH) {
-        ab = ex2(dt * c.a2[j]);
-        be = (ab - 1.0f) * c.ia[j];
-    } else {
+    if (DISC == LR_DISC_BILINEAR) {
         float r = rcp(fmaf(-dt, c.a2[j], 1.0f));
         ab = fmaf(dt * c.a2[j], r, r);  // (1 + dt A/2) r
         be = dt * r;
+    } else {
+        ab = ex2(dt * c.a2[j]);
+        be = DISC == LR_DISC_ZOH ? (ab - 1.0f) * c.ia[j] : (DISC == LR_DISC_DIRAC ? 1.0f : dt);
     }
 }
 
@@ -115,7 +119,9 @@ __device__ __forceinline__ void coef(const Disc& c, int j, float dt, float& ab, 
 template <int DISC>
 __device__ __forceinline__ float beta_of(const Disc& c, int j, float dt, float ab) {
     if (DISC == LR_DISC_ZOH) return (ab - 1.0f) * c.ia[j];
-    return dt * 0.5f * (ab + 1.0f);  // dt / (1 - dt A/2) = dt (abar + 1) / 2
+    if (DISC == LR_DISC_DIRAC) return 1.0f;
+    if (DISC == LR_DISC_ZOH_EULER) return dt;
+    return dt * 0.5f * (ab + 1.0f);  // bilinear: dt / (1 - dt A/2) = dt (abar + 1) / 2
 }
 
 __device__ __forceinline__ char* smem_base() {
@@ -170,7 +176,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     for (int j = 0; j < kNH; ++j) {
         float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
         c.A[j] = A;
-        c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
+        c.a2[j] = DISC == LR_DISC_BILINEAR ? 0.5f * A : A * kLog2e;
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
@@ -276,7 +282,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     for (int j = 0; j < kNH; ++j) {
         float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
         c.A[j] = A;
-        c.a2[j] = DISC == LR_DISC_ZOH ? A * kLog2e : 0.5f * A;
+        c.a2[j] = DISC == LR_DISC_BILINEAR ? 0.5f * A : A * kLog2e;
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
@@ -394,6 +400,12 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                         if (DISC == LR_DISC_ZOH) {
                             dta = fmaf(dab, c.A[j] * ab, fmaf(w, ab, dta));
                             dA[j] = fmaf(dab, dt * ab, fmaf(w, (dt * ab - be) * c.ia[j], dA[j]));
+                        } else if (DISC == LR_DISC_ZOH_EULER) {  // d beta / d dt = 1, d beta / dA = 0
+                            dta = fmaf(dab, c.A[j] * ab, dta + w);
+                            dA[j] = fmaf(dab, dt * ab, dA[j]);
+                        } else if (DISC == LR_DISC_DIRAC) {      // beta = 1
+                            dta = fmaf(dab, c.A[j] * ab, dta);
+                            dA[j] = fmaf(dab, dt * ab, dA[j]);
                         } else {
                             const float r = 0.5f * (ab + 1.0f);  // 1 / (1 - dt A / 2)
                             const float r2 = r * r;
@@ -556,14 +568,16 @@ lr_status s6_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, cha
               make_tmap_3d(&mY, y, 2, d.D, d.L, d.B, kDB, S);
     if (!ok) return LR_ERR_INVALID_ARG;
     const int grid = a.B * a.ncb;
-    if (d.disc == LR_DISC_ZOH) {
-        set_smem(s6_fwd_kernel<LR_DISC_ZOH>, kFwdSmem);
-        note_launch("s6_fwd_zoh");
-        s6_fwd_kernel<LR_DISC_ZOH><<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
-    } else {
-        set_smem(s6_fwd_kernel<LR_DISC_BILINEAR>, kFwdSmem);
-        note_launch("s6_fwd_bilinear");
-        s6_fwd_kernel<LR_DISC_BILINEAR><<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
+    auto run = [&](auto kernel, const char* name) {
+        set_smem(kernel, kFwdSmem);
+        note_launch(name);
+        kernel<<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
+    };
+    switch (d.disc) {
+        case LR_DISC_ZOH: run(s6_fwd_kernel<LR_DISC_ZOH>, "s6_fwd_zoh"); break;
+        case LR_DISC_BILINEAR: run(s6_fwd_kernel<LR_DISC_BILINEAR>, "s6_fwd_bilinear"); break;
+        case LR_DISC_DIRAC: run(s6_fwd_kernel<LR_DISC_DIRAC>, "s6_fwd_dirac"); break;
+        default: run(s6_fwd_kernel<LR_DISC_ZOH_EULER>, "s6_fwd_zoh_euler"); break;
     }
     return check_launch();
 }
@@ -584,14 +598,16 @@ lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const vo
               make_tmap_3d(&mdZ, a.has_z ? gr.dz : gr.dx, 2, d.D, d.L, d.B, kDB, S);
     if (!ok) return LR_ERR_INVALID_ARG;
     const int grid = a.B * a.ncb;
-    if (d.disc == LR_DISC_ZOH) {
-        set_smem(s6_bwd_kernel<LR_DISC_ZOH>, kBwdSmem);
-        note_launch("s6_bwd_zoh");
-        s6_bwd_kernel<LR_DISC_ZOH><<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
-    } else {
-        set_smem(s6_bwd_kernel<LR_DISC_BILINEAR>, kBwdSmem);
-        note_launch("s6_bwd_bilinear");
-        s6_bwd_kernel<LR_DISC_BILINEAR><<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
+    auto run = [&](auto kernel, const char* name) {
+        set_smem(kernel, kBwdSmem);
+        note_launch(name);
+        kernel<<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
+    };
+    switch (d.disc) {
+        case LR_DISC_ZOH: run(s6_bwd_kernel<LR_DISC_ZOH>, "s6_bwd_zoh"); break;
+        case LR_DISC_BILINEAR: run(s6_bwd_kernel<LR_DISC_BILINEAR>, "s6_bwd_bilinear"); break;
+        case LR_DISC_DIRAC: run(s6_bwd_kernel<LR_DISC_DIRAC>, "s6_bwd_dirac"); break;
+        default: run(s6_bwd_kernel<LR_DISC_ZOH_EULER>, "s6_bwd_zoh_euler"); break;
     }
     lr_status s = check_launch();
     if (s != LR_OK) return s;

@@ -4,7 +4,8 @@
 // Recurrence per head h ("mlx-recurrence", Apple Developer Forums thread 840535, "Current
 // kernels": ssd_scan, state [B, H, Dh, N]; the chunked evaluation of the K-Search / mlx-mamba
 // post, paragraph after Table 1):
-//   S_t = e^{dt_t A_h} S_{t-1} + beta_t B_t x_t^T,  beta_t = (e^{dt_t A_h} - 1) / A_h  (ZOH)
+//   S_t = e^{dt_t A_h} S_{t-1} + beta_t B_t x_t^T,  beta_t = (e^{dt_t A_h} - 1) / A_h  (ZOH; dirac:
+//   beta_t = 1; ZOH-Euler: beta_t = dt_t -- the lrnnx summary's Key Contribution 2 names the schemes)
 //   y_t = S_t^T C_t + D_h x_t
 // With 128-step chunks, l_t the chunk-local inclusive cumulative log decay, w_t = e^{l_Q - l_t}
 // beta_t and E_t = e^{l_t}:
@@ -29,12 +30,21 @@ constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf1
 
 struct SsdArgs {
     int B, L, H, G, HpG, nchunk;  // HpG: heads per group
+    int disc;                     // LR_DISC_ZOH, LR_DISC_DIRAC or LR_DISC_ZOH_EULER
     const __nv_bfloat16* dt;      // [B, L, H]
     const float* A;               // [H]
     const float* Dskip;           // [H] or null
     const float* ckpt;            // [nchunk][B][H][N][P] f32 (state entering each chunk)
     WsHeader* hdr;
 };
+
+// beta of one step inside the sequence (lam = dt A_h): ZOH (e^{lam} - 1) / A_h, dirac 1,
+// ZOH-Euler dt.  abar = e^{lam} in all three.
+__device__ __forceinline__ float ssd_beta(int disc, float lam, float dt, float Ah) {
+    if (disc == LR_DISC_DIRAC) return 1.0f;
+    if (disc == LR_DISC_ZOH_EULER) return dt;
+    return (ex2(lam * kLog2e) - 1.0f) / Ah;
+}
 
 // Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
 __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
@@ -164,8 +174,9 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             for (int j = 0; j < NG; ++j) {
                 const int k = k0 + j;
                 ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
-                l[j] = dtr[(k % kDtRing) * kQ + t] * Ah;  // a step past L has dt = 0: no decay, no input
-                beta[j] = (ex2(l[j] * kLog2e) - 1.0f) / Ah;
+                const float dtv = dtr[(k % kDtRing) * kQ + t];  // 0 past L: no decay
+                l[j] = dtv * Ah;
+                beta[j] = chunk_of(k) * kQ + t < a.L ? ssd_beta(a.disc, l[j], dtv, Ah) : 0.0f;  // no input past L
             }
             wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
             if (t == 0) {
@@ -471,7 +482,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         if (t0 + wt < a.L) {
             const float Ah = ad[i];
             lam = dts[i * kQ + wt] * Ah;
-            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+            beta = ssd_beta(a.disc, lam, dts[i * kQ + wt], Ah);
         }
         const float lt2 = wg_inclusive_sum(lam, tmp, wg) * kLog2e;
         l2s[wt] = lt2;
@@ -614,6 +625,7 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     a.G = (int)d.G;
     a.HpG = (int)(d.H / d.G);
     a.nchunk = (int)((d.L + kQ - 1) / kQ);
+    a.disc = d.disc;
     a.dt = (const __nv_bfloat16*)in.delta;
     a.A = in.A;
     a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
@@ -669,6 +681,7 @@ int out_heads_per_cta(const lr_desc& d, int nchunk) {
 //   X = <G, S_out> = e^{l_Q} <G, S_in> + sum_s w_s x_s . (B G)_s
 //   d lam_r = sum_{t >= r} dl_t;  d beta_s = (colsum_s(R) + w_s x_s . (B G)_s) / beta_s
 //   d dt = d lam A + d beta e^{dt A};  dA_h += d lam dt + d beta (dt e^{dt A} - beta) / A;  dD_h += dy . x
+//   (ZOH; dirac: d beta / d dt = 0, ZOH-Euler: 1; neither has a d beta / dA term)
 // (rowsum_t(R) = C_t . dC_t and colsum_s(R) = B_s . dB_s restricted to the chunk's own terms;
 // here they come straight from the fp32 accumulators of M and S2.)
 // =========================================================================================
@@ -817,7 +830,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (t0 + row < a.L) {
             const float Ah = ad[i];
             lam = dts[i * kQ + row] * Ah;
-            beta = (ex2(lam * kLog2e) - 1.0f) / Ah;
+            beta = ssd_beta(a.disc, lam, dts[i * kQ + row], Ah);
         }
         const float lt = wg0_inclusive_sum(lam, tmp);
         l2s[row] = lt * kLog2e;
@@ -1074,8 +1087,10 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 const float dt_raw = dts[i * kQ + t];
                 const float ab = ex2(dt_raw * Ah * kLog2e);
                 const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
-                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(dlam * Ah + dbeta * ab);
-                dA_part = dlam * dt_raw + dbeta * (dt_raw * ab - bt) / Ah;
+                // d beta / d dt: ZOH e^{dt A}, ZOH-Euler 1, dirac 0;  d beta / dA: ZOH only
+                const float dbdt = a.disc == LR_DISC_ZOH ? ab : (a.disc == LR_DISC_ZOH_EULER ? 1.0f : 0.0f);
+                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(dlam * Ah + dbeta * dbdt);
+                dA_part = dlam * dt_raw + (a.disc == LR_DISC_ZOH ? dbeta * (dt_raw * ab - bt) / Ah : 0.0f);
             }
             const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
             if (t == 0) {

@@ -70,12 +70,13 @@ rotlru_step_kernel(const T* __restrict__ b, const T* __restrict__ g, const float
 }
 
 // --------------------------------------------------------------------------------- S6
-// abar, beta of one (dt, A) under ZOH (exact zero-order hold) or bilinear (Tustin).
+// abar, beta of one (dt, A): ZOH (exact zero-order hold), dirac (beta = 1), ZOH-Euler (beta = dt)
+// or bilinear (Tustin).
 __device__ __forceinline__ void disc_coef(int disc, float dt, float A, float& ab, float& be) {
-    if (disc == LR_DISC_ZOH) {
+    if (disc != LR_DISC_BILINEAR) {
         const float u = dt * A;
         ab = ex2(u * kLog2eS);
-        be = A != 0.0f ? expm1f(u) / A : dt;
+        be = disc == LR_DISC_ZOH ? (A != 0.0f ? expm1f(u) / A : dt) : (disc == LR_DISC_DIRAC ? 1.0f : dt);
     } else {
         const float u = 0.5f * dt * A, r = 1.0f / (1.0f - u);
         ab = (1.0f + u) * r;

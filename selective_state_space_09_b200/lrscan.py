@@ -20,7 +20,7 @@ if not os.path.exists(LIB_PATH):
                       "or __graft_entry__.build())" % LIB_PATH)
 
 KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
-DISC = {"none": 0, "zoh": 1, "bilinear": 2}
+DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 IO = {torch.float32: 0, torch.bfloat16: 1}
 HAS_Z, HAS_DSKIP = 1, 2
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks

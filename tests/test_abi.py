@@ -172,5 +172,11 @@ def test_every_gpu_test_case_passes_host_validation(L):
     for B, Lq, H, P, G in gc.SSD_CASES:
         assert _ok(L, kind="ssd", io=bf, B=B, L=Lq, H=H, P=P, N=128, G=G, segment=128, chunk=128,
                    disc="zoh", has_d=True) == 0
+    for disc in ("dirac", "zoh_euler"):
+        assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
+                   disc=disc, has_d=True) == 0
+    # bilinear abar can be negative: no log-space decays, so the chunked SSD path refuses it
+    assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
+               disc="bilinear", has_d=True) == 2
     for B, Lq, H, V in gc.GLA_CASES:
         assert _ok(L, kind="gla", io=bf, B=B, L=Lq, H=H, P=V, N=128, segment=128, chunk=128) == 0

@@ -20,10 +20,10 @@ SSD_FWD = ("ssd_state_scan+ssd_chunk_out",)
 SSD_BWD = ("ssd_state_scan+ssd_chunk_grad+ssd_param_reduce",)
 
 
-def _ssd_ref(inp):
+def _ssd_ref(inp, disc="zoh"):
     a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], None)
-    ry, rck = oracle.ssd_fwd(*a, disc="zoh", S=128)
-    rg = oracle.ssd_bwd(*a, inp["dy"], disc="zoh")
+    ry, rck = oracle.ssd_fwd(*a, disc=disc, S=128)
+    rg = oracle.ssd_bwd(*a, inp["dy"], disc=disc)
     return ry, rck, rg
 
 
@@ -44,6 +44,22 @@ def test_ssd_parity(B, L, H, P, G, wide):
     assert_close("dB", gr["dBm"], rg["B"], TOL)
     assert_close("dC", gr["dCm"], rg["C"], TOL)
     assert_close("dD", gr["dDskip"], rg["D"], TOL)
+    assert disp[0] in SSD_FWD and disp[1] in SSD_BWD
+    assert plan.device_error() == (0, 0)
+
+
+@pytest.mark.parametrize("disc", ["dirac", "zoh_euler"])
+@pytest.mark.parametrize("B,L,H,P,G", [(1, 512, 4, 64, 1), (2, 260, 10, 64, 2)])
+def test_ssd_parity_other_discretisations(B, L, H, P, G, disc):
+    """dirac (beta = 1) and ZOH-Euler (beta = dt): the same kernels with another beta and its
+    derivatives."""
+    inp = inputs.ssd(B, L, H, P, 128, G=G, seed=B * 37 + L)
+    y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc=disc, chunk=128)
+    ry, rck, rg = _ssd_ref(inp, disc)
+    assert_close("y", y, ry, TOL)
+    assert_close("ckpt", ck.transpose(-1, -2), rck, TOL)
+    for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D")):
+        assert_close(name, gr[name], rg[ref], TOL)
     assert disp[0] in SSD_FWD and disp[1] in SSD_BWD
     assert plan.device_error() == (0, 0)
 

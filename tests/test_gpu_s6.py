@@ -23,6 +23,10 @@ CASES = [
     (1, 40, 64, 32, "zoh", True, False),       # no D skip
     (1, 1, 64, 8, "zoh", True, True),          # single step
     (2, 129, 136, 64, "bilinear", True, True),
+    (2, 200, 128, 64, "dirac", True, True),    # beta = 1
+    (1, 77, 96, 16, "zoh_euler", True, True),  # beta = dt
+    (2, 129, 136, 64, "zoh_euler", False, True),
+    (1, 1, 64, 8, "dirac", True, False),
 ]
 
 

@@ -31,6 +31,8 @@ CASES = [
     ("s6", dict(B=1, L=3, D=20, N=5), "f32", "bilinear"),
     ("ssd", dict(B=2, L=5, H=4, P=40, N=32, G=2), "bf16", "zoh"),
     ("ssd", dict(B=1, L=2, H=3, P=64, N=128, G=1), "f32", "bilinear"),
+    ("s6", dict(B=2, L=4, D=32, N=16), "f32", "dirac"),
+    ("ssd", dict(B=1, L=3, H=2, P=16, N=64, G=1), "bf16", "zoh_euler"),
     ("gla", dict(B=2, L=4, H=3, K=48, V=72), "bf16", "none"),
     ("gla", dict(B=1, L=1, H=2, K=128, V=128), "f32", "none"),
 ]

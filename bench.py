@@ -414,8 +414,49 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
     if world == 1:
         res["decode"] = run_decode(kind, ai, w)
+        if kind in ("rglru", "rotlru", "s6"):
+            res["full_state"] = run_full_state(kind, ai, dy, w, plan, steps, flush)
     del fl
     return res
+
+
+def run_full_state(kind, ai, dy, w, plan, steps, flush):
+    """The same fwd+bwd step in the library's full-state mode (every step's state stored by the
+    forward, read by the backward: the design segment checkpoints replace), timed the same way;
+    reported beside the default mode's checkpoint bytes and time."""
+    import torch
+    from selective_state_space_09_b200 import lrscan
+    desc = lrscan.desc_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0))
+    desc.flags |= lrscan.FULL_STATE
+    fp = lrscan.Plan(desc, ai[lrscan.TOKEN_INPUTS[kind][0]].device)
+    y, grads = lrscan.alloc_outputs(kind, ai)
+    fl = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=y.device) if flush else None
+    for _ in range(2):
+        fp.fwd(ai, y)
+        fp.bwd(ai, dy, grads)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        if fl is not None:
+            fl.fill_(float(i))
+        ev[i][0].record()
+        fp.fwd(ai, y)
+        ev[i][1].record()
+        fp.bwd(ai, dy, grads)
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    st = fp.device_error()
+    if st != (0, 0):
+        raise RuntimeError("device error %s in the full-state run" % (st,))
+    fwd = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    bwd = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    ck_full, ck_seg = lrscan.ckpt_bytes(desc), lrscan.ckpt_bytes(plan.desc)
+    out = {"ms_fwd": round(fwd, 5), "ms_bwd": round(bwd, 5), "state_bytes": ck_full,
+           "checkpoint_bytes": ck_seg, "memory_ratio": round(ck_full / max(ck_seg, 1), 1)}
+    del fp, fl
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(kind, ai, w, T=256, reps=20):
@@ -695,6 +736,10 @@ def main():
             d = dict(r["decode"])
             d["tokens_per_s"] = round(d["tokens_per_s"], 1)
             per_kind[name]["decode"] = d
+        if "full_state" in r:
+            f = dict(r["full_state"])
+            f["time_ratio"] = round((f["ms_fwd"] + f["ms_bwd"]) / (r["ms_fwd"] + r["ms_bwd"]), 3)
+            per_kind[name]["full_state"] = f
     line = {
         "metric": METRIC, "value": round(h["tokens_per_s"], 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -95,6 +95,14 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
 /* flags */
 #define LR_HAS_Z 1u       /* S6 / SSD: multiply the readout by silu(z)   */
 #define LR_HAS_DSKIP 2u   /* S6 / SSD: add the D-skip term D * x         */
+/* Full-state mode (rglru, rotlru, S6): the forward pass checkpoints the state entering every step
+ * (the checkpoint buffer holds L states, slot t = state entering step t, as with segment 1) and
+ * the backward pass reads those states instead of recomputing them from segment checkpoints --
+ * the "original full-state" design that the mlx-recurrence post (Apple Developer Forums thread
+ * 840535, opening paragraphs) compares segment checkpoint-and-recompute against.  Outputs and
+ * gradients are those of the default mode; the memory is L / S times the checkpoint memory.  The
+ * segment length still sets the tiling.  SSD and GLA: LR_ERR_UNSUPPORTED. */
+#define LR_FULL_STATE 4u
 /* Test hook for the failure path: the tiles of the first segment never publish their carry, so
  * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
  * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
@@ -146,7 +154,8 @@ typedef struct {
  * limits, ALIGNMENT for innermost extents that are not multiples of 16 bytes). */
 lr_status lr_validate(const lr_desc *desc);
 
-/* Bytes of the checkpoint buffer: ceil(L/S) states, f32 (slot k = state after k*S steps).
+/* Bytes of the checkpoint buffer: ceil(L/S) states, f32 (slot k = state after k*S steps); L
+ * states with LR_FULL_STATE.
  * The forward pass writes it and the backward pass reads it.  0 on an invalid descriptor.
  * Layout per slot: rglru / rotlru [B, D]; s6 [B, D, N]; ssd [B, H, N, P]; gla [B, H, K, V].
  * SSD and GLA: the f32 slots are followed by a bf16 copy of every slot's per-head state blocks in

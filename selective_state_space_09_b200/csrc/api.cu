@@ -29,6 +29,8 @@ lr_status validate(const lr_desc* d) {
     if (d->io != LR_F32 && d->io != LR_BF16) return LR_ERR_INVALID_ARG;
     if (d->B < 1 || d->L < 1 || d->segment < 1) return LR_ERR_INVALID_ARG;
     if (d->B > (1 << 20) || d->L > (1ll << 30)) return LR_ERR_UNSUPPORTED;
+    if ((d->flags & LR_FULL_STATE) && d->kind != LR_RGLRU && d->kind != LR_ROTLRU && d->kind != LR_S6)
+        return LR_ERR_UNSUPPORTED;
     const int es = esize(d->io);
     switch (d->kind) {
         case LR_RGLRU:
@@ -179,7 +181,8 @@ lr_status lr_validate(const lr_desc* desc) { return validate(desc); }
 
 size_t lr_ckpt_bytes(const lr_desc* desc) {
     if (validate(desc) != LR_OK) return 0;
-    size_t nseg = (size_t)((desc->L + desc->segment - 1) / desc->segment);
+    size_t nseg = (desc->flags & LR_FULL_STATE) ? (size_t)desc->L
+                                                : (size_t)((desc->L + desc->segment - 1) / desc->segment);
     // SSD, GLA: the f32 states are followed by a bf16 copy of each in tensor-core tile order
     const size_t per = (desc->kind == LR_SSD || desc->kind == LR_GLA) ? sizeof(float) + 2 : sizeof(float);
     return nseg * state_elems(*desc) * per;

@@ -113,10 +113,12 @@ template <typename T> struct Kind<LR_ROTLRU, T> {
         IO<T>::st2(Bs + t * BW + 2 * u, make_float2(v.r, v.i));
     }
     static __device__ __forceinline__ void st_ckpt(float* p, int chan0, V v) {
-        p[chan0] = v.r;
-        p[chan0 + 1] = v.i;
+        *reinterpret_cast<float2*>(p + chan0) = make_float2(v.r, v.i);
     }
-    static __device__ __forceinline__ V ld_ckpt(const float* p, int chan0) { return {p[chan0], p[chan0 + 1]}; }
+    static __device__ __forceinline__ V ld_ckpt(const float* p, int chan0) {
+        const float2 v = *reinterpret_cast<const float2*>(p + chan0);
+        return {v.x, v.y};
+    }
     static constexpr int chans_per_unit = 2;
 };
 
@@ -221,7 +223,7 @@ __device__ __forceinline__ char* smem_base() {
 }
 
 // --------------------------------------------------------------------------------- forward
-template <int KIND, typename T>
+template <int KIND, typename T, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapY, DiagArgs a) {
@@ -238,6 +240,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     int* misc = reinterpret_cast<int*>(sm + SM::off_misc());
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr bool full = FULL;  // LR_FULL_STATE: checkpoint every step
     const int grp = tid / CB, u = tid % CB;
 
     if (tid == 0) {
@@ -310,7 +313,8 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             carry = lookback_carry(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane, act, a.hdr, 101);
         }
         pub = fmax_(tile.m, carry, tile.v);
-        if (act) K::st_ckpt(a.ckpt + ((size_t)seg * a.B + b) * a.D, unit * K::chans_per_unit, carry);
+        const size_t slot = full ? (size_t)t0g : (size_t)seg;  // state entering the segment
+        if (act) K::st_ckpt(a.ckpt + (slot * a.B + b) * a.D, unit * K::chans_per_unit, carry);
         if (lane < CB) carryS[lane] = carry;
     }
     __syncthreads();
@@ -335,6 +339,10 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             V c = U.coef(Cs, j, u);
             hh = fmax_(c, hh, K::ldb(Bs, j, u));
             K::stb(Bs, j, u, hh);
+            // full state: slot t + 1 is the state entering step t + 1 (the slot after the segment
+            // is the next segment's carry, written there)
+            if (full && j + 1 < a.S && t0g + j + 1 < a.L && unit < units)
+                K::st_ckpt(a.ckpt + ((size_t)(t0g + j + 1) * a.B + b) * a.D, unit * K::chans_per_unit, hh);
         }
     }
     fence_proxy_async_smem();
@@ -347,7 +355,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 }
 
 // -------------------------------------------------------------------------------- backward
-template <int KIND, typename T>
+template <int KIND, typename T, bool FULL>
 __global__ void __launch_bounds__(kThreads, 2)  // two tiles per SM (shared memory)
 diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapDY, const __grid_constant__ CUtensorMap mapDC,
@@ -370,6 +378,9 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = tid / CB, u = tid % CB;
+    // full state: the forward checkpointed every step, so the states are read, not recomputed (b
+    // is not needed)
+    constexpr bool full = FULL;
 
     if (tid == 0) {
         unsigned int tk = take_ticket(a.hdr, 1);
@@ -388,9 +399,9 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int t0g = seg * a.S;
     // coefficients and b (the forward recompute) on bar[0], dy (the adjoint) on bar[1]
     if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(a.S * (K::CW + K::BW) * sizeof(T)));
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(a.S * (K::CW + (full ? 0 : K::BW)) * sizeof(T)));
         tma_load_3d(Cs, &mapC, &bar[0], cb * K::CW, t0g, b);
-        tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
+        if (!full) tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
         mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
         tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
     }
@@ -404,7 +415,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     bool have = false;
     if (warp == 0) have = early_carry(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
-    if (tid < CB) {
+    if (tid < CB && !full) {
         V c0 = zero_of(V{});
         if (unit < units)
             c0 = K::ld_ckpt(a.ckpt + ((size_t)seg * a.B + b) * a.D, unit * K::chans_per_unit);
@@ -416,35 +427,41 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int n = max(j1 - j0, 0);
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 200);
 
-    // forward aggregate of the group
-    {
-        V P = one_of(V{}), h = zero_of(V{});
-        if (ok)
-            for (int j = j0; j < j1; ++j) {
-                V c = U.coef(Cs, j, u);
-                P = mulx(c, P);
-                h = fmax_(c, h, K::ldb(Bs, j, u));
-            }
-        aggF[grp * CB + u] = {P, h};
-    }
-    __syncthreads();
-    // states of the group, from the segment checkpoint, kept in registers
-    V hin = carryS[u];
-    for (int g = 0; g < grp; ++g) {
-        Agg<V> ag = aggF[g * CB + u];
-        hin = fmax_(ag.m, hin, ag.v);
-    }
-    V hreg[SPG];
-    {
-        V h = hin;
+    // state entering each step of the group, in registers: recomputed from the segment
+    // checkpoint, or (full state) read from that step's checkpoint slot
+    V hprev[SPG];
+    if (!full) {
+        // forward aggregate of the group
+        {
+            V P = one_of(V{}), h = zero_of(V{});
+            if (ok)
+                for (int j = j0; j < j1; ++j) {
+                    V c = U.coef(Cs, j, u);
+                    P = mulx(c, P);
+                    h = fmax_(c, h, K::ldb(Bs, j, u));
+                }
+            aggF[grp * CB + u] = {P, h};
+        }
+        __syncthreads();
+        V h = carryS[u];
+        for (int g = 0; g < grp; ++g) {
+            Agg<V> ag = aggF[g * CB + u];
+            h = fmax_(ag.m, h, ag.v);
+        }
 #pragma unroll
         for (int j = 0; j < SPG; ++j) {
+            hprev[j] = h;
             if (j < n) {
                 V c = U.coef(Cs, j0 + j, u);
                 h = fmax_(c, h, K::ldb(Bs, j0 + j, u));
             }
-            hreg[j] = h;
         }
+    } else {
+#pragma unroll
+        for (int j = 0; j < SPG; ++j)
+            hprev[j] = (j < n && unit < units)
+                           ? K::ld_ckpt(a.ckpt + ((size_t)(t0g + j0 + j) * a.B + b) * a.D, unit * K::chans_per_unit)
+                           : zero_of(V{});
     }
     // reverse aggregate of the group: outgoing carry = v + m * incoming
     ok = mbar_wait(&bar[1], 0, a.hdr, 202) && ok;
@@ -507,7 +524,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         if (jj < n && ok) {
             const int j = j0 + jj;
             V G = addx(K::ldb(Ds, j, u), r);
-            V hp = jj > 0 ? hreg[jj > 0 ? jj - 1 : 0] : hin;
+            const V hp = hprev[jj];
             if constexpr (KIND == LR_RGLRU) {
                 float c = IO<T>::ld(Cs + j * K::CW + u);
                 IO<T>::st(Ds + j * K::BW + u, G);       // db
@@ -623,7 +640,7 @@ DiagWs ws_plan(const lr_desc& d, bool bwd) {
     return w;
 }
 
-template <int KIND, typename T, bool BWD>
+template <int KIND, typename T, bool BWD, bool FULL>
 void set_smem_attr(const void* fn) {
     static bool done = false;  // per instantiation
     if (!done) {
@@ -650,8 +667,12 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
     DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
                (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                nullptr};
-    auto fn = diag_fwd_kernel<KIND, T>;
-    set_smem_attr<KIND, T, false>((const void*)fn);
+    const bool full = (d.flags & LR_FULL_STATE) != 0;
+    auto fn = full ? diag_fwd_kernel<KIND, T, true> : diag_fwd_kernel<KIND, T, false>;
+    if (full)
+        set_smem_attr<KIND, T, false, true>((const void*)fn);
+    else
+        set_smem_attr<KIND, T, false, false>((const void*)fn);
     note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : "rotlru_fwd_tile");
     fn<<<g.tiles, kThreads, Smem<KIND, T, false>::total(), st>>>(mC, mB, mY, a);
     return check_launch();
@@ -677,8 +698,12 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
     DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
                (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                w.partial ? (float2*)(ws + w.partial) : nullptr};
-    auto fn = diag_bwd_kernel<KIND, T>;
-    set_smem_attr<KIND, T, true>((const void*)fn);
+    const bool full = (d.flags & LR_FULL_STATE) != 0;
+    auto fn = full ? diag_bwd_kernel<KIND, T, true> : diag_bwd_kernel<KIND, T, false>;
+    if (full)
+        set_smem_attr<KIND, T, true, true>((const void*)fn);
+    else
+        set_smem_attr<KIND, T, true, false>((const void*)fn);
     note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : "rotlru_bwd_tile");
     fn<<<g.tiles, kThreads, Smem<KIND, T, true>::total(), st>>>(mC, mB, mDY, mDC, mDB, a);
     lr_status s = check_launch();

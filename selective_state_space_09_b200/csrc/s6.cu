@@ -88,7 +88,7 @@ struct S6Args {
     int has_z, has_d;
     const float* A;      // [D, N]
     const float* Dskip;  // [D]
-    float* ckpt;         // [nseg, B, D, N]
+    float* ckpt;         // [nseg, B, D, N] (full state: [L, B, D, N])
     WsHeader* hdr;
     float* pdB;          // [ncb, B, L, N]
     float* pdC;          // [ncb, B, L, N]
@@ -138,7 +138,7 @@ constexpr size_t kTileBC = size_t(kMaxS) * kN * 2;   // [S][16] bf16
 constexpr size_t kFwdStage = 3 * kTileDT + 2 * kTileBC;
 constexpr size_t kFwdSmem = 128 + 2 * kFwdStage + 128;
 
-template <int DISC>
+template <int DISC, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mB,
@@ -193,7 +193,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             issue(k + 1, s ^ 1);
         }
         ok = ok && mbar_wait(&bar[s], (k >> 1) & 1, a.hdr, 300);
-        if (dok) {
+        if (dok && !FULL) {
             float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + part * kNH;
 #pragma unroll
             for (int j = 0; j < kNH; ++j) ck[j] = h[j];
@@ -210,6 +210,12 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                 float Bv[kNH], Cv[kNH];
                 ldn(Bs + t * kN + part * kNH, Bv);
                 ldn(Cs + t * kN + part * kNH, Cv);
+                if (FULL && dok) {  // the state entering step k S + t
+                    float4* ck = reinterpret_cast<float4*>(
+                        a.ckpt + ((((size_t)k * a.S + t) * a.B + b) * a.D + d) * kN + part * kNH);
+                    ck[0] = make_float4(h[0], h[1], h[2], h[3]);
+                    ck[1] = make_float4(h[4], h[5], h[6], h[7]);
+                }
                 float sacc = 0.0f;
 #pragma unroll
                 for (int j = 0; j < kNH; ++j) {
@@ -249,7 +255,7 @@ constexpr size_t kOffRed = kOffBnd + kBndBytes;
 constexpr size_t kRedBytes = size_t(kWarps) * kSub * 2 * kN * 4;  // per-warp dB / dC of one sub-block
 constexpr size_t kBwdSmem = kOffRed + kRedBytes + 128;
 
-template <int DISC>
+template <int DISC, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mDY,
@@ -312,12 +318,12 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         {
             const float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + (dok ? d : 0)) * kN + part * kNH;
 #pragma unroll
-            for (int j = 0; j < kNH; ++j) h[j] = dok ? ck[j] : 0.0f;
+            for (int j = 0; j < kNH; ++j) h[j] = (dok && !FULL) ? ck[j] : 0.0f;
         }
         ok = ok && mbar_wait(&bar[0], phase, a.hdr, 400);
         const int nsb = (nt + kSub - 1) / kSub;
-        // (A) segment forward, keeping sub-block boundary states
-        for (int sb = 0; sb < nsb; ++sb) {
+        // (A) segment forward, keeping sub-block boundary states (not with the full state)
+        for (int sb = 0; sb < (FULL ? 0 : nsb); ++sb) {
             float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
 #pragma unroll
             for (int j = 0; j < kNH; ++j) bp[j] = h[j];
@@ -339,14 +345,43 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             const int tb = sb * kSub;
             const int n = min(kSub, nt - tb);
             float h0[kNH], hr[kSub][kNH], ar[kSub][kNH];
-            {
+            if constexpr (!FULL) {
                 const float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
 #pragma unroll
                 for (int j = 0; j < kNH; ++j) h0[j] = h[j] = bp[j];
+            } else {  // the full state: the state entering every step of the sub-block is stored
+                float hs[kSub][kNH];
+#pragma unroll
+                for (int i = 0; i < kSub; ++i) {
+                    const float4* ck = reinterpret_cast<const float4*>(
+                        a.ckpt + ((((size_t)t0 + tb + i) * a.B + b) * a.D + (dok ? d : 0)) * kN + part * kNH);
+                    const float4 v0 = (i < n && dok) ? ck[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 v1 = (i < n && dok) ? ck[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    hs[i][0] = v0.x; hs[i][1] = v0.y; hs[i][2] = v0.z; hs[i][3] = v0.w;
+                    hs[i][4] = v1.x; hs[i][5] = v1.y; hs[i][6] = v1.z; hs[i][7] = v1.w;
+                }
+#pragma unroll
+                for (int j = 0; j < kNH; ++j) h0[j] = hs[0][j];
+#pragma unroll
+                for (int i = 0; i < kSub; ++i) {  // h after step i from the state entering it
+                    if (i < n) {
+                        const int t = tb + i;
+                        const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                        float Bv[kNH];
+                        ldn(Bs + t * kN + part * kNH, Bv);
+#pragma unroll
+                        for (int j = 0; j < kNH; ++j) {
+                            float ab, be;
+                            coef<DISC>(c, j, dt, ab, be);
+                            hr[i][j] = fmaf(ab, hs[i][j], be * (Bv[j] * xv));
+                            ar[i][j] = ab;
+                        }
+                    }
+                }
             }
 #pragma unroll
             for (int i = 0; i < kSub; ++i) {
-                if (i < n) {
+                if (i < n && !FULL) {
                     const int t = tb + i;
                     const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
                     float Bv[kNH];
@@ -573,11 +608,23 @@ lr_status s6_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, cha
         note_launch(name);
         kernel<<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
     };
+    // LR_FULL_STATE: the state entering every step is checkpointed (compile-time variant)
+    const bool full = (d.flags & LR_FULL_STATE) != 0;
     switch (d.disc) {
-        case LR_DISC_ZOH: run(s6_fwd_kernel<LR_DISC_ZOH>, "s6_fwd_zoh"); break;
-        case LR_DISC_BILINEAR: run(s6_fwd_kernel<LR_DISC_BILINEAR>, "s6_fwd_bilinear"); break;
-        case LR_DISC_DIRAC: run(s6_fwd_kernel<LR_DISC_DIRAC>, "s6_fwd_dirac"); break;
-        default: run(s6_fwd_kernel<LR_DISC_ZOH_EULER>, "s6_fwd_zoh_euler"); break;
+        case LR_DISC_ZOH:
+            run(full ? s6_fwd_kernel<LR_DISC_ZOH, true> : s6_fwd_kernel<LR_DISC_ZOH, false>, "s6_fwd_zoh");
+            break;
+        case LR_DISC_BILINEAR:
+            run(full ? s6_fwd_kernel<LR_DISC_BILINEAR, true> : s6_fwd_kernel<LR_DISC_BILINEAR, false>,
+                "s6_fwd_bilinear");
+            break;
+        case LR_DISC_DIRAC:
+            run(full ? s6_fwd_kernel<LR_DISC_DIRAC, true> : s6_fwd_kernel<LR_DISC_DIRAC, false>, "s6_fwd_dirac");
+            break;
+        default:
+            run(full ? s6_fwd_kernel<LR_DISC_ZOH_EULER, true> : s6_fwd_kernel<LR_DISC_ZOH_EULER, false>,
+                "s6_fwd_zoh_euler");
+            break;
     }
     return check_launch();
 }
@@ -603,11 +650,22 @@ lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const vo
         note_launch(name);
         kernel<<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
     };
+    const bool full = (d.flags & LR_FULL_STATE) != 0;  // the states are read, not recomputed
     switch (d.disc) {
-        case LR_DISC_ZOH: run(s6_bwd_kernel<LR_DISC_ZOH>, "s6_bwd_zoh"); break;
-        case LR_DISC_BILINEAR: run(s6_bwd_kernel<LR_DISC_BILINEAR>, "s6_bwd_bilinear"); break;
-        case LR_DISC_DIRAC: run(s6_bwd_kernel<LR_DISC_DIRAC>, "s6_bwd_dirac"); break;
-        default: run(s6_bwd_kernel<LR_DISC_ZOH_EULER>, "s6_bwd_zoh_euler"); break;
+        case LR_DISC_ZOH:
+            run(full ? s6_bwd_kernel<LR_DISC_ZOH, true> : s6_bwd_kernel<LR_DISC_ZOH, false>, "s6_bwd_zoh");
+            break;
+        case LR_DISC_BILINEAR:
+            run(full ? s6_bwd_kernel<LR_DISC_BILINEAR, true> : s6_bwd_kernel<LR_DISC_BILINEAR, false>,
+                "s6_bwd_bilinear");
+            break;
+        case LR_DISC_DIRAC:
+            run(full ? s6_bwd_kernel<LR_DISC_DIRAC, true> : s6_bwd_kernel<LR_DISC_DIRAC, false>, "s6_bwd_dirac");
+            break;
+        default:
+            run(full ? s6_bwd_kernel<LR_DISC_ZOH_EULER, true> : s6_bwd_kernel<LR_DISC_ZOH_EULER, false>,
+                "s6_bwd_zoh_euler");
+            break;
     }
     lr_status s = check_launch();
     if (s != LR_OK) return s;

@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
 DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 IO = {torch.float32: 0, torch.bfloat16: 1}
-HAS_Z, HAS_DSKIP = 1, 2
+HAS_Z, HAS_DSKIP, FULL_STATE = 1, 2, 4
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
 TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
 STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
@@ -178,9 +178,9 @@ class Plan:
         return int(s), int(info.value)
 
     def ckpt_view(self):
-        """The checkpoint buffer as an f32 tensor of ceil(L/S) states."""
+        """The checkpoint buffer as an f32 tensor of ceil(L/S) states (L with FULL_STATE)."""
         d = self.desc
-        nseg = (d.L + d.segment - 1) // d.segment
+        nseg = d.L if d.flags & FULL_STATE else (d.L + d.segment - 1) // d.segment
         shapes = {0: (nseg, d.B, d.D), 1: (nseg, d.B, d.D), 2: (nseg, d.B, d.D, d.N),
                   3: (nseg, d.B, d.H, d.N, d.P), 4: (nseg, d.B, d.H, d.N, d.P)}
         shp = shapes[d.kind]

@@ -34,8 +34,9 @@ def run_gpu(kind, inp, segment, disc="none", chunk=0, flags=0):
     from selective_state_space_09_b200 import lrscan
     g = gpu_inputs(inp)
     dy = g.pop("dy")
-    plan = lrscan.plan_for(kind, g, segment, disc, chunk)
-    plan.desc.flags |= flags
+    desc = lrscan.desc_for(kind, g, segment, disc, chunk)
+    desc.flags |= flags  # before the Plan sizes its buffers (LR_FULL_STATE changes the checkpoint)
+    plan = lrscan.Plan(desc, "cuda")
     y, grads = lrscan.alloc_outputs(kind, g)
     plan.fwd(g, y)
     fwd_dispatch = lrscan.last_dispatch()

@@ -120,3 +120,36 @@ def test_rotlru_full_size_sampled():
         assert_close("dg[%d]" % k, gr["dg"][:, :, k:k + 1], rg["g"], 1e-5)
         assert_close("dmag[%d]" % k, gr["dmag"][k:k + 1], rg["mag"], 1e-5)
         assert_close("dtheta[%d]" % k, gr["dtheta"][k:k + 1], rg["theta"], 1e-5)
+
+
+@pytest.mark.parametrize("kind,B,L,D,S,io", [("rglru", 2, 700, 96, 128, "f32"), ("rotlru", 2, 600, 64, 256, "f32"),
+                                           ("rotlru", 1, 333, 64, 64, "bf16")])
+def test_full_state_mode(kind, B, L, D, S, io):
+    """LR_FULL_STATE: the checkpoint holds the state entering every step (the oracle's segment-1
+    checkpoints) and the backward reads them.  Outputs equal the default mode's bitwise; the
+    gradients agree to fp32 rounding (the default backward rebuilds each time group's entering
+    state by folding group aggregates, while the full state stores the forward's sequential value
+    of the same quantity) and match the oracle."""
+    from selective_state_space_09_b200 import lrscan
+    inp = (inputs.rglru if kind == "rglru" else inputs.rotlru)(B, L, D, seed=L, io=io)
+    y0, _, g0, _, _ = run_gpu(kind, inp, S)
+    y1, ck, g1, plan, disp = run_gpu(kind, inp, S, flags=lrscan.FULL_STATE)
+    assert ck.shape[0] == L
+    if kind == "rglru":
+        _, rck = oracle.rglru_fwd(inp["a"], inp["b"], S=1)
+    else:
+        _, rck = oracle.rotlru_fwd(inp["b"], inp["g"], inp["mag"], inp["theta"], S=1)
+    assert_close("full-state ckpt", ck, rck, max(TOL[inp["b"].dtype], 1e-5))
+    assert torch.equal(y0, y1)
+    tol = TOL[inp["b"].dtype]
+    for k in g0:
+        assert_close(k + " (full vs default)", g1[k], to64(g0[k]), 1e-6 if io == "f32" else tol)
+    if kind == "rglru":
+        rg = oracle.rglru_bwd(inp["a"], inp["b"], inp["dy"])
+        pairs = (("da", "a"), ("db", "b"))
+    else:
+        rg = oracle.rotlru_bwd(inp["b"], inp["g"], inp["mag"], inp["theta"], inp["dy"])
+        pairs = (("db", "b"), ("dg", "g"), ("dmag", "mag"), ("dtheta", "theta"))
+    for k, r in pairs:
+        assert_close(k, g1[k], rg[r], tol)
+    assert plan.device_error() == (0, 0)

@@ -98,3 +98,21 @@ def test_s6_full_size_sampled(disc):
     _, _, rg = _oracle(sub, disc, w["segment"])
     assert_close("dB[b=0]", gr["dBm"][0:1], rg["B"], TOL)
     assert_close("dC[b=0]", gr["dCm"][0:1], rg["C"], TOL)
+
+
+@pytest.mark.parametrize("disc", ["zoh", "bilinear"])
+def test_s6_full_state_mode(disc):
+    """LR_FULL_STATE: every step's state checkpointed (the oracle's segment-1 checkpoints) and read
+    by the backward; outputs and gradients equal the default mode's bitwise."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.s6(2, 200, 128, 16, seed=9)
+    y0, _, g0, _, _ = run_gpu("s6", inp, 64, disc=disc)
+    y1, ck, g1, plan, _ = run_gpu("s6", inp, 64, disc=disc, flags=lrscan.FULL_STATE)
+    assert ck.shape[0] == 200
+    _, rck = oracle.s6_fwd(inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"],
+                           disc=disc, S=1)
+    assert_close("full-state ckpt", ck, rck, TOL)
+    assert torch.equal(y0, y1)
+    for k in g0:
+        assert torch.equal(g0[k], g1[k]), k
+    assert plan.device_error() == (0, 0)

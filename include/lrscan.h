@@ -103,6 +103,11 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * gradients are those of the default mode; the memory is L / S times the checkpoint memory.  The
  * segment length still sets the tiling.  SSD and GLA: LR_ERR_UNSUPPORTED. */
 #define LR_FULL_STATE 4u
+/* S6 / SSD: the step length is dt = softplus(delta + delta_bias) computed in the kernels (the
+ * layer's raw delta and an f32 bias per channel (S6, [D]) or head (SSD, [H]), NULL = no bias);
+ * the backward writes ddelta for the raw delta, dd * sigma(delta + bias), and, if ddelta_bias is
+ * non-NULL, ddelta_bias = its sum over batch and time. */
+#define LR_DELTA_SOFTPLUS 8u
 /* Test hook for the failure path: the tiles of the first segment never publish their carry, so
  * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
  * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
@@ -137,6 +142,7 @@ typedef struct {
     const float *Dskip;           /* s6 [D] / ssd [H] (LR_HAS_DSKIP)         */
     const void *z;                /* s6 / ssd (LR_HAS_Z)                     */
     const void *q, *k, *v;        /* gla                                     */
+    const float *delta_bias;      /* s6 [D] / ssd [H] (LR_DELTA_SOFTPLUS)     */
 } lr_inputs;
 
 /* Gradients, per kind (unused members NULL).  Device pointers. */
@@ -147,6 +153,7 @@ typedef struct {
     float *dA, *dBm, *dCm, *dDskip;
     void *dz;
     void *dq, *dk, *dv;           /* gla                                     */
+    float *ddelta_bias;           /* s6 [D] / ssd [H] (LR_DELTA_SOFTPLUS)     */
 } lr_grads;
 
 /* Host-side check of a descriptor: LR_OK, or the status lr_scan_fwd would return for it

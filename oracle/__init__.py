@@ -13,6 +13,11 @@ when omitted) and, with ``final=True``, also returns the state after the last st
 kind's state layout: rglru / rotlru [B, D], S6 [B, D, N], SSD [B, H, P, N], GLA [B, H, K, V].
 Results are returned as ``y``, ``(y, ck)``, ``(y, hL)`` or ``(y, ck, hL)``.
 
+S6 and SSD take ``delta_softplus=True`` with an optional ``delta_bias`` (per channel / head): the
+step length is then ``dt = softplus(delta + delta_bias)`` (an elementwise front-end, written out
+here in numpy), and the backward returns the gradient for the raw ``delta``,
+``d dt * sigmoid(delta + bias)``, and ``delta_bias``, its sum over batch and time.
+
 Sources: the mlx-recurrence post (Apple Developer Forums thread 840535, "Current kernels" and the
 segment-checkpointing paragraph), "lrnnx: A library for Linear RNNs" (ai.info summary, Key
 Contributions 2-3), and the K-Search / mlx-mamba blog post (techtrendfeed repost, the paragraph
@@ -78,6 +83,12 @@ def _p(x):
     return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def _softplus_front(delta, bias, axis_shape):
+    """dt = softplus(delta + bias) and sigmoid(delta + bias) (bias broadcast along the last axis)."""
+    v = delta + (0.0 if bias is None else _f64(bias).reshape(axis_shape))
+    return np.logaddexp(0.0, v), 0.5 * (1.0 + np.tanh(0.5 * v))
+
+
 def _nseg(L, S):
     return (L + S - 1) // S if S and S > 0 else 0
 
@@ -141,8 +152,11 @@ def rotlru_bwd(b, g, mag, theta, dy):
 
 
 # ------------------------------------------------------------------------------------------- S6
-def s6_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False):
+def s6_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False,
+           delta_softplus=False, delta_bias=None):
     x, delta, A, Bm, Cm = map(_f64, (x, delta, A, Bm, Cm))
+    if delta_softplus:
+        delta, _ = _softplus_front(delta, delta_bias, (1, 1, -1))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, D = x.shape
     N = A.shape[1]
@@ -155,8 +169,11 @@ def s6_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, fi
     return _ret(y, ck, hL, S, final)
 
 
-def s6_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
+def s6_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh", delta_softplus=False, delta_bias=None):
     x, delta, A, Bm, Cm, dy = map(_f64, (x, delta, A, Bm, Cm, dy))
+    sg = None
+    if delta_softplus:
+        delta, sg = _softplus_front(delta, delta_bias, (1, 1, -1))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, D = x.shape
     N = A.shape[1]
@@ -167,12 +184,19 @@ def s6_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
     lib().orc_s6_bwd(B, L, D, N, DISC[disc], _p(x), _p(delta), _p(A), _p(Bm), _p(Cm),
                      _p(Dskip), _p(z), _p(dy), _p(dx), _p(ddt), _p(dA), _p(dB), _p(dC),
                      _p(dD), _p(dz))
-    return {"x": dx, "delta": ddt, "A": dA, "B": dB, "C": dC, "D": dD, "z": dz}
+    out = {"x": dx, "delta": ddt, "A": dA, "B": dB, "C": dC, "D": dD, "z": dz}
+    if sg is not None:
+        out["delta"] = ddt * sg
+        out["delta_bias"] = out["delta"].sum(axis=(0, 1))
+    return out
 
 
 # ------------------------------------------------------------------------------------------ SSD
-def ssd_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False):
+def ssd_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, final=False,
+            delta_softplus=False, delta_bias=None):
     x, delta, A, Bm, Cm = map(_f64, (x, delta, A, Bm, Cm))
+    if delta_softplus:
+        delta, _ = _softplus_front(delta, delta_bias, (1, 1, -1))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
@@ -185,8 +209,11 @@ def ssd_fwd(x, delta, A, Bm, Cm, Dskip=None, z=None, disc="zoh", S=0, h0=None, f
     return _ret(y, ck, hL, S, final)
 
 
-def ssd_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
+def ssd_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh", delta_softplus=False, delta_bias=None):
     x, delta, A, Bm, Cm, dy = map(_f64, (x, delta, A, Bm, Cm, dy))
+    sg = None
+    if delta_softplus:
+        delta, sg = _softplus_front(delta, delta_bias, (1, 1, -1))
     Dskip, z = _f64(Dskip), _f64(z)
     B, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
@@ -197,7 +224,11 @@ def ssd_bwd(x, delta, A, Bm, Cm, Dskip, z, dy, disc="zoh"):
     lib().orc_ssd_bwd(B, L, H, P, N, G, DISC[disc], _p(x), _p(delta), _p(A), _p(Bm), _p(Cm),
                       _p(Dskip), _p(z), _p(dy), _p(dx), _p(ddt), _p(dA), _p(dB), _p(dC),
                       _p(dD), _p(dz))
-    return {"x": dx, "delta": ddt, "A": dA, "B": dB, "C": dC, "D": dD, "z": dz}
+    out = {"x": dx, "delta": ddt, "A": dA, "B": dB, "C": dC, "D": dD, "z": dz}
+    if sg is not None:
+        out["delta"] = ddt * sg
+        out["delta_bias"] = out["delta"].sum(axis=(0, 1))
+    return out
 
 
 # ------------------------------------------------------------------------------------------ GLA

@@ -31,6 +31,7 @@ lr_status validate(const lr_desc* d) {
     if (d->B > (1 << 20) || d->L > (1ll << 30)) return LR_ERR_UNSUPPORTED;
     if ((d->flags & LR_FULL_STATE) && d->kind != LR_RGLRU && d->kind != LR_ROTLRU && d->kind != LR_S6)
         return LR_ERR_UNSUPPORTED;
+    if ((d->flags & LR_DELTA_SOFTPLUS) && d->kind != LR_S6 && d->kind != LR_SSD) return LR_ERR_INVALID_ARG;
     const int es = esize(d->io);
     switch (d->kind) {
         case LR_RGLRU:
@@ -282,6 +283,7 @@ lr_status lr_step(const lr_desc* desc, const lr_inputs* in, const void* state_in
     if (d.io != LR_F32 && d.io != LR_BF16) return LR_ERR_INVALID_ARG;
     if (d.B < 1 || d.L < 1) return LR_ERR_INVALID_ARG;
     if (d.B > (1 << 20) || d.L > (1ll << 30)) return LR_ERR_UNSUPPORTED;
+    if ((d.flags & LR_DELTA_SOFTPLUS) && d.kind != LR_S6 && d.kind != LR_SSD) return LR_ERR_INVALID_ARG;
     const size_t es = (size_t)esize(d.io);
     struct Need {
         const void* p;

@@ -94,7 +94,17 @@ struct S6Args {
     float* pdC;          // [ncb, B, L, N]
     float* pdA;          // [B, D, N]
     float* pdD;          // [B, D]
+    int softplus;        // LR_DELTA_SOFTPLUS: dt = softplus(delta + bias)
+    const float* dbias;  // [D] or null (bias 0)
+    float* pdE;          // [B, D] partials of d bias
 };
+
+__device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
+
+// dt of one step: the raw delta, or softplus(delta + bias) (LR_DELTA_SOFTPLUS)
+__device__ __forceinline__ float step_dt(const S6Args& a, float raw, float bias) {
+    return a.softplus ? softplus_f(raw + bias) : raw;
+}
 
 // Per-thread constants of the discretisation for its 8 states.
 struct Disc {
@@ -180,6 +190,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
+    const float dbias = (a.softplus && a.dbias && dok) ? a.dbias[d] : 0.0f;
     float h[kNH];
 #pragma unroll
     for (int j = 0; j < kNH; ++j) h[j] = 0.0f;
@@ -206,7 +217,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         const __nv_bfloat16* Cs = stageBC(s, 1);
         if (ok) {
             for (int t = 0; t < nt; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
                 float Bv[kNH], Cv[kNH];
                 ldn(Bs + t * kN + part * kNH, Bv);
                 ldn(Cs + t * kN + part * kNH, Cv);
@@ -292,10 +303,11 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
+    const float dbias = (a.softplus && a.dbias && dok) ? a.dbias[d] : 0.0f;
     float G[kNH], anext[kNH], dA[kNH];
 #pragma unroll
     for (int j = 0; j < kNH; ++j) G[j] = anext[j] = dA[j] = 0.0f;
-    float dD = 0.0f;
+    float dD = 0.0f, dE = 0.0f;
     const uint32_t bytes = (uint32_t)(a.S * kDB * 2 * (a.has_z ? 4 : 3) + 2 * a.S * kN * 2);
     __syncthreads();
 
@@ -329,7 +341,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int j = 0; j < kNH; ++j) bp[j] = h[j];
             const int te = min(nt, (sb + 1) * kSub);
             for (int t = sb * kSub; t < te; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
                 float Bv[kNH];
                 ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -366,7 +378,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                 for (int i = 0; i < kSub; ++i) {  // h after step i from the state entering it
                     if (i < n) {
                         const int t = tb + i;
-                        const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                        const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
                         float Bv[kNH];
                         ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -383,7 +395,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int i = 0; i < kSub; ++i) {
                 if (i < n && !FULL) {
                     const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                    const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
                     float Bv[kNH];
                     ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -400,7 +412,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int i = kSub - 1; i >= 0; --i) {
                 if (i < n) {
                     const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = bf(DT + t * kDB + dl);
+                    const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
                     const float dyv = bf(DY + t * kDB + dl);
                     float Bv[kNH], Cv[kNH];
                     ldn(Bs + t * kN + part * kNH, Bv);
@@ -466,8 +478,12 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     }
                     red[((size_t)(warp * kSub + i) * 2 + q / kNH) * kN + part * kNH + (q % kNH)] = v[0];
                     if (part == 0) {
+                        // softplus: d delta = d dt sigma(delta + bias), and sigma(delta + bias) =
+                        // 1 - e^{-dt}
+                        const float ddr = a.softplus ? dta * -expm1f(-dt) : dta;
+                        dE += ddr;
                         X[t * kDB + dl] = __float2bfloat16_rn(fmaf(ds, Dd, dxa));
-                        DT[t * kDB + dl] = __float2bfloat16_rn(dta);
+                        DT[t * kDB + dl] = __float2bfloat16_rn(ddr);
                         if (a.has_z) Z[t * kDB + dl] = __float2bfloat16_rn(dz);
                         dD = fmaf(ds, xv, dD);
                     }
@@ -500,17 +516,18 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
 #pragma unroll
         for (int j = 0; j < kNH; ++j) pa[j] = dA[j];
         if (part == 0) a.pdD[(size_t)b * a.D + d] = dD;
+        if (part == 0 && a.softplus) a.pdE[(size_t)b * a.D + d] = dE;
     }
     if (tid == 0) bulk_wait_read_all();
 }
 
 // Fixed-order sums of the partials: dB, dC over channel blocks; dA, dD over batch rows.
 __global__ void s6_reduce_kernel(S6Args a, float* __restrict__ dBm, float* __restrict__ dCm,
-                                 float* __restrict__ dAo, float* __restrict__ dDo) {
+                                 float* __restrict__ dAo, float* __restrict__ dDo, float* __restrict__ dEo) {
     const size_t nBC = (size_t)a.B * a.L * kN;
     const size_t nA = (size_t)a.D * kN;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nBC + nA + a.D;
-         i += (size_t)gridDim.x * blockDim.x) {
+    const size_t n = nBC + nA + a.D + (dEo ? a.D : 0);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         if (i < nBC) {
             float sb = 0.0f, sc = 0.0f;
             for (int cb = 0; cb < a.ncb; ++cb) {
@@ -524,18 +541,25 @@ __global__ void s6_reduce_kernel(S6Args a, float* __restrict__ dBm, float* __res
             float s = 0.0f;
             for (int bb = 0; bb < a.B; ++bb) s += a.pdA[(size_t)bb * nA + j];
             dAo[j] = s;
-        } else if (dDo) {
-            const size_t j = i - nBC - nA;
+        } else if (i < nBC + nA + a.D) {
+            if (dDo) {
+                const size_t j = i - nBC - nA;
+                float s = 0.0f;
+                for (int bb = 0; bb < a.B; ++bb) s += a.pdD[(size_t)bb * a.D + j];
+                dDo[j] = s;
+            }
+        } else {  // d bias of the softplus front-end
+            const size_t j = i - nBC - nA - a.D;
             float s = 0.0f;
-            for (int bb = 0; bb < a.B; ++bb) s += a.pdD[(size_t)bb * a.D + j];
-            dDo[j] = s;
+            for (int bb = 0; bb < a.B; ++bb) s += a.pdE[(size_t)bb * a.D + j];
+            dEo[j] = s;
         }
     }
 }
 
 // ------------------------------------------------------------------------------ host side
 struct S6Ws {
-    size_t pdB, pdC, pdA, pdD, end;
+    size_t pdB, pdC, pdA, pdD, pdE, end;
 };
 
 S6Ws ws_plan(const lr_desc& d) {
@@ -546,6 +570,7 @@ S6Ws ws_plan(const lr_desc& d) {
     w.pdC = c.take(sizeof(float) * ncb * d.B * d.L * kN);
     w.pdA = c.take(sizeof(float) * d.B * d.D * kN);
     w.pdD = c.take(sizeof(float) * d.B * d.D);
+    w.pdE = c.take(sizeof(float) * d.B * d.D);
     w.end = c.off;
     return w;
 }
@@ -561,6 +586,8 @@ S6Args make_args(const lr_desc& d, const lr_inputs& in, void* ckpt, char* ws, bo
     a.disc = d.disc;
     a.has_z = (d.flags & LR_HAS_Z) ? 1 : 0;
     a.has_d = (d.flags & LR_HAS_DSKIP) ? 1 : 0;
+    a.softplus = (d.flags & LR_DELTA_SOFTPLUS) ? 1 : 0;
+    a.dbias = a.softplus ? in.delta_bias : nullptr;
     a.A = in.A;
     a.Dskip = in.Dskip;
     a.ckpt = (float*)ckpt;
@@ -571,6 +598,7 @@ S6Args make_args(const lr_desc& d, const lr_inputs& in, void* ckpt, char* ws, bo
         a.pdC = (float*)(ws + w.pdC);
         a.pdA = (float*)(ws + w.pdA);
         a.pdD = (float*)(ws + w.pdD);
+        a.pdE = (float*)(ws + w.pdE);
     }
     return a;
 }
@@ -670,7 +698,8 @@ lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const vo
     lr_status s = check_launch();
     if (s != LR_OK) return s;
     note_launch("s6_param_reduce");
-    s6_reduce_kernel<<<4 * 148, 256, 0, st>>>(a, gr.dBm, gr.dCm, gr.dA, a.has_d ? gr.dDskip : nullptr);
+    s6_reduce_kernel<<<4 * 148, 256, 0, st>>>(a, gr.dBm, gr.dCm, gr.dA, a.has_d ? gr.dDskip : nullptr,
+                                              a.softplus ? gr.ddelta_bias : nullptr);
     return check_launch();
 }
 

@@ -31,6 +31,8 @@ constexpr uint32_t kTileBytes = kKD * kP * 2;  // one N x P state block as a bf1
 struct SsdArgs {
     int B, L, H, G, HpG, nchunk;  // HpG: heads per group
     int disc;                     // LR_DISC_ZOH, LR_DISC_DIRAC or LR_DISC_ZOH_EULER
+    int softplus;                 // LR_DELTA_SOFTPLUS: dt = softplus(delta + bias_h)
+    const float* dbias;           // [H] or null
     const __nv_bfloat16* dt;      // [B, L, H]
     const float* A;               // [H]
     const float* Dskip;           // [H] or null
@@ -44,6 +46,13 @@ __device__ __forceinline__ float ssd_beta(int disc, float lam, float dt, float A
     if (disc == LR_DISC_DIRAC) return 1.0f;
     if (disc == LR_DISC_ZOH_EULER) return dt;
     return (ex2(lam * kLog2e) - 1.0f) / Ah;
+}
+
+// dt of head h from the raw delta: itself, or softplus(delta + bias_h) (LR_DELTA_SOFTPLUS)
+__device__ __forceinline__ float ssd_dt(const SsdArgs& a, float raw, int h) {
+    if (!a.softplus) return raw;
+    const float v = raw + (a.dbias ? a.dbias[h] : 0.0f);
+    return v > 20.0f ? v : log1pf(expf(v));
 }
 
 // Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
@@ -262,7 +271,8 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < kQ / 32; ++i) {
                     const int k = k0 + j, tt = chunk_of(k) * kQ + lane + 32 * i;
-                    v[j][i] = k < nk && tt < a.L ? __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]) : 0.0f;
+                    v[j][i] = k < nk && tt < a.L ? ssd_dt(a, __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]), h)
+                                                 : 0.0f;
                 }
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
@@ -358,7 +368,7 @@ __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad
     const __nv_bfloat16* src = a.dt + ((size_t)b * a.L + (valid ? t0 + row : 0)) * a.H + hfirst;
     float v[kMaxHB];
 #pragma unroll
-    for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? __bfloat162float(src[i]) : 0.0f;
+    for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? ssd_dt(a, __bfloat162float(src[i]), hfirst + i) : 0.0f;
 #pragma unroll
     for (int i = 0; i < kMaxHB; ++i) dts[i * kQ + row] = v[i];
 }
@@ -626,6 +636,8 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     a.HpG = (int)(d.H / d.G);
     a.nchunk = (int)((d.L + kQ - 1) / kQ);
     a.disc = d.disc;
+    a.softplus = (d.flags & LR_DELTA_SOFTPLUS) ? 1 : 0;
+    a.dbias = a.softplus ? in.delta_bias : nullptr;
     a.dt = (const __nv_bfloat16*)in.delta;
     a.A = in.A;
     a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
@@ -695,6 +707,7 @@ struct SsdGradArgs {
     float* dC;
     float* pdA;            // [B][H][nchunk] per-chunk partials of dA_h, dD_h
     float* pdD;
+    float* pdE;            // [B][H][nchunk] partials of d bias (LR_DELTA_SOFTPLUS)
     int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
 };
 
@@ -1080,7 +1093,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             float total;
             const float incl = wg0_inclusive_sum(dl, tmp, &total);
             const float dlam = total - incl + dl;
-            float dA_part = 0.0f;
+            float dA_part = 0.0f, ddr = 0.0f;
             if (valid) {
                 const float Ah = ad[i];
                 const float bt = betas[t];
@@ -1089,14 +1102,20 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
                 // d beta / d dt: ZOH e^{dt A}, ZOH-Euler 1, dirac 0;  d beta / dA: ZOH only
                 const float dbdt = a.disc == LR_DISC_ZOH ? ab : (a.disc == LR_DISC_ZOH_EULER ? 1.0f : 0.0f);
-                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(dlam * Ah + dbeta * dbdt);
+                // softplus front-end: d delta = d dt sigma(delta + bias), sigma(delta + bias) = 1 - e^{-dt}
+                ddr = (dlam * Ah + dbeta * dbdt) * (a.softplus ? -expm1f(-dt_raw) : 1.0f);
+                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(ddr);
                 dA_part = dlam * dt_raw + (a.disc == LR_DISC_ZOH ? dbeta * (dt_raw * ab - bt) / Ah : 0.0f);
             }
             const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
+            const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
             if (t == 0) {
-                const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
                 ga.pdA[tile] = sAD.x;
                 ga.pdD[tile] = sAD.y;
+            }
+            if (a.softplus) {  // uniform: the d bias partial of this (row, head, chunk)
+                const float2 sE = wg0_sum2(ddr, 0.0f, tmp);
+                if (t == 0) ga.pdE[tile] = sE.x;
             }
         }
     }
@@ -1138,32 +1157,36 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
 
 // dA_h, dD_h: fixed-order sums of the per-chunk partials over batch rows and chunks (one warp per
 // head; lane-strided partial sums, then a fixed butterfly).
-__global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __restrict__ pdD, int B, int H, int nchunk,
-                              float* __restrict__ dA, float* __restrict__ dD) {
+__global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __restrict__ pdD,
+                              const float* __restrict__ pdE, int B, int H, int nchunk, float* __restrict__ dA,
+                              float* __restrict__ dD, float* __restrict__ dE) {
     pdl_wait();
     const int h = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (h >= H) return;
-    float sa = 0.0f, sd = 0.0f;
+    float sa = 0.0f, sd = 0.0f, se = 0.0f;
     for (int bb = 0; bb < B; ++bb)
         for (int c = lane; c < nchunk; c += 32) {
             const size_t t = ((size_t)bb * H + h) * nchunk + c;
             sa += pdA[t];
             sd += pdD[t];
+            if (dE) se += pdE[t];
         }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         sa += __shfl_xor_sync(0xffffffffu, sa, o);
         sd += __shfl_xor_sync(0xffffffffu, sd, o);
+        se += __shfl_xor_sync(0xffffffffu, se, o);
     }
     if (lane == 0) {
         dA[h] = sa;
         if (dD) dD[h] = sd;
+        if (dE) dE[h] = se;
     }
 }
 
 struct SsdBwdWs {
-    size_t pdA, pdD, gtiles, end;
+    size_t pdA, pdD, pdE, gtiles, end;
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
@@ -1172,6 +1195,7 @@ SsdBwdWs bwd_plan(const lr_desc& d) {
     SsdBwdWs w;
     w.pdA = cur.take(sizeof(float) * tiles);
     w.pdD = cur.take(sizeof(float) * tiles);
+    w.pdE = cur.take(sizeof(float) * tiles);
     w.gtiles = cur.take((size_t)kTileBytes * tiles);
     w.end = cur.off;
     return w;
@@ -1240,6 +1264,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.dC = gr.dCm;
     ga.pdA = (float*)(ws + w.pdA);
     ga.pdD = (float*)(ws + w.pdD);
+    ga.pdE = (float*)(ws + w.pdE);
     CUtensorMap mC, mB, mX, mdY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true);
@@ -1269,7 +1294,9 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     if (s != LR_OK) return s;
     note_launch("ssd_param_reduce");
     if (launch_pdl(ssd_param_sum, dim3((a.H + 7) / 8), dim3(256), 0, st, (const float*)ga.pdA, (const float*)ga.pdD,
-                   a.B, a.H, a.nchunk, gr.dA, (d.flags & LR_HAS_DSKIP) ? gr.dDskip : (float*)nullptr) != cudaSuccess)
+                   (const float*)ga.pdE, a.B, a.H, a.nchunk, gr.dA,
+                   (d.flags & LR_HAS_DSKIP) ? gr.dDskip : (float*)nullptr,
+                   a.softplus ? gr.ddelta_bias : (float*)nullptr) != cudaSuccess)
         return LR_ERR_CUDA;
     return check_launch();
 }

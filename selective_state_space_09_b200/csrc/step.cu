@@ -86,6 +86,13 @@ __device__ __forceinline__ void disc_coef(int disc, float dt, float A, float& ab
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + ex2(-z * kLog2eS)); }
 
+// dt from the raw delta: itself, or softplus(delta + bias) (LR_DELTA_SOFTPLUS; bias may be null)
+__device__ __forceinline__ float step_dt(float raw, int softplus, const float* bias, int i) {
+    if (!softplus) return raw;
+    const float v = raw + (bias ? bias[i] : 0.0f);
+    return v > 20.0f ? v : log1pf(expf(v));
+}
+
 constexpr int kS6MaxN = 32;
 
 // One thread per (b, d, n): NL lanes (a power of two >= N, at most 32) per channel, the readout
@@ -95,7 +102,7 @@ __global__ void __launch_bounds__(256)
 s6_step_kernel(const T* __restrict__ x, const T* __restrict__ delta, const float* __restrict__ A,
                const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ Dskip,
                const T* __restrict__ z, T* __restrict__ y, const float* s_in, float* s_out, int B, int L, int D,
-               int N, int NL, int disc) {
+               int N, int NL, int disc, int softplus, const float* __restrict__ dbias) {
     const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t u = gtid / NL;  // channel (b, d)
     const int n = (int)(gtid % NL);
@@ -112,7 +119,7 @@ s6_step_kernel(const T* __restrict__ x, const T* __restrict__ delta, const float
             const size_t bt = ((size_t)bi * L + t) * N + n;
             xv = IO<T>::ld(x + i);
             float ab, be;
-            disc_coef(disc, IO<T>::ld(delta + i), An, ab, be);
+            disc_coef(disc, step_dt(IO<T>::ld(delta + i), softplus, dbias, d), An, ab, be);
             h = fmaf(ab, h, be * IO<T>::ld(Bm + bt) * xv);
             s = IO<T>::ld(Cm + bt) * h;
         }
@@ -131,10 +138,10 @@ constexpr int kMatCols = 32, kMatSlices = 8, kMatMaxK = 128, kMatRows = kMatMaxK
 
 struct MatStepArgs {
     int B, L, H, K, V, G, HpG;  // K: state rows (GLA K, SSD N); V: columns (GLA V, SSD P)
-    int ssd, disc;
+    int ssd, disc, softplus;
     const void *q, *k, *v, *g;  // GLA: q, k [B,L,H,K]; v [B,L,H,V]; g [B,L,H]
     const void *x, *dt, *Bm, *Cm, *z;  // SSD: x, z [B,L,H,P]; dt [B,L,H]; Bm, Cm [B,L,G,N]
-    const float *A, *Dskip;
+    const float *A, *Dskip, *dbias;
     void* y;                    // [B, L, H, V]
     const float* s_in;          // [B, H, K, V] or null
     float* s_out;
@@ -165,7 +172,7 @@ mat_step_kernel(MatStepArgs a) {
         const size_t bt = (size_t)bi * a.L + t;
         if (a.ssd) {
             float ab, be;
-            disc_coef(a.disc, IO<T>::ld((const T*)a.dt + bt * a.H + h), Ah, ab, be);
+            disc_coef(a.disc, step_dt(IO<T>::ld((const T*)a.dt + bt * a.H + h), a.softplus, a.dbias, h), Ah, ab, be);
             const int gi = h / a.HpG;
             const T* Bt = (const T*)a.Bm + (bt * a.G + gi) * a.K;
             const T* Ct = (const T*)a.Cm + (bt * a.G + gi) * a.K;
@@ -245,7 +252,8 @@ lr_status step_impl(const lr_desc& d, const lr_inputs& in, const float* s_in, fl
             s6_step_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
                 (const T*)in.x, (const T*)in.delta, in.A, (const T*)in.Bm, (const T*)in.Cm,
                 (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr, (d.flags & LR_HAS_Z) ? (const T*)in.z : nullptr,
-                (T*)y, s_in, s_out, B, L, (int)d.D, (int)d.N, NL, (int)d.disc);
+                (T*)y, s_in, s_out, B, L, (int)d.D, (int)d.N, NL, (int)d.disc, (d.flags & LR_DELTA_SOFTPLUS) ? 1 : 0,
+                in.delta_bias);
             return check_launch();
         }
         default: {
@@ -270,6 +278,8 @@ lr_status step_impl(const lr_desc& d, const lr_inputs& in, const float* s_in, fl
             a.z = (a.ssd && (d.flags & LR_HAS_Z)) ? in.z : nullptr;
             a.A = in.A;
             a.Dskip = (a.ssd && (d.flags & LR_HAS_DSKIP)) ? in.Dskip : nullptr;
+            a.softplus = (a.ssd && (d.flags & LR_DELTA_SOFTPLUS)) ? 1 : 0;
+            a.dbias = a.softplus ? in.delta_bias : nullptr;
             a.y = y;
             a.s_in = s_in;
             a.s_out = s_out;

@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
 DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 IO = {torch.float32: 0, torch.bfloat16: 1}
-HAS_Z, HAS_DSKIP, FULL_STATE = 1, 2, 4
+HAS_Z, HAS_DSKIP, FULL_STATE, DELTA_SOFTPLUS = 1, 2, 4, 8
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
 TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
 STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
@@ -45,9 +45,10 @@ class Desc(ctypes.Structure):
                 ("segment", ctypes.c_int32)]
 
 
-_IN = ["a", "b", "g", "mag", "theta", "x", "delta", "A", "Bm", "Cm", "Dskip", "z", "q", "k", "v"]
+_IN = ["a", "b", "g", "mag", "theta", "x", "delta", "A", "Bm", "Cm", "Dskip", "z", "q", "k", "v",
+       "delta_bias"]
 _GR = ["da", "db", "dg", "dmag", "dtheta", "dx", "ddelta", "dA", "dBm", "dCm", "dDskip", "dz",
-       "dq", "dk", "dv"]
+       "dq", "dk", "dv", "ddelta_bias"]
 
 
 class Inputs(ctypes.Structure):
@@ -191,8 +192,9 @@ class Plan:
 
 
 # ------------------------------------------------------------------ per-kind convenience plans
-def desc_for(kind, inp, segment=1, disc="none", chunk=0):
-    """Descriptor of a kind from its input tensors (shapes read from the tensors)."""
+def desc_for(kind, inp, segment=1, disc="none", chunk=0, delta_softplus=False):
+    """Descriptor of a kind from its input tensors (shapes read from the tensors).
+    delta_softplus (S6, SSD): dt = softplus(delta + inp["delta_bias"]) in the kernels."""
     if kind == "rglru":
         B, L, D = inp["a"].shape
         d = make_desc("rglru", inp["a"].dtype, B, L, D=D, segment=segment)
@@ -216,12 +218,14 @@ def desc_for(kind, inp, segment=1, disc="none", chunk=0):
         d = make_desc("gla", inp["q"].dtype, B, L, H=H, P=V, N=K, segment=segment, chunk=chunk)
     else:
         raise KeyError(kind)
+    if delta_softplus:
+        d.flags |= DELTA_SOFTPLUS
     return d
 
 
-def plan_for(kind, inp, segment, disc="none", chunk=0):
+def plan_for(kind, inp, segment, disc="none", chunk=0, delta_softplus=False):
     """Build the Plan of a kind from its input tensors (shapes read from the tensors)."""
-    d = desc_for(kind, inp, segment, disc, chunk)
+    d = desc_for(kind, inp, segment, disc, chunk, delta_softplus)
     return Plan(d, inp[next(k for k in inp if inp[k] is not None)].device)
 
 
@@ -292,6 +296,8 @@ def alloc_outputs(kind, inp):
             g["dDskip"] = e(inp["Dskip"])
         if inp.get("z") is not None:
             g["dz"] = e(inp["z"])
+        if inp.get("delta_bias") is not None:
+            g["ddelta_bias"] = e(inp["delta_bias"])
         return e(inp["x"]), g
     if kind == "gla":
         return e(inp["v"]), {"dq": e(inp["q"]), "dk": e(inp["k"]), "dv": e(inp["v"]), "dg": e(inp["g"])}
@@ -301,9 +307,9 @@ def alloc_outputs(kind, inp):
 # ---------------------------------------------------------------------- autograd wrappers
 class _ScanFn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, kind, names, segment, disc, chunk, *tensors):
+    def forward(ctx, kind, names, segment, disc, chunk, softplus, *tensors):
         inp = {n: t.contiguous() if t is not None else None for n, t in zip(names, tensors)}
-        plan = plan_for(kind, inp, segment, disc, chunk)
+        plan = plan_for(kind, inp, segment, disc, chunk, softplus)
         y, _ = alloc_outputs(kind, inp)
         plan.fwd(inp, y)
         ctx.kind, ctx.names, ctx.plan = kind, names, plan
@@ -319,31 +325,34 @@ class _ScanFn(torch.autograd.Function):
         for n in ctx.names:
             t = inp[n]
             out.append(grads.get("d" + n) if t is not None else None)
-        return (None, None, None, None, None) + tuple(out)
+        return (None, None, None, None, None, None) + tuple(out)
 
 
 def rglru(a, b, segment=128):
     """y = rglru_scan(a, b): h_t = a_t h_{t-1} + b_t, y_t = h_t.  a, b: [B, L, D]."""
-    return _ScanFn.apply("rglru", ("a", "b"), segment, "none", 0, a, b)
+    return _ScanFn.apply("rglru", ("a", "b"), segment, "none", 0, False, a, b)
 
 
 def rotlru(b, g, mag, theta, segment=256):
     """y = rotlru_scan: lambda_t = mag g_t e^{i theta}, h_t = lambda_t h_{t-1} + b_t (pairs)."""
-    return _ScanFn.apply("rotlru", ("b", "g", "mag", "theta"), segment, "none", 0, b, g, mag, theta)
+    return _ScanFn.apply("rotlru", ("b", "g", "mag", "theta"), segment, "none", 0, False, b, g, mag, theta)
 
 
-def s6(x, delta, A, B, C, D=None, z=None, disc="zoh", segment=256):
-    """Selective scan S6 with fused D skip and silu(z) gate.  x, delta, z: [B, L, D]."""
-    return _ScanFn.apply("s6", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z"), segment, disc, 0,
-                         x, delta, A, B, C, D, z)
+def s6(x, delta, A, B, C, D=None, z=None, disc="zoh", segment=256, delta_softplus=False, delta_bias=None):
+    """Selective scan S6 with fused D skip and silu(z) gate.  x, delta, z: [B, L, D].  With
+    delta_softplus the step length is softplus(delta + delta_bias) (delta_bias [D] or None)."""
+    return _ScanFn.apply("s6", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"), segment, disc, 0,
+                         delta_softplus, x, delta, A, B, C, D, z, delta_bias)
 
 
-def ssd(x, delta, A, B, C, D=None, z=None, disc="zoh", chunk=64, segment=256):
-    """Head-wise SSD scan.  x, z: [B, L, H, P]; delta: [B, L, H]; B, C: [B, L, G, N]."""
-    return _ScanFn.apply("ssd", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z"), segment, disc, chunk,
-                         x, delta, A, B, C, D, z)
+def ssd(x, delta, A, B, C, D=None, z=None, disc="zoh", chunk=64, segment=256, delta_softplus=False,
+        delta_bias=None):
+    """Head-wise SSD scan.  x, z: [B, L, H, P]; delta: [B, L, H]; B, C: [B, L, G, N].  With
+    delta_softplus the step length is softplus(delta + delta_bias) (delta_bias [H] or None)."""
+    return _ScanFn.apply("ssd", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"), segment, disc,
+                         chunk, delta_softplus, x, delta, A, B, C, D, z, delta_bias)
 
 
 def gla(q, k, v, g, chunk=64, segment=256):
     """GLA scan: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t."""
-    return _ScanFn.apply("gla", ("q", "k", "v", "g"), segment, "none", chunk, q, k, v, g)
+    return _ScanFn.apply("gla", ("q", "k", "v", "g"), segment, "none", chunk, False, q, k, v, g)

@@ -64,6 +64,24 @@ def test_ssd_parity_other_discretisations(B, L, H, P, G, disc):
     assert plan.device_error() == (0, 0)
 
 
+def test_ssd_softplus_front_end():
+    """LR_DELTA_SOFTPLUS on the chunked SSD path: gradients for the raw delta and the bias."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.ssd(2, 260, 10, 64, 128, G=2, seed=23)
+    gen = torch.Generator().manual_seed(6)
+    inp["delta"] = (torch.randn(inp["delta"].shape, generator=gen) - 2.0).to(torch.bfloat16)
+    inp["delta_bias"] = 0.5 * torch.randn(10, generator=gen)
+    y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc="zoh", chunk=128, flags=lrscan.DELTA_SOFTPLUS)
+    a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], None)
+    ry = oracle.ssd_fwd(*a, disc="zoh", delta_softplus=True, delta_bias=inp["delta_bias"])
+    rg = oracle.ssd_bwd(*a, inp["dy"], disc="zoh", delta_softplus=True, delta_bias=inp["delta_bias"])
+    assert_close("y", y, ry, TOL)
+    for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D"),
+                      ("ddelta_bias", "delta_bias")):
+        assert_close(name, gr[name], rg[ref], TOL)
+    assert plan.device_error() == (0, 0)
+
+
 def test_ssd_head_blocking_bitwise():
     """The head blocking of the output kernel changes only which CTA computes a head."""
     from selective_state_space_09_b200 import lrscan

@@ -116,3 +116,30 @@ def test_s6_full_state_mode(disc):
     for k in g0:
         assert torch.equal(g0[k], g1[k]), k
     assert plan.device_error() == (0, 0)
+
+
+@pytest.mark.parametrize("disc", ["zoh", "zoh_euler"])
+def test_s6_softplus_front_end(disc):
+    """LR_DELTA_SOFTPLUS: dt = softplus(delta + bias) in the kernels; gradients for the raw delta
+    and the bias against the oracle; the autograd wrapper gives the same values."""
+    inp = inputs.s6(2, 200, 128, 16, seed=21)
+    gen = torch.Generator().manual_seed(5)
+    inp["delta"] = (torch.randn(inp["delta"].shape, generator=gen) - 2.0).to(torch.bfloat16)
+    inp["delta_bias"] = 0.5 * torch.randn(128, generator=gen)
+    y, ck, gr, plan, disp = run_gpu("s6", inp, 64, disc=disc, flags=lrscan.DELTA_SOFTPLUS)
+    a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"])
+    ry = oracle.s6_fwd(*a, disc=disc, delta_softplus=True, delta_bias=inp["delta_bias"])
+    rg = oracle.s6_bwd(*a, inp["dy"], disc=disc, delta_softplus=True, delta_bias=inp["delta_bias"])
+    assert_close("y", y, ry, TOL)
+    for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"),
+                      ("dDskip", "D"), ("dz", "z"), ("ddelta_bias", "delta_bias")):
+        assert_close(name, gr[name], rg[ref], TOL)
+    assert plan.device_error() == (0, 0)
+    # the autograd wrapper (lrscan.s6) runs the same kernels
+    g = gpu_inputs(inp)
+    leaves = {k: g[k].clone().requires_grad_(True) for k in ("delta", "delta_bias")}
+    out = lrscan.s6(g["x"], leaves["delta"], g["A"], g["Bm"], g["Cm"], g["Dskip"], g["z"], disc=disc, segment=64,
+                    delta_softplus=True, delta_bias=leaves["delta_bias"])
+    out.backward(g["dy"])
+    assert torch.equal(out, y)
+    assert torch.equal(leaves["delta"].grad, gr["ddelta"]) and torch.equal(leaves["delta_bias"].grad, gr["ddelta_bias"])

@@ -95,6 +95,33 @@ def test_step_parity(kind, shape, io, disc):
         assert_close("state", s_out, rh, tol)
 
 
+@pytest.mark.parametrize("kind", ["s6", "ssd"])
+def test_step_softplus_front_end(kind):
+    """lr_step with dt = softplus(delta + bias)."""
+    shape = dict(B=2, L=5, D=32, N=16) if kind == "s6" else dict(B=2, L=5, H=4, P=16, N=32, G=2)
+    inp = make_inputs(kind, shape, "f32", seed=13)
+    gen = torch.Generator().manual_seed(8)
+    inp["delta"] = torch.randn(inp["delta"].shape, generator=gen) - 1.0
+    inp["delta_bias"] = 0.5 * torch.randn(shape["D"] if kind == "s6" else shape["H"], generator=gen)
+    g = gpu_inputs(api_inputs(kind, inp))
+    desc = lrscan.desc_for(kind, g, 1, "zoh", delta_softplus=True)
+    shp = lrscan.state_shape(desc)
+    y = out_like(kind, g)
+    s_out = torch.empty(shp, dtype=torch.float32, device="cuda")
+    lrscan.step(desc, g, y, s_out)
+    torch.cuda.synchronize()
+    ai = api_inputs(kind, inp)
+    if kind == "s6":
+        ry, rh = oracle.s6_fwd(ai["x"], ai["delta"], ai["A"], ai["Bm"], ai["Cm"], ai.get("Dskip"), ai.get("z"),
+                               disc="zoh", final=True, delta_softplus=True, delta_bias=ai["delta_bias"])
+    else:
+        ry, rh = oracle.ssd_fwd(ai["x"], ai["delta"], ai["A"], ai["Bm"], ai["Cm"], ai.get("Dskip"), ai.get("z"),
+                                disc="zoh", final=True, delta_softplus=True, delta_bias=ai["delta_bias"])
+        rh = np.swapaxes(rh, 2, 3)
+    assert_close("y", y, ry, TOL[torch.float32])
+    assert_close("state", s_out, rh, TOL[torch.float32])
+
+
 @pytest.mark.parametrize("kind,shape,io,disc", CASES[::2])
 def test_step_modes_bitwise(kind, shape, io, disc):
     """One call of L steps == L one-step calls (state in place) == the CUDA-graph decode loop."""

@@ -439,6 +439,39 @@ def test_fd_gla(orc):
               inp, ["q", "k", "v", "g"], dy)
 
 
+def test_softplus_front_end(orc):
+    """delta_softplus: the same scan on dt = softplus(delta + bias) computed outside the oracle by
+    torch's softplus; the raw-delta and bias gradients by finite differences (S6 and SSD)."""
+    import torch
+    rng = np.random.default_rng(19)
+    B, L, D, N = 2, 5, 3, 2
+    inp = {"x": rng.normal(size=(B, L, D)), "delta": rng.normal(-1.0, 1.0, (B, L, D)),
+           "A": -rng.uniform(0.3, 3, (D, N)), "B": rng.normal(size=(B, L, N)),
+           "C": rng.normal(size=(B, L, N)), "D": rng.normal(size=D), "z": rng.normal(size=(B, L, D)),
+           "bias": rng.normal(size=D)}
+    dt = torch.nn.functional.softplus(torch.from_numpy(inp["delta"] + inp["bias"])).numpy()
+    ref = orc.s6_fwd(inp["x"], dt, inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], disc="zoh")
+    got = orc.s6_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], disc="zoh",
+                     delta_softplus=True, delta_bias=inp["bias"])
+    assert rel_err(got, ref) < 1e-14
+    f = lambda i: orc.s6_fwd(i["x"], i["delta"], i["A"], i["B"], i["C"], i["D"], i["z"], disc="zoh",
+                             delta_softplus=True, delta_bias=i["bias"])
+    b2 = lambda i, d: {**(g := orc.s6_bwd(i["x"], i["delta"], i["A"], i["B"], i["C"], i["D"], i["z"], d,
+                                          disc="zoh", delta_softplus=True, delta_bias=i["bias"])),
+                       "bias": g["delta_bias"]}
+    _fd_check(f, b2, inp, ["delta", "bias", "A", "x"], rng.normal(size=(B, L, D)))
+    H, P, Ns, G = 4, 2, 3, 2
+    si = {"x": rng.normal(size=(1, L, H, P)), "delta": rng.normal(-1.0, 1.0, (1, L, H)),
+          "A": -rng.uniform(0.3, 3, H), "B": rng.normal(size=(1, L, G, Ns)), "C": rng.normal(size=(1, L, G, Ns)),
+          "D": rng.normal(size=H), "bias": rng.normal(size=H)}
+    fs = lambda i: orc.ssd_fwd(i["x"], i["delta"], i["A"], i["B"], i["C"], i["D"], None, disc="zoh_euler",
+                               delta_softplus=True, delta_bias=i["bias"])
+    bs = lambda i, d: {**(g := orc.ssd_bwd(i["x"], i["delta"], i["A"], i["B"], i["C"], i["D"], None, d,
+                                           disc="zoh_euler", delta_softplus=True, delta_bias=i["bias"])),
+                       "bias": g["delta_bias"]}
+    _fd_check(fs, bs, si, ["delta", "bias", "A"], rng.normal(size=(1, L, H, P)))
+
+
 # ------------------------------------------------------ P7: execution-mode equivalence
 def test_prefix_and_stepwise_equivalence(orc):
     """Running on a prefix reproduces the full run's first steps (causality), and restarting

@@ -48,9 +48,24 @@ __device__ __forceinline__ float ssd_beta(int disc, float lam, float dt, float A
     return (ex2(lam * kLog2e) - 1.0f) / Ah;
 }
 
+// The kernels come in two variants: the default one (ZOH, raw dt) with both fixed at compile time,
+// and the general one (GEN) that takes the discretisation and the softplus front-end from the
+// arguments.
+template <bool GEN>
+__device__ __forceinline__ int disc_of(const SsdArgs& a) {
+    if constexpr (GEN) return a.disc;
+    return LR_DISC_ZOH;
+}
+template <bool GEN>
+__device__ __forceinline__ bool softplus_of(const SsdArgs& a) {
+    if constexpr (GEN) return a.softplus != 0;
+    return false;
+}
+
 // dt of head h from the raw delta: itself, or softplus(delta + bias_h) (LR_DELTA_SOFTPLUS)
+template <bool GEN>
 __device__ __forceinline__ float ssd_dt(const SsdArgs& a, float raw, int h) {
-    if (!a.softplus) return raw;
+    if (!softplus_of<GEN>(a)) return raw;
     const float v = raw + (a.dbias ? a.dbias[h] : 0.0f);
     return v > 20.0f ? v : log1pf(expf(v));
 }
@@ -118,7 +133,7 @@ template <int NS, bool F32> struct ScanSmem {
     static_assert(kDtRing % kScanPrepGroup == 0 && kDtRing >= 2 * kScanPrepGroup, "dt ring holds two prep groups");
 };
 
-template <int NS, bool F32>
+template <int NS, bool F32, bool GEN>
 __global__ void __launch_bounds__(kScanThreads, 1)
 ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
                 const __grid_constant__ CUtensorMap mS, SsdArgs a, char* __restrict__ tiles, int dir,
@@ -185,7 +200,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
                 ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
                 const float dtv = dtr[(k % kDtRing) * kQ + t];  // 0 past L: no decay
                 l[j] = dtv * Ah;
-                beta[j] = chunk_of(k) * kQ + t < a.L ? ssd_beta(a.disc, l[j], dtv, Ah) : 0.0f;  // no input past L
+                beta[j] = chunk_of(k) * kQ + t < a.L ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
             }
             wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
             if (t == 0) {
@@ -271,7 +286,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < kQ / 32; ++i) {
                     const int k = k0 + j, tt = chunk_of(k) * kQ + lane + 32 * i;
-                    v[j][i] = k < nk && tt < a.L ? ssd_dt(a, __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]), h)
+                    v[j][i] = k < nk && tt < a.L ? ssd_dt<GEN>(a, __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]), h)
                                                  : 0.0f;
                 }
 #pragma unroll
@@ -358,6 +373,7 @@ constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernel
 
 // dt of the CTA's heads at the chunk's steps into shared memory ([head][step], 0 past L), and
 // A_h, D_h of the heads (ad[0 .. kMaxHB), ad[kMaxHB ..)).
+template <bool GEN>
 __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad, int b, int t0, int hfirst, int nh,
                                          int row) {
     if (row < nh) {
@@ -368,7 +384,7 @@ __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad
     const __nv_bfloat16* src = a.dt + ((size_t)b * a.L + (valid ? t0 + row : 0)) * a.H + hfirst;
     float v[kMaxHB];
 #pragma unroll
-    for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? ssd_dt(a, __bfloat162float(src[i]), hfirst + i) : 0.0f;
+    for (int i = 0; i < kMaxHB; ++i) v[i] = (i < nh && valid) ? ssd_dt<GEN>(a, __bfloat162float(src[i]), hfirst + i) : 0.0f;
 #pragma unroll
     for (int i = 0; i < kMaxHB; ++i) dts[i * kQ + row] = v[i];
 }
@@ -405,6 +421,7 @@ __device__ __forceinline__ uint32_t col_y2(int w) { return 256u + 192u * w; }
 //   issue (one thread): Y = P X (A from TMEM), Y2 = C S_in;
 //   finish: y = Y + E Y2 + D x -> the x tile -> TMA store; the freed S_in slot loads the
 //   warpgroup's next head and the x slot freed one head earlier the head after next.
+template <bool GEN>
 __global__ void __launch_bounds__(256, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
@@ -471,7 +488,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             bulk_load(St, stile(hfirst + wg), kTileBytes, &wbar[3]);
         }
     }
-    if (wg == 0) load_dts(a, dts, ad, b, t0, hfirst, nh, wt);
+    if (wg == 0) load_dts<GEN>(a, dts, ad, b, t0, hfirst, nh, wt);
     __syncthreads();
     bool ok = true;
     if (tid == 0) {
@@ -492,7 +509,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         if (t0 + wt < a.L) {
             const float Ah = ad[i];
             lam = dts[i * kQ + wt] * Ah;
-            beta = ssd_beta(a.disc, lam, dts[i * kQ + wt], Ah);
+            beta = ssd_beta(disc_of<GEN>(a), lam, dts[i * kQ + wt], Ah);
         }
         const float lt2 = wg_inclusive_sum(lam, tmp, wg) * kLog2e;
         l2s[wt] = lt2;
@@ -615,6 +632,11 @@ bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
     uint64_t str[3] = {kP * 4, (uint64_t)kKD * kP * 4, (uint64_t)BH * kKD * kP * 4};
     uint32_t box[4] = {32, (uint32_t)kKD, 1, 1};
     return make_tmap(m, base, 4, 4, dims, str, box, true);
+}
+
+// The general kernel variant: a discretisation other than ZOH, or the softplus front-end.
+bool general_variant(const lr_desc& d) {
+    return d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS);
 }
 
 struct SsdFwdWs {
@@ -755,6 +777,7 @@ constexpr int kLoader = 160;
 //   E2: dx, the inter-chunk row dots, dy scaled by E and x by w in place;
 //   batch 2: diag(E) dy S_in^T, diag(w) x G^T into dC, dB, issued with phase A of head i + 1
 //     (M = C B^T, S2 = dy x^T) while warpgroup 0 turns head i's row terms into d dt.
+template <bool GEN>
 __global__ void __launch_bounds__(256, 1)
 ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                 const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY, SsdGradArgs ga,
@@ -843,7 +866,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (t0 + row < a.L) {
             const float Ah = ad[i];
             lam = dts[i * kQ + row] * Ah;
-            beta = ssd_beta(a.disc, lam, dts[i * kQ + row], Ah);
+            beta = ssd_beta(disc_of<GEN>(a), lam, dts[i * kQ + row], Ah);
         }
         const float lt = wg0_inclusive_sum(lam, tmp);
         l2s[row] = lt * kLog2e;
@@ -867,7 +890,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     pdl_wait();  // the G tiles (and the zeroed dB, dC) come from the previous kernel
     if (tid == 0) load_sg(hfirst);
     if (wg == 0) {
-        load_dts(a, dts, ad, b, t0, hfirst, nh, row);
+        load_dts<GEN>(a, dts, ad, b, t0, hfirst, nh, row);
         wg0_bar();
         decays(0);
     }
@@ -1101,11 +1124,13 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 const float ab = ex2(dt_raw * Ah * kLog2e);
                 const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
                 // d beta / d dt: ZOH e^{dt A}, ZOH-Euler 1, dirac 0;  d beta / dA: ZOH only
-                const float dbdt = a.disc == LR_DISC_ZOH ? ab : (a.disc == LR_DISC_ZOH_EULER ? 1.0f : 0.0f);
+                const int disc = disc_of<GEN>(a);
+                const float dbdt = disc == LR_DISC_ZOH ? ab : (disc == LR_DISC_ZOH_EULER ? 1.0f : 0.0f);
                 // softplus front-end: d delta = d dt sigma(delta + bias), sigma(delta + bias) = 1 - e^{-dt}
-                ddr = (dlam * Ah + dbeta * dbdt) * (a.softplus ? -expm1f(-dt_raw) : 1.0f);
+                ddr = dlam * Ah + dbeta * dbdt;
+                if (softplus_of<GEN>(a)) ddr *= -expm1f(-dt_raw);
                 ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(ddr);
-                dA_part = dlam * dt_raw + (a.disc == LR_DISC_ZOH ? dbeta * (dt_raw * ab - bt) / Ah : 0.0f);
+                dA_part = dlam * dt_raw + (disc == LR_DISC_ZOH ? dbeta * (dt_raw * ab - bt) / Ah : 0.0f);
             }
             const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
             const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
@@ -1113,7 +1138,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 ga.pdA[tile] = sAD.x;
                 ga.pdD[tile] = sAD.y;
             }
-            if (a.softplus) {  // uniform: the d bias partial of this (row, head, chunk)
+            if (softplus_of<GEN>(a)) {  // uniform: the d bias partial of this (row, head, chunk)
                 const float2 sE = wg0_sum2(ddr, 0.0f, tmp);
                 if (t == 0) ga.pdE[tile] = sE.x;
             }
@@ -1224,13 +1249,14 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
     char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     if (!ok) return LR_ERR_INVALID_ARG;
+    const bool gen = general_variant(d);
     using ScanF = ScanSmem<3, true>;
-    cudaFuncSetAttribute(ssd_scan_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
+    auto scan = gen ? ssd_scan_kernel<3, true, true> : ssd_scan_kernel<3, true, false>;
+    cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
     note_launch("ssd_state_scan");
     CUtensorMap mS;
     if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
-    if (launch_pdl(ssd_scan_kernel<3, true>, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, a,
-                   stiles, +1,
+    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, a, stiles, +1,
                    (float4*)nullptr, (float4*)nullptr, (size_t)0) != cudaSuccess)
         return LR_ERR_CUDA;
     {
@@ -1239,9 +1265,10 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     }
     const int hb = out_heads_per_cta(d, a.nchunk);
     const int nblk_o = (a.HpG + hb - 1) / hb;
-    cudaFuncSetAttribute(ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
+    auto out = gen ? ssd_out_kernel<true> : ssd_out_kernel<false>;
+    cudaFuncSetAttribute(out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
-    if (launch_pdl(ssd_out_kernel, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
+    if (launch_pdl(out, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
                    a, (const char*)stiles, hb, nblk_o) != cudaSuccess)
         return LR_ERR_CUDA;
     return check_launch();
@@ -1275,19 +1302,20 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     {
         const size_t nzero4 = ga.accumulate ? (size_t)d.B * d.L * d.G * kKD / 4 : 0;
         using ScanB = ScanSmem<4, false>;
-        cudaFuncSetAttribute(ssd_scan_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
+        auto scan = general_variant(d) ? ssd_scan_kernel<4, false, true> : ssd_scan_kernel<4, false, false>;
+        cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
         note_launch("ssd_state_scan");
         // no f32 states in this direction (the map argument is unused)
-        if (launch_pdl(ssd_scan_kernel<4, false>, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC,
-                       a,
-                       ws + w.gtiles, -1, (float4*)gr.dBm, (float4*)gr.dCm, nzero4) != cudaSuccess)
+        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, a, ws + w.gtiles, -1,
+                       (float4*)gr.dBm, (float4*)gr.dCm, nzero4) != cudaSuccess)
             return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
-    cudaFuncSetAttribute(ssd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
+    auto grad = general_variant(d) ? ssd_grad_kernel<true> : ssd_grad_kernel<false>;
+    cudaFuncSetAttribute(grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
     note_launch("ssd_chunk_grad");
-    if (launch_pdl(ssd_grad_kernel, dim3(a.nchunk * a.B * a.G * nblk), dim3(256), GradSmem::kAlloc, st, mC, mB, mX, mdY,
+    if (launch_pdl(grad, dim3(a.nchunk * a.B * a.G * nblk), dim3(256), GradSmem::kAlloc, st, mC, mB, mX, mdY,
                    ga, hb, nblk) != cudaSuccess)
         return LR_ERR_CUDA;
     lr_status s = check_launch();

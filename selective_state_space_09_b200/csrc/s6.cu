@@ -101,9 +101,11 @@ struct S6Args {
 
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
 
-// dt of one step: the raw delta, or softplus(delta + bias) (LR_DELTA_SOFTPLUS)
-__device__ __forceinline__ float step_dt(const S6Args& a, float raw, float bias) {
-    return a.softplus ? softplus_f(raw + bias) : raw;
+// dt of one step: the raw delta, or softplus(delta + bias) (SP: LR_DELTA_SOFTPLUS)
+template <bool SP>
+__device__ __forceinline__ float step_dt(float raw, float bias) {
+    if constexpr (SP) return softplus_f(raw + bias);
+    return raw;
 }
 
 // Per-thread constants of the discretisation for its 8 states.
@@ -148,7 +150,7 @@ constexpr size_t kTileBC = size_t(kMaxS) * kN * 2;   // [S][16] bf16
 constexpr size_t kFwdStage = 3 * kTileDT + 2 * kTileBC;
 constexpr size_t kFwdSmem = 128 + 2 * kFwdStage + 128;
 
-template <int DISC, bool FULL>
+template <int DISC, bool FULL, bool SP>
 __global__ void __launch_bounds__(kThreads)
 s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mB,
@@ -190,7 +192,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
-    const float dbias = (a.softplus && a.dbias && dok) ? a.dbias[d] : 0.0f;
+    const float dbias = (SP && a.dbias && dok) ? a.dbias[d] : 0.0f;
     float h[kNH];
 #pragma unroll
     for (int j = 0; j < kNH; ++j) h[j] = 0.0f;
@@ -217,7 +219,7 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         const __nv_bfloat16* Cs = stageBC(s, 1);
         if (ok) {
             for (int t = 0; t < nt; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
+                const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
                 float Bv[kNH], Cv[kNH];
                 ldn(Bs + t * kN + part * kNH, Bv);
                 ldn(Cs + t * kN + part * kNH, Cv);
@@ -266,7 +268,7 @@ constexpr size_t kOffRed = kOffBnd + kBndBytes;
 constexpr size_t kRedBytes = size_t(kWarps) * kSub * 2 * kN * 4;  // per-warp dB / dC of one sub-block
 constexpr size_t kBwdSmem = kOffRed + kRedBytes + 128;
 
-template <int DISC, bool FULL>
+template <int DISC, bool FULL, bool SP>
 __global__ void __launch_bounds__(kThreads)
 s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mDY,
@@ -303,7 +305,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         c.ia[j] = 1.0f / A;
     }
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
-    const float dbias = (a.softplus && a.dbias && dok) ? a.dbias[d] : 0.0f;
+    const float dbias = (SP && a.dbias && dok) ? a.dbias[d] : 0.0f;
     float G[kNH], anext[kNH], dA[kNH];
 #pragma unroll
     for (int j = 0; j < kNH; ++j) G[j] = anext[j] = dA[j] = 0.0f;
@@ -341,7 +343,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int j = 0; j < kNH; ++j) bp[j] = h[j];
             const int te = min(nt, (sb + 1) * kSub);
             for (int t = sb * kSub; t < te; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
+                const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
                 float Bv[kNH];
                 ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -378,7 +380,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                 for (int i = 0; i < kSub; ++i) {  // h after step i from the state entering it
                     if (i < n) {
                         const int t = tb + i;
-                        const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
+                        const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
                         float Bv[kNH];
                         ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -395,7 +397,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int i = 0; i < kSub; ++i) {
                 if (i < n && !FULL) {
                     const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
+                    const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
                     float Bv[kNH];
                     ldn(Bs + t * kN + part * kNH, Bv);
 #pragma unroll
@@ -412,7 +414,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             for (int i = kSub - 1; i >= 0; --i) {
                 if (i < n) {
                     const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = step_dt(a, bf(DT + t * kDB + dl), dbias);
+                    const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
                     const float dyv = bf(DY + t * kDB + dl);
                     float Bv[kNH], Cv[kNH];
                     ldn(Bs + t * kN + part * kNH, Bv);
@@ -480,7 +482,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                     if (part == 0) {
                         // softplus: d delta = d dt sigma(delta + bias), and sigma(delta + bias) =
                         // 1 - e^{-dt}
-                        const float ddr = a.softplus ? dta * -expm1f(-dt) : dta;
+                        const float ddr = SP ? dta * -expm1f(-dt) : dta;
                         dE += ddr;
                         X[t * kDB + dl] = __float2bfloat16_rn(fmaf(ds, Dd, dxa));
                         DT[t * kDB + dl] = __float2bfloat16_rn(ddr);
@@ -516,7 +518,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
 #pragma unroll
         for (int j = 0; j < kNH; ++j) pa[j] = dA[j];
         if (part == 0) a.pdD[(size_t)b * a.D + d] = dD;
-        if (part == 0 && a.softplus) a.pdE[(size_t)b * a.D + d] = dE;
+        if (part == 0 && SP) a.pdE[(size_t)b * a.D + d] = dE;
     }
     if (tid == 0) bulk_wait_read_all();
 }
@@ -608,6 +610,17 @@ void set_smem(F fn, size_t bytes) {
     cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+template <int DISC>
+auto fwd_variant(bool full, bool sp) {
+    return full ? (sp ? s6_fwd_kernel<DISC, true, true> : s6_fwd_kernel<DISC, true, false>)
+                : (sp ? s6_fwd_kernel<DISC, false, true> : s6_fwd_kernel<DISC, false, false>);
+}
+template <int DISC>
+auto bwd_variant(bool full, bool sp) {
+    return full ? (sp ? s6_bwd_kernel<DISC, true, true> : s6_bwd_kernel<DISC, true, false>)
+                : (sp ? s6_bwd_kernel<DISC, false, true> : s6_bwd_kernel<DISC, false, false>);
+}
+
 }  // namespace
 
 bool s6_supported(const lr_desc& d) {
@@ -636,23 +649,13 @@ lr_status s6_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, cha
         note_launch(name);
         kernel<<<grid, kThreads, kFwdSmem, st>>>(mX, mDT, mZ, mB, mC, mY, a);
     };
-    // LR_FULL_STATE: the state entering every step is checkpointed (compile-time variant)
-    const bool full = (d.flags & LR_FULL_STATE) != 0;
+    // compile-time variants: LR_FULL_STATE (every step's state checkpointed) and LR_DELTA_SOFTPLUS
+    const bool full = (d.flags & LR_FULL_STATE) != 0, sp = a.softplus != 0;
     switch (d.disc) {
-        case LR_DISC_ZOH:
-            run(full ? s6_fwd_kernel<LR_DISC_ZOH, true> : s6_fwd_kernel<LR_DISC_ZOH, false>, "s6_fwd_zoh");
-            break;
-        case LR_DISC_BILINEAR:
-            run(full ? s6_fwd_kernel<LR_DISC_BILINEAR, true> : s6_fwd_kernel<LR_DISC_BILINEAR, false>,
-                "s6_fwd_bilinear");
-            break;
-        case LR_DISC_DIRAC:
-            run(full ? s6_fwd_kernel<LR_DISC_DIRAC, true> : s6_fwd_kernel<LR_DISC_DIRAC, false>, "s6_fwd_dirac");
-            break;
-        default:
-            run(full ? s6_fwd_kernel<LR_DISC_ZOH_EULER, true> : s6_fwd_kernel<LR_DISC_ZOH_EULER, false>,
-                "s6_fwd_zoh_euler");
-            break;
+        case LR_DISC_ZOH: run(fwd_variant<LR_DISC_ZOH>(full, sp), "s6_fwd_zoh"); break;
+        case LR_DISC_BILINEAR: run(fwd_variant<LR_DISC_BILINEAR>(full, sp), "s6_fwd_bilinear"); break;
+        case LR_DISC_DIRAC: run(fwd_variant<LR_DISC_DIRAC>(full, sp), "s6_fwd_dirac"); break;
+        default: run(fwd_variant<LR_DISC_ZOH_EULER>(full, sp), "s6_fwd_zoh_euler"); break;
     }
     return check_launch();
 }
@@ -678,22 +681,12 @@ lr_status s6_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const vo
         note_launch(name);
         kernel<<<grid, kThreads, kBwdSmem, st>>>(mX, mDT, mZ, mDY, mB, mC, mdX, mdDT, mdZ, a);
     };
-    const bool full = (d.flags & LR_FULL_STATE) != 0;  // the states are read, not recomputed
+    const bool full = (d.flags & LR_FULL_STATE) != 0, sp = a.softplus != 0;  // compile-time variants
     switch (d.disc) {
-        case LR_DISC_ZOH:
-            run(full ? s6_bwd_kernel<LR_DISC_ZOH, true> : s6_bwd_kernel<LR_DISC_ZOH, false>, "s6_bwd_zoh");
-            break;
-        case LR_DISC_BILINEAR:
-            run(full ? s6_bwd_kernel<LR_DISC_BILINEAR, true> : s6_bwd_kernel<LR_DISC_BILINEAR, false>,
-                "s6_bwd_bilinear");
-            break;
-        case LR_DISC_DIRAC:
-            run(full ? s6_bwd_kernel<LR_DISC_DIRAC, true> : s6_bwd_kernel<LR_DISC_DIRAC, false>, "s6_bwd_dirac");
-            break;
-        default:
-            run(full ? s6_bwd_kernel<LR_DISC_ZOH_EULER, true> : s6_bwd_kernel<LR_DISC_ZOH_EULER, false>,
-                "s6_bwd_zoh_euler");
-            break;
+        case LR_DISC_ZOH: run(bwd_variant<LR_DISC_ZOH>(full, sp), "s6_bwd_zoh"); break;
+        case LR_DISC_BILINEAR: run(bwd_variant<LR_DISC_BILINEAR>(full, sp), "s6_bwd_bilinear"); break;
+        case LR_DISC_DIRAC: run(bwd_variant<LR_DISC_DIRAC>(full, sp), "s6_bwd_dirac"); break;
+        default: run(bwd_variant<LR_DISC_ZOH_EULER>(full, sp), "s6_bwd_zoh_euler"); break;
     }
     lr_status s = check_launch();
     if (s != LR_OK) return s;

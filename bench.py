@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fwd+bwd scan tokens/s & achieved HBM GB/s (% of B200 peak) per scan kind"
-BENCH_ORDER = ["ssd", "rglru", "gla", "s6_zoh", "s6_bilinear", "rotlru"]
+BENCH_ORDER = ["ssd", "rglru", "gla", "s6_zoh", "s6_bilinear", "rotlru", "ssd_mamba2"]
 NAMES = {
     "ssd": "Mamba-2 SSD scan (mamba-370m-like), bf16, B=2 H=32 P=64 N=128 L=4096, chunk 128, S=128, ZOH",
     "rglru": "rglru_scan, f32, B=1 D=256 L=1024, S=128",
@@ -41,10 +41,13 @@ NAMES = {
     "s6_zoh": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, ZOH, D skip + silu(z)",
     "s6_bilinear": "Mamba-1 S6 selective scan, bf16, B=8 D=2048 N=16 L=2048, S=64, bilinear, D skip + silu(z)",
     "rotlru": "rotlru_scan, f32, B=16 D=4096 L=16384, S=256",
+    "ssd_mamba2": "SSD scan, Mamba-2 step length: dt = softplus(delta + bias) in-kernel, ZOH-Euler (beta = dt), "
+                  "bf16, B=2 H=32 P=64 N=128 L=4096, chunk 128, S=128",
 }
 INPUT_NAMES = {
     "rglru": ["a", "b"], "rotlru": ["b", "g", "mag", "theta"],
-    "s6": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z"], "ssd": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z"],
+    "s6": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"],
+    "ssd": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"],
     "gla": ["q", "k", "v", "g"],
 }
 FALLBACK_HBM = 6650.0
@@ -305,7 +308,7 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
     w, inp = workload_inputs(name, device, seed=1000 + rank)
     kind = w["kind"]
     ai = api_inputs(kind, inp)
-    plan = lrscan.plan_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0))
+    plan = lrscan.plan_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0), w.get("softplus", False))
     y, grads = lrscan.alloc_outputs(kind, ai)
     dy = inp["dy"]
 
@@ -470,11 +473,11 @@ def run_decode(kind, ai, w, T=256, reps=20):
     seq = {n: (v[:, :T].transpose(0, 1).unsqueeze(2).contiguous() if n in toks and v is not None else v)
            for n, v in ai.items()}
     first = {n: (v[0] if n in toks and v is not None else v) for n, v in seq.items()}
-    desc = lrscan.desc_for(kind, first, 1, w.get("disc", "none"))
+    desc = lrscan.desc_for(kind, first, 1, w.get("disc", "none"), delta_softplus=w.get("softplus", False))
     state = torch.zeros(lrscan.state_shape(desc), dtype=torch.float32, device=ai[toks[0]].device)
     out = ai["v"] if kind == "gla" else (ai["b"] if kind in ("rglru", "rotlru") else ai["x"])
     y = torch.empty((T, out.shape[0], 1) + tuple(out.shape[2:]), dtype=out.dtype, device=out.device)
-    graph = lrscan.DecodeGraph(kind, seq, state, y, w.get("disc", "none"))
+    graph = lrscan.DecodeGraph(kind, seq, state, y, w.get("disc", "none"), w.get("softplus", False))
     for _ in range(3):
         graph.replay()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -487,8 +490,13 @@ def run_decode(kind, ai, w, T=256, reps=20):
     ms = e0.elapsed_time(e1)
     us = ms * 1e3 / (T * reps)
     B = out.shape[0]
+    tok_bytes = sum(v[0].numel() * v.element_size() for n, v in seq.items() if n in toks and v is not None)
+    step_bytes = 2 * state.numel() * 4 + tok_bytes + y[0].numel() * y.element_size()  # state in and out
     return {"tokens_per_s": B / (us * 1e-6), "us_per_step": round(us, 3), "batch": B, "steps_per_graph": T,
-            "state_bytes": state.numel() * 4, "kernel": lrscan.last_dispatch() or kind + "_step"}
+            "state_bytes": state.numel() * 4, "bytes_per_step": step_bytes,
+            "achieved_gbs": round(step_bytes / (us * 1e-6) / 1e9, 1),
+            "note": "state L2-resident between steps: latency / launch bound",
+            "kernel": lrscan.last_dispatch() or kind + "_step"}
 
 
 def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
@@ -543,6 +551,7 @@ SAMPLES = {
     # workload: (slice description, slicer of the CPU inputs, fraction of one step's tokens)
     "rglru": "the whole workload",
     "ssd": "batch row 0, heads 0-3 of 32, full L=4096",
+    "ssd_mamba2": "batch row 0, heads 0-3 of 32, full L=4096",
     "gla": "batch row 0, heads 0-1 of 16, full L=2048",
     "s6_zoh": "batch row 0, channels 0-127 of 2048, full L=2048",
     "s6_bilinear": "batch row 0, channels 0-127 of 2048, full L=2048",
@@ -560,7 +569,7 @@ def oracle_sample(name):
         inp = inputs.rglru(w["B"], w["L"], w["D"], seed=0)
         return kind, inp, 1.0, w
     if kind == "ssd":
-        inp = inputs.ssd(1, w["L"], 4, w["P"], w["N"], 1, seed=0)
+        inp = inputs.workload(name, seed=0, B=1, H=4)
         return kind, inp, (1 / w["B"]) * (4 / w["H"]), w
     if kind == "gla":
         inp = inputs.gla(1, w["L"], 2, w["K"], w["V"], seed=0)
@@ -588,8 +597,9 @@ def oracle_step(kind, inp, w):
         oracle.s6_bwd(*a, inp["dy"], disc=w["disc"])
     elif kind == "ssd":
         a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"])
-        oracle.ssd_fwd(*a, disc=w["disc"], S=w["segment"])
-        oracle.ssd_bwd(*a, inp["dy"], disc=w["disc"])
+        sp = dict(delta_softplus=True, delta_bias=inp["delta_bias"]) if w.get("softplus") else {}
+        oracle.ssd_fwd(*a, disc=w["disc"], S=w["segment"], **sp)
+        oracle.ssd_bwd(*a, inp["dy"], disc=w["disc"], **sp)
     elif kind == "gla":
         oracle.gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], S=w["segment"])
         oracle.gla_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["dy"])
@@ -639,7 +649,10 @@ def built_workloads():
         if kind == "gla":
             w["N"], w["P"] = w.pop("K"), w.pop("V")
         seg = w.pop("segment")
+        softplus = w.pop("softplus", False)
         d = lrscan.make_desc(kind, io, segment=seg, **w)
+        if softplus:
+            d.flags |= lrscan.DELTA_SOFTPLUS
         if lrscan.validate(d) == 0:
             ok.append(name)
     return ok

@@ -48,6 +48,28 @@ __device__ __forceinline__ float ssd_beta(int disc, float lam, float dt, float A
     return (ex2(lam * kLog2e) - 1.0f) / Ah;
 }
 
+// Sums of three values over the 128 threads of warpgroup 0, fixed order, results in every thread
+// (tmp: 32 floats, the layout wg0_sum2 uses for two).
+__device__ __forceinline__ float3 wg0_sum3(float x, float y, float z, float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+        y += __shfl_xor_sync(0xffffffffu, y, o);
+        z += __shfl_xor_sync(0xffffffffu, z, o);
+    }
+    if (lane == 0) {
+        tmp[8 + warp] = x;
+        tmp[12 + warp] = y;
+        tmp[16 + warp] = z;
+    }
+    wg0_bar();
+    const float3 s = make_float3((tmp[8] + tmp[9]) + (tmp[10] + tmp[11]), (tmp[12] + tmp[13]) + (tmp[14] + tmp[15]),
+                                 (tmp[16] + tmp[17]) + (tmp[18] + tmp[19]));
+    wg0_bar();
+    return s;
+}
+
 // The kernels come in two variants: the default one (ZOH, raw dt) with both fixed at compile time,
 // and the general one (GEN) that takes the discretisation and the softplus front-end from the
 // arguments.
@@ -67,7 +89,7 @@ template <bool GEN>
 __device__ __forceinline__ float ssd_dt(const SsdArgs& a, float raw, int h) {
     if (!softplus_of<GEN>(a)) return raw;
     const float v = raw + (a.dbias ? a.dbias[h] : 0.0f);
-    return v > 20.0f ? v : log1pf(expf(v));
+    return v > 20.0f ? v : log1pf(__expf(v));
 }
 
 // Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
@@ -198,9 +220,10 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             for (int j = 0; j < NG; ++j) {
                 const int k = k0 + j;
                 ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
-                const float dtv = dtr[(k % kDtRing) * kQ + t];  // 0 past L: no decay
+                const bool in_seq = chunk_of(k) * kQ + t < a.L;
+                const float dtv = in_seq ? ssd_dt<GEN>(a, dtr[(k % kDtRing) * kQ + t], h) : 0.0f;  // 0 past L
                 l[j] = dtv * Ah;
-                beta[j] = chunk_of(k) * kQ + t < a.L ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
+                beta[j] = in_seq ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
             }
             wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
             if (t == 0) {
@@ -286,8 +309,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < kQ / 32; ++i) {
                     const int k = k0 + j, tt = chunk_of(k) * kQ + lane + 32 * i;
-                    v[j][i] = k < nk && tt < a.L ? ssd_dt<GEN>(a, __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]), h)
-                                                 : 0.0f;
+                    v[j][i] = k < nk && tt < a.L ? __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]) : 0.0f;
                 }
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
@@ -1132,15 +1154,20 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(ddr);
                 dA_part = dlam * dt_raw + (disc == LR_DISC_ZOH ? dbeta * (dt_raw * ab - bt) / Ah : 0.0f);
             }
-            const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
             const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
-            if (t == 0) {
-                ga.pdA[tile] = sAD.x;
-                ga.pdD[tile] = sAD.y;
-            }
-            if (softplus_of<GEN>(a)) {  // uniform: the d bias partial of this (row, head, chunk)
-                const float2 sE = wg0_sum2(ddr, 0.0f, tmp);
-                if (t == 0) ga.pdE[tile] = sE.x;
+            if (!softplus_of<GEN>(a)) {
+                const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
+                if (t == 0) {
+                    ga.pdA[tile] = sAD.x;
+                    ga.pdD[tile] = sAD.y;
+                }
+            } else {  // uniform: also the d bias partial of this (row, head, chunk)
+                const float3 sADE = wg0_sum3(dA_part, valid ? ddv : 0.0f, ddr, tmp);
+                if (t == 0) {
+                    ga.pdA[tile] = sADE.x;
+                    ga.pdD[tile] = sADE.y;
+                    ga.pdE[tile] = sADE.z;
+                }
             }
         }
     }

@@ -41,6 +41,10 @@ WORKLOADS = {
     "s6_bilinear": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64,
                         disc="bilinear"),
     "rotlru": dict(kind="rotlru", io="f32", B=16, D=4096, L=16384, segment=256),
+    # the SSD workload's shapes through the general kernel variant, as Mamba-2 layers run it:
+    # dt = softplus(delta + bias) in the kernels, abar = e^{dt A}, beta = dt (ZOH-Euler)
+    "ssd_mamba2": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=128,
+                       segment=128, disc="zoh_euler", softplus=True),
 }
 
 _DT = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -142,7 +146,13 @@ def workload(name, seed=0, device="cpu", **override):
     if k == "s6":
         return s6(w["B"], w["L"], w["D"], w["N"], seed, w["io"], device)
     if k == "ssd":
-        return ssd(w["B"], w["L"], w["H"], w["P"], w["N"], w.get("G", 1), seed, w["io"], device)
+        inp = ssd(w["B"], w["L"], w["H"], w["P"], w["N"], w.get("G", 1), seed, w["io"], device)
+        if w.get("softplus"):  # raw step lengths N(-2, 1) and a bias U(-1, 0) per head, drawn after
+            g = torch.Generator(device="cpu").manual_seed(seed + 7919)
+            raw = torch.randn(inp["delta"].shape, generator=g) - 2.0
+            inp["delta"] = raw.to(_DT[w["io"]]).to(device)
+            inp["delta_bias"] = (-torch.rand(w["H"], generator=g)).to(device)
+        return inp
     if k == "gla":
         return gla(w["B"], w["L"], w["H"], w["K"], w["V"], seed, w["io"], device)
     raise KeyError(k)

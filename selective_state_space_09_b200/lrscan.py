@@ -258,12 +258,12 @@ class DecodeGraph:
     inputs are ``seq[name][t]``), parameters as usual; ``state``: the f32 state, advanced in place;
     ``y``: [T, B, 1, ...] outputs.  Every replay continues from whatever ``state`` holds."""
 
-    def __init__(self, kind, seq, state, y, disc="none"):
+    def __init__(self, kind, seq, state, y, disc="none", delta_softplus=False):
         toks = TOKEN_INPUTS[kind]
         T = y.shape[0]
         self.kind, self.T, self.state, self.y = kind, T, state, y
         first = {n: (seq[n][0] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}
-        self.desc = desc_for(kind, first, 1, disc)
+        self.desc = desc_for(kind, first, 1, disc, delta_softplus=delta_softplus)
         self.calls = [({n: (seq[n][t] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}, y[t])
                       for t in range(T)]
         side = torch.cuda.Stream()

@@ -128,6 +128,39 @@ def rglru_bwd(a, b, dy):
     return {"a": da, "b": db}
 
 
+# --------------------------------------------------------------------- rglru with gate front-end
+RG_LRU_C = 8.0  # the exponent constant of a = sigmoid(Lambda)^(c r)
+
+
+def _rg_gates(r, i, x, lam):
+    """a = sigmoid(Lambda)^(c r), s = sqrt(1 - a^2), b = s (i x): the RG-LRU gate front-end."""
+    logsig = -np.logaddexp(0.0, -lam)          # log sigmoid(Lambda), per channel
+    a = np.exp(RG_LRU_C * r * logsig)
+    s = np.sqrt(1.0 - a * a)
+    return a, s, s * i * x, logsig
+
+
+def rglru_gated_fwd(r, i, x, lam, S=0, h0=None, final=False):
+    """rglru on the gates: a = sigmoid(Lambda)^(c r), b = sqrt(1 - a^2) (i x) (r, i, x: [B, L, D],
+    Lambda: [D]); the recurrence itself is the rglru oracle above."""
+    r, i, x, lam = map(_f64, (r, i, x, lam))
+    a, _, b, _ = _rg_gates(r, i, x, lam)
+    return rglru_fwd(a, b, S=S, h0=h0, final=final)
+
+
+def rglru_gated_bwd(r, i, x, lam, dy):
+    """Gradients of the gated rglru by the chain rule through the rglru oracle's (da, db):
+    di = db s x, dx = db s i, da_tot = da - db (i x) a / s, dr = da_tot a c log sigmoid(Lambda),
+    dLambda = sum_{b,t} da_tot a c r (1 - sigmoid(Lambda))."""
+    r, i, x, lam, dy = map(_f64, (r, i, x, lam, dy))
+    a, s, b, logsig = _rg_gates(r, i, x, lam)
+    g = rglru_bwd(a, b, dy)
+    da_tot = g["a"] - g["b"] * i * x * a / s
+    sig = 0.5 * (1.0 + np.tanh(0.5 * lam))
+    return {"r": da_tot * a * RG_LRU_C * logsig, "i": g["b"] * s * x, "x": g["b"] * s * i,
+            "lam": (da_tot * a * RG_LRU_C * r * (1.0 - sig)).sum(axis=(0, 1))}
+
+
 # --------------------------------------------------------------------------------------- rotlru
 def rotlru_fwd(b, g, mag, theta, S=0, h0=None, final=False):
     b, g, mag, theta = _f64(b), _f64(g), _f64(mag), _f64(theta)

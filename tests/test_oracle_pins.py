@@ -472,6 +472,24 @@ def test_softplus_front_end(orc):
     _fd_check(fs, bs, si, ["delta", "bias", "A"], rng.normal(size=(1, L, H, P)))
 
 
+def test_rglru_gate_front_end(orc):
+    """RG-LRU gates: the output is rglru on a = sigmoid(Lambda)^(8 r), b = sqrt(1 - a^2) i x
+    evaluated here with torch (a separate evaluation of the gate formulas); all four gradients by
+    finite differences."""
+    import torch
+    rng = np.random.default_rng(29)
+    B, L, D = 2, 6, 3
+    inp = {"r": rng.uniform(0.05, 0.95, (B, L, D)), "i": rng.uniform(0.05, 0.95, (B, L, D)),
+           "x": rng.normal(size=(B, L, D)), "lam": rng.uniform(2.0, 6.0, D)}
+    t = {k: torch.from_numpy(v) for k, v in inp.items()}
+    a = torch.sigmoid(t["lam"]) ** (8.0 * t["r"])
+    b = torch.sqrt(1.0 - a * a) * t["i"] * t["x"]
+    assert rel_err(orc.rglru_gated_fwd(inp["r"], inp["i"], inp["x"], inp["lam"]), orc.rglru_fwd(a.numpy(), b.numpy())) < 1e-14
+    _fd_check(lambda q: orc.rglru_gated_fwd(q["r"], q["i"], q["x"], q["lam"]),
+              lambda q, d: orc.rglru_gated_bwd(q["r"], q["i"], q["x"], q["lam"], d),
+              inp, ["r", "i", "x", "lam"], rng.normal(size=(B, L, D)))
+
+
 # ------------------------------------------------------ P7: execution-mode equivalence
 def test_prefix_and_stepwise_equivalence(orc):
     """Running on a prefix reproduces the full run's first steps (causality), and restarting

@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fwd+bwd scan tokens/s & achieved HBM GB/s (% of B200 peak) per scan kind"
-BENCH_ORDER = ["ssd", "rglru", "gla", "s6_zoh", "s6_bilinear", "rotlru", "ssd_mamba2"]
+BENCH_ORDER = ["ssd", "rglru", "gla", "s6_zoh", "s6_bilinear", "rotlru", "ssd_mamba2", "rglru_gated"]
 NAMES = {
     "ssd": "Mamba-2 SSD scan (mamba-370m-like), bf16, B=2 H=32 P=64 N=128 L=4096, chunk 128, S=128, ZOH",
     "rglru": "rglru_scan, f32, B=1 D=256 L=1024, S=128",
@@ -43,9 +43,11 @@ NAMES = {
     "rotlru": "rotlru_scan, f32, B=16 D=4096 L=16384, S=256",
     "ssd_mamba2": "SSD scan, Mamba-2 step length: dt = softplus(delta + bias) in-kernel, ZOH-Euler (beta = dt), "
                   "bf16, B=2 H=32 P=64 N=128 L=4096, chunk 128, S=128",
+    "rglru_gated": "rglru_scan with the RG-LRU gates in-kernel (a = sigmoid(Lambda)^(8 r), b = sqrt(1 - a^2) i x), "
+                   "f32, B=1 D=256 L=1024, S=128",
 }
 INPUT_NAMES = {
-    "rglru": ["a", "b"], "rotlru": ["b", "g", "mag", "theta"],
+    "rglru": ["a", "b", "x", "A"], "rotlru": ["b", "g", "mag", "theta"],
     "s6": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"],
     "ssd": ["x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"],
     "gla": ["q", "k", "v", "g"],
@@ -308,7 +310,8 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
     w, inp = workload_inputs(name, device, seed=1000 + rank)
     kind = w["kind"]
     ai = api_inputs(kind, inp)
-    plan = lrscan.plan_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0), w.get("softplus", False))
+    plan = lrscan.plan_for(kind, ai, w["segment"], w.get("disc", "none"), w.get("chunk", 0), w.get("softplus", False),
+                           w.get("gates", False))
     y, grads = lrscan.alloc_outputs(kind, ai)
     dy = inp["dy"]
 
@@ -417,7 +420,7 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
     if world == 1:
         res["decode"] = run_decode(kind, ai, w)
-        if kind in ("rglru", "rotlru", "s6"):
+        if kind in ("rglru", "rotlru", "s6") and not w.get("gates"):
             res["full_state"] = run_full_state(kind, ai, dy, w, plan, steps, flush)
     del fl
     return res
@@ -473,11 +476,13 @@ def run_decode(kind, ai, w, T=256, reps=20):
     seq = {n: (v[:, :T].transpose(0, 1).unsqueeze(2).contiguous() if n in toks and v is not None else v)
            for n, v in ai.items()}
     first = {n: (v[0] if n in toks and v is not None else v) for n, v in seq.items()}
-    desc = lrscan.desc_for(kind, first, 1, w.get("disc", "none"), delta_softplus=w.get("softplus", False))
+    desc = lrscan.desc_for(kind, first, 1, w.get("disc", "none"), delta_softplus=w.get("softplus", False),
+                           gates=w.get("gates", False))
     state = torch.zeros(lrscan.state_shape(desc), dtype=torch.float32, device=ai[toks[0]].device)
     out = ai["v"] if kind == "gla" else (ai["b"] if kind in ("rglru", "rotlru") else ai["x"])
     y = torch.empty((T, out.shape[0], 1) + tuple(out.shape[2:]), dtype=out.dtype, device=out.device)
-    graph = lrscan.DecodeGraph(kind, seq, state, y, w.get("disc", "none"), w.get("softplus", False))
+    graph = lrscan.DecodeGraph(kind, seq, state, y, w.get("disc", "none"), w.get("softplus", False),
+                               w.get("gates", False))
     for _ in range(3):
         graph.replay()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -550,6 +555,7 @@ def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
 SAMPLES = {
     # workload: (slice description, slicer of the CPU inputs, fraction of one step's tokens)
     "rglru": "the whole workload",
+    "rglru_gated": "the whole workload",
     "ssd": "batch row 0, heads 0-3 of 32, full L=4096",
     "ssd_mamba2": "batch row 0, heads 0-3 of 32, full L=4096",
     "gla": "batch row 0, heads 0-1 of 16, full L=2048",
@@ -566,8 +572,7 @@ def oracle_sample(name):
     w = inputs.WORKLOADS[name]
     kind = w["kind"]
     if kind == "rglru":
-        inp = inputs.rglru(w["B"], w["L"], w["D"], seed=0)
-        return kind, inp, 1.0, w
+        return kind, inputs.workload(name, seed=0), 1.0, w
     if kind == "ssd":
         inp = inputs.workload(name, seed=0, B=1, H=4)
         return kind, inp, (1 / w["B"]) * (4 / w["H"]), w
@@ -585,7 +590,10 @@ def oracle_sample(name):
 
 def oracle_step(kind, inp, w):
     import oracle
-    if kind == "rglru":
+    if kind == "rglru" and w.get("gates"):
+        oracle.rglru_gated_fwd(inp["a"], inp["b"], inp["x"], inp["A"], S=w["segment"])
+        oracle.rglru_gated_bwd(inp["a"], inp["b"], inp["x"], inp["A"], inp["dy"])
+    elif kind == "rglru":
         oracle.rglru_fwd(inp["a"], inp["b"], S=w["segment"])
         oracle.rglru_bwd(inp["a"], inp["b"], inp["dy"])
     elif kind == "rotlru":
@@ -650,9 +658,12 @@ def built_workloads():
             w["N"], w["P"] = w.pop("K"), w.pop("V")
         seg = w.pop("segment")
         softplus = w.pop("softplus", False)
+        gates = w.pop("gates", False)
         d = lrscan.make_desc(kind, io, segment=seg, **w)
         if softplus:
             d.flags |= lrscan.DELTA_SOFTPLUS
+        if gates:
+            d.flags |= lrscan.RGLRU_GATES
         if lrscan.validate(d) == 0:
             ok.append(name)
     return ok

@@ -32,6 +32,7 @@
  *
  * Layouts.  Row-major, last index contiguous, token-major:
  *   rglru   a, b, y, dy, da, db            [B, L, D]              io dtype
+ *           (LR_RGLRU_GATES: r, i, x, dr, di, dx [B, L, D]; Lambda, dLambda [D] f32)
  *   rotlru  b, y, dy, db                   [B, L, D] (re, im interleaved)   io dtype
  *           g, dg                          [B, L, D/2]            io dtype
  *           mag, theta, dmag, dtheta       [D/2]                  f32
@@ -108,6 +109,21 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * the backward writes ddelta for the raw delta, dd * sigma(delta + bias), and, if ddelta_bias is
  * non-NULL, ddelta_bias = its sum over batch and time. */
 #define LR_DELTA_SOFTPLUS 8u
+/* rglru, f32 I/O: the RG-LRU gate front-end computed in the kernels.  The pages name the rglru
+ * kernel for "Griffin and RecurrentGemma-style architectures" (mlx-recurrence post, Apple
+ * Developer Forums thread 840535, "Current kernels") without stating its gates; this library
+ * reads them as Griffin's: a_t = sigmoid(Lambda)^(8 r_t), b_t = sqrt(1 - a_t^2) (i_t x_t), then
+ * h_t = a_t h_{t-1} + b_t, y_t = h_t.  With this flag the rglru members take other meanings:
+ *   in->a   recurrence gate r [B, L, D] (values in (0, 1), typically a sigmoid output)
+ *   in->b   input gate i      [B, L, D]
+ *   in->x   the layer input x [B, L, D]
+ *   in->A   Lambda [D] f32
+ *   gr->da, gr->db, gr->dx   dr, di, dx [B, L, D];  gr->dA  dLambda [D] f32 (NULL = not wanted)
+ * a is formed as e^{8 r log sigmoid(Lambda)} and 1 - a^2 as -expm1(2 log a), so b keeps its
+ * relative precision as a approaches 1.  dr is undefined where r = 0 exactly (b's derivative
+ * contains 1 / sqrt(1 - a^2)).  Not combined with LR_FULL_STATE (LR_ERR_UNSUPPORTED); other
+ * kinds: LR_ERR_INVALID_ARG.  lr_step accepts it (forward only). */
+#define LR_RGLRU_GATES 16u
 /* Test hook for the failure path: the tiles of the first segment never publish their carry, so
  * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
  * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
@@ -186,7 +202,7 @@ lr_status lr_scan_fwd(const lr_desc *desc, const lr_inputs *in, void *y, void *c
 
 /* Backward pass: recomputes the states inside each segment from ckpt and runs the adjoint
  * recurrence in reverse; writes every non-NULL gradient required by the kind
- * (rglru: da, db; rotlru: db, dg, dmag, dtheta; s6: dx, ddelta, dA, dBm, dCm, dDskip if
+ * (rglru: da, db, and with LR_RGLRU_GATES dx and (optional) dA; rotlru: db, dg, dmag, dtheta; s6: dx, ddelta, dA, dBm, dCm, dDskip if
  * LR_HAS_DSKIP, dz if LR_HAS_Z; ssd: the same with per-head dA, dDskip; gla: dq, dk, dv, dg).
  *   dy         upstream gradient of y (io dtype, y's layout)
  *   ckpt       the buffer the matching lr_scan_fwd call wrote
@@ -264,7 +280,8 @@ int lr_version(void);
  * on the GPU (unordered streams) race and must be avoided.  With `check` non-zero the call
  * synchronises `stream` and returns the kernel's device-side status (LR_ERR_TIMEOUT if a bounded
  * wait gave up); otherwise it returns once the work is enqueued.  Other statuses as
- * lr_scan_fwd (LR_ERR_INVALID_ARG also for a kind other than LR_RGLRU). */
+ * lr_scan_fwd (LR_ERR_INVALID_ARG also for a kind other than LR_RGLRU; LR_ERR_UNSUPPORTED with
+ * LR_RGLRU_GATES, whose inputs this signature does not carry). */
 lr_status lr_rglru_fwd_noalloc(const lr_desc *desc, const void *a, const void *b, void *y,
                                void *ckpt, void *stream, int check);
 

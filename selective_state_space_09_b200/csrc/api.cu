@@ -32,6 +32,10 @@ lr_status validate(const lr_desc* d) {
     if ((d->flags & LR_FULL_STATE) && d->kind != LR_RGLRU && d->kind != LR_ROTLRU && d->kind != LR_S6)
         return LR_ERR_UNSUPPORTED;
     if ((d->flags & LR_DELTA_SOFTPLUS) && d->kind != LR_S6 && d->kind != LR_SSD) return LR_ERR_INVALID_ARG;
+    if (d->flags & LR_RGLRU_GATES) {
+        if (d->kind != LR_RGLRU) return LR_ERR_INVALID_ARG;
+        if (d->io != LR_F32 || (d->flags & LR_FULL_STATE)) return LR_ERR_UNSUPPORTED;
+    }
     const int es = esize(d->io);
     switch (d->kind) {
         case LR_RGLRU:
@@ -204,7 +208,10 @@ lr_status lr_scan_fwd(const lr_desc* desc, const lr_inputs* in, void* y, void* c
     const void* need[8] = {nullptr};
     int nn = 0;
     switch (d.kind) {
-        case LR_RGLRU: need[nn++] = in->a; need[nn++] = in->b; break;
+        case LR_RGLRU:
+            need[nn++] = in->a; need[nn++] = in->b;
+            if (d.flags & LR_RGLRU_GATES) { need[nn++] = in->x; need[nn++] = in->A; }
+            break;
         case LR_ROTLRU: need[nn++] = in->b; need[nn++] = in->g; need[nn++] = in->mag; need[nn++] = in->theta; break;
         case LR_S6:
         case LR_SSD:
@@ -242,7 +249,12 @@ lr_status lr_scan_bwd(const lr_desc* desc, const lr_inputs* in, const void* dy, 
     int nn = 0;
     switch (d.kind) {
         case LR_RGLRU:
-            need[nn++] = in->a; need[nn++] = in->b; need[nn++] = gr->da; need[nn++] = gr->db; break;
+            need[nn++] = in->a; need[nn++] = in->b; need[nn++] = gr->da; need[nn++] = gr->db;
+            if (d.flags & LR_RGLRU_GATES) {  // dA (dLambda) may be NULL
+                need[nn++] = in->x; need[nn++] = in->A; need[nn++] = gr->dx;
+                if (gr->dA && !aligned16(gr->dA)) return LR_ERR_ALIGNMENT;
+            }
+            break;
         case LR_ROTLRU:
             need[nn++] = in->b; need[nn++] = in->g; need[nn++] = in->mag; need[nn++] = in->theta;
             need[nn++] = gr->db; need[nn++] = gr->dg; need[nn++] = gr->dmag; need[nn++] = gr->dtheta; break;
@@ -284,6 +296,7 @@ lr_status lr_step(const lr_desc* desc, const lr_inputs* in, const void* state_in
     if (d.B < 1 || d.L < 1) return LR_ERR_INVALID_ARG;
     if (d.B > (1 << 20) || d.L > (1ll << 30)) return LR_ERR_UNSUPPORTED;
     if ((d.flags & LR_DELTA_SOFTPLUS) && d.kind != LR_S6 && d.kind != LR_SSD) return LR_ERR_INVALID_ARG;
+    if ((d.flags & LR_RGLRU_GATES) && d.kind != LR_RGLRU) return LR_ERR_INVALID_ARG;
     const size_t es = (size_t)esize(d.io);
     struct Need {
         const void* p;
@@ -296,6 +309,10 @@ lr_status lr_step(const lr_desc* desc, const lr_inputs* in, const void* state_in
             need[nn++] = {in->a, es};
             need[nn++] = {in->b, es};
             need[nn++] = {y, es};
+            if (d.flags & LR_RGLRU_GATES) {
+                need[nn++] = {in->x, es};
+                need[nn++] = {in->A, 4};
+            }
             break;
         case LR_ROTLRU:
             if (d.disc != LR_DISC_NONE || d.D < 2 || d.D % 2) return LR_ERR_INVALID_ARG;

@@ -56,12 +56,13 @@ struct DiagArgs {
     unsigned int dflags;        // lr_desc flags (LR_TEST_WITHHOLD_CARRY)
     const float* mag;           // rotlru
     const float* theta;         // rotlru
+    const float* lam;           // rglru with gates: Lambda [D]
     float* ckpt;                // [nseg, B, D] f32
     WsHeader* hdr;
     unsigned int* flags;        // [B * ncb * nseg]
     void* agg;                  // Agg<V>[tiles][CB]
     void* pre;                  // V[tiles][CB]
-    float2* partial;            // rotlru bwd: [B * nseg][D/2] (dmag, dtheta)
+    float2* partial;            // bwd: rotlru [B * nseg][D/2] (dmag, dtheta); gated rglru [B * nseg][D] (dLambda, 0)
 };
 
 // Per-kind description.  Unit = the element one thread carries through time.
@@ -84,6 +85,26 @@ template <typename T> struct Kind<LR_RGLRU, T> {
     static __device__ __forceinline__ void st_ckpt(float* p, int chan0, V v) { p[chan0] = v; }
     static __device__ __forceinline__ V ld_ckpt(const float* p, int chan0) { return p[chan0]; }
     static constexpr int chans_per_unit = 1;
+};
+
+// rglru with the RG-LRU gate front-end (LR_RGLRU_GATES, f32): the coefficient tensor holds the
+// recurrence gate r, a = sigmoid(Lambda)^(c r) = e^{c r log sigmoid(Lambda)} is formed where it is
+// read; b = sqrt(1 - a^2) (i x) is formed once per tile from the input gate i and x.
+constexpr int kRgGated = 5;         // internal kind id
+constexpr float kRgC = 8.0f;        // the exponent constant c
+template <typename T> struct Kind<kRgGated, T> : Kind<LR_RGLRU, T> {
+    struct Unit {
+        float clog;      // c log sigmoid(Lambda) (<= 0)
+        float oms;       // 1 - sigmoid(Lambda)
+        __device__ Unit(const DiagArgs& a, int d) {
+            const float lam = d < a.D ? a.lam[d] : 1.0f;
+            clog = -kRgC * log1pf(expf(-lam));
+            oms = 1.0f / (1.0f + expf(lam));
+        }
+        __device__ __forceinline__ float coef(const T* C, int t, int u) const {
+            return expf(IO<T>::ld(C + t * Kind<LR_RGLRU, T>::CW + u) * clog);
+        }
+    };
 };
 
 template <typename T> struct Kind<LR_ROTLRU, T> {
@@ -126,12 +147,15 @@ template <typename T> struct Kind<LR_ROTLRU, T> {
 template <int KIND, typename T, bool BWD> struct Smem {
     using K = Kind<KIND, T>;
     using V = typename K::V;
+    static constexpr bool G = KIND == kRgGated;  // x tile (and, backward, a tile of b values)
     static __host__ __device__ constexpr size_t coef_bytes() { return size_t(kMaxSeg) * K::CW * sizeof(T); }
     static __host__ __device__ constexpr size_t b_bytes() { return size_t(kMaxSeg) * K::BW * sizeof(T); }
     static __host__ __device__ constexpr size_t off_coef() { return 128; }
     static __host__ __device__ constexpr size_t off_b() { return off_coef() + coef_bytes(); }
     static __host__ __device__ constexpr size_t off_dy() { return off_b() + b_bytes(); }
-    static __host__ __device__ constexpr size_t off_aggf() { return off_dy() + (BWD ? b_bytes() : 0); }
+    static __host__ __device__ constexpr size_t off_x() { return off_dy() + (BWD ? b_bytes() : 0); }
+    static __host__ __device__ constexpr size_t off_e() { return off_x() + (G ? b_bytes() : 0); }
+    static __host__ __device__ constexpr size_t off_aggf() { return off_e() + (G && BWD ? b_bytes() : 0); }
     static __host__ __device__ constexpr size_t off_aggr() { return off_aggf() + sizeof(Agg<V>) * K::NG * K::CB; }
     static __host__ __device__ constexpr size_t off_carry() {
         return off_aggr() + (BWD ? sizeof(Agg<V>) * K::NG * K::CB : 0);
@@ -226,7 +250,7 @@ __device__ __forceinline__ char* smem_base() {
 template <int KIND, typename T, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
-                const __grid_constant__ CUtensorMap mapY, DiagArgs a) {
+                const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapY, DiagArgs a) {
     using K = Kind<KIND, T>;
     using V = typename K::V;
     using SM = Smem<KIND, T, false>;
@@ -235,6 +259,8 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
     T* Cs = reinterpret_cast<T*>(sm + SM::off_coef());
     T* Bs = reinterpret_cast<T*>(sm + SM::off_b());
+    T* Xs = reinterpret_cast<T*>(sm + SM::off_x());  // gated: x
+    constexpr bool gated = KIND == kRgGated;
     Agg<V>* aggF = reinterpret_cast<Agg<V>*>(sm + SM::off_aggf());
     V* carryS = reinterpret_cast<V*>(sm + SM::off_carry());
     int* misc = reinterpret_cast<int*>(sm + SM::off_misc());
@@ -258,9 +284,10 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + K::BW) * sizeof(T)));
+        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + (gated ? 2 : 1) * K::BW) * sizeof(T)));
         tma_load_3d(Cs, &mapC, bar, cb * K::CW, t0g, b);
         tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
+        if (gated) tma_load_3d(Xs, &mapX, bar, cb * K::BW, t0g, b);
     }
     const int unit = cb * CB + u;  // global unit index (channel or pair)
     const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
@@ -276,6 +303,14 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int spg = (a.S + NG - 1) / NG;
     const int j0 = grp * spg, j1 = min(j0 + spg, nt);
     bool ok = mbar_wait(bar, 0, a.hdr, 100);
+    if constexpr (gated) {  // b = sqrt(1 - a^2) (i x) over the thread's own steps, into i's slot
+        if (ok)
+            for (int j = j0; j < j1; ++j) {
+                const float L = IO<T>::ld(Cs + j * K::CW + u) * U.clog;  // log a
+                const float bj = sqrtf(-expm1f(2.0f * L)) * IO<T>::ld(Bs + j * K::BW + u) * IO<T>::ld(Xs + j * K::BW + u);
+                IO<T>::st(Bs + j * K::BW + u, bj);
+            }
+    }
 
     // group aggregate with zero carry-in
     V P = one_of(V{}), h = zero_of(V{});
@@ -358,8 +393,9 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 template <int KIND, typename T, bool FULL>
 __global__ void __launch_bounds__(kThreads, 2)  // two tiles per SM (shared memory)
 diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
-                const __grid_constant__ CUtensorMap mapDY, const __grid_constant__ CUtensorMap mapDC,
-                const __grid_constant__ CUtensorMap mapDB, DiagArgs a) {
+                const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapDY,
+                const __grid_constant__ CUtensorMap mapDC, const __grid_constant__ CUtensorMap mapDB,
+                const __grid_constant__ CUtensorMap mapDX, DiagArgs a) {
     using K = Kind<KIND, T>;
     using V = typename K::V;
     using SM = Smem<KIND, T, true>;
@@ -370,6 +406,11 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     T* Cs = reinterpret_cast<T*>(sm + SM::off_coef());
     T* Bs = reinterpret_cast<T*>(sm + SM::off_b());
     T* Ds = reinterpret_cast<T*>(sm + SM::off_dy());
+    // gated: x, and b = sqrt(1 - a^2) (i x) (the recompute's input; i stays for its gradient)
+    constexpr bool gated = KIND == kRgGated;
+    T* Xs = reinterpret_cast<T*>(sm + SM::off_x());
+    T* Es = reinterpret_cast<T*>(sm + SM::off_e());
+    T* Brec = gated ? Es : Bs;
     Agg<V>* aggF = reinterpret_cast<Agg<V>*>(sm + SM::off_aggf());
     Agg<V>* aggR = reinterpret_cast<Agg<V>*>(sm + SM::off_aggr());
     V* carryS = reinterpret_cast<V*>(sm + SM::off_carry());
@@ -399,9 +440,11 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int t0g = seg * a.S;
     // coefficients and b (the forward recompute) on bar[0], dy (the adjoint) on bar[1]
     if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(a.S * (K::CW + (full ? 0 : K::BW)) * sizeof(T)));
+        mbar_arrive_expect_tx(&bar[0],
+                              (uint32_t)(a.S * (K::CW + (full ? 0 : K::BW) + (gated ? K::BW : 0)) * sizeof(T)));
         tma_load_3d(Cs, &mapC, &bar[0], cb * K::CW, t0g, b);
         if (!full) tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
+        if (gated) tma_load_3d(Xs, &mapX, &bar[0], cb * K::BW, t0g, b);
         mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
         tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
     }
@@ -426,6 +469,14 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const int j0 = grp * spg, j1 = min(j0 + spg, nt);
     const int n = max(j1 - j0, 0);
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 200);
+    if constexpr (gated) {  // b of the thread's own steps, from r, i, x
+        if (ok)
+            for (int j = j0; j < j1; ++j) {
+                const float L = IO<T>::ld(Cs + j * K::CW + u) * U.clog;  // log a
+                IO<T>::st(Es + j * K::BW + u,
+                          sqrtf(-expm1f(2.0f * L)) * IO<T>::ld(Bs + j * K::BW + u) * IO<T>::ld(Xs + j * K::BW + u));
+            }
+    }
 
     // state entering each step of the group, in registers: recomputed from the segment
     // checkpoint, or (full state) read from that step's checkpoint slot
@@ -438,7 +489,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
                 for (int j = j0; j < j1; ++j) {
                     V c = U.coef(Cs, j, u);
                     P = mulx(c, P);
-                    h = fmax_(c, h, K::ldb(Bs, j, u));
+                    h = fmax_(c, h, K::ldb(Brec, j, u));
                 }
             aggF[grp * CB + u] = {P, h};
         }
@@ -453,7 +504,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             hprev[j] = h;
             if (j < n) {
                 V c = U.coef(Cs, j0 + j, u);
-                h = fmax_(c, h, K::ldb(Bs, j0 + j, u));
+                h = fmax_(c, h, K::ldb(Brec, j0 + j, u));
             }
         }
     } else {
@@ -530,6 +581,19 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
                 IO<T>::st(Ds + j * K::BW + u, G);       // db
                 IO<T>::st(Cs + j * K::CW + u, G * hp);  // da
                 r = c * G;
+            } else if constexpr (gated) {
+                // db = G, da = G h_{t-1}, carried through b = s (i x), s = sqrt(1 - a^2), and
+                // a = e^{c r log sigmoid(Lambda)}: ds/da = -a / s
+                const float rg = IO<T>::ld(Cs + j * K::CW + u);
+                const float L = rg * U.clog;
+                const float av = expf(L), sv = sqrtf(-expm1f(2.0f * L));
+                const float iv = IO<T>::ld(Bs + j * K::BW + u), xv = IO<T>::ld(Xs + j * K::BW + u);
+                const float da_tot = G * hp - G * iv * xv * av / sv;
+                IO<T>::st(Bs + j * K::BW + u, G * sv * xv);           // di
+                IO<T>::st(Xs + j * K::BW + u, G * sv * iv);           // dx
+                IO<T>::st(Cs + j * K::CW + u, da_tot * av * U.clog);  // dr
+                acc_mag = fmaf(da_tot * av * kRgC * rg, U.oms, acc_mag);  // dLambda
+                r = av * G;
             } else {
                 float gt = IO<T>::ld(Cs + j * K::CW + u);
                 float m = U.mag * gt;
@@ -544,12 +608,12 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             }
         }
     }
-    if constexpr (KIND == LR_ROTLRU) {
+    if constexpr (KIND == LR_ROTLRU || gated) {
         red[grp * CB + u] = make_float2(acc_mag, acc_th);
     }
     fence_proxy_async_smem();
     __syncthreads();
-    if constexpr (KIND == LR_ROTLRU) {
+    if constexpr (KIND == LR_ROTLRU || gated) {  // rotlru: dmag, dtheta; gated rglru: dLambda
         if (tid < CB && unit < units) {
             float sm_ = 0.0f, st_ = 0.0f;
             for (int g = 0; g < NG; ++g) {
@@ -557,12 +621,17 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
                 sm_ += v.x;
                 st_ += v.y;
             }
-            a.partial[((size_t)b * a.nseg + seg) * (a.D / 2) + unit] = make_float2(sm_, st_);
+            a.partial[((size_t)b * a.nseg + seg) * units + unit] = make_float2(sm_, st_);
         }
     }
     if (tid == 0 && ok) {
         tma_store_3d(&mapDC, Cs, cb * K::CW, t0g, b);
-        tma_store_3d(&mapDB, Ds, cb * K::BW, t0g, b);
+        if constexpr (gated) {
+            tma_store_3d(&mapDB, Bs, cb * K::BW, t0g, b);  // di
+            tma_store_3d(&mapDX, Xs, cb * K::BW, t0g, b);  // dx
+        } else {
+            tma_store_3d(&mapDB, Ds, cb * K::BW, t0g, b);
+        }
         bulk_commit();
         bulk_wait_read_all();
     }
@@ -600,7 +669,7 @@ rotlru_param_reduce(const float2* __restrict__ partial, int rows, int K, float* 
     }
     if (y == 0 && k < K) {
         dmag[k] = red[0][x].x;
-        dtheta[k] = red[0][x].y;
+        if (dtheta) dtheta[k] = red[0][x].y;
     }
 }
 
@@ -635,7 +704,10 @@ DiagWs ws_plan(const lr_desc& d, bool bwd) {
     w.flags = c.take(sizeof(unsigned int) * g.tiles);
     w.agg = c.take(2 * vs * g.cb * (size_t)g.tiles);
     w.pre = c.take(vs * g.cb * (size_t)g.tiles);
-    w.partial = (bwd && d.kind == LR_ROTLRU) ? c.take(sizeof(float2) * d.B * g.nseg * (d.D / 2)) : 0;
+    const bool gates = d.kind == LR_RGLRU && (d.flags & LR_RGLRU_GATES);
+    w.partial = (bwd && (d.kind == LR_ROTLRU || gates))
+                    ? c.take(sizeof(float2) * d.B * g.nseg * (d.kind == LR_ROTLRU ? d.D / 2 : d.D))
+                    : 0;
     w.end = c.off;
     return w;
 }
@@ -657,15 +729,20 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
     Geo g = geo(d);
     DiagWs w = ws_plan(d, false);
     const int es = sizeof(T);
-    CUtensorMap mC, mB, mY;
-    const void* coef = KIND == LR_RGLRU ? in.a : in.g;
-    uint64_t coefC = KIND == LR_RGLRU ? d.D : d.D / 2;
+    constexpr bool rg = KIND != LR_ROTLRU;
+    CUtensorMap mC, mB, mX, mY;
+    const void* coef = rg ? in.a : in.g;
+    uint64_t coefC = rg ? d.D : d.D / 2;
     bool ok = make_tmap_3d(&mC, coef, es, coefC, d.L, d.B, K::CW, d.segment) &&
               make_tmap_3d(&mB, in.b, es, d.D, d.L, d.B, K::BW, d.segment) &&
               make_tmap_3d(&mY, y, es, d.D, d.L, d.B, K::BW, d.segment);
+    if (KIND == kRgGated)
+        ok = ok && make_tmap_3d(&mX, in.x, es, d.D, d.L, d.B, K::BW, d.segment);
+    else
+        mX = mB;  // not read
     if (!ok) return LR_ERR_INVALID_ARG;
     DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
-               (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
+               in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
     auto fn = full ? diag_fwd_kernel<KIND, T, true> : diag_fwd_kernel<KIND, T, false>;
@@ -673,8 +750,8 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
         set_smem_attr<KIND, T, false, true>((const void*)fn);
     else
         set_smem_attr<KIND, T, false, false>((const void*)fn);
-    note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : "rotlru_fwd_tile");
-    fn<<<g.tiles, kThreads, Smem<KIND, T, false>::total(), st>>>(mC, mB, mY, a);
+    note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : KIND == kRgGated ? "rglru_gated_fwd_tile" : "rotlru_fwd_tile");
+    fn<<<g.tiles, kThreads, Smem<KIND, T, false>::total(), st>>>(mC, mB, mX, mY, a);
     return check_launch();
 }
 
@@ -685,18 +762,26 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
     Geo g = geo(d);
     DiagWs w = ws_plan(d, true);
     const int es = sizeof(T);
-    CUtensorMap mC, mB, mDY, mDC, mDB;
-    const void* coef = KIND == LR_RGLRU ? in.a : in.g;
-    void* dcoef = KIND == LR_RGLRU ? gr.da : gr.dg;
-    uint64_t coefC = KIND == LR_RGLRU ? d.D : d.D / 2;
+    constexpr bool rg = KIND != LR_ROTLRU;
+    CUtensorMap mC, mB, mX, mDY, mDC, mDB, mDX;
+    const void* coef = rg ? in.a : in.g;
+    void* dcoef = rg ? gr.da : gr.dg;
+    uint64_t coefC = rg ? d.D : d.D / 2;
     bool ok = make_tmap_3d(&mC, coef, es, coefC, d.L, d.B, K::CW, d.segment) &&
               make_tmap_3d(&mB, in.b, es, d.D, d.L, d.B, K::BW, d.segment) &&
               make_tmap_3d(&mDY, dy, es, d.D, d.L, d.B, K::BW, d.segment) &&
               make_tmap_3d(&mDC, dcoef, es, coefC, d.L, d.B, K::CW, d.segment) &&
               make_tmap_3d(&mDB, gr.db, es, d.D, d.L, d.B, K::BW, d.segment);
+    if (KIND == kRgGated) {
+        ok = ok && make_tmap_3d(&mX, in.x, es, d.D, d.L, d.B, K::BW, d.segment) &&
+             make_tmap_3d(&mDX, gr.dx, es, d.D, d.L, d.B, K::BW, d.segment);
+    } else {
+        mX = mB;  // not read
+        mDX = mDB;  // not written
+    }
     if (!ok) return LR_ERR_INVALID_ARG;
     DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
-               (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
+               in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                w.partial ? (float2*)(ws + w.partial) : nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
     auto fn = full ? diag_bwd_kernel<KIND, T, true> : diag_bwd_kernel<KIND, T, false>;
@@ -704,8 +789,8 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
         set_smem_attr<KIND, T, true, true>((const void*)fn);
     else
         set_smem_attr<KIND, T, true, false>((const void*)fn);
-    note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : "rotlru_bwd_tile");
-    fn<<<g.tiles, kThreads, Smem<KIND, T, true>::total(), st>>>(mC, mB, mDY, mDC, mDB, a);
+    note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : KIND == kRgGated ? "rglru_gated_bwd_tile" : "rotlru_bwd_tile");
+    fn<<<g.tiles, kThreads, Smem<KIND, T, true>::total(), st>>>(mC, mB, mX, mDY, mDC, mDB, mDX, a);
     lr_status s = check_launch();
     if (s != LR_OK) return s;
     if (KIND == LR_ROTLRU) {
@@ -713,6 +798,12 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
         note_launch("rotlru_param_reduce");
         rotlru_param_reduce<<<(K2 + kRedPairs - 1) / kRedPairs, kRedPairs * kRedSlices, 0, st>>>(
             a.partial, (int)d.B * g.nseg, K2, gr.dmag, gr.dtheta);
+        s = check_launch();
+    } else if (KIND == kRgGated && gr.dA) {  // dLambda: the same fixed-order reduction, one value
+        int K1 = (int)d.D;
+        note_launch("rglru_param_reduce");
+        rotlru_param_reduce<<<(K1 + kRedPairs - 1) / kRedPairs, kRedPairs * kRedSlices, 0, st>>>(
+            a.partial, (int)d.B * g.nseg, K1, gr.dA, nullptr);
         s = check_launch();
     }
     return s;
@@ -725,6 +816,7 @@ size_t diag_flag_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).agg;
 
 lr_status diag_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
                    cudaStream_t st) {
+    if (d.kind == LR_RGLRU && (d.flags & LR_RGLRU_GATES)) return launch_fwd<kRgGated, float>(d, in, y, ckpt, ws, st);
     if (d.kind == LR_RGLRU)
         return d.io == LR_F32 ? launch_fwd<LR_RGLRU, float>(d, in, y, ckpt, ws, st)
                               : launch_fwd<LR_RGLRU, __nv_bfloat16>(d, in, y, ckpt, ws, st);
@@ -734,6 +826,8 @@ lr_status diag_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, c
 
 lr_status diag_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt,
                    const lr_grads& gr, char* ws, cudaStream_t st) {
+    if (d.kind == LR_RGLRU && (d.flags & LR_RGLRU_GATES))
+        return launch_bwd<kRgGated, float>(d, in, dy, ckpt, gr, ws, st);
     if (d.kind == LR_RGLRU)
         return d.io == LR_F32 ? launch_bwd<LR_RGLRU, float>(d, in, dy, ckpt, gr, ws, st)
                               : launch_bwd<LR_RGLRU, __nv_bfloat16>(d, in, dy, ckpt, gr, ws, st);

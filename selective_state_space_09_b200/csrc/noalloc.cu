@@ -55,6 +55,7 @@ extern "C" lr_status lr_rglru_fwd_noalloc(const lr_desc* desc, const void* a, co
                                           void* y, void* ckpt, void* stream, int check) {
     reset_dispatch();
     if (!desc || desc->kind != LR_RGLRU) return LR_ERR_INVALID_ARG;
+    if (desc->flags & LR_RGLRU_GATES) return LR_ERR_UNSUPPORTED;  // no gate inputs in this signature
     lr_status s = lr_validate(desc);
     if (s != LR_OK) return s;
     if (!a || !b || !y || !ckpt) return LR_ERR_INVALID_ARG;

@@ -29,17 +29,27 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x, the MUFU approximation
 }
 
 // ------------------------------------------------------------------------ diagonal kinds
-template <typename T>
+// GATES: the RG-LRU gate front-end -- a holds the recurrence gate r, b the input gate i, and the
+// step is h = a h + sqrt(1 - a^2) (i x) with a = sigmoid(Lambda)^(8 r), formed in the log domain
+template <typename T, bool GATES>
 __global__ void __launch_bounds__(256)
-rglru_step_kernel(const T* __restrict__ a, const T* __restrict__ b, T* __restrict__ y, const float* s_in,
-                  float* s_out, int B, int L, int D) {
+rglru_step_kernel(const T* __restrict__ a, const T* __restrict__ b, const T* __restrict__ x,
+                  const float* __restrict__ lam, T* __restrict__ y, const float* s_in, float* s_out, int B, int L,
+                  int D) {
     const size_t u = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (u >= (size_t)B * D) return;
     const int bi = (int)(u / D), d = (int)(u % D);
+    float clog = 0.0f;  // 8 log sigmoid(Lambda)
+    if (GATES) clog = -8.0f * log1pf(expf(-lam[d]));
     float h = s_in ? s_in[u] : 0.0f;
     for (int t = 0; t < L; ++t) {
         const size_t i = ((size_t)bi * L + t) * D + d;
-        h = fmaf(IO<T>::ld(a + i), h, IO<T>::ld(b + i));
+        if (GATES) {
+            const float Lg = IO<T>::ld(a + i) * clog;
+            h = fmaf(expf(Lg), h, sqrtf(-expm1f(2.0f * Lg)) * IO<T>::ld(b + i) * IO<T>::ld(x + i));
+        } else {
+            h = fmaf(IO<T>::ld(a + i), h, IO<T>::ld(b + i));
+        }
         IO<T>::st(y + i, h);
     }
     s_out[u] = h;
@@ -232,9 +242,16 @@ lr_status step_impl(const lr_desc& d, const lr_inputs& in, const float* s_in, fl
     switch (d.kind) {
         case LR_RGLRU: {
             const size_t n = (size_t)d.B * d.D;
-            note_launch("rglru_step");
-            rglru_step_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-                (const T*)in.a, (const T*)in.b, (T*)y, s_in, s_out, B, L, (int)d.D);
+            const unsigned grid = (unsigned)((n + 255) / 256);
+            if (d.flags & LR_RGLRU_GATES) {
+                note_launch("rglru_gated_step");
+                rglru_step_kernel<T, true><<<grid, 256, 0, st>>>((const T*)in.a, (const T*)in.b, (const T*)in.x,
+                                                                 in.A, (T*)y, s_in, s_out, B, L, (int)d.D);
+            } else {
+                note_launch("rglru_step");
+                rglru_step_kernel<T, false><<<grid, 256, 0, st>>>((const T*)in.a, (const T*)in.b, nullptr,
+                                                                  nullptr, (T*)y, s_in, s_out, B, L, (int)d.D);
+            }
             return check_launch();
         }
         case LR_ROTLRU: {

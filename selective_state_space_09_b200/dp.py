@@ -8,10 +8,10 @@ import torch
 import torch.distributed as dist
 
 # parameter gradients (names as in the C ABI's lr_grads) that sum over the batch
-PARAM_GRADS = {"rglru": (), "rotlru": ("dmag", "dtheta"), "s6": ("dA", "dDskip"),
-               "ssd": ("dA", "dDskip"), "gla": ()}
+PARAM_GRADS = {"rglru": ("dA",), "rotlru": ("dmag", "dtheta"), "s6": ("dA", "dDskip", "ddelta_bias"),
+               "ssd": ("dA", "dDskip", "ddelta_bias"), "gla": ()}
 # per-token inputs (batch-major) of each kind; everything else is a parameter
-TOKEN_INPUTS = {"rglru": ("a", "b", "dy"), "rotlru": ("b", "g", "dy"),
+TOKEN_INPUTS = {"rglru": ("a", "b", "x", "dy"), "rotlru": ("b", "g", "dy"),
                 "s6": ("x", "delta", "Bm", "Cm", "z", "dy"), "ssd": ("x", "delta", "Bm", "Cm", "z", "dy"),
                 "gla": ("q", "k", "v", "g", "dy")}
 

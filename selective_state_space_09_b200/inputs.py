@@ -14,6 +14,9 @@ Workloads (token-major layouts, last index contiguous):
 * ``rglru``  fp32, B=1, D=256, L=1024, segment 128.
   ``a = sigmoid(Lam)^(8 r)``, ``Lam ~ U(2, 6)`` per channel, ``r = sigmoid(N(0,1))`` per step and
   channel; ``b = sqrt(1 - a^2) N(0,1)``.
+* ``rglru_gated`` the same shapes with the RG-LRU gate front-end formed in the kernels: inputs
+  ``r = sigmoid(N(0,1))``, ``i = sigmoid(N(0,1))``, ``x ~ N(0,1)`` per step and channel and
+  ``Lam ~ U(2, 6)`` per channel (key names ``a, b, x, A``: the C ABI members that carry them).
 * ``ssd``    bf16 I/O, B=2, H=32, P=64, N=128, L=4096, G=1, ZOH; evaluated in chunks of 128 steps,
   which are also the checkpoint segments.
   ``dt = softplus(N(-2,1))`` per (b,t,h); ``A_h = -exp(U(log 1, log 16))``;
@@ -41,6 +44,8 @@ WORKLOADS = {
     "s6_bilinear": dict(kind="s6", io="bf16", B=8, D=2048, N=16, L=2048, segment=64,
                         disc="bilinear"),
     "rotlru": dict(kind="rotlru", io="f32", B=16, D=4096, L=16384, segment=256),
+    # the rglru workload's shapes with the gates formed in the kernels (r, i, x, Lambda)
+    "rglru_gated": dict(kind="rglru", io="f32", B=1, D=256, L=1024, segment=128, gates=True),
     # the SSD workload's shapes through the general kernel variant, as Mamba-2 layers run it:
     # dt = softplus(delta + bias) in the kernels, abar = e^{dt A}, beta = dt (ZOH-Euler)
     "ssd_mamba2": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=128,
@@ -72,6 +77,17 @@ def rglru(B, L, D, seed=0, io="f32", device="cpu"):
     dy = r.randn(B, L, D)
     t = _DT[io]
     return {"a": a.to(t), "b": b.to(t), "dy": dy.to(t)}
+
+
+def rglru_gated(B, L, D, seed=0, device="cpu"):
+    """Gate-level rglru inputs (f32): a = r (recurrence gate), b = i (input gate), x, A = Lambda."""
+    r = _Draw(seed, device)
+    lam = 2.0 + 4.0 * r.rand(D)
+    rr = torch.sigmoid(r.randn(B, L, D))
+    ii = torch.sigmoid(r.randn(B, L, D))
+    x = r.randn(B, L, D)
+    dy = r.randn(B, L, D)
+    return {"a": rr, "b": ii, "x": x, "A": lam, "dy": dy}
 
 
 def rotlru(B, L, D, seed=0, io="f32", device="cpu"):
@@ -139,6 +155,8 @@ def workload(name, seed=0, device="cpu", **override):
     w = dict(WORKLOADS[name])
     w.update(override)
     k = w["kind"]
+    if k == "rglru" and w.get("gates"):
+        return rglru_gated(w["B"], w["L"], w["D"], seed, device)
     if k == "rglru":
         return rglru(w["B"], w["L"], w["D"], seed, w["io"], device)
     if k == "rotlru":

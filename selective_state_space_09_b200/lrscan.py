@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 KIND = {"rglru": 0, "rotlru": 1, "s6": 2, "ssd": 3, "gla": 4}
 DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 IO = {torch.float32: 0, torch.bfloat16: 1}
-HAS_Z, HAS_DSKIP, FULL_STATE, DELTA_SOFTPLUS = 1, 2, 4, 8
+HAS_Z, HAS_DSKIP, FULL_STATE, DELTA_SOFTPLUS, RGLRU_GATES = 1, 2, 4, 8, 16
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
 TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
 STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
@@ -192,9 +192,11 @@ class Plan:
 
 
 # ------------------------------------------------------------------ per-kind convenience plans
-def desc_for(kind, inp, segment=1, disc="none", chunk=0, delta_softplus=False):
+def desc_for(kind, inp, segment=1, disc="none", chunk=0, delta_softplus=False, gates=False):
     """Descriptor of a kind from its input tensors (shapes read from the tensors).
-    delta_softplus (S6, SSD): dt = softplus(delta + inp["delta_bias"]) in the kernels."""
+    delta_softplus (S6, SSD): dt = softplus(delta + inp["delta_bias"]) in the kernels.
+    gates (rglru): the RG-LRU gate front-end; inp["a"], inp["b"], inp["x"], inp["A"] hold the
+    recurrence gate r, the input gate i, x and Lambda."""
     if kind == "rglru":
         B, L, D = inp["a"].shape
         d = make_desc("rglru", inp["a"].dtype, B, L, D=D, segment=segment)
@@ -220,18 +222,20 @@ def desc_for(kind, inp, segment=1, disc="none", chunk=0, delta_softplus=False):
         raise KeyError(kind)
     if delta_softplus:
         d.flags |= DELTA_SOFTPLUS
+    if gates:
+        d.flags |= RGLRU_GATES
     return d
 
 
-def plan_for(kind, inp, segment, disc="none", chunk=0, delta_softplus=False):
+def plan_for(kind, inp, segment, disc="none", chunk=0, delta_softplus=False, gates=False):
     """Build the Plan of a kind from its input tensors (shapes read from the tensors)."""
-    d = desc_for(kind, inp, segment, disc, chunk, delta_softplus)
+    d = desc_for(kind, inp, segment, disc, chunk, delta_softplus, gates)
     return Plan(d, inp[next(k for k in inp if inp[k] is not None)].device)
 
 
 # ------------------------------------------------------------------------ decode / continuation
 # per-token inputs of each kind (the rest are parameters)
-TOKEN_INPUTS = {"rglru": ("a", "b"), "rotlru": ("b", "g"), "s6": ("x", "delta", "Bm", "Cm", "z"),
+TOKEN_INPUTS = {"rglru": ("a", "b", "x"), "rotlru": ("b", "g"), "s6": ("x", "delta", "Bm", "Cm", "z"),
                 "ssd": ("x", "delta", "Bm", "Cm", "z"), "gla": ("q", "k", "v", "g")}
 
 
@@ -258,12 +262,12 @@ class DecodeGraph:
     inputs are ``seq[name][t]``), parameters as usual; ``state``: the f32 state, advanced in place;
     ``y``: [T, B, 1, ...] outputs.  Every replay continues from whatever ``state`` holds."""
 
-    def __init__(self, kind, seq, state, y, disc="none", delta_softplus=False):
+    def __init__(self, kind, seq, state, y, disc="none", delta_softplus=False, gates=False):
         toks = TOKEN_INPUTS[kind]
         T = y.shape[0]
         self.kind, self.T, self.state, self.y = kind, T, state, y
         first = {n: (seq[n][0] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}
-        self.desc = desc_for(kind, first, 1, disc, delta_softplus=delta_softplus)
+        self.desc = desc_for(kind, first, 1, disc, delta_softplus=delta_softplus, gates=gates)
         self.calls = [({n: (seq[n][t] if n in toks and seq.get(n) is not None else seq.get(n)) for n in seq}, y[t])
                       for t in range(T)]
         side = torch.cuda.Stream()
@@ -285,7 +289,11 @@ def alloc_outputs(kind, inp):
     e = torch.empty_like
     f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
     if kind == "rglru":
-        return e(inp["b"]), {"da": e(inp["a"]), "db": e(inp["b"])}
+        g = {"da": e(inp["a"]), "db": e(inp["b"])}
+        if inp.get("x") is not None:  # gate front-end: dx, dLambda
+            g["dx"] = e(inp["x"])
+            g["dA"] = e(inp["A"])
+        return e(inp["b"]), g
     if kind == "rotlru":
         return e(inp["b"]), {"db": e(inp["b"]), "dg": e(inp["g"]), "dmag": e(inp["mag"]),
                              "dtheta": e(inp["theta"])}
@@ -307,9 +315,9 @@ def alloc_outputs(kind, inp):
 # ---------------------------------------------------------------------- autograd wrappers
 class _ScanFn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, kind, names, segment, disc, chunk, softplus, *tensors):
+    def forward(ctx, kind, names, segment, disc, chunk, opts, *tensors):
         inp = {n: t.contiguous() if t is not None else None for n, t in zip(names, tensors)}
-        plan = plan_for(kind, inp, segment, disc, chunk, softplus)
+        plan = plan_for(kind, inp, segment, disc, chunk, **opts)
         y, _ = alloc_outputs(kind, inp)
         plan.fwd(inp, y)
         ctx.kind, ctx.names, ctx.plan = kind, names, plan
@@ -330,19 +338,26 @@ class _ScanFn(torch.autograd.Function):
 
 def rglru(a, b, segment=128):
     """y = rglru_scan(a, b): h_t = a_t h_{t-1} + b_t, y_t = h_t.  a, b: [B, L, D]."""
-    return _ScanFn.apply("rglru", ("a", "b"), segment, "none", 0, False, a, b)
+    return _ScanFn.apply("rglru", ("a", "b"), segment, "none", 0, {}, a, b)
+
+
+def rglru_gated(r, i, x, lam, segment=128):
+    """RG-LRU with its gates formed in the kernels: a = sigmoid(lam)^(8 r), b = sqrt(1 - a^2) (i x),
+    h_t = a_t h_{t-1} + b_t, y_t = h_t.  r, i, x: [B, L, D] f32; lam: [D] f32.  Gradients flow to
+    r, i, x and lam."""
+    return _ScanFn.apply("rglru", ("a", "b", "x", "A"), segment, "none", 0, {"gates": True}, r, i, x, lam)
 
 
 def rotlru(b, g, mag, theta, segment=256):
     """y = rotlru_scan: lambda_t = mag g_t e^{i theta}, h_t = lambda_t h_{t-1} + b_t (pairs)."""
-    return _ScanFn.apply("rotlru", ("b", "g", "mag", "theta"), segment, "none", 0, False, b, g, mag, theta)
+    return _ScanFn.apply("rotlru", ("b", "g", "mag", "theta"), segment, "none", 0, {}, b, g, mag, theta)
 
 
 def s6(x, delta, A, B, C, D=None, z=None, disc="zoh", segment=256, delta_softplus=False, delta_bias=None):
     """Selective scan S6 with fused D skip and silu(z) gate.  x, delta, z: [B, L, D].  With
     delta_softplus the step length is softplus(delta + delta_bias) (delta_bias [D] or None)."""
     return _ScanFn.apply("s6", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"), segment, disc, 0,
-                         delta_softplus, x, delta, A, B, C, D, z, delta_bias)
+                         {"delta_softplus": delta_softplus}, x, delta, A, B, C, D, z, delta_bias)
 
 
 def ssd(x, delta, A, B, C, D=None, z=None, disc="zoh", chunk=64, segment=256, delta_softplus=False,
@@ -350,9 +365,9 @@ def ssd(x, delta, A, B, C, D=None, z=None, disc="zoh", chunk=64, segment=256, de
     """Head-wise SSD scan.  x, z: [B, L, H, P]; delta: [B, L, H]; B, C: [B, L, G, N].  With
     delta_softplus the step length is softplus(delta + delta_bias) (delta_bias [H] or None)."""
     return _ScanFn.apply("ssd", ("x", "delta", "A", "Bm", "Cm", "Dskip", "z", "delta_bias"), segment, disc,
-                         chunk, delta_softplus, x, delta, A, B, C, D, z, delta_bias)
+                         chunk, {"delta_softplus": delta_softplus}, x, delta, A, B, C, D, z, delta_bias)
 
 
 def gla(q, k, v, g, chunk=64, segment=256):
     """GLA scan: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t."""
-    return _ScanFn.apply("gla", ("q", "k", "v", "g"), segment, "none", chunk, False, q, k, v, g)
+    return _ScanFn.apply("gla", ("q", "k", "v", "g"), segment, "none", chunk, {}, q, k, v, g)

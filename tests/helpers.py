@@ -28,13 +28,13 @@ def gpu_inputs(inp, device="cuda"):
     return {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inp.items()}
 
 
-def run_gpu(kind, inp, segment, disc="none", chunk=0, flags=0):
+def run_gpu(kind, inp, segment, disc="none", chunk=0, flags=0, gates=False):
     """Forward + backward through the C ABI on the current CUDA device.  Returns
     (y, ckpt view, grads dict, plan)."""
     from selective_state_space_09_b200 import lrscan
     g = gpu_inputs(inp)
     dy = g.pop("dy")
-    desc = lrscan.desc_for(kind, g, segment, disc, chunk)
+    desc = lrscan.desc_for(kind, g, segment, disc, chunk, gates=gates)
     desc.flags |= flags  # before the Plan sizes its buffers (LR_FULL_STATE changes the checkpoint)
     plan = lrscan.Plan(desc, "cuda")
     y, grads = lrscan.alloc_outputs(kind, g)

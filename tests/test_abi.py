@@ -145,6 +145,39 @@ def test_step_calls_rejected_before_any_launch(L):
     assert L.last_launch_count() == 0
 
 
+def test_rglru_gates_rules(L):
+    """LR_RGLRU_GATES: rglru f32 only, not with the full-state mode; a scan call without x or
+    Lambda, and an lr_rglru_fwd_noalloc call with the flag, are rejected before any launch; the
+    backward workspace holds the per-tile dLambda partials."""
+    import torch
+    V = ctypes.c_void_p
+
+    def gated(kind="rglru", io=torch.float32, **kw):
+        d = L.make_desc(kind, io, **kw)
+        d.flags |= L.RGLRU_GATES
+        return d
+    assert L.validate(gated(B=1, L=1024, D=256, segment=128)) == 0
+    assert L.validate(gated(io=torch.bfloat16, B=1, L=64, D=64, segment=16)) == 2
+    d = gated(B=1, L=64, D=64, segment=16)
+    d.flags |= L.FULL_STATE
+    assert L.validate(d) == 2
+    assert L.validate(gated("rotlru", B=1, L=64, D=64, segment=16)) == 1
+    assert L.validate(gated("s6", io=torch.bfloat16, B=1, L=64, D=64, N=16, segment=16, disc="zoh")) == 1
+    d = gated(B=1, L=64, D=64, segment=16)
+    plain = L.make_desc("rglru", torch.float32, B=1, L=64, D=64, segment=16)
+    assert L.workspace_bytes(d, False) == L.workspace_bytes(plain, False)
+    assert L.workspace_bytes(d, True) >= L.workspace_bytes(plain, True) + 8 * 4 * 64
+    no_x = L.Inputs(a=V(0x1000), b=V(0x2000), A=V(0x3000))
+    assert L.lib.lr_scan_fwd(ctypes.byref(d), ctypes.byref(no_x), V(0x4000), V(0x5000), V(0x6000), 1 << 20,
+                             None) == 1
+    no_lam = L.Inputs(a=V(0x1000), b=V(0x2000), x=V(0x3000))
+    assert L.lib.lr_step(ctypes.byref(d), ctypes.byref(no_lam), None, V(0x4000), V(0x5000), None) == 1
+    so = ctypes.CDLL(L.LIB_PATH)
+    so.lr_rglru_fwd_noalloc.restype = ctypes.c_int
+    assert so.lr_rglru_fwd_noalloc(ctypes.byref(d), V(0x1000), V(0x2000), V(0x3000), V(0x4000), None, 0) == 2
+    assert L.last_launch_count() == 0
+
+
 def test_plan_buffers_cover_the_queried_sizes(L):
     import torch
     for d in (L.make_desc("rotlru", torch.float32, B=2, L=1000, D=64, segment=64),

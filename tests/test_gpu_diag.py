@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import TOL, assert_close, run_gpu, to64
+from helpers import TOL, assert_close, gpu_inputs, run_gpu, to64
 from selective_state_space_09_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +42,80 @@ def test_rglru_parity(B, L, D, S, io):
     assert_close("db", gr["db"], rg["b"], tol)
     assert disp == ("rglru_fwd_tile", "rglru_bwd_tile")
     assert plan.device_error() == (0, 0)
+
+
+GATED_CASES = [
+    # B, L, D, S
+    (1, 1024, 256, 128),    # the rglru workload's shapes
+    (2, 1000, 96, 64),      # ragged L, 3 channel blocks
+    (3, 37, 40, 8),         # ragged channels
+    (1, 1, 32, 1),          # single step
+    (1, 700, 64, 256),      # maximum segment
+]
+
+
+@pytest.mark.parametrize("B,L,D,S", GATED_CASES)
+def test_rglru_gated_parity(B, L, D, S):
+    """The RG-LRU gate front-end formed in the kernels (LR_RGLRU_GATES) against the oracle's gate
+    composition: y, checkpoints, dr, di, dx and dLambda."""
+    inp = inputs.rglru_gated(B, L, D, seed=B * 100 + L)
+    y, ck, gr, plan, disp = run_gpu("rglru", inp, S, gates=True)
+    tol = TOL[torch.float32]
+    r, i, x, lam = inp["a"], inp["b"], inp["x"], inp["A"]
+    ry, rck = oracle.rglru_gated_fwd(r, i, x, lam, S=S)
+    rg = oracle.rglru_gated_bwd(r, i, x, lam, inp["dy"])
+    assert_close("y", y, ry, tol)
+    assert_close("ckpt", ck, rck, tol)
+    assert_close("dr", gr["da"], rg["r"], tol)
+    assert_close("di", gr["db"], rg["i"], tol)
+    assert_close("dx", gr["dx"], rg["x"], tol)
+    assert_close("dLambda", gr["dA"], rg["lam"], tol)
+    assert disp == ("rglru_gated_fwd_tile", "rglru_gated_bwd_tile+rglru_param_reduce")
+    assert plan.device_error() == (0, 0)
+
+
+def test_rglru_gated_edge_gates():
+    """Gates at the ends of their range: r near 0 (a -> 1, where sqrt(1 - a^2) is formed from
+    expm1 to keep its relative precision) and near 1, i = 0 and 1 exactly, Lambda large."""
+    B, L, D, S = 2, 200, 64, 32
+    inp = inputs.rglru_gated(B, L, D, seed=77)
+    gen = torch.Generator().manual_seed(4)
+    u = torch.rand(B, L, D, generator=gen)
+    inp["a"] = torch.where(u < 0.3, torch.full_like(u, 1e-3), torch.where(u > 0.7, torch.full_like(u, 0.999), inp["a"]))
+    inp["b"] = torch.where(u < 0.1, torch.zeros_like(u), torch.where(u > 0.9, torch.ones_like(u), inp["b"]))
+    inp["A"][: D // 2] = 9.0
+    y, ck, gr, plan, _ = run_gpu("rglru", inp, S, gates=True)
+    ry = oracle.rglru_gated_fwd(inp["a"], inp["b"], inp["x"], inp["A"])
+    rg = oracle.rglru_gated_bwd(inp["a"], inp["b"], inp["x"], inp["A"], inp["dy"])
+    tol = TOL[torch.float32]
+    assert_close("y", y, ry, tol)
+    for k, rk in (("da", "r"), ("db", "i"), ("dx", "x"), ("dA", "lam")):
+        assert_close(k, gr[k], rg[rk], tol)
+
+
+def test_rglru_gated_autograd_and_optional_dlambda():
+    """lrscan.rglru_gated under torch autograd gives the ABI's gradients; a NULL dA skips the
+    Lambda reduction and leaves the other gradients unchanged."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.rglru_gated(2, 300, 96, seed=9)
+    y, ck, gr, plan, _ = run_gpu("rglru", inp, 64, gates=True)
+    t = {k: v.cuda().requires_grad_(k != "dy") for k, v in inp.items()}
+    yy = lrscan.rglru_gated(t["a"], t["b"], t["x"], t["A"], segment=64)
+    yy.backward(t["dy"])
+    assert torch.equal(yy.detach(), y)
+    for k, gk in (("a", "da"), ("b", "db"), ("x", "dx"), ("A", "dA")):
+        assert torch.equal(t[k].grad, gr[gk]), k
+    g = gpu_inputs({k: v for k, v in inp.items() if k != "dy"})
+    desc = lrscan.desc_for("rglru", g, 64, gates=True)
+    p2 = lrscan.Plan(desc)
+    y2, g2 = lrscan.alloc_outputs("rglru", g)
+    p2.fwd(g, y2)
+    del g2["dA"]
+    p2.bwd(g, inp["dy"].cuda(), g2)
+    torch.cuda.synchronize()
+    assert lrscan.last_dispatch() == "rglru_gated_bwd_tile"
+    for k in ("da", "db", "dx"):
+        assert torch.equal(g2[k], gr[k]), k
 
 
 ROTLRU_CASES = [

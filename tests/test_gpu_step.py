@@ -122,6 +122,31 @@ def test_step_softplus_front_end(kind):
     assert_close("state", s_out, rh, TOL[torch.float32])
 
 
+def test_step_rglru_gates():
+    """lr_step with the RG-LRU gate front-end: parity with the oracle's gate composition from a
+    random initial state, and the CUDA-graph decode loop equal to the one-call result bitwise."""
+    inp = inputs.rglru_gated(2, 9, 40, seed=21)
+    g = gpu_inputs(api_inputs("rglru", inp))
+    desc = lrscan.desc_for("rglru", g, 1, gates=True)
+    shp = lrscan.state_shape(desc)
+    h0 = torch.randn(shp, dtype=torch.float32, generator=torch.Generator().manual_seed(5))
+    y = torch.empty_like(g["b"])
+    s_out = torch.empty(shp, dtype=torch.float32, device="cuda")
+    lrscan.step(desc, g, y, s_out, h0.cuda())
+    torch.cuda.synchronize()
+    assert lrscan.last_dispatch() == "rglru_gated_step"
+    ry, rh = oracle.rglru_gated_fwd(inp["a"], inp["b"], inp["x"], inp["A"], h0=to64(h0), final=True)
+    assert_close("y", y, ry, TOL[torch.float32])
+    assert_close("state", s_out, rh, TOL[torch.float32])
+    toks = lrscan.TOKEN_INPUTS["rglru"]
+    seq = {n: (v.transpose(0, 1).unsqueeze(2).contiguous() if n in toks else v) for n, v in g.items()}
+    yg = torch.empty((9, 2, 1, 40), dtype=torch.float32, device="cuda")
+    sg = h0.cuda()
+    lrscan.DecodeGraph("rglru", seq, sg, yg, gates=True).replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg.squeeze(2).transpose(0, 1), y) and torch.equal(sg, s_out)
+
+
 @pytest.mark.parametrize("kind,shape,io,disc", CASES[::2])
 def test_step_modes_bitwise(kind, shape, io, disc):
     """One call of L steps == L one-step calls (state in place) == the CUDA-graph decode loop."""

@@ -177,6 +177,13 @@ __device__ __forceinline__ void bulk_wait_read_1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// All but the most recent bulk group have completed (their writes performed).
+__device__ __forceinline__ void bulk_wait_all_but_1() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
+// Orders this thread's global accesses through the async proxy (bulk / TMA copies) against its
+// generic-proxy accesses (flag stores and loads).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -201,6 +208,15 @@ __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
 __device__ __forceinline__ void st_release(unsigned int* p, unsigned int v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// The same between the threads of one CTA, on a shared-memory word.
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
 
 // Status of a tile's carry record in the chained scan.
 enum : unsigned int { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2 };
@@ -219,6 +235,29 @@ __device__ __forceinline__ unsigned int wait_flag(const unsigned int* flag, WsHe
     }
     record_error(hdr, LR_ERR_TIMEOUT, info);
     return kFlagNone;
+}
+
+// Poll the n consecutive flags f[0 .. n) until all are non-zero (relaxed loads issued together,
+// then one acquire fence), for at most kWaitLimitNs.  Returns false after giving up (an error is
+// then recorded).
+__device__ __forceinline__ bool wait_flags(const unsigned int* f, int n, WsHeader* hdr, int info) {
+    const unsigned long long t0 = global_ns();
+    for (int i = 0;; ++i) {
+        bool all = true;
+        for (int k = 0; k < n; ++k) {
+            unsigned int v;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f + k) : "memory");
+            all = all && v != kFlagNone;
+        }
+        if (all) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            return true;
+        }
+        if (i > 16) __nanosleep(128);
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_error(hdr, LR_ERR_TIMEOUT, info);
+    return false;
 }
 
 // Dynamic tile ticket: tiles are numbered in the order CTAs start, so that every tile a CTA may

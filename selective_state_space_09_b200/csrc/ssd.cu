@@ -14,11 +14,15 @@
 // M is the same for every head of a group: the output kernel computes it once per (batch row,
 // chunk) and runs the group's heads through it.
 //
-// Forward = two launches, none of which waits on another CTA:
+// Forward = two launches that run side by side:
 //   ssd_scan_kernel   (batch row, head): runs through the chunks, S_{c+1} = e^{l_Q,c} S_c + Sl_c
 //                     with Sl_c on tcgen05 and S in registers; slot c of the checkpoint <- S_c
-//                     (f32, and a bf16 tile copy for the tensor cores);
-//   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x.
+//                     (f32, and a bf16 tile copy for the tensor cores), flagged once written;
+//   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x; launched as a
+//                     programmatic dependent of the scan, it starts on the SMs the scan leaves
+//                     free and waits only for the flags of its own slot.
+// The scan kernel never waits for another CTA, so the waits always end.  The backward pass has
+// the same shape (the scan in reverse, then the gradient kernel waiting per slot).
 #include "chunk_common.cuh"
 
 namespace lrs {
@@ -127,10 +131,14 @@ __device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
 //   warps 4-7 (fold, thread = state row n, all 64 columns in registers): S <- e^{l_Q} S + product,
 //     then S leaves through shared memory (f32: TMA store of two 32-column boxes; bf16 tile: one
 //     bulk copy, the tile already in its global format);
-//   warp 9: zeroes the dB, dC accumulators of the gradient kernel when asked to (backward);
+//   warp 9: zeroes the dB, dC rows the gradient kernel adds into (backward, by chunk, flagged),
+//     then flags the slots whose copies have landed (see below);
 //   warp 11 (dt): dt of every chunk into a ring in shared memory, kDtRing chunks ahead (kept out of
 //     the prep warps: their barriers and arrivals would wait for loads in flight).
-// No CTA waits on another.
+// No scan CTA waits on another.  Once the copies of a slot have landed the fold tells warp 9 (a counter
+// in shared memory), which flags the slot in global memory (a.ready), so that the output kernel
+// (forward) or the gradient kernel (backward) can start on a chunk before the whole scan has
+// finished; the fold itself never waits for a global-scope release.
 // NS stages: 3 when the f32 states are staged too (forward), 4 otherwise.
 constexpr int kScanBufs = 4, kDecRing = 16, kScanPrepGroup = 4, kDtRing = 8;
 constexpr int kScanThreads = 384;
@@ -145,6 +153,7 @@ template <int NS, bool F32> struct ScanSmem {
     static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128] f32
     static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 4;   // full, scaled, prod, bfree, dt full / empty
     static constexpr size_t kTmem = kBar + 8 * (NS + 3 * kScanBufs + 2 * kDtRing);
+    static constexpr size_t kPub = kTmem + 8;                        // puts whose copies landed, minus 1
     static constexpr size_t kEnd = kTmem + 16;
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of SW128 tiles");
@@ -159,7 +168,7 @@ template <int NS, bool F32, bool GEN>
 __global__ void __launch_bounds__(kScanThreads, 1)
 ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
                 const __grid_constant__ CUtensorMap mS, SsdArgs a, char* __restrict__ tiles, int dir,
-                float4* zero0, float4* zero1, size_t nzero4) {
+                unsigned int* ready, float* zero0, float* zero1, unsigned int* zready) {
     using SM = ScanSmem<NS, F32>;
     char* sm = smem_base1024();
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + SM::kBar);
@@ -170,6 +179,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
     uint64_t* dtempty = dtfull + kDtRing;
     float* dtr = reinterpret_cast<float*>(sm + SM::kDt);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
+    int* pubdone = reinterpret_cast<int*>(sm + SM::kPub);
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
     float* decp = reinterpret_cast<float*>(sm + SM::kDecP);
     float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
@@ -199,6 +209,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             mbar_init(&dtfull[i], 32);
             mbar_init(&dtempty[i], 1);
         }
+        *pubdone = -1;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -320,16 +331,58 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             }
         }
     } else if (warp == 9) {
-        // ------------------------------------------------------------------------- zero
-        pdl_wait();  // the previous kernel of the stream may still read dB, dC
-        for (size_t z = (size_t)blockIdx.x * 32 + lane; z < nzero4; z += (size_t)gridDim.x * 32) {
-            zero0[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            zero1[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        // --------------------------------------------------------------- zero, publish
+        // backward, several head blocks per group: the dB, dC rows [B, L, G, N] of chunk c, group
+        // g are zeroed by head g HpG + (c mod HpG) of the batch row and flagged (zready), for the
+        // gradient kernel's reduction-adds
+        if (zready) {
+            pdl_wait();  // the previous kernel of the stream may still read dB, dC
+            const int hg = h - g * a.HpG;
+            for (int c = hg; c < a.nchunk; c += a.HpG) {
+                const int rows = min(kQ, a.L - c * kQ);
+                for (int r = 0; r < rows; ++r) {
+                    const size_t off = (((size_t)b * a.L + c * kQ + r) * a.G + g) * kKD + 4 * lane;
+                    *reinterpret_cast<float4*>(zero0 + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    *reinterpret_cast<float4*>(zero1 + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(&zready[((size_t)c * a.B + b) * a.G + g], 1u);
+            }
+        }
+        // the fold's puts in order (put q writes slot q forward, slot nchunk - 1 - q backward)
+        if (ready && lane == 0) {
+            int next = 0;
+            unsigned long long t0 = global_ns();
+            while (next < a.nchunk) {
+                const int done = ld_acquire_cta(pubdone);
+                if (done >= next) {
+                    for (; next <= done; ++next) {
+                        const int slot = dir > 0 ? next : a.nchunk - 1 - next;
+                        st_release(&ready[((size_t)slot * a.B + b) * a.H + h], 1u);
+                    }
+                    t0 = global_ns();
+                    continue;
+                }
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    record_error(a.hdr, LR_ERR_TIMEOUT, 747);
+                    break;
+                }
+                __nanosleep(100);
+            }
         }
     } else {
         // ------------------------------------------------------------------------- fold
         const int n = tid - 128, fl = n == 0;  // fl: the thread that issues the copies
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        // fl: the last two puts whose copies were issued (pub1 the latest); a put is handed to the
+        // publishing warp once the copies of the put after it have been issued, by which time its
+        // own have landed
+        int nput = 0, pub1 = -1, pub2 = -1;
+        auto publish = [&](int q) {  // puts 0 .. q have landed
+            fence_proxy_async_global();
+            st_release_cta(pubdone, q);
+        };
         float S[kP];
 #pragma unroll
         for (int i = 0; i < kP; ++i) S[i] = 0.0f;
@@ -337,7 +390,13 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
         // S into slot c through the staging buffers (free: the copies of the previous slot have
         // read them before the first barrier)
         auto put = [&](int c) {
-            if (fl) bulk_wait_read_all();
+            if (fl) {
+                if (ready && pub2 >= 0) {
+                    bulk_wait_all_but_1();
+                    publish(pub2);
+                }
+                bulk_wait_read_all();
+            }
             wg_sync(1);
             if constexpr (F32) {
 #pragma unroll
@@ -363,6 +422,8 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
                 bulk_store(tiles + ((size_t)c * BH + bh) * kTileBytes, sm + SM::kBf, kTileBytes);
                 bulk_commit();
             }
+            pub2 = pub1;
+            pub1 = nput++;
         };
         put(dir > 0 ? 0 : a.nchunk - 1);
         for (int k = 0; k < nk; ++k) {
@@ -380,7 +441,10 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             for (int i = 0; i < kP; ++i) S[i] = fmaf(d, S[i], v[i]);
             put(chunk_of(k) + dir);
         }
-        if (fl) bulk_wait_all();
+        if (fl) {
+            bulk_wait_all();
+            if (ready) publish(pub1);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -447,7 +511,7 @@ template <bool GEN>
 __global__ void __launch_bounds__(256, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
-               const char* stiles, int hb, int nblk) {
+               const char* stiles, const unsigned int* ready, int hb, int nblk) {
     using SM = OutSmem;
     char* sm = smem_base1024();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
@@ -503,8 +567,14 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             tma_load_4d(Xs + u * kQ * 128, &mX, &wbar[u], 0, hfirst + wg + 2 * u, t0, b);
         }
     }
-    pdl_wait();  // the S_in tiles come from the previous kernel
+    // S_in tiles of chunk c: written by the scan kernel, which flags each slot once its copies
+    // have landed, so this kernel runs beside the scan instead of after all of it (slot 0, the
+    // zero state, is waited for too: the scan flags it only after the kernels before it are done)
+    bool ok = true;
     if (wt == 0) {
+        for (int u = 0; u < nmine; ++u)
+            ok = ok && wait_flag(&ready[((size_t)c * a.B + b) * a.H + hfirst + wg + 2 * u], a.hdr, 716) != 0;
+        fence_proxy_async_global();
         if (has_in && nmine > 0) {
             mbar_arrive_expect_tx(&wbar[3], kTileBytes);
             bulk_load(St, stile(hfirst + wg), kTileBytes, &wbar[3]);
@@ -512,9 +582,8 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     }
     if (wg == 0) load_dts<GEN>(a, dts, ad, b, t0, hfirst, nh, wt);
     __syncthreads();
-    bool ok = true;
     if (tid == 0) {
-        ok = mbar_wait(&bar[0], 0, a.hdr, 710);
+        ok = ok && mbar_wait(&bar[0], 0, a.hdr, 710);
         if (ok) {
             tc::fence_after_sync();
             tc::mma_tiles(tmem, sC, 0, kQ, sB, 0, kQ, kQ, kQ, kKD, 0);  // M = C B^T
@@ -662,11 +731,13 @@ bool general_variant(const lr_desc& d) {
 }
 
 struct SsdFwdWs {
-    size_t end;  // the workspace holds only the header
+    size_t ready, end;  // after the header: the slot flags of the scan kernel (reset every call)
 };
-SsdFwdWs fwd_plan(const lr_desc&) {
+SsdFwdWs fwd_plan(const lr_desc& d) {
     WsCursor cur;
     SsdFwdWs w;
+    const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
+    w.ready = cur.take(sizeof(unsigned int) * nchunk * d.B * d.H);
     w.end = cur.off;
     return w;
 }
@@ -704,25 +775,32 @@ int sm_count() {
     return n;
 }
 
-// Heads per output CTA (at most 16; 16 under LR_TEST_MAX_HEAD_BLOCK): the block size that
-// minimises waves x per-CTA time, a CTA taking about 2 units per head of each warpgroup (two
-// warpgroups alternate heads) plus 1 unit of prologue (C, B loads and C B^T).
+// Heads per output CTA (at most 16; 16 under LR_TEST_MAX_HEAD_BLOCK).  A CTA takes about 2 units
+// per head of each warpgroup (two warpgroups alternate heads) plus 1 unit of prologue (C, B loads
+// and C B^T); a unit is about 3.2 us.  The output kernel runs beside the scan kernel, whose B*H
+// CTAs hold their SMs for about 0.56 units per chunk, on the SMs the scan leaves free, and ends
+// after it: the block size minimises the estimated time past the scan's end, the longer of one
+// CTA (the last chunk's CTAs start when the scan ends) and the work the free SMs could not take
+// spread over all SMs.
 int out_heads_per_cta(const lr_desc& d, int nchunk) {
     const int HpG = (int)(d.H / d.G);
     const long units = (long)nchunk * d.B * d.G;
     const int top = HpG < 16 ? HpG : 16;
     if (d.flags & LR_TEST_MAX_HEAD_BLOCK) return top;
+    const long sms = sm_count();
+    const long free_sms = sms > d.B * d.H ? sms - d.B * d.H : 0;
+    const long absorbed = free_sms * nchunk * 9 / 16;  // unit-SMs the free SMs offer during the scan
     int best = top;
     long best_cost = -1;
-    for (int hb = top; hb >= 1; hb = hb > 1 ? (hb + 1) / 2 : 0) {
-        const long ctas = units * ((HpG + hb - 1) / hb);
-        const long waves = (ctas + sm_count() - 1) / sm_count();
-        const long cost = waves * (2 * ((hb + 1) / 2) + 1);
+    for (int hb = top; hb >= 1; --hb) {
+        const long cta = 2 * ((hb + 1) / 2) + 1;
+        const long work = units * ((HpG + hb - 1) / hb) * cta;
+        const long rest = work > absorbed ? (work - absorbed + sms - 1) / sms : 0;
+        const long cost = 4 * (cta > rest ? cta : rest) + (cta > rest ? rest : cta);  // ties: the other term
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = hb;
         }
-        if (hb == 1) break;
     }
     return best;
 }
@@ -752,6 +830,8 @@ struct SsdGradArgs {
     float* pdA;            // [B][H][nchunk] per-chunk partials of dA_h, dD_h
     float* pdD;
     float* pdE;            // [B][H][nchunk] partials of d bias (LR_DELTA_SOFTPLUS)
+    const unsigned int* gready;  // [nchunk][B][H]: G tile of the slot written (by the scan kernel)
+    const unsigned int* zready;  // [nchunk][B][G]: the chunk's dB, dC rows zeroed (by the scan kernel)
     int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
 };
 
@@ -775,6 +855,7 @@ struct GradSmem {
     static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
     static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 + 7 slots, 3 phase A (+ batch 2), 4 batch 1 (dV1, BG, Y2), 5 batch 1 (dC, dB), 6 S_in/G
     static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kTicket = kTmem + 8;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kAlloc <= 232448, "gradient CTA exceeds the shared memory of one CTA");
@@ -827,17 +908,10 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     const int row = tid & 127;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
 
-    int idx = blockIdx.x;
-    const int blk = idx % nblk;
-    idx /= nblk;
-    const int g = idx % a.G;
-    idx /= a.G;
-    const int b = idx % a.B;
-    const int c = idx / a.B;
-    const int t0 = c * kQ;
-    const int hfirst = g * a.HpG + blk * hb;
-    const int nh = min(hb, a.HpG - blk * hb);
-    const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
+    // tile from a ticket taken at the start: chunks from the last (whose adjoint the scan kernel
+    // writes first), and head block 0 of a (chunk, row, group) before the blocks that wait for it
+    unsigned int* ticket = reinterpret_cast<unsigned int*>(sm + SM::kTicket);
+    if (tid == 0) *ticket = take_ticket(a.hdr, 0);
     pdl_launch_dependents();
 
     if (tid == 0) {
@@ -850,6 +924,17 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    int idx = (int)*ticket;
+    const int blk = idx % nblk;
+    idx /= nblk;
+    const int g = idx % a.G;
+    idx /= a.G;
+    const int b = idx % a.B;
+    const int c = a.nchunk - 1 - idx / a.B;
+    const int t0 = c * kQ;
+    const int hfirst = g * a.HpG + blk * hb;
+    const int nh = min(hb, a.HpG - blk * hb);
+    const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
     // Three 32 KB slots rotate per head i: {x, dy} in slot i % 3, P in (i + 1) % 3, Pd in (i + 2) % 3.
     // P is consumed first (batch 1a), so its slot takes {x, dy} of head i + 1; Pd's slot takes P of
     // head i + 1 and the {x, dy} slot (free after batch 2) Pd of head i + 1.
@@ -909,16 +994,22 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         }
         load_xdy(0, hfirst);
     }
-    pdl_wait();  // the G tiles (and the zeroed dB, dC) come from the previous kernel
-    if (tid == 0) load_sg(hfirst);
+    // the G tiles of slot c, written by the scan kernel, which flags each slot once its copies have
+    // landed (the last chunk's slot, the zero adjoint, too: the scan flags it only after the kernels
+    // before it are done), so this kernel runs beside the scan instead of after all of it
+    bool ok = true;
+    if (tid == 0) {
+        ok = wait_flags(&ga.gready[((size_t)c * a.B + b) * a.H + hfirst], nh, a.hdr, 728);
+        fence_proxy_async_global();
+        load_sg(hfirst);
+    }
     if (wg == 0) {
         load_dts<GEN>(a, dts, ad, b, t0, hfirst, nh, row);
         wg0_bar();
         decays(0);
     }
-    bool ok = true;
     if (tid == 0) {
-        ok = mbar_wait(&bar[0], 0, a.hdr, 721) && mbar_wait(&bar[1], 0, a.hdr, 722);
+        ok = ok && mbar_wait(&bar[0], 0, a.hdr, 721) && mbar_wait(&bar[1], 0, a.hdr, 722);
         if (ok) {
             tc::fence_after_sync();
             phase_a(0);
@@ -1172,8 +1263,13 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         }
     }
     // dC, dB of this (batch row, chunk, group): rows t, columns [64 wg, 64 wg + 64).  Every lane
-    // takes part in the (warp-collective) TMEM loads; rows past L are not stored.
+    // takes part in the (warp-collective) TMEM loads; rows past L are not stored.  Several head
+    // blocks add onto rows the scan kernel has zeroed (and flagged).
     ok = ok && mbar_wait(&bar[3], (uint32_t)(nh & 1), a.hdr, 725);
+    if (ga.accumulate) {
+        if (tid == 0) ok = ok && wait_flag(&ga.zready[((size_t)c * a.B + b) * a.G + g], a.hdr, 726) != 0;
+        __syncthreads();
+    }
     tc::fence_after_sync();
     {
         const bool vrow = t0 + row < a.L;
@@ -1238,13 +1334,16 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
 }
 
 struct SsdBwdWs {
-    size_t pdA, pdD, pdE, gtiles, end;
+    size_t gready, dbc, flags_end, pdA, pdD, pdE, gtiles, end;  // flags first: reset every call
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     const size_t tiles = (size_t)d.B * d.H * nchunk;
     WsCursor cur;
     SsdBwdWs w;
+    w.gready = cur.take(sizeof(unsigned int) * tiles);
+    w.dbc = cur.take(sizeof(unsigned int) * nchunk * d.B * d.G);
+    w.flags_end = cur.off;
     w.pdA = cur.take(sizeof(float) * tiles);
     w.pdD = cur.take(sizeof(float) * tiles);
     w.pdE = cur.take(sizeof(float) * tiles);
@@ -1267,10 +1366,11 @@ int grad_heads_per_cta(const lr_desc& d, int nchunk) {
 }  // namespace
 
 size_t ssd_fwd_ws_bytes(const lr_desc& d) { return fwd_plan(d).end; }
-size_t ssd_fwd_flag_bytes(const lr_desc&) { return 256; }
+size_t ssd_fwd_flag_bytes(const lr_desc& d) { return fwd_plan(d).end; }
 
 lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
     SsdArgs a = make_args(d, in, ckpt, ws);
+    unsigned int* ready = (unsigned int*)(ws + fwd_plan(d).ready);
     CUtensorMap mC, mB, mX, mY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
@@ -1284,7 +1384,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     CUtensorMap mS;
     if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
     if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, a, stiles, +1,
-                   (float4*)nullptr, (float4*)nullptr, (size_t)0) != cudaSuccess)
+                   ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr) != cudaSuccess)
         return LR_ERR_CUDA;
     {
         lr_status s = check_launch();
@@ -1296,13 +1396,13 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     cudaFuncSetAttribute(out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
     if (launch_pdl(out, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
-                   a, (const char*)stiles, hb, nblk_o) != cudaSuccess)
+                   a, (const char*)stiles, (const unsigned int*)ready, hb, nblk_o) != cudaSuccess)
         return LR_ERR_CUDA;
     return check_launch();
 }
 
 size_t ssd_bwd_ws_bytes(const lr_desc& d) { return bwd_plan(d).end; }
-size_t ssd_bwd_flag_bytes(const lr_desc&) { return 256; }
+size_t ssd_bwd_flag_bytes(const lr_desc& d) { return bwd_plan(d).flags_end; }
 
 lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const void* ckpt, const lr_grads& gr,
                   char* ws, cudaStream_t st) {
@@ -1325,16 +1425,18 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     if (!ok) return LR_ERR_INVALID_ARG;
     const int hb = grad_heads_per_cta(d, a.nchunk);
     const int nblk = (a.HpG + hb - 1) / hb;
-    ga.accumulate = nblk > 1 ? 1 : 0;  // several head blocks add into dB, dC: the scan kernel zeroes them
+    ga.accumulate = nblk > 1 ? 1 : 0;
+    ga.gready = (const unsigned int*)(ws + w.gready);
+    ga.zready = (const unsigned int*)(ws + w.dbc);
     {
-        const size_t nzero4 = ga.accumulate ? (size_t)d.B * d.L * d.G * kKD / 4 : 0;
         using ScanB = ScanSmem<4, false>;
         auto scan = general_variant(d) ? ssd_scan_kernel<4, false, true> : ssd_scan_kernel<4, false, false>;
         cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
         note_launch("ssd_state_scan");
         // no f32 states in this direction (the map argument is unused)
         if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, a, ws + w.gtiles, -1,
-                       (float4*)gr.dBm, (float4*)gr.dCm, nzero4) != cudaSuccess)
+                       (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
+                       ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;

@@ -150,13 +150,14 @@ template <int NS, bool F32> struct ScanSmem {
     static constexpr size_t kTmp = kBf + kTileBytes;                 // prep scan scratch [4][4], l_Q [4]
     static constexpr size_t kDecP = kTmp + 128;                      // e^{l_Q}: prep -> issue [kDecRing]
     static constexpr size_t kDecF = kDecP + 4 * kDecRing;            // e^{l_Q}: issue -> fold [kDecRing]
-    static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128] f32
-    static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 4;   // full, scaled, prod, bfree, dt full / empty
+    static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128][8] bf16
+    static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 16;  // full, scaled, prod, bfree, dt full / empty
     static constexpr size_t kTmem = kBar + 8 * (NS + 3 * kScanBufs + 2 * kDtRing);
     static constexpr size_t kPub = kTmem + 8;                        // puts whose copies landed, minus 1
     static constexpr size_t kEnd = kTmem + 16;
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of SW128 tiles");
+    static_assert(kDt % 128 == 0, "dt ring slots are TMA destinations");
     static_assert(kAlloc <= 232448, "scan CTA exceeds the shared memory of one CTA");
     // the prep role writes e^{l_Q} at most NS + kScanPrepGroup chunks ahead of the issuing thread;
     // kScanBufs >= NS keeps every mbarrier at most one phase ahead of its waiters
@@ -167,8 +168,9 @@ template <int NS, bool F32> struct ScanSmem {
 template <int NS, bool F32, bool GEN>
 __global__ void __launch_bounds__(kScanThreads, 1)
 ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
-                const __grid_constant__ CUtensorMap mS, SsdArgs a, char* __restrict__ tiles, int dir,
-                unsigned int* ready, float* zero0, float* zero1, unsigned int* zready) {
+                const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mDt, int dt_tma,
+                SsdArgs a, char* __restrict__ tiles, int dir, unsigned int* ready, float* zero0, float* zero1,
+                unsigned int* zready) {
     using SM = ScanSmem<NS, F32>;
     char* sm = smem_base1024();
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + SM::kBar);
@@ -177,7 +179,9 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
     uint64_t* bfree = prod + kScanBufs;
     uint64_t* dtfull = bfree + kScanBufs;
     uint64_t* dtempty = dtfull + kDtRing;
-    float* dtr = reinterpret_cast<float*>(sm + SM::kDt);
+    // dt ring: slot s, step t holds the raw dt of heads 8 (h / 8) .. 8 (h / 8) + 7 (a TMA box of
+    // the [B, L, H] tensor when H is a multiple of 8; else only head h's entry is written)
+    __nv_bfloat16* dtb = reinterpret_cast<__nv_bfloat16*>(sm + SM::kDt);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
     int* pubdone = reinterpret_cast<int*>(sm + SM::kPub);
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
@@ -185,6 +189,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
     float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, g = h / a.HpG;
+    const int hx = h & 7;  // this head's column of a dt ring row
     const int BH = a.B * a.H;
     const int nk = a.nchunk - 1;  // chunks with a product
     auto chunk_of = [&](int k) { return dir > 0 ? k : a.nchunk - 1 - k; };
@@ -206,7 +211,7 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             mbar_init(&bfree[i], 128);
         }
         for (int i = 0; i < kDtRing; ++i) {
-            mbar_init(&dtfull[i], 32);
+            mbar_init(&dtfull[i], dt_tma ? 1 : 32);
             mbar_init(&dtempty[i], 1);
         }
         *pubdone = -1;
@@ -232,7 +237,8 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
                 const int k = k0 + j;
                 ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
                 const bool in_seq = chunk_of(k) * kQ + t < a.L;
-                const float dtv = in_seq ? ssd_dt<GEN>(a, dtr[(k % kDtRing) * kQ + t], h) : 0.0f;  // 0 past L
+                const float dtv =  // 0 past L
+                    in_seq ? ssd_dt<GEN>(a, __bfloat162float(dtb[((k % kDtRing) * kQ + t) * 8 + hx]), h) : 0.0f;
                 l[j] = dtv * Ah;
                 beta[j] = in_seq ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
             }
@@ -303,9 +309,28 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
         }
     } else if (warp == 11) {
         // --------------------------------------------------------------------------- dt
-        // one prep group (kScanPrepGroup chunks) per batch of loads: an arrival waits for every load
-        // of the thread in flight, so the loads of a group are all issued before the first one
+        // TMA: one box of 8 heads x 128 steps per chunk.  Loads: one prep group (kScanPrepGroup
+        // chunks) per batch of loads: an arrival waits for every load of the thread in flight, so
+        // the loads of a group are all issued before the first one.
         constexpr int NG = kScanPrepGroup;
+        if (dt_tma) {
+            if (lane == 0)
+                for (int k = 0; k < nk; ++k) {
+                    const int slot = k % kDtRing;
+                    if (k >= kDtRing)
+                        ok = ok && mbar_wait(&dtempty[slot], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
+                    mbar_arrive_expect_tx(&dtfull[slot], (uint32_t)(kQ * 16));
+                    tma_load_3d(dtb + (size_t)slot * kQ * 8, &mDt, &dtfull[slot], h & ~7, chunk_of(k) * kQ, b);
+                }
+            // the prep group's chunks past the last product: nothing to load
+            if (lane == 0)
+                for (int k = nk; k % NG != 0; ++k) {
+                    const int slot = k % kDtRing;
+                    if (k >= kDtRing)
+                        ok = ok && mbar_wait(&dtempty[slot], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
+                    mbar_arrive(&dtfull[slot]);
+                }
+        } else
         for (int k0 = 0; k0 < nk; k0 += NG) {
             if (k0 >= kDtRing) {
 #pragma unroll
@@ -326,7 +351,8 @@ ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ 
             for (int j = 0; j < NG; ++j) {
                 const int slot = (k0 + j) % kDtRing;
 #pragma unroll
-                for (int i = 0; i < kQ / 32; ++i) dtr[slot * kQ + lane + 32 * i] = v[j][i];
+                for (int i = 0; i < kQ / 32; ++i)
+                    dtb[(slot * kQ + lane + 32 * i) * 8 + hx] = __float2bfloat16_rn(v[j][i]);
                 mbar_arrive(&dtfull[slot]);
             }
         }
@@ -723,6 +749,13 @@ bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
     uint64_t str[3] = {kP * 4, (uint64_t)kKD * kP * 4, (uint64_t)BH * kKD * kP * 4};
     uint32_t box[4] = {32, (uint32_t)kKD, 1, 1};
     return make_tmap(m, base, 4, 4, dims, str, box, true);
+}
+
+// TMA map of the raw dt [B, L, H] bf16 with boxes of 8 heads x 128 steps (16-byte rows): only
+// when a row of H heads spans a multiple of 16 bytes (H a multiple of 8); false otherwise.
+bool map_dt(CUtensorMap* m, const lr_desc& d, const void* dt) {
+    if (d.H % 8 != 0) return false;
+    return make_tmap_3d(m, dt, 2, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.B, 8, (uint32_t)kQ);
 }
 
 // The general kernel variant: a discretisation other than ZOH, or the softplus front-end.
@@ -1383,8 +1416,11 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     note_launch("ssd_state_scan");
     CUtensorMap mS;
     if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
-    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, a, stiles, +1,
-                   ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr) != cudaSuccess)
+    CUtensorMap mDt;
+    const int dt_tma = map_dt(&mDt, d, in.delta) ? 1 : 0;
+    if (!dt_tma) mDt = mB;  // not read
+    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, mDt, dt_tma, a, stiles,
+                   +1, ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr) != cudaSuccess)
         return LR_ERR_CUDA;
     {
         lr_status s = check_launch();
@@ -1434,8 +1470,11 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
         note_launch("ssd_state_scan");
         // no f32 states in this direction (the map argument is unused)
-        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, a, ws + w.gtiles, -1,
-                       (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
+        CUtensorMap mDt;
+        const int dt_tma = map_dt(&mDt, d, in.delta) ? 1 : 0;
+        if (!dt_tma) mDt = mC;  // not read
+        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, mDt, dt_tma, a,
+                       ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
                        ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;
         lr_status s = check_launch();

@@ -14,8 +14,11 @@ from selective_state_space_09_b200 import inputs
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
 
+# (B, L, H, P, G).  Also covers: dt boxes by TMA (H a multiple of 8) and by per-lane loads (other
+# H); several head blocks adding into dB, dC rows zeroed by the scan kernel, with more chunks than
+# heads per group (1, 1000, 2: each head zeroes four chunks' rows).
 SSD_CASES = [(1, 512, 4, 64, 1), (2, 300, 8, 64, 2), (1, 128, 2, 64, 1), (1, 77, 8, 64, 1),
-             (1, 384, 12, 64, 1), (2, 260, 10, 64, 2), (1, 520, 40, 64, 2)]
+             (1, 384, 12, 64, 1), (2, 260, 10, 64, 2), (1, 520, 40, 64, 2), (1, 1000, 2, 64, 1)]
 SSD_FWD = ("ssd_state_scan+ssd_chunk_out",)
 SSD_BWD = ("ssd_state_scan+ssd_chunk_grad+ssd_param_reduce",)
 

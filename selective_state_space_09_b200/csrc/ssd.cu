@@ -15,7 +15,7 @@
 // chunk) and runs the group's heads through it.
 //
 // Forward = two launches that run side by side:
-//   ssd_scan_kernel   (batch row, head): runs through the chunks, S_{c+1} = e^{l_Q,c} S_c + Sl_c
+//   chunk_scan_kernel (batch row, head; chunk_scan.cuh): runs through the chunks, S_{c+1} = e^{l_Q,c} S_c + Sl_c
 //                     with Sl_c on tcgen05 and S in registers; slot c of the checkpoint <- S_c
 //                     (f32, and a bf16 tile copy for the tensor cores), flagged once written;
 //   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x; launched as a
@@ -23,7 +23,7 @@
 //                     free and waits only for the flags of its own slot.
 // The scan kernel never waits for another CTA, so the waits always end.  The backward pass has
 // the same shape (the scan in reverse, then the gradient kernel waiting per slot).
-#include "chunk_common.cuh"
+#include "chunk_scan.cuh"
 
 namespace lrs {
 using namespace chunkc;
@@ -44,13 +44,25 @@ struct SsdArgs {
     WsHeader* hdr;
 };
 
-// beta of one step inside the sequence (lam = dt A_h): ZOH (e^{lam} - 1) / A_h, dirac 1,
-// ZOH-Euler dt.  abar = e^{lam} in all three.
-__device__ __forceinline__ float ssd_beta(int disc, float lam, float dt, float Ah) {
-    if (disc == LR_DISC_DIRAC) return 1.0f;
-    if (disc == LR_DISC_ZOH_EULER) return dt;
-    return (ex2(lam * kLog2e) - 1.0f) / Ah;
+// The scan kernel's view of the problem (chunk_scan.cuh).
+__host__ ScanArgs scan_args(const SsdArgs& a) {
+    ScanArgs s{};
+    s.B = a.B;
+    s.L = a.L;
+    s.H = a.H;
+    s.G = a.G;
+    s.HpG = a.HpG;
+    s.nchunk = a.nchunk;
+    s.halves = 1;
+    s.disc = a.disc;
+    s.softplus = a.softplus;
+    s.dbias = a.dbias;
+    s.dt = a.dt;
+    s.A = a.A;
+    s.hdr = a.hdr;
+    return s;
 }
+
 
 // Sums of three values over the 128 threads of warpgroup 0, fixed order, results in every thread
 // (tmp: 32 floats, the layout wg0_sum2 uses for two).
@@ -74,411 +86,6 @@ __device__ __forceinline__ float3 wg0_sum3(float x, float y, float z, float* tmp
     return s;
 }
 
-// The kernels come in two variants: the default one (ZOH, raw dt) with both fixed at compile time,
-// and the general one (GEN) that takes the discretisation and the softplus front-end from the
-// arguments.
-template <bool GEN>
-__device__ __forceinline__ int disc_of(const SsdArgs& a) {
-    if constexpr (GEN) return a.disc;
-    return LR_DISC_ZOH;
-}
-template <bool GEN>
-__device__ __forceinline__ bool softplus_of(const SsdArgs& a) {
-    if constexpr (GEN) return a.softplus != 0;
-    return false;
-}
-
-// dt of head h from the raw delta: itself, or softplus(delta + bias_h) (LR_DELTA_SOFTPLUS)
-template <bool GEN>
-__device__ __forceinline__ float ssd_dt(const SsdArgs& a, float raw, int h) {
-    if (!softplus_of<GEN>(a)) return raw;
-    const float v = raw + (a.dbias ? a.dbias[h] : 0.0f);
-    return v > 20.0f ? v : log1pf(__expf(v));
-}
-
-// Barrier of the 128 threads of warpgroup wg (named barrier 1 + wg).
-__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
-
-// Inclusive prefix sum over the 128 threads of warpgroup wg (same order as cta_inclusive_sum).
-__device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
-    const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 3;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) tmp[w] = x;
-    wg_sync(wg);
-    float add = 0.0f;
-    for (int k = 0; k < w; ++k) add += tmp[k];
-    wg_sync(wg);
-    return x + add;
-}
-
-// -------------------------------------------------------------------- chunk states, scanned
-// One CTA per (batch row, head) walks the chunks in order (dir > 0) or in reverse (dir < 0):
-//   dir > 0: S_0 = 0,      S_{c+1} = e^{l_Q,c} S_c + B_c^T diag(w) x_c    slot c <- S_c
-//            (the f32 checkpoint and its bf16 tile copy);
-//   dir < 0: G_{last} = 0, G_{c-1} = e^{l_Q,c} G_c + C_c^T diag(E) dy_c   slot c <- G_c (bf16 tile).
-// Only the fold is sequential; the chunk products are independent, so the CTA runs as a pipeline of
-// roles joined by mbarriers:
-//   warps 0-3 (prep, thread = step t): decays of kScanPrepGroup chunks at a time (inclusive sums of
-//     dt A), then per chunk, once its tiles are in, row t of x (dy) scaled by w_t (E_t) in place;
-//   warp 8 lane 0 (issue): the tcgen05 product of each prepared chunk into one of kScanBufs TMEM
-//     buffers;
-//   warp 10 lane 0 (load): the TMA loads of the chunk tiles into a ring of NS stages, each stage
-//     refilled as soon as the product that reads it has completed;
-//   warps 4-7 (fold, thread = state row n, all 64 columns in registers): S <- e^{l_Q} S + product,
-//     then S leaves through shared memory (f32: TMA store of two 32-column boxes; bf16 tile: one
-//     bulk copy, the tile already in its global format);
-//   warp 9: zeroes the dB, dC rows the gradient kernel adds into (backward, by chunk, flagged),
-//     then flags the slots whose copies have landed (see below);
-//   warp 11 (dt): dt of every chunk into a ring in shared memory, kDtRing chunks ahead (kept out of
-//     the prep warps: their barriers and arrivals would wait for loads in flight).
-// No scan CTA waits on another.  Once the copies of a slot have landed the fold tells warp 9 (a counter
-// in shared memory), which flags the slot in global memory (a.ready), so that the output kernel
-// (forward) or the gradient kernel (backward) can start on a chunk before the whole scan has
-// finished; the fold itself never waits for a global-scope release.
-// NS stages: 3 when the f32 states are staged too (forward), 4 otherwise.
-constexpr int kScanBufs = 4, kDecRing = 16, kScanPrepGroup = 4, kDtRing = 8;
-constexpr int kScanThreads = 384;
-template <int NS, bool F32> struct ScanSmem {
-    static constexpr size_t kRt = (size_t)kQ * kKD * 2;            // R tile (B or C), 128 x 128 bf16
-    static constexpr size_t kStage = kRt + (size_t)kQ * kP * 2;      // then the Z tile (x or dy)
-    static constexpr size_t kF32 = (size_t)NS * kStage;             // f32 state staging, 2 boxes
-    static constexpr size_t kBf = kF32 + (F32 ? (size_t)kKD * kP * 4 : 0);  // bf16 tile staging
-    static constexpr size_t kTmp = kBf + kTileBytes;                 // prep scan scratch [4][4], l_Q [4]
-    static constexpr size_t kDecP = kTmp + 128;                      // e^{l_Q}: prep -> issue [kDecRing]
-    static constexpr size_t kDecF = kDecP + 4 * kDecRing;            // e^{l_Q}: issue -> fold [kDecRing]
-    static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128][8] bf16
-    static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 16;  // full, scaled, prod, bfree, dt full / empty
-    static constexpr size_t kTmem = kBar + 8 * (NS + 3 * kScanBufs + 2 * kDtRing);
-    static constexpr size_t kPub = kTmem + 8;                        // puts whose copies landed, minus 1
-    static constexpr size_t kEnd = kTmem + 16;
-    static constexpr size_t kAlloc = kEnd + 1024;
-    static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of SW128 tiles");
-    static_assert(kDt % 128 == 0, "dt ring slots are TMA destinations");
-    static_assert(kAlloc <= 232448, "scan CTA exceeds the shared memory of one CTA");
-    // the prep role writes e^{l_Q} at most NS + kScanPrepGroup chunks ahead of the issuing thread;
-    // kScanBufs >= NS keeps every mbarrier at most one phase ahead of its waiters
-    static_assert(kScanBufs >= NS && NS + kScanPrepGroup < kDecRing, "ring sizes");
-    static_assert(kDtRing % kScanPrepGroup == 0 && kDtRing >= 2 * kScanPrepGroup, "dt ring holds two prep groups");
-};
-
-template <int NS, bool F32, bool GEN>
-__global__ void __launch_bounds__(kScanThreads, 1)
-ssd_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
-                const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mDt, int dt_tma,
-                SsdArgs a, char* __restrict__ tiles, int dir, unsigned int* ready, float* zero0, float* zero1,
-                unsigned int* zready) {
-    using SM = ScanSmem<NS, F32>;
-    char* sm = smem_base1024();
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + SM::kBar);
-    uint64_t* scaled = full + NS;
-    uint64_t* prod = scaled + kScanBufs;
-    uint64_t* bfree = prod + kScanBufs;
-    uint64_t* dtfull = bfree + kScanBufs;
-    uint64_t* dtempty = dtfull + kDtRing;
-    // dt ring: slot s, step t holds the raw dt of heads 8 (h / 8) .. 8 (h / 8) + 7 (a TMA box of
-    // the [B, L, H] tensor when H is a multiple of 8; else only head h's entry is written)
-    __nv_bfloat16* dtb = reinterpret_cast<__nv_bfloat16*>(sm + SM::kDt);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
-    int* pubdone = reinterpret_cast<int*>(sm + SM::kPub);
-    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
-    float* decp = reinterpret_cast<float*>(sm + SM::kDecP);
-    float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, g = h / a.HpG;
-    const int hx = h & 7;  // this head's column of a dt ring row
-    const int BH = a.B * a.H;
-    const int nk = a.nchunk - 1;  // chunks with a product
-    auto chunk_of = [&](int k) { return dir > 0 ? k : a.nchunk - 1 - k; };
-    auto stage = [&](int k) { return sm + (size_t)(k % NS) * SM::kStage; };
-    auto load = [&](int k) {
-        char* st = stage(k);
-        uint64_t* bar = &full[k % NS];
-        const int t0 = chunk_of(k) * kQ;
-        mbar_arrive_expect_tx(bar, (uint32_t)SM::kStage);
-        for (int j = 0; j < kKD / 64; ++j) tma_load_4d(st + j * kQ * 128, &mR, bar, 64 * j, g, t0, b);
-        tma_load_4d(st + SM::kRt, &mZ, bar, 0, h, t0, b);
-    };
-    pdl_launch_dependents();
-    if (tid == 256) {
-        for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
-        for (int i = 0; i < kScanBufs; ++i) {
-            mbar_init(&scaled[i], 128);
-            mbar_init(&prod[i], 2);  // the product's commit and the issuing thread (e^{l_Q} handed on)
-            mbar_init(&bfree[i], 128);
-        }
-        for (int i = 0; i < kDtRing; ++i) {
-            mbar_init(&dtfull[i], dt_tma ? 1 : 32);
-            mbar_init(&dtempty[i], 1);
-        }
-        *pubdone = -1;
-        fence_barrier_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 8) tc::tmem_alloc(tmem_slot, 64 * kScanBufs);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    bool ok = true;
-
-    if (warp < 4) {
-        // ------------------------------------------------------------------------- prep
-        constexpr int NG = kScanPrepGroup;
-        const int t = tid;
-        const float Ah = a.A[h];
-        for (int k0 = 0; k0 < nk; k0 += NG) {
-            float l[NG], beta[NG], f[NG];
-#pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                const int k = k0 + j;
-                ok = ok && mbar_wait(&dtfull[k % kDtRing], (uint32_t)((k / kDtRing) & 1), a.hdr, 745);
-                const bool in_seq = chunk_of(k) * kQ + t < a.L;
-                const float dtv =  // 0 past L
-                    in_seq ? ssd_dt<GEN>(a, __bfloat162float(dtb[((k % kDtRing) * kQ + t) * 8 + hx]), h) : 0.0f;
-                l[j] = dtv * Ah;
-                beta[j] = in_seq ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
-            }
-            wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
-            if (t == 0) {
-#pragma unroll
-                for (int j = 0; j < NG; ++j) mbar_arrive(&dtempty[(k0 + j) % kDtRing]);
-            }
-            if (t == kQ - 1) {
-#pragma unroll
-                for (int j = 0; j < NG; ++j) tmp[4 * NG + j] = l[j];
-            }
-            wg_sync(0);
-#pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                const float lQ2 = tmp[4 * NG + j] * kLog2e, lt2 = l[j] * kLog2e;
-                f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] : ex2(lt2);
-                if (t == 0) decp[(k0 + j) % kDecRing] = ex2(lQ2);
-            }
-#pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                const int k = k0 + j;
-                if (k >= nk) break;
-                ok = ok && mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1), a.hdr, 740);
-                char* z = stage(k) + SM::kRt;
-                uint4 raw[kP / 8];  // the whole row first: its loads overlap
-#pragma unroll
-                for (int c = 0; c < kP / 8; ++c) raw[c] = *reinterpret_cast<const uint4*>(z + tc::sw128_off(t, 8 * c, kQ));
-#pragma unroll
-                for (int c = 0; c < kP / 8; ++c) {
-                    __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&raw[c]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 v = __bfloat1622float2(hv[i]);
-                        hv[i] = __floats2bfloat162_rn(v.x * f[j], v.y * f[j]);
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < kP / 8; ++c) *reinterpret_cast<uint4*>(z + tc::sw128_off(t, 8 * c, kQ)) = raw[c];
-                fence_proxy_async_smem();
-                mbar_arrive(&scaled[k % kScanBufs]);
-            }
-        }
-    } else if (warp == 8) {
-        // ------------------------------------------------------------------------ issue
-        if (lane == 0) {
-            for (int k = 0; k < nk; ++k) {
-                const int buf = k % kScanBufs, use = k / kScanBufs;
-                ok = ok && mbar_wait(&scaled[buf], (uint32_t)(use & 1), a.hdr, 741);
-                if (k >= kScanBufs) ok = ok && mbar_wait(&bfree[buf], (uint32_t)((use - 1) & 1), a.hdr, 742);
-                tc::fence_after_sync();
-                decf[k % kDecRing] = decp[k % kDecRing];
-                if (ok)
-                    tc::mma_tiles(tmem + 64 * buf, smem_u32(stage(k)), 1, kQ, smem_u32(stage(k) + SM::kRt), 1, kQ,
-                                  kKD, kP, kQ, 0);
-                tc::commit(&prod[buf]);
-                mbar_arrive(&prod[buf]);
-            }
-        }
-    } else if (warp == 10) {
-        // ------------------------------------------------------------------------- load
-        if (lane == 0) {
-            for (int k = 0; k < nk && k < NS; ++k) load(k);
-            for (int k = 0; k + NS < nk; ++k) {  // the product of chunk k has read its stage
-                ok = ok && mbar_wait(&prod[k % kScanBufs], (uint32_t)((k / kScanBufs) & 1), a.hdr, 743);
-                if (ok) load(k + NS);
-            }
-        }
-    } else if (warp == 11) {
-        // --------------------------------------------------------------------------- dt
-        // TMA: one box of 8 heads x 128 steps per chunk.  Loads: one prep group (kScanPrepGroup
-        // chunks) per batch of loads: an arrival waits for every load of the thread in flight, so
-        // the loads of a group are all issued before the first one.
-        constexpr int NG = kScanPrepGroup;
-        if (dt_tma) {
-            if (lane == 0)
-                for (int k = 0; k < nk; ++k) {
-                    const int slot = k % kDtRing;
-                    if (k >= kDtRing)
-                        ok = ok && mbar_wait(&dtempty[slot], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
-                    mbar_arrive_expect_tx(&dtfull[slot], (uint32_t)(kQ * 16));
-                    tma_load_3d(dtb + (size_t)slot * kQ * 8, &mDt, &dtfull[slot], h & ~7, chunk_of(k) * kQ, b);
-                }
-            // the prep group's chunks past the last product: nothing to load
-            if (lane == 0)
-                for (int k = nk; k % NG != 0; ++k) {
-                    const int slot = k % kDtRing;
-                    if (k >= kDtRing)
-                        ok = ok && mbar_wait(&dtempty[slot], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
-                    mbar_arrive(&dtfull[slot]);
-                }
-        } else
-        for (int k0 = 0; k0 < nk; k0 += NG) {
-            if (k0 >= kDtRing) {
-#pragma unroll
-                for (int j = 0; j < NG; ++j) {
-                    const int k = k0 + j;
-                    ok = ok && mbar_wait(&dtempty[k % kDtRing], (uint32_t)(((k / kDtRing) - 1) & 1), a.hdr, 746);
-                }
-            }
-            float v[NG][kQ / 32];
-#pragma unroll
-            for (int j = 0; j < NG; ++j)
-#pragma unroll
-                for (int i = 0; i < kQ / 32; ++i) {
-                    const int k = k0 + j, tt = chunk_of(k) * kQ + lane + 32 * i;
-                    v[j][i] = k < nk && tt < a.L ? __bfloat162float(a.dt[((size_t)b * a.L + tt) * a.H + h]) : 0.0f;
-                }
-#pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                const int slot = (k0 + j) % kDtRing;
-#pragma unroll
-                for (int i = 0; i < kQ / 32; ++i)
-                    dtb[(slot * kQ + lane + 32 * i) * 8 + hx] = __float2bfloat16_rn(v[j][i]);
-                mbar_arrive(&dtfull[slot]);
-            }
-        }
-    } else if (warp == 9) {
-        // --------------------------------------------------------------- zero, publish
-        // backward, several head blocks per group: the dB, dC rows [B, L, G, N] of chunk c, group
-        // g are zeroed by head g HpG + (c mod HpG) of the batch row and flagged (zready), for the
-        // gradient kernel's reduction-adds
-        if (zready) {
-            pdl_wait();  // the previous kernel of the stream may still read dB, dC
-            const int hg = h - g * a.HpG;
-            for (int c = hg; c < a.nchunk; c += a.HpG) {
-                const int rows = min(kQ, a.L - c * kQ);
-                for (int r = 0; r < rows; ++r) {
-                    const size_t off = (((size_t)b * a.L + c * kQ + r) * a.G + g) * kKD + 4 * lane;
-                    *reinterpret_cast<float4*>(zero0 + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    *reinterpret_cast<float4*>(zero1 + off) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                }
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release(&zready[((size_t)c * a.B + b) * a.G + g], 1u);
-            }
-        }
-        // the fold's puts in order (put q writes slot q forward, slot nchunk - 1 - q backward)
-        if (ready && lane == 0) {
-            int next = 0;
-            unsigned long long t0 = global_ns();
-            while (next < a.nchunk) {
-                const int done = ld_acquire_cta(pubdone);
-                if (done >= next) {
-                    for (; next <= done; ++next) {
-                        const int slot = dir > 0 ? next : a.nchunk - 1 - next;
-                        st_release(&ready[((size_t)slot * a.B + b) * a.H + h], 1u);
-                    }
-                    t0 = global_ns();
-                    continue;
-                }
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    record_error(a.hdr, LR_ERR_TIMEOUT, 747);
-                    break;
-                }
-                __nanosleep(100);
-            }
-        }
-    } else {
-        // ------------------------------------------------------------------------- fold
-        const int n = tid - 128, fl = n == 0;  // fl: the thread that issues the copies
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        // fl: the last two puts whose copies were issued (pub1 the latest); a put is handed to the
-        // publishing warp once the copies of the put after it have been issued, by which time its
-        // own have landed
-        int nput = 0, pub1 = -1, pub2 = -1;
-        auto publish = [&](int q) {  // puts 0 .. q have landed
-            fence_proxy_async_global();
-            st_release_cta(pubdone, q);
-        };
-        float S[kP];
-#pragma unroll
-        for (int i = 0; i < kP; ++i) S[i] = 0.0f;
-        pdl_wait();  // the previous kernel of the stream may still read the slots
-        // S into slot c through the staging buffers (free: the copies of the previous slot have
-        // read them before the first barrier)
-        auto put = [&](int c) {
-            if (fl) {
-                if (ready && pub2 >= 0) {
-                    bulk_wait_all_but_1();
-                    publish(pub2);
-                }
-                bulk_wait_read_all();
-            }
-            wg_sync(1);
-            if constexpr (F32) {
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    char* box = sm + SM::kF32 + j * (kKD * 128);  // columns 32 j .. 32 j + 31
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        *reinterpret_cast<float4*>(box + n * 128 + ((i ^ (n & 7)) << 4)) =
-                            make_float4(S[32 * j + 4 * i], S[32 * j + 4 * i + 1], S[32 * j + 4 * i + 2],
-                                        S[32 * j + 4 * i + 3]);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                *reinterpret_cast<uint4*>(sm + SM::kBf + tc::sw128_off(n, 8 * i, kKD)) = pack_bf16x8(S + 8 * i);
-            fence_proxy_async_smem();
-            wg_sync(1);
-            if (fl) {
-                if constexpr (F32) {
-                    tma_store_4d(&mS, sm + SM::kF32, 0, 0, bh, c);
-                    tma_store_4d(&mS, sm + SM::kF32 + kKD * 128, 32, 0, bh, c);
-                }
-                bulk_store(tiles + ((size_t)c * BH + bh) * kTileBytes, sm + SM::kBf, kTileBytes);
-                bulk_commit();
-            }
-            pub2 = pub1;
-            pub1 = nput++;
-        };
-        put(dir > 0 ? 0 : a.nchunk - 1);
-        for (int k = 0; k < nk; ++k) {
-            const int buf = k % kScanBufs;
-            ok = ok && mbar_wait(&prod[buf], (uint32_t)((k / kScanBufs) & 1), a.hdr, 744);
-            tc::fence_after_sync();
-            float v[kP];
-#pragma unroll
-            for (int j = 0; j < kP; j += 16) tc::ld16(tmem + 64 * buf + j + lane_off, v + j);
-            tc::wait_ld();
-            tc::fence_before_sync();
-            mbar_arrive(&bfree[buf]);
-            const float d = decf[k % kDecRing];
-#pragma unroll
-            for (int i = 0; i < kP; ++i) S[i] = fmaf(d, S[i], v[i]);
-            put(chunk_of(k) + dir);
-        }
-        if (fl) {
-            bulk_wait_all();
-            if (ready) publish(pub1);
-        }
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 8) {
-        tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 64 * kScanBufs);
-    }
-}
 
 // ---------------------------------------------------------------------------------- outputs
 constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernels)
@@ -742,22 +349,6 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     }
 }
 
-// TMA map of the f32 state slots [nslot][B*H][N][P], boxes of 32 columns x 128 rows (128-byte
-// swizzle), written by the scan kernel.
-bool map_states(CUtensorMap* m, void* base, int64_t BH, int64_t nslot) {
-    uint64_t dims[4] = {(uint64_t)kP, (uint64_t)kKD, (uint64_t)BH, (uint64_t)nslot};
-    uint64_t str[3] = {kP * 4, (uint64_t)kKD * kP * 4, (uint64_t)BH * kKD * kP * 4};
-    uint32_t box[4] = {32, (uint32_t)kKD, 1, 1};
-    return make_tmap(m, base, 4, 4, dims, str, box, true);
-}
-
-// TMA map of the raw dt [B, L, H] bf16 with boxes of 8 heads x 128 steps (16-byte rows): only
-// when a row of H heads spans a multiple of 16 bytes (H a multiple of 8); false otherwise.
-bool map_dt(CUtensorMap* m, const lr_desc& d, const void* dt) {
-    if (d.H % 8 != 0) return false;
-    return make_tmap_3d(m, dt, 2, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.B, 8, (uint32_t)kQ);
-}
-
 // The general kernel variant: a discretisation other than ZOH, or the softplus front-end.
 bool general_variant(const lr_desc& d) {
     return d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS);
@@ -840,7 +431,7 @@ int out_heads_per_cta(const lr_desc& d, int nchunk) {
 
 // =========================================================================================
 // Backward.  With G_c the adjoint of the state leaving chunk c (G_{last} = 0):
-//   G_{c-1} = e^{l_Q, c} G_c + U_c,  U_c = C^T diag(E) dy_h      (ssd_scan_kernel, dir < 0)
+//   G_{c-1} = e^{l_Q, c} G_c + U_c,  U_c = C^T diag(E) dy_h      (chunk_scan_kernel, dir < 0)
 // and per (chunk, head), with S2 = dy x^T, Pd = S2 o Lmask, P = M o Lmask, R = Pd o M:
 //   dC += Pd B + diag(E) dy S_in^T            dB += Pd^T C + diag(w) x G^T   (summed over heads)
 //   dx  = P^T dy + diag(w) B G + D dy
@@ -1411,15 +1002,15 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     if (!ok) return LR_ERR_INVALID_ARG;
     const bool gen = general_variant(d);
     using ScanF = ScanSmem<3, true>;
-    auto scan = gen ? ssd_scan_kernel<3, true, true> : ssd_scan_kernel<3, true, false>;
+    auto scan = gen ? chunk_scan_kernel<3, true, kScanSsdGen> : chunk_scan_kernel<3, true, kScanSsd>;
     cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
     note_launch("ssd_state_scan");
     CUtensorMap mS;
-    if (!map_states(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk)) return LR_ERR_INVALID_ARG;
+    if (!map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk, kP)) return LR_ERR_INVALID_ARG;
     CUtensorMap mDt;
-    const int dt_tma = map_dt(&mDt, d, in.delta) ? 1 : 0;
+    const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
     if (!dt_tma) mDt = mB;  // not read
-    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, mDt, dt_tma, a, stiles,
+    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, mDt, dt_tma, scan_args(a), stiles,
                    +1, ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr) != cudaSuccess)
         return LR_ERR_CUDA;
     {
@@ -1466,14 +1057,15 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.zready = (const unsigned int*)(ws + w.dbc);
     {
         using ScanB = ScanSmem<4, false>;
-        auto scan = general_variant(d) ? ssd_scan_kernel<4, false, true> : ssd_scan_kernel<4, false, false>;
+        auto scan = general_variant(d) ? chunk_scan_kernel<4, false, kScanSsdGen>
+                                       : chunk_scan_kernel<4, false, kScanSsd>;
         cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
         note_launch("ssd_state_scan");
         // no f32 states in this direction (the map argument is unused)
         CUtensorMap mDt;
-        const int dt_tma = map_dt(&mDt, d, in.delta) ? 1 : 0;
+        const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
         if (!dt_tma) mDt = mC;  // not read
-        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, mDt, dt_tma, a,
+        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, mDt, dt_tma, scan_args(a),
                        ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
                        ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;

@@ -239,12 +239,9 @@ def kernel_cost(w, name, pas, pass_bytes):
         tile = B * H * K * V * 2
         hc = nc * B * H
         prod = 2 * Q * Q * max(K, V)       # one 128 x 128 x 128 product
-        if name == "gla_chunk_state":
-            return tk + tv + g + (nc - 1) * slot, (nc - 1) * B * H * 2 * K * V * Q
-        if name == "gla_state_pass":
-            if pas == "fwd":
-                return (nc - 1) * slot + nc * slot + nc * tile, 0
-            return (nc - 1) * slot + nc * tile, 0
+        if name == "gla_state_scan":       # k (q), v (dO), g in; every slot out (f32 + tile; tile)
+            out = nc * (slot + tile) if pas == "fwd" else nc * tile
+            return tk + tv + g + out, (nc - 1) * B * H * 2 * K * V * Q
         if name == "gla_chunk_out":
             return 2 * tk + 2 * tv + g + nc * tile, hc * 3 * prod
         if name == "gla_chunk_grad":

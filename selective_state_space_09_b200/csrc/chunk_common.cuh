@@ -1,6 +1,7 @@
-// chunk_common.cuh -- pieces shared by the chunked-matmul kernels (chunk.cu, ssd.cu): the chunk
-// geometry, the base-2 exponential, CTA-wide prefix sums, row scaling of 128-byte-swizzled tiles,
-// vector reductions to global memory, and the TMA map of a [B, L, X, W] bf16 tensor.
+// chunk_common.cuh -- pieces shared by the chunked-matmul kernels (ssd.cu, gla.cu, chunk_scan.cuh):
+// the chunk geometry, the base-2 exponential, CTA-wide prefix sums, row scaling of
+// 128-byte-swizzled tiles, vector reductions to global memory, and the TMA map of a [B, L, X, W]
+// bf16 tensor.
 #pragma once
 
 #include "common.cuh"
@@ -169,63 +170,6 @@ inline bool map4(CUtensorMap* m, const void* p, uint64_t W, uint64_t X, uint64_t
     uint64_t str[3] = {W * 2, X * W * 2, L * X * W * 2};
     uint32_t box[4] = {64, 1, (uint32_t)kQ, 1};
     return make_tmap(m, p, 2, 4, dims, str, box, swz);
-}
-
-// ---------------------------------------------------------------------------- state passing
-// One thread per (b h, four consecutive state elements (n, p .. p+3)) of the f32 slots of `buf`
-// ([nchunk][B*H][N*VD/4] float4; N = 128 state rows, VD value columns), walking the chunks:
-//   dir > 0: slot 0 = 0; slot c = decay_{c-1} slot_{c-1} + slot_c (c = 1 .. nchunk-1), in place;
-//            every slot is also written as bf16 into `tiles` ([nchunk][B*H] tiles, tensor-core
-//            order), the B operand of C S_in in the output and gradient kernels;
-//   dir < 0: G_{nchunk-1} = 0; G_c = decay_{c+1} G_{c+1} + slot_c (slot c holds U_{c+1}), written
-//            only as bf16 tiles.
-// Loads of eight slots are issued ahead of their dependent updates.
-template <int VD>
-__global__ void __launch_bounds__(256)
-state_pass_kernel(float4* buf, char* tiles, const float* __restrict__ decay, int BH, int n4, int nchunk, int dir,
-                  float4* zero0, float4* zero1, size_t nzero4) {
-    constexpr size_t kTile = (size_t)kKD * VD * 2;
-    pdl_launch_dependents();
-    pdl_wait();
-    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    // zero0 / zero1 (the backward's dB, dC when several CTAs add into them): nzero4 float4 each
-    for (size_t z = e; z < nzero4; z += (size_t)gridDim.x * blockDim.x) {
-        zero0[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        zero1[z] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
-    if (e >= (size_t)BH * n4) return;
-    const size_t stride = (size_t)BH * n4;
-    const int bh = (int)(e / n4), q = (int)(e % n4);
-    const float* dec = decay + (size_t)bh * nchunk;
-    const uint32_t toff = tc::sw128_off(q / (VD / 4), (q % (VD / 4)) * 4, kKD);
-    auto put = [&](int c, float4 v) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-        uint2 u = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-        *reinterpret_cast<uint2*>(tiles + ((size_t)c * BH + bh) * kTile + toff) = u;
-    };
-    float4* p = buf + e;
-    float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const int first = dir > 0 ? 0 : nchunk - 1;
-    if (dir > 0) p[(size_t)first * stride] = s;
-    put(first, s);
-    for (int k0 = 1; k0 < nchunk; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
-            if (k0 + k < nchunk) v[k] = __ldcg(p + (size_t)c * stride);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            if (k0 + k < nchunk) {
-                const int c = dir > 0 ? k0 + k : nchunk - 1 - (k0 + k);
-                const float d = dec[c - dir];
-                s = make_float4(fmaf(d, s.x, v[k].x), fmaf(d, s.y, v[k].y), fmaf(d, s.z, v[k].z), fmaf(d, s.w, v[k].w));
-                if (dir > 0) p[(size_t)c * stride] = s;
-                put(c, s);
-            }
-        }
-    }
 }
 
 }  // namespace chunkc

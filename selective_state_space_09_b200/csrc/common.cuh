@@ -260,6 +260,13 @@ __device__ __forceinline__ bool wait_flags(const unsigned int* f, int n, WsHeade
     return false;
 }
 
+// The same with one acquire load per flag (no fence: cheaper for a few flags).
+__device__ __forceinline__ bool wait_flags_acquire(const unsigned int* f, int n, WsHeader* hdr, int info) {
+    for (int k = 0; k < n; ++k)
+        if (wait_flag(f + k, hdr, info) == kFlagNone) return false;
+    return true;
+}
+
 // Dynamic tile ticket: tiles are numbered in the order CTAs start, so that every tile a CTA may
 // wait on belongs to a CTA that has already started.
 __device__ __forceinline__ unsigned int take_ticket(WsHeader* hdr, int which) {

@@ -9,11 +9,12 @@
 //   S_out = e^{l_Q} S_in + Sl,  Sl = K^T diag(w) V
 //   O     = (M o Lmask) V + diag(E) Q S_in
 // (the chunked evaluation of the K-Search / mlx-mamba post, paragraph after Table 1, with a
-// scalar decay and a matrix state).  Forward = gla_state_kernel (Sl of every chunk but the last),
-// state_pass_kernel (entering states = checkpoints, with bf16 tile copies), gla_out_kernel.
-// Backward = gla_state_kernel (U = Q^T diag(E) dO), state_pass_kernel (adjoint states G),
-// gla_grad_kernel.
-#include "chunk_common.cuh"
+// scalar decay and a matrix state).  Forward = chunk_scan_kernel (chunk_scan.cuh: one CTA per (row,
+// head, 64 value columns) folding Sl = K^T diag(w) V into the entering states, checkpoints and
+// bf16 tiles) and gla_out_kernel beside it.  Backward = chunk_scan_kernel in reverse (adjoint
+// states G from U = Q^T diag(E) dO) and gla_grad_kernel beside it.  The chunk kernels wait for the
+// scan's per-slot flags, not for the whole scan.
+#include "chunk_scan.cuh"
 
 namespace lrs {
 using namespace chunkc;
@@ -22,7 +23,6 @@ namespace {
 struct GlaArgs {
     int B, L, H, nchunk;
     const __nv_bfloat16* g;   // [B, L, H] gate in (0, 1)
-    float* decay;             // [B][H][nchunk] e^{l_Q}
     WsHeader* hdr;
 };
 
@@ -30,109 +30,6 @@ struct GlaArgs {
 __device__ __forceinline__ float gla_lam(const GlaArgs& a, int b, int h, int t) {
     if (t >= a.L) return 0.0f;
     return __logf(__bfloat162float(a.g[((size_t)b * a.L + t) * a.H + h]));
-}
-
-// ------------------------------------------------------------------------- state increments
-template <int VD>
-struct GStateSmem {
-    static constexpr size_t kR = 0;                       // 128 x 128 bf16 (k or q)
-    static constexpr size_t kZ = kR + kQ * kKD * 2;       // 128 x VD bf16 (v or dO)
-    static constexpr size_t kTmp = kZ + kQ * VD * 2;      // scan scratch
-    static constexpr size_t kBar = kTmp + 64;
-    static constexpr size_t kTmem = kBar + 64;
-    static constexpr size_t kEnd = kTmem + 64;
-    static constexpr size_t kAlloc = kEnd + 1024;
-    // the f32 result (128 x VD x 4 bytes) is staged over R and Z once the product is done
-    static_assert(kQ * VD * 4 <= kTmp, "staging fits over the operand tiles");
-};
-
-// One CTA per (chunk, batch row, head):
-//   dir > 0: Sl_c = K^T diag(w) V for chunk c = 0 .. nchunk-2, into slot c + 1 of the state map;
-//   dir < 0: U_c = Q^T diag(E) dO for chunk c = 1 .. nchunk-1, into slot c - 1.
-// decay[(b H + h) nchunk + c] = e^{l_Q}.
-template <int VD>
-__global__ void __launch_bounds__(kThreads, 3)
-gla_state_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mZ,
-                 const __grid_constant__ CUtensorMap mOut, GlaArgs a, int dir) {
-    using SM = GStateSmem<VD>;
-    char* sm = smem_base1024();
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::kBar);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmem);
-    float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    int idx = blockIdx.x;
-    const int h = idx % a.H;
-    idx /= a.H;
-    const int b = idx % a.B;
-    const int c = idx / a.B + (dir > 0 ? 0 : 1);
-    const int slot = dir > 0 ? c + 1 : c - 1;
-    const int t0 = c * kQ;
-    pdl_launch_dependents();
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        fence_barrier_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 128);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(kQ * kKD * 2 + kQ * VD * 2));
-        for (int j = 0; j < kKD / 64; ++j) tma_load_4d(sm + SM::kR + j * kQ * 128, &mR, &bar[0], 64 * j, h, t0, b);
-        for (int j = 0; j < VD / 64; ++j) tma_load_4d(sm + SM::kZ + j * kQ * 128, &mZ, &bar[0], 64 * j, h, t0, b);
-    }
-    const float lt = cta_inclusive_sum(gla_lam(a, b, h, t0 + tid), tmp);
-    if (tid == kQ - 1) tmp[8] = lt;
-    __syncthreads();
-    const float lQ2 = tmp[8] * kLog2e, lt2 = lt * kLog2e;
-    const float f = dir > 0 ? ex2(lQ2 - lt2) : ex2(lt2);
-    pdl_wait();  // the previous kernel of the stream may still read what this one writes
-    if (tid == 0) a.decay[((size_t)b * a.H + h) * a.nchunk + c] = ex2(lQ2);
-    bool ok = mbar_wait(&bar[0], 0, a.hdr, 800);
-    scale_row(sm + SM::kZ, tid, VD, kQ, f);
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && ok) {  // R^T (f o Z): M = 128 state rows, N = VD, K = 128 steps
-        tc::fence_after_sync();
-        tc::mma_tiles(tmem, smem_u32(sm + SM::kR), 1, kQ, smem_u32(sm + SM::kZ), 1, kQ, kKD, VD, kQ, 0);
-        tc::commit(&bar[1]);
-    }
-    __syncwarp();
-    ok = ok && mbar_wait(&bar[1], 0, a.hdr, 801);
-    tc::fence_after_sync();
-    // f32 result through shared memory in 32-column, 128-byte-swizzled boxes
-#pragma unroll
-    for (int v0 = 0; v0 < VD; v0 += 16) {
-        float v[16];
-        tc::ld16(tmem + lane_off + v0, v);
-        tc::wait_ld();
-        char* box = sm + (v0 >> 5) * (kKD * 128);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int chunk = ((v0 & 31) >> 2) + k;
-            *reinterpret_cast<float4*>(box + tid * 128 + ((chunk ^ (tid & 7)) << 4)) =
-                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-        }
-    }
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && ok) {
-        const int bh = b * a.H + h;
-        for (int j = 0; j < VD / 32; ++j) tma_store_4d(&mOut, sm + j * (kKD * 128), 32 * j, 0, bh, slot);
-        bulk_commit();
-        bulk_wait_read_all();
-    }
-    __syncthreads();
-    if (warp == 0) {
-        tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 128);
-    }
 }
 
 // ---------------------------------------------------------------------------------- outputs
@@ -158,7 +55,7 @@ template <int VD>
 __global__ void __launch_bounds__(kThreads, 2)
 gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mO, GlaArgs a,
-               const char* stiles) {
+               const char* stiles, const unsigned int* ready, int halves) {
     using SM = GOutSmem<VD>;
     constexpr uint32_t kColO = 64;
     char* sm = smem_base1024();
@@ -203,7 +100,6 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     const float l0 = l2s[32 * warp];
     for (int s = lane; s < 32 * warp; s += 32) cfw[s] = ex2(l0 - l2s[s]);
     __syncwarp();
-    pdl_wait();  // the S_in tiles come from the previous kernel
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 810);
     if (tid == 0 && ok) {
         tc::fence_after_sync();
@@ -212,6 +108,14 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     }
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 811);
     tc::fence_after_sync();
+    // the S_in tile of slot c: written by the scan kernel, which flags each 64-column half once its
+    // copies have landed; polled only now (the flag loads' latency hides behind the loads and
+    // Q K^T above), and for slot 0, the zero state, too: the scan flags it only after the kernels
+    // before it are done, and no global write of this kernel comes before this
+    if (tid == 0) {
+        ok = wait_flags_acquire(&ready[(((size_t)c * a.B + b) * a.H + h) * halves], halves, a.hdr, 813) && ok;
+        fence_proxy_async_global();
+    }
     if (tid == 0 && ok && has_in) {  // k is consumed: its slot takes the S_in tile
         mbar_arrive_expect_tx(&bar[3], (uint32_t)(kKD * VD * 2));
         bulk_load(sm + SM::kKt, stiles + (((size_t)c * a.B + b) * a.H + h) * (size_t)(kKD * VD * 2),
@@ -319,6 +223,7 @@ struct GGradSmem {
     static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
     static constexpr size_t kBar = kTmp + 256;             // 0 loads, 1 A, 2 B, 3 S_in/G, 4 C, 5 D
     static constexpr size_t kTmem = kBar + 64;
+    static constexpr size_t kTicket = kTmem + 8;
     static constexpr size_t kEnd = kTmem + 64;
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kAlloc <= 232448, "gradient CTA exceeds the shared memory of one CTA");
@@ -328,6 +233,8 @@ struct GlaGradArgs {
     GlaArgs a;
     const char* stiles;      // [nchunk][B][H] bf16 tiles of the entering states
     const char* gtiles;      // [nchunk][B][H] bf16 tiles of the adjoint states
+    const unsigned int* gready;  // [nchunk][B][H][halves]: G tile half written (by the scan kernel)
+    int halves;
     __nv_bfloat16* dq;       // [B, L, H, K]
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;       // [B, L, H, V]
@@ -362,15 +269,10 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
     const int row = tid & 127;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    int idx = blockIdx.x;
-    const int h = idx % a.H;
-    idx /= a.H;
-    const int b = idx % a.B;
-    const int c = idx / a.B;
-    const int t0 = c * kQ;
-    const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
-    const bool vrow = t0 + row < a.L;
-    const size_t tok = ((size_t)b * a.L + (vrow ? t0 + row : 0)) * a.H + h;  // token index of this row
+    // tile from a ticket taken at the start, chunks from the last (whose adjoint the scan kernel
+    // writes first)
+    unsigned int* ticket = reinterpret_cast<unsigned int*>(sm + SM::kTicket);
+    if (tid == 0) *ticket = take_ticket(a.hdr, 0);
     pdl_launch_dependents();
 
     if (tid == 0) {
@@ -383,6 +285,15 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    int idx = (int)*ticket;
+    const int h = idx % a.H;
+    idx /= a.H;
+    const int b = idx % a.B;
+    const int c = a.nchunk - 1 - idx / a.B;
+    const int t0 = c * kQ;
+    const bool has_in = c > 0, has_out = c + 1 < a.nchunk;
+    const bool vrow = t0 + row < a.L;
+    const size_t tok = ((size_t)b * a.L + (vrow ? t0 + row : 0)) * a.H + h;  // token index of this row
     if (tid == 0) {
         mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * kQ * kKD * 2 + 2 * kQ * VD * 2));
         for (int j = 0; j < kKD / 64; ++j) {
@@ -402,7 +313,6 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         const int w = k >> 7, s = k & 127;
         if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]);
     }
-    pdl_wait();  // the G tiles come from the previous kernel
     bool ok = mbar_wait(&bar[0], 0, a.hdr, 820);
     __syncthreads();
     if (tid == 0 && ok) {  // phase A
@@ -495,6 +405,11 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 822);
     tc::fence_after_sync();
     if (tid == 0) {  // P, Pd are consumed: their slots take S_in and G
+        // the G tile of slot c: written by the scan kernel, which flags each 64-column half once
+        // its copies have landed (the last chunk's zero adjoint too, flagged only after the
+        // kernels before the scan are done); no global write of this kernel comes before this
+        ok = wait_flags_acquire(&ga.gready[(((size_t)c * a.B + b) * a.H + h) * ga.halves], ga.halves, a.hdr, 828) && ok;
+        fence_proxy_async_global();
         const size_t tile = (((size_t)c * a.B + b) * a.H + h) * (size_t)(kKD * VD * 2);
         const uint32_t bytes = (has_in ? kKD * VD * 2 : 0u) + (has_out ? kKD * VD * 2 : 0u);
         if (bytes == 0) {
@@ -668,79 +583,95 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     }
 }
 
-// TMA map of f32 state slots [nslot][B*H][128][VD], boxes of 32 columns x 128 rows (128-byte swizzle)
-bool map_states_vd(CUtensorMap* m, void* base, int64_t BH, int64_t nslot, int VD) {
-    uint64_t dims[4] = {(uint64_t)VD, (uint64_t)kKD, (uint64_t)BH, (uint64_t)nslot};
-    uint64_t str[3] = {(uint64_t)VD * 4, (uint64_t)kKD * VD * 4, (uint64_t)BH * kKD * VD * 4};
-    uint32_t box[4] = {32, (uint32_t)kKD, 1, 1};
-    return make_tmap(m, base, 4, 4, dims, str, box, true);
-}
-
 struct GlaWs {
-    size_t decay, U, gtiles, end;
+    size_t ready, flags_end, gtiles, end;  // the slot flags first (reset every call)
 };
 GlaWs gla_plan(const lr_desc& d, bool bwd) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     const size_t tiles = (size_t)d.B * d.H * nchunk;
     WsCursor cur;
     GlaWs w{};
-    w.decay = cur.take(sizeof(float) * tiles);
-    if (bwd) {
-        w.U = cur.take(sizeof(float) * tiles * kKD * d.P);
-        w.gtiles = cur.take((size_t)2 * tiles * kKD * d.P);
-    }
+    w.ready = cur.take(sizeof(unsigned int) * tiles * (size_t)(d.P / kScanP));
+    w.flags_end = cur.off;
+    if (bwd) w.gtiles = cur.take((size_t)2 * tiles * kKD * d.P);
     w.end = cur.off;
     return w;
 }
 
-GlaArgs gla_args(const lr_desc& d, const lr_inputs& in, char* ws, float* decay) {
+GlaArgs gla_args(const lr_desc& d, const lr_inputs& in, char* ws) {
     GlaArgs a{};
     a.B = (int)d.B;
     a.L = (int)d.L;
     a.H = (int)d.H;
     a.nchunk = (int)((d.L + kQ - 1) / kQ);
     a.g = (const __nv_bfloat16*)in.g;
-    a.decay = decay;
     a.hdr = (WsHeader*)ws;
     return a;
+}
+
+// The scan kernel's view of the problem (chunk_scan.cuh): per-head rows (G = H), decay log g.
+ScanArgs scan_args(const GlaArgs& a, int VD) {
+    ScanArgs s{};
+    s.B = a.B;
+    s.L = a.L;
+    s.H = a.H;
+    s.G = a.H;
+    s.HpG = 1;
+    s.nchunk = a.nchunk;
+    s.halves = VD / kScanP;
+    s.dt = a.g;
+    s.hdr = a.hdr;
+    return s;
+}
+
+// The chunk-state scan over (row, head, 64 value columns): dir > 0 folds K^T diag(w) V into the
+// entering states (f32 checkpoint slots and bf16 tiles); dir < 0 folds Q^T diag(E) dO into the
+// adjoint states (bf16 tiles).  Each slot half is flagged in `ready` once written.
+template <int VD>
+lr_status gla_scan(const lr_desc& d, const GlaArgs& a, const CUtensorMap& mR, const CUtensorMap& mZ, void* ckpt,
+                   char* tiles, int dir, unsigned int* ready, cudaStream_t st) {
+    CUtensorMap mS, mDt;
+    if (dir > 0 && !map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk, VD)) return LR_ERR_INVALID_ARG;
+    if (dir < 0) mS = mR;  // no f32 states in this direction
+    const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, a.g) ? 1 : 0;
+    if (!dt_tma) mDt = mR;  // not read
+    const ScanArgs sa = scan_args(a, VD);
+    const dim3 grid((unsigned)(a.B * a.H * sa.halves));
+    note_launch("gla_state_scan");
+    cudaError_t e;
+    if (dir > 0) {
+        using SF = ScanSmem<3, true>;
+        cudaFuncSetAttribute(chunk_scan_kernel<3, true, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SF::kAlloc);
+        e = launch_pdl(chunk_scan_kernel<3, true, kScanGla>, grid, dim3(kScanThreads), SF::kAlloc, st, mR, mZ, mS,
+                       mDt, dt_tma, sa, tiles, +1, ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr);
+    } else {
+        using SB = ScanSmem<4, false>;
+        cudaFuncSetAttribute(chunk_scan_kernel<4, false, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SB::kAlloc);
+        e = launch_pdl(chunk_scan_kernel<4, false, kScanGla>, grid, dim3(kScanThreads), SB::kAlloc, st, mR, mZ, mS,
+                       mDt, dt_tma, sa, tiles, -1, ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr);
+    }
+    if (e != cudaSuccess) return LR_ERR_CUDA;
+    return check_launch();
 }
 
 template <int VD>
 lr_status gla_fwd_t(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
     const GlaWs w = gla_plan(d, false);
-    GlaArgs a = gla_args(d, in, ws, (float*)(ws + w.decay));
+    GlaArgs a = gla_args(d, in, ws);
     CUtensorMap mQ, mK, mV, mO;
     if (!(map4(&mQ, in.q, kKD, d.H, d.L, d.B, true) && map4(&mK, in.k, kKD, d.H, d.L, d.B, true) &&
           map4(&mV, in.v, VD, d.H, d.L, d.B, true) && map4(&mO, y, VD, d.H, d.L, d.B, true)))
         return LR_ERR_INVALID_ARG;
     char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float);
-    if (a.nchunk > 1) {
-        CUtensorMap mS;
-        if (!map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk, VD)) return LR_ERR_INVALID_ARG;
-        cudaFuncSetAttribute(gla_state_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)GStateSmem<VD>::kAlloc);
-        note_launch("gla_chunk_state");
-        if (launch_pdl(gla_state_kernel<VD>, dim3((a.nchunk - 1) * a.B * a.H), dim3(kThreads), GStateSmem<VD>::kAlloc,
-                       st, mK, mV, mS, a, +1) != cudaSuccess)
-            return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
-    {
-        const int n4 = kKD * VD / 4;
-        const size_t total = (size_t)a.B * a.H * n4;
-        note_launch("gla_state_pass");
-        if (launch_pdl(state_pass_kernel<VD>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st, (float4*)ckpt,
-                       stiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, +1, (float4*)nullptr, (float4*)nullptr,
-                       (size_t)0) != cudaSuccess)
-            return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
+    unsigned int* ready = (unsigned int*)(ws + w.ready);
+    lr_status s = gla_scan<VD>(d, a, mK, mV, ckpt, stiles, +1, ready, st);
+    if (s != LR_OK) return s;
     cudaFuncSetAttribute(gla_out_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GOutSmem<VD>::kAlloc);
     note_launch("gla_chunk_out");
     if (launch_pdl(gla_out_kernel<VD>, dim3(a.nchunk * a.B * a.H), dim3(kThreads), GOutSmem<VD>::kAlloc, st, mQ, mK,
-                   mV, mO, a, (const char*)stiles) != cudaSuccess)
+                   mV, mO, a, (const char*)stiles, (const unsigned int*)ready, VD / kScanP) != cudaSuccess)
         return LR_ERR_CUDA;
     return check_launch();
 }
@@ -750,10 +681,12 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
                     char* ws, cudaStream_t st) {
     const GlaWs w = gla_plan(d, true);
     GlaGradArgs ga{};
-    ga.a = gla_args(d, in, ws, (float*)(ws + w.decay));
+    ga.a = gla_args(d, in, ws);
     const GlaArgs& a = ga.a;
     ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float);
     ga.gtiles = ws + w.gtiles;
+    ga.gready = (const unsigned int*)(ws + w.ready);
+    ga.halves = VD / kScanP;
     ga.dq = (__nv_bfloat16*)gr.dq;
     ga.dk = (__nv_bfloat16*)gr.dk;
     ga.dv = (__nv_bfloat16*)gr.dv;
@@ -762,30 +695,8 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
     if (!(map4(&mQ, in.q, kKD, d.H, d.L, d.B, true) && map4(&mK, in.k, kKD, d.H, d.L, d.B, true) &&
           map4(&mV, in.v, VD, d.H, d.L, d.B, true) && map4(&mO, dy, VD, d.H, d.L, d.B, true)))
         return LR_ERR_INVALID_ARG;
-    float* Ubuf = (float*)(ws + w.U);
-    if (a.nchunk > 1) {
-        CUtensorMap mU;
-        if (!map_states_vd(&mU, Ubuf, (int64_t)a.B * a.H, a.nchunk, VD)) return LR_ERR_INVALID_ARG;
-        cudaFuncSetAttribute(gla_state_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)GStateSmem<VD>::kAlloc);
-        note_launch("gla_chunk_state");
-        if (launch_pdl(gla_state_kernel<VD>, dim3((a.nchunk - 1) * a.B * a.H), dim3(kThreads), GStateSmem<VD>::kAlloc,
-                       st, mQ, mO, mU, a, -1) != cudaSuccess)
-            return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
-    {
-        const int n4 = kKD * VD / 4;
-        const size_t total = (size_t)a.B * a.H * n4;
-        note_launch("gla_state_pass");
-        if (launch_pdl(state_pass_kernel<VD>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st, (float4*)Ubuf,
-                       ws + w.gtiles, (const float*)a.decay, a.B * a.H, n4, a.nchunk, -1, (float4*)nullptr,
-                       (float4*)nullptr, (size_t)0) != cudaSuccess)
-            return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
+    lr_status s = gla_scan<VD>(d, a, mQ, mO, nullptr, ws + w.gtiles, -1, (unsigned int*)(ws + w.ready), st);
+    if (s != LR_OK) return s;
     cudaFuncSetAttribute(gla_grad_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GGradSmem<VD>::kAlloc);
     note_launch("gla_chunk_grad");
     if (launch_pdl(gla_grad_kernel<VD>, dim3(a.nchunk * a.B * a.H), dim3(256), GGradSmem<VD>::kAlloc, st, mQ, mK, mV,
@@ -797,7 +708,7 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
 }  // namespace
 
 size_t gla_ws_bytes(const lr_desc& d, bool bwd) { return gla_plan(d, bwd).end; }
-size_t gla_flag_bytes(const lr_desc&, bool) { return 256; }
+size_t gla_flag_bytes(const lr_desc& d, bool bwd) { return gla_plan(d, bwd).flags_end; }
 
 lr_status gla_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
     return d.P == 64 ? gla_fwd_t<64>(d, in, y, ckpt, ws, st) : gla_fwd_t<128>(d, in, y, ckpt, ws, st);

@@ -1,7 +1,7 @@
 // chunk_scan.cuh -- the chunk-state scan shared by the matrix-state kinds (SSD and GLA) on
 // tcgen05: one CTA per (batch row, head, 64 value columns) folds the chunk products
 // S_{c+1} = e^{l_Q,c} S_c + R_c^T diag(w) Z_c (or the adjoint in reverse) into a register-resident
-// state and writes every chunk's entering state (the checkpoint slots), flagging each slot as it
+// state and writes every chunk's entering state (the checkpoint slots), counting each slot as it
 // lands so that the chunk kernels can run beside it.
 //
 // Recurrence ("mlx-recurrence", Apple Developer Forums thread 840535, "Current kernels": ssd_scan
@@ -103,12 +103,13 @@ __device__ __forceinline__ float wg_inclusive_sum(float x, float* tmp, int wg) {
 //     then S leaves through shared memory (f32: TMA store of two 32-column boxes; bf16 tile: one
 //     bulk copy, the tile already in its global format);
 //   warp 9: zeroes the dB, dC rows the SSD gradient kernel adds into (backward, by chunk, flagged),
-//     then flags the slots whose copies have landed (see below);
+//     then counts the slots whose copies have landed (see below);
 //   warp 11 (dt): the raw per-step decay input (SSD dt, GLA g) of every chunk into a ring in shared
 //     memory, kDtRing chunks ahead (kept out of the prep warps: their barriers and arrivals would
 //     wait for loads in flight).
 // No scan CTA waits on another.  Once the copies of a slot have landed the fold tells warp 9 (a counter
-// in shared memory), which flags the slot in global memory (a.ready), so that the output kernel
+// in shared memory), which counts the slot in global memory (ready[slot][b][g], one count per head
+// and half of the group, so that a consumer needs one acquire load for all of them), so that the output kernel
 // (forward) or the gradient kernel (backward) can start on a chunk before the whole scan has
 // finished; the fold itself never waits for a global-scope release.
 // NS stages: 3 when the f32 states are staged too (forward), 4 otherwise.
@@ -366,7 +367,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                 if (done >= next) {
                     for (; next <= done; ++next) {
                         const int slot = dir > 0 ? next : a.nchunk - 1 - next;
-                        st_release(&ready[(((size_t)slot * a.B + b) * a.H + h) * a.halves + half], 1u);
+                        red_release_add(&ready[((size_t)slot * a.B + b) * a.G + g], 1u);
                     }
                     t0 = global_ns();
                     continue;

@@ -237,34 +237,22 @@ __device__ __forceinline__ unsigned int wait_flag(const unsigned int* flag, WsHe
     return kFlagNone;
 }
 
-// Poll the n consecutive flags f[0 .. n) until all are non-zero (relaxed loads issued together,
-// then one acquire fence), for at most kWaitLimitNs.  Returns false after giving up (an error is
-// then recorded).
-__device__ __forceinline__ bool wait_flags(const unsigned int* f, int n, WsHeader* hdr, int info) {
+// Counter protocol: producers add 1 with release semantics, a consumer polls with acquire loads
+// until the counter reaches `target` (at most kWaitLimitNs; false after giving up, an error is
+// then recorded).  One acquire load covers every producer counted.
+__device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_count(const unsigned int* p, unsigned int target, WsHeader* hdr, int info) {
+    if (ld_acquire(p) >= target) return true;
     const unsigned long long t0 = global_ns();
     for (int i = 0;; ++i) {
-        bool all = true;
-        for (int k = 0; k < n; ++k) {
-            unsigned int v;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f + k) : "memory");
-            all = all && v != kFlagNone;
-        }
-        if (all) {
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            return true;
-        }
+        if (ld_acquire(p) >= target) return true;
         if (i > 16) __nanosleep(128);
         if (global_ns() - t0 > kWaitLimitNs) break;
     }
     record_error(hdr, LR_ERR_TIMEOUT, info);
     return false;
-}
-
-// The same with one acquire load per flag (no fence: cheaper for a few flags).
-__device__ __forceinline__ bool wait_flags_acquire(const unsigned int* f, int n, WsHeader* hdr, int info) {
-    for (int k = 0; k < n; ++k)
-        if (wait_flag(f + k, hdr, info) == kFlagNone) return false;
-    return true;
 }
 
 // Dynamic tile ticket: tiles are numbered in the order CTAs start, so that every tile a CTA may

@@ -108,12 +108,12 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     }
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 811);
     tc::fence_after_sync();
-    // the S_in tile of slot c: written by the scan kernel, which flags each 64-column half once its
+    // the S_in tile of slot c: written by the scan kernel, which counts each 64-column half once its
     // copies have landed; polled only now (the flag loads' latency hides behind the loads and
     // Q K^T above), and for slot 0, the zero state, too: the scan flags it only after the kernels
     // before it are done, and no global write of this kernel comes before this
     if (tid == 0) {
-        ok = wait_flags_acquire(&ready[(((size_t)c * a.B + b) * a.H + h) * halves], halves, a.hdr, 813) && ok;
+        ok = wait_count(&ready[((size_t)c * a.B + b) * a.H + h], (unsigned int)halves, a.hdr, 813) && ok;
         fence_proxy_async_global();
     }
     if (tid == 0 && ok && has_in) {  // k is consumed: its slot takes the S_in tile
@@ -233,7 +233,7 @@ struct GlaGradArgs {
     GlaArgs a;
     const char* stiles;      // [nchunk][B][H] bf16 tiles of the entering states
     const char* gtiles;      // [nchunk][B][H] bf16 tiles of the adjoint states
-    const unsigned int* gready;  // [nchunk][B][H][halves]: G tile half written (by the scan kernel)
+    const unsigned int* gready;  // [nchunk][B][H]: halves of the slot's G tile written (by the scan kernel)
     int halves;
     __nv_bfloat16* dq;       // [B, L, H, K]
     __nv_bfloat16* dk;
@@ -405,10 +405,10 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 822);
     tc::fence_after_sync();
     if (tid == 0) {  // P, Pd are consumed: their slots take S_in and G
-        // the G tile of slot c: written by the scan kernel, which flags each 64-column half once
+        // the G tile of slot c: written by the scan kernel, which counts each 64-column half once
         // its copies have landed (the last chunk's zero adjoint too, flagged only after the
         // kernels before the scan are done); no global write of this kernel comes before this
-        ok = wait_flags_acquire(&ga.gready[(((size_t)c * a.B + b) * a.H + h) * ga.halves], ga.halves, a.hdr, 828) && ok;
+        ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828) && ok;
         fence_proxy_async_global();
         const size_t tile = (((size_t)c * a.B + b) * a.H + h) * (size_t)(kKD * VD * 2);
         const uint32_t bytes = (has_in ? kKD * VD * 2 : 0u) + (has_out ? kKD * VD * 2 : 0u);

@@ -20,7 +20,7 @@
 //                     (f32, and a bf16 tile copy for the tensor cores), flagged once written;
 //   ssd_out_kernel    (batch row, chunk, head block): Y from M, the checkpoint and x; launched as a
 //                     programmatic dependent of the scan, it starts on the SMs the scan leaves
-//                     free and waits only for the flags of its own slot.
+//                     free and waits only for its own slot (a per-group count of the heads written).
 // The scan kernel never waits for another CTA, so the waits always end.  The backward pass has
 // the same shape (the scan in reverse, then the gradient kernel waiting per slot).
 #include "chunk_scan.cuh"
@@ -200,13 +200,13 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             tma_load_4d(Xs + u * kQ * 128, &mX, &wbar[u], 0, hfirst + wg + 2 * u, t0, b);
         }
     }
-    // S_in tiles of chunk c: written by the scan kernel, which flags each slot once its copies
-    // have landed, so this kernel runs beside the scan instead of after all of it (slot 0, the
-    // zero state, is waited for too: the scan flags it only after the kernels before it are done)
+    // S_in tiles of chunk c: written by the scan kernel, which counts each head of a slot once its
+    // copies have landed, so this kernel runs beside the scan instead of after all of it (slot 0,
+    // the zero state, is waited for too: the scan counts it only after the kernels before it are
+    // done).  One acquire load of the group's count covers every head of the block.
     bool ok = true;
     if (wt == 0) {
-        for (int u = 0; u < nmine; ++u)
-            ok = ok && wait_flag(&ready[((size_t)c * a.B + b) * a.H + hfirst + wg + 2 * u], a.hdr, 716) != 0;
+        ok = wait_count(&ready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 716);
         fence_proxy_async_global();
         if (has_in && nmine > 0) {
             mbar_arrive_expect_tx(&wbar[3], kTileBytes);
@@ -454,7 +454,7 @@ struct SsdGradArgs {
     float* pdA;            // [B][H][nchunk] per-chunk partials of dA_h, dD_h
     float* pdD;
     float* pdE;            // [B][H][nchunk] partials of d bias (LR_DELTA_SOFTPLUS)
-    const unsigned int* gready;  // [nchunk][B][H]: G tile of the slot written (by the scan kernel)
+    const unsigned int* gready;  // [nchunk][B][G]: heads of the group whose G tile of the slot is written
     const unsigned int* zready;  // [nchunk][B][G]: the chunk's dB, dC rows zeroed (by the scan kernel)
     int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
 };
@@ -618,12 +618,13 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         }
         load_xdy(0, hfirst);
     }
-    // the G tiles of slot c, written by the scan kernel, which flags each slot once its copies have
-    // landed (the last chunk's slot, the zero adjoint, too: the scan flags it only after the kernels
-    // before it are done), so this kernel runs beside the scan instead of after all of it
+    // the G tiles of slot c, written by the scan kernel, which counts each head of a slot once its
+    // copies have landed (the last chunk's slot, the zero adjoint, too: the scan counts it only
+    // after the kernels before it are done), so this kernel runs beside the scan instead of after
+    // all of it; one acquire load of the group's count covers every head of the block
     bool ok = true;
     if (tid == 0) {
-        ok = wait_flags(&ga.gready[((size_t)c * a.B + b) * a.H + hfirst], nh, a.hdr, 728);
+        ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 728);
         fence_proxy_async_global();
         load_sg(hfirst);
     }

@@ -503,39 +503,66 @@ def run_decode(kind, ai, w, T=256, reps=20):
 
 def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
     """Same step through the public API from pinned host buffers: every step copies its inputs
-    host->device, runs forward and backward, and copies y and all gradients back."""
+    host->device, runs forward and backward, and copies y and all gradients back.  Copies run on
+    their own streams with two sets of device (and host) buffers, so that the inputs of step i + 1
+    land and the results of step i - 1 leave while step i's kernels run (PCIe in both directions
+    beside the GPU work, as a training loop feeding the layer would overlap them)."""
     import torch
     import torch.distributed as dist
     from selective_state_space_09_b200 import dp
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     h_in = {k: v.to("cpu").pin_memory() for k, v in ai.items()}
     h_dy = dy.to("cpu").pin_memory()
-    h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    h_g = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
-    d_in = {k: torch.empty_like(v) for k, v in ai.items()}
-    d_dy = torch.empty_like(dy)
+    sets = []
+    for j in range(2):
+        sets.append({
+            "in": {k: torch.empty_like(v) for k, v in ai.items()}, "dy": torch.empty_like(dy),
+            "y": y if j == 0 else torch.empty_like(y),
+            "g": grads if j == 0 else {k: torch.empty_like(v) for k, v in grads.items()},
+            "hy": torch.empty(y.shape, dtype=y.dtype).pin_memory(),
+            "hg": {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()},
+            "ev_in": torch.cuda.Event(), "ev_comp": torch.cuda.Event(), "ev_out": torch.cuda.Event(),
+            "used": False})
 
-    def step():
-        for k in d_in:
-            d_in[k].copy_(h_in[k], non_blocking=True)
-        d_dy.copy_(h_dy, non_blocking=True)
-        plan.fwd(d_in, y)
-        plan.bwd(d_in, d_dy, grads)
+    def step(i):
+        S = sets[i % 2]
+        with torch.cuda.stream(s_in):
+            if S["used"]:
+                s_in.wait_event(S["ev_comp"])  # the kernels of two steps ago have read these inputs
+            for k in S["in"]:
+                S["in"][k].copy_(h_in[k], non_blocking=True)
+            S["dy"].copy_(h_dy, non_blocking=True)
+            S["ev_in"].record(s_in)
+        comp.wait_event(S["ev_in"])
+        if S["used"]:
+            comp.wait_event(S["ev_out"])  # the results of two steps ago have left
+        plan.fwd(S["in"], S["y"])
+        plan.bwd(S["in"], S["dy"], S["g"])
         if world > 1:
-            dp.reduce_param_grads(kind, grads)
-        h_y.copy_(y, non_blocking=True)
-        for k in grads:
-            h_g[k].copy_(grads[k], non_blocking=True)
+            dp.reduce_param_grads(kind, S["g"])
+        S["ev_comp"].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(S["ev_comp"])
+            S["hy"].copy_(S["y"], non_blocking=True)
+            for k in S["g"]:
+                S["hg"][k].copy_(S["g"][k], non_blocking=True)
+            S["ev_out"].record(s_out)
+        S["used"] = True
 
-    for _ in range(max(1, warmup)):
-        step()
+    for i in range(max(1, warmup)):
+        step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
+    e0.record(comp)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(steps):
+        step(i)
+    comp.wait_stream(s_out)  # the last results have left
+    e1.record(comp)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     if world > 1:
@@ -543,9 +570,10 @@ def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     bi = sum(nbytes(v) for v in h_in.values()) + nbytes(h_dy)
-    bo = nbytes(h_y) + sum(nbytes(v) for v in h_g.values())
+    bo = nbytes(sets[0]["hy"]) + sum(nbytes(v) for v in sets[0]["hg"].values())
     return {"value": tokens_of(w) * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "note": "inputs of step i + 1 and results of step i - 1 cross PCIe while step i runs"}
 
 
 # ------------------------------------------------------------------------ oracle (CPU)

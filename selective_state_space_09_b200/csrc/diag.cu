@@ -158,11 +158,14 @@ template <int KIND, typename T, bool BWD> struct Smem {
     using K = Kind<KIND, T>;
     using V = typename K::V;
     static constexpr bool G = KIND == kRgGated;  // x tile (and, backward, a tile of b values)
+    // rotlru backward: dy lands in b's slot once the forward recompute is done with b (three tiles
+    // per SM instead of two)
+    static constexpr bool AL = BWD && KIND == LR_ROTLRU;
     static __host__ __device__ constexpr size_t coef_bytes() { return size_t(kMaxSeg) * K::CW * sizeof(T); }
     static __host__ __device__ constexpr size_t b_bytes() { return size_t(kMaxSeg) * K::BW * sizeof(T); }
     static __host__ __device__ constexpr size_t off_coef() { return 128; }
     static __host__ __device__ constexpr size_t off_b() { return off_coef() + coef_bytes(); }
-    static __host__ __device__ constexpr size_t off_dy() { return off_b() + b_bytes(); }
+    static __host__ __device__ constexpr size_t off_dy() { return off_b() + (AL ? 0 : b_bytes()); }
     static __host__ __device__ constexpr size_t off_x() { return off_dy() + (BWD ? b_bytes() : 0); }
     static __host__ __device__ constexpr size_t off_e() { return off_x() + (G ? b_bytes() : 0); }
     static __host__ __device__ constexpr size_t off_aggf() { return off_e() + (G && BWD ? b_bytes() : 0); }
@@ -401,7 +404,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 
 // -------------------------------------------------------------------------------- backward
 template <int KIND, typename T, bool FULL>
-__global__ void __launch_bounds__(kThreads, 2)  // two tiles per SM (shared memory)
+__global__ void __launch_bounds__(kThreads, KIND == LR_ROTLRU ? 3 : 2)  // tiles per SM (shared memory)
 diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapDY,
                 const __grid_constant__ CUtensorMap mapDC, const __grid_constant__ CUtensorMap mapDB,
@@ -455,8 +458,10 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         tma_load_3d(Cs, &mapC, &bar[0], cb * K::CW, t0g, b);
         if (!full) tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
         if (gated) tma_load_3d(Xs, &mapX, &bar[0], cb * K::BW, t0g, b);
-        mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
-        tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
+        if (!(SM::AL && !full)) {
+            mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
+            tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
+        }
     }
     const int unit = cb * CB + u;
     const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
@@ -523,6 +528,14 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             hprev[j] = (j < n && unit < units)
                            ? K::ld_ckpt(a.ckpt + ((size_t)(t0g + j0 + j) * a.B + b) * a.D, unit * K::chans_per_unit)
                            : zero_of(V{});
+    }
+    if constexpr (SM::AL && !full) {  // dy into b's slot, now that every thread is done with b
+        __syncthreads();
+        if (tid == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
+            tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
+        }
     }
     // reverse aggregate of the group: outgoing carry = v + m * incoming
     ok = mbar_wait(&bar[1], 0, a.hdr, 202) && ok;

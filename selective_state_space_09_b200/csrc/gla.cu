@@ -93,6 +93,13 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
         mbar_arrive_expect_tx(&bar[1], (uint32_t)(kQ * VD * 2));
         for (int j = 0; j < VD / 64; ++j) tma_load_4d(sm + SM::kVt + j * kQ * 128, &mV, &bar[1], 64 * j, h, t0, b);
     }
+    // the S_in tile of slot c: written by the scan kernel, which counts each 64-column half once its
+    // copies have landed; polled here by a thread with no copies in flight, so that the poll's
+    // latency hides behind the loads above (slot 0, the zero state, is waited for too: the scan
+    // counts it only after the kernels before it are done, and no global write of this kernel
+    // comes before the barrier below)
+    bool ready_ok = true;
+    if (tid == 32) ready_ok = wait_count(&ready[((size_t)c * a.B + b) * a.H + h], (unsigned int)halves, a.hdr, 813);
     const float lt2 = cta_inclusive_sum(gla_lam(a, b, h, t0 + tid), tmp) * kLog2e;
     l2s[tid] = lt2;
     __syncthreads();
@@ -108,15 +115,9 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     }
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 811);
     tc::fence_after_sync();
-    // the S_in tile of slot c: written by the scan kernel, which counts each 64-column half once its
-    // copies have landed; polled only now (the flag loads' latency hides behind the loads and
-    // Q K^T above), and for slot 0, the zero state, too: the scan flags it only after the kernels
-    // before it are done, and no global write of this kernel comes before this
-    if (tid == 0) {
-        ok = wait_count(&ready[((size_t)c * a.B + b) * a.H + h], (unsigned int)halves, a.hdr, 813) && ok;
-        fence_proxy_async_global();
-    }
+    ok = ok && ready_ok;
     if (tid == 0 && ok && has_in) {  // k is consumed: its slot takes the S_in tile
+        fence_proxy_async_global();  // the copy comes after the count polled above
         mbar_arrive_expect_tx(&bar[3], (uint32_t)(kKD * VD * 2));
         bulk_load(sm + SM::kKt, stiles + (((size_t)c * a.B + b) * a.H + h) * (size_t)(kKD * VD * 2),
                   (uint32_t)(kKD * VD * 2), &bar[3]);
@@ -305,6 +306,12 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
             tma_load_4d(sm + SM::kOt + j * kQ * 128, &mO, &bar[0], 64 * j, h, t0, b);
         }
     }
+    // the G tile of slot c: written by the scan kernel, which counts each 64-column half once its
+    // copies have landed (the last chunk's zero adjoint too, counted only after the kernels before
+    // the scan are done); polled here by a thread of warpgroup 1, idle while warpgroup 0 forms the
+    // decays, and no global write of this kernel comes before the barrier below
+    bool ready_ok = true;
+    if (tid == 224) ready_ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
     // decays (warpgroup 0), column factors cf[w][s] = e^{l_{32 w} - l_s} (s < 32 w)
     if (wg == 0) l2s[row] = wg0_inclusive_sum(gla_lam(a, b, h, t0 + row), tmp) * kLog2e;
     __syncthreads();
@@ -313,7 +320,7 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         const int w = k >> 7, s = k & 127;
         if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]);
     }
-    bool ok = mbar_wait(&bar[0], 0, a.hdr, 820);
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 820) && ready_ok;
     __syncthreads();
     if (tid == 0 && ok) {  // phase A
         tc::fence_after_sync();
@@ -405,11 +412,7 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 822);
     tc::fence_after_sync();
     if (tid == 0) {  // P, Pd are consumed: their slots take S_in and G
-        // the G tile of slot c: written by the scan kernel, which counts each 64-column half once
-        // its copies have landed (the last chunk's zero adjoint too, flagged only after the
-        // kernels before the scan are done); no global write of this kernel comes before this
-        ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828) && ok;
-        fence_proxy_async_global();
+        fence_proxy_async_global();  // the copies below come after the count polled above
         const size_t tile = (((size_t)c * a.B + b) * a.H + h) * (size_t)(kKD * VD * 2);
         const uint32_t bytes = (has_in ? kKD * VD * 2 : 0u) + (has_out ? kKD * VD * 2 : 0u);
         if (bytes == 0) {

@@ -124,9 +124,11 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * contains 1 / sqrt(1 - a^2)).  Not combined with LR_FULL_STATE (LR_ERR_UNSUPPORTED); other
  * kinds: LR_ERR_INVALID_ARG.  lr_step accepts it (forward only). */
 #define LR_RGLRU_GATES 16u
-/* Test hook for the failure path: the tiles of the first segment never publish their carry, so
- * the tiles after them wait out their bound (about 1 s), record LR_ERR_TIMEOUT and finish with an
- * incomplete carry.  Results of such a call are meaningless; lr_get_error reports the timeout. */
+/* Test hook for the failure path: the tiles of the first segment never publish their carry
+ * (rglru, rotlru), or the state scan never counts checkpoint slot 0 (SSD, GLA), so the tiles or
+ * chunk kernels that depend on it wait out their bound (about 1 s), record LR_ERR_TIMEOUT and
+ * finish with incomplete inputs.  Results of such a call are meaningless; lr_get_error reports
+ * the timeout. */
 #define LR_TEST_WITHHOLD_CARRY 0x80000000u
 /* Test hook for the work distribution: SSD kernels that loop over the heads of a group inside one
  * CTA take the largest head blocks they support (16 heads) instead of sizing the blocks to fill

@@ -31,6 +31,7 @@ struct ScanArgs {
     const __nv_bfloat16* dt;      // [B, L, H]: SSD raw dt, GLA gate g in (0, 1)
     const float* A;               // SSD [H]
     WsHeader* hdr;
+    int withhold;                 // LR_TEST_WITHHOLD_CARRY: slot 0 is never counted (failure-path test)
 };
 
 // beta of one step inside the sequence (lam = dt A_h): ZOH (e^{lam} - 1) / A_h, dirac 1,
@@ -367,7 +368,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                 if (done >= next) {
                     for (; next <= done; ++next) {
                         const int slot = dir > 0 ? next : a.nchunk - 1 - next;
-                        red_release_add(&ready[((size_t)slot * a.B + b) * a.G + g], 1u);
+                        if (!(a.withhold && slot == 0)) red_release_add(&ready[((size_t)slot * a.B + b) * a.G + g], 1u);
                     }
                     t0 = global_ns();
                     continue;

@@ -24,6 +24,7 @@ struct GlaArgs {
     int B, L, H, nchunk;
     const __nv_bfloat16* g;   // [B, L, H] gate in (0, 1)
     WsHeader* hdr;
+    int withhold;             // LR_TEST_WITHHOLD_CARRY (the scan never counts slot 0)
 };
 
 // log decay of step t of head h (0 past L)
@@ -98,8 +99,8 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     // latency hides behind the loads above (slot 0, the zero state, is waited for too: the scan
     // counts it only after the kernels before it are done, and no global write of this kernel
     // comes before the barrier below)
-    bool ready_ok = true;
-    if (tid == 32) ready_ok = wait_count(&ready[((size_t)c * a.B + b) * a.H + h], (unsigned int)halves, a.hdr, 813);
+    // (a timeout is recorded in the workspace; the kernel finishes)
+    if (tid == 32) wait_count(&ready[((size_t)c * a.B + b) * a.H + h], (unsigned int)halves, a.hdr, 813);
     const float lt2 = cta_inclusive_sum(gla_lam(a, b, h, t0 + tid), tmp) * kLog2e;
     l2s[tid] = lt2;
     __syncthreads();
@@ -115,7 +116,6 @@ gla_out_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ C
     }
     ok = ok && mbar_wait(&bar[2], 0, a.hdr, 811);
     tc::fence_after_sync();
-    ok = ok && ready_ok;
     if (tid == 0 && ok && has_in) {  // k is consumed: its slot takes the S_in tile
         fence_proxy_async_global();  // the copy comes after the count polled above
         mbar_arrive_expect_tx(&bar[3], (uint32_t)(kKD * VD * 2));
@@ -310,8 +310,8 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     // copies have landed (the last chunk's zero adjoint too, counted only after the kernels before
     // the scan are done); polled here by a thread of warpgroup 1, idle while warpgroup 0 forms the
     // decays, and no global write of this kernel comes before the barrier below
-    bool ready_ok = true;
-    if (tid == 224) ready_ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
+    // (a timeout is recorded in the workspace; the kernel finishes)
+    if (tid == 224) wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
     // decays (warpgroup 0), column factors cf[w][s] = e^{l_{32 w} - l_s} (s < 32 w)
     if (wg == 0) l2s[row] = wg0_inclusive_sum(gla_lam(a, b, h, t0 + row), tmp) * kLog2e;
     __syncthreads();
@@ -320,7 +320,7 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         const int w = k >> 7, s = k & 127;
         if (s < 32 * w) cf[k] = ex2(l2s[32 * w] - l2s[s]);
     }
-    bool ok = mbar_wait(&bar[0], 0, a.hdr, 820) && ready_ok;
+    bool ok = mbar_wait(&bar[0], 0, a.hdr, 820);
     __syncthreads();
     if (tid == 0 && ok) {  // phase A
         tc::fence_after_sync();
@@ -609,6 +609,7 @@ GlaArgs gla_args(const lr_desc& d, const lr_inputs& in, char* ws) {
     a.nchunk = (int)((d.L + kQ - 1) / kQ);
     a.g = (const __nv_bfloat16*)in.g;
     a.hdr = (WsHeader*)ws;
+    a.withhold = (d.flags & LR_TEST_WITHHOLD_CARRY) ? 1 : 0;
     return a;
 }
 
@@ -624,6 +625,7 @@ ScanArgs scan_args(const GlaArgs& a, int VD) {
     s.halves = VD / kScanP;
     s.dt = a.g;
     s.hdr = a.hdr;
+    s.withhold = a.withhold;
     return s;
 }
 

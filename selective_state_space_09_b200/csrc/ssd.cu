@@ -42,6 +42,7 @@ struct SsdArgs {
     const float* Dskip;           // [H] or null
     const float* ckpt;            // [nchunk][B][H][N][P] f32 (state entering each chunk)
     WsHeader* hdr;
+    int withhold;                 // LR_TEST_WITHHOLD_CARRY (the scan never counts slot 0)
 };
 
 // The scan kernel's view of the problem (chunk_scan.cuh).
@@ -60,6 +61,7 @@ __host__ ScanArgs scan_args(const SsdArgs& a) {
     s.dt = a.dt;
     s.A = a.A;
     s.hdr = a.hdr;
+    s.withhold = a.withhold;
     return s;
 }
 
@@ -206,7 +208,8 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     // done).  One acquire load of the group's count covers every head of the block.
     bool ok = true;
     if (wt == 0) {
-        ok = wait_count(&ready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 716);
+        // (a timeout is recorded in the workspace; the kernel finishes)
+        wait_count(&ready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 716);
         fence_proxy_async_global();
         if (has_in && nmine > 0) {
             mbar_arrive_expect_tx(&wbar[3], kTileBytes);
@@ -382,6 +385,7 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
     a.ckpt = (const float*)ckpt;
     a.hdr = (WsHeader*)ws;
+    a.withhold = (d.flags & LR_TEST_WITHHOLD_CARRY) ? 1 : 0;
     return a;
 }
 
@@ -624,7 +628,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     // all of it; one acquire load of the group's count covers every head of the block
     bool ok = true;
     if (tid == 0) {
-        ok = wait_count(&ga.gready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 728);
+        // (a timeout is recorded in the workspace; the kernel finishes)
+        wait_count(&ga.gready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 728);
         fence_proxy_async_global();
         load_sg(hfirst);
     }

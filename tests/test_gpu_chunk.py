@@ -85,6 +85,26 @@ def test_ssd_softplus_front_end():
     assert plan.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("kind", ["ssd", "gla"])
+def test_withheld_slot_times_out_and_context_survives(kind):
+    """Failure path of the scan / chunk-kernel protocol: the state scan never counts slot 0, so the
+    chunk kernels of the first chunk wait out their bound, record LR_ERR_TIMEOUT (status 6) with
+    the waiting site and finish.  A normal call afterwards on the same context is correct."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.ssd(1, 300, 8, 64, 128, seed=41) if kind == "ssd" else inputs.gla(1, 300, 8, 128, 128, seed=41)
+    disc = "zoh" if kind == "ssd" else "none"
+    y, ck, gr, plan, _ = run_gpu(kind, inp, 128, disc=disc, chunk=128, flags=lrscan.TEST_WITHHOLD_CARRY)
+    status, info = plan.device_error()
+    assert status == 6 and info in ((716, 728) if kind == "ssd" else (813, 828)), (status, info)
+    y, ck, gr, plan, _ = run_gpu(kind, inp, 128, disc=disc, chunk=128)
+    assert plan.device_error() == (0, 0)
+    if kind == "ssd":
+        ref = oracle.ssd_fwd(inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], None, disc="zoh")
+    else:
+        ref = oracle.gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"])
+    assert_close("y", y, ref, TOL)
+
+
 def test_ssd_head_blocking_bitwise():
     """The head blocking of the output kernel changes only which CTA computes a head."""
     from selective_state_space_09_b200 import lrscan

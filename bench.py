@@ -71,8 +71,8 @@ def peaks():
 # Sources each kernel family is built from (its own file and the headers it includes): a committed
 # ncu figure stays valid while these are unchanged.
 KERNEL_SOURCES = {
-    "ssd": ("ssd.cu", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
-    "gla": ("gla.cu", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
+    "ssd": ("ssd.cu", "chunk_scan.cuh", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
+    "gla": ("gla.cu", "chunk_scan.cuh", "chunk_common.cuh", "common.cuh", "tc.cuh", "host_common.h"),
     "s6": ("s6.cu", "common.cuh", "host_common.h"),
     "rglru": ("diag.cu", "common.cuh", "host_common.h"),
     "rotlru": ("diag.cu", "common.cuh", "host_common.h"),

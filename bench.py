@@ -671,7 +671,7 @@ def time_oracle(name, repeats=1, min_seconds=1.0):
 
 # ---------------------------------------------------------------------------------- main
 def built_workloads():
-    """Workloads whose kind this build implements (lr_validate reports UNSUPPORTED otherwise)."""
+    """Workloads whose kind the library implements (lr_validate reports UNSUPPORTED otherwise)."""
     import torch
     from selective_state_space_09_b200 import inputs, lrscan
     ok = []

@@ -75,7 +75,7 @@ extern "C" {
 typedef enum {
     LR_OK = 0,
     LR_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, non-positive or inconsistent shape   */
-    LR_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (see lr_validate) */
+    LR_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement (see lr_validate) */
     LR_ERR_ALIGNMENT = 3,     /* pointer or innermost extent not 16-byte aligned                */
     LR_ERR_WORKSPACE = 4,     /* workspace smaller than lr_workspace_bytes                      */
     LR_ERR_CUDA = 5,          /* a CUDA runtime call failed (launch, memset, copy)              */
@@ -175,7 +175,7 @@ typedef struct {
 } lr_grads;
 
 /* Host-side check of a descriptor: LR_OK, or the status lr_scan_fwd would return for it
- * (INVALID_ARG for inconsistent shapes, UNSUPPORTED for a valid request outside this build's
+ * (INVALID_ARG for inconsistent shapes, UNSUPPORTED for a valid request outside the library's
  * limits, ALIGNMENT for innermost extents that are not multiples of 16 bytes). */
 lr_status lr_validate(const lr_desc *desc);
 

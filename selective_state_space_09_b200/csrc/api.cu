@@ -22,7 +22,7 @@ thread_local cudaStream_t t_stream = nullptr;  // stream of the current entry-po
 int esize(int io) { return io == LR_BF16 ? 2 : 4; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Shape rules of this build (also reported by lr_validate).
+// Shape rules of the library (also reported by lr_validate).
 lr_status validate(const lr_desc* d) {
     if (!d) return LR_ERR_INVALID_ARG;
     if (d->kind < LR_RGLRU || d->kind > LR_GLA) return LR_ERR_INVALID_ARG;
@@ -372,7 +372,7 @@ const char* lr_status_string(lr_status s) {
     switch (s) {
         case LR_OK: return "ok";
         case LR_ERR_INVALID_ARG: return "invalid argument";
-        case LR_ERR_UNSUPPORTED: return "unsupported by this build";
+        case LR_ERR_UNSUPPORTED: return "unsupported by this library";
         case LR_ERR_ALIGNMENT: return "misaligned pointer or innermost extent";
         case LR_ERR_WORKSPACE: return "workspace too small";
         case LR_ERR_CUDA: return "CUDA runtime error";

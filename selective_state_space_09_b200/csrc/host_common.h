@@ -67,7 +67,7 @@ struct WsCursor {
     }
 };
 
-// Per-kind entry points (defined in the kernel files).  *_supported: whether this build has
+// Per-kind entry points (defined in the kernel files).  *_supported: whether the library has
 // kernels for the (already validated) descriptor.
 bool s6_supported(const lr_desc& d);
 bool chunk_supported(const lr_desc& d);

@@ -25,7 +25,7 @@ IO = {torch.float32: 0, torch.bfloat16: 1}
 HAS_Z, HAS_DSKIP, FULL_STATE, DELTA_SOFTPLUS, RGLRU_GATES = 1, 2, 4, 8, 16
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
 TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
-STATUS = ["ok", "invalid argument", "unsupported by this build", "misaligned pointer or innermost extent",
+STATUS = ["ok", "invalid argument", "unsupported by this library", "misaligned pointer or innermost extent",
           "workspace too small", "CUDA runtime error", "device wait timed out",
           "device consistency check failed"]
 

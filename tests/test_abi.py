@@ -189,7 +189,7 @@ def test_plan_buffers_cover_the_queried_sizes(L):
 
 
 def test_every_gpu_test_case_passes_host_validation(L):
-    """The descriptors of the GPU parity cases are valid for this build (checked on the CPU, so a
+    """The descriptors of the GPU parity cases are valid for the library (checked on the CPU, so a
     shape-rule mistake does not cost a GPU run)."""
     import torch
     import test_gpu_diag as gd

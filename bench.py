@@ -191,119 +191,182 @@ def nbytes(t):
     return t.numel() * t.element_size()
 
 
-def algorithmic_bytes(kind, inp, y, grads, ckpt_bytes):
-    """Bytes the step must move at minimum: every input read once and every output written once
-    per pass, plus the checkpoints (written by the forward pass, read by the backward pass)."""
-    ins = sum(nbytes(v) for v in api_inputs(kind, inp).values())
-    fwd = ins + nbytes(y) + ckpt_bytes
-    bwd = ins + nbytes(inp["dy"]) + ckpt_bytes + sum(nbytes(v) for v in grads.values())
+def operand_bytes(kind, inp, y, grads, dy, ckpt_bytes):
+    """Bytes of every operand of one step (each tensor once): the inputs, the output, the upstream
+    gradient, every gradient, and the f32 checkpoint states at the configured segment length
+    (written by the forward pass, read by the backward pass).  Intermediates a kernel creates for
+    another kernel (per-chunk state tiles, partial sums) are not operands."""
+    ops = {k: nbytes(v) for k, v in api_inputs(kind, inp).items()}
+    ops["y"] = nbytes(y)
+    ops["dy"] = nbytes(dy)
+    ops.update({k: nbytes(v) for k, v in grads.items()})
+    ops["ckpt"] = ckpt_bytes
+    return ops
+
+
+def algorithmic_bytes(kind, ops, grad_names):
+    """Bytes a pass must move at minimum: every input read once and every output written once,
+    plus the checkpoints (forward: written; backward: read)."""
+    ins = sum(ops[k] for k in INPUT_NAMES[kind] if k in ops)
+    fwd = ins + ops["y"] + ops["ckpt"]
+    bwd = ins + ops["dy"] + ops["ckpt"] + sum(ops[k] for k in grad_names)
     return fwd, bwd
 
 
-def kernel_cost(w, name, pas, pass_bytes):
-    """Algorithmic bytes and FLOPs of one launch of kernel `name` of a workload's pass: what the
-    kernel must read and write at minimum (each operand once) and the products of the method it
-    evaluates.  Kernels that are a whole pass carry the pass's bytes; small fixed-order reductions
-    are counted as 0 (they are not candidates for the dominant kernel)."""
-    kind = w["kind"]
-    if name.endswith("param_reduce"):
-        return 0, 0
-    if kind == "ssd":
-        B, L, H, P, N, G = w["B"], w["L"], w["H"], w["P"], w["N"], w.get("G", 1)
-        Q = 128
-        nc = -(-L // Q)
-        tok = B * L * H * P * 2            # x, dy, y, dx (bf16)
-        bc = B * L * G * N * 2             # B or C (bf16)
-        dt = B * L * H * 2
-        slot = B * H * N * P * 4           # one f32 state slot
-        tile = B * H * N * P * 2           # one bf16 state slot
-        head_chunks = nc * B * H
-        if name == "ssd_state_scan":       # x (dy), B (C), dt in; every slot out (f32 + tile; tile)
-            out = nc * (slot + tile) if pas == "fwd" else nc * tile
-            return tok + bc + dt + out, (nc - 1) * B * H * 2 * N * P * Q
+# Operands each kernel of the chunked kinds reads or writes (names as in operand_bytes); the
+# kernels that are a whole pass (diagonal kinds, S6) carry the pass's bytes.
+CHUNK_KERNEL_OPERANDS = {
+    ("ssd_state_scan", "fwd"): ("x", "Bm", "delta", "ckpt"),
+    ("ssd_chunk_out", "fwd"): ("x", "Bm", "Cm", "delta", "Dskip", "z", "y"),
+    ("ssd_state_scan", "bwd"): ("Cm", "dy", "delta", "z"),
+    ("ssd_chunk_grad", "bwd"): ("x", "Bm", "Cm", "delta", "Dskip", "z", "dy", "ckpt",
+                                "dx", "ddelta", "dBm", "dCm", "dz"),
+    ("gla_state_scan", "fwd"): ("k", "v", "g", "ckpt"),
+    ("gla_chunk_out", "fwd"): ("q", "k", "v", "g", "y"),
+    ("gla_state_scan", "bwd"): ("q", "dy", "g"),
+    ("gla_chunk_grad", "bwd"): ("q", "k", "v", "g", "dy", "ckpt", "dq", "dk", "dv", "dg"),
+}
+
+
+def chunk_flops(w, name):
+    """FLOPs of the method's products in one launch of a chunked kind's kernel (M = C B^T counted
+    once per row, chunk and group for SSD)."""
+    Q = w.get("chunk") or 128
+    nc = -(-w["L"] // Q)
+    if w["kind"] == "ssd":
+        B, H, P, N, G = w["B"], w["H"], w["P"], w["N"], w.get("G", 1)
+        hc = nc * B * H
+        if name == "ssd_state_scan":
+            return (nc - 1) * B * H * 2 * N * P * Q
         if name == "ssd_chunk_out":
-            fl = head_chunks * (2 * Q * P * Q + 2 * Q * P * N) + nc * B * G * 2 * Q * Q * N
-            return 2 * tok + 2 * bc + dt + nc * tile, fl
+            return hc * (2 * Q * P * Q + 2 * Q * P * N) + nc * B * G * 2 * Q * Q * N
         if name == "ssd_chunk_grad":
             per = 2 * Q * (Q * P + 2 * Q * N + Q * P + 2 * P * N + 2 * N * P)
-            fl = head_chunks * per + nc * B * G * 2 * Q * Q * N
-            return 3 * tok + 2 * bc + 2 * dt + 2 * nc * tile + 2 * B * L * G * N * 4, fl
-    if kind == "gla":
-        B, L, H, K, V = w["B"], w["L"], w["H"], w["K"], w["V"]
-        Q = 128
-        nc = -(-L // Q)
-        tk = B * L * H * K * 2             # q, k, dq, dk (bf16)
-        tv = B * L * H * V * 2             # v, o, dO, dv
-        g = B * L * H * 2
-        slot = B * H * K * V * 4
-        tile = B * H * K * V * 2
+            return hc * per + nc * B * G * 2 * Q * Q * N
+    if w["kind"] == "gla":
+        B, H, K, V = w["B"], w["H"], w["K"], w["V"]
         hc = nc * B * H
-        prod = 2 * Q * Q * max(K, V)       # one 128 x 128 x 128 product
-        if name == "gla_state_scan":       # k (q), v (dO), g in; every slot out (f32 + tile; tile)
-            out = nc * (slot + tile) if pas == "fwd" else nc * tile
-            return tk + tv + g + out, (nc - 1) * B * H * 2 * K * V * Q
+        prod = 2 * Q * Q * max(K, V)
+        if name == "gla_state_scan":
+            return (nc - 1) * B * H * 2 * K * V * Q
         if name == "gla_chunk_out":
-            return 2 * tk + 2 * tv + g + nc * tile, hc * 3 * prod
+            return hc * 3 * prod
         if name == "gla_chunk_grad":
-            return 4 * tk + 3 * tv + 2 * g + 2 * nc * tile, hc * 9 * prod
+            return hc * 9 * prod
+    return 0
+
+
+def kernel_cost(w, name, pas, ops, pass_bytes):
+    """Algorithmic bytes and FLOPs of one launch of kernel `name` of a workload's pass: the
+    operands the kernel must read and write at minimum (each once) and the products of the method
+    it evaluates.  Kernels that are a whole pass carry the pass's bytes; small fixed-order
+    reductions are counted as 0 (they are not candidates for the dominant kernel)."""
+    if name.endswith("param_reduce"):
+        return 0, 0
+    key = (name, pas)
+    if key in CHUNK_KERNEL_OPERANDS:
+        return sum(ops.get(k, 0) for k in CHUNK_KERNEL_OPERANDS[key]), chunk_flops(w, name)
     return pass_bytes, 0
 
 
-# S6 is bound by plain ALU work: per (t, d, n) element, FMA-pipe ops and MUFU (ex2 / rcp) results
-# (forward 7 + 1, backward 25 + 2).  Peak element rate = 148 SMs x min(128 FMA lanes / ops,
-# 16 MUFU lanes / results) x the maximum SM clock (1,965 MHz).
-S6_ALU = {"fwd": (7, 1), "bwd": (25, 2)}
-SM_COUNT, SM_MAX_HZ = 148, 1.965e9
+# S6 is bound by plain arithmetic, not memory.  Per (b, t, d, n) element, the method needs at
+# least one exponential (or, bilinear, one reciprocal) per pass -- the forward forms abar, the
+# backward re-forms it from the checkpoint -- and the fp32 FMA-pipe operations counted below
+# (forward: beta, the state update, the readout term; backward: the state recompute, the adjoint
+# update and the six gradient terms).  The peak rate of each pipe is measured on the device by
+# lr_probe_pipe at the start of the run.
+S6_ALU = {"fwd": {"ffma": 5, "mufu": 1}, "bwd": {"ffma": 15, "mufu": 1}}
 
 
-def kernel_alu(w, name, pas):
-    if w["kind"] != "s6" or name.endswith("param_reduce"):
+def kernel_alu(w, name, pas, rates):
+    if w["kind"] != "s6" or name.endswith("param_reduce") or not rates:
         return None
-    fma, mufu = S6_ALU[pas]
+    c = S6_ALU[pas]
     elems = w["B"] * w["L"] * w["D"] * w["N"]
-    peak = SM_COUNT * SM_MAX_HZ * min(128.0 / fma, 16.0 / mufu)
-    return {"elements": elems, "peak_elems_per_s": peak}
+    t_mufu = elems * c["mufu"] / rates["ex2_per_s"]
+    t_fma = elems * c["ffma"] / rates["ffma_per_s"]
+    return {"elements": elems, "pipe": "mufu" if t_mufu >= t_fma else "ffma",
+            "peak_elems_per_s": elems / max(t_mufu, t_fma), "ops_per_element": c}
 
 
-def kernel_table(w, names, ms, pas, pass_bytes):
+def kernel_table(w, names, ms, pas, ops, pass_bytes, rates):
     rows = []
     for k, (n, t) in enumerate(zip(names, ms)):
-        b, f = kernel_cost(w, n, pas, pass_bytes)
+        b, f = kernel_cost(w, n, pas, ops, pass_bytes)
         rows.append({"pass": pas, "index": k, "kernel": n, "ms": t, "bytes": b, "flops": f,
-                     "alu": kernel_alu(w, n, pas)})
+                     "alu": kernel_alu(w, n, pas, rates)})
     return rows
 
 
 def kernel_roofline(row, pk):
     """Roofline entry of one timed kernel: the bound is whichever of its algorithmic bytes at the
-    measured copy bandwidth and its FLOPs at the measured bf16 GEMM rate takes longer."""
+    measured copy bandwidth, its FLOPs at the measured bf16 GEMM rate and (S6) its arithmetic at
+    the measured pipe rates takes longer.  Chunked kinds also carry their tensor-pipe figure."""
     t_hbm = row["bytes"] / (pk["hbm_gbs"] * 1e9)
     t_tc = row["flops"] / (pk["bf16_tflops"] * 1e12)
     sec = row["ms"] * 1e-3
     alu = row.get("alu")
+    out = None
     if alu and alu["elements"] / alu["peak_elems_per_s"] > max(t_hbm, t_tc):
         ach = alu["elements"] / sec / 1e9
         pk_g = alu["peak_elems_per_s"] / 1e9
-        return {"bound": "alu", "achieved": round(ach, 1), "peak": round(pk_g, 1), "unit": "Gelem/s",
-                "frac": round(ach / pk_g, 4)}
-    if t_tc > t_hbm:
+        out = {"bound": "alu", "achieved": round(ach, 2), "peak": round(pk_g, 2), "unit": "Gelem/s",
+               "frac": round(ach / pk_g, 4), "pipe": alu["pipe"], "ops_per_element": alu["ops_per_element"]}
+    elif t_tc > t_hbm:
         ach = row["flops"] / sec / 1e12
-        return {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(ach / pk["bf16_tflops"], 4)}
-    ach = row["bytes"] / sec / 1e9
-    return {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(ach / pk["hbm_gbs"], 4)}
+        out = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+               "frac": round(ach / pk["bf16_tflops"], 4)}
+    else:
+        ach = row["bytes"] / sec / 1e9
+        out = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+               "frac": round(ach / pk["hbm_gbs"], 4)}
+    if row["flops"]:
+        tf = row["flops"] / sec / 1e12
+        out["tensor"] = {"achieved_tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 4),
+                         "hbm_frac": round(row["bytes"] / sec / 1e9 / pk["hbm_gbs"], 4)}
+    return out
+
+
+def measure_pipe_rates(device):
+    """Rates of the special-function unit (ex2) and the fp32 FMA pipe on this device, from one
+    timed launch each of lr_probe_pipe (CUDA events; best of 3)."""
+    import torch
+    from selective_state_space_09_b200 import lrscan
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    blocks, threads = sms * 8, 256
+    out = torch.empty(blocks * threads, dtype=torch.float32, device=device)
+    res = {"sms": sms}
+    for which, iters in (("ex2", 2048), ("ffma", 8192)):
+        best = None
+        for _ in range(4):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            n = lrscan.probe_pipe(which, out, blocks, threads, iters)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        res[which + "_per_s"] = n / (best * 1e-3)
+        res[which + "_per_clk_per_sm_at_max_clock"] = round(res[which + "_per_s"] / (sms * SM_MAX_HZ), 2)
+    del out
+    return res
+
+
+SM_MAX_HZ = 1.965e9
 
 
 def tokens_of(w):
     return w["B"] * w["L"]
 
 
-def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu_sample=False):
+def run_workload(name, steps, warmup, device, rank, world, flush_buf, e2e=False, rates=None):
     import torch
     import torch.distributed as dist
     from selective_state_space_09_b200 import dp, lrscan
 
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(device)
+    mem0 = torch.cuda.memory_allocated(device)
     w, inp = workload_inputs(name, device, seed=1000 + rank)
     kind = w["kind"]
     ai = api_inputs(kind, inp)
@@ -330,7 +393,8 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
     if st != (0, 0):
         raise RuntimeError("device error %s in %s" % (st, name))
 
-    fl = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device) if flush else None
+    flush = flush_buf is not None
+    fl = flush_buf
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
             torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     # per-kernel start events (the library's timing hook records kev[k] before its k-th launch)
@@ -379,6 +443,27 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
             dp.reduce_param_grads(kind, grads)
     torch.cuda.synchronize()
 
+    # The same steps back to back without the flush (inputs left in L2 by the previous step):
+    # reported beside the flushed figure for workloads small enough to stay in L2.
+    warm = None
+    if flush:
+        wev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            wev[i][0].record()
+            plan.fwd(ai, y)
+            wev[i][1].record()
+            plan.bwd(ai, dy, grads)
+            if world > 1:
+                dp.reduce_param_grads(kind, grads)
+            wev[i][2].record()
+        torch.cuda.synchronize()
+        wf = statistics.mean(a.elapsed_time(b) for a, b, _ in wev)
+        wb = statistics.mean(b.elapsed_time(c) for _, b, c in wev)
+        warm = {"ms_fwd": round(wf, 5), "ms_bwd": round(wb, 5),
+                "tokens_per_s": round(tokens_of(w) * world / ((wf + wb) * 1e-3), 1)}
+
     def kernel_ms(kev, ends):
         n = len(kev[0])
         return [statistics.mean(kev[s][k].elapsed_time(kev[s][k + 1] if k + 1 < n else ends[s])
@@ -396,7 +481,9 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         t = torch.tensor([step_ms, fwd_mean, bwd_mean], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         step_ms, fwd_mean, bwd_mean = (float(v) for v in t.tolist())
-    fwd_b, bwd_b = algorithmic_bytes(kind, inp, y, grads, plan.ckpt_view().numel() * 4)  # f32 states
+    ckpt_b = plan.ckpt_view().numel() * 4  # the f32 states at the configured segment length
+    ops = operand_bytes(kind, inp, y, grads, dy, ckpt_b)
+    fwd_b, bwd_b = algorithmic_bytes(kind, ops, list(grads))
     res = {
         "workload": name, "kind": kind, "desc": NAMES[name],
         "tokens_per_step": tokens_of(w) * world,
@@ -406,24 +493,26 @@ def run_workload(name, steps, warmup, device, rank, world, flush, e2e=False, cpu
         "fwd_gbs": fwd_b / (fwd_mean * 1e-3) / 1e9, "bwd_gbs": bwd_b / (bwd_mean * 1e-3) / 1e9,
         "step_gbs": (fwd_b + bwd_b) / (step_ms * 1e-3) / 1e9,
         "launches_per_step": fwd_launch + bwd_launch,
-        "kernels_timed": kernel_table(w, fnames, kms_f, "fwd", fwd_b) + kernel_table(w, bnames, kms_b, "bwd", bwd_b),
+        "kernels_timed": kernel_table(w, fnames, kms_f, "fwd", ops, fwd_b, rates)
+                         + kernel_table(w, bnames, kms_b, "bwd", ops, bwd_b, rates),
+        "ckpt_bytes": ckpt_b, "segment": w["segment"],
         "fwd_kernels": fwd_names, "bwd_kernels": bwd_names,
         "window": (t0, t1), "wall_s": t1 - t0,
-        "peak_mem_bytes": torch.cuda.max_memory_allocated(device),
+        "peak_mem_bytes": torch.cuda.max_memory_allocated(device) - mem0,
         "io_dtype": "bf16" if y.dtype == torch.bfloat16 else "f32",
         "l2": "flushed between steps" if flush else "inputs larger than L2",
+        "l2_warm": warm,
     }
     if e2e:
         res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
     if world == 1:
         res["decode"] = run_decode(kind, ai, w)
         if kind in ("rglru", "rotlru", "s6") and not w.get("gates"):
-            res["full_state"] = run_full_state(kind, ai, dy, w, plan, steps, flush)
-    del fl
+            res["full_state"] = run_full_state(kind, ai, dy, w, plan, steps, flush_buf)
     return res
 
 
-def run_full_state(kind, ai, dy, w, plan, steps, flush):
+def run_full_state(kind, ai, dy, w, plan, steps, flush_buf):
     """The same fwd+bwd step in the library's full-state mode (every step's state stored by the
     forward, read by the backward: the design segment checkpoints replace), timed the same way;
     reported beside the default mode's checkpoint bytes and time."""
@@ -433,7 +522,7 @@ def run_full_state(kind, ai, dy, w, plan, steps, flush):
     desc.flags |= lrscan.FULL_STATE
     fp = lrscan.Plan(desc, ai[lrscan.TOKEN_INPUTS[kind][0]].device)
     y, grads = lrscan.alloc_outputs(kind, ai)
-    fl = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=y.device) if flush else None
+    fl = flush_buf
     for _ in range(2):
         fp.fwd(ai, y)
         fp.bwd(ai, dy, grads)
@@ -457,7 +546,7 @@ def run_full_state(kind, ai, dy, w, plan, steps, flush):
     ck_full, ck_seg = lrscan.ckpt_bytes(desc), lrscan.ckpt_bytes(plan.desc)
     out = {"ms_fwd": round(fwd, 5), "ms_bwd": round(bwd, 5), "state_bytes": ck_full,
            "checkpoint_bytes": ck_seg, "memory_ratio": round(ck_full / max(ck_seg, 1), 1)}
-    del fp, fl
+    del fp
     torch.cuda.empty_cache()
     return out
 
@@ -577,39 +666,43 @@ def run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w):
 
 
 # ------------------------------------------------------------------------ oracle (CPU)
-SAMPLES = {
-    # workload: (slice description, slicer of the CPU inputs, fraction of one step's tokens)
-    "rglru": "the whole workload",
-    "rglru_gated": "the whole workload",
-    "ssd": "batch row 0, heads 0-3 of 32, full L=4096",
-    "ssd_mamba2": "batch row 0, heads 0-3 of 32, full L=4096",
-    "gla": "batch row 0, heads 0-1 of 16, full L=2048",
-    "s6_zoh": "batch row 0, channels 0-127 of 2048, full L=2048",
-    "s6_bilinear": "batch row 0, channels 0-127 of 2048, full L=2048",
-    "rotlru": "batch row 0, pairs 0-31 of 2048, full L=16384",
-}
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
-def oracle_sample(name):
-    """CPU inputs of the bounded sample and the fraction of one step's tokens they represent."""
-    import torch
+def oracle_sample(name, units):
+    """CPU inputs of a bounded sample of the workload with at least `units` independent units
+    (as far as the workload has them), a description, and the fraction of one step's tokens the
+    sample represents.  Units are the oracle's parallel loop: (row, head) for SSD and GLA, batch
+    rows for S6's backward, pairs for rotlru, channels for rglru."""
     from selective_state_space_09_b200 import inputs
     w = inputs.WORKLOADS[name]
     kind = w["kind"]
+    units = max(1, int(units))
     if kind == "rglru":
-        return kind, inputs.workload(name, seed=0), 1.0, w
-    if kind == "ssd":
-        inp = inputs.workload(name, seed=0, B=1, H=4)
-        return kind, inp, (1 / w["B"]) * (4 / w["H"]), w
-    if kind == "gla":
-        inp = inputs.gla(1, w["L"], 2, w["K"], w["V"], seed=0)
-        return kind, inp, (1 / w["B"]) * (2 / w["H"]), w
+        return kind, inputs.workload(name, seed=0), 1.0, w, "the whole workload (%d channels)" % w["D"]
+    if kind in ("ssd", "gla"):
+        H = min(w["H"], units)
+        B = min(w["B"], -(-units // H))
+        if kind == "ssd":
+            inp = inputs.workload(name, seed=0, B=B, H=H)
+        else:
+            inp = inputs.gla(B, w["L"], H, w["K"], w["V"], seed=0)
+        return kind, inp, (B / w["B"]) * (H / w["H"]), w, \
+            "batch rows 0-%d, heads 0-%d of %d, full L=%d" % (B - 1, H - 1, w["H"], w["L"])
     if kind == "s6":
-        inp = inputs.s6(1, w["L"], 128, w["N"], seed=0)
-        return kind, inp, (1 / w["B"]) * (128 / w["D"]), w
+        B = min(w["B"], units)
+        inp = inputs.s6(B, w["L"], 128, w["N"], seed=0)
+        return kind, inp, (B / w["B"]) * (128 / w["D"]), w, \
+            "batch rows 0-%d, channels 0-127 of %d, full L=%d" % (B - 1, w["D"], w["L"])
     if kind == "rotlru":
-        inp = inputs.rotlru(1, w["L"], 64, seed=0)
-        return kind, inp, (1 / w["B"]) * (64 / w["D"]), w
+        K = max(32, units)
+        inp = inputs.rotlru(1, w["L"], 2 * K, seed=0)
+        return kind, inp, (1 / w["B"]) * (2 * K / w["D"]), w, \
+            "batch row 0, pairs 0-%d of %d, full L=%d" % (K - 1, w["D"] // 2, w["L"])
     raise KeyError(name)
 
 
@@ -646,27 +739,41 @@ def parallel_units(kind, inp):
     if kind == "s6":
         return inp["x"].shape[0]
     if kind in ("ssd", "gla"):
-        return inp["v" if kind == "gla" else "x"].shape[0] * inp["v" if kind == "gla" else "x"].shape[2]
+        t = inp["v" if kind == "gla" else "x"]
+        return t.shape[0] * t.shape[2]
     return 1
 
 
-def time_oracle(name, repeats=1, min_seconds=1.0):
+def time_oracle(name, threads, min_seconds=1.0):
+    """The fp64 oracle's forward + backward on a bounded sample with at least `threads` units, on
+    `threads` host threads; tokens/s scaled to the workload's tokens."""
     import oracle
-    kind, inp, frac, w = oracle_sample(name)
-    threads = oracle.get_threads()
+    kind, inp, frac, w, desc = oracle_sample(name, threads)
+    oracle.set_threads(threads)
     oracle_step(kind, inp, w)  # warm (page-in, library load)
     n, t0 = 0, time.perf_counter()
     while True:
         oracle_step(kind, inp, w)
         n += 1
         el = time.perf_counter() - t0
-        if n >= repeats and el >= min_seconds:
+        if el >= min_seconds:
             break
     per = el / n
     toks = tokens_of(w) * frac
     return {"value": toks / per, "unit": "tokens/s", "cores": min(threads, parallel_units(kind, inp)),
-            "kind": "oracle", "sample": SAMPLES[name] + " (fp64 C oracle, forward + backward, %d run(s))" % n,
+            "kind": "oracle", "sample": desc + " (fp64 C oracle, forward + backward, %d run(s))" % n,
             "seconds_per_sample": per}
+
+
+def cpu_baseline(name):
+    """The oracle at all host cores (the reported value) and at one thread."""
+    cores = host_cores()
+    allc = time_oracle(name, cores)
+    one = time_oracle(name, 1)
+    out = {k: allc[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    out["host_cores"] = cores
+    out["one_thread"] = {"value": one["value"], "unit": "tokens/s", "sample": one["sample"]}
+    return out
 
 
 # ---------------------------------------------------------------------------------- main
@@ -694,13 +801,26 @@ def built_workloads():
     return ok
 
 
+def relaunch_ranks(args):
+    """`--gpus N` with N > 1 outside a torchrun launch: start N ranks, one per GPU, through
+    torch.distributed.run on this host and return its exit status (rank 0 prints the line)."""
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(args.gpus),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=None, help="headline workload (default: ssd if built)")
+    ap.add_argument("--workload", default=None, help="headline workload (default: ssd)")
     ap.add_argument("--only-headline", action="store_true", help="skip the per-kind lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
@@ -710,9 +830,13 @@ def main():
     BATCH_OVERRIDE = args.batch
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_ranks(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print("bench: --gpus %d but WORLD_SIZE %d; timing %d rank(s)" % (args.gpus, world, world), file=sys.stderr)
 
     if args.impl == "reference":
         if rank != 0:
@@ -734,39 +858,48 @@ def main():
     others = [] if args.only_headline else [n for n in BENCH_ORDER if n in built and n != head]
 
     pk = peaks()
+    rates = measure_pipe_rates(device)
+    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MiB > L2
     props = torch.cuda.get_device_properties(device)
     sampler = ClockSampler(getattr(props, "uuid", None) and ("GPU-" + str(props.uuid)) or local)
     sampler.start()
     time.sleep(0.3)
     results = {}
     for name in [head] + others:
-        big = name == "rotlru"
-        r = run_workload(name, args.steps, args.warmup, device, rank, world, flush=not big,
-                         e2e=(name == head))
+        big = name == "rotlru"  # 10 GiB of inputs: far larger than L2, no flush needed
+        r = run_workload(name, args.steps, args.warmup, device, rank, world, None if big else flush_buf,
+                         e2e=(name == head), rates=rates)
         sampler.mark(*r["window"])
         results[name] = r
         torch.cuda.empty_cache()
     time.sleep(0.2)
     sampler.stop()
     clocks = sampler.summary()
+    del flush_buf
 
     h = results[head]
     dom_row = max(h["kernels_timed"], key=lambda r: r["ms"])
     roofline = kernel_roofline(dom_row, pk)
+    step_bytes = h["fwd_bytes"] + h["bwd_bytes"]
     roofline.update({
         "traffic": ncu_traffic(dom_row["kernel"], dom_row["pass"]), "kernel": dom_row["kernel"], "pass": dom_row["pass"],
         "algorithmic_bytes_per_launch": dom_row["bytes"], "algorithmic_flops_per_launch": dom_row["flops"],
-        "ms_per_launch": round(dom_row["ms"], 5),
-        "note": "of %s peak (burst GEMM / copy); kernel time from CUDA events the library records "
-                "before each launch on the call's stream, in a second timed loop of the same steps "
-                "(events between kernels stop the next kernel from starting early, so the headline "
-                "loop runs without them)" % pk["source"]})
+        "ms_per_launch": round(dom_row["ms"], 5), "segment": h["segment"],
+        "step": {"algorithmic_bytes": step_bytes, "ms": round(h["ms_per_step"], 5),
+                 "achieved_gbs": round(h["step_gbs"], 1), "frac": round(h["step_gbs"] / pk["hbm_gbs"], 4)},
+        "kernels": [dict(kernel_roofline(r, pk), kernel=r["kernel"], **{"pass": r["pass"], "ms": round(r["ms"], 5)})
+                    for r in h["kernels_timed"] if r["bytes"] or r["flops"]],
+        "note": "of %s peak (burst GEMM / copy); algorithmic bytes = the kernel's operands each once "
+                "(inputs, outputs, gradients, f32 checkpoints at the configured segment length; no "
+                "intermediates); kernel time from CUDA events the library records before each launch "
+                "on the call's stream, in a second timed loop of the same steps (events between kernels "
+                "stop the next kernel from starting early, so the headline loop runs without them)" % pk["source"]})
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = time_oracle(head)
-        cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        cpu = cpu_baseline(head)
     per_kind = {}
     for name, r in results.items():
+        dom = max(r["kernels_timed"], key=lambda q: q["ms"])
         per_kind[name] = {
             "desc": r["desc"], "tokens_per_s": round(r["tokens_per_s"], 1),
             "ms_fwd": round(r["ms_fwd"], 5), "ms_bwd": round(r["ms_bwd"], 5),
@@ -777,10 +910,14 @@ def main():
             "kernels": r["fwd_kernels"] + " | " + r["bwd_kernels"],
             "kernel_ms": {"%s:%d:%s" % (k["pass"], k["index"], k["kernel"]): round(k["ms"], 5)
                           for k in r["kernels_timed"]},
-            "dominant_kernel": dict(kernel_roofline(max(r["kernels_timed"], key=lambda q: q["ms"]), pk),
-                                    kernel=max(r["kernels_timed"], key=lambda q: q["ms"])["kernel"]),
+            "kernel_roofline": {"%s:%d:%s" % (k["pass"], k["index"], k["kernel"]): kernel_roofline(k, pk)
+                                for k in r["kernels_timed"] if k["bytes"] or k["flops"]},
+            "dominant_kernel": dict(kernel_roofline(dom, pk), kernel=dom["kernel"]),
             "peak_mem_gib": round(r["peak_mem_bytes"] / 2 ** 30, 3), "l2": r["l2"],
+            "segment": r["segment"], "checkpoint_bytes": r["ckpt_bytes"],
         }
+        if r.get("l2_warm"):
+            per_kind[name]["l2_warm"] = r["l2_warm"]
         if "decode" in r:
             d = dict(r["decode"])
             d["tokens_per_s"] = round(d["tokens_per_s"], 1)
@@ -802,6 +939,7 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clocks,
+        "pipe_rates": {k: (round(v, 1) if isinstance(v, float) and v > 1e6 else v) for k, v in rates.items()},
         "per_kind": per_kind,
         "src_sha": src_sha(),
     }
@@ -818,12 +956,16 @@ def inputs_L(name):
 
 
 def reference_arm(args, world):
-    """The fp64 CPU oracle on the host cores: each step is a bounded sample of the workload."""
-    import torch  # noqa: F401
-    built = built_workloads()
-    name = args.workload or ("ssd" if "ssd" in built else built[0])
+    """The fp64 CPU oracle on all host cores: each step is a bounded sample of the workload.  The
+    workload is chosen by name; nothing here loads the CUDA library."""
     import oracle
-    kind, inp, frac, w = oracle_sample(name)
+    from selective_state_space_09_b200 import inputs
+    name = args.workload or "ssd"
+    if name not in inputs.WORKLOADS:
+        raise SystemExit("unknown workload %s" % name)
+    cores = host_cores()
+    kind, inp, frac, w, desc = oracle_sample(name, cores)
+    oracle.set_threads(cores)
     for _ in range(args.warmup):
         oracle_step(kind, inp, w)
     t0 = time.perf_counter()
@@ -838,11 +980,12 @@ def reference_arm(args, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; distributions of the workload)",
-        "config": {"workload": NAMES[name], "global_batch": w["B"], "seq_len": w["L"],
-                   "parallelism": "single", "l2": "n/a (CPU)"},
+        "config": {"workload": NAMES[name], "global_batch": w["B"] * world, "seq_len": w["L"],
+                   "parallelism": "dp%d" % world if world > 1 else "single",
+                   "l2": "inputs larger than L2" if name == "rotlru" else "flushed between steps"},
         "cpu_baseline": {"value": round(v, 1), "unit": "tokens/s",
-                         "cores": min(oracle.get_threads(), parallel_units(kind, inp)), "kind": "oracle",
-                         "sample": SAMPLES[name] + " per step (fp64 C oracle, forward + backward)"},
+                         "cores": min(cores, parallel_units(kind, inp)), "kind": "oracle",
+                         "sample": desc + " per step (fp64 C oracle, forward + backward)"},
         "e2e": {"value": round(v, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))

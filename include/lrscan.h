@@ -261,6 +261,17 @@ int lr_last_launch_count(void);
 
 int lr_version(void);
 
+/* Calibration probe (benchmarks).  The pages give no rates for the arithmetic pipes a scan may be
+ * bound by; the S6 scan is bound by exponentials and fp32 FMAs rather than by memory, so its
+ * roofline needs the rate of each pipe on the part it runs on.  Enqueues one kernel on `stream`
+ * that keeps one pipe busy: which = 0 the special-function unit (ex2.approx.ftz.f32), which = 1
+ * the fp32 FMA pipe (fma.rn.f32); `blocks` x `threads` threads each run `iters` iterations of 8
+ * independent dependency chains and write one float to out[blocks * threads] (device, caller
+ * owned).  Returns the number of results the launch produces (time it with CUDA events recorded
+ * around the call; results / seconds is the pipe's rate), or -1 for invalid arguments (threads
+ * a multiple of 32 in [32, 1024], blocks and iters >= 1) or a failed launch. */
+int64_t lr_probe_pipe(int which, float *out, int blocks, int threads, int iters, void *stream);
+
 /* lr_rglru_fwd_noalloc -- the rglru forward pass for callers that cannot allocate device memory.
  * The pages have no counterpart: this entry point exists for deployment, not for the method.
  *
@@ -286,6 +297,15 @@ int lr_version(void);
  * LR_RGLRU_GATES, whose inputs this signature does not carry). */
 lr_status lr_rglru_fwd_noalloc(const lr_desc *desc, const void *a, const void *b, void *y,
                                void *ckpt, void *stream, int check);
+
+/* The device-side status of the last lr_rglru_fwd_noalloc call on the current device, for callers
+ * that enqueue it with check = 0 (it has no workspace to hand to lr_get_error).  Synchronises
+ * `stream`, then reads and clears the error record at the start of the library's array: LR_OK,
+ * LR_ERR_TIMEOUT or LR_ERR_DEVICE_CHECK (`info`, if non-NULL, receives the kernel's detail code);
+ * LR_ERR_CUDA if the synchronisation or the read failed.  Every lr_rglru_fwd_noalloc call clears
+ * the record when it starts, so a status must be read before the next call on that device is
+ * enqueued. */
+lr_status lr_rglru_noalloc_error(void *stream, int32_t *info);
 
 #ifdef __cplusplus
 }

@@ -737,14 +737,11 @@ DiagWs ws_plan(const lr_desc& d, bool bwd) {
     return w;
 }
 
+// The dynamic shared-memory limit is a per-device attribute of the function, so it is set on every
+// call (a host-side call of about a microsecond): a process may drive several devices.
 template <int KIND, typename T, bool BWD, bool FULL>
 void set_smem_attr(const void* fn) {
-    static bool done = false;  // per instantiation
-    if (!done) {
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Smem<KIND, T, BWD>::total());
-        done = true;
-    }
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem<KIND, T, BWD>::total());
 }
 
 template <int KIND, typename T>

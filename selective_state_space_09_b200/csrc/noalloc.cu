@@ -79,3 +79,20 @@ extern "C" lr_status lr_rglru_fwd_noalloc(const lr_desc* desc, const void* a, co
     if (cudaMemcpy(&err, ws, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return LR_ERR_CUDA;
     return static_cast<lr_status>(err);
 }
+
+// The device-side status of the last lr_rglru_fwd_noalloc call on the current device, for callers
+// that enqueue with check = 0: synchronises `stream`, reads the error record at the start of the
+// array and clears it (the record lr_get_error reads from a caller's workspace).  Each call of
+// lr_rglru_fwd_noalloc clears the record when it starts, so a status is lost once the next call
+// on the device is enqueued.
+extern "C" lr_status lr_rglru_noalloc_error(void* stream, int32_t* info) {
+    void* ws = nullptr;
+    lr_status s = scratch_address(&ws);
+    if (s != LR_OK) return s;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LR_ERR_CUDA;
+    WsHeader h;
+    if (cudaMemcpy(&h, ws, 8, cudaMemcpyDeviceToHost) != cudaSuccess) return LR_ERR_CUDA;
+    if (cudaMemset(ws, 0, 8) != cudaSuccess) return LR_ERR_CUDA;
+    if (info) *info = h.info;
+    return static_cast<lr_status>(h.err);
+}

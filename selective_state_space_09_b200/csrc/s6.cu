@@ -46,7 +46,7 @@ constexpr int kN = 16;                 // states per channel
 constexpr int kTPC = 2;                // threads per channel
 constexpr int kNH = kN / kTPC;         // states per thread
 constexpr int kCPW = 32 / kTPC;        // channels per warp
-constexpr int kThreads = kDB * kTPC;   // 512
+constexpr int kThreads = kDB * kTPC;   // 128
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxS = 64;              // segment rows per TMA box
 constexpr int kSub = 8;                // backward sub-block length

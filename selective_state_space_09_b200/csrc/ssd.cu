@@ -389,18 +389,13 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     return a;
 }
 
-// Number of SMs of the current device (queried once).
+// Number of SMs of the current device (queried on every call: a process may drive several devices).
 int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
-                                                          cudaSuccess && v > 0)
-            n = v;
-        else
-            n = 148;
-    }
-    return n;
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+                                                      cudaSuccess && v > 0)
+        return v;
+    return 148;
 }
 
 // Heads per output CTA (at most 16; 16 under LR_TEST_MAX_HEAD_BLOCK).  A CTA takes about 2 units

@@ -84,6 +84,8 @@ def _load():
     L.lr_version.restype = ctypes.c_int
     L.lr_step.argtypes = [pd, ctypes.POINTER(Inputs), vp, vp, vp, vp]
     L.lr_step.restype = st
+    L.lr_probe_pipe.argtypes = [ctypes.c_int, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+    L.lr_probe_pipe.restype = ctypes.c_int64
     return L
 
 
@@ -134,6 +136,17 @@ def set_launch_events(events):
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     set_launch_events._keep = arr  # the library keeps the pointer until the hook is reset
     lib.lr_set_launch_events(arr, len(events))
+
+
+def probe_pipe(which, out, blocks, threads, iters):
+    """lr_probe_pipe: one launch that keeps the special-function unit (which = "ex2") or the fp32
+    FMA pipe (which = "ffma") busy; out: f32 device tensor of blocks * threads elements.  Returns
+    the number of results the launch produces."""
+    assert out.numel() >= blocks * threads and out.dtype == torch.float32 and out.is_cuda
+    n = int(lib.lr_probe_pipe({"ex2": 0, "ffma": 1}[which], _ptr(out), blocks, threads, iters, _stream()))
+    if n < 0:
+        raise LrScanError(1, "lr_probe_pipe")
+    return n
 
 
 def _check(status, where):

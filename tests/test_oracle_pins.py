@@ -660,7 +660,7 @@ def test_planted_mistakes_are_caught(tmp_path):
         "shifted_gate": ("h = a[i] * h + b[i];", "h = (t > 0 ? a[i - D] : a[i]) * h + b[i];"),
         # rotation applied clockwise (sign of the imaginary part of lambda)
         "wrong_rotation": ("double lr = m * c, li = m * s;", "double lr = m * c, li = -m * s;"),
-        # GLA readout with the state transposed (q contracted against the value index)
+        # GLA state update without the forget gate (the decay g_t dropped)
         "gla_dropped_decay": ("St[i * V + j] = gt * St[i * V + j] + kt[i] * vt[j];",
                               "St[i * V + j] = St[i * V + j] + kt[i] * vt[j];"),
         # ZOH beta = dt instead of expm1(u)/A

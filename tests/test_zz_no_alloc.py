@@ -58,3 +58,34 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     assert f(ctypes.byref(big), p, p, p, p, None, 0) == 4          # LR_ERR_WORKSPACE
     other = lrscan.make_desc("rotlru", torch.float32, B=1, L=64, D=64, segment=64)
     assert f(ctypes.byref(other), p, p, p, p, None, 0) == 1        # not the rglru kind
+
+
+def test_noalloc_reports_a_bounded_wait_that_gave_up():
+    """The failure path through the library's array: with the test hook that makes the first
+    segment's tiles withhold their carry, the tiles of the later segments wait out their 1 s bound
+    and record LR_ERR_TIMEOUT.  check = 1 returns it; with check = 0 the error query reads it, and
+    the next call (without the hook) clears it and succeeds."""
+    from selective_state_space_09_b200 import lrscan
+    f = _noalloc(lrscan)
+    q = lrscan.lib.lr_rglru_noalloc_error
+    q.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)]
+    q.restype = ctypes.c_int
+    inp = {k: v.cuda() for k, v in inputs.rglru(1, 512, 64, seed=21).items()}
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    desc = lrscan.make_desc("rglru", torch.float32, B=1, L=512, D=64, segment=128)
+    desc.flags |= lrscan.TEST_WITHHOLD_CARRY
+    y = torch.empty_like(inp["b"])
+    ck = torch.empty((lrscan.ckpt_bytes(desc) // 4,), device="cuda")
+    args = (inp["a"].data_ptr(), inp["b"].data_ptr(), y.data_ptr(), ck.data_ptr(), stream)
+    assert f(ctypes.byref(desc), *args, 1) == 6                      # LR_ERR_TIMEOUT
+    assert f(ctypes.byref(desc), *args, 0) == 0                      # enqueued
+    info = ctypes.c_int32(0)
+    assert q(stream, ctypes.byref(info)) == 6                        # read ...
+    assert q(stream, ctypes.byref(info)) == 0                        # ... and cleared
+    desc.flags &= ~lrscan.TEST_WITHHOLD_CARRY
+    assert f(ctypes.byref(desc), *args, 1) == 0                      # the context is still usable
+    ref = lrscan.plan_for("rglru", {"a": inp["a"], "b": inp["b"]}, 128)
+    y_ref = torch.empty_like(y)
+    ref.fwd({"a": inp["a"], "b": inp["b"]}, y_ref)
+    torch.cuda.synchronize()
+    assert_close("y after the timeout", y, y_ref.cpu().double().numpy(), 1e-5)

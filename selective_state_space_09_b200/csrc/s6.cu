@@ -15,26 +15,31 @@
 // thread 840535, segment checkpointing with recomputation during the backward pass).
 //
 // Work split.  The scan is bound by the per-(t, d, n) arithmetic (one exp or reciprocal and a
-// handful of FMAs per state per step), not by HBM, so the layout keeps states in registers and
-// avoids cross-thread traffic on the recurrence: a CTA owns one batch row and 64 channels for the
-// whole sequence; kTPC = 2 threads per channel (lanes q and q + 16 of a warp) hold 8 of its 16
-// states each, so the readout sum over n is one shuffle.  (4 or 8 threads per channel give more
-// warps but repeat the per-(step, channel) work -- loads, gate, reductions, outputs -- on every
-// thread; both measured slower on the S6 workload.)
+// handful of FMAs per state per step), not by HBM, so the states stay in registers and the
+// recurrence never crosses threads: a CTA owns one batch row and 64 channels for the whole
+// sequence; kTPC = 4 threads per channel (lanes q, q + 8, q + 16, q + 24 of a warp) hold 4 of its
+// 16 states each, so the readout sum over n is two shuffles.  Four threads per channel (rather
+// than two) halve the registers a thread needs, so twice the warps fit on an SM; the per-(t, d)
+// work that every thread of a channel would repeat -- the silu(z) gate and the softplus step
+// length -- is instead split over the four lanes (lane p takes the steps t = p mod 4) and shared
+// by shuffles or shared memory.  Steps run in batches of kSub = 8: the exponentials and input
+// terms of a batch do not depend on the state, so they are formed first (32 independent
+// exponentials per thread), then the 8 dependent state updates.
 // Segments of S <= 64 steps are staged in shared memory by TMA (x, dt, z, dy as [S][64] bf16
 // tiles, B, C as [S][16]); outputs are written back into the consumed tile slots and stored with
 // TMA.  The forward pass double-buffers segments and writes the state entering each segment to the
 // checkpoint buffer.
 //
 // Backward, per segment in reverse order (the adjoint carry G stays in registers across
-// segments): (A) from the checkpoint, run the segment forward and keep the state at every 8-step
-// sub-block boundary in shared memory; (C) for each sub-block in reverse, recompute its 8 steps
-// keeping h_t and abar_t in registers, then run the adjoint recurrence
-// G_t[n] = ds_t C_t[n] + abar_{t+1} G_{t+1}[n] (ds = dy silu(z)) backwards through them and form
-// every gradient.  dB_t[n] and dC_t[n] (sums over channels) are reduced over the 16 channels of a
-// warp with a butterfly, then over the CTA's warps in a fixed order once per sub-block, giving
-// one partial per 64-channel block; dA and dD partials are per batch row.  A small kernel sums the
-// partials in a fixed order (deterministic results).
+// segments): the gate terms ds = dy silu(z) and dz / s are formed for the whole tile first; (A)
+// from the checkpoint, run the segment forward and keep the state at every 8-step sub-block
+// boundary in shared memory; (C) for each sub-block in reverse, recompute its 8 steps keeping h_t
+// and abar_t in registers, then run the adjoint recurrence
+// G_t[n] = ds_t C_t[n] + abar_{t+1} G_{t+1}[n] backwards through them and form every gradient.
+// dB_t[n] and dC_t[n] (sums over channels) are reduced over the 8 channels of a warp with a
+// butterfly, then over the CTA's warps in a fixed order once per sub-block, giving one partial per
+// 64-channel block; dA and dD partials are per batch row.  A small kernel sums the partials in a
+// fixed order (deterministic results).
 #include "common.cuh"
 #include "host_common.h"
 
@@ -43,14 +48,16 @@ namespace {
 
 constexpr int kDB = 64;                // channels per CTA
 constexpr int kN = 16;                 // states per channel
-constexpr int kTPC = 2;                // threads per channel
-constexpr int kNH = kN / kTPC;         // states per thread
-constexpr int kCPW = 32 / kTPC;        // channels per warp
-constexpr int kThreads = kDB * kTPC;   // 128
-constexpr int kWarps = kThreads / 32;
+constexpr int kTPC = 4;                // threads per channel
+constexpr int kNH = kN / kTPC;         // states per thread (4)
+constexpr int kCPW = 32 / kTPC;        // channels per warp (8)
+constexpr int kThreads = kDB * kTPC;   // 256
+constexpr int kWarps = kThreads / 32;  // 8
 constexpr int kMaxS = 64;              // segment rows per TMA box
-constexpr int kSub = 8;                // backward sub-block length
+constexpr int kSub = 8;                // step batch (forward) and backward sub-block length
 static_assert(2 * kNH == kCPW, "the dB / dC reduce-scatter over a warp's channels leaves one value per lane");
+static_assert(kSub == 2 * kTPC, "each lane of a channel takes two steps of a batch for the per-(t, d) work");
+static_assert(kSub * 32 == kThreads, "the cross-warp dB / dC reduction gives one (step, lane) pair per thread");
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float ex2(float x) {
@@ -66,14 +73,13 @@ __device__ __forceinline__ float rcp(float x) {
 __device__ __forceinline__ float sigm(float z) { return rcp(1.0f + ex2(-z * kLog2e)); }
 __device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// kNH consecutive bf16 -> float (this thread's states of a B or C row)
-__device__ __forceinline__ void ldn(const __nv_bfloat16* p, float* out) {
-#pragma unroll
-    for (int i = 0; i < kNH; i += 2) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p + i));
-        out[i] = f.x;
-        out[i + 1] = f.y;
-    }
+// kNH consecutive f32 (this thread's states of a B or C row; one 16-byte access)
+__device__ __forceinline__ void ldn(const float* p, float* out) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    out[0] = v.x;
+    out[1] = v.y;
+    out[2] = v.z;
+    out[3] = v.w;
 }
 // sum over the kTPC threads of a channel (lanes l, l + kCPW, l + 2 kCPW, ...)
 __device__ __forceinline__ float chan_sum(float x) {
@@ -101,39 +107,103 @@ struct S6Args {
 
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
 
-// dt of one step: the raw delta, or softplus(delta + bias) (SP: LR_DELTA_SOFTPLUS)
+// x and dt of the steps t0 .. t0 + kSub - 1 of a tile for channel column `dl` (x = 0 and dt = 0
+// beyond `nb` steps: such a step leaves the state unchanged and is never read back).  With the
+// softplus front-end (SP) lane part p forms dt of steps p and p + kTPC and the lanes of a channel
+// exchange them, instead of all four forming all eight.
 template <bool SP>
-__device__ __forceinline__ float step_dt(float raw, float bias) {
-    if constexpr (SP) return softplus_f(raw + bias);
-    return raw;
+__device__ __forceinline__ void load_steps(const __nv_bfloat16* X, const __nv_bfloat16* DT, int t0, int nb, int dl,
+                                           int part, int q, float bias, float* xs, float* dts) {
+#pragma unroll
+    for (int i = 0; i < kSub; ++i) xs[i] = i < nb ? bf(X + (t0 + i) * kDB + dl) : 0.0f;
+    if constexpr (!SP) {
+#pragma unroll
+        for (int i = 0; i < kSub; ++i) dts[i] = i < nb ? bf(DT + (t0 + i) * kDB + dl) : 0.0f;
+    } else {
+        float mine[kSub / kTPC];
+#pragma unroll
+        for (int r = 0; r < kSub / kTPC; ++r) {
+            const int i = part + kTPC * r;
+            mine[r] = i < nb ? softplus_f(bf(DT + (t0 + i) * kDB + dl) + bias) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kSub; ++i) dts[i] = __shfl_sync(0xffffffffu, mine[i / kTPC], q + kCPW * (i % kTPC));
+    }
 }
 
-// Per-thread constants of the discretisation for its 8 states.
+// Per-thread constants of the discretisation for its kNH states.  The per-step scale of dt
+// (log2(e) for the exponential forms, 1/2 for bilinear) is applied once per step, not per state.
 struct Disc {
-    float a2[kNH];  // bilinear: A / 2; the others (abar = e^{dt A}): A log2(e)
-    float ia[kNH];  // ZOH: 1 / A
     float A[kNH];
+    float ia[kNH];  // ZOH: 1 / A
 };
 
 template <int DISC>
-__device__ __forceinline__ void coef(const Disc& c, int j, float dt, float& ab, float& be) {
+__device__ __forceinline__ float dt_scale(float dt) {
+    return DISC == LR_DISC_BILINEAR ? 0.5f * dt : dt * kLog2e;
+}
+
+// abar and beta of one state; dsc = dt_scale(dt)
+template <int DISC>
+__device__ __forceinline__ void coef(const Disc& c, int j, float dt, float dsc, float& ab, float& be) {
     if (DISC == LR_DISC_BILINEAR) {
-        float r = rcp(fmaf(-dt, c.a2[j], 1.0f));
-        ab = fmaf(dt * c.a2[j], r, r);  // (1 + dt A/2) r
+        float r = rcp(fmaf(-dsc, c.A[j], 1.0f));
+        ab = fmaf(dsc * c.A[j], r, r);  // (1 + dt A/2) r
         be = dt * r;
     } else {
-        ab = ex2(dt * c.a2[j]);
-        be = DISC == LR_DISC_ZOH ? (ab - 1.0f) * c.ia[j] : (DISC == LR_DISC_DIRAC ? 1.0f : dt);
+        ab = ex2(dsc * c.A[j]);
+        be = DISC == LR_DISC_ZOH ? fmaf(ab, c.ia[j], -c.ia[j]) : (DISC == LR_DISC_DIRAC ? 1.0f : dt);
     }
 }
 
 // beta from abar (cheaper than a second transcendental in the backward sweep)
 template <int DISC>
 __device__ __forceinline__ float beta_of(const Disc& c, int j, float dt, float ab) {
-    if (DISC == LR_DISC_ZOH) return (ab - 1.0f) * c.ia[j];
+    if (DISC == LR_DISC_ZOH) return fmaf(ab, c.ia[j], -c.ia[j]);
     if (DISC == LR_DISC_DIRAC) return 1.0f;
     if (DISC == LR_DISC_ZOH_EULER) return dt;
     return dt * 0.5f * (ab + 1.0f);  // bilinear: dt / (1 - dt A/2) = dt (abar + 1) / 2
+}
+
+// abar and beta B x of the kSub steps of a batch (state-independent: formed before the updates);
+// Bf: the tile's B rows as f32 ([S][16])
+template <int DISC>
+__device__ __forceinline__ void batch_coefs(const Disc& c, const float* Bf, int t0, int part,
+                                            const float* xs, const float* dts, float (&ab)[kSub][kNH],
+                                            float (&bx)[kSub][kNH]) {
+#pragma unroll
+    for (int i = 0; i < kSub; ++i) {
+        const float4 B4 = *reinterpret_cast<const float4*>(Bf + (t0 + i) * kN + part * kNH);
+        const float Bv[kNH] = {B4.x, B4.y, B4.z, B4.w};
+        const float dsc = dt_scale<DISC>(dts[i]);
+#pragma unroll
+        for (int j = 0; j < kNH; ++j) {
+            float be;
+            coef<DISC>(c, j, dts[i], dsc, ab[i][j], be);
+            bx[i][j] = be * (Bv[j] * xs[i]);
+        }
+    }
+}
+
+// The B and C rows of a tile ([S][16] bf16, as TMA lands them) as f32, by all threads.
+__device__ __forceinline__ void widen_bc(const __nv_bfloat16* Bs, const __nv_bfloat16* Cs, float* Bf, float* Cf,
+                                         int nt, int tid) {
+    for (int e = tid; e < nt * kN / 2; e += kThreads) {
+        const float2 b2 = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Bs)[e]);
+        const float2 c2 = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Cs)[e]);
+        reinterpret_cast<float2*>(Bf)[e] = b2;
+        reinterpret_cast<float2*>(Cf)[e] = c2;
+    }
+}
+
+template <int DISC>
+__device__ __forceinline__ void load_disc(Disc& c, const float* A, int d, bool dok, int part) {
+#pragma unroll
+    for (int j = 0; j < kNH; ++j) {
+        float Av = dok ? A[(size_t)d * kN + part * kNH + j] : -1.0f;
+        c.A[j] = Av;
+        c.ia[j] = DISC == LR_DISC_ZOH ? 1.0f / Av : 0.0f;
+    }
 }
 
 __device__ __forceinline__ char* smem_base() {
@@ -144,21 +214,23 @@ __device__ __forceinline__ char* smem_base() {
 
 constexpr size_t kTileDT = size_t(kMaxS) * kDB * 2;  // [S][64] bf16
 constexpr size_t kTileBC = size_t(kMaxS) * kN * 2;   // [S][16] bf16
+constexpr size_t kTileF = size_t(kMaxS) * kDB * 4;   // [S][64] f32
 
 // ----------------------------------------------------------------------------------- forward
 // Shared memory per stage: X, DT, Z tiles and B, C tiles.
+constexpr size_t kTileBCf = size_t(kMaxS) * kN * 4;  // [S][16] f32
 constexpr size_t kFwdStage = 3 * kTileDT + 2 * kTileBC;
-constexpr size_t kFwdSmem = 128 + 2 * kFwdStage + 128;
+constexpr size_t kFwdSmem = 128 + 2 * kFwdStage + 2 * kTileBCf + 128;
 
 template <int DISC, bool FULL, bool SP>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mB,
               const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mY, S6Args a) {
     char* sm = smem_base();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm);  // bar[0], bar[1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int part = lane / kCPW, dl = warp * kCPW + (lane % kCPW);
+    const int part = lane / kCPW, q = lane % kCPW, dl = warp * kCPW + q;
     const int b = blockIdx.x / a.ncb, cb = blockIdx.x % a.ncb;
     const int d = cb * kDB + dl;
     const bool dok = d < a.D;
@@ -184,15 +256,11 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         issue(0, 0);
     }
     Disc c;
-#pragma unroll
-    for (int j = 0; j < kNH; ++j) {
-        float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
-        c.A[j] = A;
-        c.a2[j] = DISC == LR_DISC_BILINEAR ? 0.5f * A : A * kLog2e;
-        c.ia[j] = 1.0f / A;
-    }
+    load_disc<DISC>(c, a.A, d, dok, part);
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
     const float dbias = (SP && a.dbias && dok) ? a.dbias[d] : 0.0f;
+    float* Bf = reinterpret_cast<float*>(sm + 128 + 2 * kFwdStage);  // the stage's B, C rows as f32
+    float* Cf = Bf + kMaxS * kN;
     float h[kNH];
 #pragma unroll
     for (int j = 0; j < kNH; ++j) h[j] = 0.0f;
@@ -206,45 +274,54 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             issue(k + 1, s ^ 1);
         }
         ok = ok && mbar_wait(&bar[s], (k >> 1) & 1, a.hdr, 300);
-        if (dok && !FULL) {
-            float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + part * kNH;
-#pragma unroll
-            for (int j = 0; j < kNH; ++j) ck[j] = h[j];
-        }
+        if (dok && !FULL)
+            *reinterpret_cast<float4*>(a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + part * kNH) =
+                make_float4(h[0], h[1], h[2], h[3]);
         const int nt = min(a.S, a.L - k * a.S);
         __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(stage(s, 0));
         const __nv_bfloat16* DT = reinterpret_cast<const __nv_bfloat16*>(stage(s, 1));
         const __nv_bfloat16* Z = reinterpret_cast<const __nv_bfloat16*>(stage(s, 2));
-        const __nv_bfloat16* Bs = stageBC(s, 0);
-        const __nv_bfloat16* Cs = stageBC(s, 1);
-        if (ok) {
-            for (int t = 0; t < nt; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
-                float Bv[kNH], Cv[kNH];
-                ldn(Bs + t * kN + part * kNH, Bv);
-                ldn(Cs + t * kN + part * kNH, Cv);
-                if (FULL && dok) {  // the state entering step k S + t
-                    float4* ck = reinterpret_cast<float4*>(
-                        a.ckpt + ((((size_t)k * a.S + t) * a.B + b) * a.D + d) * kN + part * kNH);
-                    ck[0] = make_float4(h[0], h[1], h[2], h[3]);
-                    ck[1] = make_float4(h[4], h[5], h[6], h[7]);
-                }
-                float sacc = 0.0f;
+        widen_bc(stageBC(s, 0), stageBC(s, 1), Bf, Cf, nt, tid);
+        __syncthreads();
+        for (int t0 = 0; ok && t0 < nt; t0 += kSub) {
+            const int nb = min(kSub, nt - t0);
+            float xs[kSub], dts[kSub], ab[kSub][kNH], bx[kSub][kNH];
+            load_steps<SP>(X, DT, t0, nb, dl, part, q, dbias, xs, dts);
+            batch_coefs<DISC>(c, Bf, t0, part, xs, dts, ab, bx);
+            float sv[kSub];
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) {
+                float Cv[kNH];
+                ldn(Cf + (t0 + i) * kN + part * kNH, Cv);
+                if (FULL && dok && i < nb)  // the state entering step k S + t0 + i
+                    *reinterpret_cast<float4*>(
+                        a.ckpt + ((((size_t)k * a.S + t0 + i) * a.B + b) * a.D + d) * kN + part * kNH) =
+                        make_float4(h[0], h[1], h[2], h[3]);
+                float acc = 0.0f;
 #pragma unroll
                 for (int j = 0; j < kNH; ++j) {
-                    float ab, be;
-                    coef<DISC>(c, j, dt, ab, be);
-                    h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
-                    sacc = fmaf(Cv[j], h[j], sacc);
+                    h[j] = fmaf(ab[i][j], h[j], bx[i][j]);
+                    acc = fmaf(Cv[j], h[j], acc);
                 }
-                sacc = chan_sum(sacc);
-                if (part == 0) {
-                    float yv = fmaf(Dd, xv, sacc);
+                sv[i] = acc;
+            }
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) sv[i] = chan_sum(sv[i]);
+            // lane part p writes the outputs of steps p and p + kTPC (the gate formed once per (t, d))
+#pragma unroll
+            for (int r = 0; r < kSub / kTPC; ++r) {
+                const int i = part + kTPC * r;
+                float yv = 0.0f, xi = 0.0f, si = 0.0f;
+#pragma unroll
+                for (int u = 0; u < kSub; ++u)  // register select (i is lane-dependent)
+                    if (u % kTPC == part % kTPC && u / kTPC == r) { xi = xs[u]; si = sv[u]; }
+                if (i < nb) {
+                    yv = fmaf(Dd, xi, si);
                     if (a.has_z) {
-                        const float zv = bf(Z + t * kDB + dl);
+                        const float zv = bf(Z + (t0 + i) * kDB + dl);
                         yv *= zv * sigm(zv);
                     }
-                    X[t * kDB + dl] = __float2bfloat16_rn(yv);
+                    X[(t0 + i) * kDB + dl] = __float2bfloat16_rn(yv);
                 }
             }
         }
@@ -259,17 +336,22 @@ s6_fwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------------------------- backward
-// Shared memory: X, DT, Z, DY tiles, B, C tiles, sub-block boundary states, per-warp dB/dC.
+// Shared memory: X, DT, Z, DY tiles, B, C tiles (bf16 as TMA lands them, and f32), ds = dy silu(z)
+// (f32), sub-block boundary states, per-warp dB / dC of one sub-block.  After the tile's gate
+// terms are formed, the Z slot holds dz / s = dy sigma(z) (1 + z (1 - sigma(z))) in bf16 and then
+// dz itself.
 constexpr size_t kOffX = 128;
 constexpr size_t kOffB = kOffX + 4 * kTileDT;
-constexpr size_t kOffBnd = kOffB + 2 * kTileBC;
+constexpr size_t kOffBf = kOffB + 2 * kTileBC;
+constexpr size_t kOffDS = kOffBf + 2 * kTileBCf;
+constexpr size_t kOffBnd = kOffDS + kTileF;
 constexpr size_t kBndBytes = size_t(kMaxS / kSub) * kThreads * kNH * 4;
 constexpr size_t kOffRed = kOffBnd + kBndBytes;
-constexpr size_t kRedBytes = size_t(kWarps) * kSub * 2 * kN * 4;  // per-warp dB / dC of one sub-block
+constexpr size_t kRedBytes = size_t(kWarps) * kSub * 32 * 4;  // per-warp dB / dC of one sub-block
 constexpr size_t kBwdSmem = kOffRed + kRedBytes + 128;
 
 template <int DISC, bool FULL, bool SP>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mDT,
               const __grid_constant__ CUtensorMap mZ, const __grid_constant__ CUtensorMap mDY,
               const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
@@ -283,8 +365,11 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
     __nv_bfloat16* DY = reinterpret_cast<__nv_bfloat16*>(sm + kOffX + 3 * kTileDT);
     const __nv_bfloat16* Bs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB);
     const __nv_bfloat16* Cs = reinterpret_cast<const __nv_bfloat16*>(sm + kOffB + kTileBC);
+    float* Bf = reinterpret_cast<float*>(sm + kOffBf);    // [S][16] B as f32
+    float* Cf = Bf + kMaxS * kN;                           // [S][16] C as f32
+    float* DS = reinterpret_cast<float*>(sm + kOffDS);    // [S][64] ds = dy silu(z)
     float* bnd = reinterpret_cast<float*>(sm + kOffBnd);  // [sub-block][thread][kNH]
-    float* red = reinterpret_cast<float*>(sm + kOffRed);  // [warp][step of the sub-block][2][kN]
+    float* red = reinterpret_cast<float*>(sm + kOffRed);  // [warp][step of the sub-block][lane]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int part = lane / kCPW, q = lane % kCPW, dl = warp * kCPW + q;
@@ -297,13 +382,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         fence_proxy_async_smem();
     }
     Disc c;
-#pragma unroll
-    for (int j = 0; j < kNH; ++j) {
-        float A = dok ? a.A[(size_t)d * kN + part * kNH + j] : -1.0f;
-        c.A[j] = A;
-        c.a2[j] = DISC == LR_DISC_BILINEAR ? 0.5f * A : A * kLog2e;
-        c.ia[j] = 1.0f / A;
-    }
+    load_disc<DISC>(c, a.A, d, dok, part);
     const float Dd = (a.has_d && dok) ? a.Dskip[d] : 0.0f;
     const float dbias = (SP && a.dbias && dok) ? a.dbias[d] : 0.0f;
     float G[kNH], anext[kNH], dA[kNH];
@@ -329,137 +408,157 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
             tma_load_3d(const_cast<__nv_bfloat16*>(Cs), &mC, &bar[0], 0, t0, b);
         }
         float h[kNH];
-        {
-            const float* ck = a.ckpt + (((size_t)k * a.B + b) * a.D + (dok ? d : 0)) * kN + part * kNH;
+        if (!FULL && dok) {
+            const float4 v = *reinterpret_cast<const float4*>(a.ckpt + (((size_t)k * a.B + b) * a.D + d) * kN + part * kNH);
+            h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+        } else {
 #pragma unroll
-            for (int j = 0; j < kNH; ++j) h[j] = (dok && !FULL) ? ck[j] : 0.0f;
+            for (int j = 0; j < kNH; ++j) h[j] = 0.0f;
         }
         ok = ok && mbar_wait(&bar[0], phase, a.hdr, 400);
+        // gate terms of the tile, once per (t, d); B and C rows as f32
+        for (int e = tid; e < nt * kDB; e += kThreads) {
+            const float dyv = bf(DY + e);
+            if (a.has_z) {
+                const float zv = bf(Z + e);
+                const float sg = sigm(zv);
+                DS[e] = dyv * zv * sg;
+                Z[e] = __float2bfloat16_rn(dyv * sg * fmaf(zv, 1.0f - sg, 1.0f));
+            } else {
+                DS[e] = dyv;
+            }
+        }
+        widen_bc(Bs, Cs, Bf, Cf, nt, tid);
+        __syncthreads();
         const int nsb = (nt + kSub - 1) / kSub;
         // (A) segment forward, keeping sub-block boundary states (not with the full state)
         for (int sb = 0; sb < (FULL ? 0 : nsb); ++sb) {
-            float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
+            *reinterpret_cast<float4*>(bnd + ((size_t)sb * kThreads + tid) * kNH) = make_float4(h[0], h[1], h[2], h[3]);
+            if (sb + 1 == nsb) break;  // the last sub-block's end state is not needed
+            float xs[kSub], dts[kSub], ab[kSub][kNH], bx[kSub][kNH];
+            load_steps<SP>(X, DT, sb * kSub, kSub, dl, part, q, dbias, xs, dts);
+            batch_coefs<DISC>(c, Bf, sb * kSub, part, xs, dts, ab, bx);
 #pragma unroll
-            for (int j = 0; j < kNH; ++j) bp[j] = h[j];
-            const int te = min(nt, (sb + 1) * kSub);
-            for (int t = sb * kSub; t < te; ++t) {
-                const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
-                float Bv[kNH];
-                ldn(Bs + t * kN + part * kNH, Bv);
+            for (int i = 0; i < kSub; ++i)
 #pragma unroll
-                for (int j = 0; j < kNH; ++j) {
-                    float ab, be;
-                    coef<DISC>(c, j, dt, ab, be);
-                    h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
-                }
-            }
+                for (int j = 0; j < kNH; ++j) h[j] = fmaf(ab[i][j], h[j], bx[i][j]);
         }
         // (C) sub-blocks in reverse: recompute into registers, then the adjoint sweep
         for (int sb = nsb - 1; sb >= 0; --sb) {
             const int tb = sb * kSub;
             const int n = min(kSub, nt - tb);
+            // x and dt of the sub-block: kept in registers only with the softplus front-end
+            // (its dt is formed, not loaded); otherwise the sweep re-reads them from the tile
+            // (step t's row is overwritten with its gradients only after its last use)
+            float xs_sp[SP ? kSub : 1], dts_sp[SP ? kSub : 1];
             float h0[kNH], hr[kSub][kNH], ar[kSub][kNH];
-            if constexpr (!FULL) {
-                const float* bp = bnd + ((size_t)sb * kThreads + tid) * kNH;
+            {
+                float xs[kSub], dts[kSub];
+                load_steps<SP>(X, DT, tb, n, dl, part, q, dbias, xs, dts);
+                if constexpr (SP) {
 #pragma unroll
-                for (int j = 0; j < kNH; ++j) h0[j] = h[j] = bp[j];
-            } else {  // the full state: the state entering every step of the sub-block is stored
-                float hs[kSub][kNH];
-#pragma unroll
-                for (int i = 0; i < kSub; ++i) {
-                    const float4* ck = reinterpret_cast<const float4*>(
-                        a.ckpt + ((((size_t)t0 + tb + i) * a.B + b) * a.D + (dok ? d : 0)) * kN + part * kNH);
-                    const float4 v0 = (i < n && dok) ? ck[0] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float4 v1 = (i < n && dok) ? ck[1] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    hs[i][0] = v0.x; hs[i][1] = v0.y; hs[i][2] = v0.z; hs[i][3] = v0.w;
-                    hs[i][4] = v1.x; hs[i][5] = v1.y; hs[i][6] = v1.z; hs[i][7] = v1.w;
-                }
-#pragma unroll
-                for (int j = 0; j < kNH; ++j) h0[j] = hs[0][j];
-#pragma unroll
-                for (int i = 0; i < kSub; ++i) {  // h after step i from the state entering it
-                    if (i < n) {
-                        const int t = tb + i;
-                        const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
-                        float Bv[kNH];
-                        ldn(Bs + t * kN + part * kNH, Bv);
-#pragma unroll
-                        for (int j = 0; j < kNH; ++j) {
-                            float ab, be;
-                            coef<DISC>(c, j, dt, ab, be);
-                            hr[i][j] = fmaf(ab, hs[i][j], be * (Bv[j] * xv));
-                            ar[i][j] = ab;
-                        }
+                    for (int i = 0; i < kSub; ++i) {
+                        xs_sp[i] = xs[i];
+                        dts_sp[i] = dts[i];
                     }
                 }
-            }
+                float bx[kSub][kNH];
+                batch_coefs<DISC>(c, Bf, tb, part, xs, dts, ar, bx);
+                if constexpr (!FULL) {
+                    const float4 v = *reinterpret_cast<const float4*>(bnd + ((size_t)sb * kThreads + tid) * kNH);
+                    h0[0] = v.x; h0[1] = v.y; h0[2] = v.z; h0[3] = v.w;
 #pragma unroll
-            for (int i = 0; i < kSub; ++i) {
-                if (i < n && !FULL) {
-                    const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
-                    float Bv[kNH];
-                    ldn(Bs + t * kN + part * kNH, Bv);
+                    for (int i = 0; i < kSub; ++i)
 #pragma unroll
-                    for (int j = 0; j < kNH; ++j) {
-                        float ab, be;
-                        coef<DISC>(c, j, dt, ab, be);
-                        h[j] = fmaf(ab, h[j], be * (Bv[j] * xv));
-                        hr[i][j] = h[j];
-                        ar[i][j] = ab;
+                        for (int j = 0; j < kNH; ++j)
+                            hr[i][j] = fmaf(ar[i][j], i > 0 ? hr[i > 0 ? i - 1 : 0][j] : h0[j], bx[i][j]);
+                } else {  // the full state: the state entering every step of the sub-block is stored
+                    float hs[kSub][kNH];
+#pragma unroll
+                    for (int i = 0; i < kSub; ++i) {
+                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (i < n && dok)
+                            v = *reinterpret_cast<const float4*>(
+                                a.ckpt + ((((size_t)t0 + tb + i) * a.B + b) * a.D + d) * kN + part * kNH);
+                        hs[i][0] = v.x; hs[i][1] = v.y; hs[i][2] = v.z; hs[i][3] = v.w;
                     }
+#pragma unroll
+                    for (int j = 0; j < kNH; ++j) h0[j] = hs[0][j];
+#pragma unroll
+                    for (int i = 0; i < kSub; ++i)
+#pragma unroll
+                        for (int j = 0; j < kNH; ++j) hr[i][j] = fmaf(ar[i][j], hs[i][j], bx[i][j]);
+                    // the sweep reads the state entering step i > 0 as hr[i - 1], which equals the
+                    // stored one up to the rounding of the same operations
                 }
             }
 #pragma unroll
             for (int i = kSub - 1; i >= 0; --i) {
                 if (i < n) {
                     const int t = tb + i;
-                    const float xv = bf(X + t * kDB + dl), dt = step_dt<SP>(bf(DT + t * kDB + dl), dbias);
-                    const float dyv = bf(DY + t * kDB + dl);
+                    float xv, dt;
+                    if constexpr (SP) {
+                        xv = xs_sp[i];
+                        dt = dts_sp[i];
+                    } else {
+                        xv = bf(X + t * kDB + dl);
+                        dt = bf(DT + t * kDB + dl);
+                    }
+                    const float ds = DS[t * kDB + dl];
                     float Bv[kNH], Cv[kNH];
-                    ldn(Bs + t * kN + part * kNH, Bv);
-                    ldn(Cs + t * kN + part * kNH, Cv);
-                    // readout and gate
-                    float sacc = 0.0f;
+                    ldn(Bf + t * kN + part * kNH, Bv);
+                    ldn(Cf + t * kN + part * kNH, Cv);
+                    float s = 0.0f;
+                    if (a.has_z) {  // the readout s is needed only for dz = s (dz / s)
+                        float sacc = 0.0f;
 #pragma unroll
-                    for (int j = 0; j < kNH; ++j) sacc = fmaf(Cv[j], hr[i][j], sacc);
-                    sacc = chan_sum(sacc);
-                    const float s = fmaf(Dd, xv, sacc);
-                    float ds = dyv, dz = 0.0f;
-                    if (a.has_z) {
-                        const float zv = bf(Z + t * kDB + dl);
-                        const float sg = sigm(zv);
-                        ds = dyv * zv * sg;
-                        dz = dyv * s * sg * fmaf(zv, 1.0f - sg, 1.0f);
+                        for (int j = 0; j < kNH; ++j) sacc = fmaf(Cv[j], hr[i][j], sacc);
+                        s = fmaf(Dd, xv, chan_sum(sacc));
                     }
                     float v[2 * kNH];  // dB (x n), dC (x n) contributions of this channel
                     float dxa = 0.0f, dta = 0.0f;
+                    const float hdt = 0.5f * dt;
 #pragma unroll
                     for (int j = 0; j < kNH; ++j) {
                         const float ab = ar[i][j];
-                        const float be = beta_of<DISC>(c, j, dt, ab);
                         const float hp = i > 0 ? hr[i > 0 ? i - 1 : 0][j] : h0[j];
                         G[j] = fmaf(anext[j], G[j], ds * Cv[j]);
                         v[kNH + j] = ds * hr[i][j];
-                        const float u = G[j] * be;
-                        v[j] = u * xv;
-                        dxa = fmaf(u, Bv[j], dxa);
-                        const float dab = G[j] * hp;
-                        const float w = G[j] * (Bv[j] * xv);  // d loss / d beta
-                        if (DISC == LR_DISC_ZOH) {
-                            dta = fmaf(dab, c.A[j] * ab, fmaf(w, ab, dta));
-                            dA[j] = fmaf(dab, dt * ab, fmaf(w, (dt * ab - be) * c.ia[j], dA[j]));
-                        } else if (DISC == LR_DISC_ZOH_EULER) {  // d beta / d dt = 1, d beta / dA = 0
-                            dta = fmaf(dab, c.A[j] * ab, dta + w);
-                            dA[j] = fmaf(dab, dt * ab, dA[j]);
-                        } else if (DISC == LR_DISC_DIRAC) {      // beta = 1
-                            dta = fmaf(dab, c.A[j] * ab, dta);
-                            dA[j] = fmaf(dab, dt * ab, dA[j]);
-                        } else {
-                            const float r = 0.5f * (ab + 1.0f);  // 1 / (1 - dt A / 2)
-                            const float r2 = r * r;
-                            dta = fmaf(dab, c.A[j] * r2, fmaf(w, fmaf(0.5f * dt * c.A[j], r2, r), dta));
-                            dA[j] = fmaf(dab, dt * r2, fmaf(w, 0.5f * dt * dt * r2, dA[j]));
+                        const float xB = xv * Bv[j];
+                        if (DISC == LR_DISC_DIRAC) {  // beta = 1
+                            v[j] = G[j] * xv;
+                            dxa = fmaf(G[j], Bv[j], dxa);
+                            const float r = ab * (G[j] * hp);
+                            dta = fmaf(r, c.A[j], dta);
+                            dA[j] = fmaf(r, dt, dA[j]);
+                        } else if (DISC == LR_DISC_ZOH_EULER) {  // beta = dt
+                            const float Gb = G[j] * dt;
+                            v[j] = Gb * xv;
+                            dxa = fmaf(Gb, Bv[j], dxa);
+                            const float r = ab * (G[j] * hp);
+                            dta = fmaf(r, c.A[j], fmaf(G[j], xB, dta));  // + d loss / d beta
+                            dA[j] = fmaf(r, dt, dA[j]);
+                        } else if (DISC == LR_DISC_ZOH) {
+                            // with dab = G h_{t-1} (d loss / d abar) and w = G B x (d loss / d beta):
+                            // d dt = abar (dab A + w) = abar G (h_{t-1} A + B x);
+                            // d A = (dt abar G (h_{t-1} A + B x) - w beta) / A, w beta = (G beta x) B;
+                            // the 1 / A is applied once, to the sum, at the end
+                            const float be = beta_of<DISC>(c, j, dt, ab);
+                            const float Gb = G[j] * be;
+                            v[j] = Gb * xv;
+                            dxa = fmaf(Gb, Bv[j], dxa);
+                            const float r = ab * (G[j] * fmaf(hp, c.A[j], xB));
+                            dta += r;
+                            dA[j] = fmaf(-v[j], Bv[j], fmaf(dt, r, dA[j]));
+                        } else {  // bilinear, rr = 1 / (1 - dt A / 2) = (abar + 1) / 2
+                            // d dt = rr^2 A (dab + w dt / 2) + w rr;  d A = rr^2 dt (dab + w dt / 2)
+                            const float rr = 0.5f * (ab + 1.0f);
+                            const float Gb = G[j] * (dt * rr);
+                            v[j] = Gb * xv;
+                            dxa = fmaf(Gb, Bv[j], dxa);
+                            const float rm = (rr * rr) * (G[j] * fmaf(xB, hdt, hp));
+                            dta = fmaf(rm, c.A[j], fmaf(G[j] * xB, rr, dta));
+                            dA[j] = fmaf(rm, dt, dA[j]);
                         }
                         anext[j] = ab;
                     }
@@ -478,7 +577,7 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                             v[i2] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                         }
                     }
-                    red[((size_t)(warp * kSub + i) * 2 + q / kNH) * kN + part * kNH + (q % kNH)] = v[0];
+                    red[(warp * kSub + i) * 32 + lane] = v[0];
                     if (part == 0) {
                         // softplus: d delta = d dt sigma(delta + bias), and sigma(delta + bias) =
                         // 1 - e^{-dt}
@@ -486,20 +585,25 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
                         dE += ddr;
                         X[t * kDB + dl] = __float2bfloat16_rn(fmaf(ds, Dd, dxa));
                         DT[t * kDB + dl] = __float2bfloat16_rn(ddr);
-                        if (a.has_z) Z[t * kDB + dl] = __float2bfloat16_rn(dz);
+                        if (a.has_z) Z[t * kDB + dl] = __float2bfloat16_rn(s * bf(Z + t * kDB + dl));
                         dD = fmaf(ds, xv, dD);
                     }
                 }
             }
-            // this sub-block's dB / dC partial of the CTA: fixed-order sum over the warps
+            // this sub-block's dB / dC partial of the CTA: fixed-order sum over the warps, one
+            // (step, lane) pair per thread
             __syncthreads();
-            for (int e = tid; e < n * 2 * kN; e += kThreads) {
-                const int i = e / (2 * kN), r = e % (2 * kN);
-                float sum = 0.0f;
+            {
+                const int i = tid >> 5, ln = tid & 31;
+                if (i < n) {
+                    float sum = 0.0f;
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w) sum += red[((size_t)(w * kSub + i) * 2) * kN + r];
-                float* dst = (r < kN ? a.pdB : a.pdC) + (((size_t)cb * a.B + b) * a.L + t0 + tb + i) * kN + (r % kN);
-                *dst = sum;
+                    for (int w = 0; w < kWarps; ++w) sum += red[(w * kSub + i) * 32 + ln];
+                    const int p = ln / kCPW, qq = ln % kCPW;
+                    float* dst = (qq < kNH ? a.pdB : a.pdC) +
+                                 (((size_t)cb * a.B + b) * a.L + t0 + tb + i) * kN + p * kNH + (qq % kNH);
+                    *dst = sum;
+                }
             }
             __syncthreads();
         }
@@ -514,9 +618,12 @@ s6_bwd_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CU
         __syncthreads();
     }
     if (dok) {
-        float* pa = a.pdA + ((size_t)b * a.D + d) * kN + part * kNH;
-#pragma unroll
-        for (int j = 0; j < kNH; ++j) pa[j] = dA[j];
+        float4 o;
+        if (DISC == LR_DISC_ZOH)
+            o = make_float4(dA[0] * c.ia[0], dA[1] * c.ia[1], dA[2] * c.ia[2], dA[3] * c.ia[3]);
+        else
+            o = make_float4(dA[0], dA[1], dA[2], dA[3]);
+        *reinterpret_cast<float4*>(a.pdA + ((size_t)b * a.D + d) * kN + part * kNH) = o;
         if (part == 0) a.pdD[(size_t)b * a.D + d] = dD;
         if (part == 0 && SP) a.pdE[(size_t)b * a.D + d] = dE;
     }

@@ -14,9 +14,9 @@ bool chunk_supported(const lr_desc& d) {
     if (d.io != LR_BF16) return false;
     if (d.N != kKD || (d.P != 64 && d.P != 128)) return false;
     if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
-    // SSD: the decays are kept as chunk-local log sums, so abar = e^{dt A} > 0 is required (ZOH,
-    // dirac, ZOH-Euler; bilinear abar can be negative)
-    if (d.kind == LR_SSD && (d.disc == LR_DISC_BILINEAR || (d.flags & LR_HAS_Z) || d.P != 64)) return false;
+    // SSD: the decays are kept as chunk-local log sums (with a sign parity for bilinear, whose abar
+    // can be negative)
+    if (d.kind == LR_SSD && ((d.flags & LR_HAS_Z) || d.P != 64)) return false;
     return d.L <= (1 << 28) && d.H <= 4096;
 }
 

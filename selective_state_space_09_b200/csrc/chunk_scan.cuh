@@ -19,8 +19,28 @@ constexpr int kScanP = 64;                               // value columns of one
 constexpr uint32_t kScanTile = kKD * kScanP * 2;         // one 128 x 64 block of a bf16 state tile
 
 // Per-step decay of the scan: SSD with the default kernel variant (ZOH, raw dt), SSD with the
-// general one (discretisation and softplus front-end from the arguments), GLA.
-enum { kScanSsd = 0, kScanSsdGen = 1, kScanGla = 2 };
+// general one (discretisation and softplus front-end from the arguments), GLA, and SSD with the
+// bilinear discretisation (abar may be negative: a sign parity is carried beside the log
+// magnitude, see bilinear_step).
+enum { kScanSsd = 0, kScanSsdGen = 1, kScanGla = 2, kScanSsdBil = 3 };
+
+// Floor of a step's log decay: e^{-87} is still a normal fp32 number, so products of decays stay
+// finite and an exact zero decay (bilinear abar at dt A = -2) enters as e^{-87}.
+constexpr float kMinLogDecay = -87.0f;
+
+// Bilinear step (Tustin): u = dt A / 2, abar = (1 + u) / (1 - u), beta = dt / (1 - u).  abar lies
+// in (-1, 1] for A < 0 and is negative where dt |A| > 2, so products of decays are carried as a
+// log magnitude lam = log|abar| (floored at kMinLogDecay) and a sign: neg = 1 where abar < 0, and
+// the sign of a product over steps (s, t] is (-1)^(#neg in (s, t]).
+__device__ __forceinline__ void bilinear_step(float dt, float Ah, float& lam, float& beta, float& neg) {
+    const float u = 0.5f * dt * Ah;
+    const float num = 1.0f + u, den = 1.0f - u;
+    lam = fmaxf(__logf(fabsf(num)) - __logf(den), kMinLogDecay);
+    beta = dt / den;
+    neg = num < 0.0f ? 1.0f : 0.0f;
+}
+// (-1)^n for an inclusive count n of negative steps (exact small integers in fp32)
+__device__ __forceinline__ float parity_sign(float n) { return (__float2int_rn(n) & 1) ? -1.0f : 1.0f; }
 
 struct ScanArgs {
     int B, L, H, G, HpG, nchunk;  // GLA: G = H, HpG = 1
@@ -121,8 +141,8 @@ template <int NS, bool F32> struct ScanSmem {
     static constexpr size_t kStage = kRt + (size_t)kQ * kScanP * 2;  // then the Z tile
     static constexpr size_t kF32 = (size_t)NS * kStage;             // f32 state staging, 2 boxes
     static constexpr size_t kBf = kF32 + (F32 ? (size_t)kKD * kScanP * 4 : 0);  // bf16 tile staging
-    static constexpr size_t kTmp = kBf + kScanTile;                  // prep scan scratch [4][4], l_Q [4]
-    static constexpr size_t kDecP = kTmp + 128;                      // e^{l_Q}: prep -> issue [kDecRing]
+    static constexpr size_t kTmp = kBf + kScanTile;                  // prep scan scratch [4][8], l_Q and sign [8]
+    static constexpr size_t kDecP = kTmp + 256;                      // e^{l_Q}: prep -> issue [kDecRing]
     static constexpr size_t kDecF = kDecP + 4 * kDecRing;            // e^{l_Q}: issue -> fold [kDecRing]
     static constexpr size_t kDt = kDecF + 4 * kDecRing;              // dt ring [kDtRing][128][8] bf16
     static constexpr size_t kBar = kDt + (size_t)kDtRing * kQ * 16;  // full, scaled, prod, bfree, dt full / empty
@@ -146,7 +166,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                   ScanArgs a, char* __restrict__ tiles, int dir, unsigned int* ready, float* zero0, float* zero1,
                   unsigned int* zready) {
     using SM = ScanSmem<NS, F32>;
-    constexpr bool GEN = MODE == kScanSsdGen;
+    constexpr bool GEN = MODE == kScanSsdGen || MODE == kScanSsdBil;
     char* sm = smem_base1024();
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + SM::kBar);
     uint64_t* scaled = full + NS;
@@ -208,7 +228,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
         const int t = tid;
         const float Ah = MODE == kScanGla ? 0.0f : a.A[h];
         for (int k0 = 0; k0 < nk; k0 += NG) {
-            float l[NG], beta[NG], f[NG];
+            // l[j]: log decay of step t of chunk k0 + j; for bilinear l[NG + j]: its negative-step count
+            constexpr int NV = MODE == kScanSsdBil ? 2 * NG : NG;
+            float l[NV], beta[NG], f[NG];
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
                 const int k = k0 + j;
@@ -218,27 +240,36 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                 if constexpr (MODE == kScanGla) {  // lam = log g, beta = 1 (0 past L)
                     l[j] = in_seq ? __logf(raw) : 0.0f;
                     beta[j] = in_seq ? 1.0f : 0.0f;
+                } else if constexpr (MODE == kScanSsdBil) {  // log|abar|, sign count (0 past L)
+                    l[j] = beta[j] = l[NG + j] = 0.0f;
+                    if (in_seq) bilinear_step(ssd_dt<true>(a, raw, h), Ah, l[j], beta[j], l[NG + j]);
                 } else {
                     const float dtv = in_seq ? ssd_dt<GEN>(a, raw, h) : 0.0f;  // 0 past L
                     l[j] = dtv * Ah;
                     beta[j] = in_seq ? ssd_beta(disc_of<GEN>(a), l[j], dtv, Ah) : 0.0f;  // no input past L
                 }
             }
-            wg0_inclusive_sum_n<NG>(l, tmp);  // its barriers: every prep thread has read the dt slots
+            wg0_inclusive_sum_n<NV>(l, tmp);  // its barriers: every prep thread has read the dt slots
             if (t == 0) {
 #pragma unroll
                 for (int j = 0; j < NG; ++j) mbar_arrive(&dtempty[(k0 + j) % kDtRing]);
             }
             if (t == kQ - 1) {
 #pragma unroll
-                for (int j = 0; j < NG; ++j) tmp[4 * NG + j] = l[j];
+                for (int j = 0; j < NV; ++j) tmp[32 + j] = l[j];
             }
             wg_sync(0);
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
-                const float lQ2 = tmp[4 * NG + j] * kLog2e, lt2 = l[j] * kLog2e;
-                f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] : ex2(lt2);
-                if (t == 0) decp[(k0 + j) % kDecRing] = ex2(lQ2);
+                const float lQ2 = tmp[32 + j] * kLog2e, lt2 = l[j] * kLog2e;
+                // signs of the decay products (bilinear): over (t, Q] and over (0, t]
+                float sgQ = 1.0f, sgt = 1.0f;
+                if constexpr (MODE == kScanSsdBil) {
+                    sgQ = parity_sign(tmp[32 + NG + j]);
+                    sgt = parity_sign(l[NG + j]);
+                }
+                f[j] = dir > 0 ? ex2(lQ2 - lt2) * beta[j] * (sgQ * sgt) : ex2(lt2) * sgt;
+                if (t == 0) decp[(k0 + j) % kDecRing] = ex2(lQ2) * sgQ;
             }
 #pragma unroll
             for (int j = 0; j < NG; ++j) {

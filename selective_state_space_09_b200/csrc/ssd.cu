@@ -89,6 +89,50 @@ __device__ __forceinline__ float3 wg0_sum3(float x, float y, float z, float* tmp
 }
 
 
+// Kernel variants: the default one (ZOH, raw dt), the general one (dirac / ZOH-Euler and the
+// softplus front-end, from the arguments) and the bilinear one (signed decays).
+enum { kVarZoh = 0, kVarGen = 1, kVarBil = 2 };
+
+// Log decay lam, input weight beta and negative-step indicator of one step (neg: bilinear only).
+template <int VAR>
+__device__ __forceinline__ void step_decay(const SsdArgs& a, float dtv, float Ah, float& lam, float& beta,
+                                           float& neg) {
+    if constexpr (VAR == kVarBil) {
+        bilinear_step(dtv, Ah, lam, beta, neg);
+    } else {
+        lam = dtv * Ah;
+        beta = ssd_beta(disc_of<VAR == kVarGen>(a), lam, dtv, Ah);
+        neg = 0.0f;
+    }
+}
+
+// Suffix sums x_t + ... + x_127 of NV values over the 128 threads of warpgroup 0, each term added
+// to its neighbours only (no difference of partial sums; tmp: 4 * NV floats).
+template <int NV>
+__device__ __forceinline__ void wg0_suffix_sum_n(float (&x)[NV], float* tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const float y = __shfl_down_sync(0xffffffffu, x[j], o);
+            if (lane + o < 32) x[j] += y;
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) tmp[warp * NV + j] = x[j];
+    }
+    wg0_bar();
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        float add = 0.0f;
+        for (int w = 3; w > warp; --w) add += tmp[w * NV + j];
+        x[j] += add;
+    }
+    wg0_bar();
+}
+
 // ---------------------------------------------------------------------------------- outputs
 constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernels)
 
@@ -96,7 +140,7 @@ constexpr int kMaxHB = 16;  // heads per CTA at most (output and gradient kernel
 // A_h, D_h of the heads (ad[0 .. kMaxHB), ad[kMaxHB ..)).
 template <bool GEN>
 __device__ __forceinline__ void load_dts(const SsdArgs& a, float* dts, float* ad, int b, int t0, int hfirst, int nh,
-                                         int row) {
+                                         int row) {  // GEN: the softplus front-end may apply
     if (row < nh) {
         ad[row] = a.A[hfirst + row];
         ad[kMaxHB + row] = a.Dskip ? a.Dskip[hfirst + row] : 0.0f;
@@ -142,7 +186,7 @@ __device__ __forceinline__ uint32_t col_y2(int w) { return 256u + 192u * w; }
 //   issue (one thread): Y = P X (A from TMEM), Y2 = C S_in;
 //   finish: y = Y + E Y2 + D x -> the x tile -> TMA store; the freed S_in slot loads the
 //   warpgroup's next head and the x slot freed one head earlier the head after next.
-template <bool GEN>
+template <int VAR>
 __global__ void __launch_bounds__(256, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
@@ -216,7 +260,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
             bulk_load(St, stile(hfirst + wg), kTileBytes, &wbar[3]);
         }
     }
-    if (wg == 0) load_dts<GEN>(a, dts, ad, b, t0, hfirst, nh, wt);
+    if (wg == 0) load_dts<VAR != kVarZoh>(a, dts, ad, b, t0, hfirst, nh, wt);
     __syncthreads();
     if (tid == 0) {
         ok = ok && mbar_wait(&bar[0], 0, a.hdr, 710);
@@ -232,23 +276,23 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     for (int u = 0; u < nmine; ++u) {
         const int i = wg + 2 * u, xs = u % 3;
         // ---- prep: decays, column factors, P
-        float lam = 0.0f, beta = 0.0f;
-        if (t0 + wt < a.L) {
-            const float Ah = ad[i];
-            lam = dts[i * kQ + wt] * Ah;
-            beta = ssd_beta(disc_of<GEN>(a), lam, dts[i * kQ + wt], Ah);
-        }
+        float lam = 0.0f, beta = 0.0f, neg = 0.0f;
+        if (t0 + wt < a.L) step_decay<VAR>(a, dts[i * kQ + wt], ad[i], lam, beta, neg);
         const float lt2 = wg_inclusive_sum(lam, tmp, wg) * kLog2e;
+        // bilinear: sign of the decay product over (0, t]; the column factor of step s carries
+        // the sign of (0, s], so row factor x column factor has the sign of (s, t]
+        float sg = 1.0f;
+        if constexpr (VAR == kVarBil) sg = parity_sign(wg_inclusive_sum(neg, tmp, wg));
         l2s[wt] = lt2;
-        betas[wt] = beta;
+        betas[wt] = beta * sg;
         wg_sync(wg);
-        const float E = ex2(lt2);
+        const float E = ex2(lt2) * sg;
         const float Dh = ad[kMaxHB + i];
         const float l0 = l2s[32 * wq];
         for (int s = lane; s < 32 * wq; s += 32) cfw[s] = ex2(l0 - l2s[s]) * betas[s];
         __syncwarp();
         {
-            const float rf = ex2(lt2 - l0);
+            const float rf = ex2(lt2 - l0) * sg;
             const uint32_t pcol = tmem + col_p(wg) + lane_off;
 #pragma unroll 1
             for (int sb = 0; sb < 4; ++sb) {
@@ -275,8 +319,8 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const int s = 32 * sb + 2 * q;
-                        const float p0 = s <= wt ? v[2 * q] * (ex2(lt2 - l2s[s]) * betas[s]) : 0.0f;
-                        const float p1 = s + 1 <= wt ? v[2 * q + 1] * (ex2(lt2 - l2s[s + 1]) * betas[s + 1]) : 0.0f;
+                        const float p0 = s <= wt ? v[2 * q] * (ex2(lt2 - l2s[s]) * betas[s] * sg) : 0.0f;
+                        const float p1 = s + 1 <= wt ? v[2 * q + 1] * (ex2(lt2 - l2s[s + 1]) * betas[s + 1] * sg) : 0.0f;
                         __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                         pk[q] = *reinterpret_cast<uint32_t*>(&pr);
                     }
@@ -352,9 +396,11 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
     }
 }
 
-// The general kernel variant: a discretisation other than ZOH, or the softplus front-end.
-bool general_variant(const lr_desc& d) {
-    return d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS);
+// Kernel variant of a descriptor: bilinear (signed decays), the general one (dirac, ZOH-Euler or
+// the softplus front-end), or the default ZOH one.
+int variant_of(const lr_desc& d) {
+    if (d.disc == LR_DISC_BILINEAR) return kVarBil;
+    return (d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS)) ? kVarGen : kVarZoh;
 }
 
 struct SsdFwdWs {
@@ -475,7 +521,10 @@ struct GradSmem {
     static constexpr size_t kKdk = kQdq + 2 * kQ * 4;      // w x . BG [2][128]
     static constexpr size_t kDd = kKdk + 2 * kQ * 4;       // dy . x [2][128]
     static constexpr size_t kGs = kDd + 2 * kQ * 4;        // <G, S_in> partials [256]
-    static constexpr size_t kTmp = kGs + 256 * 4;          // scan scratch
+    static constexpr size_t kSg = kGs + 256 * 4;           // bilinear: sign of the decay over (0, t] [2][128]
+    static constexpr size_t kRect = kSg + 2 * kQ * 4;      // bilinear: column sums of the masked row prefixes [4][128]
+    static constexpr size_t kBase = kRect + 4 * kQ * 4;    // bilinear: row sums of R over columns 0..63 [128]
+    static constexpr size_t kTmp = kBase + kQ * 4;         // scan scratch
     static constexpr size_t kBar = kTmp + 256;             // 0 C/B, 1..2 + 7 slots, 3 phase A (+ batch 2), 4 batch 1 (dV1, BG, Y2), 5 batch 1 (dC, dB), 6 S_in/G
     static constexpr size_t kTmem = kBar + 64;
     static constexpr size_t kTicket = kTmem + 8;
@@ -503,7 +552,7 @@ constexpr int kLoader = 160;
 //   E2: dx, the inter-chunk row dots, dy scaled by E and x by w in place;
 //   batch 2: diag(E) dy S_in^T, diag(w) x G^T into dC, dB, issued with phase A of head i + 1
 //     (M = C B^T, S2 = dy x^T) while warpgroup 0 turns head i's row terms into d dt.
-template <bool GEN>
+template <int VAR>
 __global__ void __launch_bounds__(256, 1)
 ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                 const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY, SsdGradArgs ga,
@@ -525,6 +574,10 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     float* tmp = reinterpret_cast<float*>(sm + SM::kTmp);
     float* dts = reinterpret_cast<float*>(sm + SM::kDt);
     float* ad = reinterpret_cast<float*>(sm + SM::kAD);
+    float* sgall = reinterpret_cast<float*>(sm + SM::kSg);
+    float* rectp = reinterpret_cast<float*>(sm + SM::kRect);
+    float* basep = reinterpret_cast<float*>(sm + SM::kBase);
+    constexpr bool GEN = VAR != kVarZoh;
     const uint32_t sQ = smem_u32(sm + SM::kQt), sK = smem_u32(sm + SM::kKt), sS = smem_u32(sm + SM::kSt),
                    sG = smem_u32(sm + SM::kGt);
     const int tid = threadIdx.x, wg = tid >> 7, wq = (tid >> 5) & 3, lane = tid & 31;
@@ -592,15 +645,17 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         float* l2s = l2all + (i & 1) * kQ;
         float* betas = betall + (i & 1) * kQ;
         float* cf = cfall + (i & 1) * 4 * kQ;
-        float lam = 0.0f, beta = 0.0f;
-        if (t0 + row < a.L) {
-            const float Ah = ad[i];
-            lam = dts[i * kQ + row] * Ah;
-            beta = ssd_beta(disc_of<GEN>(a), lam, dts[i * kQ + row], Ah);
-        }
+        float lam = 0.0f, beta = 0.0f, neg = 0.0f;
+        if (t0 + row < a.L) step_decay<VAR>(a, dts[i * kQ + row], ad[i], lam, beta, neg);
         const float lt = wg0_inclusive_sum(lam, tmp);
+        // bilinear: betas carry the sign of the decay over (0, s] (see the output kernel)
+        float sg = 1.0f;
+        if constexpr (VAR == kVarBil) {
+            sg = parity_sign(wg0_inclusive_sum(neg, tmp));
+            sgall[(i & 1) * kQ + row] = sg;
+        }
         l2s[row] = lt * kLog2e;
-        betas[row] = beta;
+        betas[row] = beta * sg;
         wg0_bar();
 #pragma unroll
         for (int k = row; k < 4 * kQ; k += kQ) {
@@ -659,7 +714,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         if (tid == 0 && i > 0) load_sg(h);
         __syncthreads();
         // ---- E1
-        {
+        if constexpr (VAR != kVarBil) {
             const float l2r = l2s[row];
             const float rf = ex2(l2r - l2s[32 * wq]);
             float rsum = 0.0f;
@@ -725,6 +780,90 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 colp[wq * kQ + s0 + lane] = rr[0];
             }
             rowp[wg * kQ + row] = rsum;
+        } else {
+            // Bilinear: besides P, Pd and the column sums of R (for d beta), the decay gradient
+            // needs rect(t) = sum_{i >= t} sum_{s < t} R[i, s] as a sum of its own terms (every term
+            // holds the factor abar_t, which is divided out afterwards; a difference of row and
+            // column sums would leave an absolute error that the division amplifies where abar_t
+            // is near 0).  Warpgroup wg takes columns [64 wg, 64 wg + 64) in order, keeps the row's
+            // running prefix and sums the masked prefixes Q[i][t] = [i >= t] sum_{s < t} R[i, s]
+            // (s within its columns) over the rows; the columns of warpgroup 0 reach the other
+            // half through the row sums `basep`.
+            const float l2r = l2s[row];
+            const float sgr = sgall[r * kQ + row];
+            const float rf = ex2(l2r - l2s[32 * wq]) * sgr;
+            float pre = 0.0f;
+#pragma unroll 1
+            for (int sb = 2 * wg; sb < 2 * wg + 2; ++sb) {
+                const int s0 = 32 * sb;
+                if (sb > wq) {  // above the diagonal: zero rows of P and Pd
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < 32; k += 8) {
+                        *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = z;
+                        *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = z;
+                    }
+                    colp[wq * kQ + s0 + lane] = 0.0f;
+                    rectp[wq * kQ + s0 + lane] = 0.0f;
+                    continue;
+                }
+                float m[32], s2[32];
+                tc::ld16(tmem + kGM + lane_off + s0, m);
+                tc::ld16(tmem + kGM + lane_off + s0 + 16, m + 16);
+                tc::ld16(tmem + kGS2 + lane_off + s0, s2);
+                tc::ld16(tmem + kGS2 + lane_off + s0 + 16, s2 + 16);
+                tc::wait_ld();
+                float rr[32];
+                if (sb < wq) {
+                    const float* cfb = cf + wq * kQ + s0;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const float f = rf * cfb[k];
+                        const float mk = m[k];
+                        m[k] = mk * f;
+                        s2[k] *= f;
+                        rr[k] = s2[k] * mk;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int s = s0 + k;
+                        const float f = s <= row ? ex2(l2r - l2s[s]) * betas[s] * sgr : 0.0f;
+                        const float mk = m[k];
+                        m[k] = mk * f;
+                        s2[k] *= f;
+                        rr[k] = s2[k] * mk;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 32; k += 8) {
+                    *reinterpret_cast<uint4*>(Pt + tc::sw128_off(row, s0 + k, kQ)) = pack_bf16x8(m + k);
+                    *reinterpret_cast<uint4*>(Pdt + tc::sw128_off(row, s0 + k, kQ)) = pack_bf16x8(s2 + k);
+                }
+                float qv[32];  // masked exclusive row prefix: [row >= s] (pre + R[row, s0 .. s - 1])
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    qv[k] = s0 + k <= row ? pre : 0.0f;
+                    pre += rr[k];
+                }
+                // column sums over this warp's 32 rows: lane l ends with column s0 + l
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const bool up = (lane & off) != 0;
+#pragma unroll
+                    for (int k = 0; k < off; ++k) {
+                        const float send = up ? rr[k] : rr[k + off];
+                        const float keep = up ? rr[k + off] : rr[k];
+                        rr[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                        const float sendq = up ? qv[k] : qv[k + off];
+                        const float keepq = up ? qv[k + off] : qv[k];
+                        qv[k] = keepq + __shfl_xor_sync(0xffffffffu, sendq, off);
+                    }
+                }
+                colp[wq * kQ + s0 + lane] = rr[0];
+                rectp[wq * kQ + s0 + lane] = qv[0];
+            }
+            if (wg == 0) basep[row] = pre;
         }
         // S_in and G tiles of this head: <G, S_in> partial over this thread's row / columns
         ok = ok && mbar_wait(&bar[6], (uint32_t)(i & 1), a.hdr, 726);
@@ -770,8 +909,12 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
         // ---- E2
         {
             const float l2r = l2s[row];
-            const float E = ex2(l2r);
-            const float w = ex2(l2s[kQ - 1] - l2r) * betas[row];
+            float E = ex2(l2r);
+            float w = ex2(l2s[kQ - 1] - l2r) * betas[row];
+            if constexpr (VAR == kVarBil) {  // signs of the decays over (0, t] and (t, Q]
+                E *= sgall[r * kQ + row];
+                w *= sgall[r * kQ + kQ - 1];
+            }
             const float Dh = ad[kMaxHB + i];
             __nv_bfloat16* dxrow = ga.dx + (((size_t)b * a.L + min(t0 + row, a.L - 1)) * a.H + h) * kP;
             float qdq = 0.0f, kdk = 0.0f, dd = 0.0f;
@@ -839,7 +982,63 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             tc::commit(&bar[3]);
         }
         // ---- d dt, dA, dD of head i (warpgroup 0)
-        if (wg == 0) {
+        if (wg == 0 && VAR == kVarBil) {
+            // d lam_t = rect(t) + sum_{i >= t} E_i dy_i . (C S_in)_i + sum_{s < t} w_s x_s . (B G)_s
+            //           + e^{l_Q} <G, S_in>, every sum over terms that hold abar_t; d abar_t = d lam_t / abar_t
+            const int t = row;
+            const bool valid = t0 + t < a.L;
+            const float cs = (colp[t] + colp[kQ + t]) + (colp[2 * kQ + t] + colp[3 * kQ + t]);
+            const float rect = (rectp[t] + rectp[kQ + t]) + (rectp[2 * kQ + t] + rectp[3 * kQ + t]);
+            const float qi = qdqp[t] + qdqp[kQ + t];
+            const float ki = kdkp[t] + kdkp[kQ + t];
+            const float ddv = ddp[t] + ddp[kQ + t];
+            const float2 kg = wg0_sum2(0.0f, gsp[t] + gsp[kQ + t], tmp);  // <G, S_in>
+            // exclusive prefix of the w x . BG terms: shift by one row through rowp (free here)
+            rowp[t] = ki;
+            wg0_bar();
+            float kprev = t > 0 ? rowp[t - 1] : 0.0f;
+            wg0_bar();
+            kprev = wg0_inclusive_sum(kprev, tmp);
+            float suf[2] = {qi, basep[t]};
+            wg0_suffix_sum_n<2>(suf, tmp);
+            const float sgQ = sgall[r * kQ + kQ - 1];
+            const float dlam = rect + (t >= 64 ? suf[1] : 0.0f) + suf[0] + kprev + ex2(l2s[kQ - 1]) * sgQ * kg.y;
+            float dA_part = 0.0f, ddr = 0.0f;
+            if (valid) {
+                const float Ah = ad[i];
+                const float dt_raw = dts[i * kQ + t];
+                const float u = 0.5f * dt_raw * Ah;
+                const float rr = 1.0f / (1.0f - u);
+                const float ab = (1.0f + u) * rr;
+                const float bt = betas[t] * sgall[r * kQ + t];  // beta_t (positive)
+                const float dab = ab != 0.0f ? dlam / ab : 0.0f;
+                const float dbeta = bt != 0.0f ? (cs + ki) / bt : 0.0f;
+                // abar = (1 + u) / (1 - u), beta = dt / (1 - u), u = dt A / 2:
+                // d abar / d dt = A rr^2, d abar / dA = dt rr^2, d beta / d dt = rr + u rr^2,
+                // d beta / dA = dt^2 rr^2 / 2
+                const float rr2 = rr * rr;
+                ddr = dab * Ah * rr2 + dbeta * fmaf(u, rr2, rr);
+                if (softplus_of<GEN>(a)) ddr *= -expm1f(-dt_raw);
+                ga.ddt[((size_t)b * a.L + t0 + t) * a.H + h] = __float2bfloat16_rn(ddr);
+                dA_part = (dab + dbeta * 0.5f * dt_raw) * dt_raw * rr2;
+            }
+            const size_t tile = ((size_t)b * a.H + h) * a.nchunk + c;
+            if (!softplus_of<GEN>(a)) {
+                const float2 sAD = wg0_sum2(dA_part, valid ? ddv : 0.0f, tmp);
+                if (t == 0) {
+                    ga.pdA[tile] = sAD.x;
+                    ga.pdD[tile] = sAD.y;
+                }
+            } else {
+                const float3 sADE = wg0_sum3(dA_part, valid ? ddv : 0.0f, ddr, tmp);
+                if (t == 0) {
+                    ga.pdA[tile] = sADE.x;
+                    ga.pdD[tile] = sADE.y;
+                    ga.pdE[tile] = sADE.z;
+                }
+            }
+        }
+        if (wg == 0 && VAR != kVarBil) {
             const int t = row;
             const bool valid = t0 + t < a.L;
             const float cs = (colp[t] + colp[kQ + t]) + (colp[2 * kQ + t] + colp[3 * kQ + t]);
@@ -1001,9 +1200,10 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
     char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
     if (!ok) return LR_ERR_INVALID_ARG;
-    const bool gen = general_variant(d);
+    const int var = variant_of(d);
     using ScanF = ScanSmem<3, true>;
-    auto scan = gen ? chunk_scan_kernel<3, true, kScanSsdGen> : chunk_scan_kernel<3, true, kScanSsd>;
+    auto scan = var == kVarBil ? chunk_scan_kernel<3, true, kScanSsdBil>
+                : var == kVarGen ? chunk_scan_kernel<3, true, kScanSsdGen> : chunk_scan_kernel<3, true, kScanSsd>;
     cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
     note_launch("ssd_state_scan");
     CUtensorMap mS;
@@ -1020,7 +1220,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     }
     const int hb = out_heads_per_cta(d, a.nchunk);
     const int nblk_o = (a.HpG + hb - 1) / hb;
-    auto out = gen ? ssd_out_kernel<true> : ssd_out_kernel<false>;
+    auto out = var == kVarBil ? ssd_out_kernel<kVarBil> : var == kVarGen ? ssd_out_kernel<kVarGen> : ssd_out_kernel<kVarZoh>;
     cudaFuncSetAttribute(out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
     if (launch_pdl(out, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
@@ -1058,8 +1258,9 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.zready = (const unsigned int*)(ws + w.dbc);
     {
         using ScanB = ScanSmem<4, false>;
-        auto scan = general_variant(d) ? chunk_scan_kernel<4, false, kScanSsdGen>
-                                       : chunk_scan_kernel<4, false, kScanSsd>;
+        const int var = variant_of(d);
+        auto scan = var == kVarBil ? chunk_scan_kernel<4, false, kScanSsdBil>
+                    : var == kVarGen ? chunk_scan_kernel<4, false, kScanSsdGen> : chunk_scan_kernel<4, false, kScanSsd>;
         cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanB::kAlloc);
         note_launch("ssd_state_scan");
         // no f32 states in this direction (the map argument is unused)
@@ -1073,7 +1274,8 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
-    auto grad = general_variant(d) ? ssd_grad_kernel<true> : ssd_grad_kernel<false>;
+    const int var = variant_of(d);
+    auto grad = var == kVarBil ? ssd_grad_kernel<kVarBil> : var == kVarGen ? ssd_grad_kernel<kVarGen> : ssd_grad_kernel<kVarZoh>;
     cudaFuncSetAttribute(grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
     note_launch("ssd_chunk_grad");
     if (launch_pdl(grad, dim3(a.nchunk * a.B * a.G * nblk), dim3(256), GradSmem::kAlloc, st, mC, mB, mX, mdY,

@@ -73,7 +73,7 @@ def test_validation_rules(L):
     assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=256,
                chunk=64, disc="zoh") == 2                                        # chunk != 128
     assert _ok(L, kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, segment=128,
-               disc="bilinear") == 2
+               disc="bilinear") == 0                                             # signed decays
     assert _ok(L, kind="ssd", io=bf, B=2, L=64, H=32, P=64, N=128, G=3, segment=64,
                disc="zoh") == 1                                                  # H % G
     assert _ok(L, kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, segment=128, chunk=128) == 0
@@ -205,11 +205,8 @@ def test_every_gpu_test_case_passes_host_validation(L):
     for B, Lq, H, P, G in gc.SSD_CASES:
         assert _ok(L, kind="ssd", io=bf, B=B, L=Lq, H=H, P=P, N=128, G=G, segment=128, chunk=128,
                    disc="zoh", has_d=True) == 0
-    for disc in ("dirac", "zoh_euler"):
+    for disc in ("dirac", "zoh_euler", "bilinear"):  # bilinear: signed decays (log magnitude + parity)
         assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
                    disc=disc, has_d=True) == 0
-    # bilinear abar can be negative: no log-space decays, so the chunked SSD path refuses it
-    assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
-               disc="bilinear", has_d=True) == 2
     for B, Lq, H, V in gc.GLA_CASES:
         assert _ok(L, kind="gla", io=bf, B=B, L=Lq, H=H, P=V, N=128, segment=128, chunk=128) == 0

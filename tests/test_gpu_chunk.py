@@ -67,6 +67,50 @@ def test_ssd_parity_other_discretisations(B, L, H, P, G, disc):
     assert plan.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("B,L,H,P,G,dt_shift", [(1, 512, 4, 64, 1, 0.0), (2, 260, 10, 64, 2, 0.0),
+                                                 (1, 77, 8, 64, 1, 0.0), (1, 384, 12, 64, 1, 1.5)])
+def test_ssd_parity_bilinear(B, L, H, P, G, dt_shift):
+    """Bilinear (Tustin) SSD on the chunked path: abar = (1 + u) / (1 - u), u = dt A / 2, is negative
+    wherever dt |A| > 2 and passes through 0 at dt |A| = 2.  The decays are carried as a log
+    magnitude and a sign parity; the decay gradient is formed from sums whose every term holds
+    abar_t, so dividing by abar_t stays accurate near 0.  dt_shift raises the step lengths so that
+    most steps have abar < 0."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.ssd(B, L, H, P, 128, G=G, seed=B * 41 + L)
+    if dt_shift:
+        inp["delta"] = (inp["delta"].float() + dt_shift).to(torch.bfloat16)
+    u = 0.5 * inp["delta"].double() * inp["A"].double()
+    neg = float((1.0 + u < 0).double().mean())
+    assert neg > 0.05, neg  # the case exercises negative decays
+    for flags in (0, lrscan.TEST_MAX_HEAD_BLOCK):
+        y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc="bilinear", chunk=128, flags=flags)
+        ry, rck, rg = _ssd_ref(inp, "bilinear")
+        assert_close("y", y, ry, TOL)
+        assert_close("ckpt", ck.transpose(-1, -2), rck, TOL)
+        for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D")):
+            assert_close(name, gr[name], rg[ref], TOL)
+        assert disp[0] in SSD_FWD and disp[1] in SSD_BWD
+        assert plan.device_error() == (0, 0)
+
+
+def test_ssd_bilinear_softplus_front_end():
+    """Bilinear with dt = softplus(delta + bias) formed in the kernels."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.ssd(1, 300, 8, 64, 128, G=1, seed=29)
+    gen = torch.Generator().manual_seed(8)
+    inp["delta"] = (torch.randn(inp["delta"].shape, generator=gen) - 1.0).to(torch.bfloat16)
+    inp["delta_bias"] = 0.5 * torch.randn(8, generator=gen)
+    y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc="bilinear", chunk=128, flags=lrscan.DELTA_SOFTPLUS)
+    a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], None)
+    ry = oracle.ssd_fwd(*a, disc="bilinear", delta_softplus=True, delta_bias=inp["delta_bias"])
+    rg = oracle.ssd_bwd(*a, inp["dy"], disc="bilinear", delta_softplus=True, delta_bias=inp["delta_bias"])
+    assert_close("y", y, ry, TOL)
+    for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D"),
+                      ("ddelta_bias", "delta_bias")):
+        assert_close(name, gr[name], rg[ref], TOL)
+    assert plan.device_error() == (0, 0)
+
+
 def test_ssd_softplus_front_end():
     """LR_DELTA_SOFTPLUS on the chunked SSD path: gradients for the raw delta and the bias."""
     from selective_state_space_09_b200 import lrscan

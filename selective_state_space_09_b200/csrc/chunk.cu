@@ -16,7 +16,7 @@ bool chunk_supported(const lr_desc& d) {
     if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
     // SSD: the decays are kept as chunk-local log sums (with a sign parity for bilinear, whose abar
     // can be negative)
-    if (d.kind == LR_SSD && ((d.flags & LR_HAS_Z) || d.P != 64)) return false;
+    if (d.kind == LR_SSD && d.P != 64) return false;
     return d.L <= (1 << 28) && d.H <= 4096;
 }
 

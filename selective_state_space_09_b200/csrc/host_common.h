@@ -38,12 +38,12 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int esize, uint64_t d0, ui
 bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const uint64_t* dims,
                const uint64_t* strides, const uint32_t* box, bool swizzle128);
 
-// Launches `kernel` on `st` with programmatic stream serialization: it may start while the
-// previous kernel of the stream runs and must call pdl_wait before touching that kernel's outputs
-// (or anything it reads).
+// Launches `kernel` on `st` with programmatic stream serialization (launch_ex: unless
+// `programmatic` is false): it may start while the previous kernel of the stream runs and must
+// call pdl_wait before touching that kernel's outputs (or anything it reads).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args... args) {
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      bool programmatic, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -53,8 +53,13 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = programmatic ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    return launch_ex(kernel, grid, block, smem, st, true, args...);
 }
 
 // Byte offset bookkeeping for a workspace: a 256-byte header followed by regions.

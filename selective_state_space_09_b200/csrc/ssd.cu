@@ -40,6 +40,7 @@ struct SsdArgs {
     const __nv_bfloat16* dt;      // [B, L, H]
     const float* A;               // [H]
     const float* Dskip;           // [H] or null
+    const __nv_bfloat16* z;       // [B, L, H, P] or null (LR_HAS_Z: y = (S^T C + D x) silu(z))
     const float* ckpt;            // [nchunk][B][H][N][P] f32 (state entering each chunk)
     WsHeader* hdr;
     int withhold;                 // LR_TEST_WITHHOLD_CARRY (the scan never counts slot 0)
@@ -103,6 +104,34 @@ __device__ __forceinline__ void step_decay(const SsdArgs& a, float dtv, float Ah
         lam = dtv * Ah;
         beta = ssd_beta(disc_of<VAR == kVarGen>(a), lam, dtv, Ah);
         neg = 0.0f;
+    }
+}
+
+__device__ __forceinline__ float sigm_f(float z) { return 1.0f / (1.0f + ex2(-z * kLog2e)); }
+
+// Backward of the z gate, elementwise over [B, L, H, P] (8 elements per thread and step): with
+// s the readout before the gate and y = s silu(z), ds = dy silu(z) replaces dy in every
+// product of the scan and gradient kernels, and dz = s * gz with gz = dy sigma(z) (1 + z (1 -
+// sigma(z))), s being formed in the gradient kernel.
+__global__ void ssd_gate_prep(const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ z,
+                              __nv_bfloat16* __restrict__ ds, __nv_bfloat16* __restrict__ gz, size_t n8) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+        const uint4 dr = reinterpret_cast<const uint4*>(dy)[i];
+        const uint4 zr = reinterpret_cast<const uint4*>(z)[i];
+        const __nv_bfloat162* dv = reinterpret_cast<const __nv_bfloat162*>(&dr);
+        const __nv_bfloat162* zv = reinterpret_cast<const __nv_bfloat162*>(&zr);
+        uint4 o1, o2;
+        __nv_bfloat162* w1 = reinterpret_cast<__nv_bfloat162*>(&o1);
+        __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&o2);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 d2 = __bfloat1622float2(dv[e]), z2 = __bfloat1622float2(zv[e]);
+            const float s0 = sigm_f(z2.x), s1 = sigm_f(z2.y);
+            w1[e] = __floats2bfloat162_rn(d2.x * z2.x * s0, d2.y * z2.y * s1);
+            w2[e] = __floats2bfloat162_rn(d2.x * s0 * fmaf(z2.x, 1.0f - s0, 1.0f), d2.y * s1 * fmaf(z2.y, 1.0f - s1, 1.0f));
+        }
+        reinterpret_cast<uint4*>(ds)[i] = o1;
+        reinterpret_cast<uint4*>(gz)[i] = o2;
     }
 }
 
@@ -345,6 +374,9 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         ok = ok && mbar_wait(&wbar[xs], (uint32_t)((u / 3) & 1), a.hdr, 714);  // x rows read below
         tc::fence_after_sync();
         char* X = Xs + xs * kQ * 128;
+        // z gate: this row's z of the head, read straight from global memory (16 bytes per 8 columns)
+        const bool zrow = a.z && t0 + wt < a.L;
+        const __nv_bfloat16* zr = zrow ? a.z + (((size_t)b * a.L + t0 + wt) * a.H + hfirst + i) * kP : nullptr;
 #pragma unroll
         for (int v0 = 0; v0 < kP; v0 += 16) {
             float y1[16], y2[16];
@@ -356,6 +388,9 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
                 uint4* px = reinterpret_cast<uint4*>(X + tc::sw128_off(wt, v0 + hh, kQ));
                 uint4 raw = *px;
                 __nv_bfloat162* xv = reinterpret_cast<__nv_bfloat162*>(&raw);
+                uint4 zraw = make_uint4(0, 0, 0, 0);
+                if (zrow) zraw = *reinterpret_cast<const uint4*>(zr + v0 + hh);
+                const __nv_bfloat162* zv = reinterpret_cast<const __nv_bfloat162*>(&zraw);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 xf = __bfloat1622float2(xv[e]);
@@ -364,7 +399,14 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
                         o0 = fmaf(E, y2[hh + 2 * e], o0);
                         o1 = fmaf(E, y2[hh + 2 * e + 1], o1);
                     }
-                    xv[e] = __floats2bfloat162_rn(fmaf(Dh, xf.x, o0), fmaf(Dh, xf.y, o1));
+                    o0 = fmaf(Dh, xf.x, o0);
+                    o1 = fmaf(Dh, xf.y, o1);
+                    if (a.z) {  // y = s silu(z)
+                        const float2 zf = __bfloat1622float2(zv[e]);
+                        o0 *= zf.x * sigm_f(zf.x);
+                        o1 *= zf.y * sigm_f(zf.y);
+                    }
+                    xv[e] = __floats2bfloat162_rn(o0, o1);
                 }
                 *px = raw;
             }
@@ -429,6 +471,7 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     a.dt = (const __nv_bfloat16*)in.delta;
     a.A = in.A;
     a.Dskip = (d.flags & LR_HAS_DSKIP) ? in.Dskip : nullptr;
+    a.z = (d.flags & LR_HAS_Z) ? (const __nv_bfloat16*)in.z : nullptr;
     a.ckpt = (const float*)ckpt;
     a.hdr = (WsHeader*)ws;
     a.withhold = (d.flags & LR_TEST_WITHHOLD_CARRY) ? 1 : 0;
@@ -502,6 +545,8 @@ struct SsdGradArgs {
     const unsigned int* gready;  // [nchunk][B][G]: heads of the group whose G tile of the slot is written
     const unsigned int* zready;  // [nchunk][B][G]: the chunk's dB, dC rows zeroed (by the scan kernel)
     int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
+    const __nv_bfloat16* gz;  // z gate: dy sigma(z) (1 + z (1 - sigma(z))) [B, L, H, P], or null
+    __nv_bfloat16* dz;        // z gate: dz [B, L, H, P]
 };
 
 struct GradSmem {
@@ -532,8 +577,9 @@ struct GradSmem {
     static constexpr size_t kAlloc = kEnd + 1024;
     static_assert(kAlloc <= 232448, "gradient CTA exceeds the shared memory of one CTA");
 };
-// TMEM columns: dC (0), dB (128); phase A: M (256), S2 (384); phase B: dV1 (256), BG (320), Y2 (384).
-constexpr uint32_t kGdC = 0, kGdB = 128, kGM = 256, kGS2 = 384, kGdV = 256, kGBG = 320, kGY2 = 384;
+// TMEM columns: dC (0), dB (128); phase A: M (256), S2 (384); phase B: dV1 (256), BG (320), Y2 (384),
+// and with the z gate Y = P x (448).
+constexpr uint32_t kGdC = 0, kGdB = 128, kGM = 256, kGS2 = 384, kGdV = 256, kGBG = 320, kGY2 = 384, kGY = 448;
 
 // Thread that issues the gradient kernel's products after the prologue: warpgroup 1 idles while
 // they run, and an issuing thread blocks while the tensor pipe is full, so warpgroup 0 stays free
@@ -897,6 +943,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             tc::mma_tiles(tmem + kGdV, sP, 1, kQ, sO, 1, kQ, kQ, kP, kQ, 0);      // dV1 = P^T dy
             if (has_out) tc::mma_tiles(tmem + kGBG, sK, 0, kQ, sG, 1, kKD, kQ, kP, kKD, 0);  // B G
             if (has_in) tc::mma_tiles(tmem + kGY2, sQ, 0, kQ, sS, 1, kKD, kQ, kP, kKD, 0);   // C S_in
+            if (ga.gz) tc::mma_tiles(tmem + kGY, sP, 0, kQ, sX, 1, kQ, kQ, kP, kQ, 0);        // Y = P x
             tc::commit(&bar[4]);
             tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
             tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
@@ -916,7 +963,8 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 w *= sgall[r * kQ + kQ - 1];
             }
             const float Dh = ad[kMaxHB + i];
-            __nv_bfloat16* dxrow = ga.dx + (((size_t)b * a.L + min(t0 + row, a.L - 1)) * a.H + h) * kP;
+            const size_t rowoff = (((size_t)b * a.L + min(t0 + row, a.L - 1)) * a.H + h) * kP;
+            __nv_bfloat16* dxrow = ga.dx + rowoff;
             float qdq = 0.0f, kdk = 0.0f, dd = 0.0f;
 #pragma unroll
             for (int v0 = 0; v0 < 32; v0 += 16) {
@@ -926,6 +974,34 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 if (has_out) tc::ld16(tmem + kGBG + lane_off + col, bg);
                 if (has_in) tc::ld16(tmem + kGY2 + lane_off + col, y2);
                 tc::wait_ld();
+                if (ga.gz) {
+                    // z gate: s = P x + E (C S_in) + D x, the readout before the gate; dz = s gz
+                    float yv[16];
+                    tc::ld16(tmem + kGY + lane_off + col, yv);
+                    tc::wait_ld();
+                    if (t0 + row < a.L) {
+#pragma unroll
+                        for (int hh = 0; hh < 16; hh += 8) {
+                            const uint4 xr = *reinterpret_cast<const uint4*>(Xt + tc::sw128_off(row, col + hh, kQ));
+                            const uint4 gr = *reinterpret_cast<const uint4*>(ga.gz + rowoff + col + hh);
+                            const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&xr);
+                            const __nv_bfloat162* gv = reinterpret_cast<const __nv_bfloat162*>(&gr);
+                            float dzv[8];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 xf = __bfloat1622float2(xv[e]), gf = __bfloat1622float2(gv[e]);
+                                float s0 = fmaf(Dh, xf.x, yv[hh + 2 * e]), s1 = fmaf(Dh, xf.y, yv[hh + 2 * e + 1]);
+                                if (has_in) {
+                                    s0 = fmaf(E, y2[hh + 2 * e], s0);
+                                    s1 = fmaf(E, y2[hh + 2 * e + 1], s1);
+                                }
+                                dzv[2 * e] = s0 * gf.x;
+                                dzv[2 * e + 1] = s1 * gf.y;
+                            }
+                            *reinterpret_cast<uint4*>(ga.dz + rowoff + col + hh) = pack_bf16x8(dzv);
+                        }
+                    }
+                }
 #pragma unroll
                 for (int hh = 0; hh < 16; hh += 8) {
                     uint4* px = reinterpret_cast<uint4*>(Xt + tc::sw128_off(row, col + hh, kQ));
@@ -1158,7 +1234,7 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
 }
 
 struct SsdBwdWs {
-    size_t gready, dbc, flags_end, pdA, pdD, pdE, gtiles, end;  // flags first: reset every call
+    size_t gready, dbc, flags_end, pdA, pdD, pdE, gtiles, ds, gz, end;  // flags first: reset every call
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
@@ -1172,6 +1248,10 @@ SsdBwdWs bwd_plan(const lr_desc& d) {
     w.pdD = cur.take(sizeof(float) * tiles);
     w.pdE = cur.take(sizeof(float) * tiles);
     w.gtiles = cur.take((size_t)kTileBytes * tiles);
+    // z gate: ds = dy silu(z) and dz / s (bf16, [B, L, H, P] each)
+    const size_t tok = (d.flags & LR_HAS_Z) ? (size_t)d.B * d.L * d.H * d.P * 2 : 0;
+    w.ds = tok ? cur.take(tok) : 0;
+    w.gz = tok ? cur.take(tok) : 0;
     w.end = cur.off;
     return w;
 }
@@ -1247,6 +1327,19 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.pdA = (float*)(ws + w.pdA);
     ga.pdD = (float*)(ws + w.pdD);
     ga.pdE = (float*)(ws + w.pdE);
+    // z gate: ds = dy silu(z) takes dy's place in the scan and gradient kernels
+    const bool hz = (d.flags & LR_HAS_Z) != 0;
+    if (hz) {
+        ga.gz = (const __nv_bfloat16*)(ws + w.gz);
+        ga.dz = (__nv_bfloat16*)gr.dz;
+        note_launch("ssd_gate_prep");
+        const size_t n8 = (size_t)d.B * d.L * d.H * d.P / 8;
+        ssd_gate_prep<<<4 * sm_count(), 256, 0, st>>>((const __nv_bfloat16*)dy, (const __nv_bfloat16*)in.z,
+                                                      (__nv_bfloat16*)(ws + w.ds), (__nv_bfloat16*)(ws + w.gz), n8);
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+        dy = ws + w.ds;
+    }
     CUtensorMap mC, mB, mX, mdY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mdY, dy, kP, d.H, d.L, d.B, true);
@@ -1267,8 +1360,9 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         CUtensorMap mDt;
         const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
         if (!dt_tma) mDt = mC;  // not read
-        if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, mC, mdY, mC, mDt, dt_tma, scan_args(a),
-                       ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
+        // after the gate prep the scan starts only once ds is written (its loads do not wait)
+        if (launch_ex(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, !hz, mC, mdY, mC, mDt, dt_tma,
+                       scan_args(a), ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
                        ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;
         lr_status s = check_launch();

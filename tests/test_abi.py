@@ -206,7 +206,8 @@ def test_every_gpu_test_case_passes_host_validation(L):
         assert _ok(L, kind="ssd", io=bf, B=B, L=Lq, H=H, P=P, N=128, G=G, segment=128, chunk=128,
                    disc="zoh", has_d=True) == 0
     for disc in ("dirac", "zoh_euler", "bilinear"):  # bilinear: signed decays (log magnitude + parity)
-        assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
-                   disc=disc, has_d=True) == 0
+        for hz in (False, True):
+            assert _ok(L, kind="ssd", io=bf, B=1, L=512, H=4, P=64, N=128, G=1, segment=128, chunk=128,
+                       disc=disc, has_d=True, has_z=hz) == 0
     for B, Lq, H, V in gc.GLA_CASES:
         assert _ok(L, kind="gla", io=bf, B=B, L=Lq, H=H, P=V, N=128, segment=128, chunk=128) == 0

@@ -93,6 +93,28 @@ def test_ssd_parity_bilinear(B, L, H, P, G, dt_shift):
         assert plan.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("disc", ["zoh", "bilinear", "zoh_euler"])
+@pytest.mark.parametrize("B,L,H,P,G", [(1, 512, 4, 64, 1), (2, 260, 10, 64, 2), (1, 77, 8, 64, 1)])
+def test_ssd_parity_z_gate(B, L, H, P, G, disc):
+    """The silu(z) gate on the chunked SSD path: y = (C h + D x) silu(z); the backward forms
+    ds = dy silu(z) once, and dz from the readout before the gate (one more product, P x)."""
+    from selective_state_space_09_b200 import lrscan
+    inp = inputs.ssd(B, L, H, P, 128, G=G, seed=B * 43 + L, with_z=True)
+    for flags in (0, lrscan.TEST_MAX_HEAD_BLOCK):
+        y, ck, gr, plan, disp = run_gpu("ssd", inp, 128, disc=disc, chunk=128, flags=flags)
+        a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"])
+        ry, rck = oracle.ssd_fwd(*a, disc=disc, S=128)
+        rg = oracle.ssd_bwd(*a, inp["dy"], disc=disc)
+        assert_close("y", y, ry, TOL)
+        assert_close("ckpt", ck.transpose(-1, -2), rck, TOL)
+        for name, ref in (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D"),
+                          ("dz", "z")):
+            assert_close(name, gr[name], rg[ref], TOL)
+        assert disp[0] in SSD_FWD
+        assert disp[1] == "ssd_gate_prep+ssd_state_scan+ssd_chunk_grad+ssd_param_reduce"
+        assert plan.device_error() == (0, 0)
+
+
 def test_ssd_bilinear_softplus_front_end():
     """Bilinear with dt = softplus(delta + bias) formed in the kernels."""
     from selective_state_space_09_b200 import lrscan

@@ -183,8 +183,10 @@ lr_status lr_validate(const lr_desc *desc);
  * states with LR_FULL_STATE.
  * The forward pass writes it and the backward pass reads it.  0 on an invalid descriptor.
  * Layout per slot: rglru / rotlru [B, D]; s6 [B, D, N]; ssd [B, H, N, P]; gla [B, H, K, V].
- * SSD and GLA: the f32 slots are followed by a bf16 copy of every slot's per-head state blocks in
- * the library's internal tensor-core tile order (read back by the kernels only). */
+ * SSD and GLA with segment == chunk (128): the f32 slots are followed by a bf16 copy of every
+ * slot's per-head state blocks in the library's internal tensor-core tile order (read back by the
+ * kernels only).  With longer segments (a whole number of chunks) the buffer holds the f32 segment
+ * states only; the backward pass rebuilds the state entering every chunk from them. */
 size_t lr_ckpt_bytes(const lr_desc *desc);
 
 /* Bytes of scratch the forward (backward = 0) or backward (backward = 1) pass needs: per-tile

@@ -188,8 +188,10 @@ size_t lr_ckpt_bytes(const lr_desc* desc) {
     if (validate(desc) != LR_OK) return 0;
     size_t nseg = (desc->flags & LR_FULL_STATE) ? (size_t)desc->L
                                                 : (size_t)((desc->L + desc->segment - 1) / desc->segment);
-    // SSD, GLA: the f32 states are followed by a bf16 copy of each in tensor-core tile order
-    const size_t per = (desc->kind == LR_SSD || desc->kind == LR_GLA) ? sizeof(float) + 2 : sizeof(float);
+    // SSD, GLA with one chunk per segment: the f32 states are followed by a bf16 copy of each in
+    // tensor-core tile order (longer segments: the f32 states only)
+    const bool tiles = (desc->kind == LR_SSD || desc->kind == LR_GLA) && desc->segment == 128;
+    const size_t per = tiles ? sizeof(float) + 2 : sizeof(float);
     return nseg * state_elems(*desc) * per;
 }
 

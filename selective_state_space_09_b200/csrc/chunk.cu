@@ -13,7 +13,7 @@ using namespace chunkc;
 bool chunk_supported(const lr_desc& d) {
     if (d.io != LR_BF16) return false;
     if (d.N != kKD || (d.P != 64 && d.P != 128)) return false;
-    if (d.segment != kQ || (d.chunk != 0 && d.chunk != kQ)) return false;
+    if (d.segment % kQ != 0 || (d.chunk != 0 && d.chunk != kQ)) return false;  // segments of whole chunks
     // SSD: the decays are kept as chunk-local log sums (with a sign parity for bilinear, whose abar
     // can be negative)
     if (d.kind == LR_SSD && d.P != 64) return false;

@@ -52,6 +52,12 @@ struct ScanArgs {
     const float* A;               // SSD [H]
     WsHeader* hdr;
     int withhold;                 // LR_TEST_WITHHOLD_CARRY: slot 0 is never counted (failure-path test)
+    int f32_every;                // forward: the f32 state of chunk c is a checkpoint when c % f32_every == 0
+                                  // (slot c / f32_every); 0 or 1 = every chunk
+    int seg_k;                    // segment mode (dir > 0, recompute): one CTA per segment of seg_k chunks,
+                                  // its state read from s_init; 0 = one CTA walks the whole sequence
+    const float* s_init;          // segment mode: f32 state entering each segment [nseg][B*H][kKD][vd]
+    int vd;                       // value width of s_init rows
 };
 
 // beta of one step inside the sequence (lam = dt A_h): ZOH (e^{lam} - 1) / A_h, dirac 1,
@@ -183,13 +189,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
     float* decp = reinterpret_cast<float*>(sm + SM::kDecP);
     float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int half = blockIdx.x % a.halves, bh = blockIdx.x / a.halves, b = bh / a.H, h = bh % a.H;
+    const int nbh = a.B * a.H * a.halves;
+    const int seg = a.seg_k ? (int)blockIdx.x / nbh : 0;  // segment mode: this CTA's segment
+    const int bidx = (int)blockIdx.x % nbh;
+    const int half = bidx % a.halves, bh = bidx / a.halves, b = bh / a.H, h = bh % a.H;
     const int g = h / a.HpG, rsel = MODE == kScanGla ? h : g;  // R: per group (SSD) or head (GLA)
     const int hx = h & 7;  // this head's column of a dt ring row
     const size_t slot_bytes = (size_t)kScanTile * a.halves;  // one bf16 state tile, all halves
     const int BH = a.B * a.H;
-    const int nk = a.nchunk - 1;  // chunks with a product
-    auto chunk_of = [&](int k) { return dir > 0 ? k : a.nchunk - 1 - k; };
+    // chunks this CTA covers: the whole sequence, or (segment mode) chunks c_first .. c_first + ncs - 1
+    const int c_first = a.seg_k ? seg * a.seg_k : 0;
+    const int ncs = a.seg_k ? min(a.seg_k, a.nchunk - c_first) : a.nchunk;
+    const int nk = ncs - 1;  // chunks with a product
+    auto chunk_of = [&](int k) { return dir > 0 ? c_first + k : a.nchunk - 1 - k; };
     auto stage = [&](int k) { return sm + (size_t)(k % NS) * SM::kStage; };
     auto load = [&](int k) {
         char* st = stage(k);
@@ -394,11 +406,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
         if (ready && lane == 0) {
             int next = 0;
             unsigned long long t0 = global_ns();
-            while (next < a.nchunk) {
+            while (next < ncs) {
                 const int done = ld_acquire_cta(pubdone);
                 if (done >= next) {
                     for (; next <= done; ++next) {
-                        const int slot = dir > 0 ? next : a.nchunk - 1 - next;
+                        const int slot = dir > 0 ? c_first + next : a.nchunk - 1 - next;
                         if (!(a.withhold && slot == 0)) red_release_add(&ready[((size_t)slot * a.B + b) * a.G + g], 1u);
                     }
                     t0 = global_ns();
@@ -424,8 +436,21 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
             st_release_cta(pubdone, q);
         };
         float S[kScanP];
+        if (a.s_init) {  // segment mode: the checkpointed state entering the segment, row n
+            const float4* src = reinterpret_cast<const float4*>(
+                a.s_init + (((size_t)seg * BH + bh) * kKD + n) * a.vd + kScanP * half);
 #pragma unroll
-        for (int i = 0; i < kScanP; ++i) S[i] = 0.0f;
+            for (int i = 0; i < kScanP / 4; ++i) {
+                const float4 v = src[i];
+                S[4 * i] = v.x;
+                S[4 * i + 1] = v.y;
+                S[4 * i + 2] = v.z;
+                S[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kScanP; ++i) S[i] = 0.0f;
+        }
         pdl_wait();  // the previous kernel of the stream may still read the slots
         // S into slot c through the staging buffers (free: the copies of the previous slot have
         // read them before the first barrier)
@@ -438,7 +463,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                 bulk_wait_read_all();
             }
             wg_sync(1);
-            if constexpr (F32) {
+            const int every = a.f32_every > 1 ? a.f32_every : 1;
+            const bool f32_slot = F32 && c % every == 0;  // a checkpoint slot (forward)
+            if (f32_slot) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     char* box = sm + SM::kF32 + j * (kKD * 128);  // columns 32 j .. 32 j + 31
@@ -455,9 +482,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
             fence_proxy_async_smem();
             wg_sync(1);
             if (fl) {
-                if constexpr (F32) {
-                    tma_store_4d(&mS, sm + SM::kF32, 64 * half, 0, bh, c);
-                    tma_store_4d(&mS, sm + SM::kF32 + kKD * 128, 64 * half + 32, 0, bh, c);
+                if (f32_slot) {
+                    tma_store_4d(&mS, sm + SM::kF32, 64 * half, 0, bh, c / every);
+                    tma_store_4d(&mS, sm + SM::kF32 + kKD * 128, 64 * half + 32, 0, bh, c / every);
                 }
                 bulk_store(tiles + (size_t)c * BH * slot_bytes + (size_t)bh * slot_bytes + (size_t)half * kScanTile,
                            sm + SM::kBf, kScanTile);
@@ -466,7 +493,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
             pub2 = pub1;
             pub1 = nput++;
         };
-        put(dir > 0 ? 0 : a.nchunk - 1);
+        put(dir > 0 ? c_first : a.nchunk - 1);
         for (int k = 0; k < nk; ++k) {
             const int buf = k % kScanBufs;
             ok = ok && mbar_wait(&prod[buf], (uint32_t)((k / kScanBufs) & 1), a.hdr, 744);

@@ -235,6 +235,8 @@ struct GlaGradArgs {
     const char* stiles;      // [nchunk][B][H] bf16 tiles of the entering states
     const char* gtiles;      // [nchunk][B][H] bf16 tiles of the adjoint states
     const unsigned int* gready;  // [nchunk][B][H]: halves of the slot's G tile written (by the scan kernel)
+    const unsigned int* sready;  // [nchunk][B][H]: halves of the recomputed S_in tile written, or null (one
+                                 // chunk per segment: the tiles come with the checkpoint)
     int halves;
     __nv_bfloat16* dq;       // [B, L, H, K]
     __nv_bfloat16* dk;
@@ -311,7 +313,10 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     // the scan are done); polled here by a thread of warpgroup 1, idle while warpgroup 0 forms the
     // decays, and no global write of this kernel comes before the barrier below
     // (a timeout is recorded in the workspace; the kernel finishes)
-    if (tid == 224) wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
+    if (tid == 224) {
+        wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
+        if (ga.sready) wait_count(&ga.sready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 830);
+    }
     // decays (warpgroup 0), column factors cf[w][s] = e^{l_{32 w} - l_s} (s < 32 w)
     if (wg == 0) l2s[row] = wg0_inclusive_sum(gla_lam(a, b, h, t0 + row), tmp) * kLog2e;
     __syncthreads();
@@ -586,17 +591,26 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
     }
 }
 
+// Chunks per checkpoint segment.  With one chunk per segment the checkpoint buffer also holds the
+// bf16 tile copy of every state; with longer segments it holds the f32 segment states only, the
+// forward pass keeps the tiles of every chunk in its workspace and the backward pass recomputes
+// them from the segment states.
+int chunks_per_segment(const lr_desc& d) { return d.segment / kQ; }
+
 struct GlaWs {
-    size_t ready, flags_end, gtiles, end;  // the slot flags first (reset every call)
+    size_t ready, sready, flags_end, gtiles, stiles, end;  // the slot flags first (reset every call)
 };
 GlaWs gla_plan(const lr_desc& d, bool bwd) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     const size_t tiles = (size_t)d.B * d.H * nchunk;
+    const bool seg = chunks_per_segment(d) > 1;
     WsCursor cur;
     GlaWs w{};
     w.ready = cur.take(sizeof(unsigned int) * tiles * (size_t)(d.P / kScanP));
+    if (bwd && seg) w.sready = cur.take(sizeof(unsigned int) * tiles);
     w.flags_end = cur.off;
     if (bwd) w.gtiles = cur.take((size_t)2 * tiles * kKD * d.P);
+    if (seg) w.stiles = cur.take((size_t)2 * tiles * kKD * d.P);
     w.end = cur.off;
     return w;
 }
@@ -626,25 +640,44 @@ ScanArgs scan_args(const GlaArgs& a, int VD) {
     s.dt = a.g;
     s.hdr = a.hdr;
     s.withhold = a.withhold;
+    s.f32_every = 1;
     return s;
 }
 
 // The chunk-state scan over (row, head, 64 value columns): dir > 0 folds K^T diag(w) V into the
-// entering states (f32 checkpoint slots and bf16 tiles); dir < 0 folds Q^T diag(E) dO into the
-// adjoint states (bf16 tiles).  Each slot half is flagged in `ready` once written.
+// entering states (f32 checkpoint slots every `kseg` chunks, bf16 tiles of every chunk); dir < 0
+// folds Q^T diag(E) dO into the adjoint states (bf16 tiles).  With `recompute` (dir > 0, kseg > 1)
+// one CTA per (segment, row, head, half) rebuilds the tiles of its segment's chunks from the f32
+// segment state in `ckpt`.  Each slot half is flagged in `ready` once written.
 template <int VD>
 lr_status gla_scan(const lr_desc& d, const GlaArgs& a, const CUtensorMap& mR, const CUtensorMap& mZ, void* ckpt,
-                   char* tiles, int dir, unsigned int* ready, cudaStream_t st) {
+                   char* tiles, int dir, unsigned int* ready, int kseg, bool recompute, cudaStream_t st) {
+    const int nseg = (a.nchunk + kseg - 1) / kseg;
     CUtensorMap mS, mDt;
-    if (dir > 0 && !map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk, VD)) return LR_ERR_INVALID_ARG;
-    if (dir < 0) mS = mR;  // no f32 states in this direction
+    if (dir > 0 && !recompute && !map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, nseg, VD)) return LR_ERR_INVALID_ARG;
+    if (dir < 0 || recompute) mS = mR;  // no f32 states written
     const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, a.g) ? 1 : 0;
     if (!dt_tma) mDt = mR;  // not read
-    const ScanArgs sa = scan_args(a, VD);
+    ScanArgs sa = scan_args(a, VD);
+    cudaError_t e;
+    if (recompute) {
+        sa.seg_k = kseg;
+        sa.s_init = (const float*)ckpt;
+        sa.vd = VD;
+        using SR = ScanSmem<1, false>;
+        cudaFuncSetAttribute(chunk_scan_kernel<1, false, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SR::kAlloc);
+        note_launch("gla_state_recompute");
+        e = launch_pdl(chunk_scan_kernel<1, false, kScanGla>, dim3((unsigned)(nseg * a.B * a.H * sa.halves)),
+                       dim3(kScanThreads), SR::kAlloc, st, mR, mZ, mS, mDt, dt_tma, sa, tiles, +1, ready,
+                       (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr);
+        if (e != cudaSuccess) return LR_ERR_CUDA;
+        return check_launch();
+    }
     const dim3 grid((unsigned)(a.B * a.H * sa.halves));
     note_launch("gla_state_scan");
-    cudaError_t e;
     if (dir > 0) {
+        sa.f32_every = kseg;  // f32 checkpoints at segment starts only
         using SF = ScanSmem<3, true>;
         cudaFuncSetAttribute(chunk_scan_kernel<3, true, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SF::kAlloc);
@@ -669,9 +702,10 @@ lr_status gla_fwd_t(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, 
     if (!(map4(&mQ, in.q, kKD, d.H, d.L, d.B, true) && map4(&mK, in.k, kKD, d.H, d.L, d.B, true) &&
           map4(&mV, in.v, VD, d.H, d.L, d.B, true) && map4(&mO, y, VD, d.H, d.L, d.B, true)))
         return LR_ERR_INVALID_ARG;
-    char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float);
+    const int kseg = chunks_per_segment(d);
+    char* stiles = kseg == 1 ? (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float) : ws + w.stiles;
     unsigned int* ready = (unsigned int*)(ws + w.ready);
-    lr_status s = gla_scan<VD>(d, a, mK, mV, ckpt, stiles, +1, ready, st);
+    lr_status s = gla_scan<VD>(d, a, mK, mV, ckpt, stiles, +1, ready, kseg, false, st);
     if (s != LR_OK) return s;
     cudaFuncSetAttribute(gla_out_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GOutSmem<VD>::kAlloc);
     note_launch("gla_chunk_out");
@@ -688,7 +722,10 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
     GlaGradArgs ga{};
     ga.a = gla_args(d, in, ws);
     const GlaArgs& a = ga.a;
-    ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float);
+    const int kseg = chunks_per_segment(d);
+    ga.stiles = kseg == 1 ? (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * VD * sizeof(float)
+                          : (const char*)(ws + w.stiles);
+    ga.sready = kseg > 1 ? (const unsigned int*)(ws + w.sready) : nullptr;
     ga.gtiles = ws + w.gtiles;
     ga.gready = (const unsigned int*)(ws + w.ready);
     ga.halves = VD / kScanP;
@@ -700,7 +737,13 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
     if (!(map4(&mQ, in.q, kKD, d.H, d.L, d.B, true) && map4(&mK, in.k, kKD, d.H, d.L, d.B, true) &&
           map4(&mV, in.v, VD, d.H, d.L, d.B, true) && map4(&mO, dy, VD, d.H, d.L, d.B, true)))
         return LR_ERR_INVALID_ARG;
-    lr_status s = gla_scan<VD>(d, a, mQ, mO, nullptr, ws + w.gtiles, -1, (unsigned int*)(ws + w.ready), st);
+    lr_status s;
+    if (kseg > 1) {  // the states entering every chunk, rebuilt from the f32 segment states
+        s = gla_scan<VD>(d, a, mK, mV, const_cast<void*>(ckpt), ws + w.stiles, +1, (unsigned int*)(ws + w.sready),
+                         kseg, true, st);
+        if (s != LR_OK) return s;
+    }
+    s = gla_scan<VD>(d, a, mQ, mO, nullptr, ws + w.gtiles, -1, (unsigned int*)(ws + w.ready), kseg, false, st);
     if (s != LR_OK) return s;
     cudaFuncSetAttribute(gla_grad_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GGradSmem<VD>::kAlloc);
     note_launch("gla_chunk_grad");

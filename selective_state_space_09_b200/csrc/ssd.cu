@@ -63,6 +63,7 @@ __host__ ScanArgs scan_args(const SsdArgs& a) {
     s.A = a.A;
     s.hdr = a.hdr;
     s.withhold = a.withhold;
+    s.f32_every = 1;
     return s;
 }
 
@@ -445,14 +446,23 @@ int variant_of(const lr_desc& d) {
     return (d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS)) ? kVarGen : kVarZoh;
 }
 
+// Chunks per checkpoint segment (the segment is a multiple of the chunk).  With one chunk per
+// segment the checkpoint buffer also holds the bf16 tile copy of every state the tensor cores
+// read; with longer segments it holds the f32 segment states only, the forward pass keeps the
+// tiles of every chunk in its workspace, and the backward pass recomputes them from the segment
+// states.
+int chunks_per_segment(const lr_desc& d) { return d.segment / kQ; }
+
 struct SsdFwdWs {
-    size_t ready, end;  // after the header: the slot flags of the scan kernel (reset every call)
+    size_t ready, flags_end, stiles, end;  // after the header: the slot flags of the scan kernel (reset every call)
 };
 SsdFwdWs fwd_plan(const lr_desc& d) {
     WsCursor cur;
     SsdFwdWs w;
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     w.ready = cur.take(sizeof(unsigned int) * nchunk * d.B * d.H);
+    w.flags_end = cur.off;
+    w.stiles = chunks_per_segment(d) > 1 ? cur.take((size_t)kTileBytes * nchunk * d.B * d.H) : 0;
     w.end = cur.off;
     return w;
 }
@@ -544,6 +554,8 @@ struct SsdGradArgs {
     float* pdE;            // [B][H][nchunk] partials of d bias (LR_DELTA_SOFTPLUS)
     const unsigned int* gready;  // [nchunk][B][G]: heads of the group whose G tile of the slot is written
     const unsigned int* zready;  // [nchunk][B][G]: the chunk's dB, dC rows zeroed (by the scan kernel)
+    const unsigned int* sready;  // [nchunk][B][G]: heads whose recomputed S_in tile is written, or null
+                                 // (one chunk per segment: the tiles come with the checkpoint)
     int accumulate;        // dB / dC: 1 = reduction-add (several head blocks per group), 0 = store
     const __nv_bfloat16* gz;  // z gate: dy sigma(z) (1 + z (1 - sigma(z))) [B, L, H, P], or null
     __nv_bfloat16* dz;        // z gate: dz [B, L, H, P]
@@ -726,6 +738,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
     if (tid == 0) {
         // (a timeout is recorded in the workspace; the kernel finishes)
         wait_count(&ga.gready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 728);
+        if (ga.sready) wait_count(&ga.sready[((size_t)c * a.B + b) * a.G + g], (unsigned int)a.HpG, a.hdr, 730);
         fence_proxy_async_global();
         load_sg(hfirst);
     }
@@ -1234,15 +1247,17 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
 }
 
 struct SsdBwdWs {
-    size_t gready, dbc, flags_end, pdA, pdD, pdE, gtiles, ds, gz, end;  // flags first: reset every call
+    size_t gready, dbc, sready, flags_end, pdA, pdD, pdE, gtiles, ds, gz, stiles, end;  // flags first: reset every call
 };
 SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t nchunk = (size_t)((d.L + kQ - 1) / kQ);
     const size_t tiles = (size_t)d.B * d.H * nchunk;
+    const bool recompute = chunks_per_segment(d) > 1;
     WsCursor cur;
     SsdBwdWs w;
     w.gready = cur.take(sizeof(unsigned int) * tiles);
     w.dbc = cur.take(sizeof(unsigned int) * nchunk * d.B * d.G);
+    w.sready = recompute ? cur.take(sizeof(unsigned int) * nchunk * d.B * d.G) : 0;
     w.flags_end = cur.off;
     w.pdA = cur.take(sizeof(float) * tiles);
     w.pdD = cur.take(sizeof(float) * tiles);
@@ -1252,6 +1267,8 @@ SsdBwdWs bwd_plan(const lr_desc& d) {
     const size_t tok = (d.flags & LR_HAS_Z) ? (size_t)d.B * d.L * d.H * d.P * 2 : 0;
     w.ds = tok ? cur.take(tok) : 0;
     w.gz = tok ? cur.take(tok) : 0;
+    // segments longer than a chunk: the states entering every chunk, recomputed (bf16 tiles)
+    w.stiles = recompute ? cur.take((size_t)kTileBytes * tiles) : 0;
     w.end = cur.off;
     return w;
 }
@@ -1270,15 +1287,17 @@ int grad_heads_per_cta(const lr_desc& d, int nchunk) {
 }  // namespace
 
 size_t ssd_fwd_ws_bytes(const lr_desc& d) { return fwd_plan(d).end; }
-size_t ssd_fwd_flag_bytes(const lr_desc& d) { return fwd_plan(d).end; }
+size_t ssd_fwd_flag_bytes(const lr_desc& d) { return fwd_plan(d).flags_end; }
 
 lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws, cudaStream_t st) {
     SsdArgs a = make_args(d, in, ckpt, ws);
-    unsigned int* ready = (unsigned int*)(ws + fwd_plan(d).ready);
+    const SsdFwdWs w = fwd_plan(d);
+    unsigned int* ready = (unsigned int*)(ws + w.ready);
     CUtensorMap mC, mB, mX, mY;
     bool ok = map4(&mC, in.Cm, kKD, d.G, d.L, d.B, true) && map4(&mB, in.Bm, kKD, d.G, d.L, d.B, true) &&
               map4(&mX, in.x, kP, d.H, d.L, d.B, true) && map4(&mY, y, kP, d.H, d.L, d.B, true);
-    char* stiles = (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
+    const int kseg = chunks_per_segment(d), nseg = (a.nchunk + kseg - 1) / kseg;
+    char* stiles = kseg == 1 ? (char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float) : ws + w.stiles;
     if (!ok) return LR_ERR_INVALID_ARG;
     const int var = variant_of(d);
     using ScanF = ScanSmem<3, true>;
@@ -1287,11 +1306,13 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanF::kAlloc);
     note_launch("ssd_state_scan");
     CUtensorMap mS;
-    if (!map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, a.nchunk, kP)) return LR_ERR_INVALID_ARG;
+    if (!map_states_vd(&mS, ckpt, (int64_t)a.B * a.H, nseg, kP)) return LR_ERR_INVALID_ARG;
     CUtensorMap mDt;
     const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
     if (!dt_tma) mDt = mB;  // not read
-    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, mDt, dt_tma, scan_args(a), stiles,
+    ScanArgs sa = scan_args(a);
+    sa.f32_every = kseg;  // f32 checkpoints at segment starts only
+    if (launch_pdl(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanF::kAlloc, st, mB, mX, mS, mDt, dt_tma, sa, stiles,
                    +1, ready, (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr) != cudaSuccess)
         return LR_ERR_CUDA;
     {
@@ -1319,7 +1340,10 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.a = make_args(d, in, ckpt, ws);
     const SsdArgs& a = ga.a;
     ga.gtiles = ws + w.gtiles;
-    ga.stiles = (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float);
+    const int kseg = chunks_per_segment(d), nseg = (a.nchunk + kseg - 1) / kseg;
+    ga.stiles = kseg == 1 ? (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float)
+                          : (const char*)(ws + w.stiles);
+    ga.sready = kseg > 1 ? (const unsigned int*)(ws + w.sready) : nullptr;
     ga.ddt = (__nv_bfloat16*)gr.ddelta;
     ga.dx = (__nv_bfloat16*)gr.dx;
     ga.dB = gr.dBm;
@@ -1349,6 +1373,30 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.accumulate = nblk > 1 ? 1 : 0;
     ga.gready = (const unsigned int*)(ws + w.gready);
     ga.zready = (const unsigned int*)(ws + w.dbc);
+    if (kseg > 1) {
+        // the states entering every chunk, from the f32 segment states: one CTA per (segment, row,
+        // head) folds the segment's chunk products from its checkpoint (forward direction)
+        using ScanR = ScanSmem<1, false>;
+        const int var = variant_of(d);
+        auto rec = var == kVarBil ? chunk_scan_kernel<1, false, kScanSsdBil>
+                   : var == kVarGen ? chunk_scan_kernel<1, false, kScanSsdGen> : chunk_scan_kernel<1, false, kScanSsd>;
+        cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanR::kAlloc);
+        note_launch("ssd_state_recompute");
+        CUtensorMap mDt;
+        const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
+        if (!dt_tma) mDt = mB;  // not read
+        ScanArgs sr = scan_args(a);
+        sr.seg_k = kseg;
+        sr.s_init = (const float*)ckpt;
+        sr.vd = kP;
+        // after the gate prep: a plain launch (the kernels after it read ds)
+        if (launch_ex(rec, dim3(nseg * a.B * a.H), dim3(kScanThreads), ScanR::kAlloc, st, !hz, mB, mX, mB, mDt, dt_tma,
+                      sr, ws + w.stiles, +1, (unsigned int*)(ws + w.sready), (float*)nullptr, (float*)nullptr,
+                      (unsigned int*)nullptr) != cudaSuccess)
+            return LR_ERR_CUDA;
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
     {
         using ScanB = ScanSmem<4, false>;
         const int var = variant_of(d);
@@ -1361,7 +1409,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
         if (!dt_tma) mDt = mC;  // not read
         // after the gate prep the scan starts only once ds is written (its loads do not wait)
-        if (launch_ex(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, !hz, mC, mdY, mC, mDt, dt_tma,
+        if (launch_ex(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, !hz || kseg > 1, mC, mdY, mC, mDt, dt_tma,
                        scan_args(a), ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
                        ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;

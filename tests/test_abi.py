@@ -91,6 +91,17 @@ def test_size_queries(L):
     assert L.ckpt_bytes(d) == 8 * 1 * 256 * 4                       # ceil(1000/128) = 8
     bad = L.make_desc("rglru", torch.float32, B=1, L=1000, D=3, segment=128)
     assert L.ckpt_bytes(bad) == 0 and L.workspace_bytes(bad, True) == 0
+    # SSD / GLA: one chunk per segment keeps a bf16 tile copy beside every f32 state; longer
+    # segments (whole chunks) keep the f32 segment states only
+    bf = torch.bfloat16
+    ssd = dict(kind="ssd", io=bf, B=2, L=4096, H=32, P=64, N=128, G=1, chunk=128, disc="zoh")
+    state = 2 * 32 * 128 * 64
+    assert L.ckpt_bytes(L.make_desc(segment=128, **ssd)) == 32 * state * 6
+    assert L.ckpt_bytes(L.make_desc(segment=256, **ssd)) == 16 * state * 4
+    assert L.ckpt_bytes(L.make_desc(segment=512, **ssd)) == 8 * state * 4
+    assert L.validate(L.make_desc(segment=192, **ssd)) == 2          # not a whole number of chunks
+    gla = dict(kind="gla", io=bf, B=4, L=2048, H=16, P=128, N=128, chunk=128)
+    assert L.ckpt_bytes(L.make_desc(segment=256, **gla)) == 8 * 4 * 16 * 128 * 128 * 4
 
 
 def test_calls_rejected_before_any_launch(L):

@@ -214,6 +214,56 @@ def test_gla_parity(B, L, H, V):
     assert plan.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("S", [256, 512])
+@pytest.mark.parametrize("case", ["ssd", "ssd_bilinear_z", "gla128", "gla64"])
+def test_segments_longer_than_a_chunk(case, S):
+    """Checkpoint segments of several chunks: the checkpoint holds the f32 state entering each
+    segment only (no bf16 copies), the forward keeps the tiles of every chunk in its workspace, and
+    the backward rebuilds them from the segment states before the gradient kernels read them.  The
+    checkpoints match the oracle's at segment S; outputs and gradients match the oracle, and equal
+    the one-chunk-segment run bitwise (the rebuilt tiles are the forward's)."""
+    from selective_state_space_09_b200 import lrscan
+    L = 700  # 6 chunks, the last one ragged: segments of 2 + 2 + 2 (S = 256) or 4 + 2 (S = 512)
+    if case.startswith("ssd"):
+        kind, disc = "ssd", ("bilinear" if case == "ssd_bilinear_z" else "zoh")
+        inp = inputs.ssd(2, L, 8, 64, 128, G=2, seed=S + 3, with_z=case == "ssd_bilinear_z")
+    else:
+        kind, disc = "gla", "none"
+        inp = inputs.gla(1, L, 4, 128, 128 if case == "gla128" else 64, seed=S + 5)
+    y, ck, gr, plan, disp = run_gpu(kind, inp, S, disc=disc, chunk=128)
+    y1, ck1, gr1, plan1, _ = run_gpu(kind, inp, 128, disc=disc, chunk=128)
+    assert plan.device_error() == (0, 0) and plan1.device_error() == (0, 0)
+    nseg = -(-L // S)
+    state = 2 * 8 * 128 * 64 if kind == "ssd" else 1 * 4 * 128 * inp["v"].shape[-1]
+    assert lrscan.ckpt_bytes(plan.desc) == nseg * state * 4
+    assert disp[1].startswith(kind + "_gate_prep+" if "_z" in case else kind + "_state_recompute+")
+    if kind == "ssd":
+        a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"])
+        ry, rck = oracle.ssd_fwd(*a, disc=disc, S=S)
+        rg = oracle.ssd_bwd(*a, inp["dy"], disc=disc)
+        assert_close("ckpt", ck.transpose(-1, -2), rck, TOL)
+        names = (("dx", "x"), ("ddelta", "delta"), ("dA", "A"), ("dBm", "B"), ("dCm", "C"), ("dDskip", "D"))
+        if inp["z"] is not None:
+            names += (("dz", "z"),)
+    else:
+        ry, rck = oracle.gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], S=S)
+        rg = oracle.gla_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["dy"])
+        assert_close("ckpt", ck, rck, TOL)
+        names = (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"))
+    assert_close("y", y, ry, TOL)
+    for gk, rk in names:
+        assert_close(gk, gr[gk], rg[rk], TOL)
+    # the same numbers as with one chunk per segment (dB, dC: sums of reduction-adds over head
+    # blocks in arbitrary order, bitwise only up to two blocks per group)
+    assert torch.equal(y, y1)
+    assert torch.equal(ck, ck1[::S // 128])
+    for gk, _ in names:
+        if gk in ("dBm", "dCm"):
+            assert_close(gk, gr[gk], to64(gr1[gk]), 1e-5)
+        else:
+            assert torch.equal(gr[gk], gr1[gk]), gk
+
+
 def test_gla_deterministic():
     inp = inputs.gla(2, 384, 2, 128, 128, seed=3)
     a = run_gpu("gla", inp, 128, chunk=128)

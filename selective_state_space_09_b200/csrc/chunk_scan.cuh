@@ -54,8 +54,8 @@ struct ScanArgs {
     int withhold;                 // LR_TEST_WITHHOLD_CARRY: slot 0 is never counted (failure-path test)
     int f32_every;                // forward: the f32 state of chunk c is a checkpoint when c % f32_every == 0
                                   // (slot c / f32_every); 0 or 1 = every chunk
-    int seg_k;                    // segment mode (dir > 0, recompute): one CTA per segment of seg_k chunks,
-                                  // its state read from s_init; 0 = one CTA walks the whole sequence
+    int seg_k;                    // segment mode (dir > 0, recompute): segments of seg_k chunks, each
+                                  // restarted from its state in s_init; 0 = one chain over the sequence
     const float* s_init;          // segment mode: f32 state entering each segment [nseg][B*H][kKD][vd]
     int vd;                       // value width of s_init rows
 };
@@ -189,19 +189,31 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
     float* decp = reinterpret_cast<float*>(sm + SM::kDecP);
     float* decf = reinterpret_cast<float*>(sm + SM::kDecF);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nbh = a.B * a.H * a.halves;
-    const int seg = a.seg_k ? (int)blockIdx.x / nbh : 0;  // segment mode: this CTA's segment
-    const int bidx = (int)blockIdx.x % nbh;
-    const int half = bidx % a.halves, bh = bidx / a.halves, b = bh / a.H, h = bh % a.H;
+    const int half = blockIdx.x % a.halves, bh = blockIdx.x / a.halves, b = bh / a.H, h = bh % a.H;
     const int g = h / a.HpG, rsel = MODE == kScanGla ? h : g;  // R: per group (SSD) or head (GLA)
     const int hx = h & 7;  // this head's column of a dt ring row
     const size_t slot_bytes = (size_t)kScanTile * a.halves;  // one bf16 state tile, all halves
     const int BH = a.B * a.H;
-    // chunks this CTA covers: the whole sequence, or (segment mode) chunks c_first .. c_first + ncs - 1
-    const int c_first = a.seg_k ? seg * a.seg_k : 0;
-    const int ncs = a.seg_k ? min(a.seg_k, a.nchunk - c_first) : a.nchunk;
-    const int nk = ncs - 1;  // chunks with a product
-    auto chunk_of = [&](int k) { return dir > 0 ? c_first + k : a.nchunk - 1 - k; };
+    // Segment mode walks the segments from the last to the first (the gradient kernels that wait
+    // for the rebuilt states take the chunks from the last one), the chunks of a segment in order;
+    // each segment restarts from its checkpointed state and has one product fewer than chunks.
+    const int K = a.seg_k > 0 ? a.seg_k : a.nchunk;
+    const int nseg = (a.nchunk + K - 1) / K;
+    const int nlast = a.nchunk - (nseg - 1) * K;  // chunks of the last segment
+    const int nk = a.nchunk - nseg;               // products
+    // chunk of product k and of put q (segment mode; otherwise the sequence in order / reversed)
+    auto chunk_of = [&](int k) {
+        if (!a.seg_k) return dir > 0 ? k : a.nchunk - 1 - k;
+        if (k < nlast - 1) return (nseg - 1) * K + k;
+        const int kk = k - (nlast - 1);
+        return (nseg - 2 - kk / (K - 1)) * K + kk % (K - 1);
+    };
+    auto slot_of_put = [&](int q) {
+        if (!a.seg_k) return dir > 0 ? q : a.nchunk - 1 - q;
+        if (q < nlast) return (nseg - 1) * K + q;
+        const int qq = q - nlast;
+        return (nseg - 2 - qq / K) * K + qq % K;
+    };
     auto stage = [&](int k) { return sm + (size_t)(k % NS) * SM::kStage; };
     auto load = [&](int k) {
         char* st = stage(k);
@@ -406,11 +418,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
         if (ready && lane == 0) {
             int next = 0;
             unsigned long long t0 = global_ns();
-            while (next < ncs) {
+            while (next < a.nchunk) {
                 const int done = ld_acquire_cta(pubdone);
                 if (done >= next) {
                     for (; next <= done; ++next) {
-                        const int slot = dir > 0 ? c_first + next : a.nchunk - 1 - next;
+                        const int slot = slot_of_put(next);
                         if (!(a.withhold && slot == 0)) red_release_add(&ready[((size_t)slot * a.B + b) * a.G + g], 1u);
                     }
                     t0 = global_ns();
@@ -436,9 +448,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
             st_release_cta(pubdone, q);
         };
         float S[kScanP];
-        if (a.s_init) {  // segment mode: the checkpointed state entering the segment, row n
+#pragma unroll
+        for (int i = 0; i < kScanP; ++i) S[i] = 0.0f;
+        // segment mode: the checkpointed state entering segment sg, row n
+        auto load_state = [&](int sg) {
             const float4* src = reinterpret_cast<const float4*>(
-                a.s_init + (((size_t)seg * BH + bh) * kKD + n) * a.vd + kScanP * half);
+                a.s_init + (((size_t)sg * BH + bh) * kKD + n) * a.vd + kScanP * half);
 #pragma unroll
             for (int i = 0; i < kScanP / 4; ++i) {
                 const float4 v = src[i];
@@ -447,11 +462,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
                 S[4 * i + 2] = v.z;
                 S[4 * i + 3] = v.w;
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < kScanP; ++i) S[i] = 0.0f;
-        }
-        pdl_wait();  // the previous kernel of the stream may still read the slots
+        };
+        // the previous kernel of the stream may still read the slots; in segment mode the slots are
+        // this kernel's own workspace region, which the kernel before it (the backward scan) never
+        // touches, so it runs beside that kernel
+        if (!a.s_init) pdl_wait();
         // S into slot c through the staging buffers (free: the copies of the previous slot have
         // read them before the first barrier)
         auto put = [&](int c) {
@@ -493,8 +508,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
             pub2 = pub1;
             pub1 = nput++;
         };
-        put(dir > 0 ? c_first : a.nchunk - 1);
-        for (int k = 0; k < nk; ++k) {
+        // one product folded into S, then S put into the slot of the next chunk
+        auto fold = [&](int k) {
             const int buf = k % kScanBufs;
             ok = ok && mbar_wait(&prod[buf], (uint32_t)((k / kScanBufs) & 1), a.hdr, 744);
             tc::fence_after_sync();
@@ -508,6 +523,18 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < kScanP; ++i) S[i] = fmaf(d, S[i], v[i]);
             put(chunk_of(k) + dir);
+        };
+        if (!a.seg_k) {
+            put(dir > 0 ? 0 : a.nchunk - 1);
+            for (int k = 0; k < nk; ++k) fold(k);
+        } else {
+            int k = 0;
+            for (int sg = nseg - 1; sg >= 0; --sg) {
+                load_state(sg);
+                put(sg * K);
+                const int nc = sg == nseg - 1 ? nlast : K;
+                for (int j = 0; j + 1 < nc; ++j) fold(k++);
+            }
         }
         if (fl) {
             bulk_wait_all();

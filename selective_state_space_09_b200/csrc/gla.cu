@@ -647,8 +647,8 @@ ScanArgs scan_args(const GlaArgs& a, int VD) {
 // The chunk-state scan over (row, head, 64 value columns): dir > 0 folds K^T diag(w) V into the
 // entering states (f32 checkpoint slots every `kseg` chunks, bf16 tiles of every chunk); dir < 0
 // folds Q^T diag(E) dO into the adjoint states (bf16 tiles).  With `recompute` (dir > 0, kseg > 1)
-// one CTA per (segment, row, head, half) rebuilds the tiles of its segment's chunks from the f32
-// segment state in `ckpt`.  Each slot half is flagged in `ready` once written.
+// one CTA per (row, head, half) rebuilds the tiles of every chunk from the f32 segment states in
+// `ckpt`, the last segment first.  Each slot half is flagged in `ready` once written.
 template <int VD>
 lr_status gla_scan(const lr_desc& d, const GlaArgs& a, const CUtensorMap& mR, const CUtensorMap& mZ, void* ckpt,
                    char* tiles, int dir, unsigned int* ready, int kseg, bool recompute, cudaStream_t st) {
@@ -664,11 +664,11 @@ lr_status gla_scan(const lr_desc& d, const GlaArgs& a, const CUtensorMap& mR, co
         sa.seg_k = kseg;
         sa.s_init = (const float*)ckpt;
         sa.vd = VD;
-        using SR = ScanSmem<1, false>;
-        cudaFuncSetAttribute(chunk_scan_kernel<1, false, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        using SR = ScanSmem<4, false>;
+        cudaFuncSetAttribute(chunk_scan_kernel<4, false, kScanGla>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SR::kAlloc);
         note_launch("gla_state_recompute");
-        e = launch_pdl(chunk_scan_kernel<1, false, kScanGla>, dim3((unsigned)(nseg * a.B * a.H * sa.halves)),
+        e = launch_pdl(chunk_scan_kernel<4, false, kScanGla>, dim3((unsigned)(a.B * a.H * sa.halves)),
                        dim3(kScanThreads), SR::kAlloc, st, mR, mZ, mS, mDt, dt_tma, sa, tiles, +1, ready,
                        (float*)nullptr, (float*)nullptr, (unsigned int*)nullptr);
         if (e != cudaSuccess) return LR_ERR_CUDA;
@@ -737,14 +737,13 @@ lr_status gla_bwd_t(const lr_desc& d, const lr_inputs& in, const void* dy, const
     if (!(map4(&mQ, in.q, kKD, d.H, d.L, d.B, true) && map4(&mK, in.k, kKD, d.H, d.L, d.B, true) &&
           map4(&mV, in.v, VD, d.H, d.L, d.B, true) && map4(&mO, dy, VD, d.H, d.L, d.B, true)))
         return LR_ERR_INVALID_ARG;
-    lr_status s;
-    if (kseg > 1) {  // the states entering every chunk, rebuilt from the f32 segment states
+    lr_status s = gla_scan<VD>(d, a, mQ, mO, nullptr, ws + w.gtiles, -1, (unsigned int*)(ws + w.ready), kseg, false, st);
+    if (s != LR_OK) return s;
+    if (kseg > 1) {  // the states entering every chunk, rebuilt from the f32 segment states beside the scan
         s = gla_scan<VD>(d, a, mK, mV, const_cast<void*>(ckpt), ws + w.stiles, +1, (unsigned int*)(ws + w.sready),
                          kseg, true, st);
         if (s != LR_OK) return s;
     }
-    s = gla_scan<VD>(d, a, mQ, mO, nullptr, ws + w.gtiles, -1, (unsigned int*)(ws + w.ready), kseg, false, st);
-    if (s != LR_OK) return s;
     cudaFuncSetAttribute(gla_grad_kernel<VD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GGradSmem<VD>::kAlloc);
     note_launch("gla_chunk_grad");
     if (launch_pdl(gla_grad_kernel<VD>, dim3(a.nchunk * a.B * a.H), dim3(256), GGradSmem<VD>::kAlloc, st, mQ, mK, mV,

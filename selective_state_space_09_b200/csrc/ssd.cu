@@ -216,7 +216,7 @@ __device__ __forceinline__ uint32_t col_y2(int w) { return 256u + 192u * w; }
 //   issue (one thread): Y = P X (A from TMEM), Y2 = C S_in;
 //   finish: y = Y + E Y2 + D x -> the x tile -> TMA store; the freed S_in slot loads the
 //   warpgroup's next head and the x slot freed one head earlier the head after next.
-template <int VAR>
+template <int VAR, bool HZ>
 __global__ void __launch_bounds__(256, 1)
 ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY, SsdArgs a,
@@ -376,7 +376,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
         tc::fence_after_sync();
         char* X = Xs + xs * kQ * 128;
         // z gate: this row's z of the head, read straight from global memory (16 bytes per 8 columns)
-        const bool zrow = a.z && t0 + wt < a.L;
+        const bool zrow = HZ && t0 + wt < a.L;
         const __nv_bfloat16* zr = zrow ? a.z + (((size_t)b * a.L + t0 + wt) * a.H + hfirst + i) * kP : nullptr;
 #pragma unroll
         for (int v0 = 0; v0 < kP; v0 += 16) {
@@ -402,7 +402,7 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
                     }
                     o0 = fmaf(Dh, xf.x, o0);
                     o1 = fmaf(Dh, xf.y, o1);
-                    if (a.z) {  // y = s silu(z)
+                    if constexpr (HZ) {  // y = s silu(z)
                         const float2 zf = __bfloat1622float2(zv[e]);
                         o0 *= zf.x * sigm_f(zf.x);
                         o1 *= zf.y * sigm_f(zf.y);
@@ -440,11 +440,18 @@ ssd_out_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ C
 }
 
 // Kernel variant of a descriptor: bilinear (signed decays), the general one (dirac, ZOH-Euler or
-// the softplus front-end), or the default ZOH one.
+// the softplus front-end), or the default ZOH one.  The z gate is a second compile-time choice, so
+// the kernels without it carry none of its work.
 int variant_of(const lr_desc& d) {
     if (d.disc == LR_DISC_BILINEAR) return kVarBil;
     return (d.disc != LR_DISC_ZOH || (d.flags & LR_DELTA_SOFTPLUS)) ? kVarGen : kVarZoh;
 }
+template <bool HZ>
+auto out_variant_z(int var) {
+    return var == kVarBil ? ssd_out_kernel<kVarBil, HZ> : var == kVarGen ? ssd_out_kernel<kVarGen, HZ>
+                                                                          : ssd_out_kernel<kVarZoh, HZ>;
+}
+auto out_variant(int var, bool hz) { return hz ? out_variant_z<true>(var) : out_variant_z<false>(var); }
 
 // Chunks per checkpoint segment (the segment is a multiple of the chunk).  With one chunk per
 // segment the checkpoint buffer also holds the bf16 tile copy of every state the tensor cores
@@ -610,7 +617,7 @@ constexpr int kLoader = 160;
 //   E2: dx, the inter-chunk row dots, dy scaled by E and x by w in place;
 //   batch 2: diag(E) dy S_in^T, diag(w) x G^T into dC, dB, issued with phase A of head i + 1
 //     (M = C B^T, S2 = dy x^T) while warpgroup 0 turns head i's row terms into d dt.
-template <int VAR>
+template <int VAR, bool HZ>
 __global__ void __launch_bounds__(256, 1)
 ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                 const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY, SsdGradArgs ga,
@@ -956,7 +963,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
             tc::mma_tiles(tmem + kGdV, sP, 1, kQ, sO, 1, kQ, kQ, kP, kQ, 0);      // dV1 = P^T dy
             if (has_out) tc::mma_tiles(tmem + kGBG, sK, 0, kQ, sG, 1, kKD, kQ, kP, kKD, 0);  // B G
             if (has_in) tc::mma_tiles(tmem + kGY2, sQ, 0, kQ, sS, 1, kKD, kQ, kP, kKD, 0);   // C S_in
-            if (ga.gz) tc::mma_tiles(tmem + kGY, sP, 0, kQ, sX, 1, kQ, kQ, kP, kQ, 0);        // Y = P x
+            if (HZ) tc::mma_tiles(tmem + kGY, sP, 0, kQ, sX, 1, kQ, kQ, kP, kQ, 0);           // Y = P x
             tc::commit(&bar[4]);
             tc::mma_tiles(tmem + kGdC, sPd, 0, kQ, sK, 1, kQ, kQ, kKD, kQ, acc);  // dC += Pd B
             tc::mma_tiles(tmem + kGdB, sPd, 1, kQ, sQ, 1, kQ, kQ, kKD, kQ, acc);  // dB += Pd^T C
@@ -987,7 +994,7 @@ ssd_grad_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ 
                 if (has_out) tc::ld16(tmem + kGBG + lane_off + col, bg);
                 if (has_in) tc::ld16(tmem + kGY2 + lane_off + col, y2);
                 tc::wait_ld();
-                if (ga.gz) {
+                if constexpr (HZ) {
                     // z gate: s = P x + E (C S_in) + D x, the readout before the gate; dz = s gz
                     float yv[16];
                     tc::ld16(tmem + kGY + lane_off + col, yv);
@@ -1246,6 +1253,13 @@ __global__ void ssd_param_sum(const float* __restrict__ pdA, const float* __rest
     }
 }
 
+template <bool HZ>
+auto grad_variant_z(int var) {
+    return var == kVarBil ? ssd_grad_kernel<kVarBil, HZ> : var == kVarGen ? ssd_grad_kernel<kVarGen, HZ>
+                                                                           : ssd_grad_kernel<kVarZoh, HZ>;
+}
+auto grad_variant(int var, bool hz) { return hz ? grad_variant_z<true>(var) : grad_variant_z<false>(var); }
+
 struct SsdBwdWs {
     size_t gready, dbc, sready, flags_end, pdA, pdD, pdE, gtiles, ds, gz, stiles, end;  // flags first: reset every call
 };
@@ -1321,7 +1335,7 @@ lr_status ssd_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, ch
     }
     const int hb = out_heads_per_cta(d, a.nchunk);
     const int nblk_o = (a.HpG + hb - 1) / hb;
-    auto out = var == kVarBil ? ssd_out_kernel<kVarBil> : var == kVarGen ? ssd_out_kernel<kVarGen> : ssd_out_kernel<kVarZoh>;
+    auto out = out_variant(var, (d.flags & LR_HAS_Z) != 0);
     cudaFuncSetAttribute(out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OutSmem::kAlloc);
     note_launch("ssd_chunk_out");
     if (launch_pdl(out, dim3(a.nchunk * a.B * a.G * nblk_o), dim3(256), OutSmem::kAlloc, st, mC, mB, mX, mY,
@@ -1340,7 +1354,7 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.a = make_args(d, in, ckpt, ws);
     const SsdArgs& a = ga.a;
     ga.gtiles = ws + w.gtiles;
-    const int kseg = chunks_per_segment(d), nseg = (a.nchunk + kseg - 1) / kseg;
+    const int kseg = chunks_per_segment(d);
     ga.stiles = kseg == 1 ? (const char*)ckpt + (size_t)a.nchunk * a.B * a.H * kKD * kP * sizeof(float)
                           : (const char*)(ws + w.stiles);
     ga.sready = kseg > 1 ? (const unsigned int*)(ws + w.sready) : nullptr;
@@ -1373,30 +1387,6 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
     ga.accumulate = nblk > 1 ? 1 : 0;
     ga.gready = (const unsigned int*)(ws + w.gready);
     ga.zready = (const unsigned int*)(ws + w.dbc);
-    if (kseg > 1) {
-        // the states entering every chunk, from the f32 segment states: one CTA per (segment, row,
-        // head) folds the segment's chunk products from its checkpoint (forward direction)
-        using ScanR = ScanSmem<1, false>;
-        const int var = variant_of(d);
-        auto rec = var == kVarBil ? chunk_scan_kernel<1, false, kScanSsdBil>
-                   : var == kVarGen ? chunk_scan_kernel<1, false, kScanSsdGen> : chunk_scan_kernel<1, false, kScanSsd>;
-        cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanR::kAlloc);
-        note_launch("ssd_state_recompute");
-        CUtensorMap mDt;
-        const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
-        if (!dt_tma) mDt = mB;  // not read
-        ScanArgs sr = scan_args(a);
-        sr.seg_k = kseg;
-        sr.s_init = (const float*)ckpt;
-        sr.vd = kP;
-        // after the gate prep: a plain launch (the kernels after it read ds)
-        if (launch_ex(rec, dim3(nseg * a.B * a.H), dim3(kScanThreads), ScanR::kAlloc, st, !hz, mB, mX, mB, mDt, dt_tma,
-                      sr, ws + w.stiles, +1, (unsigned int*)(ws + w.sready), (float*)nullptr, (float*)nullptr,
-                      (unsigned int*)nullptr) != cudaSuccess)
-            return LR_ERR_CUDA;
-        lr_status s = check_launch();
-        if (s != LR_OK) return s;
-    }
     {
         using ScanB = ScanSmem<4, false>;
         const int var = variant_of(d);
@@ -1409,15 +1399,40 @@ lr_status ssd_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, const v
         const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
         if (!dt_tma) mDt = mC;  // not read
         // after the gate prep the scan starts only once ds is written (its loads do not wait)
-        if (launch_ex(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, !hz || kseg > 1, mC, mdY, mC, mDt, dt_tma,
+        if (launch_ex(scan, dim3(a.B * a.H), dim3(kScanThreads), ScanB::kAlloc, st, !hz, mC, mdY, mC, mDt, dt_tma,
                        scan_args(a), ws + w.gtiles, -1, (unsigned int*)(ws + w.gready), gr.dBm, gr.dCm,
                        ga.accumulate ? (unsigned int*)(ws + w.dbc) : (unsigned int*)nullptr) != cudaSuccess)
             return LR_ERR_CUDA;
         lr_status s = check_launch();
         if (s != LR_OK) return s;
     }
-    const int var = variant_of(d);
-    auto grad = var == kVarBil ? ssd_grad_kernel<kVarBil> : var == kVarGen ? ssd_grad_kernel<kVarGen> : ssd_grad_kernel<kVarZoh>;
+    if (kseg > 1) {
+        // the states entering every chunk, from the f32 segment states: one CTA per (row, head) walks
+        // the segments from the last, each restarted from its checkpoint, folding the chunk products
+        // (forward direction); launched after the backward scan so that it runs on the SMs the scan
+        // leaves free, and before the gradient kernel, so that all its CTAs have started before a
+        // gradient CTA waits for them
+        using ScanR = ScanSmem<4, false>;
+        const int var = variant_of(d);
+        auto rec = var == kVarBil ? chunk_scan_kernel<4, false, kScanSsdBil>
+                   : var == kVarGen ? chunk_scan_kernel<4, false, kScanSsdGen> : chunk_scan_kernel<4, false, kScanSsd>;
+        cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanR::kAlloc);
+        note_launch("ssd_state_recompute");
+        CUtensorMap mDt;
+        const int dt_tma = map_dt(&mDt, d.B, d.L, d.H, in.delta) ? 1 : 0;
+        if (!dt_tma) mDt = mB;  // not read
+        ScanArgs sr = scan_args(a);
+        sr.seg_k = kseg;
+        sr.s_init = (const float*)ckpt;
+        sr.vd = kP;
+        if (launch_ex(rec, dim3(a.B * a.H), dim3(kScanThreads), ScanR::kAlloc, st, true, mB, mX, mB, mDt, dt_tma,
+                      sr, ws + w.stiles, +1, (unsigned int*)(ws + w.sready), (float*)nullptr, (float*)nullptr,
+                      (unsigned int*)nullptr) != cudaSuccess)
+            return LR_ERR_CUDA;
+        lr_status s = check_launch();
+        if (s != LR_OK) return s;
+    }
+    auto grad = grad_variant(variant_of(d), hz);
     cudaFuncSetAttribute(grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::kAlloc);
     note_launch("ssd_chunk_grad");
     if (launch_pdl(grad, dim3(a.nchunk * a.B * a.G * nblk), dim3(256), GradSmem::kAlloc, st, mC, mB, mX, mdY,

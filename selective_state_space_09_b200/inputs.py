@@ -50,6 +50,10 @@ WORKLOADS = {
     # dt = softplus(delta + bias) in the kernels, abar = e^{dt A}, beta = dt (ZOH-Euler)
     "ssd_mamba2": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=128,
                        segment=128, disc="zoh_euler", softplus=True),
+    # the SSD workload's inputs through the bilinear (Tustin) discretisation: abar = (1 + u) / (1 - u),
+    # u = dt A / 2, negative wherever dt |A| > 2
+    "ssd_bilinear": dict(kind="ssd", io="bf16", B=2, H=32, P=64, N=128, G=1, L=4096, chunk=128,
+                         segment=128, disc="bilinear"),
 }
 
 _DT = {"f32": torch.float32, "bf16": torch.bfloat16}

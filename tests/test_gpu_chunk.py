@@ -236,7 +236,7 @@ def test_segments_longer_than_a_chunk(case, S):
     nseg = -(-L // S)
     state = 2 * 8 * 128 * 64 if kind == "ssd" else 1 * 4 * 128 * inp["v"].shape[-1]
     assert lrscan.ckpt_bytes(plan.desc) == nseg * state * 4
-    assert disp[1].startswith(kind + "_gate_prep+" if "_z" in case else kind + "_state_recompute+")
+    assert kind + "_state_recompute" in disp[1].split("+")
     if kind == "ssd":
         a = (inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], inp["Dskip"], inp["z"])
         ry, rck = oracle.ssd_fwd(*a, disc=disc, S=S)

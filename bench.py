@@ -830,6 +830,7 @@ def time_oracle(name, threads, min_seconds=1.0):
 def cpu_baseline(name):
     """The oracle at all host cores (the reported value) and at one thread."""
     cores = host_cores()
+    os.environ["OMP_NUM_THREADS"] = str(cores)  # read by the OpenMP runtime when the oracle loads
     allc = time_oracle(name, cores)
     one = time_oracle(name, 1)
     out = {k: allc[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -1028,6 +1029,9 @@ def inputs_L(name):
 def reference_arm(args, world):
     """The fp64 CPU oracle on all host cores: each step is a bounded sample of the workload.  The
     workload is chosen by name; nothing here loads the CUDA library."""
+    # torch.distributed.run exports OMP_NUM_THREADS=1, which the OpenMP runtime reads when the
+    # oracle library loads
+    os.environ["OMP_NUM_THREADS"] = str(host_cores())
     import oracle
     from selective_state_space_09_b200 import inputs
     name = args.workload or "ssd"

@@ -263,8 +263,9 @@ def kernel_cost(w, name, pas, ops, pass_bytes):
     """Algorithmic bytes and FLOPs of one launch of kernel `name` of a workload's pass: the
     operands the kernel must read and write at minimum (each once) and the products of the method
     it evaluates.  Kernels that are a whole pass carry the pass's bytes; small fixed-order
-    reductions are counted as 0 (they are not candidates for the dominant kernel)."""
-    if name.endswith("param_reduce"):
+    reductions and the workspace zeroing are counted as 0 (they are not candidates for the
+    dominant kernel)."""
+    if name.endswith("param_reduce") or name.endswith("ws_zero"):
         return 0, 0
     key = (name, pas)
     if key in CHUNK_KERNEL_OPERANDS:

@@ -138,6 +138,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     });
     return encode;
 }
+// The tensor-map encoder is a driver call and needs a current context on the calling thread; a
+// thread whose first CUDA call of the process is this one (a framework's worker thread, say) has
+// none yet.  A runtime call binds the current device's primary context to the thread.
+bool bind_context() { return cudaFree(nullptr) == cudaSuccess; }
 }  // namespace
 
 bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const uint64_t* dims,
@@ -152,10 +156,14 @@ bool make_tmap(CUtensorMap* map, const void* base, int esize, int rank, const ui
         e[i] = 1;
     }
     for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
-    CUresult r = encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    auto run = [&] {
+        return encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank,
+                      const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    };
+    CUresult r = run();
+    if (r == CUDA_ERROR_INVALID_CONTEXT && bind_context()) r = run();
     return r == CUDA_SUCCESS;
 }
 
@@ -167,10 +175,14 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int esize_, uint64_t d0, u
     cuuint64_t strides[2] = {d0 * esize_, d0 * d1 * esize_};
     cuuint32_t box[3] = {box0, box1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(map, esize_ == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    auto run = [&] {
+        return encode(map, esize_ == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    };
+    CUresult r = run();
+    if (r == CUDA_ERROR_INVALID_CONTEXT && bind_context()) r = run();
     return r == CUDA_SUCCESS;
 }
 
@@ -231,7 +243,9 @@ lr_status lr_scan_fwd(const lr_desc* desc, const lr_inputs* in, void* y, void* c
     if (ws_size < ws_bytes(d, false)) return LR_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     set_launch_stream(st);
-    if (cudaMemsetAsync(ws, 0, flag_bytes(d, false), st) != cudaSuccess) return LR_ERR_CUDA;
+    // the diagonal kinds zero their workspace head in a kernel their scan kernel overlaps
+    const bool diag = d.kind == LR_RGLRU || d.kind == LR_ROTLRU;
+    if (!diag && cudaMemsetAsync(ws, 0, flag_bytes(d, false), st) != cudaSuccess) return LR_ERR_CUDA;
     switch (d.kind) {
         case LR_RGLRU:
         case LR_ROTLRU: return diag_fwd(d, *in, y, ckpt, (char*)ws, st);
@@ -279,7 +293,8 @@ lr_status lr_scan_bwd(const lr_desc* desc, const lr_inputs* in, const void* dy, 
     if (ws_size < ws_bytes(d, true)) return LR_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     set_launch_stream(st);
-    if (cudaMemsetAsync(ws, 0, flag_bytes(d, true), st) != cudaSuccess) return LR_ERR_CUDA;
+    const bool diag = d.kind == LR_RGLRU || d.kind == LR_ROTLRU;
+    if (!diag && cudaMemsetAsync(ws, 0, flag_bytes(d, true), st) != cudaSuccess) return LR_ERR_CUDA;
     switch (d.kind) {
         case LR_RGLRU:
         case LR_ROTLRU: return diag_bwd(d, *in, dy, ckpt, *gr, (char*)ws, st);

@@ -24,6 +24,8 @@
 // per tile into partials that a second kernel reduces in a fixed order.
 #include <stdio.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "host_common.h"
 
@@ -54,6 +56,7 @@ template <typename V> struct Agg {
 struct DiagArgs {
     int B, L, D, S, nseg, ncb;  // D = real channels of b / y
     unsigned int dflags;        // lr_desc flags (LR_TEST_WITHHOLD_CARRY)
+    int direct;                 // tiles numbered by block index (the grid fits on the SMs at once)
     const float* mag;           // rotlru
     const float* theta;         // rotlru
     const float* lam;           // rglru with gates: Lambda [D]
@@ -208,31 +211,181 @@ __device__ __forceinline__ Agg<V> ld_cg_agg(const Agg<V>* p) {
     return {ld_cg(&p->m), ld_cg(&p->v)};
 }
 
-// Carry entering tile k of a row, deterministic whatever the timing: walk towards the start
-// of the chain (dir = -1: earlier segments, forward pass; dir = +1: later segments, backward
-// pass) until a tile that has published its inclusive prefix (or the end of the row), then fold
-// the aggregates of the tiles in between in chain order, x <- m x + v.  That is the same
-// sequence of operations as a purely chained scan, so the result does not depend on which
-// records happened to be ready.  Waits are bounded; a wait that gives up counts as a zero
-// prefix (the error is recorded).
+// A tile's records in the look-back.  Complex values (rotlru) are stored, fenced, and then the
+// tile's flag is set with release semantics, so a reader that sees the flag may read them.  Real
+// values are published without a fence: each 32-bit value travels with its status in one 64-bit
+// word (a single store makes both visible), the flag is set with a relaxed store and only tells a
+// reader which records to read, and a reader that finds a record's status missing reads it again.
+// The workspace holding the records is zeroed before every call, so a status is this call's.
+__device__ __forceinline__ uint64_t pack_rec(unsigned int st, float v) {
+    return ((uint64_t)st << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u32(unsigned int* p, unsigned int v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <typename V> struct Rec;
+template <> struct Rec<cpx> {  // fenced
+    static constexpr bool kFence = true;
+    using AggT = Agg<cpx>;
+    using PreT = cpx;
+    static __device__ __forceinline__ void put_agg(AggT* p, Agg<cpx> a) { st_cg_agg(p, a); }
+    static __device__ __forceinline__ void put_pre(PreT* p, cpx v) { st_cg(p, v); }
+    static __device__ __forceinline__ bool get_agg(const AggT* p, Agg<cpx>& a) {
+        a = ld_cg_agg(p);
+        return true;
+    }
+    static __device__ __forceinline__ bool get_pre(const PreT* p, cpx& v) {
+        v = ld_cg(p);
+        return true;
+    }
+};
+template <> struct Rec<float> {  // packed: status in the high word
+    static constexpr bool kFence = false;
+    struct AggT {
+        uint64_t m, v;
+    };
+    using PreT = uint64_t;
+    static __device__ __forceinline__ void put_agg(AggT* p, Agg<float> a) {
+        st_relaxed_u64(&p->m, pack_rec(kFlagAgg, a.m));
+        st_relaxed_u64(&p->v, pack_rec(kFlagAgg, a.v));
+    }
+    static __device__ __forceinline__ void put_pre(PreT* p, float v) { st_relaxed_u64(p, pack_rec(kFlagPrefix, v)); }
+    static __device__ __forceinline__ bool get_agg(const AggT* p, Agg<float>& a) {
+        const uint64_t m = ld_relaxed_u64(&p->m), v = ld_relaxed_u64(&p->v);
+        a = {__uint_as_float((unsigned int)m), __uint_as_float((unsigned int)v)};
+        return (m >> 32) == kFlagAgg && (v >> 32) == kFlagAgg;
+    }
+    static __device__ __forceinline__ bool get_pre(const PreT* p, float& v) {
+        const uint64_t w = ld_relaxed_u64(p);
+        v = __uint_as_float((unsigned int)w);
+        return (w >> 32) == kFlagPrefix;
+    }
+};
+
+// Publish a tile's aggregate (st = kFlagAgg) or inclusive prefix (kFlagPrefix); warp 0, one lane
+// per unit (act: the lane's unit exists).
 template <typename V>
-__device__ V lookback_carry(const unsigned int* flags, const Agg<V>* aggRec, const V* preRec,
-                            size_t row, int k, int dir, int nseg, int CB, int lane, bool act,
-                            WsHeader* hdr, int info) {
-    int j = k + dir;
-    V x = zero_of(V{});
-    while (j >= 0 && j < nseg) {
-        unsigned int f = wait_flag(&flags[row + j], hdr, info);
-        if (f == kFlagPrefix) {
-            if (act) x = ld_cg(&preRec[(row + j) * CB + lane]);
+__device__ __forceinline__ void publish_agg(unsigned int* flag, typename Rec<V>::AggT* rec, Agg<V> a, bool act,
+                                            int lane) {
+    if (act) Rec<V>::put_agg(rec, a);
+    if (Rec<V>::kFence) __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+        if (Rec<V>::kFence)
+            st_release(flag, kFlagAgg);
+        else
+            st_relaxed_u32(flag, kFlagAgg);
+    }
+}
+template <typename V>
+__device__ __forceinline__ void publish_pre(unsigned int* flag, typename Rec<V>::PreT* rec, V v, bool act,
+                                            int lane) {
+    if (act) Rec<V>::put_pre(rec, v);
+    if (Rec<V>::kFence) __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+        if (Rec<V>::kFence)
+            st_release(flag, kFlagPrefix);
+        else
+            st_relaxed_u32(flag, kFlagPrefix);
+    }
+}
+
+// Read a record whose status was missing again until it is there (bounded by the wait that began
+// at t0; false after giving up, with the error recorded).
+template <typename V, bool PRE, typename R, typename O>
+__device__ __forceinline__ bool reread(const R* p, O& out, unsigned long long t0, WsHeader* hdr, int info) {
+    for (int it = 0;; ++it) {
+        bool got;
+        if constexpr (PRE)
+            got = Rec<V>::get_pre(p, out);
+        else
+            got = Rec<V>::get_agg(p, out);
+        if (got) return true;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            record_error(hdr, LR_ERR_TIMEOUT, info);
+            return false;
+        }
+        if (it > 16) __nanosleep(64);
+    }
+}
+
+// Carry entering tile k of a row, deterministic whatever the timing.  Towards the start of the
+// chain (dir = -1: earlier segments, forward pass; dir = +1: later segments, backward pass) the
+// nearest tile that has published its inclusive prefix (or the end of the row) is found with
+// every tile between it and k holding its aggregate; the aggregates of those tiles are then
+// folded onto the prefix in chain order, x <- m x + v.  That is the same sequence of operations as
+// a purely chained scan, so the result does not depend on which records happened to be ready.
+//
+// The warp (all 32 lanes call this) reads the flags of 32 tiles per round trip, lane i the tile at
+// distance i + 1 of the window, and issues the aggregate loads KB at a time before folding them:
+// a tile far down a row pays a few L2 round trips, not two per tile in between.  The wait is
+// bounded; giving up records the error and yields a zero carry.
+template <int KB, typename V>
+__device__ __forceinline__ V lookback_carry(const unsigned int* flags, const typename Rec<V>::AggT* aggRec,
+                                            const typename Rec<V>::PreT* preRec, size_t row, int k, int dir,
+                                            int nseg, int CB, int lane, bool act, WsHeader* hdr, int info) {
+    using R = Rec<V>;
+    int dist = 0;  // distance of the window's first tile minus one
+    int jp;        // the tile whose prefix starts the fold (out of range: the row's end, zero)
+    const unsigned long long t0 = global_ns();
+    for (int it = 0;; ++it) {
+        const int j = k + dir * (dist + 1 + lane);
+        const bool in = j >= 0 && j < nseg;
+        const unsigned int f = in ? ld_acquire(&flags[row + j]) : (unsigned int)kFlagPrefix;
+        const unsigned int pre = __ballot_sync(0xffffffffu, f == kFlagPrefix);
+        const unsigned int none = __ballot_sync(0xffffffffu, f == kFlagNone);
+        const int p = pre ? __ffs(pre) - 1 : 32, q = none ? __ffs(none) - 1 : 32;
+        if (p < q) {  // every tile before the prefix holds its aggregate
+            jp = k + dir * (dist + 1 + p);
             break;
         }
-        if (f != kFlagAgg) break;  // gave up: zero prefix
-        j += dir;
+        if (q == 32) {  // a whole window of aggregates: look further
+            dist += 32;
+            continue;
+        }
+        if (global_ns() - t0 > kWaitLimitNs) {
+            record_error(hdr, LR_ERR_TIMEOUT, info);
+            return zero_of(V{});
+        }
+        if (it > 16) __nanosleep(128);
     }
-    for (int i = j - dir; i != k; i -= dir) {
-        Agg<V> ag = act ? ld_cg_agg(&aggRec[(row + i) * CB + lane]) : Agg<V>{one_of(V{}), zero_of(V{})};
-        x = fmax_(ag.m, x, ag.v);
+    V x = zero_of(V{});
+    if (jp >= 0 && jp < nseg && act) {
+        const typename R::PreT* pp = &preRec[(row + jp) * CB + lane];
+        if (!R::get_pre(pp, x) && !reread<V, true>(pp, x, t0, hdr, info)) return zero_of(V{});
+    }
+    for (int i = jp - dir; i != k;) {
+        Agg<V> ag[KB];
+        bool got[KB];
+        int cnt = 0;
+#pragma unroll
+        for (int b = 0; b < KB; ++b) {
+            const int ii = i - dir * b;
+            const bool use = dir < 0 ? ii < k : ii > k;
+            got[b] = true;
+            ag[b] = Agg<V>{one_of(V{}), zero_of(V{})};
+            if (use && act) got[b] = R::get_agg(&aggRec[(row + ii) * CB + lane], ag[b]);
+            cnt += use ? 1 : 0;
+        }
+#pragma unroll
+        for (int b = 0; b < KB; ++b)
+            if (b < cnt) {
+                if (!got[b] &&
+                    !reread<V, false>(&aggRec[(row + i - dir * b) * CB + lane], ag[b], t0, hdr, info))
+                    return zero_of(V{});
+                x = fmax_(ag[b].m, x, ag[b].v);
+            }
+        i -= dir * cnt;
     }
     return x;
 }
@@ -242,13 +395,14 @@ __device__ V lookback_carry(const unsigned int* flags, const Agg<V>* aggRec, con
 // found it (otherwise the caller takes the look-back above, which yields the same value once the
 // neighbour's prefix is out).
 template <typename V>
-__device__ __forceinline__ bool early_carry(const unsigned int* flags, const V* preRec, size_t row, int k, int dir,
-                                            int nseg, int CB, int lane, bool act, V& x) {
+__device__ __forceinline__ bool early_carry(const unsigned int* flags, const typename Rec<V>::PreT* preRec,
+                                            size_t row, int k, int dir, int nseg, int CB, int lane, bool act,
+                                            V& x) {
     x = zero_of(V{});
     const int j = k + dir;
     if (j < 0 || j >= nseg) return true;
-    const bool ready = ld_acquire(&flags[row + j]) == kFlagPrefix;
-    if (ready && act) x = ld_cg(&preRec[(row + j) * CB + lane]);
+    bool ready = ld_acquire(&flags[row + j]) == kFlagPrefix;
+    if (ready && act) ready = Rec<V>::get_pre(&preRec[(row + j) * CB + lane], x);
     return __all_sync(0xffffffffu, ready);
 }
 
@@ -257,6 +411,24 @@ __device__ __forceinline__ char* smem_base() {
     extern __shared__ char dyn_smem[];
     uintptr_t p = reinterpret_cast<uintptr_t>(dyn_smem);
     return reinterpret_cast<char*>((p + 127) & ~uintptr_t(127)) ;
+}
+
+// Named barrier 1 over the whole CTA: warp 0 arrives once it has written the tile's carry and goes
+// on to publish the tile's prefix and checkpoint, the other warps wait only for the carry.
+__device__ __forceinline__ void carry_arrive() { asm volatile("bar.arrive 1, %0;" ::"n"(kThreads) : "memory"); }
+__device__ __forceinline__ void carry_wait() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
+
+// Aggregate loads in flight in the look-back (8 spill registers in the gated forward and rotlru's
+// backward tile kernels)
+template <int KIND> constexpr int lookback_batch() { return KIND == LR_RGLRU ? 8 : 4; }
+
+// Zeroes the head of the workspace (header, flags and, with real values, the tile records) and lets
+// the scan kernel that follows start at once (programmatic launch): that kernel waits for this one
+// only before it touches the workspace.
+__global__ void ws_zero_kernel(uint4* __restrict__ p, size_t n16) {
+    pdl_launch_dependents();
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // --------------------------------------------------------------------------------- forward
@@ -282,35 +454,40 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     constexpr bool full = FULL;  // LR_FULL_STATE: checkpoint every step
     const int grp = tid / CB, u = tid % CB;
 
+    // The tile and its loads.  The kernel starts while the workspace is being zeroed (programmatic
+    // launch after ws_zero_kernel): the inputs may be read at once, the workspace only after
+    // pdl_wait.  With tiles numbered by block index the loads are issued before that wait.
+    auto take_tile = [&](unsigned int tk) {
+        const int per_seg = a.B * a.ncb;
+        const int sg = tk / per_seg, rem = tk % per_seg, bb = rem / a.ncb, cc = rem % a.ncb;
+        misc[0] = sg;
+        misc[1] = bb;
+        misc[2] = cc;
+        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + (gated ? 2 : 1) * K::BW) * sizeof(T)));
+        tma_load_3d(Cs, &mapC, bar, cc * K::CW, sg * a.S, bb);
+        tma_load_3d(Bs, &mapB, bar, cc * K::BW, sg * a.S, bb);
+        if (gated) tma_load_3d(Xs, &mapX, bar, cc * K::BW, sg * a.S, bb);
+    };
     if (tid == 0) {
-        unsigned int tk = take_ticket(a.hdr, 0);
-        int per_seg = a.B * a.ncb;
-        int seg = tk / per_seg, rem = tk % per_seg;
-        misc[0] = seg;
-        misc[1] = rem / a.ncb;
-        misc[2] = rem % a.ncb;
         mbar_init(bar, 1);
         fence_barrier_init();
         fence_proxy_async_smem();
+        if (a.direct) take_tile(blockIdx.x);
     }
+    pdl_wait();
+    if (tid == 0 && !a.direct) take_tile(take_ticket(a.hdr, 0));
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(a.S * (K::CW + (gated ? 2 : 1) * K::BW) * sizeof(T)));
-        tma_load_3d(Cs, &mapC, bar, cb * K::CW, t0g, b);
-        tma_load_3d(Bs, &mapB, bar, cb * K::BW, t0g, b);
-        if (gated) tma_load_3d(Xs, &mapX, bar, cb * K::BW, t0g, b);
-    }
     const int unit = cb * CB + u;  // global unit index (channel or pair)
     const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
     const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
-    Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
-    V* preRec = reinterpret_cast<V*>(a.pre);
+    auto* aggRec = reinterpret_cast<typename Rec<V>::AggT*>(a.agg);
+    auto* preRec = reinterpret_cast<typename Rec<V>::PreT*>(a.pre);
     const bool act = warp == 0 && lane < CB && unit < units;
     V carry = zero_of(V{});
     bool have = false;
-    if (warp == 0) have = early_carry(a.flags, preRec, row, seg, -1, a.nseg, CB, lane, act, carry);
+    if (warp == 0) have = early_carry<V>(a.flags, preRec, row, seg, -1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     const int nt = min(a.S, a.L - t0g);
     const int spg = (a.S + NG - 1) / NG;
@@ -337,11 +514,10 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     aggF[grp * CB + u] = {P, h};
     __syncthreads();
 
-    // tile carry through the chained look-back (warp 0, one lane per unit); the carry is usually
-    // known already (early_carry), and this tile's own prefix is published after the other warps
-    // have been released
+    // tile carry through the chained look-back (warp 0, one lane per unit; usually known already,
+    // early_carry); warp 0 then releases the other warps and publishes the tile's inclusive prefix
+    // at once, since the look-backs of later tiles wait for it (the first segment's in particular)
     const bool has_succ = seg + 1 < a.nseg;
-    V pub = zero_of(V{});
     if (warp == 0) {
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB) {
@@ -353,27 +529,23 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         }
         if (!have) {
             if (seg > 0 && has_succ) {
-                if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+                publish_agg<V>(&a.flags[row + seg], &aggRec[(row + seg) * CB + lane], tile, act, lane);
             }
-            carry = lookback_carry(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane, act, a.hdr, 101);
+            carry = lookback_carry<lookback_batch<KIND>(), V>(a.flags, aggRec, preRec, row, seg, -1, a.nseg, CB, lane,
+                                                           act, a.hdr, 101);
         }
-        pub = fmax_(tile.m, carry, tile.v);
-        const size_t slot = full ? (size_t)t0g : (size_t)seg;  // state entering the segment
-        if (act) K::st_ckpt(a.ckpt + (slot * a.B + b) * a.D, unit * K::chans_per_unit, carry);
         if (lane < CB) carryS[lane] = carry;
-    }
-    __syncthreads();
-    if (warp == 0) {
+        __syncwarp();
+        carry_arrive();
         const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == 0;
         if (has_succ && !withhold) {
-            if (act) st_cg(&preRec[(row + seg) * CB + lane], pub);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
+            publish_pre<V>(&a.flags[row + seg], &preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v), act,
+                           lane);
         }
+        const size_t slot = full ? (size_t)t0g : (size_t)seg;  // state entering the segment
+        if (act) K::st_ckpt(a.ckpt + (slot * a.B + b) * a.D, unit * K::chans_per_unit, carry);
+    } else {
+        carry_wait();
     }
 
     // apply: recompute the group with its true carry-in, write y into the b slot
@@ -436,42 +608,47 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     // is not needed)
     constexpr bool full = FULL;
 
+    // The tile (later segments first) and its loads: coefficients and b (the forward recompute) on
+    // bar[0], dy (the adjoint) on bar[1].  As in the forward kernel, the workspace is touched only
+    // after pdl_wait, and with tiles numbered by block index the loads are issued before it.
+    auto take_tile = [&](unsigned int tk) {
+        const int per_seg = a.B * a.ncb;
+        const int sg = a.nseg - 1 - (int)(tk / per_seg), rem = tk % per_seg, bb = rem / a.ncb, cc = rem % a.ncb;
+        misc[0] = sg;
+        misc[1] = bb;
+        misc[2] = cc;
+        const int t0 = sg * a.S;
+        mbar_arrive_expect_tx(&bar[0],
+                              (uint32_t)(a.S * (K::CW + (full ? 0 : K::BW) + (gated ? K::BW : 0)) * sizeof(T)));
+        tma_load_3d(Cs, &mapC, &bar[0], cc * K::CW, t0, bb);
+        if (!full) tma_load_3d(Bs, &mapB, &bar[0], cc * K::BW, t0, bb);
+        if (gated) tma_load_3d(Xs, &mapX, &bar[0], cc * K::BW, t0, bb);
+        if (!(SM::AL && !full)) {
+            mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
+            tma_load_3d(Ds, &mapDY, &bar[1], cc * K::BW, t0, bb);
+        }
+    };
     if (tid == 0) {
-        unsigned int tk = take_ticket(a.hdr, 1);
-        int per_seg = a.B * a.ncb;
-        int seg = a.nseg - 1 - (int)(tk / per_seg), rem = tk % per_seg;
-        misc[0] = seg;
-        misc[1] = rem / a.ncb;
-        misc[2] = rem % a.ncb;
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
+        if (a.direct) take_tile(blockIdx.x);
     }
+    pdl_wait();
+    if (tid == 0 && !a.direct) take_tile(take_ticket(a.hdr, 1));
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
-    // coefficients and b (the forward recompute) on bar[0], dy (the adjoint) on bar[1]
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar[0],
-                              (uint32_t)(a.S * (K::CW + (full ? 0 : K::BW) + (gated ? K::BW : 0)) * sizeof(T)));
-        tma_load_3d(Cs, &mapC, &bar[0], cb * K::CW, t0g, b);
-        if (!full) tma_load_3d(Bs, &mapB, &bar[0], cb * K::BW, t0g, b);
-        if (gated) tma_load_3d(Xs, &mapX, &bar[0], cb * K::BW, t0g, b);
-        if (!(SM::AL && !full)) {
-            mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
-            tma_load_3d(Ds, &mapDY, &bar[1], cb * K::BW, t0g, b);
-        }
-    }
     const int unit = cb * CB + u;
     const int units = K::chans_per_unit == 1 ? a.D : a.D / 2;
     const size_t row = (size_t)(b * a.ncb + cb) * a.nseg;
-    Agg<V>* aggRec = reinterpret_cast<Agg<V>*>(a.agg);
-    V* preRec = reinterpret_cast<V*>(a.pre);
+    auto* aggRec = reinterpret_cast<typename Rec<V>::AggT*>(a.agg);
+    auto* preRec = reinterpret_cast<typename Rec<V>::PreT*>(a.pre);
     const bool act = warp == 0 && lane < CB && unit < units;
     V carry = zero_of(V{});
     bool have = false;
-    if (warp == 0) have = early_carry(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
+    if (warp == 0) have = early_carry<V>(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     if (tid < CB && !full) {
         V c0 = zero_of(V{});
@@ -552,9 +729,9 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     }
     __syncthreads();
 
-    // tile carry from later segments (warp 0; usually known already, see the forward kernel)
+    // tile carry from later segments (warp 0; usually known already), then the other warps are
+    // released and the tile's prefix published, as in the forward kernel
     const bool has_pred = seg > 0;  // earlier segment waits on this one
-    V pub = zero_of(V{});
     if (warp == 0) {
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB)
@@ -565,25 +742,21 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             }
         if (!have) {
             if (has_pred && seg + 1 < a.nseg) {
-                if (act) st_cg_agg(&aggRec[(row + seg) * CB + lane], tile);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release(&a.flags[row + seg], kFlagAgg);
+                publish_agg<V>(&a.flags[row + seg], &aggRec[(row + seg) * CB + lane], tile, act, lane);
             }
-            carry = lookback_carry(a.flags, aggRec, preRec, row, seg, +1, a.nseg, CB, lane, act, a.hdr, 201);
+            carry = lookback_carry<lookback_batch<KIND>(), V>(a.flags, aggRec, preRec, row, seg, +1, a.nseg, CB, lane,
+                                                           act, a.hdr, 201);
         }
-        pub = fmax_(tile.m, carry, tile.v);
         if (lane < CB) carryS[CB + lane] = carry;
-    }
-    __syncthreads();
-    if (warp == 0) {
+        __syncwarp();
+        carry_arrive();
         const bool withhold = (a.dflags & LR_TEST_WITHHOLD_CARRY) && seg == a.nseg - 1;
         if (has_pred && !withhold) {
-            if (act) st_cg(&preRec[(row + seg) * CB + lane], pub);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.flags[row + seg], kFlagPrefix);
+            publish_pre<V>(&a.flags[row + seg], &preRec[(row + seg) * CB + lane], fmax_(tile.m, carry, tile.v), act,
+                           lane);
         }
+    } else {
+        carry_wait();
     }
 
     // adjoint sweep of the group with its true carry; gradients into the shared slots
@@ -717,24 +890,44 @@ Geo geo(const lr_desc& d) {
     return g;
 }
 
+// Tiles may be numbered by block index, instead of by a ticket taken as each CTA starts, when the
+// grid has at most one CTA per SM: all of its CTAs can then be resident together, so a tile that
+// waits for another never keeps it from starting, whatever order the CTAs start in.  The ticket
+// costs a global atomic round trip before the tile's loads can be issued.
+bool direct_tiles(const Geo& g) { return g.tiles <= device_sm_count(); }
+
 struct DiagWs {
-    size_t flags, agg, pre, partial, end;
+    size_t flags, agg, pre, zero_end, partial, end;
 };
 
+// Workspace: flags, then the tiles' aggregate and prefix records (8 bytes per unit and record
+// value: a complex value, or a real value with its status word), then partials.  Zeroed before each
+// call: the flags, and with real values the records too (their status words).
 DiagWs ws_plan(const lr_desc& d, bool bwd) {
     Geo g = geo(d);
-    size_t vs = d.kind == LR_RGLRU ? 4 : 8;
+    const size_t vs = 8;
     WsCursor c;
     DiagWs w;
     w.flags = c.take(sizeof(unsigned int) * g.tiles);
     w.agg = c.take(2 * vs * g.cb * (size_t)g.tiles);
     w.pre = c.take(vs * g.cb * (size_t)g.tiles);
+    w.zero_end = d.kind == LR_RGLRU ? c.off : w.agg;
     const bool gates = d.kind == LR_RGLRU && (d.flags & LR_RGLRU_GATES);
     w.partial = (bwd && (d.kind == LR_ROTLRU || gates))
                     ? c.take(sizeof(float2) * d.B * g.nseg * (d.kind == LR_ROTLRU ? d.D / 2 : d.D))
                     : 0;
     w.end = c.off;
     return w;
+}
+
+// Zero the workspace head the scan kernel relies on (ws_zero_kernel; the scan kernel is launched
+// after it as a programmatic dependent).
+lr_status zero_ws(const lr_desc& d, bool bwd, char* ws, cudaStream_t st) {
+    const size_t n16 = ws_plan(d, bwd).zero_end / 16;
+    const int blocks = (int)std::min<size_t>((n16 + 255) / 256, (size_t)4 * device_sm_count());
+    note_launch("diag_ws_zero");
+    ws_zero_kernel<<<std::max(blocks, 1), 256, 0, st>>>(reinterpret_cast<uint4*>(ws), n16);
+    return check_launch();
 }
 
 // The dynamic shared-memory limit is a per-device attribute of the function, so it is set on every
@@ -763,7 +956,7 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
     else
         mX = mB;  // not read
     if (!ok) return LR_ERR_INVALID_ARG;
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), in.mag, in.theta,
                in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
@@ -772,8 +965,12 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
         set_smem_attr<KIND, T, false, true>((const void*)fn);
     else
         set_smem_attr<KIND, T, false, false>((const void*)fn);
+    lr_status s = zero_ws(d, false, ws, st);
+    if (s != LR_OK) return s;
     note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : KIND == kRgGated ? "rglru_gated_fwd_tile" : "rotlru_fwd_tile");
-    fn<<<g.tiles, kThreads, Smem<KIND, T, false>::total(), st>>>(mC, mB, mX, mY, a);
+    if (launch_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, false>::total(), st, true, mC, mB, mX, mY, a) !=
+        cudaSuccess)
+        return LR_ERR_CUDA;
     return check_launch();
 }
 
@@ -802,7 +999,7 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
         mDX = mDB;  // not written
     }
     if (!ok) return LR_ERR_INVALID_ARG;
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, in.mag, in.theta,
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), in.mag, in.theta,
                in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                w.partial ? (float2*)(ws + w.partial) : nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
@@ -811,9 +1008,13 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
         set_smem_attr<KIND, T, true, true>((const void*)fn);
     else
         set_smem_attr<KIND, T, true, false>((const void*)fn);
+    lr_status s = zero_ws(d, true, ws, st);
+    if (s != LR_OK) return s;
     note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : KIND == kRgGated ? "rglru_gated_bwd_tile" : "rotlru_bwd_tile");
-    fn<<<g.tiles, kThreads, Smem<KIND, T, true>::total(), st>>>(mC, mB, mX, mDY, mDC, mDB, mDX, a);
-    lr_status s = check_launch();
+    if (launch_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, true>::total(), st, true, mC, mB, mX, mDY, mDC,
+                  mDB, mDX, a) != cudaSuccess)
+        return LR_ERR_CUDA;
+    s = check_launch();
     if (s != LR_OK) return s;
     if (KIND == LR_ROTLRU) {
         int K2 = (int)(d.D / 2);
@@ -834,7 +1035,7 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
 }  // namespace
 
 size_t diag_ws_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).end; }
-size_t diag_flag_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).agg; }
+size_t diag_flag_bytes(const lr_desc& d, bool bwd) { return ws_plan(d, bwd).zero_end; }
 
 lr_status diag_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt, char* ws,
                    cudaStream_t st) {

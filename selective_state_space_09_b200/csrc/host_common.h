@@ -62,6 +62,15 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return launch_ex(kernel, grid, block, smem, st, true, args...);
 }
 
+// Number of SMs of the current device (queried on every call: a process may drive several devices).
+inline int device_sm_count() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+                                                      cudaSuccess && v > 0)
+        return v;
+    return 148;
+}
+
 // Byte offset bookkeeping for a workspace: a 256-byte header followed by regions.
 struct WsCursor {
     size_t off = 256;

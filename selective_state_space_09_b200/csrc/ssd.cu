@@ -495,14 +495,7 @@ SsdArgs make_args(const lr_desc& d, const lr_inputs& in, const void* ckpt, char*
     return a;
 }
 
-// Number of SMs of the current device (queried on every call: a process may drive several devices).
-int sm_count() {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
-                                                      cudaSuccess && v > 0)
-        return v;
-    return 148;
-}
+int sm_count() { return device_sm_count(); }
 
 // Heads per output CTA (at most 16; 16 under LR_TEST_MAX_HEAD_BLOCK).  A CTA takes about 2 units
 // per head of each warpgroup (two warpgroups alternate heads) plus 1 unit of prologue (C, B loads

@@ -40,7 +40,7 @@ def test_rglru_parity(B, L, D, S, io):
     assert_close("ckpt", ck, rck, max(tol, 1e-5))
     assert_close("da", gr["da"], rg["a"], tol)
     assert_close("db", gr["db"], rg["b"], tol)
-    assert disp == ("rglru_fwd_tile", "rglru_bwd_tile")
+    assert disp == ("diag_ws_zero+rglru_fwd_tile", "diag_ws_zero+rglru_bwd_tile")
     assert plan.device_error() == (0, 0)
 
 
@@ -70,7 +70,7 @@ def test_rglru_gated_parity(B, L, D, S):
     assert_close("di", gr["db"], rg["i"], tol)
     assert_close("dx", gr["dx"], rg["x"], tol)
     assert_close("dLambda", gr["dA"], rg["lam"], tol)
-    assert disp == ("rglru_gated_fwd_tile", "rglru_gated_bwd_tile+rglru_param_reduce")
+    assert disp == ("diag_ws_zero+rglru_gated_fwd_tile", "diag_ws_zero+rglru_gated_bwd_tile+rglru_param_reduce")
     assert plan.device_error() == (0, 0)
 
 
@@ -113,7 +113,7 @@ def test_rglru_gated_autograd_and_optional_dlambda():
     del g2["dA"]
     p2.bwd(g, inp["dy"].cuda(), g2)
     torch.cuda.synchronize()
-    assert lrscan.last_dispatch() == "rglru_gated_bwd_tile"
+    assert lrscan.last_dispatch() == "diag_ws_zero+rglru_gated_bwd_tile"
     for k in ("da", "db", "dx"):
         assert torch.equal(g2[k], gr[k]), k
 
@@ -140,7 +140,7 @@ def test_rotlru_parity(B, L, D, S, io):
     assert_close("dg", gr["dg"], rg["g"], tol)
     assert_close("dmag", gr["dmag"], rg["mag"], max(tol, 1e-5))
     assert_close("dtheta", gr["dtheta"], rg["theta"], max(tol, 1e-5))
-    assert disp == ("rotlru_fwd_tile", "rotlru_bwd_tile+rotlru_param_reduce")
+    assert disp == ("diag_ws_zero+rotlru_fwd_tile", "diag_ws_zero+rotlru_bwd_tile+rotlru_param_reduce")
     assert plan.device_error() == (0, 0)
 
 
@@ -227,3 +227,42 @@ def test_full_state_mode(kind, B, L, D, S, io):
     for k, r in pairs:
         assert_close(k, g1[k], rg[r], tol)
     assert plan.device_error() == (0, 0)
+
+
+def test_entry_points_from_a_fresh_thread():
+    """The entry points called from a thread that has made no CUDA call of its own (as a
+    framework's backward worker may be): the tensor-map encoder, a driver call, needs the thread
+    bound to the device's context, which the library does itself.  Results equal a call from the
+    main thread bitwise."""
+    import ctypes
+    import threading
+    from selective_state_space_09_b200 import lrscan
+    inp = gpu_inputs(inputs.rglru(2, 300, 96, seed=5))
+    dy = inp.pop("dy")
+    desc = lrscan.desc_for("rglru", inp, 64)
+    ref_plan = lrscan.Plan(desc)
+    y_ref, g_ref = lrscan.alloc_outputs("rglru", inp)
+    ref_plan.fwd(inp, y_ref)
+    ref_plan.bwd(inp, dy, g_ref)
+    torch.cuda.synchronize()
+    plan = lrscan.Plan(desc)
+    y, g = lrscan.alloc_outputs("rglru", inp)
+    ii = lrscan.Inputs(*[lrscan._ptr(inp.get(n)) for n in lrscan._IN])
+    gg = lrscan.Grads(*[lrscan._ptr(g.get(n)) for n in lrscan._GR])
+    args = (ctypes.byref(desc), ctypes.byref(ii))
+    status = []
+
+    def work():  # the legacy default stream; no torch call on this thread
+        status.append(lrscan.lib.lr_scan_fwd(*args, lrscan._ptr(y), lrscan._ptr(plan.ckpt), lrscan._ptr(plan.ws),
+                                             plan.ws_bytes, None))
+        status.append(lrscan.lib.lr_scan_bwd(*args, lrscan._ptr(dy), lrscan._ptr(plan.ckpt), ctypes.byref(gg),
+                                             lrscan._ptr(plan.ws), plan.ws_bytes, None))
+
+    th = threading.Thread(target=work)
+    th.start()
+    th.join()
+    torch.cuda.synchronize()
+    assert status == [0, 0]
+    assert torch.equal(y, y_ref)
+    for k in g_ref:
+        assert torch.equal(g[k], g_ref[k]), k

@@ -479,6 +479,26 @@ def run_workload(name, steps, warmup, device, rank, world, flush_buf, e2e=False,
         warm = {"ms_fwd": round(wf, 5), "ms_bwd": round(wb, 5),
                 "tokens_per_s": round(tokens_of(w) * world / ((wf + wb) * 1e-3), 1)}
 
+    # The same steps replayed from a CUDA graph of the two calls (lrscan.StepGraph), one rank: the
+    # kernels and their work are the same, the per-launch overhead is paid once per graph.
+    graph = None
+    if world == 1:
+        sg = lrscan.StepGraph(plan, ai, dy, y, grads)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            if fl is not None:
+                fl.fill_(float(i))
+            host_ahead()
+            gev[i][0].record()
+            sg.replay()
+            gev[i][1].record()
+        torch.cuda.synchronize()
+        gms = statistics.mean(a.elapsed_time(b) for a, b in gev)
+        graph = {"ms_per_step": round(gms, 5), "tokens_per_s": round(tokens_of(w) / (gms * 1e-3), 1),
+                 "l2": "flushed between steps" if flush else "inputs larger than L2"}
+        del sg
+
     def kernel_ms(kev, ends):
         n = len(kev[0])
         return [statistics.mean(kev[s][k].elapsed_time(kev[s][k + 1] if k + 1 < n else ends[s])
@@ -517,6 +537,7 @@ def run_workload(name, steps, warmup, device, rank, world, flush_buf, e2e=False,
         "io_dtype": "bf16" if y.dtype == torch.bfloat16 else "f32",
         "l2": "flushed between steps" if flush else "inputs larger than L2",
         "l2_warm": warm,
+        "graph": graph,
     }
     if e2e:
         res["e2e"] = run_e2e(plan, kind, ai, dy, y, grads, steps, warmup, world, w)
@@ -982,6 +1003,8 @@ def main():
         }
         if r.get("l2_warm"):
             per_kind[name]["l2_warm"] = r["l2_warm"]
+        if r.get("graph"):
+            per_kind[name]["graph"] = r["graph"]
         if "decode" in r:
             d = dict(r["decode"])
             d["tokens_per_s"] = round(d["tokens_per_s"], 1)
@@ -1008,6 +1031,7 @@ def main():
                    "l2": h["l2"]},
         "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in h["e2e"].items()},
         "gpu_launches": args.steps * sum(r["launches_per_step"] for r in [h]),
+        "graph": h.get("graph"),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clocks,

@@ -297,6 +297,30 @@ class DecodeGraph:
         self.graph.replay()
 
 
+class StepGraph:
+    """The forward and backward call of one training step of ``plan`` captured once in a CUDA
+    graph; ``replay()`` runs both again on the same buffers (each kernel launch is then a node of
+    one graph launch instead of a separate stream launch).  ``inp``, ``dy``, ``y`` and ``grads``
+    are the tensors given here: write a step's inputs into them before a replay, read its results
+    after.  The kernels and their work are those of ``plan.fwd`` / ``plan.bwd``."""
+
+    def __init__(self, plan, inp, dy, y, grads):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # one eager step settles lazy initialisation
+            plan.fwd(inp, y)
+            plan.bwd(inp, dy, grads)
+        torch.cuda.current_stream().wait_stream(side)
+        self.plan = plan
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            plan.fwd(inp, y)
+            plan.bwd(inp, dy, grads)
+
+    def replay(self):
+        self.graph.replay()
+
+
 def alloc_outputs(kind, inp):
     """Output tensor and empty gradient tensors for a kind (shapes/dtypes of the header)."""
     e = torch.empty_like

@@ -135,6 +135,11 @@ typedef enum { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
  * the GPU.  Results are bitwise identical with and without it; small test problems use it to
  * cover the multi-head pipelines. */
 #define LR_TEST_MAX_HEAD_BLOCK 0x40000000u
+/* Test hook for the carry exchange of rglru / rotlru: rows of at most 8 segment tiles normally run
+ * as one thread-block cluster whose tiles exchange their aggregates through distributed shared
+ * memory; with this flag they take the look-back over global-memory records that longer rows use.
+ * Results are bitwise identical either way. */
+#define LR_TEST_LOOKBACK 0x20000000u
 
 /* Problem descriptor.  Unused dimensions are 0.  S6: D, N.  SSD: H, P, N, G, chunk.
  * GLA: H, P (= V), N (= K), chunk.  rglru / rotlru: D.  segment = checkpoint segment length S

@@ -57,6 +57,7 @@ struct DiagArgs {
     int B, L, D, S, nseg, ncb;  // D = real channels of b / y
     unsigned int dflags;        // lr_desc flags (LR_TEST_WITHHOLD_CARRY)
     int direct;                 // tiles numbered by block index (the grid fits on the SMs at once)
+    int cl;                     // > 0: a row's tiles form one thread-block cluster of cl CTAs (cl = nseg)
     const float* mag;           // rotlru
     const float* theta;         // rotlru
     const float* lam;           // rglru with gates: Lambda [D]
@@ -176,7 +177,8 @@ template <int KIND, typename T, bool BWD> struct Smem {
     static __host__ __device__ constexpr size_t off_carry() {
         return off_aggr() + (BWD ? sizeof(Agg<V>) * K::NG * K::CB : 0);
     }
-    static __host__ __device__ constexpr size_t off_red() { return off_carry() + 2 * sizeof(V) * K::CB; }
+    static __host__ __device__ constexpr size_t off_cl() { return off_carry() + 2 * sizeof(V) * K::CB; }
+    static __host__ __device__ constexpr size_t off_red() { return off_cl() + sizeof(Agg<V>) * K::CB; }
     static __host__ __device__ constexpr size_t off_misc() {
         return off_red() + (BWD ? sizeof(float2) * K::NG * K::CB : 0);
     }
@@ -418,6 +420,52 @@ __device__ __forceinline__ char* smem_base() {
 __device__ __forceinline__ void carry_arrive() { asm volatile("bar.arrive 1, %0;" ::"n"(kThreads) : "memory"); }
 __device__ __forceinline__ void carry_wait() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 
+// Thread-block clusters: a row of at most 8 tiles runs as one cluster, and the tiles exchange their
+// aggregates through distributed shared memory instead of global-memory records.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, int rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ Agg<float> ld_dsmem_agg(uint32_t addr, float) {
+    float m, v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(m), "=f"(v) : "r"(addr) : "memory");
+    return {m, v};
+}
+__device__ __forceinline__ Agg<cpx> ld_dsmem_agg(uint32_t addr, cpx) {
+    float a, b, c, d;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(a), "=f"(b), "=f"(c), "=f"(d) : "r"(addr)
+                 : "memory");
+    return {{a, b}, {c, d}};
+}
+constexpr int kMaxCluster = 8;  // portable cluster size
+
+// Cluster mode: the carry entering tile `seg` from the aggregates the other tiles of the row left in
+// their cluster slot (dir = -1: ranks 0 .. seg - 1, folded in that order; dir = +1: ranks nseg - 1
+// down to seg + 1), x <- m x + v from zero -- the same operations as the chained look-back.
+// Warp 0, one lane per unit, after the cluster barrier that follows the slots' writes.
+template <typename V>
+__device__ __forceinline__ V cluster_carry(const Agg<V>* clAgg, int seg, int nseg, int dir, int lane, int CB) {
+    V x = zero_of(V{});
+    if (lane >= CB) return x;
+    const uint32_t local = smem_u32(clAgg + lane);
+    Agg<V> ag[kMaxCluster];
+#pragma unroll
+    for (int i = 0; i < kMaxCluster; ++i) {
+        const int j = dir < 0 ? i : nseg - 1 - i;
+        const bool use = dir < 0 ? j < seg : j > seg;
+        ag[i] = use ? ld_dsmem_agg(dsmem_addr(local, j), V{}) : Agg<V>{one_of(V{}), zero_of(V{})};
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxCluster; ++i) {
+        const int j = dir < 0 ? i : nseg - 1 - i;
+        if (dir < 0 ? j < seg : j > seg) x = fmax_(ag[i].m, x, ag[i].v);
+    }
+    return x;
+}
+
 // Aggregate loads in flight in the look-back (8 spill registers in the gated forward and rotlru's
 // backward tile kernels)
 template <int KIND> constexpr int lookback_batch() { return KIND == LR_RGLRU ? 8 : 4; }
@@ -433,7 +481,7 @@ __global__ void ws_zero_kernel(uint4* __restrict__ p, size_t n16) {
 
 // --------------------------------------------------------------------------------- forward
 template <int KIND, typename T, bool FULL>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, KIND == LR_ROTLRU ? 4 : 2)  // tiles per SM (registers)
 diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapY, DiagArgs a) {
     using K = Kind<KIND, T>;
@@ -472,10 +520,13 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         mbar_init(bar, 1);
         fence_barrier_init();
         fence_proxy_async_smem();
-        if (a.direct) take_tile(blockIdx.x);
+        if (a.cl)  // the row's tiles are the cluster's CTAs, in segment order
+            take_tile((blockIdx.x % a.cl) * (a.B * a.ncb) + blockIdx.x / a.cl);
+        else if (a.direct)
+            take_tile(blockIdx.x);
     }
     pdl_wait();
-    if (tid == 0 && !a.direct) take_tile(take_ticket(a.hdr, 0));
+    if (tid == 0 && !a.cl && !a.direct) take_tile(take_ticket(a.hdr, 0));
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
@@ -487,7 +538,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const bool act = warp == 0 && lane < CB && unit < units;
     V carry = zero_of(V{});
     bool have = false;
-    if (warp == 0) have = early_carry<V>(a.flags, preRec, row, seg, -1, a.nseg, CB, lane, act, carry);
+    if (warp == 0 && !a.cl) have = early_carry<V>(a.flags, preRec, row, seg, -1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     const int nt = min(a.S, a.L - t0g);
     const int spg = (a.S + NG - 1) / NG;
@@ -518,7 +569,32 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     // early_carry); warp 0 then releases the other warps and publishes the tile's inclusive prefix
     // at once, since the look-backs of later tiles wait for it (the first segment's in particular)
     const bool has_succ = seg + 1 < a.nseg;
-    if (warp == 0) {
+    Agg<V>* clAgg = reinterpret_cast<Agg<V>*>(sm + SM::off_cl());
+    if (a.cl) {  // cluster mode: slots, barrier, fold of the earlier tiles' slots
+        if (warp == 0 && lane < CB) {
+            Agg<V> tile{one_of(V{}), zero_of(V{})};
+            for (int g = 0; g < NG; ++g) {
+                Agg<V> ag = aggF[g * CB + lane];
+                tile.v = fmax_(ag.m, tile.v, ag.v);
+                tile.m = mulx(ag.m, tile.m);
+            }
+            clAgg[lane] = tile;
+        }
+        cluster_arrive();
+        cluster_wait();
+        if (warp == 0) {
+            carry = cluster_carry(clAgg, seg, a.nseg, -1, lane, CB);
+            if (lane < CB) carryS[lane] = carry;
+            __syncwarp();
+            carry_arrive();
+            cluster_arrive();  // done reading the other tiles' slots
+            const size_t slot = full ? (size_t)t0g : (size_t)seg;
+            if (act) K::st_ckpt(a.ckpt + (slot * a.B + b) * a.D, unit * K::chans_per_unit, carry);
+        } else {
+            cluster_arrive();
+            carry_wait();
+        }
+    } else if (warp == 0) {
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB) {
             for (int g = 0; g < NG; ++g) {
@@ -572,6 +648,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         bulk_commit();
         bulk_wait_read_all();
     }
+    if (a.cl) cluster_wait();  // no tile's slot is read after its CTA has exited
 }
 
 // -------------------------------------------------------------------------------- backward
@@ -633,10 +710,13 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         mbar_init(&bar[1], 1);
         fence_barrier_init();
         fence_proxy_async_smem();
-        if (a.direct) take_tile(blockIdx.x);
+        if (a.cl)  // the row's tiles are the cluster's CTAs; tile numbers count later segments first
+            take_tile((a.nseg - 1 - (int)(blockIdx.x % a.cl)) * (a.B * a.ncb) + blockIdx.x / a.cl);
+        else if (a.direct)
+            take_tile(blockIdx.x);
     }
     pdl_wait();
-    if (tid == 0 && !a.direct) take_tile(take_ticket(a.hdr, 1));
+    if (tid == 0 && !a.cl && !a.direct) take_tile(take_ticket(a.hdr, 1));
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
@@ -648,7 +728,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     const bool act = warp == 0 && lane < CB && unit < units;
     V carry = zero_of(V{});
     bool have = false;
-    if (warp == 0) have = early_carry<V>(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
+    if (warp == 0 && !a.cl) have = early_carry<V>(a.flags, preRec, row, seg, +1, a.nseg, CB, lane, act, carry);
     typename K::Unit U(a, unit);
     if (tid < CB && !full) {
         V c0 = zero_of(V{});
@@ -732,7 +812,30 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
     // tile carry from later segments (warp 0; usually known already), then the other warps are
     // released and the tile's prefix published, as in the forward kernel
     const bool has_pred = seg > 0;  // earlier segment waits on this one
-    if (warp == 0) {
+    Agg<V>* clAgg = reinterpret_cast<Agg<V>*>(sm + SM::off_cl());
+    if (a.cl) {  // cluster mode, as in the forward kernel (the later tiles' slots)
+        if (warp == 0 && lane < CB) {
+            Agg<V> tile{one_of(V{}), zero_of(V{})};
+            for (int g = NG - 1; g >= 0; --g) {
+                Agg<V> ag = aggR[g * CB + lane];
+                tile.v = fmax_(ag.m, tile.v, ag.v);
+                tile.m = mulx(ag.m, tile.m);
+            }
+            clAgg[lane] = tile;
+        }
+        cluster_arrive();
+        cluster_wait();
+        if (warp == 0) {
+            carry = cluster_carry(clAgg, seg, a.nseg, +1, lane, CB);
+            if (lane < CB) carryS[CB + lane] = carry;
+            __syncwarp();
+            carry_arrive();
+            cluster_arrive();
+        } else {
+            cluster_arrive();
+            carry_wait();
+        }
+    } else if (warp == 0) {
         Agg<V> tile{one_of(V{}), zero_of(V{})};
         if (lane < CB)
             for (int g = NG - 1; g >= 0; --g) {
@@ -831,6 +934,7 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         bulk_commit();
         bulk_wait_read_all();
     }
+    if (a.cl) cluster_wait();  // no tile's slot is read after its CTA has exited
 }
 
 // Fixed-order reduction of rotlru's per-tile parameter partials over (batch row, segment).  A
@@ -896,6 +1000,15 @@ Geo geo(const lr_desc& d) {
 // costs a global atomic round trip before the tile's loads can be issued.
 bool direct_tiles(const Geo& g) { return g.tiles <= device_sm_count(); }
 
+// A row of 2 .. 8 tiles runs as one thread-block cluster (cluster mode): its tiles exchange
+// aggregates through distributed shared memory, with no global records, flags or waits on other
+// CTAs.  Longer rows take the look-back, and so do calls with the failure-path test flag (a
+// withheld carry needs the look-back's bounded waits) or the look-back test flag.
+int cluster_size(const lr_desc& d, const Geo& g) {
+    if (d.flags & (LR_TEST_WITHHOLD_CARRY | LR_TEST_LOOKBACK)) return 0;
+    return (g.nseg >= 2 && g.nseg <= kMaxCluster) ? g.nseg : 0;
+}
+
 struct DiagWs {
     size_t flags, agg, pre, zero_end, partial, end;
 };
@@ -923,7 +1036,7 @@ DiagWs ws_plan(const lr_desc& d, bool bwd) {
 // Zero the workspace head the scan kernel relies on (ws_zero_kernel; the scan kernel is launched
 // after it as a programmatic dependent).
 lr_status zero_ws(const lr_desc& d, bool bwd, char* ws, cudaStream_t st) {
-    const size_t n16 = ws_plan(d, bwd).zero_end / 16;
+    const size_t n16 = (cluster_size(d, geo(d)) ? 256 : ws_plan(d, bwd).zero_end) / 16;  // cluster mode: header
     const int blocks = (int)std::min<size_t>((n16 + 255) / 256, (size_t)4 * device_sm_count());
     note_launch("diag_ws_zero");
     ws_zero_kernel<<<std::max(blocks, 1), 256, 0, st>>>(reinterpret_cast<uint4*>(ws), n16);
@@ -956,7 +1069,8 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
     else
         mX = mB;  // not read
     if (!ok) return LR_ERR_INVALID_ARG;
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), in.mag, in.theta,
+    const int cl = cluster_size(d, g);
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl, in.mag, in.theta,
                in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
@@ -968,8 +1082,8 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
     lr_status s = zero_ws(d, false, ws, st);
     if (s != LR_OK) return s;
     note_launch(KIND == LR_RGLRU ? "rglru_fwd_tile" : KIND == kRgGated ? "rglru_gated_fwd_tile" : "rotlru_fwd_tile");
-    if (launch_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, false>::total(), st, true, mC, mB, mX, mY, a) !=
-        cudaSuccess)
+    if (launch_cluster_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, false>::total(), st, true, cl, mC, mB, mX,
+                          mY, a) != cudaSuccess)
         return LR_ERR_CUDA;
     return check_launch();
 }
@@ -999,7 +1113,8 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
         mDX = mDB;  // not written
     }
     if (!ok) return LR_ERR_INVALID_ARG;
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), in.mag, in.theta,
+    const int cl = cluster_size(d, g);
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl, in.mag, in.theta,
                in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                w.partial ? (float2*)(ws + w.partial) : nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
@@ -1011,8 +1126,8 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
     lr_status s = zero_ws(d, true, ws, st);
     if (s != LR_OK) return s;
     note_launch(KIND == LR_RGLRU ? "rglru_bwd_tile" : KIND == kRgGated ? "rglru_gated_bwd_tile" : "rotlru_bwd_tile");
-    if (launch_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, true>::total(), st, true, mC, mB, mX, mDY, mDC,
-                  mDB, mDX, a) != cudaSuccess)
+    if (launch_cluster_ex(fn, dim3(g.tiles), dim3(kThreads), Smem<KIND, T, true>::total(), st, true, cl, mC, mB, mX,
+                          mDY, mDC, mDB, mDX, a) != cudaSuccess)
         return LR_ERR_CUDA;
     s = check_launch();
     if (s != LR_OK) return s;

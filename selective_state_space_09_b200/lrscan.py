@@ -24,7 +24,7 @@ DISC = {"none": 0, "zoh": 1, "bilinear": 2, "dirac": 3, "zoh_euler": 4}
 IO = {torch.float32: 0, torch.bfloat16: 1}
 HAS_Z, HAS_DSKIP, FULL_STATE, DELTA_SOFTPLUS, RGLRU_GATES = 1, 2, 4, 8, 16
 # test hooks (lrscan.h): withheld carry (timeout path), widest SSD head blocks
-TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK = 0x80000000, 0x40000000
+TEST_WITHHOLD_CARRY, TEST_MAX_HEAD_BLOCK, TEST_LOOKBACK = 0x80000000, 0x40000000, 0x20000000
 STATUS = ["ok", "invalid argument", "unsupported by this library", "misaligned pointer or innermost extent",
           "workspace too small", "CUDA runtime error", "device wait timed out",
           "device consistency check failed"]

@@ -266,3 +266,20 @@ def test_entry_points_from_a_fresh_thread():
     assert torch.equal(y, y_ref)
     for k in g_ref:
         assert torch.equal(g[k], g_ref[k]), k
+
+
+@pytest.mark.parametrize("kind,B,L,D,S,io", [("rglru", 1, 1024, 256, 128, "f32"), ("rglru", 3, 37, 40, 8, "f32"),
+                                           ("rotlru", 2, 600, 64, 256, "f32"), ("rotlru", 1, 333, 64, 64, "bf16")])
+def test_cluster_exchange_equals_lookback(kind, B, L, D, S, io):
+    """Rows of 2 .. 8 segment tiles run as one thread-block cluster and exchange their aggregates
+    through distributed shared memory; forced onto the look-back over global-memory records
+    (LR_TEST_LOOKBACK), the same problem gives bitwise the same outputs, checkpoints and gradients
+    (both fold the same aggregates in the same order)."""
+    from selective_state_space_09_b200 import lrscan
+    inp = (inputs.rglru if kind == "rglru" else inputs.rotlru)(B, L, D, seed=L + 7, io=io)
+    y0, c0, g0, p0, _ = run_gpu(kind, inp, S)
+    y1, c1, g1, p1, _ = run_gpu(kind, inp, S, flags=lrscan.TEST_LOOKBACK)
+    assert p0.device_error() == (0, 0) and p1.device_error() == (0, 0)
+    assert torch.equal(y0, y1) and torch.equal(c0, c1)
+    for k in g0:
+        assert torch.equal(g0[k], g1[k]), k

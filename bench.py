@@ -1021,6 +1021,19 @@ def main():
                           "rebuild the rest; per_step_state_bytes: every step's state, which the chunked "
                           "backward never reads")
             per_kind[name]["segments"] = sg
+            # the full-state comparison in the chunked form: every chunk's entering state kept
+            # (segment = chunk, the default) against the longest measured segment's checkpoints
+            ck = max((k for k in sg if k.startswith("S") and k[1:].isdigit()), key=lambda k: int(k[1:]), default=None)
+            if ck:
+                lo = sg[ck]
+                per_kind[name]["full_state"] = {
+                    "analog": "every chunk's entering state kept (segment = chunk) vs f32 checkpoints every "
+                              "%d steps" % lo["segment"],
+                    "ms_fwd": round(r["ms_fwd"], 5), "ms_bwd": round(r["ms_bwd"], 5),
+                    "state_bytes": sg["default"]["checkpoint_bytes"], "checkpoint_bytes": lo["checkpoint_bytes"],
+                    "memory_ratio": round(sg["default"]["checkpoint_bytes"] / lo["checkpoint_bytes"], 2),
+                    "time_ratio": round((r["ms_fwd"] + r["ms_bwd"]) / (lo["ms_fwd"] + lo["ms_bwd"]), 3),
+                    "per_step_state_bytes": sg["per_step_state_bytes"]}
     line = {
         "metric": METRIC, "value": round(h["tokens_per_s"], 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

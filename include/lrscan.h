@@ -291,7 +291,7 @@ int64_t lr_probe_pipe(int which, float *out, int blocks, int threads, int iters,
  * segment checkpoints `ckpt` (lr_ckpt_bytes(desc) bytes), from device inputs a, b.  Its scratch
  * is a 1 MiB array inside the library (held by every GPU that loads the library until the
  * process exits); the call allocates nothing.  Limit: problems whose forward workspace
- * (lr_workspace_bytes(desc, 0), about 390 bytes per tile of 32 channels x S steps per batch row)
+ * (lr_workspace_bytes(desc, 0), about 770 bytes per tile of 32 channels x S steps per batch row)
  * exceeds 1 MiB are rejected with LR_ERR_WORKSPACE.
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with

@@ -703,6 +703,8 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         if (!(SM::AL && !full)) {
             mbar_arrive_expect_tx(&bar[1], (uint32_t)(a.S * K::BW * sizeof(T)));
             tma_load_3d(Ds, &mapDY, &bar[1], cc * K::BW, t0, bb);
+        } else {  // dy lands in b's slot after the recompute: bring it into L2 meanwhile
+            tma_prefetch_3d(&mapDY, cc * K::BW, t0, bb);
         }
     };
     if (tid == 0) {

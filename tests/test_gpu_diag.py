@@ -2,7 +2,8 @@
 
 Cases span several tiles and ragged tails in time (L not a multiple of the segment) and in
 channels (D not a multiple of the 32-channel tile), the degenerate L = 1 / S = 1 / L < S cases,
-bf16 I/O, the rglru workload at full size and the long-sequence rotlru workload at full size on
+bf16 I/O, rows of up to 8 segment tiles (one thread-block cluster) and longer rows (the global
+look-back), the rglru workload at full size and the long-sequence rotlru workload at full size on
 sampled units.  Tolerance: max|err| <= 1e-5 max|ref| for fp32 I/O, 2e-2 for bf16, per tensor
 (y, checkpoints and every gradient).
 """
@@ -26,6 +27,8 @@ RGLRU_CASES = [
     (1, 700, 64, 256, "f32"),       # maximum segment
     (2, 300, 128, 100, "bf16"),
     (1, 129, 8, 1, "f32"),          # S = 1: a checkpoint every step
+    (2, 1024, 64, 128, "bf16"),     # rows of 8 tiles: the largest cluster
+    (1, 1025, 64, 128, "f32"),      # rows of 9 tiles (ragged): the look-back, just past the clusters
 ]
 
 

@@ -58,6 +58,7 @@ struct DiagArgs {
     unsigned int dflags;        // lr_desc flags (LR_TEST_WITHHOLD_CARRY)
     int direct;                 // tiles numbered by block index (the grid fits on the SMs at once)
     int cl;                     // > 0: a row's tiles form one thread-block cluster of cl CTAs (cl = nseg)
+    int ahead;                  // forward, ticket mode: a tile prefetches the tile `ahead` tickets later into L2
     const float* mag;           // rotlru
     const float* theta;         // rotlru
     const float* lam;           // rglru with gates: Lambda [D]
@@ -526,7 +527,22 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             take_tile(blockIdx.x);
     }
     pdl_wait();
-    if (tid == 0 && !a.cl && !a.direct) take_tile(take_ticket(a.hdr, 0));
+    if (tid == 0 && !a.cl && !a.direct) {
+        // ticket mode: the tile `ahead` (one per SM) tickets later is brought into L2 now, so its
+        // loads find it there (forward rotlru tile 2.00 -> 1.86 ms; in the backward, whose dy is
+        // prefetched by its own tile, the same made the kernel slower, and further ahead -- a
+        // whole residency wave -- both kernels)
+        const unsigned int tk = take_ticket(a.hdr, 0);
+        take_tile(tk);
+        const unsigned int nx = tk + (unsigned int)a.ahead;
+        const int per_seg = a.B * a.ncb;
+        if (a.ahead > 0 && nx < (unsigned int)(a.nseg * per_seg)) {
+            const int sg = nx / per_seg, rem = nx % per_seg, bb = rem / a.ncb, cc = rem % a.ncb;
+            tma_prefetch_3d(&mapC, cc * K::CW, sg * a.S, bb);
+            tma_prefetch_3d(&mapB, cc * K::BW, sg * a.S, bb);
+            if (gated) tma_prefetch_3d(&mapX, cc * K::BW, sg * a.S, bb);
+        }
+    }
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
     const int t0g = seg * a.S;
@@ -1072,9 +1088,9 @@ lr_status launch_fwd(const lr_desc& d, const lr_inputs& in, void* y, void* ckpt,
         mX = mB;  // not read
     if (!ok) return LR_ERR_INVALID_ARG;
     const int cl = cluster_size(d, g);
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl, in.mag, in.theta,
-               in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
-               nullptr};
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl,
+               device_sm_count(), in.mag, in.theta, in.A, (float*)ckpt, (WsHeader*)ws,
+               (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre, nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
     auto fn = full ? diag_fwd_kernel<KIND, T, true> : diag_fwd_kernel<KIND, T, false>;
     if (full)
@@ -1116,8 +1132,8 @@ lr_status launch_bwd(const lr_desc& d, const lr_inputs& in, const void* dy, cons
     }
     if (!ok) return LR_ERR_INVALID_ARG;
     const int cl = cluster_size(d, g);
-    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl, in.mag, in.theta,
-               in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
+    DiagArgs a{(int)d.B, (int)d.L, (int)d.D, d.segment, g.nseg, g.ncb, d.flags, direct_tiles(g), cl, 0, in.mag,
+               in.theta, in.A, (float*)ckpt, (WsHeader*)ws, (unsigned int*)(ws + w.flags), ws + w.agg, ws + w.pre,
                w.partial ? (float2*)(ws + w.partial) : nullptr};
     const bool full = (d.flags & LR_FULL_STATE) != 0;
     auto fn = full ? diag_bwd_kernel<KIND, T, true> : diag_bwd_kernel<KIND, T, false>;

@@ -11,10 +11,12 @@
 // (rglru: 32 real channels; rotlru: 16 complex pairs = 32 floats).  The CTA loads the whole tile
 // into shared memory with TMA (one box per tensor, ragged tails zero-filled by the TMA unit),
 // splits it into NG time groups of S/NG steps (one thread per unit per group), scans each group
-// sequentially in fp32, combines the groups in shared memory and chains the tiles of a row
-// through a single-pass look-back over per-tile carry records (aggregate first, inclusive
-// prefix once known; bounded waits).  Results are written back into the tile's shared-memory
-// slots and stored with TMA.
+// sequentially in fp32, combines the groups in shared memory and joins the tiles of a row: a row of
+// at most 8 tiles runs as one thread-block cluster whose tiles exchange their aggregates through
+// distributed shared memory; longer rows chain through a single-pass look-back over per-tile carry
+// records in global memory (aggregate first, inclusive prefix once known; bounded waits).  Both
+// fold the same aggregates in the same order.  Results are written back into the tile's
+// shared-memory slots and stored with TMA.
 //
 // Forward: carries flow to later segments; the carry entering each segment is the segment
 // checkpoint (written to ckpt).  Backward ("segment checkpointing with recomputation during the

@@ -317,8 +317,13 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         wait_count(&ga.gready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 828);
         if (ga.sready) wait_count(&ga.sready[((size_t)c * a.B + b) * a.H + h], (unsigned int)ga.halves, a.hdr, 830);
     }
-    // decays (warpgroup 0), column factors cf[w][s] = e^{l_{32 w} - l_s} (s < 32 w)
-    if (wg == 0) l2s[row] = wg0_inclusive_sum(gla_lam(a, b, h, t0 + row), tmp) * kLog2e;
+    // decays (warpgroup 0), column factors cf[w][s] = e^{l_{32 w} - l_s} (s < 32 w); the row's
+    // gate stays in a register for dg = d lam / g at the end (its load is not repeated there)
+    float gself = 1.0f;
+    if (wg == 0) {
+        if (vrow) gself = __bfloat162float(a.g[tok]);
+        l2s[row] = wg0_inclusive_sum(vrow ? __logf(gself) : 0.0f, tmp) * kLog2e;
+    }
     __syncthreads();
 #pragma unroll
     for (int k = tid; k < 4 * kQ; k += 256) {
@@ -579,10 +584,7 @@ gla_grad_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ 
         float total;
         const float incl = wg0_inclusive_sum(dl, tmp, &total);
         const float dlam = total - incl + dl;
-        if (vrow) {
-            const float gv = __bfloat162float(a.g[tok]);
-            ga.dg[tok] = __float2bfloat16_rn(dlam / gv);
-        }
+        if (vrow) ga.dg[tok] = __float2bfloat16_rn(dlam / gself);
     }
     __syncthreads();
     if (tid < 32) {

@@ -426,6 +426,11 @@ __device__ __forceinline__ void carry_wait() { asm volatile("bar.sync 1, %0;" ::
 // Thread-block clusters: a row of at most 8 tiles runs as one cluster, and the tiles exchange their
 // aggregates through distributed shared memory instead of global-memory records.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+// Arrival that only marks a CTA's reads of the other slots as done (their values are already in
+// registers), so it needs no release ordering.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 __device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, int rank) {
     uint32_t r;
@@ -605,11 +610,11 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             if (lane < CB) carryS[lane] = carry;
             __syncwarp();
             carry_arrive();
-            cluster_arrive();  // done reading the other tiles' slots
+            cluster_arrive_relaxed();  // done reading the other tiles' slots
             const size_t slot = full ? (size_t)t0g : (size_t)seg;
             if (act) K::st_ckpt(a.ckpt + (slot * a.B + b) * a.D, unit * K::chans_per_unit, carry);
         } else {
-            cluster_arrive();
+            cluster_arrive_relaxed();
             carry_wait();
         }
     } else if (warp == 0) {
@@ -850,9 +855,9 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
             if (lane < CB) carryS[CB + lane] = carry;
             __syncwarp();
             carry_arrive();
-            cluster_arrive();
+            cluster_arrive_relaxed();
         } else {
-            cluster_arrive();
+            cluster_arrive_relaxed();
             carry_wait();
         }
     } else if (warp == 0) {

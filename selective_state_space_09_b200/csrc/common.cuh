@@ -36,7 +36,12 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 
+// Records the first error of a call in the workspace header.  A kernel launched as a programmatic
+// dependent may run before the kernel ahead of it has finished zeroing that header, so it waits for
+// that kernel first (griddepcontrol.wait; immediate in any other launch).  Only failure paths get
+// here, and no kernel ahead of another waits on the one behind it.
 __device__ __forceinline__ void record_error(WsHeader* hdr, unsigned int code, int info) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (atomicCAS(&hdr->err, 0u, code) == 0u) atomicExch(&hdr->info, info);
 }
 

@@ -512,7 +512,8 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
 
     // The tile and its loads.  The kernel starts while the workspace is being zeroed (programmatic
     // launch after ws_zero_kernel): the inputs may be read at once, the workspace only after
-    // pdl_wait.  With tiles numbered by block index the loads are issued before that wait.
+    // pdl_wait (record_error waits by itself).  With tiles numbered by block index the loads are
+    // issued before that wait; in cluster mode there is no wait.
     auto take_tile = [&](unsigned int tk) {
         const int per_seg = a.B * a.ncb;
         const int sg = tk / per_seg, rem = tk % per_seg, bb = rem / a.ncb, cc = rem % a.ncb;
@@ -533,7 +534,7 @@ diag_fwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         else if (a.direct)
             take_tile(blockIdx.x);
     }
-    pdl_wait();
+    if (!a.cl) pdl_wait();  // cluster mode touches the workspace only to record an error
     if (tid == 0 && !a.cl && !a.direct) {
         // ticket mode: the tile `ahead` (one per SM) tickets later is brought into L2 now, so its
         // loads find it there (forward rotlru tile 2.00 -> 1.86 ms; in the backward, whose dy is
@@ -740,7 +741,8 @@ diag_bwd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant_
         else if (a.direct)
             take_tile(blockIdx.x);
     }
-    pdl_wait();
+    if (!a.cl) pdl_wait();  // cluster mode touches the workspace only for its partials (a region
+                            // the zeroing leaves alone) and to record an error
     if (tid == 0 && !a.cl && !a.direct) take_tile(take_ticket(a.hdr, 1));
     __syncthreads();
     const int seg = misc[0], b = misc[1], cb = misc[2];
